@@ -1,0 +1,148 @@
+"""CPU oracle for the chunkwise TTT layer and In-Place TTT.
+
+TEST INFRASTRUCTURE ONLY: only tests/, __graft_entry__.smoke() and bench.py's
+cpu_baseline / reference leg may import this package. The product library
+(weight_sequence_layers_b200) never imports it and shares no code with it.
+
+* ttt_fwd / ttt_bwd call the C++ per-token state evolver in ttt_oracle.cpp
+  (fp64 state and arithmetic; ttt_fwd_f32 is the fp32-state build).
+* inplace_fwd follows In-Place TTT (page "In-Place Test-Time Training",
+  section "核心方法和技术细节", the chunkwise apply-then-update rule
+  W^(i+1) = W^(i) + eta * Vhat_[i]^T Z_[i]) with fp64 numpy matmuls.
+
+Every function here is pinned by tests/test_oracle_pins.py; no function is
+"parity unpinned" except for absolute agreement with the authors' own
+implementation, which the pages neither ship nor print values of.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ttt_oracle.cpp")
+_LIB = os.path.join(_HERE, "libttt_oracle.so")
+_lib = None
+
+LOSS = {"mse": 0, "ip": 1}
+ACT = {"id": 0, "silu": 1}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library in-tree (g++ -O2 -fopenmp)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-fopenmp", _SRC, "-o", _LIB]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        d, f, i = ctypes.c_double, ctypes.c_float, ctypes.c_int
+        p = ctypes.c_void_p
+        lib.ttt_oracle_fwd_f64.argtypes = [i] * 8 + [d] + [p] * 9 + [i]
+        lib.ttt_oracle_fwd_f32.argtypes = [i] * 8 + [d] + [p] * 9 + [i]
+        lib.ttt_oracle_bwd_f64.argtypes = [i] * 8 + [d] + [p] * 13 + [i]
+        for fn in (lib.ttt_oracle_fwd_f64, lib.ttt_oracle_fwd_f32, lib.ttt_oracle_bwd_f64):
+            fn.restype = i
+        _lib = lib
+    return _lib
+
+
+def _np(x, dtype):
+    """torch tensor or array -> C-contiguous numpy array of `dtype` (exact upcast)."""
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=dtype))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def ttt_fwd(Q, K, V, beta, gamma, W0, *, C: int, loss: str = "mse", act: str = "id",
+            lr_bias: float, nthreads: int = 0, state: str = "f64"):
+    """Per-token fast-weight evolution. Returns (O, W_final, W_chunks, threads_used).
+
+    Q, K: [B,H,T,dk]; V: [B,H,T,dv]; beta, gamma: [B,H,T] (gamma None = no decay);
+    W0: [B,H,dk,dv]. state="f64" (parity) or "f32" (fp32 state, timed baseline).
+    """
+    lib = _load()
+    dt = np.float64 if state == "f64" else np.float32
+    q, k, v = _np(Q, dt), _np(K, dt), _np(V, dt)
+    b_, g_, w0 = _np(beta, dt), _np(gamma, dt), _np(W0, dt)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if T % C:
+        raise ValueError("T must be a multiple of C")
+    o = np.empty((B, H, T, dv), dt)
+    wf = np.empty((B, H, dk, dv), dt)
+    wc = np.empty((B, H, T // C, dk, dv), dt)
+    fn = lib.ttt_oracle_fwd_f64 if state == "f64" else lib.ttt_oracle_fwd_f32
+    used = fn(B, H, T, dk, dv, C, LOSS[loss], ACT[act], float(lr_bias), _ptr(q), _ptr(k), _ptr(v),
+              _ptr(b_), _ptr(g_), _ptr(w0), _ptr(o), _ptr(wf), _ptr(wc), int(nthreads))
+    if used < 0:
+        raise ValueError("oracle rejected the shape")
+    return o, wf, wc, used
+
+
+def ttt_bwd(Q, K, V, beta, gamma, W0, dO, dW_T=None, *, C: int, loss: str = "mse",
+            act: str = "id", lr_bias: float, nthreads: int = 0):
+    """Reverse-mode of the per-token loop for J = <dO,O> + <dW_T,W_final> (fp64).
+    Returns dict dQ, dK, dV, dbeta, dW0."""
+    lib = _load()
+    dt = np.float64
+    q, k, v = _np(Q, dt), _np(K, dt), _np(V, dt)
+    b_, g_, w0 = _np(beta, dt), _np(gamma, dt), _np(W0, dt)
+    do, dwt = _np(dO, dt), _np(dW_T, dt)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if T % C:
+        raise ValueError("T must be a multiple of C")
+    out = dict(dQ=np.empty((B, H, T, dk)), dK=np.empty((B, H, T, dk)),
+               dV=np.empty((B, H, T, dv)), dbeta=np.empty((B, H, T)),
+               dW0=np.empty((B, H, dk, dv)))
+    used = lib.ttt_oracle_bwd_f64(B, H, T, dk, dv, C, LOSS[loss], ACT[act], float(lr_bias),
+                                  _ptr(q), _ptr(k), _ptr(v), _ptr(b_), _ptr(g_), _ptr(w0),
+                                  _ptr(do), _ptr(dwt), _ptr(out["dQ"]), _ptr(out["dK"]),
+                                  _ptr(out["dV"]), _ptr(out["dbeta"]), _ptr(out["dW0"]),
+                                  int(nthreads))
+    if used < 0:
+        raise ValueError("oracle rejected the shape")
+    return out
+
+
+def inplace_fwd(Z, Vhat, W, *, C: int, lr: float, rows=None):
+    """In-Place TTT W_down forward, apply-then-update per chunk (fp64).
+
+    Z: [T, d_ff]; Vhat: [T, d_model]; W: [d_model, d_ff] (the fast weight W_down).
+    For chunk i: O_i = Z_i W_i^T, then W_{i+1} = W_i + lr * Vhat_i^T Z_i.
+    `rows` (optional index array into d_model) restricts the computation to
+    those rows of W (and columns of O and Vhat): the rows evolve independently,
+    so the restricted result is exact. Returns (O[:, rows], W_final[rows]).
+    """
+    z = _np(Z, np.float64)
+    vh = _np(Vhat, np.float64)
+    w = _np(W, np.float64)
+    if rows is not None:
+        rows = np.asarray(rows)
+        vh = vh[:, rows]
+        w = w[rows]
+    w = w.copy()
+    T = z.shape[0]
+    if T % C:
+        raise ValueError("T must be a multiple of C")
+    o = np.empty((T, w.shape[0]))
+    for i in range(T // C):
+        zi = z[i * C:(i + 1) * C]
+        o[i * C:(i + 1) * C] = zi @ w.T          # apply with the current fast weight
+        w += lr * (vh[i * C:(i + 1) * C].T @ zi)  # then update it with this chunk
+    return o, w

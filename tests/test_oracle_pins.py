@@ -1,0 +1,341 @@
+"""Pins for the CPU oracle, each against something other than the oracle itself.
+
+* the chunk dual form printed on page "Modular TTT: Rethinking Test-Time
+  Training as Composable Modules", section "方法步骤详情"
+  (O = Q W_start - Tril(Q Khat^T) dVhat, W_end = W_start - Khat^T dVhat),
+  evaluated by brute force with explicit masks and decay weights;
+* C = 1 closed forms: the delta rule (MSE, identity) and decayed Hebbian
+  linear attention (inner product, identity);
+* chunk-size invariance of the inner-product/identity case;
+* eta = 0 and the affine state transition (I - K^T diag(eta) K) W0 + K^T diag(eta) V
+  (section "内部学习规则与学习率参数化", the update matrix whose eigenvalues
+  govern stability);
+* streaming and column independence;
+* hand-worked golden values (tests/golden/scalar_chunk_worked.txt);
+* central finite differences for every backward output;
+* In-Place TTT (page "In-Place Test-Time Training", section "核心方法和技术细节"):
+  associativity of the update, plain GEMM when C = T or eta = 0, and the
+  dual form with Z_i Z_j^T corrections.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "scalar_chunk_worked.txt")
+
+
+def sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def act_np(act, z):
+    return z * sigmoid(z) if act == "silu" else z
+
+
+def dact_np(act, z):
+    if act != "silu":
+        return np.ones_like(z)
+    s = sigmoid(z)
+    return s * (1 + z * (1 - s))
+
+
+def rand_inputs(rng, B, H, T, dk, dv, decay=True, w0_scale=0.3):
+    Q = rng.standard_normal((B, H, T, dk)) / math.sqrt(dk)
+    K = rng.standard_normal((B, H, T, dk)) / math.sqrt(dk)
+    V = rng.standard_normal((B, H, T, dv))
+    beta = rng.standard_normal((B, H, T))
+    gamma = sigmoid(2.0 + rng.standard_normal((B, H, T))) if decay else None
+    W0 = w0_scale * rng.standard_normal((B, H, dk, dv))
+    return Q, K, V, beta, gamma, W0
+
+
+def dual_form(Q, K, V, beta, gamma, W0, C, loss, act, b):
+    """The page's chunk dual form, by brute force, one head at a time."""
+    B, H, T, dk = Q.shape
+    dv = V.shape[-1]
+    O = np.zeros((B, H, T, dv))
+    WF = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for hi in range(H):
+            W = W0[bi, hi].copy()
+            for c in range(T // C):
+                sl = slice(c * C, (c + 1) * C)
+                q, k, v = Q[bi, hi, sl], K[bi, hi, sl], V[bi, hi, sl]
+                eta = 2 * sigmoid(beta[bi, hi, sl] + b)
+                lg = np.log(gamma[bi, hi, sl]) if gamma is not None else np.zeros(C)
+                L = np.cumsum(lg)
+                Z = k @ W
+                Vh = act_np(act, Z)
+                A = Vh - v if loss == "mse" else -v
+                G = A * dact_np(act, Z)
+                Zq = np.zeros((C, dv))
+                for s in range(C):
+                    acc = math.exp(L[s]) * (q[s] @ W)
+                    for r in range(s + 1):  # Tril: r <= s, the diagonal included
+                        acc = acc - eta[r] * math.exp(L[s] - L[r]) * float(q[s] @ k[r]) * G[r]
+                    Zq[s] = acc
+                O[bi, hi, sl] = act_np(act, Zq)
+                u = eta * np.exp(L[-1] - L)
+                W = math.exp(L[-1]) * W - k.T @ (u[:, None] * G)
+            WF[bi, hi] = W
+    return O, WF
+
+
+COMBOS = [(l, a) for l in ("mse", "ip") for a in ("id", "silu")]
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+@pytest.mark.parametrize("C", [1, 2, 4, 8])
+@pytest.mark.parametrize("decay", [False, True])
+def test_oracle_matches_chunk_dual_form(loss, act, C, decay):
+    rng = np.random.default_rng(100 + C)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 2, 16, 5, 3, decay=decay)
+    b = -0.7
+    O, WF, WC, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=C, loss=loss, act=act, lr_bias=b)
+    O2, WF2 = dual_form(Q, K, V, beta, gamma, W0, C, loss, act, b)
+    np.testing.assert_allclose(O, O2, rtol=0, atol=1e-12 * max(1, np.abs(O2).max()))
+    np.testing.assert_allclose(WF, WF2, rtol=0, atol=1e-12 * max(1, np.abs(WF2).max()))
+    # saved chunk-start weights: first is W0, each later one equals the state after the previous chunk
+    np.testing.assert_array_equal(WC[:, :, 0], W0)
+
+
+@pytest.mark.parametrize("decay", [False, True])
+def test_c1_is_the_delta_rule(decay):
+    rng = np.random.default_rng(7)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 1, 24, 4, 3, decay=decay)
+    b = 0.3
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=1, loss="mse", act="id", lr_bias=b)
+    W = W0[0, 0].copy()
+    for t in range(24):
+        k, v, q = K[0, 0, t], V[0, 0, t], Q[0, 0, t]
+        eta = 2 * sigmoid(beta[0, 0, t] + b)
+        g = 1.0 if gamma is None else gamma[0, 0, t]
+        W = g * W - eta * np.outer(k, k @ W - v)     # textbook delta rule with decay
+        np.testing.assert_allclose(O[0, 0, t], q @ W, atol=1e-12)
+    np.testing.assert_allclose(WF[0, 0], W, atol=1e-12)
+
+
+def test_c1_inner_product_is_decayed_hebbian_attention():
+    rng = np.random.default_rng(8)
+    T = 20
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 1, T, 4, 3, decay=True)
+    b = -1.1
+    O, _, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=1, loss="ip", act="id", lr_bias=b)
+    eta = 2 * sigmoid(beta[0, 0] + b)
+    cum = np.cumprod(gamma[0, 0])
+    for t in range(T):
+        want = cum[t] * (Q[0, 0, t] @ W0[0, 0])
+        for r in range(t + 1):
+            want = want + (cum[t] / cum[r]) * eta[r] * (Q[0, 0, t] @ K[0, 0, r]) * V[0, 0, r]
+        np.testing.assert_allclose(O[0, 0, t], want, atol=1e-12)
+
+
+def test_inner_product_identity_is_chunk_invariant():
+    rng = np.random.default_rng(9)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 2, 1, 32, 4, 4, decay=True)
+    ref = None
+    for C in (1, 2, 4, 8, 16, 32):
+        O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=C, loss="ip", act="id", lr_bias=0.2)
+        if ref is None:
+            ref = (O, WF)
+        else:
+            np.testing.assert_allclose(O, ref[0], atol=1e-12)
+            np.testing.assert_allclose(WF, ref[1], atol=1e-12)
+
+
+def test_mse_depends_on_chunk_size():
+    rng = np.random.default_rng(10)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 1, 16, 4, 4)
+    O1, _, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=1, loss="mse", act="id", lr_bias=0.5)
+    O4, _, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=4, loss="mse", act="id", lr_bias=0.5)
+    assert np.abs(O1 - O4).max() > 1e-3
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+def test_eta_zero_only_decays(loss, act):
+    rng = np.random.default_rng(11)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 2, 16, 4, 3)
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=4, loss=loss, act=act, lr_bias=-1e4)
+    cum = np.cumprod(gamma, axis=-1)
+    want = act_np(act, cum[..., None] * np.einsum("bhtk,bhkv->bhtv", Q, W0))
+    np.testing.assert_allclose(O, want, atol=1e-12)
+    np.testing.assert_allclose(WF, cum[..., -1, None, None] * W0, atol=1e-12)
+
+
+def test_affine_state_transition():
+    """No decay, identity, MSE: W_end = (I - K^T diag(eta) K) W0 + K^T diag(eta) V."""
+    rng = np.random.default_rng(12)
+    C = 8
+    Q, K, V, beta, _, W0 = rand_inputs(rng, 1, 1, C, 5, 3, decay=False)
+    b = 0.1
+    _, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, None, W0, C=C, loss="mse", act="id", lr_bias=b)
+    k, v = K[0, 0], V[0, 0]
+    D = np.diag(2 * sigmoid(beta[0, 0] + b))
+    want = (np.eye(5) - k.T @ D @ k) @ W0[0, 0] + k.T @ D @ v
+    np.testing.assert_allclose(WF[0, 0], want, atol=1e-12)
+
+
+def test_streaming_equals_one_call():
+    rng = np.random.default_rng(13)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 2, 32, 4, 4)
+    kw = dict(C=8, loss="mse", act="silu", lr_bias=-0.5)
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, **kw)
+    a = slice(0, 16)
+    b_ = slice(16, 32)
+    O1, W1, _, _ = oracle.ttt_fwd(Q[:, :, a], K[:, :, a], V[:, :, a], beta[..., a], gamma[..., a], W0, **kw)
+    O2, W2, _, _ = oracle.ttt_fwd(Q[:, :, b_], K[:, :, b_], V[:, :, b_], beta[..., b_], gamma[..., b_], W1, **kw)
+    np.testing.assert_allclose(np.concatenate([O1, O2], axis=2), O, atol=1e-13)
+    np.testing.assert_allclose(W2, WF, atol=1e-13)
+
+
+def test_value_columns_are_independent():
+    rng = np.random.default_rng(14)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 1, 16, 4, 6)
+    kw = dict(C=4, loss="mse", act="silu", lr_bias=0.0)
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, **kw)
+    cols = [1, 4, 5]
+    Os, WFs, _, _ = oracle.ttt_fwd(Q, K, V[..., cols], beta, gamma, W0[..., cols], **kw)
+    np.testing.assert_allclose(Os, O[..., cols], atol=1e-14)
+    np.testing.assert_allclose(WFs, WF[..., cols], atol=1e-14)
+
+
+def _golden():
+    cases, grads = {}, {}
+    with open(GOLDEN) as f:
+        for line in f:
+            if line.startswith("case "):
+                lhs, rhs = line[5:].split("|")
+                name, loss, act, C, g1, g2 = lhs.split()
+                cases[name] = (loss, act, int(C), float(g1), float(g2), [float(x) for x in rhs.split()])
+            elif line.startswith("grad "):
+                lhs, rhs = line[5:].split("|")
+                grads[lhs.strip()] = [float(x) for x in rhs.split()]
+    return cases, grads
+
+
+def _golden_inputs():
+    Q = np.array([1.0, 3.0]).reshape(1, 1, 2, 1)
+    K = np.array([1.0, 2.0]).reshape(1, 1, 2, 1)
+    V = np.array([2.0, -1.0]).reshape(1, 1, 2, 1)
+    beta = np.zeros((1, 1, 2))
+    W0 = np.full((1, 1, 1, 1), 0.5)
+    return Q, K, V, beta, W0
+
+
+def test_golden_scalar_worked_examples():
+    cases, _ = _golden()
+    assert len(cases) == 4
+    Q, K, V, beta, W0 = _golden_inputs()
+    for name, (loss, act, C, g1, g2, (o1, o2, wf)) in cases.items():
+        gamma = None if g1 == 1 and g2 == 1 else np.array([g1, g2]).reshape(1, 1, 2)
+        O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=C, loss=loss, act=act, lr_bias=0.0)
+        np.testing.assert_allclose(O.ravel(), [o1, o2], atol=1e-14, err_msg=name)
+        np.testing.assert_allclose(WF.ravel(), [wf], atol=1e-14, err_msg=name)
+
+
+def test_golden_scalar_backward():
+    _, grads = _golden()
+    Q, K, V, beta, W0 = _golden_inputs()
+    dO = np.array([0.0, 1.0]).reshape(1, 1, 2, 1)
+    g = oracle.ttt_bwd(Q, K, V, beta, None, W0, dO, None, C=2, loss="mse", act="id", lr_bias=0.0)
+    got = np.concatenate([g["dQ"].ravel(), g["dK"].ravel(), g["dV"].ravel(), g["dbeta"].ravel(),
+                          g["dW0"].ravel()])
+    np.testing.assert_allclose(got, grads["mse_c2"], atol=1e-14)
+
+
+def _objective(Q, K, V, beta, gamma, W0, dO, dWT, kw):
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, **kw)
+    return float((O * dO).sum() + (WF * dWT).sum())
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+def test_backward_matches_finite_differences(loss, act):
+    rng = np.random.default_rng(20 + 2 * list(dict.fromkeys(COMBOS)).index((loss, act)))
+    B, H, T, dk, dv, C = 1, 2, 16, 4, 3, 4
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, B, H, T, dk, dv, decay=True, w0_scale=0.5)
+    dO = rng.standard_normal((B, H, T, dv))
+    dWT = rng.standard_normal((B, H, dk, dv))
+    kw = dict(C=C, loss=loss, act=act, lr_bias=-0.4)
+    g = oracle.ttt_bwd(Q, K, V, beta, gamma, W0, dO, dWT, **kw)
+    h = 1e-6
+    args = dict(Q=Q, K=K, V=V, beta=beta, W0=W0)
+    names = dict(Q="dQ", K="dK", V="dV", beta="dbeta", W0="dW0")
+    for name, x in args.items():
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            jp = _objective(Q, K, V, beta, gamma, W0, dO, dWT, kw)
+            x[idx] = old - h
+            jm = _objective(Q, K, V, beta, gamma, W0, dO, dWT, kw)
+            x[idx] = old
+            fd[idx] = (jp - jm) / (2 * h)
+        an = g[names[name]]
+        err = np.abs(an - fd).max() / max(1e-12, np.abs(fd).max())
+        assert err < 1e-7, (name, err)
+
+
+def test_f32_state_build_tracks_f64():
+    rng = np.random.default_rng(30)
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, 1, 2, 64, 16, 16)
+    kw = dict(C=16, loss="mse", act="silu", lr_bias=-2.0)
+    O64, W64, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, **kw)
+    O32, W32, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, state="f32", **kw)
+    assert np.abs(O32 - O64).max() / np.abs(O64).max() < 1e-5
+    assert np.abs(W32 - W64).max() / np.abs(W64).max() < 1e-5
+
+
+# --------------------------------------------------------------------------- In-Place TTT
+
+
+def _inplace_rand(rng, T, d_ff, d_model):
+    Z = rng.standard_normal((T, d_ff))
+    Vh = 0.1 * rng.standard_normal((T, d_model))
+    W = 0.1 * rng.standard_normal((d_model, d_ff))
+    return Z, Vh, W
+
+
+def test_inplace_final_state_is_associative():
+    rng = np.random.default_rng(40)
+    Z, Vh, W = _inplace_rand(rng, 32, 12, 5)
+    for C in (1, 4, 8, 32):
+        _, WF = oracle.inplace_fwd(Z, Vh, W, C=C, lr=0.05)
+        np.testing.assert_allclose(WF, W + 0.05 * Vh.T @ Z, atol=1e-12)
+
+
+def test_inplace_single_chunk_and_zero_lr_are_plain_gemm():
+    rng = np.random.default_rng(41)
+    Z, Vh, W = _inplace_rand(rng, 32, 12, 5)
+    O, _ = oracle.inplace_fwd(Z, Vh, W, C=32, lr=0.05)
+    np.testing.assert_allclose(O, Z @ W.T, atol=1e-12)
+    O0, _ = oracle.inplace_fwd(Z, Vh, W, C=4, lr=0.0)
+    np.testing.assert_allclose(O0, Z @ W.T, atol=1e-12)
+
+
+def test_inplace_dual_form():
+    """O_i = Z_i W_0^T + eta * sum_{j<i} (Z_i Z_j^T) Vhat_j  (apply-then-update, no intra-chunk term)."""
+    rng = np.random.default_rng(42)
+    T, C, eta = 24, 4, 0.03
+    Z, Vh, W = _inplace_rand(rng, T, 7, 6)
+    O, _ = oracle.inplace_fwd(Z, Vh, W, C=C, lr=eta)
+    for i in range(T // C):
+        zi = Z[i * C:(i + 1) * C]
+        want = zi @ W.T
+        for j in range(i):
+            want = want + eta * (zi @ Z[j * C:(j + 1) * C].T) @ Vh[j * C:(j + 1) * C]
+        np.testing.assert_allclose(O[i * C:(i + 1) * C], want, atol=1e-12)
+
+
+def test_inplace_row_subset_is_exact():
+    rng = np.random.default_rng(43)
+    Z, Vh, W = _inplace_rand(rng, 16, 9, 8)
+    O, WF = oracle.inplace_fwd(Z, Vh, W, C=4, lr=0.1)
+    rows = np.array([0, 3, 7])
+    Os, WFs = oracle.inplace_fwd(Z, Vh, W, C=4, lr=0.1, rows=rows)
+    np.testing.assert_array_equal(Os, O[:, rows])
+    np.testing.assert_array_equal(WFs, WF[rows])
