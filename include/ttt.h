@@ -1,0 +1,141 @@
+/*
+ * ttt.h -- C ABI of the B200 (sm_100a) chunkwise test-time-training library.
+ *
+ * The operations follow two papers, as described on the pages they are cited from:
+ *
+ *  - Modular TTT (page "Modular TTT: Rethinking Test-Time Training as Composable
+ *    Modules"): the hidden state is a fast weight W (d_k x d_v per batch and head),
+ *    trained online on keys/values and read with queries. Per chunk of C tokens,
+ *    section "方法步骤详情" (Algorithm 1) runs three passes: train-view forward
+ *    Z = K W0 (optionally one SiLU, section "实验结果": a single nonlinearity after
+ *    Linear), train-view backward of the inner loss (MSE or inner product), and the
+ *    causal query-view readout O = Q W_start - Tril(Q Khat^T) dVhat, ending with the
+ *    state transition W_end = W_start - Khat^T dVhat. The learning rate is
+ *    eta_t = 2 sigmoid(beta_t + b) (section "内部学习规则与学习率参数化"); scalar
+ *    decay shrinks past writes (section "权重衰减").
+ *  - In-Place TTT (page "In-Place Test-Time Training", section "核心方法和技术细节"):
+ *    W_down of a gated MLP is the fast weight; per chunk O_i = Z_i W_i^T, then
+ *    W_{i+1} = W_i + eta Vhat_i^T Z_i.
+ *
+ * Exact per-token semantics implemented (one head; t = token, s = position in its chunk,
+ * W0 = state at the chunk start, act = identity or SiLU):
+ *     z_t  = k_t W0;   g_t = a_t * act'(z_t),  a_t = act(z_t) - v_t (MSE) or -v_t (IP)
+ *     eta_t = 2 sigmoid(beta_t + lr_bias)
+ *     W_t  = gamma_t W_{t-1} - eta_t k_t^T g_t          (gamma_t = 1 without decay)
+ *     o_t  = act(q_t W_t)                              (the token reads its own write)
+ * which the kernels evaluate in the chunk dual form.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers to contiguous row-major buffers owned by
+ *    the caller; the library never allocates, frees or retains them. Scratch memory is
+ *    passed in as `workspace` (size from the matching *_workspace_bytes query).
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream). A call returns after argument checks and launches; results are
+ *    ready when the stream reaches that point.
+ *  - Argument checks run on the host before anything is launched. On any error nothing
+ *    is launched and no output is touched. Device pointers must be 16-byte aligned.
+ *  - No exceptions cross the ABI; the library keeps no per-call state, so calls on
+ *    different streams may overlap provided their buffers do not alias.
+ *  - Kernels never trap. Every wait inside a kernel is bounded; a wait that runs out
+ *    sets a per-device error word and the kernel returns early (outputs then invalid).
+ *    ttt_get_device_error() reports and clears it.
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_INVALID_ARG = 1,  /* NULL required pointer, bad sizes, T % C != 0, ...      */
+  TTT_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement           */
+  TTT_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                        */
+  TTT_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than the query returned       */
+  TTT_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed             */
+  TTT_ERR_TIMEOUT = 6       /* a bounded in-kernel wait ran out (device error word)     */
+} ttt_status;
+
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;    /* type of Q,K,V,O,dO,dQ,dK,dV     */
+typedef enum { TTT_LOSS_MSE = 0, TTT_LOSS_IP = 1 } ttt_loss;
+typedef enum { TTT_ACT_ID = 0, TTT_ACT_SILU = 1 } ttt_act;
+
+/* Shape and variant of one TTT layer call. */
+typedef struct {
+  int B, H;        /* batch, heads                                                     */
+  int T;           /* tokens per sequence; T % C == 0                                    */
+  int dk, dv;      /* key/query width and value width of the fast weight (1..128)        */
+  int C;           /* chunk size (semantic: gradients inside a chunk are taken at W0)    */
+  int dtype;       /* ttt_dtype                                                         */
+  int loss;        /* ttt_loss: MSE = 1/2||act(z)-v||^2, IP = -<act(z), v>               */
+  int act;         /* ttt_act applied to both the train view and the query view         */
+  float lr_bias;   /* b in eta_t = 2 sigmoid(beta_t + b)                                 */
+} ttt_config;
+
+/* Layouts (all contiguous):
+ *   Q, K, dQ, dK        [B, H, T, dk]   dtype
+ *   V, O, dO, dV        [B, H, T, dv]   dtype
+ *   beta, gamma, dbeta  [B, H, T]       float32   (gamma NULL = no decay, gamma == 1)
+ *   W0, W_final, dW_final, dW0   [B, H, dk, dv]  float32, row index = key feature
+ *   W_chunks            [B, H, T/C, dk, dv]  dtype: the state at the start of every chunk
+ */
+
+/* Bytes of workspace ttt_chunk_fwd (for_bwd = 0) or ttt_chunk_bwd (for_bwd = 1) needs for
+ * this config; 0 if none. Returns (size_t)-1 if the config is invalid. */
+size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd);
+
+/* Forward of the chunkwise TTT layer.
+ *  in : Q, K, V, beta, gamma (nullable), W0
+ *  out: O; W_final (nullable) = state after the last token; W_chunks (nullable) = chunk-start
+ *       states, needed by ttt_chunk_bwd.
+ * bf16 configs with dk == dv in {64, 128} and C in {128, 256} run on the tcgen05 kernel;
+ * other shapes (dk, dv <= 128, C <= 256) and all float32 configs run on the SIMT kernels. */
+ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
+                         const float* beta, const float* gamma, const float* W0, void* O,
+                         float* W_final, void* W_chunks, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/* Analytic backward of the layer for the objective J = <dO, O> + <dW_final, W_final>.
+ *  in : Q, K, V, beta, gamma (nullable), W0, W_chunks (from ttt_chunk_fwd, required),
+ *       dO, dW_final (nullable = 0)
+ *  out: dQ, dK, dV, dbeta, dW0 (plain stores, not accumulated). If the caller shares W0
+ *       across the batch it reduces dW0 over B itself. No gradient is returned for gamma. */
+ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
+                         const float* beta, const float* gamma, const float* W0,
+                         const void* W_chunks, const void* dO, const float* dW_final, void* dQ,
+                         void* dK, void* dV, float* dbeta, float* dW0, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Workspace bytes of inplace_ttt_fwd; (size_t)-1 for invalid sizes. */
+size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C);
+
+/* In-Place TTT forward of the W_down fast weight (one sequence).
+ *  Z     [T, d_ff]      bf16   (the gated-MLP activation phi(H W_gate^T) * (H W_up^T))
+ *  Vhat  [T, d_model]   bf16   (the update target)
+ *  W     [d_model, d_ff] float32, in: W_down at token 0, out: W_down after the last chunk
+ *  O     [T, d_model]   bf16   out: O_i = Z_i W_i^T (apply, then update: no intra-chunk term)
+ * Requirements: T % C == 0, C % 128 == 0, d_ff % 64 == 0, d_model % 128 == 0. */
+ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                           const void* Vhat, float* W, void* O, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns TTT_ERR_TIMEOUT if any kernel of this library on the
+ * current device recorded a bounded wait that ran out since the last call (and clears the
+ * word), TTT_ERR_CUDA if the stream reports an error, else TTT_OK. */
+ttt_status ttt_get_device_error(void* stream);
+
+/* Launches a one-warp kernel whose wait on an mbarrier that nothing completes is bounded
+ * by `spin_limit` polls; it must end by recording a timeout in the device error word.
+ * Used to test the failure path without faulting the GPU. */
+ttt_status ttt_selftest_bounded_wait(unsigned spin_limit, void* stream);
+
+/* Static description of a status code. */
+const char* ttt_status_string(ttt_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TTT_H_ */

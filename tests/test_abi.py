@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every function include/ttt.h declares, and rejects bad
+arguments on the host before touching a GPU (these run without one)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import weight_sequence_layers_b200 as ttt
+
+FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_ttt_workspace_bytes",
+             "inplace_ttt_fwd", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "ttt_status_string"}
+
+
+def test_header_declares_the_entry_points():
+    assert FWD_NAMES <= set(ttt.header_functions())
+
+
+def test_every_declared_symbol_is_exported():
+    out = subprocess.run(["nm", "-D", "--defined-only", ttt.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in ttt.header_functions():
+        assert name in exported, name
+        assert getattr(ttt.lib, name) is not None
+
+
+def test_library_links_no_libcuda():
+    out = subprocess.run(["ldd", ttt.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcuda.so" not in out and "libcudart.so" not in out
+
+
+def test_status_strings():
+    for s in range(7):
+        assert ttt.status_string(s)
+    assert ttt.status_string(99) == "unknown status"
+
+
+def _cfg(**kw):
+    base = dict(B=2, H=3, T=256, dk=64, dv=64, C=64, dtype="f32", loss="mse", act="id", lr_bias=-2.9)
+    base.update(kw)
+    return ttt.make_config(**base)
+
+
+def test_workspace_query_validates_config():
+    assert ttt.ttt_workspace_bytes(_cfg(), False) == 0
+    assert ttt.ttt_workspace_bytes(_cfg(), True) > 0
+    for bad in (dict(T=250), dict(C=0), dict(B=0), dict(dk=0)):
+        with pytest.raises(ttt.TTTError):
+            ttt.ttt_workspace_bytes(_cfg(**bad), False)
+    cfg = _cfg()
+    cfg.loss = 7
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_workspace_bytes(cfg, False)
+
+
+def test_unsupported_shapes_are_reported():
+    cfg = _cfg(dk=256)
+    assert ttt.lib.ttt_workspace_bytes(ctypes.byref(cfg), 0) == ctypes.c_size_t(-1).value
+    st = ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), *([16] * 3), 16, None, 16, 16, None, None, None, 0, None)
+    assert st == ttt.ERR_UNSUPPORTED
+
+
+def test_fwd_argument_errors_before_launch():
+    cfg = _cfg()
+    call = lambda *p: ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), *p, None)
+    A = 4096  # a 16-byte aligned fake address: never dereferenced on these paths
+    assert call(None, A, A, A, None, A, A, None, None, None, 0) == ttt.ERR_INVALID_ARG
+    assert call(A, A, A, A, None, A, None, None, None, None, 0) == ttt.ERR_INVALID_ARG
+    assert call(A + 4, A, A, A, None, A, A, None, None, None, 0) == ttt.ERR_ALIGNMENT
+    assert call(A, A, A, A, A + 8, A, A, None, None, None, 0) == ttt.ERR_ALIGNMENT
+    bad = _cfg(T=100)
+    assert ttt.lib.ttt_chunk_fwd(ctypes.byref(bad), A, A, A, A, None, A, A, None, None, None, 0,
+                                 None) == ttt.ERR_INVALID_ARG
+    assert ttt.lib.ttt_chunk_fwd(None, A, A, A, A, None, A, A, None, None, None, 0, None) == ttt.ERR_INVALID_ARG
+
+
+def test_bwd_requires_chunk_states_and_workspace():
+    cfg = _cfg()
+    A = 4096
+    base = [A, A, A, A, None, A, A, A, None, A, A, A, A, A]
+    args = list(base)
+    args[6] = None  # W_chunks
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *args, None, 0, None) == ttt.ERR_INVALID_ARG
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *base, None, 0, None) == ttt.ERR_WORKSPACE
+    need = ttt.ttt_workspace_bytes(cfg, True)
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *base, A, need - 1, None) == ttt.ERR_WORKSPACE
+
+
+def test_inplace_argument_errors():
+    A = 4096
+    f = ttt.lib.inplace_ttt_fwd
+    assert f(1000, 256, 256, 128, 1e-3, A, A, A, A, A, 1 << 30, None) == ttt.ERR_INVALID_ARG  # T % C
+    assert f(960, 256, 256, 96, 1e-3, A, A, A, A, A, 1 << 30, None) == ttt.ERR_UNSUPPORTED    # C % 128
+    assert f(1024, 250, 256, 128, 1e-3, A, A, A, A, A, 1 << 30, None) == ttt.ERR_UNSUPPORTED  # d_ff % 64
+    assert f(1024, 256, 256, 128, float("nan"), A, A, A, A, A, 1 << 30, None) == ttt.ERR_INVALID_ARG
+    assert f(1024, 256, 256, 128, 1e-3, None, A, A, A, A, 1 << 30, None) == ttt.ERR_INVALID_ARG
+    assert f(1024, 256, 256, 128, 1e-3, A, A, A + 4, A, A, 1 << 30, None) == ttt.ERR_ALIGNMENT
+    need = ttt.inplace_ttt_workspace_bytes(1024, 256, 256, 128)
+    assert need >= 2 * 256 * 256 * 2
+    assert f(1024, 256, 256, 128, 1e-3, A, A, A, A, A, need - 1, None) == ttt.ERR_WORKSPACE
+    with pytest.raises(ttt.TTTError):
+        ttt.inplace_ttt_workspace_bytes(1000, 256, 256, 128)
+
+
+def test_valid_call_without_a_gpu_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    cfg = _cfg()
+    A = 4096
+    st = ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), A, A, A, A, None, A, A, None, None, None, 0, None)
+    assert st == ttt.ERR_CUDA

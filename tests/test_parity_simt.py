@@ -1,0 +1,66 @@
+"""GPU parity of the SIMT kernels (float32 workloads, and bf16 shapes outside the tensor-core
+envelope) against the oracle, element by element."""
+import pytest
+import torch
+
+import synth
+from _runners import oracle_bwd, oracle_fwd, run_bwd, run_fwd
+from _util import rel_err
+
+pytestmark = pytest.mark.gpu
+
+F32_TOL = 1e-4
+BF16_TOL = 2e-2
+
+
+def test_tiny_fp32_workload_forward():
+    cfg = synth.TINY_FP32
+    inp = synth.ttt_inputs(cfg, device="cuda")
+    got = run_fwd(cfg, inp)
+    ref = oracle_fwd(cfg, inp)
+    for k in ("O", "W_final", "W_chunks"):
+        assert rel_err(got[k], ref[k]) <= F32_TOL, k
+
+
+SHAPES = [
+    # B, H, T, dk, dv, C
+    (1, 2, 96, 16, 24, 32),
+    (2, 1, 192, 64, 40, 64),
+    (1, 1, 60, 8, 8, 20),      # C not a multiple of the 32-row query tile
+    (1, 1, 512, 128, 128, 256),
+]
+COMBOS = [("mse", "id"), ("mse", "silu"), ("ip", "id"), ("ip", "silu")]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("loss,act", COMBOS)
+@pytest.mark.parametrize("decay", [False, True])
+def test_fp32_forward_backward(shape, loss, act, decay):
+    B, H, T, dk, dv, C = shape
+    cfg = synth.TINY_FP32.replace(B=B, H=H, T=T, dk=dk, dv=dv, C=C, loss=loss, act=act,
+                                  decay=decay, w0_std=0.05, normalize="qk")
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=T + dk)
+    inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(3))
+    got = run_fwd(cfg, inp)
+    ref = oracle_fwd(cfg, inp)
+    for k in ("O", "W_final", "W_chunks"):
+        assert rel_err(got[k], ref[k]) <= F32_TOL, k
+    g = run_bwd(cfg, inp, got["W_chunks"])
+    r = oracle_bwd(cfg, inp)
+    for k in ("dQ", "dK", "dV", "dbeta", "dW0"):
+        assert rel_err(g[k], r[k]) <= F32_TOL, k
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+def test_bf16_shapes_outside_the_tensor_core_envelope(loss, act):
+    cfg = synth.FWD_410M.replace(B=1, H=2, T=256, dk=32, dv=48, C=64, loss=loss, act=act,
+                                 w0_std=0.05)
+    inp = synth.ttt_inputs(cfg, device="cuda")
+    got = run_fwd(cfg, inp)
+    ref = oracle_fwd(cfg, inp)
+    for k in ("O", "W_final"):
+        assert rel_err(got[k], ref[k]) <= BF16_TOL, k
+    g = run_bwd(cfg, inp, got["W_chunks"])
+    r = oracle_bwd(cfg, inp)
+    for k in ("dQ", "dK", "dV", "dbeta", "dW0"):
+        assert rel_err(g[k], r[k]) <= BF16_TOL, k

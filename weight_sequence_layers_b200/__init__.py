@@ -1,0 +1,146 @@
+"""Python binding of the B200 chunkwise-TTT library (libttt.so, C ABI in include/ttt.h).
+
+Argument marshalling only: every function here forwards torch tensors' device pointers,
+sizes and the current CUDA stream to the C entry point of the same name and raises
+TTTError on a non-OK status. Every step of the computation runs in the library's CUDA
+kernels; there is no fallback of any kind. Importing fails loudly if libttt.so has not
+been built (python weight_sequence_layers_b200/build.py).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libttt.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "ttt.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with python weight_sequence_layers_b200/build.py")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(7)
+F32, BF16 = 0, 1
+LOSS = {"mse": 0, "ip": 1}
+ACT = {"id": 0, "silu": 1}
+
+
+class TTTError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+class ttt_config(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("loss", ctypes.c_int), ("act", ctypes.c_int),
+                ("lr_bias", ctypes.c_float)]
+
+
+_p, _i, _u, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_float, ctypes.c_size_t
+_cfgp = ctypes.POINTER(ttt_config)
+_SIGS = {
+    "ttt_workspace_bytes": ([_cfgp, _i], _sz),
+    "ttt_chunk_fwd": ([_cfgp] + [_p] * 10 + [_sz, _p], _i),
+    "ttt_chunk_bwd": ([_cfgp] + [_p] * 15 + [_sz, _p], _i),
+    "inplace_ttt_workspace_bytes": ([_i] * 4, _sz),
+    "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 5 + [_sz, _p], _i),
+    "ttt_get_device_error": ([_p], _i),
+    "ttt_selftest_bounded_wait": ([_u, _p], _i),
+    "ttt_status_string": ([_i], ctypes.c_char_p),
+}
+for _name, (_args, _ret) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _ret
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/ttt.h declares."""
+    text = open(HEADER).read()
+    return re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(\w+)\s*\(", text, flags=re.M)
+
+
+def status_string(status: int) -> str:
+    return _lib.ttt_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise TTTError(status, where)
+
+
+def make_config(B, H, T, dk, dv, C, dtype="bf16", loss="mse", act="id", lr_bias=0.0) -> ttt_config:
+    return ttt_config(B, H, T, dk, dv, C, F32 if dtype in ("f32", F32) else BF16,
+                      LOSS.get(loss, loss), ACT.get(act, act), float(lr_bias))
+
+
+def ttt_workspace_bytes(cfg: ttt_config, for_bwd: bool) -> int:
+    n = _lib.ttt_workspace_bytes(ctypes.byref(cfg), int(bool(for_bwd)))
+    if n == ctypes.c_size_t(-1).value:
+        raise TTTError(ERR_INVALID_ARG, "ttt_workspace_bytes")
+    return n
+
+
+def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None,
+                  workspace=None, workspace_bytes=0, stream=None):
+    st = _lib.ttt_chunk_fwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
+                            _ptr(W0), _ptr(O), _ptr(W_final), _ptr(W_chunks), _ptr(workspace),
+                            int(workspace_bytes), _stream(stream))
+    _check(st, "ttt_chunk_fwd")
+
+
+def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final, dQ, dK, dV, dbeta, dW0,
+                  workspace=None, workspace_bytes=0, stream=None):
+    st = _lib.ttt_chunk_bwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
+                            _ptr(W0), _ptr(W_chunks), _ptr(dO), _ptr(dW_final), _ptr(dQ), _ptr(dK),
+                            _ptr(dV), _ptr(dbeta), _ptr(dW0), _ptr(workspace),
+                            int(workspace_bytes), _stream(stream))
+    _check(st, "ttt_chunk_bwd")
+
+
+def inplace_ttt_workspace_bytes(T, d_ff, d_model, C) -> int:
+    n = _lib.inplace_ttt_workspace_bytes(T, d_ff, d_model, C)
+    if n == ctypes.c_size_t(-1).value:
+        raise TTTError(ERR_INVALID_ARG, "inplace_ttt_workspace_bytes")
+    return n
+
+
+def inplace_ttt_fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace=None, workspace_bytes=0,
+                    stream=None):
+    st = _lib.inplace_ttt_fwd(T, d_ff, d_model, C, float(lr), _ptr(Z), _ptr(Vhat), _ptr(W),
+                              _ptr(O), _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "inplace_ttt_fwd")
+
+
+def ttt_get_device_error(stream=None) -> int:
+    """Returns the status (OK, ERR_TIMEOUT or ERR_CUDA) instead of raising."""
+    return _lib.ttt_get_device_error(_stream(stream))
+
+
+def ttt_selftest_bounded_wait(spin_limit: int, stream=None):
+    _check(_lib.ttt_selftest_bounded_wait(int(spin_limit), _stream(stream)), "ttt_selftest_bounded_wait")
+
+
+# Raw C entry points (for callers that marshal pointers themselves).
+lib = _lib

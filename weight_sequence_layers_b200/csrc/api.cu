@@ -1,0 +1,283 @@
+// C ABI of the library: argument checks on the host, dispatch to the kernels, the per-device
+// error word that bounded in-kernel waits report into, and the tensor-map encoder.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/ttt.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tttk {
+
+// One error word per device: kernels OR error codes into it, ttt_get_device_error reads and
+// clears it.
+__device__ unsigned g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned* g_err_ptr[kMaxDevices];
+std::mutex g_err_mu;
+
+unsigned* error_word(cudaError_t* e) {
+  int dev = 0;
+  *e = cudaGetDevice(&dev);
+  if (*e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    if (*e == cudaSuccess) *e = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    *e = cudaGetSymbolAddress(&p, g_error_word);
+    if (*e != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<unsigned*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks the config; returns TTT_OK or the first failure.
+ttt_status check_config(const ttt_config* c) {
+  if (!c) return TTT_ERR_INVALID_ARG;
+  if (c->B < 1 || c->H < 1 || c->T < 1 || c->dk < 1 || c->dv < 1 || c->C < 1)
+    return TTT_ERR_INVALID_ARG;
+  if (c->T % c->C) return TTT_ERR_INVALID_ARG;
+  if (c->dtype != TTT_F32 && c->dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+  if (c->loss != TTT_LOSS_MSE && c->loss != TTT_LOSS_IP) return TTT_ERR_INVALID_ARG;
+  if (c->act != TTT_ACT_ID && c->act != TTT_ACT_SILU) return TTT_ERR_INVALID_ARG;
+  if (!isfinite(c->lr_bias)) return TTT_ERR_INVALID_ARG;
+  if ((long long)c->B * c->H * c->T * (c->dk > c->dv ? c->dk : c->dv) > (1ll << 40))
+    return TTT_ERR_INVALID_ARG;
+  return TTT_OK;
+}
+
+LayerArgs args_of(const ttt_config* c) {
+  LayerArgs a{};
+  a.B = c->B;
+  a.H = c->H;
+  a.T = c->T;
+  a.dk = c->dk;
+  a.dv = c->dv;
+  a.C = c->C;
+  a.dtype = c->dtype;
+  a.loss = c->loss;
+  a.act = c->act;
+  a.lr_bias = c->lr_bias;
+  return a;
+}
+
+enum Path { PATH_NONE, PATH_SIMT, PATH_TC };
+
+Path fwd_path(const LayerArgs& a) {
+  if (a.dtype == TTT_BF16 && tc_fwd_supported(a)) return PATH_TC;
+  if (simt_supported(a)) return PATH_SIMT;
+  return PATH_NONE;
+}
+Path bwd_path(const LayerArgs& a) {
+  if (a.dtype == TTT_BF16 && tc_bwd_supported(a)) return PATH_TC;
+  if (simt_supported(a)) return PATH_SIMT;
+  return PATH_NONE;
+}
+
+ttt_status launch_status(cudaError_t e) { return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA; }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+__global__ void selftest_wait_kernel(unsigned spin_limit, unsigned* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on `bar`: the wait must give up after spin_limit polls.
+    bool done = false;
+    for (unsigned it = 0; it < spin_limit && !done; ++it) done = mbar_try_wait(smem_u32(&bar), 0);
+    if (!done) atomicOr(err, ERR_WAIT_TIMEOUT);
+  }
+}
+
+}  // namespace
+
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_elems * 2};
+  cuuint32_t box[2] = {box_inner, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace tttk
+
+using namespace tttk;
+
+extern "C" {
+
+const char* ttt_status_string(ttt_status s) {
+  switch (s) {
+    case TTT_OK: return "ok";
+    case TTT_ERR_INVALID_ARG: return "invalid argument";
+    case TTT_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TTT_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case TTT_ERR_WORKSPACE: return "workspace missing or too small";
+    case TTT_ERR_CUDA: return "CUDA error";
+    case TTT_ERR_TIMEOUT: return "bounded in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
+  if (check_config(cfg) != TTT_OK) return (size_t)-1;
+  LayerArgs a = args_of(cfg);
+  if (!for_bwd) {
+    switch (fwd_path(a)) {
+      case PATH_TC: return tc_fwd_workspace(a);
+      case PATH_SIMT: return simt_fwd_workspace(a);
+      default: return (size_t)-1;
+    }
+  }
+  switch (bwd_path(a)) {
+    case PATH_TC: return tc_bwd_workspace(a);
+    case PATH_SIMT: return simt_bwd_workspace(a);
+    default: return (size_t)-1;
+  }
+}
+
+ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
+                         const float* beta, const float* gamma, const float* W0, void* O,
+                         float* W_final, void* W_chunks, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  ttt_status st = check_config(cfg);
+  if (st != TTT_OK) return st;
+  if (!Q || !K || !V || !beta || !W0 || !O) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, beta, gamma, W0, O, W_final, W_chunks, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  LayerArgs a = args_of(cfg);
+  const Path path = fwd_path(a);
+  if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
+  const size_t need = path == PATH_TC ? tc_fwd_workspace(a) : simt_fwd_workspace(a);
+  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.W0 = W0; a.O = O;
+  a.W_final = W_final; a.W_chunks = W_chunks; a.ws = workspace; a.ws_bytes = workspace_bytes;
+  a.err = err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(path == PATH_TC ? tc_fwd(a, s) : simt_fwd(a, s));
+}
+
+ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
+                         const float* beta, const float* gamma, const float* W0,
+                         const void* W_chunks, const void* dO, const float* dW_final, void* dQ,
+                         void* dK, void* dV, float* dbeta, float* dW0, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  ttt_status st = check_config(cfg);
+  if (st != TTT_OK) return st;
+  if (!Q || !K || !V || !beta || !W0 || !W_chunks || !dO || !dQ || !dK || !dV || !dbeta || !dW0)
+    return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final,
+                        dQ, dK, dV, dbeta, dW0, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  LayerArgs a = args_of(cfg);
+  const Path path = bwd_path(a);
+  if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
+  const size_t need = path == PATH_TC ? tc_bwd_workspace(a) : simt_bwd_workspace(a);
+  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.W0 = W0; a.W_chunks =
+      const_cast<void*>(W_chunks);
+  a.dO = dO; a.dW_final = dW_final; a.dQ = dQ; a.dK = dK; a.dV = dV; a.dbeta = dbeta;
+  a.dW0 = dW0; a.ws = workspace; a.ws_bytes = workspace_bytes; a.err = err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(path == PATH_TC ? tc_bwd(a, s) : simt_bwd(a, s));
+}
+
+size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C) {
+  if (T < 1 || d_ff < 1 || d_model < 1 || C < 1 || T % C || C % 128 || d_ff % 64 ||
+      d_model % 128)
+    return (size_t)-1;
+  return inplace_workspace(T, d_ff, d_model, C);
+}
+
+ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                           const void* Vhat, float* W, void* O, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  if (T < 1 || d_ff < 1 || d_model < 1 || C < 1 || T % C || !isfinite(lr))
+    return TTT_ERR_INVALID_ARG;
+  if (C % 128 || d_ff % 64 || d_model % 128) return TTT_ERR_UNSUPPORTED;
+  if ((long long)T * d_ff > (1ll << 40) || (long long)d_model * d_ff > (1ll << 40))
+    return TTT_ERR_INVALID_ARG;
+  if (!Z || !Vhat || !W || !O) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Z, Vhat, W, O, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const size_t need = inplace_workspace(T, d_ff, d_model, C);
+  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  return launch_status(inplace_run(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace, err,
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status ttt_get_device_error(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TTT_ERR_CUDA;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  unsigned h = 0;
+  if (cudaMemcpy(&h, err, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_CUDA;
+  if (h) {
+    const unsigned zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return TTT_ERR_CUDA;
+    return TTT_ERR_TIMEOUT;
+  }
+  return TTT_OK;
+}
+
+ttt_status ttt_selftest_bounded_wait(unsigned spin_limit, void* stream) {
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(spin_limit, err);
+  return launch_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Host-side interface between the C ABI (api.cu) and the kernel translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace tttk {
+
+struct LayerArgs {
+  int B, H, T, dk, dv, C, dtype, loss, act;
+  float lr_bias;
+  const void *Q, *K, *V;
+  const float *beta, *gamma, *W0;
+  void* O;
+  float* W_final;
+  void* W_chunks;
+  const void* dO;
+  const float* dW_final;
+  void *dQ, *dK, *dV;
+  float *dbeta, *dW0;
+  void* ws;
+  size_t ws_bytes;
+  unsigned* err;  // per-device error word
+};
+
+// SIMT kernels (float32 or bf16 storage, float32 arithmetic).
+size_t simt_fwd_workspace(const LayerArgs& a);
+size_t simt_bwd_workspace(const LayerArgs& a);
+bool simt_supported(const LayerArgs& a);
+cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s);
+cudaError_t simt_bwd(const LayerArgs& a, cudaStream_t s);
+
+// tcgen05 kernels (bf16 storage).
+bool tc_fwd_supported(const LayerArgs& a);
+size_t tc_fwd_workspace(const LayerArgs& a);
+cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s);
+bool tc_bwd_supported(const LayerArgs& a);
+size_t tc_bwd_workspace(const LayerArgs& a);
+cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
+
+// In-Place TTT.
+size_t inplace_workspace(int T, int d_ff, int d_model, int C);
+cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                        const void* Vhat, float* W, void* O, void* ws, unsigned* err,
+                        cudaStream_t s);
+
+// 2-D bf16 tensor map with 128-byte swizzle: `rows` rows of `inner` elements, rows
+// `row_stride_elems` apart; box = {box_inner (64), box_rows}. Returns false on failure.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_rows);
+
+}  // namespace tttk

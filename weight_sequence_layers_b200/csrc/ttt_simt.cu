@@ -1,0 +1,360 @@
+// SIMT (CUDA-core, float32 arithmetic) kernels of the chunkwise TTT layer.
+//
+// They serve the float32 configurations and bf16 shapes outside the tensor-core kernels'
+// envelope. Both evaluate the chunk dual form of page "Modular TTT: Rethinking Test-Time
+// Training as Composable Modules", section "方法步骤详情" (Algorithm 1): per chunk, with
+// W0 the chunk-start fast weight,
+//     Z  = K W0,  G = a(Z) * act'(Z)                 (train view + inner-loss gradient)
+//     S_sr = eta_r exp(L_s - L_r) (q_s . k_r), r <= s (Tril of the scaled, decayed scores)
+//     O  = act(diag(Gamma) Q W0 - S G)               (query view)
+//     W_end = Gamma_C W0 - K^T diag(u) G,  u_r = eta_r exp(L_C - L_r)
+// with eta = 2 sigmoid(beta + b) (section "内部学习规则与学习率参数化") and
+// L_s = sum_{t<=s} log gamma_t (section "权重衰减").
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "kernels.h"
+
+namespace tttk {
+namespace {
+
+constexpr int kNvs = 32;        // value columns per forward block
+constexpr int kRows = 32;       // query rows per score tile in the forward
+constexpr int kMaxC = 256;
+constexpr int kMaxD = 128;
+
+__device__ __forceinline__ float ldf(const float* p) { return *p; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void stf(float* p, float v) { *p = v; }
+__device__ __forceinline__ void stf(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+__device__ __forceinline__ float sigm(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float actf(int act, float z) { return act ? z * sigm(z) : z; }
+__device__ __forceinline__ float act1(int act, float z) {
+  if (!act) return 1.f;
+  const float s = sigm(z);
+  return s * (1.f + z * (1.f - s));
+}
+__device__ __forceinline__ float act2(int act, float z) {
+  if (!act) return 0.f;
+  const float s = sigm(z);
+  return s * (1.f - s) * (2.f + z * (1.f - 2.f * s));
+}
+
+struct Dims {
+  int T, dk, dv, C, loss, act, has_gamma;
+  float lr_bias;
+};
+
+// eta_s and the chunk-local log-decay prefix L_s for the C tokens of chunk c of head bh.
+__device__ void chunk_scans(const Dims& d, const float* beta, const float* gamma, int bh, int c,
+                            float* eta, float* L) {
+  const size_t t0 = (size_t)bh * d.T + (size_t)c * d.C;
+  for (int s = threadIdx.x; s < d.C; s += blockDim.x) {
+    eta[s] = 2.f * sigm(beta[t0 + s] + d.lr_bias);
+    L[s] = d.has_gamma ? logf(gamma[t0 + s]) : 0.f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int s = 1; s < d.C; ++s) L[s] += L[s - 1];
+  __syncthreads();
+}
+
+template <typename TI>
+__global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, const TI* K,
+                                                       const TI* V, const float* beta,
+                                                       const float* gamma, const float* W0,
+                                                       TI* O, float* Wf, TI* Wc) {
+  extern __shared__ float smem[];
+  const int bh = blockIdx.y, j0 = blockIdx.x * kNvs;
+  const int nv = min(kNvs, d.dv - j0);
+  const int dk = d.dk, dv = d.dv, C = d.C, NC = d.T / d.C;
+  float* Ws = smem;                  // [dk][kNvs] state slice
+  float* G = Ws + dk * kNvs;         // [C][kNvs]
+  float* S = G + C * kNvs;           // [kRows][C]
+  float* eta = S + kRows * C;        // [C]
+  float* L = eta + C;                // [C]
+  const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
+  for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
+    const int i = e / nv, j = e % nv;
+    Ws[i * kNvs + j] = W0[(size_t)bh * dk * dv + (size_t)i * dv + j0 + j];
+  }
+  __syncthreads();
+  for (int c = 0; c < NC; ++c) {
+    if (Wc)
+      for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
+        const int i = e / nv, j = e % nv;
+        stf(&Wc[(((size_t)bh * NC + c) * dk + i) * dv + j0 + j], Ws[i * kNvs + j]);
+      }
+    chunk_scans(d, beta, gamma, bh, c, eta, L);
+    const size_t tc = (size_t)c * C;
+    // train view: G = a(Z) * act'(Z), Z = K W0
+    for (int e = threadIdx.x; e < C * nv; e += blockDim.x) {
+      const int s = e / nv, j = e % nv;
+      const TI* kr = K + qk0 + (tc + s) * dk;
+      float z = 0.f;
+      for (int i = 0; i < dk; ++i) z += ldf(kr + i) * Ws[i * kNvs + j];
+      const float vv = ldf(V + v0 + (tc + s) * dv + j0 + j);
+      const float a = d.loss == 0 ? actf(d.act, z) - vv : -vv;
+      G[s * kNvs + j] = a * act1(d.act, z);
+    }
+    __syncthreads();
+    // query view, kRows queries at a time
+    for (int s0 = 0; s0 < C; s0 += kRows) {
+      for (int e = threadIdx.x; e < kRows * C; e += blockDim.x) {
+        const int sr = e / C, r = e % C, s = s0 + sr;
+        float v = 0.f;
+        if (r <= s && s < C) {
+          const TI* qs = Q + qk0 + (tc + s) * dk;
+          const TI* kr = K + qk0 + (tc + r) * dk;
+          float p = 0.f;
+          for (int i = 0; i < dk; ++i) p += ldf(qs + i) * ldf(kr + i);
+          v = eta[r] * expf(L[s] - L[r]) * p;
+        }
+        S[sr * C + r] = v;
+      }
+      __syncthreads();
+      for (int e = threadIdx.x; e < kRows * nv; e += blockDim.x) {
+        const int sr = e / nv, j = e % nv, s = s0 + sr;
+        if (s >= C) continue;
+        const TI* qs = Q + qk0 + (tc + s) * dk;
+        float y = 0.f;
+        for (int i = 0; i < dk; ++i) y += ldf(qs + i) * Ws[i * kNvs + j];
+        float acc = expf(L[s]) * y;
+        for (int r = 0; r <= s; ++r) acc -= S[sr * C + r] * G[r * kNvs + j];
+        stf(&O[v0 + (tc + s) * dv + j0 + j], actf(d.act, acc));
+      }
+      __syncthreads();
+    }
+    // state transition
+    const float LC = L[C - 1];
+    for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
+      const int i = e / nv, j = e % nv;
+      float w = expf(LC) * Ws[i * kNvs + j];
+      for (int r = 0; r < C; ++r)
+        w -= eta[r] * expf(LC - L[r]) * ldf(K + qk0 + (tc + r) * dk + i) * G[r * kNvs + j];
+      Ws[i * kNvs + j] = w;
+    }
+    __syncthreads();
+  }
+  if (Wf)
+    for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
+      const int i = e / nv, j = e % nv;
+      Wf[(size_t)bh * dk * dv + (size_t)i * dv + j0 + j] = Ws[i * kNvs + j];
+    }
+}
+
+// Per-head float32 scratch of the backward (in units of floats): Wh, Wn, W0 (dk x dv each),
+// Z, G, dZq, Y, dG, dZ (C x dv each), S, dS (C x C each), eta, L, deta (C each).
+__host__ __device__ inline size_t bwd_head_floats(int C, int dk, int dv) {
+  return 3 * (size_t)dk * dv + 6 * (size_t)C * dv + 2 * (size_t)C * C + 3 * (size_t)C;
+}
+
+// Analytic backward of the chunk dual form, reverse over chunks; one block per head.
+// Wh carries dJ/dW at the chunk end; every intermediate lives in the head's scratch.
+template <typename TI>
+__global__ void __launch_bounds__(512) simt_bwd_kernel(
+    Dims d, const TI* Q, const TI* K, const TI* V, const float* beta, const float* gamma,
+    const TI* Wc, const TI* dO, const float* dWf, TI* dQ, TI* dK, TI* dV, float* dbeta,
+    float* dW0, float* ws) {
+  const int bh = blockIdx.x;
+  const int dk = d.dk, dv = d.dv, C = d.C, NC = d.T / d.C;
+  float* Wh = ws + (size_t)bh * bwd_head_floats(C, dk, dv);
+  float* Wn = Wh + dk * dv;
+  float* W0 = Wn + dk * dv;  // float copy of the chunk-start state
+  float* Z = W0 + dk * dv;
+  float* G = Z + C * dv;
+  float* DZQ = G + C * dv;
+  float* Y = DZQ + C * dv;
+  float* DG = Y + C * dv;
+  float* DZ = DG + C * dv;
+  float* S = DZ + C * dv;
+  float* DS = S + C * C;
+  float* eta = DS + C * C;
+  float* L = eta + C;
+  float* deta = L + C;
+  const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
+  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
+    Wh[e] = dWf ? dWf[(size_t)bh * dk * dv + e] : 0.f;
+  __syncthreads();
+  for (int c = NC - 1; c >= 0; --c) {
+    const size_t tc = (size_t)c * C;
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
+      W0[e] = ldf(Wc + ((size_t)bh * NC + c) * dk * dv + e);
+    chunk_scans(d, beta, gamma, bh, c, eta, L);  // ends with __syncthreads
+    const float LC = L[C - 1];
+    // Z = K W0, G
+    for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
+      const int s = e / dv, j = e % dv;
+      float z = 0.f;
+      for (int i = 0; i < dk; ++i) z += ldf(K + qk0 + (tc + s) * dk + i) * W0[i * dv + j];
+      const float vv = ldf(V + v0 + (tc + s) * dv + j);
+      const float a = d.loss == 0 ? actf(d.act, z) - vv : -vv;
+      Z[e] = z;
+      G[e] = a * act1(d.act, z);
+    }
+    // S (causal, scaled)
+    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
+      const int s = e / C, r = e % C;
+      float v = 0.f;
+      if (r <= s) {
+        float p = 0.f;
+        for (int i = 0; i < dk; ++i)
+          p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i);
+        v = eta[r] * expf(L[s] - L[r]) * p;
+      }
+      S[e] = v;
+    }
+    // Y = K Wh
+    for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
+      const int r = e / dv, j = e % dv;
+      float y = 0.f;
+      for (int i = 0; i < dk; ++i) y += ldf(K + qk0 + (tc + r) * dk + i) * Wh[i * dv + j];
+      Y[e] = y;
+    }
+    __syncthreads();
+    // dZq = dO * act'(Zq), Zq = Gamma Q W0 - S G
+    for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
+      const int s = e / dv, j = e % dv;
+      float y = 0.f;
+      for (int i = 0; i < dk; ++i) y += ldf(Q + qk0 + (tc + s) * dk + i) * W0[i * dv + j];
+      float zq = expf(L[s]) * y;
+      for (int r = 0; r <= s; ++r) zq -= S[s * C + r] * G[r * dv + j];
+      DZQ[e] = ldf(dO + v0 + (tc + s) * dv + j) * act1(d.act, zq);
+    }
+    __syncthreads();
+    // dS = -dZq G^T (causal)
+    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
+      const int s = e / C, r = e % C;
+      float v = 0.f;
+      if (r <= s)
+        for (int j = 0; j < dv; ++j) v -= DZQ[s * dv + j] * G[r * dv + j];
+      DS[e] = v;
+    }
+    // dG = -S^T dZq - diag(u) Y
+    for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
+      const int r = e / dv, j = e % dv;
+      float g = 0.f;
+      for (int s = r; s < C; ++s) g -= S[s * C + r] * DZQ[s * dv + j];
+      g -= eta[r] * expf(LC - L[r]) * Y[e];
+      DG[e] = g;
+    }
+    __syncthreads();
+    // deta_r = sum_s dS_sr P_sr exp(L_s - L_r) - exp(L_C - L_r) Y_r . G_r ;  dZ, dV
+    for (int r = threadIdx.x; r < C; r += blockDim.x) {
+      float acc = 0.f;
+      for (int s = r; s < C; ++s) acc += DS[s * C + r] * S[s * C + r];
+      acc /= eta[r];
+      float yg = 0.f;
+      for (int j = 0; j < dv; ++j) yg += Y[r * dv + j] * G[r * dv + j];
+      deta[r] = acc - expf(LC - L[r]) * yg;
+    }
+    for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
+      const int r = e / dv, j = e % dv;
+      const float z = Z[e], d1 = act1(d.act, z);
+      const float vv = ldf(V + v0 + (tc + r) * dv + j);
+      const float a = d.loss == 0 ? actf(d.act, z) - vv : -vv;
+      const float da = DG[e] * d1;
+      DZ[e] = DG[e] * a * act2(d.act, z) + (d.loss == 0 ? da * d1 : 0.f);
+      stf(&dV[v0 + (tc + r) * dv + j], -da);
+    }
+    __syncthreads();
+    // dQ = diag(Gamma) dZq W0^T + (dS * M) K
+    for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+      const int s = e / dk, i = e % dk;
+      float a1 = 0.f;
+      for (int j = 0; j < dv; ++j) a1 += DZQ[s * dv + j] * W0[i * dv + j];
+      float acc = expf(L[s]) * a1;
+      for (int r = 0; r <= s; ++r)
+        acc += DS[s * C + r] * eta[r] * expf(L[s] - L[r]) * ldf(K + qk0 + (tc + r) * dk + i);
+      stf(&dQ[qk0 + (tc + s) * dk + i], acc);
+    }
+    // dK = (dS * M)^T Q - diag(u) G Wh^T + dZ W0^T
+    for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+      const int r = e / dk, i = e % dk;
+      float acc = 0.f;
+      for (int s = r; s < C; ++s)
+        acc += DS[s * C + r] * eta[r] * expf(L[s] - L[r]) * ldf(Q + qk0 + (tc + s) * dk + i);
+      float gw = 0.f, zw = 0.f;
+      for (int j = 0; j < dv; ++j) {
+        gw += G[r * dv + j] * Wh[i * dv + j];
+        zw += DZ[r * dv + j] * W0[i * dv + j];
+      }
+      acc += -eta[r] * expf(LC - L[r]) * gw + zw;
+      stf(&dK[qk0 + (tc + r) * dk + i], acc);
+    }
+    for (int r = threadIdx.x; r < C; r += blockDim.x)
+      dbeta[(size_t)bh * d.T + tc + r] = deta[r] * eta[r] * (1.f - 0.5f * eta[r]);
+    // dW at the chunk start = Gamma_C Wh + Q^T diag(Gamma) dZq + K^T dZ
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+      const int i = e / dv, j = e % dv;
+      float acc = expf(LC) * Wh[e];
+      for (int s = 0; s < C; ++s)
+        acc += expf(L[s]) * ldf(Q + qk0 + (tc + s) * dk + i) * DZQ[s * dv + j] +
+               ldf(K + qk0 + (tc + s) * dk + i) * DZ[s * dv + j];
+      Wn[e] = acc;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) Wh[e] = Wn[e];
+    __syncthreads();
+  }
+  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) dW0[(size_t)bh * dk * dv + e] = Wh[e];
+}
+
+Dims dims_of(const LayerArgs& a) {
+  return Dims{a.T, a.dk, a.dv, a.C, a.loss, a.act, a.gamma != nullptr, a.lr_bias};
+}
+
+size_t fwd_smem_bytes(const LayerArgs& a) {
+  return sizeof(float) * ((size_t)a.dk * kNvs + (size_t)a.C * kNvs + (size_t)kRows * a.C + 2 * a.C);
+}
+
+}  // namespace
+
+bool simt_supported(const LayerArgs& a) {
+  return a.dk >= 1 && a.dk <= kMaxD && a.dv >= 1 && a.dv <= kMaxD && a.C >= 1 && a.C <= kMaxC;
+}
+
+size_t simt_fwd_workspace(const LayerArgs&) { return 0; }
+
+size_t simt_bwd_workspace(const LayerArgs& a) {
+  return sizeof(float) * bwd_head_floats(a.C, a.dk, a.dv) * a.B * a.H;
+}
+
+cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
+  const Dims d = dims_of(a);
+  const size_t smem = fwd_smem_bytes(a);
+  dim3 grid((a.dv + kNvs - 1) / kNvs, a.B * a.H);
+  if (a.dtype == 0) {
+    auto k = simt_fwd_kernel<float>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 256, smem, s>>>(d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta,
+                              a.gamma, a.W0, (float*)a.O, a.W_final, (float*)a.W_chunks);
+  } else {
+    auto k = simt_fwd_kernel<__nv_bfloat16>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 256, smem, s>>>(d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K,
+                              (const __nv_bfloat16*)a.V, a.beta, a.gamma, a.W0,
+                              (__nv_bfloat16*)a.O, a.W_final, (__nv_bfloat16*)a.W_chunks);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t simt_bwd(const LayerArgs& a, cudaStream_t s) {
+  const Dims d = dims_of(a);
+  if (a.dtype == 0) {
+    simt_bwd_kernel<float><<<a.B * a.H, 512, 0, s>>>(
+        d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta, a.gamma,
+        (const float*)a.W_chunks, (const float*)a.dO, a.dW_final, (float*)a.dQ, (float*)a.dK,
+        (float*)a.dV, a.dbeta, a.dW0, (float*)a.ws);
+  } else {
+    simt_bwd_kernel<__nv_bfloat16><<<a.B * a.H, 512, 0, s>>>(
+        d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K, (const __nv_bfloat16*)a.V,
+        a.beta, a.gamma, (const __nv_bfloat16*)a.W_chunks, (const __nv_bfloat16*)a.dO,
+        a.dW_final, (__nv_bfloat16*)a.dQ, (__nv_bfloat16*)a.dK, (__nv_bfloat16*)a.dV, a.dbeta,
+        a.dW0, (float*)a.ws);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace tttk
