@@ -69,11 +69,9 @@ def oracle_bwd(cfg, inp):
 
 
 def head_slice(inp, heads):
-    """Restrict every per-head tensor to the listed (b, h) pairs (as a batch of 1 x len)."""
+    """The per-head tensors of the listed (b, h) pairs, stacked as B = 1, H = len(heads).
+    Heads evolve independently, so the oracle on this slice is exact for those heads."""
     out = {}
     for k, v in inp.items():
-        if v is None or k == "dW_T" and v is None:
-            out[k] = None
-            continue
-        out[k] = torch.stack([v[b, h] for b, h in heads]).unsqueeze(0)
+        out[k] = None if v is None else torch.stack([v[b, h] for b, h in heads]).unsqueeze(0)
     return out

@@ -1,0 +1,535 @@
+// tcgen05 forward of the chunkwise TTT layer (bf16 operands, fp32 state and accumulators).
+//
+// Page "Modular TTT: Rethinking Test-Time Training as Composable Modules", section
+// "方法步骤详情" (Algorithm 1) with the lr of section "内部学习规则与学习率参数化" and the
+// scalar decay of section "权重衰减". Per chunk of C tokens, with W0 the chunk-start state:
+//   Z   = K W0                          (train view, one MMA per 128-token block)
+//   G   = a(Z) * act'(Z)                (inner-loss gradient; MSE a = act(Z) - V, IP a = -V)
+//   Zq  = diag(Gamma) Q W0 - S G,  S_sr = eta_r exp(L_s - L_r) (q_s . k_r) for r <= s
+//   O   = act(Zq)
+//   W   = Gamma_C W0 - K^T diag(u) G,  u_r = eta_r exp(L_C - L_r)
+//
+// One CTA owns one (batch, head, 64-wide slice of d_v): the columns of W, V, G, Z, Zq and O
+// evolve independently, so d_v = 128 runs as two CTAs per head. The fp32 state lives in TMEM
+// for the whole sequence; a bf16 copy in shared memory is the MMA operand of the next chunk.
+//
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner), warps 2-9 epilogue
+// (two warpgroups; warpgroup g handles value columns [32g, 32g+32) of each 128-row block and
+// score columns [64g, 64g+64) of each 128x128 score block). Every wait is bounded.
+//
+// TMEM columns: [0,64) W (lanes = key features), [64, 64+64NB) Z blocks,
+// [64+64NB, 64+128NB) Y / Zq blocks, [64+128NB, +128) one 128x128 fp32 score block P.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace tttk {
+namespace {
+
+constexpr int NV = 64;             // value columns per CTA
+constexpr int kThreads = 320;      // 10 warps
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t PANEL128 = 128 * 128;  // 128 rows x 128 bytes
+
+struct FwdParams {
+  int BH, T, NC, nslice, loss, act;
+  float lr_bias;
+  const float* beta;
+  const float* gamma;     // nullable
+  const float* W0;        // [BH, D, D] fp32
+  __nv_bfloat16* O;       // [BH, T, D]
+  float* W_final;         // nullable
+  __nv_bfloat16* W_chunks;  // nullable, [BH, NC, D, D]
+  unsigned* err;
+};
+
+template <int D, int NB>
+struct Layout {
+  static constexpr int C = 128 * NB;
+  static constexpr int KP = D / 64;                      // 64-wide key-feature panels
+  static constexpr uint32_t K_PANEL = C * 128;           // one K panel (C rows)
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_Q = OFF_K + KP * K_PANEL;
+  static constexpr uint32_t OFF_V = OFF_Q + KP * PANEL128;  // V slice, overwritten by G
+  static constexpr uint32_t OFF_UG = OFF_V + C * 128;
+  static constexpr uint32_t OFF_W0 = OFF_UG + C * 128;      // bf16 state, MN-major [D][64]
+  static constexpr uint32_t OFF_S = OFF_W0 + D * 128;       // 2 panels of 128 x 64
+  static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;   // float arrays
+  static constexpr uint32_t OFF_BAR = OFF_F + 5 * 256 * 4;
+  static constexpr uint32_t BYTES = OFF_BAR + 256;
+  static constexpr uint32_t KV_TX = KP * K_PANEL + C * 128;
+  static constexpr uint32_t Q_TX = KP * PANEL128;
+  static constexpr int NP = NB * (NB + 1) / 2;            // score blocks per chunk
+  // TMEM columns
+  static constexpr uint32_t T_W = 0, T_Z = 64, T_Y = 64 + 64 * NB, T_P = 64 + 128 * NB;
+};
+
+struct __align__(8) FwdBars {
+  uint64_t kv_full, kv_free, q_full, q_free, z_full, g_ready, y_full, y_scaled, p_full, s_ready,
+      s_free, zq_full, y_free, w_full, w0_ready, scan_full, scan_free;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ float sigm(float x) { return 1.f / (1.f + __expf(-x)); }
+__device__ __forceinline__ float act_f(int act, float z) { return act ? z * sigm(z) : z; }
+__device__ __forceinline__ float act_d1(int act, float z) {
+  if (!act) return 1.f;
+  const float s = sigm(z);
+  return s * (1.f + z * (1.f - s));
+}
+
+// Reads 32 bf16 (16-byte chunks c0..c0+3 of `row`) of a swizzled panel as floats.
+__device__ __forceinline__ void ld_row32(uint32_t panel, int row, int c0, float (&x)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t a, b, c, d;
+    ld_shared_v4(panel + sw128_off(row, c0 + k), a, b, c, d);
+    x[8 * k + 0] = bf16lo(a); x[8 * k + 1] = bf16hi(a);
+    x[8 * k + 2] = bf16lo(b); x[8 * k + 3] = bf16hi(b);
+    x[8 * k + 4] = bf16lo(c); x[8 * k + 5] = bf16hi(c);
+    x[8 * k + 6] = bf16lo(d); x[8 * k + 7] = bf16hi(d);
+  }
+}
+__device__ __forceinline__ void st_row32(uint32_t panel, int row, int c0, const float (&x)[32]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    st_shared_v4(panel + sw128_off(row, c0 + k), pack_bf16x2(x[8 * k], x[8 * k + 1]),
+                 pack_bf16x2(x[8 * k + 2], x[8 * k + 3]), pack_bf16x2(x[8 * k + 4], x[8 * k + 5]),
+                 pack_bf16x2(x[8 * k + 6], x[8 * k + 7]));
+}
+__device__ __forceinline__ void st_global_bf16x32(__nv_bfloat16* dst, const float (&x)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    d[k] = make_uint4(pack_bf16x2(x[8 * k], x[8 * k + 1]), pack_bf16x2(x[8 * k + 2], x[8 * k + 3]),
+                      pack_bf16x2(x[8 * k + 4], x[8 * k + 5]),
+                      pack_bf16x2(x[8 * k + 6], x[8 * k + 7]));
+}
+
+template <int D, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    ttt_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = Layout<D, NB>;
+  constexpr int C = L::C;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sK = sbase + L::OFF_K, sQ = sbase + L::OFF_Q, sV = sbase + L::OFF_V,
+                 sUG = sbase + L::OFF_UG, sW0 = sbase + L::OFF_W0, sS = sbase + L::OFF_S;
+  float* f_eta = reinterpret_cast<float*>(smem + L::OFF_F);  // eta_r
+  float* f_L = f_eta + 256;                                   // L_r (chunk-local log decay)
+  float* f_gam = f_L + 256;                                   // Gamma_r = exp(L_r)
+  float* f_uneg = f_gam + 256;                                // -eta_r exp(L_C - L_r)
+  float* f_cfac = f_uneg + 256;                               // eta_r exp(L_ref(r) - L_r)
+  FwdBars* bars = reinterpret_cast<FwdBars*>(smem + L::OFF_BAR);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.x / p.nslice, slice = blockIdx.x % p.nslice;
+  Abort ab{&bars->abort_flag, p.err};
+#define BAR(x) smem_u32(&bars->x)
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(kv_full), 1);
+    mbar_init(BAR(kv_free), 1);
+    mbar_init(BAR(q_full), 1);
+    mbar_init(BAR(q_free), 1);
+    mbar_init(BAR(z_full), 1);
+    mbar_init(BAR(g_ready), kEpiWarps);
+    mbar_init(BAR(y_full), 1);
+    mbar_init(BAR(y_scaled), kEpiWarps);
+    mbar_init(BAR(p_full), 1);
+    mbar_init(BAR(s_ready), kEpiWarps);
+    mbar_init(BAR(s_free), 1);
+    mbar_init(BAR(zq_full), 1);
+    mbar_init(BAR(y_free), kEpiWarps);
+    mbar_init(BAR(w_full), 1);
+    mbar_init(BAR(w0_ready), kEpiWarps);
+    mbar_init(BAR(scan_full), 1);
+    mbar_init(BAR(scan_free), kEpiWarps);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(BAR(tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int NC = p.NC;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int qk = 0;  // Q half loads issued
+      for (int c = 0; c < NC; ++c) {
+        const int row0 = bh * p.T + c * C;
+        for (int h = 0; h < NB; ++h) {
+          if (qk > 0 && !mbar_wait(BAR(q_free), (qk - 1) & 1, ab)) goto done_prod;
+          mbar_arrive_expect_tx(BAR(q_full), L::Q_TX);
+#pragma unroll
+          for (int kp = 0; kp < L::KP; ++kp)
+            tma_load_2d(sQ + kp * PANEL128, &tmQ, BAR(q_full), 64 * kp, row0 + 128 * h);
+          ++qk;
+          if (h == 0) {
+            if (c > 0 && !mbar_wait(BAR(kv_free), (c - 1) & 1, ab)) goto done_prod;
+            mbar_arrive_expect_tx(BAR(kv_full), L::KV_TX);
+#pragma unroll
+            for (int kp = 0; kp < L::KP; ++kp)
+              tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(kv_full), 64 * kp, row0);
+            tma_load_2d(sV, &tmV, BAR(kv_full), NV * slice, row0);
+          }
+        }
+      }
+    done_prod:;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idZ = idesc_bf16(128, NV, 0, 1);   // K-major A, MN-major B
+      const uint32_t idP = idesc_bf16(128, 128, 0, 0);  // K-major A and B
+      const uint32_t idW = idesc_bf16(128, NV, 1, 1);   // MN-major A and B
+      const uint32_t lboKt = D == 128 ? L::K_PANEL : 0;  // second 64-row block of K^T
+      int kq = 0, ks = 0;
+      for (int c = 0; c < NC; ++c) {
+        if (!mbar_wait(BAR(kv_full), c & 1, ab)) break;
+        if (!mbar_wait(BAR(w0_ready), c & 1, ab)) break;
+        tc_fence_after();
+        // Z_b = K_b W0
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_Z + NV * b,
+                        sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
+        mma_commit(BAR(z_full));
+        bool ok = true;
+        for (int h = 0; h < NB && ok; ++h) {
+          if (!mbar_wait(BAR(q_full), kq & 1, ab)) { ok = false; break; }
+          ++kq;
+          if (h == 0 && c > 0 && !mbar_wait(BAR(y_free), (c - 1) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_Y + NV * h,
+                        sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
+          mma_commit(BAR(y_full));
+          for (int b = 0; b <= h; ++b) {
+#pragma unroll
+            for (int j = 0; j < D / 16; ++j)
+              mma_bf16_ss(tmem + L::T_P,
+                          sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                          sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16,
+                                      1024),
+                          idP, j > 0);
+            mma_commit(BAR(p_full));
+            if (b == h) mma_commit(BAR(q_free));
+            if (h == 0 && b == 0) {
+              // state transition W += K^T (u * -G), W already scaled by Gamma_C
+              if (!mbar_wait(BAR(g_ready), c & 1, ab)) { ok = false; break; }
+              tc_fence_after();
+              for (int j = 0; j < C / 16; ++j)
+                mma_bf16_ss(tmem + L::T_W, sdesc_sw128(sK + j * 2048, lboKt, 1024),
+                            sdesc_sw128(sUG + j * 2048, 0, 1024), idW, 1);
+              mma_commit(BAR(w_full));
+            }
+            if (!mbar_wait(BAR(s_ready), ks & 1, ab)) { ok = false; break; }
+            if (b == 0 && !mbar_wait(BAR(y_scaled), (c * NB + h) & 1, ab)) { ok = false; break; }
+            ++ks;
+            tc_fence_after();
+            // Zq_h += (-S_hb) G_b
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              mma_bf16_ss(tmem + L::T_Y + NV * h,
+                          sdesc_sw128(sS + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                          sdesc_sw128(sV + b * PANEL128 + j * 2048, 0, 1024), idZ, 1);
+            mma_commit(BAR(s_free));
+          }
+          if (ok) mma_commit(BAR(zq_full));
+        }
+        if (!ok) break;
+        mma_commit(BAR(kv_free));
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int ew = warp - 2;          // 0..7
+    const int g = ew / 4;             // warpgroup: value columns [32g, 32g+32)
+    const int q = warp & 3;           // TMEM lane quadrant
+    const int lrow = q * 32 + lane;   // TMEM lane = row inside a 128-row block
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool w_rows = q * 32 < D;   // this warp holds state rows
+    const size_t wofs = (size_t)bh * D * D + (size_t)lrow * D + NV * slice + 32 * g;
+    bool ok = true;
+    // initial state: fp32 into TMEM, bf16 operand copy, chunk-0 checkpoint
+    if (w_rows) {
+      float w[32];
+      const float4* src = reinterpret_cast<const float4*>(p.W0 + wofs);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float4 v = src[k];
+        w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+      }
+      tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
+      tmem_wait_st();
+      st_row32(sW0, lrow, 4 * g, w);
+      if (p.W_chunks)
+        st_global_bf16x32(p.W_chunks + (size_t)bh * NC * D * D + (size_t)lrow * D + NV * slice + 32 * g, w);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(w0_ready));
+
+    int kp = 0;  // score blocks consumed
+    for (int c = 0; c < NC && ok; ++c) {
+      const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
+      // -------- per-chunk scans (warp 2): eta, L, Gamma, -u, column factors
+      if (ew == 0) {
+        if (c > 0 && !mbar_wait(BAR(scan_free), (c - 1) & 1, ab)) { ok = false; break; }
+        constexpr int PER = C / 32;
+        float lg[PER];
+        float run = 0.f;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int r = lane * PER + k;
+          const float gmm = p.gamma ? p.gamma[tok0 + r] : 1.f;
+          run += p.gamma ? __logf(gmm) : 0.f;
+          lg[k] = run;
+          f_eta[r] = 2.f * sigm(p.beta[tok0 + r] + p.lr_bias);
+        }
+        float incl = run;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const float o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        const float excl = incl - run;
+        const float LC = __shfl_sync(0xffffffffu, incl, 31);
+#pragma unroll
+        for (int k = 0; k < PER; ++k) f_L[lane * PER + k] = lg[k] + excl;
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int r = lane * PER + k;
+          const float Lr = f_L[r];
+          const float eta = f_eta[r];
+          f_gam[r] = __expf(Lr);
+          f_uneg[r] = -eta * __expf(LC - Lr);
+          f_cfac[r] = eta * __expf(f_L[r | 63] - Lr);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(scan_full));
+      }
+      if (!mbar_wait(BAR(scan_full), c & 1, ab)) { ok = false; break; }
+      const float gamC = f_gam[C - 1];
+
+      // -------- train view: G = a(Z) act'(Z) in place over V, -u*G, state decay
+      if (!mbar_wait(BAR(kv_full), c & 1, ab)) { ok = false; break; }
+      if (!mbar_wait(BAR(z_full), c & 1, ab)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      for (int b = 0; b < NB; ++b) {
+        float z[32], v[32];
+        tmem_ld32(tmem + lane_off + L::T_Z + NV * b + 32 * g, z);
+        tmem_wait_ld();
+        const int row = 128 * b + lrow;
+        ld_row32(sV, row, 4 * g, v);
+        const float un = f_uneg[row];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float a = p.loss == 0 ? act_f(p.act, z[j]) - v[j] : -v[j];
+          const float gg = a * act_d1(p.act, z[j]);
+          v[j] = gg;
+          z[j] = un * gg;
+        }
+        st_row32(sV, row, 4 * g, v);
+        st_row32(sUG, row, 4 * g, z);
+      }
+      if (w_rows) {
+        float w[32];
+        tmem_ld32(tmem + lane_off + L::T_W + 32 * g, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] *= gamC;
+        tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
+        tmem_wait_st();
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(g_ready));
+
+      for (int h = 0; h < NB && ok; ++h) {
+        const int srow = 128 * h + lrow;  // chunk-local query index of this thread
+        // Y_h *= Gamma_s
+        if (!mbar_wait(BAR(y_full), (c * NB + h) & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        {
+          float y[32];
+          tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
+          tmem_wait_ld();
+          const float gs = f_gam[srow];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] *= gs;
+          tmem_st32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(y_scaled));
+
+        if (h == NB - 1) {
+          // -------- state copy for the next chunk: after the transition MMA and after the
+          // last MMA that reads the current bf16 copy (Y of this block, complete above)
+          if (!mbar_wait(BAR(w_full), c & 1, ab)) { ok = false; break; }
+          __syncwarp();
+          tc_fence_after();
+          if (w_rows) {
+            float w[32];
+            tmem_ld32(tmem + lane_off + L::T_W + 32 * g, w);
+            tmem_wait_ld();
+            if (c + 1 < NC) {
+              st_row32(sW0, lrow, 4 * g, w);
+              if (p.W_chunks)
+                st_global_bf16x32(p.W_chunks + ((size_t)bh * NC + c + 1) * D * D +
+                                      (size_t)lrow * D + NV * slice + 32 * g, w);
+            } else if (p.W_final) {
+              float4* dst = reinterpret_cast<float4*>(p.W_final + wofs);
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                dst[k] = make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            }
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(w0_ready));
+        }
+
+        const float Ls = f_L[srow];
+        for (int b = 0; b <= h; ++b) {
+          if (!mbar_wait(BAR(p_full), kp & 1, ab)) { ok = false; break; }
+          if (kp > 0 && !mbar_wait(BAR(s_free), (kp - 1) & 1, ab)) { ok = false; break; }
+          ++kp;
+          __syncwarp();
+          tc_fence_after();
+          const int r0 = 128 * b + 64 * g;  // first key of this thread's 64 columns
+          const int rlast = r0 + 63;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float s[32];
+            tmem_ld32(tmem + lane_off + L::T_P + 64 * g + 32 * half, s);
+            tmem_wait_ld();
+            const int rb = r0 + 32 * half;
+            if (rlast <= srow) {
+              // every key precedes the query: exp(L_s - L_r) = exp(L_s - L_last) * exp(L_last - L_r)
+              const float as = __expf(Ls - f_L[rlast]);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) s[j] = -s[j] * as * f_cfac[rb + j];
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int r = rb + j;
+                s[j] = r <= srow ? -s[j] * f_eta[r] * __expf(Ls - f_L[r]) : 0.f;
+              }
+            }
+            st_row32(sS + g * PANEL128, lrow, 4 * half, s);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(s_ready));
+        }
+        if (!ok) break;
+        if (h == NB - 1) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(scan_free));
+        }
+        // -------- O_h = act(Zq_h)
+        if (!mbar_wait(BAR(zq_full), (c * NB + h) & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        {
+          float o[32];
+          tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[j] = act_f(p.act, o[j]);
+          st_global_bf16x32(p.O + (tok0 + srow) * D + NV * slice + 32 * g, o);
+        }
+      }
+      if (!ok) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(y_free));
+    }
+  }
+#undef BAR
+  tc_fence_before();
+  __syncthreads();
+  if (bars->abort_flag) __nanosleep(100000);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, int NB>
+cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
+  using L = Layout<D, NB>;
+  const uint64_t rows = (uint64_t)a.B * a.H * a.T;
+  CUtensorMap tk, tq, tv;
+  if (!make_tmap_bf16(&tk, a.K, D, rows, D, 64, L::C) ||
+      !make_tmap_bf16(&tq, a.Q, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tv, a.V, D, rows, D, 64, L::C))
+    return cudaErrorInvalidValue;
+  FwdParams p{};
+  p.BH = a.B * a.H;
+  p.T = a.T;
+  p.NC = a.T / a.C;
+  p.nslice = D / NV;
+  p.loss = a.loss;
+  p.act = a.act;
+  p.lr_bias = a.lr_bias;
+  p.beta = a.beta;
+  p.gamma = a.gamma;
+  p.W0 = a.W0;
+  p.O = static_cast<__nv_bfloat16*>(a.O);
+  p.W_final = a.W_final;
+  p.W_chunks = static_cast<__nv_bfloat16*>(a.W_chunks);
+  p.err = a.err;
+  const size_t smem = L::BYTES + 1024;
+  auto k = ttt_fwd_tc_kernel<D, NB>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_fwd_supported(const LayerArgs& a) {
+  return a.dtype == 1 && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
+         (a.C == 128 || a.C == 256) && a.T % a.C == 0;
+}
+
+size_t tc_fwd_workspace(const LayerArgs&) { return 0; }
+
+cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s) {
+  if (a.dk == 64) return a.C == 128 ? launch<64, 1>(a, s) : launch<64, 2>(a, s);
+  return a.C == 128 ? launch<128, 1>(a, s) : launch<128, 2>(a, s);
+}
+
+}  // namespace tttk
