@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the chunkwise TTT layer hot path on B200.
+
+One step = ttt_chunk_fwd (saving the chunk-start states) + ttt_chunk_bwd over one batch of
+the 1.45B-shaped training workload (B=4, H=16, T=4096, d_k=d_v=128, C=256, MSE loss, scalar
+decay, bf16 storage, fp32 state), inputs resident in HBM. The In-Place TTT forward
+(T=32768, d_ff=9728, d_model=2560, C=1024) is timed beside it and reported under "inplace".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun (N > 1) every rank runs its own replica of the workload (the layer has no
+exchange step on one sequence batch; weak scaling), timed on the device with CUDA events
+and reduced as the max over ranks. Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "TTT layer fwd(+bwd) tokens/sec on 1 B200; % of bf16 tensor-core peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------- algorithmic work
+def layer_work(cfg):
+    """Algorithmic flops and bytes of one forward and one backward launch.
+
+    flops per chunk per head: fwd 6 C dk dv + C(C+1)(dk+dv), bwd 12 C dk dv + 2 C(C+1)(dk+dv)
+    (causal half of the C x C products, diagonal included; recomputation not counted).
+    bytes: every input read once and every output written once; the saved chunk-start
+    states are an implementation cost and not counted.
+    """
+    B, H, T, dk, dv, C = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C
+    units = B * H * (T // C)
+    fl_f = units * (6 * C * dk * dv + C * (C + 1) * (dk + dv))
+    fl_b = units * (12 * C * dk * dv + 2 * C * (C + 1) * (dk + dv))
+    e = 2 if cfg.dtype == "bf16" else 4
+    tok = B * H * T
+    by_f = tok * (2 * dk + dv) * e + tok * 4 * (2 if cfg.decay else 1) + 2 * B * H * dk * dv * 4 + tok * dv * e
+    by_b = (tok * (2 * dk + 2 * dv) * e + tok * 4 * (2 if cfg.decay else 1) + B * H * dk * dv * 4
+            + tok * (2 * dk + dv) * e + tok * 4 + B * H * dk * dv * 4)
+    return dict(fwd_flops=fl_f, bwd_flops=fl_b, fwd_bytes=by_f, bwd_bytes=by_b)
+
+
+def inplace_work(icfg):
+    flops = 4 * icfg.d_ff * icfg.d_model * icfg.T
+    byts = icfg.T * (icfg.d_ff + icfg.d_model) * 2 + 2 * icfg.d_model * icfg.d_ff * 4 + icfg.T * icfg.d_model * 2
+    return flops, byts
+
+
+# ------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        props = torch.cuda.get_device_properties(device)
+        self.bus = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.bus}", f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[4], hwt=parts[5], swt=parts[6], pcap=parts[7]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        busy = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in busy:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": busy[0]["smax"],
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(busy)}
+
+
+# ----------------------------------------------------------------------------- the step
+class Layer:
+    """Device buffers and the fwd+bwd step through the C ABI binding."""
+
+    def __init__(self, cfg, ttt, seed):
+        self.cfg, self.ttt = cfg, ttt
+        self.inp = synth.ttt_inputs(cfg, device="cuda", seed=seed)
+        B, H, T, dk, dv, C = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C
+        sd = synth.storage_dtype(cfg)
+        dev = "cuda"
+        self.c = ttt.make_config(B, H, T, dk, dv, C, cfg.dtype, cfg.loss, cfg.act, cfg.lr_bias)
+        self.O = torch.empty((B, H, T, dv), device=dev, dtype=sd)
+        self.Wf = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
+        self.Wc = torch.empty((B, H, T // C, dk, dv), device=dev, dtype=sd)
+        self.dQ = torch.empty((B, H, T, dk), device=dev, dtype=sd)
+        self.dK = torch.empty((B, H, T, dk), device=dev, dtype=sd)
+        self.dV = torch.empty((B, H, T, dv), device=dev, dtype=sd)
+        self.dbeta = torch.empty((B, H, T), device=dev, dtype=torch.float32)
+        self.dW0 = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
+        self.nf = ttt.ttt_workspace_bytes(self.c, False)
+        self.nb = ttt.ttt_workspace_bytes(self.c, True)
+        self.ws = torch.empty(max(self.nf, self.nb, 16), device=dev, dtype=torch.uint8)
+
+    def fwd(self):
+        i = self.inp
+        self.ttt.ttt_chunk_fwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
+                               self.O, self.Wf, self.Wc, self.ws, self.nf)
+
+    def bwd(self):
+        i = self.inp
+        self.ttt.ttt_chunk_bwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
+                               self.Wc, i["dO"], i["dW_T"], self.dQ, self.dK, self.dV, self.dbeta,
+                               self.dW0, self.ws, self.nb)
+
+
+def time_steps(layer, steps, warmup, sampler=None):
+    """Device time of `steps` fwd+bwd steps; events around every launch for per-kernel times."""
+    for _ in range(warmup):
+        layer.fwd()
+        layer.bwd()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n0 = layer.ttt.ttt_kernel_launches()
+    if sampler:
+        sampler.mark("t0")
+    barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for a, b, c in ev:
+        a.record()
+        layer.fwd()
+        b.record()
+        layer.bwd()
+        c.record()
+    end.record()
+    torch.cuda.synchronize()
+    barrier()
+    if sampler:
+        sampler.mark("t1")
+    launches = layer.ttt.ttt_kernel_launches() - n0
+    total = start.elapsed_time(end)
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in ev)
+    bwd_ms = statistics.mean(b.elapsed_time(c) for _, b, c in ev)
+    return total, fwd_ms, bwd_ms, launches
+
+
+def time_e2e(layer, steps, warmup):
+    """Same step through the binding with the inputs in pinned HOST memory: every step copies
+    the inputs host->device and the gradients device->host inside the timed region."""
+    i = layer.inp
+    names_in = ["Q", "K", "V", "dO", "beta", "gamma", "W0"]
+    host_in = {k: i[k].to("cpu").pin_memory() for k in names_in if i[k] is not None}
+    outs = {"dQ": layer.dQ, "dK": layer.dK, "dV": layer.dV, "dbeta": layer.dbeta, "dW0": layer.dW0}
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def step():
+        for k, t in host_in.items():
+            i[k].copy_(t, non_blocking=True)
+        layer.fwd()
+        layer.bwd()
+        for k, t in outs.items():
+            host_out[k].copy_(t, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    barrier()
+    return s.elapsed_time(e), h2d, d2h
+
+
+def time_inplace(ttt, steps, warmup):
+    icfg = synth.INPLACE_QWEN4B
+    inp = synth.inplace_inputs(icfg, device="cuda")
+    W = inp["W"].clone()
+    O = torch.empty((icfg.T, icfg.d_model), device="cuda", dtype=torch.bfloat16)
+    n = ttt.inplace_ttt_workspace_bytes(icfg.T, icfg.d_ff, icfg.d_model, icfg.C)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+
+    def run():
+        W.copy_(inp["W"])
+        ttt.inplace_ttt_fwd(icfg.T, icfg.d_ff, icfg.d_model, icfg.C, icfg.lr, inp["Z"], inp["Vhat"],
+                            W, O, ws, n)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        W.copy_(inp["W"])
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        ttt.inplace_ttt_fwd(icfg.T, icfg.d_ff, icfg.d_model, icfg.C, icfg.lr, inp["Z"], inp["Vhat"],
+                            W, O, ws, n)
+        b.record()
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    return icfg, ms
+
+
+# --------------------------------------------------------------------------- oracle legs
+def cpu_oracle_step(cfg, inp_cpu, nthreads):
+    """The oracle as it stands: forward with the fp32-state build, backward in fp64."""
+    import oracle
+    b32 = float(torch.tensor(cfg.lr_bias, dtype=torch.float32))
+    t0 = time.perf_counter()
+    _, _, _, used = oracle.ttt_fwd(inp_cpu["Q"], inp_cpu["K"], inp_cpu["V"], inp_cpu["beta"],
+                                   inp_cpu["gamma"], inp_cpu["W0"], C=cfg.C, loss=cfg.loss,
+                                   act=cfg.act, lr_bias=b32, state="f32", nthreads=nthreads)
+    oracle.ttt_bwd(inp_cpu["Q"], inp_cpu["K"], inp_cpu["V"], inp_cpu["beta"], inp_cpu["gamma"],
+                   inp_cpu["W0"], inp_cpu["dO"], inp_cpu["dW_T"], C=cfg.C, loss=cfg.loss,
+                   act=cfg.act, lr_bias=b32, nthreads=nthreads)
+    return time.perf_counter() - t0, used
+
+
+def cpu_sample(cfg, batches):
+    scfg = cfg.replace(B=batches)
+    return scfg, synth.ttt_inputs(scfg, device="cpu")
+
+
+def cpu_baseline(cfg, batches=2):
+    scfg, inp = cpu_sample(cfg, batches)
+    secs, used = cpu_oracle_step(scfg, inp, os.cpu_count() or 1)
+    return {"value": scfg.B * scfg.T / secs, "unit": "tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{scfg.B} of {cfg.B} sequences (all {cfg.H} heads, T={cfg.T}) fwd "
+                      f"(fp32-state oracle) + bwd (fp64 oracle), {secs:.1f} s"}
+
+
+# ---------------------------------------------------------------------------- distributed
+_dist = None
+
+
+def barrier():
+    if _dist is not None:
+        _dist.barrier()
+
+
+def reduce_max(x: float) -> float:
+    if _dist is None:
+        return x
+    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    _dist.all_reduce(t, op=_dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    global _dist
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-inplace", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = synth.TRAIN_1P45B
+    config = {"workload": cfg.name, "B": cfg.B, "H": cfg.H, "T": cfg.T, "dk": cfg.dk, "dv": cfg.dv,
+              "C": cfg.C, "loss": cfg.loss, "act": cfg.act, "decay": "scalar",
+              "parallelism": f"replicas x{world}",
+              "l2": "inputs larger than L2 (Q,K,V,dO = 268 MB per step)"}
+
+    if args.impl == "reference":
+        # The oracle on the host cores: rank 0 only; other ranks exit without work.
+        if rank != 0:
+            return
+        scfg, inp = cpu_sample(cfg, 1)
+        for _ in range(args.warmup):
+            cpu_oracle_step(scfg, inp, os.cpu_count() or 1)
+        secs, used = 0.0, 1
+        for _ in range(args.steps):
+            s, used = cpu_oracle_step(scfg, inp, os.cpu_count() or 1)
+            secs += s
+        val = args.steps * scfg.B * scfg.T / secs
+        print(json.dumps({
+            "impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32/f64",
+            "data": "synthetic", "config": config,
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": used, "kind": "oracle",
+                             "sample": f"1 of {cfg.B} sequences (all heads) per step"},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }))
+        return
+
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        _dist = dist
+    else:
+        torch.cuda.set_device(0)
+    import weight_sequence_layers_b200 as ttt
+
+    peaks, peak_src = load_peaks()
+    layer = Layer(cfg, ttt, seed=cfg.seed + rank)
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    total_ms, fwd_ms, bwd_ms, launches = time_steps(layer, args.steps, args.warmup, sampler)
+    clocks = sampler.stop() if sampler else None
+    assert ttt.ttt_get_device_error() == ttt.OK
+    total_ms = reduce_max(total_ms)
+    ms_step = total_ms / args.steps
+    tokens = cfg.B * cfg.T * world
+    value = tokens / (ms_step * 1e-3)
+
+    work = layer_work(cfg)
+    dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
+    dom_ms = bwd_ms if dom == "bwd" else fwd_ms
+    dom_bytes = work[f"{dom}_bytes"]
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "kernel": f"ttt_chunk_{dom}", "peak_source": peak_src}
+    step_flops = work["fwd_flops"] + work["bwd_flops"]
+    tc_frac = step_flops / (ms_step * 1e-3) / (peaks["bf16_tflops"] * 1e12)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config, "roofline": roofline,
+        "tc_frac_of_bf16_peak": tc_frac,
+        "kernels_ms": {"ttt_chunk_fwd": fwd_ms, "ttt_chunk_bwd": bwd_ms},
+        "gpu_launches": launches, "clocks": clocks,
+    }
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(layer, args.steps, args.warmup)
+        e2e_ms = reduce_max(e2e_ms)
+        out["e2e"] = {"value": tokens / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del layer
+    torch.cuda.empty_cache()
+    if not args.no_inplace:
+        icfg, ims = time_inplace(ttt, steps=3, warmup=1)
+        fl, by = inplace_work(icfg)
+        tf = fl / (ims * 1e-3) / 1e12
+        out["inplace"] = {"workload": icfg.name, "ms": ims, "tokens_per_s": icfg.T / (ims * 1e-3),
+                          "roofline": {"bound": "tensor", "achieved": tf,
+                                       "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                                       "frac": tf / peaks["bf16_tflops_sustained"]}}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(cfg)
+    if _dist is not None:
+        _dist.barrier()
+        _dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

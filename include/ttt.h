@@ -132,6 +132,10 @@ ttt_status ttt_get_device_error(void* stream);
  * Used to test the failure path without faulting the GPU. */
 ttt_status ttt_selftest_bounded_wait(unsigned spin_limit, void* stream);
 
+/* Number of kernels this library has launched in this process (all devices, all entry
+ * points) since it was loaded. Lets a caller check what ran without a profiler. */
+unsigned long long ttt_kernel_launches(void);
+
 /* Static description of a status code. */
 const char* ttt_status_string(ttt_status s);
 

@@ -51,6 +51,7 @@ _SIGS = {
     "ttt_get_device_error": ([_p], _i),
     "ttt_selftest_bounded_wait": ([_u, _p], _i),
     "ttt_status_string": ([_i], ctypes.c_char_p),
+    "ttt_kernel_launches": ([], ctypes.c_ulonglong),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -140,6 +141,10 @@ def ttt_get_device_error(stream=None) -> int:
 
 def ttt_selftest_bounded_wait(spin_limit: int, stream=None):
     _check(_lib.ttt_selftest_bounded_wait(int(spin_limit), _stream(stream)), "ttt_selftest_bounded_wait")
+
+
+def ttt_kernel_launches() -> int:
+    return int(_lib.ttt_kernel_launches())
 
 
 # Raw C entry points (for callers that marshal pointers themselves).

@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/ttt.h"
@@ -122,6 +123,9 @@ __global__ void selftest_wait_kernel(unsigned spin_limit, unsigned* err) {
 }
 
 }  // namespace
+
+std::atomic<unsigned long long> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_rows) {
@@ -272,11 +276,14 @@ ttt_status ttt_get_device_error(void* stream) {
   return TTT_OK;
 }
 
+unsigned long long ttt_kernel_launches(void) { return g_launches.load(); }
+
 ttt_status ttt_selftest_bounded_wait(unsigned spin_limit, void* stream) {
   cudaError_t e;
   unsigned* err = error_word(&e);
   if (!err) return TTT_ERR_CUDA;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(spin_limit, err);
+  count_launches(1);
   return launch_status(cudaGetLastError());
 }
 

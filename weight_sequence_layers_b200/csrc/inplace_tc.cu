@@ -324,6 +324,7 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
     p.counter = counters + i;
     inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, twb, tvh, p);
   }
+  count_launches(NC + 1);
   return cudaGetLastError();
 }
 

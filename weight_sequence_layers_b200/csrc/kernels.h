@@ -44,6 +44,9 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
                         const void* Vhat, float* W, void* O, void* ws, unsigned* err,
                         cudaStream_t s);
 
+// Adds n to the process-wide count of kernel launches (reported by ttt_kernel_launches).
+void count_launches(int n);
+
 // 2-D bf16 tensor map with 128-byte swizzle: `rows` rows of `inner` elements, rows
 // `row_stride_elems` apart; box = {box_inner (64), box_rows}. Returns false on failure.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,

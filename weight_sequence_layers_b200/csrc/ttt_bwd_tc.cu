@@ -1,9 +1,885 @@
-// tcgen05 backward of the chunkwise TTT layer (bf16 storage, fp32 state).
+// tcgen05 analytic backward of the chunkwise TTT layer (identity activation, MSE or
+// inner-product inner loss, scalar decay; bf16 operands, fp32 accumulators and states).
+//
+// Forward per chunk (page "Modular TTT: Rethinking Test-Time Training as Composable
+// Modules", section "方法步骤详情"): Z = K W0, G = Z - V (MSE) or -V (IP),
+// O = diag(Gamma) Q W0 - S G with S = (Q K^T) * M, M_sr = eta_r exp(L_s - L_r) (r <= s),
+// W_end = Gamma_C W0 - K^T diag(u) G, u_r = eta_r exp(L_C - L_r).
+// For J = <dO, O> + <dW_T, W_T>, with dW the adjoint of the state at the chunk end:
+//   X  = S^T dO,  Y = K dW,  dG = -X - diag(u) Y,  dV = -dG,  dZ = dG (MSE) or 0 (IP)
+//   dW_start = Gamma_C dW + Q^T diag(Gamma) dO + K^T dZ                (carried to chunk c-1)
+//   dS = -dO G^T (causal),  dP = dS * M
+//   dQ = diag(Gamma) dO W0^T + dP K
+//   dK = dP^T Q - diag(u) G dW^T + dZ W0^T
+//   deta_r = sum_s dS_sr P_sr exp(L_s - L_r) - exp(L_C - L_r) K_r . (G_r dW^T)
+//   dbeta = deta * eta (1 - eta / 2)
+//
+// Three kernels:
+//   chain : one CTA per (batch, head, 64-wide value slice) walks the chunks backwards with
+//           dW (fp32) resident in TMEM, writing dV, dW0 and the bf16 adjoint at the end of
+//           every chunk (workspace). Columns of dW, X, Y, dG, dV are independent.
+//   dk    : one CTA per (batch, head, chunk, 128-key block): dK and dbeta of those keys.
+//   dq    : one CTA per (batch, head, chunk, 128-query block): dQ of those queries.
+// The two chunk-parallel kernels recompute G and the score blocks from the saved chunk-start
+// state and hold dP (bf16) in TMEM as the A operand of their last contraction.
+#include <cuda_bf16.h>
+#include <math.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_util.cuh"
 
 namespace tttk {
-bool tc_bwd_supported(const LayerArgs&) { return false; }
-size_t tc_bwd_workspace(const LayerArgs&) { return 0; }
-cudaError_t tc_bwd(const LayerArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int NV = 64;
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t PANEL128 = 128 * 128;
+
+struct BwdParams {
+  int BH, T, NC, nslice, loss;
+  float lr_bias;
+  const float* beta;
+  const float* gamma;
+  const float* dW_final;      // nullable
+  __nv_bfloat16* dV;          // chain: out; dk: in (dZ = -dV for MSE)
+  float* dW0;
+  __nv_bfloat16* dWs;         // [BH, NC, D, D] adjoint at the end of each chunk
+  __nv_bfloat16* dQ;
+  __nv_bfloat16* dK;
+  float* dbeta;
+  unsigned* err;
+};
+
+struct __align__(8) Bars {
+  uint64_t b[20];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+#define BAR(i) smem_u32(&bars->b[i])
+
+__device__ __forceinline__ void setup(Bars* bars, const int* counts, int n, uint32_t& tmem) {
+  const int warp = threadIdx.x / 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < n; ++i) mbar_init(BAR(i), counts[i]);
+    bars->abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  tmem = bars->tmem_base;
+}
+
+__device__ __forceinline__ void teardown(Bars* bars, uint32_t tmem) {
+  tc_fence_before();
+  __syncthreads();
+  if (bars->abort_flag) __nanosleep(100000);
+  if (threadIdx.x / 32 == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Epilogue warps signal an mbarrier once per warp after their shared/TMEM writes.
+__device__ __forceinline__ void epi_arrive(uint32_t bar) {
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// =============================================================================== chain
+template <int D, int NB>
+struct ChainL {
+  static constexpr int C = 128 * NB, KP = D / 64;
+  static constexpr uint32_t K_PANEL = C * 128;
+  static constexpr uint32_t OFF_K = 0, OFF_Q = KP * K_PANEL, OFF_DO = 2 * KP * K_PANEL;
+  static constexpr uint32_t OFF_DW = OFF_DO + C * 128;   // bf16 adjoint, MN-major [D][64]
+  static constexpr uint32_t OFF_S = OFF_DW + D * 128;    // S^T blocks, then dZ (C rows)
+  static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;
+  static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
+  static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
+  static constexpr uint32_t TX = 2 * KP * K_PANEL + C * 128;
+  static constexpr uint32_t T_DW = 0, T_X = 64, T_Y = 64 + 64 * NB, T_P = 64 + 128 * NB;
+};
+enum { C_KV_FULL, C_KV_FREE, C_P_FULL, C_S_READY, C_S_FREE, C_X_FULL, C_W_READY, C_Y_FULL,
+       C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_NBARS };
+
+template <int D, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_chain_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+  using L = ChainL<D, NB>;
+  constexpr int C = L::C;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb0 = smem_u32(smem);
+  const uint32_t sK = sb0 + L::OFF_K, sQ = sb0 + L::OFF_Q, sDO = sb0 + L::OFF_DO,
+                 sDW = sb0 + L::OFF_DW, sS = sb0 + L::OFF_S;
+  float* f = reinterpret_cast<float*>(smem + L::OFF_F);
+  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cfac = f + 1024,
+        *f_cfacT = f + 1280;
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.x / p.nslice, slice = blockIdx.x % p.nslice;
+  const int NC = p.NC;
+  const bool mse = p.loss == 0;
+  const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
+                               kEpiWarps};
+  uint32_t tmem;
+  setup(bars, counts, C_NBARS, tmem);
+  Abort ab{&bars->abort_flag, p.err};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int it = 0; it < NC; ++it) {
+        const int c = NC - 1 - it;
+        const int row0 = bh * p.T + c * C;
+        if (it > 0 && !mbar_wait(BAR(C_KV_FREE), (it - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(BAR(C_KV_FULL), L::TX);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp) {
+          tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(C_KV_FULL), 64 * kp, row0);
+          tma_load_2d(sQ + kp * L::K_PANEL, &tmQ, BAR(C_KV_FULL), 64 * kp, row0);
+        }
+        tma_load_2d(sDO, &tmDO, BAR(C_KV_FULL), NV * slice, row0);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idP = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idX = idesc_bf16(128, NV, 0, 1);
+      const uint32_t idW = idesc_bf16(128, NV, 1, 1);
+      const uint32_t lboT = D == 128 ? L::K_PANEL : 0;
+      int kp = 0;
+      for (int it = 0; it < NC; ++it) {
+        if (!mbar_wait(BAR(C_KV_FULL), it & 1, ab)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int rb = 0; rb < NB && ok; ++rb)
+          for (int sb = rb; sb < NB; ++sb) {
+            // P^T block = K_rb Q_sb^T
+#pragma unroll
+            for (int j = 0; j < D / 16; ++j)
+              mma_bf16_ss(tmem + L::T_P,
+                          sdesc_sw128(sK + (j / 4) * L::K_PANEL + rb * PANEL128 + (j % 4) * 32, 16, 1024),
+                          sdesc_sw128(sQ + (j / 4) * L::K_PANEL + sb * PANEL128 + (j % 4) * 32, 16, 1024),
+                          idP, j > 0);
+            mma_commit(BAR(C_P_FULL));
+            if (!mbar_wait(BAR(C_S_READY), kp & 1, ab)) { ok = false; break; }
+            ++kp;
+            tc_fence_after();
+            // X_rb += S^T_(rb,sb) dO_sb
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              mma_bf16_ss(tmem + L::T_X + NV * rb,
+                          sdesc_sw128(sS + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                          sdesc_sw128(sDO + sb * PANEL128 + j * 2048, 0, 1024), idX,
+                          (sb != rb) || (j > 0));
+            mma_commit(BAR(C_S_FREE));
+          }
+        if (!ok) break;
+        mma_commit(BAR(C_X_FULL));
+        // Y_b = K_b dW
+        if (!mbar_wait(BAR(C_W_READY), it & 1, ab)) break;
+        tc_fence_after();
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_Y + NV * b,
+                        sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sDW + j * 2048, 0, 1024), idX, j > 0);
+        mma_commit(BAR(C_Y_FULL));
+        // dW (already Gamma_C-scaled) += (Gamma Q)^T dO + K^T dZ
+        if (!mbar_wait(BAR(C_QS_READY), it & 1, ab)) break;
+        tc_fence_after();
+        for (int j = 0; j < C / 16; ++j)
+          mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sQ + j * 2048, lboT, 1024),
+                      sdesc_sw128(sDO + j * 2048, 0, 1024), idW, 1);
+        if (!mbar_wait(BAR(C_DZ_READY), it & 1, ab)) break;
+        tc_fence_after();
+        if (mse)
+          for (int j = 0; j < C / 16; ++j)
+            mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sK + j * 2048, lboT, 1024),
+                        sdesc_sw128(sS + j * 2048, 0, 1024), idW, 1);
+        mma_commit(BAR(C_DW_FULL));
+        mma_commit(BAR(C_KV_FREE));
+      }
+    }
+  } else {
+    const int ew = warp - 2, g = ew / 4, q = warp & 3, lrow = q * 32 + lane;
+    const uint32_t loff = (uint32_t)(q * 32) << 16;
+    const bool w_rows = q * 32 < D;
+    const size_t wcol = (size_t)lrow * D + NV * slice + 32 * g;
+    bool ok = true;
+    if (w_rows) {
+      float w[32];
+      if (p.dW_final) {
+        const float4* src = reinterpret_cast<const float4*>(p.dW_final + (size_t)bh * D * D + wcol);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float4 v = src[k];
+          w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) w[k] = 0.f;
+      }
+      tmem_st32(tmem + loff + L::T_DW + 32 * g, w);
+      tmem_wait_st();
+      st_row32(sDW, lrow, 4 * g, w);
+      st_global_bf16x32(p.dWs + ((size_t)bh * NC + NC - 1) * D * D + wcol, w);
+    }
+    epi_arrive(BAR(C_W_READY));
+    int kp = 0;
+    for (int it = 0; it < NC && ok; ++it) {
+      const int c = NC - 1 - it;
+      const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
+      if (ew == 0) {
+        if (it > 0 && !mbar_wait(BAR(C_SCAN_FREE), (it - 1) & 1, ab)) { ok = false; break; }
+        chunk_scan_warp<C>(p.beta, p.gamma, tok0, p.lr_bias, f_eta, f_L, f_gam, f_eLC, f_cfac,
+                           f_cfacT);
+        if (lane == 0) mbar_arrive(BAR(C_SCAN_FULL));
+      }
+      if (!mbar_wait(BAR(C_SCAN_FULL), it & 1, ab)) { ok = false; break; }
+      // ---- S^T blocks: S^T_rs = P^T_rs eta_r exp(L_s - L_r), s >= r
+      for (int rb = 0; rb < NB && ok; ++rb) {
+        const int r = 128 * rb + lrow;
+        const float Lr = f_L[r], er = f_eta[r];
+        for (int sb = rb; sb < NB; ++sb) {
+          if (!mbar_wait(BAR(C_P_FULL), kp & 1, ab)) { ok = false; break; }
+          if (kp > 0 && !mbar_wait(BAR(C_S_FREE), (kp - 1) & 1, ab)) { ok = false; break; }
+          ++kp;
+          __syncwarp();
+          tc_fence_after();
+          const int s0 = 128 * sb + 64 * g;
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            float v[32];
+            tmem_ld32(tmem + loff + L::T_P + 64 * g + 32 * half, v);
+            tmem_wait_ld();
+            const int sbase = s0 + 32 * half;
+            if (s0 >= r) {
+              const float a = er * __expf(f_L[s0] - Lr);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= a * f_cfacT[sbase + j];
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int s = sbase + j;
+                v[j] = s >= r ? v[j] * er * __expf(f_L[s] - Lr) : 0.f;
+              }
+            }
+            st_row32(sS + g * PANEL128, lrow, 4 * half, v);
+          }
+          epi_arrive(BAR(C_S_READY));
+        }
+      }
+      if (!ok) break;
+      // ---- scale Q rows by Gamma_s (all score MMAs are done) and the state by Gamma_C
+      if (!mbar_wait(BAR(C_X_FULL), it & 1, ab)) { ok = false; break; }
+      for (int s = ew * 32 + lane; s < C; s += kEpiWarps * 32) {
+        const float gs = f_gam[s];
+        for (int kp2 = 0; kp2 < L::KP; ++kp2)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t a = sQ + kp2 * L::K_PANEL + sw128_off(s, ch);
+            uint32_t w0, w1, w2, w3;
+            ld_shared_v4(a, w0, w1, w2, w3);
+            st_shared_v4(a, pack_bf16x2(bf16lo(w0) * gs, bf16hi(w0) * gs),
+                         pack_bf16x2(bf16lo(w1) * gs, bf16hi(w1) * gs),
+                         pack_bf16x2(bf16lo(w2) * gs, bf16hi(w2) * gs),
+                         pack_bf16x2(bf16lo(w3) * gs, bf16hi(w3) * gs));
+          }
+      }
+      __syncwarp();
+      tc_fence_after();
+      if (w_rows) {
+        float w[32];
+        tmem_ld32(tmem + loff + L::T_DW + 32 * g, w);
+        tmem_wait_ld();
+        const float gC = f_gam[C - 1];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] *= gC;
+        tmem_st32(tmem + loff + L::T_DW + 32 * g, w);
+        tmem_wait_st();
+      }
+      epi_arrive(BAR(C_QS_READY));
+      // ---- dG = -X - u Y ; dV = -dG ; dZ = dG (MSE)
+      if (!mbar_wait(BAR(C_Y_FULL), it & 1, ab)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      for (int b = 0; b < NB; ++b) {
+        const int r = 128 * b + lrow;
+        float x[32], y[32];
+        tmem_ld32(tmem + loff + L::T_X + NV * b + 32 * g, x);
+        tmem_ld32(tmem + loff + L::T_Y + NV * b + 32 * g, y);
+        tmem_wait_ld();
+        const float u = f_eta[r] * f_eLC[r];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          x[j] = -x[j] - u * y[j];  // dG
+          y[j] = -x[j];             // dV
+        }
+        st_global_bf16x32(p.dV + (tok0 + r) * D + NV * slice + 32 * g, y);
+        if (mse) st_row32(sS, r, 4 * g, x);
+      }
+      epi_arrive(BAR(C_DZ_READY));
+      // ---- adjoint at the end of chunk c-1 (or dW0)
+      if (!mbar_wait(BAR(C_DW_FULL), it & 1, ab)) { ok = false; break; }
+      __syncwarp();
+      tc_fence_after();
+      if (w_rows) {
+        float w[32];
+        tmem_ld32(tmem + loff + L::T_DW + 32 * g, w);
+        tmem_wait_ld();
+        if (c > 0) {
+          st_row32(sDW, lrow, 4 * g, w);
+          st_global_bf16x32(p.dWs + ((size_t)bh * NC + c - 1) * D * D + wcol, w);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(p.dW0 + (size_t)bh * D * D + wcol);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+        }
+      }
+      epi_arrive(BAR(C_W_READY));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C_SCAN_FREE));
+    }
+  }
+  teardown(bars, tmem);
+}
+
+// ================================================================================== dK
+template <int D, int NB>
+struct DkL {
+  static constexpr int C = 128 * NB, KP = D / 64;
+  static constexpr uint32_t BLK = KP * PANEL128;  // 128 rows x D
+  static constexpr uint32_t WSZ = KP * D * 128;   // D rows x D
+  static constexpr uint32_t OFF_K = 0, OFF_G = BLK, OFF_W0 = 2 * BLK, OFF_DW = 2 * BLK + WSZ,
+                            OFF_Q = 2 * BLK + 2 * WSZ, OFF_DO = 3 * BLK + 2 * WSZ,
+                            OFF_F = 4 * BLK + 2 * WSZ;
+  static constexpr uint32_t OFF_BAR = OFF_F + 8 * 256 * 4;
+  static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
+  static constexpr uint32_t T_ZDP = 0, T_DK = 128, T_DS = 256, T_P = 384;
+};
+enum { K_LD_FULL, K_Z_FULL, K_G_READY, K_H_FULL, K_H_SCALED, K_QDO_FULL, K_QDO_FREE, K_SP_FULL,
+       K_DP_READY, K_DP_FREE, K_DV_FULL, K_DK_FULL, K_PART, K_SCAN, K_NBARS };
+
+template <int D, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmW,
+                  const __grid_constant__ CUtensorMap tmDW, const BwdParams p) {
+  using L = DkL<D, NB>;
+  constexpr int C = L::C;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb0 = smem_u32(smem);
+  const uint32_t sK = sb0 + L::OFF_K, sG = sb0 + L::OFF_G, sW0 = sb0 + L::OFF_W0,
+                 sDW = sb0 + L::OFF_DW, sQ = sb0 + L::OFF_Q, sDO = sb0 + L::OFF_DO;
+  float* f = reinterpret_cast<float*>(smem + L::OFF_F);
+  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cfac = f + 1024,
+        *f_cfacT = f + 1280, *f_part = f + 1536;  // f_part[2][128]
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int rb = blockIdx.x % NB;
+  const int c = (blockIdx.x / NB) % p.NC;
+  const int bh = blockIdx.x / (NB * p.NC);
+  const int NC = p.NC;
+  const bool mse = p.loss == 0;
+  const int counts[K_NBARS] = {1, 1, kEpiWarps, 1, kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1,
+                               kEpiWarps, 1};
+  uint32_t tmem;
+  setup(bars, counts, K_NBARS, tmem);
+  Abort ab{&bars->abort_flag, p.err};
+  const int tokc = bh * p.T + c * C;                 // first token of the chunk
+  const int wrow = (bh * NC + c) * D;                // first row of this chunk's state
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(BAR(K_LD_FULL), 2 * L::BLK + 2 * L::WSZ);
+#pragma unroll
+      for (int kp = 0; kp < L::KP; ++kp) {
+        tma_load_2d(sK + kp * PANEL128, &tmK, BAR(K_LD_FULL), 64 * kp, tokc + 128 * rb);
+        tma_load_2d(sG + kp * PANEL128, &tmV, BAR(K_LD_FULL), 64 * kp, tokc + 128 * rb);
+        tma_load_2d(sW0 + kp * D * 128, &tmW, BAR(K_LD_FULL), 64 * kp, wrow);
+        tma_load_2d(sDW + kp * D * 128, &tmDW, BAR(K_LD_FULL), 64 * kp, wrow);
+      }
+      int k = 0;
+      for (int sb = rb; sb < NB; ++sb, ++k) {
+        if (k > 0 && !mbar_wait(BAR(K_QDO_FREE), (k - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(BAR(K_QDO_FULL), 2 * L::BLK);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp) {
+          tma_load_2d(sQ + kp * PANEL128, &tmQ, BAR(K_QDO_FULL), 64 * kp, tokc + 128 * sb);
+          tma_load_2d(sDO + kp * PANEL128, &tmDO, BAR(K_QDO_FULL), 64 * kp, tokc + 128 * sb);
+        }
+      }
+      if (mse && mbar_wait(BAR(K_QDO_FREE), (k - 1) & 1, ab)) {
+        mbar_arrive_expect_tx(BAR(K_DV_FULL), L::BLK);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sDO + kp * PANEL128, &tmDV, BAR(K_DV_FULL), 64 * kp, tokc + 128 * rb);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idZ = idesc_bf16(128, D, 0, 1);
+      const uint32_t idKK = idesc_bf16(128, D, 0, 0);
+      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idQ = idesc_bf16(128, D, 0, 1);
+      const uint32_t idZW = idesc_bf16(128, D, 0, 0, 1);
+      do {
+        if (!mbar_wait(BAR(K_LD_FULL), 0, ab)) break;
+        tc_fence_after();
+        if (mse) {
+          // Z = K_rb W0
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_ZDP, sdesc_sw128(sK + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sW0 + j * 2048, D * 128, 1024), idZ, j > 0);
+          mma_commit(BAR(K_Z_FULL));
+        }
+        if (!mbar_wait(BAR(K_G_READY), 0, ab)) break;
+        tc_fence_after();
+        // H = G dW^T into the dK accumulator
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j)
+          mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                      sdesc_sw128(sDW + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idKK, j > 0);
+        mma_commit(BAR(K_H_FULL));
+        bool ok = true;
+        int k = 0;
+        for (int sb = rb; sb < NB; ++sb, ++k) {
+          if (!mbar_wait(BAR(K_QDO_FULL), k & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          // dS^T accumulator = G dO_sb^T ; P^T = K_rb Q_sb^T
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_DS, sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_P, sdesc_sw128(sK + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
+          mma_commit(BAR(K_SP_FULL));
+          if (!mbar_wait(BAR(K_DP_READY), k & 1, ab)) { ok = false; break; }
+          if (k == 0 && !mbar_wait(BAR(K_H_SCALED), 0, ab)) { ok = false; break; }
+          tc_fence_after();
+          // dK += dP^T Q_sb   (A = dP^T, bf16 in TMEM)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mma_bf16_ts(tmem + L::T_DK, tmem + L::T_ZDP + 8 * j,
+                        sdesc_sw128(sQ + j * 2048, PANEL128, 1024), idQ, 1);
+          mma_commit(BAR(K_QDO_FREE));
+          mma_commit(BAR(K_DP_FREE));
+        }
+        if (!ok) break;
+        if (mse) {
+          // dK += dZ W0^T with dZ = -dV
+          if (!mbar_wait(BAR(K_DV_FULL), 0, ab)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sW0 + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idZW, 1);
+        }
+        mma_commit(BAR(K_DK_FULL));
+      } while (0);
+    }
+  } else {
+    const int ew = warp - 2, g = ew / 4, q = warp & 3, lrow = q * 32 + lane;
+    const uint32_t loff = (uint32_t)(q * 32) << 16;
+    const int r = 128 * rb + lrow;  // chunk-local key index
+    do {
+      if (ew == 0) {
+        chunk_scan_warp<C>(p.beta, p.gamma, (size_t)tokc, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
+                           f_cfac, f_cfacT);
+        if (lane == 0) mbar_arrive(BAR(K_SCAN));
+      }
+      if (!mbar_wait(BAR(K_SCAN), 0, ab)) break;
+      if (!mbar_wait(BAR(K_LD_FULL), 0, ab)) break;
+      if (mse && !mbar_wait(BAR(K_Z_FULL), 0, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+      const float Lr = f_L[r], er = f_eta[r], eLCr = f_eLC[r];
+      // G = Z - V (MSE) or -V (IP), in place over V
+      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+        float v[32], z[32];
+        ld_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+        if (mse) {
+          tmem_ld32(tmem + loff + L::T_ZDP + 32 * cc, z);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = z[j] - v[j];
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = -v[j];
+        }
+        st_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+      }
+      epi_arrive(BAR(K_G_READY));
+      // H = G dW^T: deta partial -exp(L_C - L_r) K_r . H_r and the dK term -u_r H_r
+      if (!mbar_wait(BAR(K_H_FULL), 0, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+      float dot = 0.f;
+      const float ur = er * eLCr;
+      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+        float h[32], kr[32];
+        tmem_ld32(tmem + loff + L::T_DK + 32 * cc, h);
+        ld_row32(sK + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), kr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          dot += h[j] * kr[j];
+          h[j] *= -ur;
+        }
+        tmem_st32(tmem + loff + L::T_DK + 32 * cc, h);
+      }
+      tmem_wait_st();
+      epi_arrive(BAR(K_H_SCALED));
+      float deta = -eLCr * dot;
+      // score blocks: dP^T = dS^T M^T into TMEM (bf16), deta += sum_s dS^T P^T exp(L_s - L_r)
+      bool ok = true;
+      int k = 0;
+      for (int sb = rb; sb < NB; ++sb, ++k) {
+        if (!mbar_wait(BAR(K_SP_FULL), k & 1, ab)) { ok = false; break; }
+        if (k > 0 && !mbar_wait(BAR(K_DP_FREE), (k - 1) & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        const int s0 = 128 * sb + 64 * g;
+        const float a = s0 >= r ? __expf(f_L[s0] - Lr) : 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float ds[32], pp[32];
+          tmem_ld32(tmem + loff + L::T_DS + 64 * g + 32 * half, ds);
+          tmem_ld32(tmem + loff + L::T_P + 64 * g + 32 * half, pp);
+          tmem_wait_ld();
+          const int sbase = s0 + 32 * half;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int s = sbase + j;
+            const float e = s0 >= r ? a * f_cfacT[s] : (s >= r ? __expf(f_L[s] - Lr) : 0.f);
+            const float dsT = -ds[j];
+            deta += dsT * pp[j] * e;
+            ds[j] = dsT * er * e;  // dP^T
+          }
+          uint32_t w[16];
+          pack32(ds, w);
+          tmem_st16u(tmem + loff + L::T_ZDP + 32 * g + 16 * half, w);
+        }
+        tmem_wait_st();
+        epi_arrive(BAR(K_DP_READY));
+      }
+      if (!ok) break;
+      // dK out; dbeta from both warpgroups' partial sums
+      if (!mbar_wait(BAR(K_DK_FULL), 0, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+        float v[32];
+        tmem_ld32(tmem + loff + L::T_DK + 32 * cc, v);
+        tmem_wait_ld();
+        st_global_bf16x32(p.dK + ((size_t)tokc + r) * D + 32 * cc, v);
+      }
+      f_part[g * 128 + lrow] = deta;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(K_PART));
+      if (!mbar_wait(BAR(K_PART), 0, ab)) break;
+      if (g == 0) {
+        const float d = f_part[lrow] + f_part[128 + lrow];
+        p.dbeta[(size_t)tokc + r] = d * er * (1.f - 0.5f * er);
+      }
+    } while (0);
+  }
+  teardown(bars, tmem);
+}
+
+// ================================================================================== dQ
+template <int D, int NB>
+struct DqL {
+  static constexpr int C = 128 * NB, KP = D / 64;
+  static constexpr uint32_t BLK = KP * PANEL128;
+  static constexpr uint32_t WSZ = KP * D * 128;
+  static constexpr uint32_t OFF_DO = 0, OFF_W0 = BLK, OFF_K = BLK + WSZ, OFF_G = 2 * BLK + WSZ,
+                            OFF_F = 3 * BLK + WSZ;
+  static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
+  static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
+  static constexpr uint32_t T_DQ = 0, T_Z = 128, T_DS = 256, T_DP = 384;
+};
+enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_KV_FULL, Q_KV_FREE, Q_Z_FULL, Q_G_READY, Q_DS_FULL,
+       Q_DP_READY, Q_DP_FREE, Q_DQ_FULL, Q_SCAN, Q_NBARS };
+
+template <int D, int NB>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmW,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const BwdParams p) {
+  using L = DqL<D, NB>;
+  constexpr int C = L::C;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb0 = smem_u32(smem);
+  const uint32_t sDO = sb0 + L::OFF_DO, sW0 = sb0 + L::OFF_W0, sK = sb0 + L::OFF_K,
+                 sG = sb0 + L::OFF_G;
+  float* f = reinterpret_cast<float*>(smem + L::OFF_F);
+  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cfac = f + 1024,
+        *f_cfacT = f + 1280;
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int sb = blockIdx.x % NB;
+  const int c = (blockIdx.x / NB) % p.NC;
+  const int bh = blockIdx.x / (NB * p.NC);
+  const int NC = p.NC;
+  const bool mse = p.loss == 0;
+  const int counts[Q_NBARS] = {1, 1, kEpiWarps, 1, 1, 1, kEpiWarps, 1, kEpiWarps, 1, 1, 1};
+  uint32_t tmem;
+  setup(bars, counts, Q_NBARS, tmem);
+  Abort ab{&bars->abort_flag, p.err};
+  const int tokc = bh * p.T + c * C;
+  const int wrow = (bh * NC + c) * D;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(BAR(Q_LD0), L::BLK + L::WSZ);
+#pragma unroll
+      for (int kp = 0; kp < L::KP; ++kp) {
+        tma_load_2d(sDO + kp * PANEL128, &tmDO, BAR(Q_LD0), 64 * kp, tokc + 128 * sb);
+        tma_load_2d(sW0 + kp * D * 128, &tmW, BAR(Q_LD0), 64 * kp, wrow);
+      }
+      for (int rb = 0; rb <= sb; ++rb) {
+        if (rb > 0 && !mbar_wait(BAR(Q_KV_FREE), (rb - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(BAR(Q_KV_FULL), 2 * L::BLK);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp) {
+          tma_load_2d(sK + kp * PANEL128, &tmK, BAR(Q_KV_FULL), 64 * kp, tokc + 128 * rb);
+          tma_load_2d(sG + kp * PANEL128, &tmV, BAR(Q_KV_FULL), 64 * kp, tokc + 128 * rb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idKK = idesc_bf16(128, D, 0, 0);
+      const uint32_t idZ = idesc_bf16(128, D, 0, 1);
+      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      do {
+        if (!mbar_wait(BAR(Q_LD0), 0, ab)) break;
+        tc_fence_after();
+        // dQ = dO_sb W0^T (scaled by Gamma_s in the epilogue)
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j)
+          mma_bf16_ss(tmem + L::T_DQ, sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                      sdesc_sw128(sW0 + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idKK, j > 0);
+        mma_commit(BAR(Q_DQ0));
+        bool ok = true;
+        for (int rb = 0; rb <= sb; ++rb) {
+          if (!mbar_wait(BAR(Q_KV_FULL), rb & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          if (mse) {
+#pragma unroll
+            for (int j = 0; j < D / 16; ++j)
+              mma_bf16_ss(tmem + L::T_Z, sdesc_sw128(sK + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                          sdesc_sw128(sW0 + j * 2048, D * 128, 1024), idZ, j > 0);
+            mma_commit(BAR(Q_Z_FULL));
+          }
+          if (!mbar_wait(BAR(Q_G_READY), rb & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          // dS accumulator = dO_sb G_rb^T
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_DS, sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
+          mma_commit(BAR(Q_DS_FULL));
+          if (!mbar_wait(BAR(Q_DP_READY), rb & 1, ab)) { ok = false; break; }
+          if (rb == 0 && !mbar_wait(BAR(Q_DQ_SCALED), 0, ab)) { ok = false; break; }
+          tc_fence_after();
+          // dQ += dP K_rb   (A = dP, bf16 in TMEM)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mma_bf16_ts(tmem + L::T_DQ, tmem + L::T_DP + 8 * j,
+                        sdesc_sw128(sK + j * 2048, PANEL128, 1024), idZ, 1);
+          mma_commit(BAR(Q_KV_FREE));
+          mma_commit(BAR(Q_DP_FREE));
+        }
+        if (!ok) break;
+        mma_commit(BAR(Q_DQ_FULL));
+      } while (0);
+    }
+  } else {
+    const int ew = warp - 2, g = ew / 4, q = warp & 3, lrow = q * 32 + lane;
+    const uint32_t loff = (uint32_t)(q * 32) << 16;
+    const int s = 128 * sb + lrow;  // chunk-local query index
+    do {
+      if (ew == 0) {
+        chunk_scan_warp<C>(p.beta, p.gamma, (size_t)tokc, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
+                           f_cfac, f_cfacT);
+        if (lane == 0) mbar_arrive(BAR(Q_SCAN));
+      }
+      if (!mbar_wait(BAR(Q_SCAN), 0, ab)) break;
+      const float Ls = f_L[s];
+      // dQ *= Gamma_s
+      if (!mbar_wait(BAR(Q_DQ0), 0, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+        float v[32];
+        tmem_ld32(tmem + loff + L::T_DQ + 32 * cc, v);
+        tmem_wait_ld();
+        const float gs = f_gam[s];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= gs;
+        tmem_st32(tmem + loff + L::T_DQ + 32 * cc, v);
+      }
+      tmem_wait_st();
+      epi_arrive(BAR(Q_DQ_SCALED));
+      bool ok = true;
+      for (int rb = 0; rb <= sb; ++rb) {
+        // G_rb = K_rb W0 - V_rb (MSE) or -V_rb (IP), rows of the key block
+        if (!mbar_wait(BAR(Q_KV_FULL), rb & 1, ab)) { ok = false; break; }
+        if (mse && !mbar_wait(BAR(Q_Z_FULL), rb & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+          float v[32], z[32];
+          ld_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+          if (mse) {
+            tmem_ld32(tmem + loff + L::T_Z + 32 * cc, z);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = z[j] - v[j];
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = -v[j];
+          }
+          st_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+        }
+        epi_arrive(BAR(Q_G_READY));
+        // dP_sr = -acc * eta_r exp(L_s - L_r), r <= s
+        if (!mbar_wait(BAR(Q_DS_FULL), rb & 1, ab)) { ok = false; break; }
+        if (rb > 0 && !mbar_wait(BAR(Q_DP_FREE), (rb - 1) & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        const int r0 = 128 * rb + 64 * g, rlast = r0 + 63;
+        const float a = rlast <= s ? __expf(Ls - f_L[rlast]) : 0.f;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float v[32];
+          tmem_ld32(tmem + loff + L::T_DS + 64 * g + 32 * half, v);
+          tmem_wait_ld();
+          const int rbase = r0 + 32 * half;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int r = rbase + j;
+            const float m = rlast <= s ? a * f_cfac[r] : (r <= s ? f_eta[r] * __expf(Ls - f_L[r]) : 0.f);
+            v[j] = -v[j] * m;
+          }
+          uint32_t w[16];
+          pack32(v, w);
+          tmem_st16u(tmem + loff + L::T_DP + 32 * g + 16 * half, w);
+        }
+        tmem_wait_st();
+        epi_arrive(BAR(Q_DP_READY));
+      }
+      if (!ok) break;
+      if (!mbar_wait(BAR(Q_DQ_FULL), 0, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+        float v[32];
+        tmem_ld32(tmem + loff + L::T_DQ + 32 * cc, v);
+        tmem_wait_ld();
+        st_global_bf16x32(p.dQ + ((size_t)tokc + s) * D + 32 * cc, v);
+      }
+    } while (0);
+  }
+  teardown(bars, tmem);
+}
+
+#undef BAR
+
+template <int D, int NB>
+cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
+  constexpr int C = 128 * NB;
+  const uint64_t rows = (uint64_t)a.B * a.H * a.T;
+  const int BH = a.B * a.H, NC = a.T / a.C;
+  const uint64_t wrows = (uint64_t)BH * NC * D;
+  __nv_bfloat16* dWs = static_cast<__nv_bfloat16*>(a.ws);
+  CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tW, tDW;
+  if (!make_tmap_bf16(&tK, a.K, D, rows, D, 64, C) || !make_tmap_bf16(&tQ, a.Q, D, rows, D, 64, C) ||
+      !make_tmap_bf16(&tDO, a.dO, D, rows, D, 64, C) ||
+      !make_tmap_bf16(&tK1, a.K, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tV1, a.V, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tQ1, a.Q, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tDO1, a.dO, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tDV1, a.dV, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tW, a.W_chunks, D, wrows, D, 64, D) ||
+      !make_tmap_bf16(&tDW, dWs, D, wrows, D, 64, D))
+    return cudaErrorInvalidValue;
+  BwdParams p{};
+  p.BH = BH;
+  p.T = a.T;
+  p.NC = NC;
+  p.nslice = D / NV;
+  p.loss = a.loss;
+  p.lr_bias = a.lr_bias;
+  p.beta = a.beta;
+  p.gamma = a.gamma;
+  p.dW_final = a.dW_final;
+  p.dV = static_cast<__nv_bfloat16*>(a.dV);
+  p.dW0 = a.dW0;
+  p.dWs = dWs;
+  p.dQ = static_cast<__nv_bfloat16*>(a.dQ);
+  p.dK = static_cast<__nv_bfloat16*>(a.dK);
+  p.dbeta = a.dbeta;
+  p.err = a.err;
+
+  const size_t sm_chain = ChainL<D, NB>::BYTES + 1024;
+  const size_t sm_dk = DkL<D, NB>::BYTES + 1024;
+  const size_t sm_dq = DqL<D, NB>::BYTES + 1024;
+  auto kc = bwd_chain_kernel<D, NB>;
+  auto kk = bwd_dk_kernel<D, NB>;
+  auto kq = bwd_dq_kernel<D, NB>;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chain)) ||
+      (e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dk)) ||
+      (e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dq)))
+    return e;
+  kc<<<BH * p.nslice, kThreads, sm_chain, s>>>(tK, tQ, tDO, p);
+  kq<<<BH * NC * NB, kThreads, sm_dq, s>>>(tDO1, tW, tK1, tV1, p);
+  kk<<<BH * NC * NB, kThreads, sm_dk, s>>>(tK1, tV1, tQ1, tDO1, tDV1, tW, tDW, p);
+  count_launches(3);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_bwd_supported(const LayerArgs& a) {
+  return a.dtype == 1 && a.act == 0 && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
+         (a.C == 128 || a.C == 256) && a.T % a.C == 0;
+}
+
+size_t tc_bwd_workspace(const LayerArgs& a) {
+  return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2;
+}
+
+cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s) {
+  if (a.dk == 64) return a.C == 128 ? launch<64, 1>(a, s) : launch<64, 2>(a, s);
+  return a.C == 128 ? launch<128, 1>(a, s) : launch<128, 2>(a, s);
+}
+
 }  // namespace tttk

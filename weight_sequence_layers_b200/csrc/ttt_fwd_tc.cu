@@ -24,6 +24,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_util.cuh"
 
 namespace tttk {
 namespace {
@@ -73,42 +74,6 @@ struct __align__(8) FwdBars {
   uint32_t tmem_base;
   int abort_flag;
 };
-
-__device__ __forceinline__ float sigm(float x) { return 1.f / (1.f + __expf(-x)); }
-__device__ __forceinline__ float act_f(int act, float z) { return act ? z * sigm(z) : z; }
-__device__ __forceinline__ float act_d1(int act, float z) {
-  if (!act) return 1.f;
-  const float s = sigm(z);
-  return s * (1.f + z * (1.f - s));
-}
-
-// Reads 32 bf16 (16-byte chunks c0..c0+3 of `row`) of a swizzled panel as floats.
-__device__ __forceinline__ void ld_row32(uint32_t panel, int row, int c0, float (&x)[32]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    uint32_t a, b, c, d;
-    ld_shared_v4(panel + sw128_off(row, c0 + k), a, b, c, d);
-    x[8 * k + 0] = bf16lo(a); x[8 * k + 1] = bf16hi(a);
-    x[8 * k + 2] = bf16lo(b); x[8 * k + 3] = bf16hi(b);
-    x[8 * k + 4] = bf16lo(c); x[8 * k + 5] = bf16hi(c);
-    x[8 * k + 6] = bf16lo(d); x[8 * k + 7] = bf16hi(d);
-  }
-}
-__device__ __forceinline__ void st_row32(uint32_t panel, int row, int c0, const float (&x)[32]) {
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    st_shared_v4(panel + sw128_off(row, c0 + k), pack_bf16x2(x[8 * k], x[8 * k + 1]),
-                 pack_bf16x2(x[8 * k + 2], x[8 * k + 3]), pack_bf16x2(x[8 * k + 4], x[8 * k + 5]),
-                 pack_bf16x2(x[8 * k + 6], x[8 * k + 7]));
-}
-__device__ __forceinline__ void st_global_bf16x32(__nv_bfloat16* dst, const float (&x)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    d[k] = make_uint4(pack_bf16x2(x[8 * k], x[8 * k + 1]), pack_bf16x2(x[8 * k + 2], x[8 * k + 3]),
-                      pack_bf16x2(x[8 * k + 4], x[8 * k + 5]),
-                      pack_bf16x2(x[8 * k + 6], x[8 * k + 7]));
-}
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -515,6 +480,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, p);
+  count_launches(1);
   return cudaGetLastError();
 }
 

@@ -337,6 +337,7 @@ cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
                               (const __nv_bfloat16*)a.V, a.beta, a.gamma, a.W0,
                               (__nv_bfloat16*)a.O, a.W_final, (__nv_bfloat16*)a.W_chunks);
   }
+  count_launches(1);
   return cudaGetLastError();
 }
 
@@ -354,6 +355,7 @@ cudaError_t simt_bwd(const LayerArgs& a, cudaStream_t s) {
         a.dW_final, (__nv_bfloat16*)a.dQ, (__nv_bfloat16*)a.dK, (__nv_bfloat16*)a.dV, a.dbeta,
         a.dW0, (float*)a.ws);
   }
+  count_launches(1);
   return cudaGetLastError();
 }
 
