@@ -109,6 +109,29 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
                          void* dK, void* dV, float* dbeta, float* dW0, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Backward without caller-provided scratch (no counterpart in the papers: a deployment aid).
+ * Some callers cannot allocate device memory when they call the library: a host framework
+ * that owns every byte of device memory through its own pool, or a plugin that is handed only
+ * its input and output buffers. For them this variant takes the same arguments as
+ * ttt_chunk_bwd minus the workspace, and keeps its scratch (the per-chunk adjoint states) in
+ * a fixed array of TTT_NOALLOC_SCRATCH_BYTES that the library holds on every GPU it is loaded
+ * on, until the process exits. It allocates nothing and calls no allocating routine.
+ *  - Only configs of the tensor-core backward are accepted (bf16, identity activation,
+ *    dk == dv in {64, 128}, C in {128, 256}); others return TTT_ERR_UNSUPPORTED.
+ *  - Configs needing more than the fixed scratch (B*H*(T/C)*dk*dv*2 bytes) return
+ *    TTT_ERR_WORKSPACE with nothing launched; ttt_chunk_bwd serves those.
+ *  - The first call on a device looks up the array's device address (with that device
+ *    current); make that first call before any stream capture.
+ *  - Every call shares the one array and leaves its contents behind. Calls that overlap on
+ *    the GPU (different streams, or different host threads) race on it: serialise them.
+ *    Nothing in the array has to start at zero. */
+#define TTT_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q, const void* K, const void* V,
+                                 const float* beta, const float* gamma, const float* W0,
+                                 const void* W_chunks, const void* dO, const float* dW_final,
+                                 void* dQ, void* dK, void* dV, float* dbeta, float* dW0,
+                                 void* stream);
+
 /* Workspace bytes of inplace_ttt_fwd; (size_t)-1 for invalid sizes. */
 size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C);
 

@@ -1,0 +1,65 @@
+"""ttt_chunk_bwd_noalloc: the backward for callers that cannot allocate device memory when they
+call the library (a host framework that owns all device memory, a plugin handed only its
+buffers). It must give the same gradients as ttt_chunk_bwd with a caller workspace, on two
+calls in a row that share its fixed scratch array, and refuse configs whose scratch would not
+fit. This file is collected last on purpose."""
+import ctypes
+
+import pytest
+import torch
+
+import synth
+import weight_sequence_layers_b200 as ttt
+from _runners import abi_config, run_bwd, run_fwd
+from _util import rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+GRADS = ("dQ", "dK", "dV", "dbeta", "dW0")
+
+
+def noalloc_bwd(cfg, inp, W_chunks):
+    c = abi_config(cfg)
+    sd = synth.storage_dtype(cfg)
+    B, H, T, dk, dv = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv
+    out = dict(dQ=torch.full((B, H, T, dk), float("nan"), device="cuda", dtype=sd),
+               dK=torch.full((B, H, T, dk), float("nan"), device="cuda", dtype=sd),
+               dV=torch.full((B, H, T, dv), float("nan"), device="cuda", dtype=sd),
+               dbeta=torch.full((B, H, T), float("nan"), device="cuda"),
+               dW0=torch.full((B, H, dk, dv), float("nan"), device="cuda"))
+    st = ttt.lib.ttt_chunk_bwd_noalloc(
+        ctypes.byref(c), inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(),
+        inp["beta"].data_ptr(), inp["gamma"].data_ptr(), inp["W0"].data_ptr(), W_chunks.data_ptr(),
+        inp["dO"].data_ptr(), inp["dW_T"].data_ptr(), out["dQ"].data_ptr(), out["dK"].data_ptr(),
+        out["dV"].data_ptr(), out["dbeta"].data_ptr(), out["dW0"].data_ptr(),
+        torch.cuda.current_stream().cuda_stream)
+    assert st == ttt.OK, ttt.status_string(st)
+    torch.cuda.synchronize()
+    assert ttt.ttt_get_device_error() == ttt.OK
+    return out
+
+
+def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
+    # scratch needed: 4 heads x 4 chunks x 128 x 128 x 2 bytes = 512 KiB (limit 8 MiB)
+    cfg = synth.TRAIN_1P45B.replace(B=1, H=4, T=1024)
+    for seed in (21, 22):
+        inp = synth.ttt_inputs(cfg, device="cuda", seed=seed)
+        inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(seed))
+        fwd = run_fwd(cfg, inp)
+        ref = run_bwd(cfg, inp, fwd["W_chunks"])
+        got = noalloc_bwd(cfg, inp, fwd["W_chunks"])
+        for k in GRADS:
+            assert rel_err(got[k], ref[k]) <= TOL, (seed, k)
+
+
+def test_noalloc_backward_refuses_configs_beyond_its_scratch():
+    big = abi_config(synth.TRAIN_1P45B)  # needs 32 MiB of scratch
+    A = 4096  # never dereferenced: the size check comes first
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(big), A, A, A, A, A, A, A, A, None, A, A, A, A,
+                                       A, None)
+    assert st == ttt.ERR_WORKSPACE
+    silu = abi_config(synth.TRAIN_1P45B.replace(B=1, H=1, T=256, act="silu"))
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(silu), A, A, A, A, A, A, A, A, None, A, A, A,
+                                       A, A, None)
+    assert st == ttt.ERR_UNSUPPORTED

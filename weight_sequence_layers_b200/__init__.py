@@ -52,6 +52,7 @@ _SIGS = {
     "ttt_selftest_bounded_wait": ([_u, _p], _i),
     "ttt_status_string": ([_i], ctypes.c_char_p),
     "ttt_kernel_launches": ([], ctypes.c_ulonglong),
+    "ttt_chunk_bwd_noalloc": ([_cfgp] + [_p] * 14 + [_p], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -118,6 +119,19 @@ def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final, dQ, dK,
                             _ptr(dV), _ptr(dbeta), _ptr(dW0), _ptr(workspace),
                             int(workspace_bytes), _stream(stream))
     _check(st, "ttt_chunk_bwd")
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def ttt_chunk_bwd_noalloc(cfg, Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final, dQ, dK, dV, dbeta,
+                          dW0, stream=None):
+    """ttt_chunk_bwd for callers that cannot allocate: scratch is the library's fixed array."""
+    st = _lib.ttt_chunk_bwd_noalloc(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
+                                    _ptr(gamma), _ptr(W0), _ptr(W_chunks), _ptr(dO),
+                                    _ptr(dW_final), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta),
+                                    _ptr(dW0), _stream(stream))
+    _check(st, "ttt_chunk_bwd_noalloc")
 
 
 def inplace_ttt_workspace_bytes(T, d_ff, d_model, C) -> int:

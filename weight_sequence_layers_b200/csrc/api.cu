@@ -124,6 +124,11 @@ __global__ void selftest_wait_kernel(unsigned spin_limit, unsigned* err) {
 
 }  // namespace
 
+unsigned* current_error_word() {
+  cudaError_t e;
+  return error_word(&e);
+}
+
 std::atomic<unsigned long long> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 

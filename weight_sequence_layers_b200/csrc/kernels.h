@@ -44,6 +44,9 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
                         const void* Vhat, float* W, void* O, void* ws, unsigned* err,
                         cudaStream_t s);
 
+// Address of the current device's error word (looked up once per device); NULL on failure.
+unsigned* current_error_word();
+
 // Adds n to the process-wide count of kernel launches (reported by ttt_kernel_launches).
 void count_launches(int n);
 
