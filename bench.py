@@ -44,6 +44,29 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def measured_traffic(call: str, workload: str):
+    """DRAM bytes per launch of `call` from the committed ncu counters, or None if the kernel
+    sources changed since those counters were taken (or none exist for this workload)."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            entry = json.load(f)[call]
+    except (OSError, KeyError, ValueError):
+        return None
+    if entry.get("workload") != workload:
+        return None
+    m = hashlib.sha256()
+    for rel in sorted(entry["sources"]):
+        try:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                data = f.read()
+        except OSError:
+            return None
+        m.update(rel.encode())
+        m.update(data)
+    return entry["bytes"] if m.hexdigest()[:16] == entry["sha"] else None
+
+
 # ------------------------------------------------------------------------- algorithmic work
 def layer_work(cfg):
     """Algorithmic flops and bytes of one forward and one backward launch.
@@ -380,8 +403,10 @@ def main():
     dom_bytes = work[f"{dom}_bytes"]
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "kernel": f"ttt_chunk_{dom}", "peak_source": peak_src}
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": measured_traffic(f"ttt_chunk_{dom}", cfg.name),
+                "kernel": f"ttt_chunk_{dom}", "algorithmic_bytes": dom_bytes,
+                "peak_source": peak_src}
     step_flops = work["fwd_flops"] + work["bwd_flops"]
     tc_frac = step_flops / (ms_step * 1e-3) / (peaks["bf16_tflops"] * 1e12)
 
@@ -408,7 +433,10 @@ def main():
         out["inplace"] = {"workload": icfg.name, "ms": ims, "tokens_per_s": icfg.T / (ims * 1e-3),
                           "roofline": {"bound": "tensor", "achieved": tf,
                                        "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                                       "frac": tf / peaks["bf16_tflops_sustained"]}}
+                                       "frac": tf / peaks["bf16_tflops_sustained"],
+                                       "traffic": measured_traffic("inplace_chunk", icfg.name),
+                                       "traffic_unit": "bytes per chunk launch",
+                                       "peak_source": peak_src}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg)
     if _dist is not None:
