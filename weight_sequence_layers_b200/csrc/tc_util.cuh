@@ -9,12 +9,23 @@
 namespace tttk {
 namespace {
 
-__device__ __forceinline__ float sigm(float x) { return 1.f / (1.f + __expf(-x)); }
-__device__ __forceinline__ float act_f(int act, float z) { return act ? z * sigm(z) : z; }
-__device__ __forceinline__ float act_d1(int act, float z) {
-  if (!act) return 1.f;
-  const float s = sigm(z);
-  return s * (1.f + z * (1.f - s));
+// Sigmoid with the hardware exponential and reciprocal (bf16-level accuracy is enough here).
+__device__ __forceinline__ float sigm(float x) { return __frcp_rn(1.f + __expf(-x)); }
+
+// Activation of the fast-weight network (ACT = 0 identity, 1 SiLU) and its derivative; a
+// compile-time choice so the identity path carries no transcendental at all.
+template <int ACT>
+__device__ __forceinline__ float act_f(float z) {
+  if constexpr (ACT == 1) return z * sigm(z);
+  return z;
+}
+template <int ACT>
+__device__ __forceinline__ float act_d1(float z) {
+  if constexpr (ACT == 1) {
+    const float s = sigm(z);
+    return s * (1.f + z * (1.f - s));
+  }
+  return 1.f;
 }
 
 // Reads 32 bf16 (16-byte chunks c0..c0+3 of `row`) of a swizzled panel as floats.
@@ -49,13 +60,12 @@ __device__ __forceinline__ void st_global_bf16x32(__nv_bfloat16* dst, const floa
 // Per-chunk scans by one warp (C = 32 * PER tokens starting at tok0):
 //   eta_r = 2 sigmoid(beta_r + b), L_r = sum_{t<=r} log gamma_t (chunk-local),
 //   gam_r = exp(L_r), eLC_r = exp(L_C - L_r),
-//   cfac_r  = eta_r exp(L_{last of r's 64-group} - L_r)   (<= eta_r),
-//   cfacT_r = exp(L_r - L_{first of r's 64-group})         (<= 1).
-// Every exponent is <= 0: no 1/Gamma is formed, strong decay underflows to 0 instead.
+//   cF16_r = eta_r exp(L_{r16} - L_r) and cT16_r = exp(L_r - L_{r16}) with r16 = r & ~15.
+// beta and gamma may point to global or shared memory (gamma NULL: no decay).
 template <int C>
-__device__ __forceinline__ void chunk_scan_warp(const float* beta, const float* gamma, size_t tok0,
-                                                float lr_bias, float* eta, float* L, float* gam,
-                                                float* eLC, float* cfac, float* cfacT) {
+__device__ __forceinline__ void chunk_scan_warp(const float* beta, const float* gamma, float lr_bias,
+                                                float* eta, float* L, float* gam, float* eLC,
+                                                float* cF16, float* cT16) {
   constexpr int PER = C / 32;
   const int lane = threadIdx.x & 31;
   float lg[PER];
@@ -63,9 +73,9 @@ __device__ __forceinline__ void chunk_scan_warp(const float* beta, const float* 
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
     const int r = lane * PER + k;
-    run += gamma ? __logf(gamma[tok0 + r]) : 0.f;
+    run += gamma ? __logf(gamma[r]) : 0.f;
     lg[k] = run;
-    eta[r] = 2.f * sigm(beta[tok0 + r] + lr_bias);
+    eta[r] = 2.f * sigm(beta[r] + lr_bias);
   }
   float incl = run;
 #pragma unroll
@@ -81,13 +91,50 @@ __device__ __forceinline__ void chunk_scan_warp(const float* beta, const float* 
 #pragma unroll
   for (int k = 0; k < PER; ++k) {
     const int r = lane * PER + k;
-    const float Lr = L[r];
+    const float Lr = L[r], L16 = L[r & ~15];
     gam[r] = __expf(Lr);
     eLC[r] = __expf(LC - Lr);
-    cfac[r] = eta[r] * __expf(L[r | 63] - Lr);
-    cfacT[r] = __expf(Lr - L[r & ~63]);
+    cF16[r] = eta[r] * __expf(L16 - Lr);
+    cT16[r] = __expf(Lr - L16);
   }
   __syncwarp();
+}
+
+// Causal decay weights of one query s against 32 consecutive keys r0..r0+31 (r0 % 16 == 0):
+//   w_j = [r <= s] eta_r exp(L_s - L_r) = [r <= s] exp(L_s - L_{r16}) * cF16_r.
+// One exponential per 16 keys, no division; the first factor is <= 1 whenever a key of the
+// group precedes s, the second is bounded by the decay of at most 15 tokens.
+__device__ __forceinline__ void causal_weights_q(const float* L, const float* cF16, int s, float Ls,
+                                                 int r0, float (&w)[32]) {
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int r16 = r0 + 16 * g;
+    const float a = s >= r16 ? __expf(Ls - L[r16]) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[16 * g + j] = (r16 + j <= s) ? a * cF16[r16 + j] : 0.f;
+  }
+}
+
+// Causal decay weights of one key r against 32 consecutive queries s0..s0+31 (s0 % 16 == 0):
+//   w_j = [s >= r] exp(L_s - L_r) = [s >= r] exp(L_{s16} - L_r) * cT16_s.
+__device__ __forceinline__ void causal_weights_k(const float* L, const float* cT16, int r, float Lr,
+                                                 int s0, float (&w)[32]) {
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    const int s16 = s0 + 16 * g;
+    const float b = s16 + 15 >= r ? __expf(L[s16] - Lr) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) w[16 * g + j] = (s16 + j >= r) ? b * cT16[s16 + j] : 0.f;
+  }
+}
+
+// Bulk copy of `bytes` (multiple of 16, 16-byte aligned) from global to shared memory,
+// completing on `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
 }
 
 // 32 consecutive floats -> 16 packed bf16 pairs (even index in the low half).

@@ -126,8 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sK = sb0 + L::OFF_K, sQ = sb0 + L::OFF_Q, sDO = sb0 + L::OFF_DO,
                  sDW = sb0 + L::OFF_DW, sS = sb0 + L::OFF_S;
   float* f = reinterpret_cast<float*>(smem + L::OFF_F);
-  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cfac = f + 1024,
-        *f_cfacT = f + 1280;
+  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
+        *f_cT16 = f + 1280;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / p.nslice, slice = blockIdx.x % p.nslice;
@@ -246,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
       if (ew == 0) {
         if (it > 0 && !mbar_wait(BAR(C_SCAN_FREE), (it - 1) & 1, ab)) { ok = false; break; }
-        chunk_scan_warp<C>(p.beta, p.gamma, tok0, p.lr_bias, f_eta, f_L, f_gam, f_eLC, f_cfac,
-                           f_cfacT);
+        chunk_scan_warp<C>(p.beta + tok0, p.gamma ? p.gamma + tok0 : nullptr, p.lr_bias, f_eta, f_L,
+                           f_gam, f_eLC, f_cF16, f_cT16);
         if (lane == 0) mbar_arrive(BAR(C_SCAN_FULL));
       }
       if (!mbar_wait(BAR(C_SCAN_FULL), it & 1, ab)) { ok = false; break; }
@@ -264,21 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s0 = 128 * sb + 64 * g;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            float v[32];
+            float v[32], w[32];
             tmem_ld32(tmem + loff + L::T_P + 64 * g + 32 * half, v);
+            causal_weights_k(f_L, f_cT16, r, Lr, s0 + 32 * half, w);
             tmem_wait_ld();
-            const int sbase = s0 + 32 * half;
-            if (s0 >= r) {
-              const float a = er * __expf(f_L[s0] - Lr);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] *= a * f_cfacT[sbase + j];
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int s = sbase + j;
-                v[j] = s >= r ? v[j] * er * __expf(f_L[s] - Lr) : 0.f;
-              }
-            }
+            for (int j = 0; j < 32; ++j) v[j] *= er * w[j];
             st_row32(sS + g * PANEL128, lrow, 4 * half, v);
           }
           epi_arrive(BAR(C_S_READY));
@@ -391,8 +382,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sK = sb0 + L::OFF_K, sG = sb0 + L::OFF_G, sW0 = sb0 + L::OFF_W0,
                  sDW = sb0 + L::OFF_DW, sQ = sb0 + L::OFF_Q, sDO = sb0 + L::OFF_DO;
   float* f = reinterpret_cast<float*>(smem + L::OFF_F);
-  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cfac = f + 1024,
-        *f_cfacT = f + 1280, *f_part = f + 1536;  // f_part[2][128]
+  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
+        *f_cT16 = f + 1280, *f_part = f + 1536;  // f_part[2][128]
   Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int rb = blockIdx.x % NB;
@@ -506,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = 128 * rb + lrow;  // chunk-local key index
     do {
       if (ew == 0) {
-        chunk_scan_warp<C>(p.beta, p.gamma, (size_t)tokc, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
-                           f_cfac, f_cfacT);
+        chunk_scan_warp<C>(p.beta + tokc, p.gamma ? p.gamma + tokc : nullptr, p.lr_bias, f_eta,
+                           f_L, f_gam, f_eLC, f_cF16, f_cT16);
         if (lane == 0) mbar_arrive(BAR(K_SCAN));
       }
       if (!mbar_wait(BAR(K_SCAN), 0, ab)) break;
@@ -562,21 +553,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         tc_fence_after();
         const int s0 = 128 * sb + 64 * g;
-        const float a = s0 >= r ? __expf(f_L[s0] - Lr) : 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          float ds[32], pp[32];
+          float ds[32], pp[32], wt[32];
           tmem_ld32(tmem + loff + L::T_DS + 64 * g + 32 * half, ds);
           tmem_ld32(tmem + loff + L::T_P + 64 * g + 32 * half, pp);
+          causal_weights_k(f_L, f_cT16, r, Lr, s0 + 32 * half, wt);
           tmem_wait_ld();
-          const int sbase = s0 + 32 * half;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int s = sbase + j;
-            const float e = s0 >= r ? a * f_cfacT[s] : (s >= r ? __expf(f_L[s] - Lr) : 0.f);
             const float dsT = -ds[j];
-            deta += dsT * pp[j] * e;
-            ds[j] = dsT * er * e;  // dP^T
+            deta += dsT * pp[j] * wt[j];
+            ds[j] = dsT * er * wt[j];  // dP^T
           }
           uint32_t w[16];
           pack32(ds, w);
@@ -638,8 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sDO = sb0 + L::OFF_DO, sW0 = sb0 + L::OFF_W0, sK = sb0 + L::OFF_K,
                  sG = sb0 + L::OFF_G;
   float* f = reinterpret_cast<float*>(smem + L::OFF_F);
-  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cfac = f + 1024,
-        *f_cfacT = f + 1280;
+  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
+        *f_cT16 = f + 1280;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int sb = blockIdx.x % NB;
@@ -726,8 +714,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int s = 128 * sb + lrow;  // chunk-local query index
     do {
       if (ew == 0) {
-        chunk_scan_warp<C>(p.beta, p.gamma, (size_t)tokc, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
-                           f_cfac, f_cfacT);
+        chunk_scan_warp<C>(p.beta + tokc, p.gamma ? p.gamma + tokc : nullptr, p.lr_bias, f_eta,
+                           f_L, f_gam, f_eLC, f_cF16, f_cT16);
         if (lane == 0) mbar_arrive(BAR(Q_SCAN));
       }
       if (!mbar_wait(BAR(Q_SCAN), 0, ab)) break;
@@ -774,20 +762,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (rb > 0 && !mbar_wait(BAR(Q_DP_FREE), (rb - 1) & 1, ab)) { ok = false; break; }
         __syncwarp();
         tc_fence_after();
-        const int r0 = 128 * rb + 64 * g, rlast = r0 + 63;
-        const float a = rlast <= s ? __expf(Ls - f_L[rlast]) : 0.f;
+        const int r0 = 128 * rb + 64 * g;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          float v[32];
+          float v[32], m[32];
           tmem_ld32(tmem + loff + L::T_DS + 64 * g + 32 * half, v);
+          causal_weights_q(f_L, f_cF16, s, Ls, r0 + 32 * half, m);
           tmem_wait_ld();
-          const int rbase = r0 + 32 * half;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int r = rbase + j;
-            const float m = rlast <= s ? a * f_cfac[r] : (r <= s ? f_eta[r] * __expf(Ls - f_L[r]) : 0.f);
-            v[j] = -v[j] * m;
-          }
+          for (int j = 0; j < 32; ++j) v[j] = -v[j] * m[j];
           uint32_t w[16];
           pack32(v, w);
           tmem_st16u(tmem + loff + L::T_DP + 32 * g + 16 * half, w);

@@ -36,7 +36,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t PANEL128 = 128 * 128;  // 128 rows x 128 bytes
 
 struct FwdParams {
-  int BH, T, NC, nslice, loss, act;
+  int BH, T, NC, nslice;
   float lr_bias;
   const float* beta;
   const float* gamma;     // nullable
@@ -58,8 +58,9 @@ struct Layout {
   static constexpr uint32_t OFF_UG = OFF_V + C * 128;
   static constexpr uint32_t OFF_W0 = OFF_UG + C * 128;      // bf16 state, MN-major [D][64]
   static constexpr uint32_t OFF_S = OFF_W0 + D * 128;       // 2 panels of 128 x 64
-  static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;   // float arrays
-  static constexpr uint32_t OFF_BAR = OFF_F + 5 * 256 * 4;
+  static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;   // float arrays (6 x 256)
+  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;   // beta, gamma of 2 chunks (4 x C)
+  static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + 256;
   static constexpr uint32_t KV_TX = KP * K_PANEL + C * 128;
   static constexpr uint32_t Q_TX = KP * PANEL128;
@@ -75,7 +76,7 @@ struct __align__(8) FwdBars {
   int abort_flag;
 };
 
-template <int D, int NB>
+template <int D, int NB, int ACT, int LOSS>
 __global__ void __launch_bounds__(kThreads, 1)
     ttt_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -90,8 +91,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* f_eta = reinterpret_cast<float*>(smem + L::OFF_F);  // eta_r
   float* f_L = f_eta + 256;                                   // L_r (chunk-local log decay)
   float* f_gam = f_L + 256;                                   // Gamma_r = exp(L_r)
-  float* f_uneg = f_gam + 256;                                // -eta_r exp(L_C - L_r)
-  float* f_cfac = f_uneg + 256;                               // eta_r exp(L_ref(r) - L_r)
+  float* f_eLC = f_gam + 256;                                 // exp(L_C - L_r)
+  float* f_cF16 = f_eLC + 256;                                // eta_r exp(L_{r16} - L_r)
+  float* f_cT16 = f_cF16 + 256;                               // exp(L_r - L_{r16})
+  float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);   // [parity][beta, gamma][C]
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / p.nslice, slice = blockIdx.x % p.nslice;
@@ -147,7 +150,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++qk;
           if (h == 0) {
             if (c > 0 && !mbar_wait(BAR(kv_free), (c - 1) & 1, ab)) goto done_prod;
-            mbar_arrive_expect_tx(BAR(kv_full), L::KV_TX);
+            mbar_arrive_expect_tx(BAR(kv_full), L::KV_TX + (p.gamma ? 2 : 1) * C * 4);
+            {
+              const uint32_t bg = smem_u32(f_bg + (c & 1) * 2 * C);
+              bulk_g2s(bg, p.beta + (size_t)row0, C * 4, BAR(kv_full));
+              if (p.gamma) bulk_g2s(bg + C * 4, p.gamma + (size_t)row0, C * 4, BAR(kv_full));
+            }
 #pragma unroll
             for (int kp = 0; kp < L::KP; ++kp)
               tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(kv_full), 64 * kp, row0);
@@ -259,41 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kp = 0;  // score blocks consumed
     for (int c = 0; c < NC && ok; ++c) {
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
-      // -------- per-chunk scans (warp 2): eta, L, Gamma, -u, column factors
+      // -------- per-chunk scans (warp 2) from the prefetched beta, gamma
       if (ew == 0) {
         if (c > 0 && !mbar_wait(BAR(scan_free), (c - 1) & 1, ab)) { ok = false; break; }
-        constexpr int PER = C / 32;
-        float lg[PER];
-        float run = 0.f;
-#pragma unroll
-        for (int k = 0; k < PER; ++k) {
-          const int r = lane * PER + k;
-          const float gmm = p.gamma ? p.gamma[tok0 + r] : 1.f;
-          run += p.gamma ? __logf(gmm) : 0.f;
-          lg[k] = run;
-          f_eta[r] = 2.f * sigm(p.beta[tok0 + r] + p.lr_bias);
-        }
-        float incl = run;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const float o = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += o;
-        }
-        const float excl = incl - run;
-        const float LC = __shfl_sync(0xffffffffu, incl, 31);
-#pragma unroll
-        for (int k = 0; k < PER; ++k) f_L[lane * PER + k] = lg[k] + excl;
-        __syncwarp();
-#pragma unroll
-        for (int k = 0; k < PER; ++k) {
-          const int r = lane * PER + k;
-          const float Lr = f_L[r];
-          const float eta = f_eta[r];
-          f_gam[r] = __expf(Lr);
-          f_uneg[r] = -eta * __expf(LC - Lr);
-          f_cfac[r] = eta * __expf(f_L[r | 63] - Lr);
-        }
-        __syncwarp();
+        if (!mbar_wait(BAR(kv_full), c & 1, ab)) { ok = false; break; }
+        const float* bg = f_bg + (c & 1) * 2 * C;
+        chunk_scan_warp<C>(bg, p.gamma ? bg + C : nullptr, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
+                           f_cF16, f_cT16);
         if (lane == 0) mbar_arrive(BAR(scan_full));
       }
       if (!mbar_wait(BAR(scan_full), c & 1, ab)) { ok = false; break; }
@@ -310,11 +290,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         const int row = 128 * b + lrow;
         ld_row32(sV, row, 4 * g, v);
-        const float un = f_uneg[row];
+        const float un = -f_eta[row] * f_eLC[row];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float a = p.loss == 0 ? act_f(p.act, z[j]) - v[j] : -v[j];
-          const float gg = a * act_d1(p.act, z[j]);
+          const float a = LOSS == 0 ? act_f<ACT>(z[j]) - v[j] : -v[j];
+          const float gg = a * act_d1<ACT>(z[j]);
           v[j] = gg;
           z[j] = un * gg;
         }
@@ -391,26 +371,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           __syncwarp();
           tc_fence_after();
           const int r0 = 128 * b + 64 * g;  // first key of this thread's 64 columns
-          const int rlast = r0 + 63;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            float s[32];
-            tmem_ld32(tmem + lane_off + L::T_P + 64 * g + 32 * half, s);
+            float sv[32], w[32];
+            tmem_ld32(tmem + lane_off + L::T_P + 64 * g + 32 * half, sv);
+            causal_weights_q(f_L, f_cF16, srow, Ls, r0 + 32 * half, w);
             tmem_wait_ld();
-            const int rb = r0 + 32 * half;
-            if (rlast <= srow) {
-              // every key precedes the query: exp(L_s - L_r) = exp(L_s - L_last) * exp(L_last - L_r)
-              const float as = __expf(Ls - f_L[rlast]);
 #pragma unroll
-              for (int j = 0; j < 32; ++j) s[j] = -s[j] * as * f_cfac[rb + j];
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int r = rb + j;
-                s[j] = r <= srow ? -s[j] * f_eta[r] * __expf(Ls - f_L[r]) : 0.f;
-              }
-            }
-            st_row32(sS + g * PANEL128, lrow, 4 * half, s);
+            for (int j = 0; j < 32; ++j) sv[j] = -sv[j] * w[j];
+            st_row32(sS + g * PANEL128, lrow, 4 * half, sv);
           }
           fence_proxy_async_smem();
           tc_fence_before();
@@ -431,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = act_f(p.act, o[j]);
+          for (int j = 0; j < 32; ++j) o[j] = act_f<ACT>(o[j]);
           st_global_bf16x32(p.O + (tok0 + srow) * D + NV * slice + 32 * g, o);
         }
       }
@@ -451,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int NB>
+template <int D, int NB, int ACT, int LOSS>
 cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   using L = Layout<D, NB>;
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
@@ -465,8 +434,6 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.T = a.T;
   p.NC = a.T / a.C;
   p.nslice = D / NV;
-  p.loss = a.loss;
-  p.act = a.act;
   p.lr_bias = a.lr_bias;
   p.beta = a.beta;
   p.gamma = a.gamma;
@@ -476,7 +443,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.W_chunks = static_cast<__nv_bfloat16*>(a.W_chunks);
   p.err = a.err;
   const size_t smem = L::BYTES + 1024;
-  auto k = ttt_fwd_tc_kernel<D, NB>;
+  auto k = ttt_fwd_tc_kernel<D, NB, ACT, LOSS>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, p);
@@ -493,9 +460,15 @@ bool tc_fwd_supported(const LayerArgs& a) {
 
 size_t tc_fwd_workspace(const LayerArgs&) { return 0; }
 
+template <int D, int NB>
+cudaError_t launch_variant(const LayerArgs& a, cudaStream_t s) {
+  if (a.act == 0) return a.loss == 0 ? launch<D, NB, 0, 0>(a, s) : launch<D, NB, 0, 1>(a, s);
+  return a.loss == 0 ? launch<D, NB, 1, 0>(a, s) : launch<D, NB, 1, 1>(a, s);
+}
+
 cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s) {
-  if (a.dk == 64) return a.C == 128 ? launch<64, 1>(a, s) : launch<64, 2>(a, s);
-  return a.C == 128 ? launch<128, 1>(a, s) : launch<128, 2>(a, s);
+  if (a.dk == 64) return a.C == 128 ? launch_variant<64, 1>(a, s) : launch_variant<64, 2>(a, s);
+  return a.C == 128 ? launch_variant<128, 1>(a, s) : launch_variant<128, 2>(a, s);
 }
 
 }  // namespace tttk
