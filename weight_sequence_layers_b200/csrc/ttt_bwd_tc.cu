@@ -105,13 +105,15 @@ struct ChainL {
   static constexpr uint32_t OFF_DW = OFF_DO + C * 128;   // bf16 adjoint, MN-major [D][64]
   static constexpr uint32_t OFF_S = OFF_DW + D * 128;    // S^T blocks, then dZ (C rows)
   static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;
-  static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
+  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of 2 chunks
+  static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t TX = 2 * KP * K_PANEL + C * 128;
   static constexpr uint32_t T_DW = 0, T_X = 64, T_Y = 64 + 64 * NB, T_P = 64 + 128 * NB;
 };
 enum { C_KV_FULL, C_KV_FREE, C_P_FULL, C_S_READY, C_S_FREE, C_X_FULL, C_W_READY, C_Y_FULL,
-       C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_NBARS };
+       C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_BG_FULL, C_BG_FULL1,
+       C_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -134,13 +136,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NC = p.NC;
   const bool mse = p.loss == 0;
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
-                               kEpiWarps};
+                               kEpiWarps, 1, 1};
+  float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   uint32_t tmem;
   setup(bars, counts, C_NBARS, tmem);
   Abort ab{&bars->abort_flag, p.err};
 
   if (warp == 0) {
     if (lane == 0) {
+      // beta, gamma of iteration it go to buffer it & 1 on barrier C_BG_FULL + (it & 1)
+      // (phase (it >> 1) & 1), one iteration ahead of the scan that reads them
+      auto load_bg = [&](int i2) {
+        const uint32_t bg = smem_u32(f_bg + (i2 & 1) * 2 * C);
+        const uint32_t bar = BAR(C_BG_FULL + (i2 & 1));
+        const size_t r0 = (size_t)bh * p.T + (size_t)(NC - 1 - i2) * C;
+        mbar_arrive_expect_tx(bar, (p.gamma ? 2 : 1) * C * 4);
+        bulk_g2s(bg, p.beta + r0, C * 4, bar);
+        if (p.gamma) bulk_g2s(bg + C * 4, p.gamma + r0, C * 4, bar);
+      };
+      load_bg(0);
       for (int it = 0; it < NC; ++it) {
         const int c = NC - 1 - it;
         const int row0 = bh * p.T + c * C;
@@ -152,6 +166,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sQ + kp * L::K_PANEL, &tmQ, BAR(C_KV_FULL), 64 * kp, row0);
         }
         tma_load_2d(sDO, &tmDO, BAR(C_KV_FULL), NV * slice, row0);
+        if (it + 1 < NC) {
+          if (it > 0 && !mbar_wait(BAR(C_SCAN_FULL), (it - 1) & 1, ab)) break;
+          load_bg(it + 1);
+        }
       }
     }
   } else if (warp == 1) {
@@ -246,8 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
       if (ew == 0) {
         if (it > 0 && !mbar_wait(BAR(C_SCAN_FREE), (it - 1) & 1, ab)) { ok = false; break; }
-        chunk_scan_warp<C>(p.beta + tok0, p.gamma ? p.gamma + tok0 : nullptr, p.lr_bias, f_eta, f_L,
-                           f_gam, f_eLC, f_cF16, f_cT16);
+        if (!mbar_wait(BAR(C_BG_FULL + (it & 1)), (it >> 1) & 1, ab)) { ok = false; break; }
+        const float* bg = f_bg + (it & 1) * 2 * C;
+        chunk_scan_warp<C>(bg, p.gamma ? bg + C : nullptr, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
+                           f_cF16, f_cT16);
         if (lane == 0) mbar_arrive(BAR(C_SCAN_FULL));
       }
       if (!mbar_wait(BAR(C_SCAN_FULL), it & 1, ab)) { ok = false; break; }
@@ -357,15 +377,16 @@ struct DkL {
   static constexpr int C = 128 * NB, KP = D / 64;
   static constexpr uint32_t BLK = KP * PANEL128;  // 128 rows x D
   static constexpr uint32_t WSZ = KP * D * 128;   // D rows x D
+  // the dW slot later receives a 128-row dV block, so it holds the larger of the two
+  static constexpr uint32_t DWSZ = WSZ > BLK ? WSZ : BLK;
   static constexpr uint32_t OFF_K = 0, OFF_G = BLK, OFF_W0 = 2 * BLK, OFF_DW = 2 * BLK + WSZ,
-                            OFF_Q = 2 * BLK + 2 * WSZ, OFF_DO = 3 * BLK + 2 * WSZ,
-                            OFF_F = 4 * BLK + 2 * WSZ;
+                            OFF_Q = OFF_DW + DWSZ, OFF_DO = OFF_Q + BLK, OFF_F = OFF_DO + BLK;
   static constexpr uint32_t OFF_BAR = OFF_F + 8 * 256 * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t T_ZDP = 0, T_DK = 128, T_DS = 256, T_P = 384;
 };
 enum { K_LD_FULL, K_Z_FULL, K_G_READY, K_H_FULL, K_H_SCALED, K_QDO_FULL, K_QDO_FREE, K_SP_FULL,
-       K_DP_READY, K_DP_FREE, K_DV_FULL, K_DK_FULL, K_PART, K_SCAN, K_NBARS };
+       K_DP_READY, K_DP_FREE, K_DV_FULL, K_DK_FULL, K_PART, K_SCAN, K_H_DONE, K_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -392,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NC = p.NC;
   const bool mse = p.loss == 0;
   const int counts[K_NBARS] = {1, 1, kEpiWarps, 1, kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1,
-                               kEpiWarps, 1};
+                               kEpiWarps, 1, 1};
   uint32_t tmem;
   setup(bars, counts, K_NBARS, tmem);
   Abort ab{&bars->abort_flag, p.err};
@@ -419,11 +440,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sDO + kp * PANEL128, &tmDO, BAR(K_QDO_FULL), 64 * kp, tokc + 128 * sb);
         }
       }
-      if (mse && mbar_wait(BAR(K_QDO_FREE), (k - 1) & 1, ab)) {
+      // dV (dZ = -dV) goes into the dW slot once the only MMA that reads dW (H) is done
+      if (mse && mbar_wait(BAR(K_H_DONE), 0, ab)) {
         mbar_arrive_expect_tx(BAR(K_DV_FULL), L::BLK);
 #pragma unroll
         for (int kp = 0; kp < L::KP; ++kp)
-          tma_load_2d(sDO + kp * PANEL128, &tmDV, BAR(K_DV_FULL), 64 * kp, tokc + 128 * rb);
+          tma_load_2d(sDW + kp * PANEL128, &tmDV, BAR(K_DV_FULL), 64 * kp, tokc + 128 * rb);
       }
     }
   } else if (warp == 1) {
@@ -452,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                       sdesc_sw128(sDW + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idKK, j > 0);
         mma_commit(BAR(K_H_FULL));
+        mma_commit(BAR(K_H_DONE));
         bool ok = true;
         int k = 0;
         for (int sb = rb; sb < NB; ++sb, ++k) {
@@ -485,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int j = 0; j < D / 16; ++j)
-            mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+            mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sDW + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                         sdesc_sw128(sW0 + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idZW, 1);
         }
         mma_commit(BAR(K_DK_FULL));
@@ -603,13 +626,14 @@ struct DqL {
   static constexpr int C = 128 * NB, KP = D / 64;
   static constexpr uint32_t BLK = KP * PANEL128;
   static constexpr uint32_t WSZ = KP * D * 128;
-  static constexpr uint32_t OFF_DO = 0, OFF_W0 = BLK, OFF_K = BLK + WSZ, OFF_G = 2 * BLK + WSZ,
-                            OFF_F = 3 * BLK + WSZ;
+  // per key block rb: K_rb at OFF_K + 2 rb BLK, V_rb (then G_rb) at OFF_K + (2 rb + 1) BLK
+  static constexpr uint32_t OFF_DO = 0, OFF_W0 = BLK, OFF_K = BLK + WSZ,
+                            OFF_F = BLK + WSZ + 2 * NB * BLK;
   static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t T_DQ = 0, T_Z = 128, T_DS = 256, T_DP = 384;
 };
-enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_KV_FULL, Q_KV_FREE, Q_Z_FULL, Q_G_READY, Q_DS_FULL,
+enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_KV_FULL, Q_KV_FULL1, Q_Z_FULL, Q_G_READY, Q_DS_FULL,
        Q_DP_READY, Q_DP_FREE, Q_DQ_FULL, Q_SCAN, Q_NBARS };
 
 template <int D, int NB>
@@ -623,8 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sb0 = smem_u32(smem);
-  const uint32_t sDO = sb0 + L::OFF_DO, sW0 = sb0 + L::OFF_W0, sK = sb0 + L::OFF_K,
-                 sG = sb0 + L::OFF_G;
+  const uint32_t sDO = sb0 + L::OFF_DO, sW0 = sb0 + L::OFF_W0, sKV = sb0 + L::OFF_K;
   float* f = reinterpret_cast<float*>(smem + L::OFF_F);
   float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
         *f_cT16 = f + 1280;
@@ -651,12 +674,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(sW0 + kp * D * 128, &tmW, BAR(Q_LD0), 64 * kp, wrow);
       }
       for (int rb = 0; rb <= sb; ++rb) {
-        if (rb > 0 && !mbar_wait(BAR(Q_KV_FREE), (rb - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(BAR(Q_KV_FULL), 2 * L::BLK);
+        const uint32_t bar = BAR(Q_KV_FULL + rb);
+        const uint32_t sK = sKV + 2 * rb * L::BLK, sG = sK + L::BLK;
+        mbar_arrive_expect_tx(bar, 2 * L::BLK);
 #pragma unroll
         for (int kp = 0; kp < L::KP; ++kp) {
-          tma_load_2d(sK + kp * PANEL128, &tmK, BAR(Q_KV_FULL), 64 * kp, tokc + 128 * rb);
-          tma_load_2d(sG + kp * PANEL128, &tmV, BAR(Q_KV_FULL), 64 * kp, tokc + 128 * rb);
+          tma_load_2d(sK + kp * PANEL128, &tmK, bar, 64 * kp, tokc + 128 * rb);
+          tma_load_2d(sG + kp * PANEL128, &tmV, bar, 64 * kp, tokc + 128 * rb);
         }
       }
     }
@@ -676,7 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(BAR(Q_DQ0));
         bool ok = true;
         for (int rb = 0; rb <= sb; ++rb) {
-          if (!mbar_wait(BAR(Q_KV_FULL), rb & 1, ab)) { ok = false; break; }
+          const uint32_t sK = sKV + 2 * rb * L::BLK, sG = sK + L::BLK;
+          if (!mbar_wait(BAR(Q_KV_FULL + rb), 0, ab)) { ok = false; break; }
           tc_fence_after();
           if (mse) {
 #pragma unroll
@@ -701,7 +726,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 8; ++j)
             mma_bf16_ts(tmem + L::T_DQ, tmem + L::T_DP + 8 * j,
                         sdesc_sw128(sK + j * 2048, PANEL128, 1024), idZ, 1);
-          mma_commit(BAR(Q_KV_FREE));
           mma_commit(BAR(Q_DP_FREE));
         }
         if (!ok) break;
@@ -737,8 +761,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_arrive(BAR(Q_DQ_SCALED));
       bool ok = true;
       for (int rb = 0; rb <= sb; ++rb) {
+        const uint32_t sG = sKV + (2 * rb + 1) * L::BLK;
         // G_rb = K_rb W0 - V_rb (MSE) or -V_rb (IP), rows of the key block
-        if (!mbar_wait(BAR(Q_KV_FULL), rb & 1, ab)) { ok = false; break; }
+        if (!mbar_wait(BAR(Q_KV_FULL + rb), 0, ab)) { ok = false; break; }
         if (mse && !mbar_wait(BAR(Q_Z_FULL), rb & 1, ab)) { ok = false; break; }
         __syncwarp();
         tc_fence_after();

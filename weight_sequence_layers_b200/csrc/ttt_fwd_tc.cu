@@ -71,7 +71,7 @@ struct Layout {
 
 struct __align__(8) FwdBars {
   uint64_t kv_full, kv_free, q_full, q_free, z_full, g_ready, y_full, y_scaled, p_full, s_ready,
-      s_free, zq_full, y_free, w_full, w0_ready, scan_full, scan_free;
+      s_free, zq_full, y_free, w_full, w0_ready, scan_full, scan_free, bg_full[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(BAR(w0_ready), kEpiWarps);
     mbar_init(BAR(scan_full), 1);
     mbar_init(BAR(scan_free), kEpiWarps);
+    mbar_init(BAR(bg_full[0]), 1);
+    mbar_init(BAR(bg_full[1]), 1);
     bars->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -139,6 +141,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int qk = 0;  // Q half loads issued
+      // beta, gamma of chunk c go to buffer c & 1 on bg_full[c & 1] (phase (c >> 1) & 1),
+      // one chunk ahead of the scan that reads them
+      auto load_bg = [&](int cc) {
+        const uint32_t bg = smem_u32(f_bg + (cc & 1) * 2 * C);
+        const uint32_t bar = BAR(bg_full[cc & 1]);
+        const size_t r0 = (size_t)bh * p.T + (size_t)cc * C;
+        mbar_arrive_expect_tx(bar, (p.gamma ? 2 : 1) * C * 4);
+        bulk_g2s(bg, p.beta + r0, C * 4, bar);
+        if (p.gamma) bulk_g2s(bg + C * 4, p.gamma + r0, C * 4, bar);
+      };
+      load_bg(0);
       for (int c = 0; c < NC; ++c) {
         const int row0 = bh * p.T + c * C;
         for (int h = 0; h < NB; ++h) {
@@ -150,16 +163,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++qk;
           if (h == 0) {
             if (c > 0 && !mbar_wait(BAR(kv_free), (c - 1) & 1, ab)) goto done_prod;
-            mbar_arrive_expect_tx(BAR(kv_full), L::KV_TX + (p.gamma ? 2 : 1) * C * 4);
-            {
-              const uint32_t bg = smem_u32(f_bg + (c & 1) * 2 * C);
-              bulk_g2s(bg, p.beta + (size_t)row0, C * 4, BAR(kv_full));
-              if (p.gamma) bulk_g2s(bg + C * 4, p.gamma + (size_t)row0, C * 4, BAR(kv_full));
-            }
+            mbar_arrive_expect_tx(BAR(kv_full), L::KV_TX);
 #pragma unroll
             for (int kp = 0; kp < L::KP; ++kp)
               tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(kv_full), 64 * kp, row0);
             tma_load_2d(sV, &tmV, BAR(kv_full), NV * slice, row0);
+            if (c + 1 < NC) {
+              // buffer (c+1)&1 was last read by the scan of chunk c-1
+              if (c > 0 && !mbar_wait(BAR(scan_full), (c - 1) & 1, ab)) goto done_prod;
+              load_bg(c + 1);
+            }
           }
         }
       }
@@ -270,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // -------- per-chunk scans (warp 2) from the prefetched beta, gamma
       if (ew == 0) {
         if (c > 0 && !mbar_wait(BAR(scan_free), (c - 1) & 1, ab)) { ok = false; break; }
-        if (!mbar_wait(BAR(kv_full), c & 1, ab)) { ok = false; break; }
+        if (!mbar_wait(BAR(bg_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
         const float* bg = f_bg + (c & 1) * 2 * C;
         chunk_scan_warp<C>(bg, p.gamma ? bg + C : nullptr, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
                            f_cF16, f_cT16);
