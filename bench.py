@@ -322,11 +322,20 @@ def barrier():
 
 
 def reduce_max(x: float) -> float:
+    """Max over ranks (device tensor for NCCL, host tensor for gloo)."""
     if _dist is None:
         return x
-    t = torch.tensor([x], device="cuda", dtype=torch.float64)
+    dev = "cuda" if _dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], device=dev, dtype=torch.float64)
     _dist.all_reduce(t, op=_dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(local_ms: float, steps: int, tokens_per_rank: int, world: int):
+    """Whole-job throughput of `world` replicas: every rank processed tokens_per_rank per step;
+    the job's step time is the slowest rank's. Returns (ms_per_step, tokens_per_s)."""
+    ms = reduce_max(local_ms) / steps
+    return ms, world * tokens_per_rank / (ms * 1e-3)
 
 
 def main():
@@ -392,10 +401,8 @@ def main():
     total_ms, fwd_ms, bwd_ms, launches = time_steps(layer, args.steps, args.warmup, sampler)
     clocks = sampler.stop() if sampler else None
     assert ttt.ttt_get_device_error() == ttt.OK
-    total_ms = reduce_max(total_ms)
-    ms_step = total_ms / args.steps
+    ms_step, value = replica_throughput(total_ms, args.steps, cfg.B * cfg.T, world)
     tokens = cfg.B * cfg.T * world
-    value = tokens / (ms_step * 1e-3)
 
     work = layer_work(cfg)
     dom = "bwd" if bwd_ms >= fwd_ms else "fwd"

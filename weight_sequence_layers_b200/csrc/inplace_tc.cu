@@ -12,7 +12,8 @@
 //                 that the next chunk's apply tiles read.
 // Apply tiles (long, K = d_ff) are handed out first, update tiles fill the remaining SMs.
 // Warp roles: warp 0 issues TMA loads into a 4-stage ring, warp 1 issues tcgen05.mma into
-// two TMEM accumulators of 128 x 256 fp32, warps 2-5 drain the accumulators.
+// two TMEM accumulators of 128 x 256 fp32, warps 2-9 drain the accumulators (two warps per
+// TMEM lane quadrant, each taking 128 of the 256 columns).
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -25,7 +26,8 @@ constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, RING = 4;
 constexpr uint32_t A_BYTES = BM * BK * 2;      // 16 KB
 constexpr uint32_t B_BYTES = BN * BK * 2;      // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;            // two 256-column accumulators
 
 struct Params {
@@ -90,11 +92,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&bars->acc_full[a]), 1);
-      mbar_init(smem_u32(&bars->acc_empty[a]), 4);
+      mbar_init(smem_u32(&bars->acc_empty[a]), kEpiWarps);
     }
     for (int r = 0; r < RING; ++r) {
       mbar_init(smem_u32(&bars->tile_full[r]), 1);
-      mbar_init(smem_u32(&bars->tile_empty[r]), 5);
+      mbar_init(smem_u32(&bars->tile_empty[r]), 1 + kEpiWarps);
     }
     bars->abort_flag = 0;
     fence_barrier_init();
@@ -187,9 +189,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // Epilogue: warp w drains TMEM lanes 32*(w%4) .. +31; thread = one accumulator row.
+    // Epilogue: warp w drains TMEM lanes 32*(w%4) .. +31 (thread = one accumulator row) and
+    // columns [128 h, 128 h + 128) with h = (w - 2) / 4.
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    const int hcol = (warp - 2) / 4;
     int r = 0, acc = 0;
     uint32_t rph = 0, aph = 0;
     for (;;) {
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(smem_u32(&bars->acc_full[acc]), aph, ab)) break;
       __syncwarp();
       tc_fence_after();
-      for (int cb = 0; cb < BN / 32; ++cb) {
+      for (int cb = hcol * (BN / 64); cb < (hcol + 1) * (BN / 64); ++cb) {
         float v[32];
         tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
         tmem_wait_ld();
