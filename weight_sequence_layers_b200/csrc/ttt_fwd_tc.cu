@@ -18,7 +18,10 @@
 // score columns [64g, 64g+64) of each 128x128 score block). Every wait is bounded.
 //
 // TMEM columns: [0,64) W (lanes = key features), [64, 64+64NB) Z blocks,
-// [64+64NB, 64+128NB) Y / Zq blocks, [64+128NB, +128) one 128x128 fp32 score block P.
+// [64+64NB, 64+128NB) Y / Zq blocks, [64+128NB, +128) one 128x128 fp32 score block P, then
+// 64 columns of bf16 S (the A operand of S G, read by the MMA straight from TMEM).
+// Shared memory: K as two 128-row halves with their own full/free barriers, V double-buffered,
+// so the next chunk's loads start as soon as each buffer's last reader has finished.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -51,27 +54,26 @@ template <int D, int NB>
 struct Layout {
   static constexpr int C = 128 * NB;
   static constexpr int KP = D / 64;                      // 64-wide key-feature panels
-  static constexpr uint32_t K_PANEL = C * 128;           // one K panel (C rows)
-  static constexpr uint32_t OFF_K = 0;
-  static constexpr uint32_t OFF_Q = OFF_K + KP * K_PANEL;
-  static constexpr uint32_t OFF_V = OFF_Q + KP * PANEL128;  // V slice, overwritten by G
-  static constexpr uint32_t OFF_UG = OFF_V + C * 128;
-  static constexpr uint32_t OFF_W0 = OFF_UG + C * 128;      // bf16 state, MN-major [D][64]
-  static constexpr uint32_t OFF_S = OFF_W0 + D * 128;       // 2 panels of 128 x 64
-  static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;   // float arrays (6 x 256)
-  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;   // beta, gamma of 2 chunks (4 x C)
+  static constexpr uint32_t KH = KP * PANEL128;          // one 128-row half of K (or of Q)
+  static constexpr uint32_t OFF_K = 0;                   // K half b, panel p at OFF_K + (b KP + p) PANEL128
+  static constexpr uint32_t OFF_Q = OFF_K + NB * KH;     // one 128-row half of Q
+  static constexpr uint32_t OFF_V = OFF_Q + KH;          // V slice of chunk c in buffer c & 1; G in place
+  static constexpr uint32_t OFF_UG = OFF_V + 2 * C * 128;
+  static constexpr uint32_t OFF_W0 = OFF_UG + C * 128;   // bf16 state, MN-major [D][64]
+  static constexpr uint32_t OFF_F = OFF_W0 + D * 128;    // float arrays (6 x 256)
+  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of 2 chunks (4 x C)
   static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + 256;
-  static constexpr uint32_t KV_TX = KP * K_PANEL + C * 128;
-  static constexpr uint32_t Q_TX = KP * PANEL128;
-  static constexpr int NP = NB * (NB + 1) / 2;            // score blocks per chunk
+  static constexpr uint32_t V_TX = C * 128;
   // TMEM columns
-  static constexpr uint32_t T_W = 0, T_Z = 64, T_Y = 64 + 64 * NB, T_P = 64 + 128 * NB;
+  static constexpr uint32_t T_W = 0, T_Z = 64, T_Y = 64 + 64 * NB, T_P = 64 + 128 * NB,
+                            T_S = T_P + 128;
 };
 
 struct __align__(8) FwdBars {
-  uint64_t kv_full, kv_free, q_full, q_free, z_full, g_ready, y_full, y_scaled, p_full, s_ready,
-      s_free, zq_full, y_free, w_full, w0_ready, scan_full, scan_free, bg_full[2];
+  uint64_t k_full[2], k_free[2], v_full[2], v_free[2], q_full, q_free, z_full, g_ready, y_full,
+      y_scaled, p_full, s_ready, s_free, zq_full, y_free, w_full, w0_ready, scan_full, scan_free,
+      bg_full[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -87,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sK = sbase + L::OFF_K, sQ = sbase + L::OFF_Q, sV = sbase + L::OFF_V,
-                 sUG = sbase + L::OFF_UG, sW0 = sbase + L::OFF_W0, sS = sbase + L::OFF_S;
+                 sUG = sbase + L::OFF_UG, sW0 = sbase + L::OFF_W0;
   float* f_eta = reinterpret_cast<float*>(smem + L::OFF_F);  // eta_r
   float* f_L = f_eta + 256;                                   // L_r (chunk-local log decay)
   float* f_gam = f_L + 256;                                   // Gamma_r = exp(L_r)
@@ -102,8 +104,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #define BAR(x) smem_u32(&bars->x)
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(kv_full), 1);
-    mbar_init(BAR(kv_free), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(k_full[i]), 1);
+      mbar_init(BAR(k_free[i]), 1);
+      mbar_init(BAR(v_full[i]), 1);
+      mbar_init(BAR(v_free[i]), 1);
+    }
     mbar_init(BAR(q_full), 1);
     mbar_init(BAR(q_free), 1);
     mbar_init(BAR(z_full), 1);
@@ -154,25 +160,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_bg(0);
       for (int c = 0; c < NC; ++c) {
         const int row0 = bh * p.T + c * C;
+        // V slice of chunk c into buffer c & 1, free once chunk c-2's last S G MMA is done
+        const int vb = c & 1;
+        if (c >= 2 && !mbar_wait(BAR(v_free[vb]), ((c - 2) >> 1) & 1, ab)) goto done_prod;
+        mbar_arrive_expect_tx(BAR(v_full[vb]), L::V_TX);
+        tma_load_2d(sV + vb * C * 128, &tmV, BAR(v_full[vb]), NV * slice, row0);
         for (int h = 0; h < NB; ++h) {
+          // K half h of chunk c, free once its last reader of chunk c-1 is done
+          if (c > 0 && !mbar_wait(BAR(k_free[h]), (c - 1) & 1, ab)) goto done_prod;
+          mbar_arrive_expect_tx(BAR(k_full[h]), L::KH);
+#pragma unroll
+          for (int kp = 0; kp < L::KP; ++kp)
+            tma_load_2d(sK + (h * L::KP + kp) * PANEL128, &tmK, BAR(k_full[h]), 64 * kp,
+                        row0 + 128 * h);
           if (qk > 0 && !mbar_wait(BAR(q_free), (qk - 1) & 1, ab)) goto done_prod;
-          mbar_arrive_expect_tx(BAR(q_full), L::Q_TX);
+          mbar_arrive_expect_tx(BAR(q_full), L::KH);
 #pragma unroll
           for (int kp = 0; kp < L::KP; ++kp)
             tma_load_2d(sQ + kp * PANEL128, &tmQ, BAR(q_full), 64 * kp, row0 + 128 * h);
           ++qk;
-          if (h == 0) {
-            if (c > 0 && !mbar_wait(BAR(kv_free), (c - 1) & 1, ab)) goto done_prod;
-            mbar_arrive_expect_tx(BAR(kv_full), L::KV_TX);
-#pragma unroll
-            for (int kp = 0; kp < L::KP; ++kp)
-              tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(kv_full), 64 * kp, row0);
-            tma_load_2d(sV, &tmV, BAR(kv_full), NV * slice, row0);
-            if (c + 1 < NC) {
-              // buffer (c+1)&1 was last read by the scan of chunk c-1
-              if (c > 0 && !mbar_wait(BAR(scan_full), (c - 1) & 1, ab)) goto done_prod;
-              load_bg(c + 1);
-            }
+          if (h == 0 && c + 1 < NC) {
+            // buffer (c+1)&1 was last read by the scan of chunk c-1
+            if (c > 0 && !mbar_wait(BAR(scan_full), (c - 1) & 1, ab)) goto done_prod;
+            load_bg(c + 1);
           }
         }
       }
@@ -184,21 +194,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idZ = idesc_bf16(128, NV, 0, 1);   // K-major A, MN-major B
       const uint32_t idP = idesc_bf16(128, 128, 0, 0);  // K-major A and B
       const uint32_t idW = idesc_bf16(128, NV, 1, 1);   // MN-major A and B
-      const uint32_t lboKt = D == 128 ? L::K_PANEL : 0;  // second 64-row block of K^T
+      const uint32_t lboKt = D == 128 ? PANEL128 : 0;  // second 64-row block of K^T
       int kq = 0, ks = 0;
       for (int c = 0; c < NC; ++c) {
-        if (!mbar_wait(BAR(kv_full), c & 1, ab)) break;
+        const uint32_t sVc = sV + (c & 1) * C * 128;
         if (!mbar_wait(BAR(w0_ready), c & 1, ab)) break;
-        tc_fence_after();
         // Z_b = K_b W0
-        for (int b = 0; b < NB; ++b)
+        bool ok = true;
+        for (int b = 0; b < NB; ++b) {
+          if (!mbar_wait(BAR(k_full[b]), c & 1, ab)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
           for (int j = 0; j < D / 16; ++j)
             mma_bf16_ss(tmem + L::T_Z + NV * b,
-                        sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sK + (b * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                         sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
+        }
+        if (!ok) break;
         mma_commit(BAR(z_full));
-        bool ok = true;
         for (int h = 0; h < NB && ok; ++h) {
           if (!mbar_wait(BAR(q_full), kq & 1, ab)) { ok = false; break; }
           ++kq;
@@ -215,8 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < D / 16; ++j)
               mma_bf16_ss(tmem + L::T_P,
                           sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                          sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16,
-                                      1024),
+                          sdesc_sw128(sK + (b * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                           idP, j > 0);
             mma_commit(BAR(p_full));
             if (b == h) mma_commit(BAR(q_free));
@@ -225,26 +237,28 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!mbar_wait(BAR(g_ready), c & 1, ab)) { ok = false; break; }
               tc_fence_after();
               for (int j = 0; j < C / 16; ++j)
-                mma_bf16_ss(tmem + L::T_W, sdesc_sw128(sK + j * 2048, lboKt, 1024),
+                mma_bf16_ss(tmem + L::T_W,
+                            sdesc_sw128(sK + (j / 8) * L::KH + (j % 8) * 2048, lboKt, 1024),
                             sdesc_sw128(sUG + j * 2048, 0, 1024), idW, 1);
               mma_commit(BAR(w_full));
             }
+            // release K half b after its last reader (P_{NB-1,b}; with one block also W)
+            if (h == NB - 1) mma_commit(BAR(k_free[b]));
             if (!mbar_wait(BAR(s_ready), ks & 1, ab)) { ok = false; break; }
             if (b == 0 && !mbar_wait(BAR(y_scaled), (c * NB + h) & 1, ab)) { ok = false; break; }
             ++ks;
             tc_fence_after();
-            // Zq_h += (-S_hb) G_b
+            // Zq_h += (-S_hb) G_b, S (bf16) read from TMEM
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              mma_bf16_ss(tmem + L::T_Y + NV * h,
-                          sdesc_sw128(sS + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                          sdesc_sw128(sV + b * PANEL128 + j * 2048, 0, 1024), idZ, 1);
+              mma_bf16_ts(tmem + L::T_Y + NV * h, tmem + L::T_S + 8 * j,
+                          sdesc_sw128(sVc + b * PANEL128 + j * 2048, 0, 1024), idZ, 1);
             mma_commit(BAR(s_free));
           }
           if (ok) mma_commit(BAR(zq_full));
         }
         if (!ok) break;
-        mma_commit(BAR(kv_free));
+        mma_commit(BAR(v_free[c & 1]));
       }
     }
   } else {
@@ -293,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float gamC = f_gam[C - 1];
 
       // -------- train view: G = a(Z) act'(Z) in place over V, -u*G, state decay
-      if (!mbar_wait(BAR(kv_full), c & 1, ab)) { ok = false; break; }
+      const uint32_t sVc = sV + (c & 1) * C * 128;
+      if (!mbar_wait(BAR(v_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
       if (!mbar_wait(BAR(z_full), c & 1, ab)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
@@ -302,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem + lane_off + L::T_Z + NV * b + 32 * g, z);
         tmem_wait_ld();
         const int row = 128 * b + lrow;
-        ld_row32(sV, row, 4 * g, v);
+        ld_row32(sVc, row, 4 * g, v);
         const float un = -f_eta[row] * f_eLC[row];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -311,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           v[j] = gg;
           z[j] = un * gg;
         }
-        st_row32(sV, row, 4 * g, v);
+        st_row32(sVc, row, 4 * g, v);
         st_row32(sUG, row, 4 * g, z);
       }
       if (w_rows) {
@@ -392,9 +407,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; ++j) sv[j] = -sv[j] * w[j];
-            st_row32(sS + g * PANEL128, lrow, 4 * half, sv);
+            uint32_t pk[16];
+            pack32(sv, pk);
+            tmem_st16u(tmem + lane_off + L::T_S + 32 * g + 16 * half, pk);
           }
-          fence_proxy_async_smem();
+          tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(BAR(s_ready));
@@ -438,7 +455,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   using L = Layout<D, NB>;
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
   CUtensorMap tk, tq, tv;
-  if (!make_tmap_bf16(&tk, a.K, D, rows, D, 64, L::C) ||
+  if (!make_tmap_bf16(&tk, a.K, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tq, a.Q, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tv, a.V, D, rows, D, 64, L::C))
     return cudaErrorInvalidValue;
