@@ -15,7 +15,8 @@
 //
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner), warps 2-9 epilogue
 // (two warpgroups; warpgroup g handles value columns [32g, 32g+32) of each 128-row block and
-// score columns [64g, 64g+64) of each 128x128 score block). Every wait is bounded.
+// score columns [64g, 64g+64) of each 128x128 score block), warp 10 computes the lr and decay
+// scans of the next chunk into the other of two buffers. Every wait is bounded.
 //
 // TMEM columns: [0,64) W (lanes = key features), [64, 64+64NB) Z blocks,
 // [64+64NB, 64+128NB) Y / Zq blocks, [64+128NB, +128) one 128x128 fp32 score block P, then
@@ -33,7 +34,7 @@ namespace tttk {
 namespace {
 
 constexpr int NV = 64;             // value columns per CTA
-constexpr int kThreads = 320;      // 10 warps
+constexpr int kThreads = 352;      // 11 warps
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t PANEL128 = 128 * 128;  // 128 rows x 128 bytes
@@ -60,8 +61,8 @@ struct Layout {
   static constexpr uint32_t OFF_V = OFF_Q + KH;          // V slice of chunk c in buffer c & 1; G in place
   static constexpr uint32_t OFF_UG = OFF_V + 2 * C * 128;
   static constexpr uint32_t OFF_W0 = OFF_UG + C * 128;   // bf16 state, MN-major [D][64]
-  static constexpr uint32_t OFF_F = OFF_W0 + D * 128;    // float arrays (6 x 256)
-  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of 2 chunks (4 x C)
+  static constexpr uint32_t OFF_F = OFF_W0 + D * 128;    // scan arrays, 2 buffers x 6 x 256
+  static constexpr uint32_t OFF_BG = OFF_F + 2 * 6 * 256 * 4;  // beta, gamma of 2 chunks
   static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + 256;
   static constexpr uint32_t V_TX = C * 128;
@@ -72,8 +73,8 @@ struct Layout {
 
 struct __align__(8) FwdBars {
   uint64_t k_full[2], k_free[2], v_full[2], v_free[2], q_full, q_free, z_full, g_ready, y_full,
-      y_scaled, p_full, s_ready, s_free, zq_full, y_free, w_full, w0_ready, scan_full, scan_free,
-      bg_full[2];
+      y_scaled, p_full, s_ready, s_free, zq_full, y_free, w_full, w0_ready, scan_full[2],
+      scan_free[2], bg_full[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -90,12 +91,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
   const uint32_t sK = sbase + L::OFF_K, sQ = sbase + L::OFF_Q, sV = sbase + L::OFF_V,
                  sUG = sbase + L::OFF_UG, sW0 = sbase + L::OFF_W0;
-  float* f_eta = reinterpret_cast<float*>(smem + L::OFF_F);  // eta_r
-  float* f_L = f_eta + 256;                                   // L_r (chunk-local log decay)
-  float* f_gam = f_L + 256;                                   // Gamma_r = exp(L_r)
-  float* f_eLC = f_gam + 256;                                 // exp(L_C - L_r)
-  float* f_cF16 = f_eLC + 256;                                // eta_r exp(L_{r16} - L_r)
-  float* f_cT16 = f_cF16 + 256;                               // exp(L_r - L_{r16})
+  // scan arrays of buffer i: eta, L (chunk-local log decay), Gamma = exp(L), exp(L_C - L),
+  // cF16 = eta exp(L_{r16} - L), cT16 = exp(L - L_{r16})
+  float* f_scan = reinterpret_cast<float*>(smem + L::OFF_F);
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);   // [parity][beta, gamma][C]
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -123,8 +121,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(BAR(y_free), kEpiWarps);
     mbar_init(BAR(w_full), 1);
     mbar_init(BAR(w0_ready), kEpiWarps);
-    mbar_init(BAR(scan_full), 1);
-    mbar_init(BAR(scan_free), kEpiWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(scan_full[i]), 1);
+      mbar_init(BAR(scan_free[i]), kEpiWarps);
+    }
     mbar_init(BAR(bg_full[0]), 1);
     mbar_init(BAR(bg_full[1]), 1);
     bars->abort_flag = 0;
@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++qk;
           if (h == 0 && c + 1 < NC) {
             // buffer (c+1)&1 was last read by the scan of chunk c-1
-            if (c > 0 && !mbar_wait(BAR(scan_full), (c - 1) & 1, ab)) goto done_prod;
+            if (c > 0 && !mbar_wait(BAR(scan_full[(c - 1) & 1]), ((c - 1) >> 1) & 1, ab))
+              goto done_prod;
             load_bg(c + 1);
           }
         }
@@ -261,6 +262,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(BAR(v_free[c & 1]));
       }
     }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------------ scans, one chunk ahead
+    for (int c = 0; c < NC; ++c) {
+      const int sb = c & 1;
+      if (c >= 2 && !mbar_wait(BAR(scan_free[sb]), ((c - 2) >> 1) & 1, ab)) break;
+      if (!mbar_wait(BAR(bg_full[sb]), (c >> 1) & 1, ab)) break;
+      const float* bg = f_bg + sb * 2 * C;
+      float* fs = f_scan + sb * 6 * 256;
+      chunk_scan_warp<C>(bg, p.gamma ? bg + C : nullptr, p.lr_bias, fs, fs + 256, fs + 512,
+                         fs + 768, fs + 1024, fs + 1280);
+      if (lane == 0) mbar_arrive(BAR(scan_full[sb]));
+    }
   } else {
     // ------------------------------------------------------------------ epilogue
     const int ew = warp - 2;          // 0..7
@@ -294,16 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kp = 0;  // score blocks consumed
     for (int c = 0; c < NC && ok; ++c) {
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
-      // -------- per-chunk scans (warp 2) from the prefetched beta, gamma
-      if (ew == 0) {
-        if (c > 0 && !mbar_wait(BAR(scan_free), (c - 1) & 1, ab)) { ok = false; break; }
-        if (!mbar_wait(BAR(bg_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
-        const float* bg = f_bg + (c & 1) * 2 * C;
-        chunk_scan_warp<C>(bg, p.gamma ? bg + C : nullptr, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
-                           f_cF16, f_cT16);
-        if (lane == 0) mbar_arrive(BAR(scan_full));
-      }
-      if (!mbar_wait(BAR(scan_full), c & 1, ab)) { ok = false; break; }
+      // -------- this chunk's scan arrays (computed by warp 10)
+      if (!mbar_wait(BAR(scan_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
+      const float* f_eta = f_scan + (c & 1) * 6 * 256;
+      const float* f_L = f_eta + 256;
+      const float* f_gam = f_eta + 512;
+      const float* f_eLC = f_eta + 768;
+      const float* f_cF16 = f_eta + 1024;
       const float gamC = f_gam[C - 1];
 
       // -------- train view: G = a(Z) act'(Z) in place over V, -u*G, state decay
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (h == NB - 1) {
           __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(scan_free));
+          if (lane == 0) mbar_arrive(BAR(scan_free[c & 1]));
         }
         // -------- O_h = act(Zq_h)
         if (!mbar_wait(BAR(zq_full), (c * NB + h) & 1, ab)) { ok = false; break; }
