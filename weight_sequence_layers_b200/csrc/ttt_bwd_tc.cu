@@ -109,11 +109,14 @@ struct ChainL {
   static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t TX = 2 * KP * K_PANEL + C * 128;
-  static constexpr uint32_t T_DW = 0, T_X = 64, T_Y = 64 + 64 * NB, T_P = 64 + 128 * NB;
+  // P^T blocks alternate between two TMEM buffers; Y reuses buffer 0 after the score loop
+  static constexpr uint32_t T_DW = 0, T_X = 64, T_P0 = 64 + 64 * NB, T_P1 = T_P0 + 128,
+                            T_Y = T_P0;
+  static constexpr int NP = NB * (NB + 1) / 2;
 };
 enum { C_KV_FULL, C_KV_FREE, C_P_FULL, C_S_READY, C_S_FREE, C_X_FULL, C_W_READY, C_Y_FULL,
        C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_BG_FULL, C_BG_FULL1,
-       C_NBARS };
+       C_P_FULL1, C_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -136,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NC = p.NC;
   const bool mse = p.loss == 0;
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
-                               kEpiWarps, 1, 1};
+                               kEpiWarps, 1, 1, 1};
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   uint32_t tmem;
   setup(bars, counts, C_NBARS, tmem);
@@ -183,28 +186,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(BAR(C_KV_FULL), it & 1, ab)) break;
         tc_fence_after();
         bool ok = true;
-        for (int rb = 0; rb < NB && ok; ++rb)
-          for (int sb = rb; sb < NB; ++sb) {
-            // P^T block = K_rb Q_sb^T
+        // score blocks in order k = (rb, sb), sb >= rb; P^T_k goes to TMEM buffer k & 1 and the
+        // next-but-one block is issued as soon as the epilogue has consumed this buffer
+        auto issue_p = [&](int k) {
+          const int rb = k < NB ? 0 : 1, sb = k < NB ? k : 1;  // NB <= 2
 #pragma unroll
-            for (int j = 0; j < D / 16; ++j)
-              mma_bf16_ss(tmem + L::T_P,
-                          sdesc_sw128(sK + (j / 4) * L::K_PANEL + rb * PANEL128 + (j % 4) * 32, 16, 1024),
-                          sdesc_sw128(sQ + (j / 4) * L::K_PANEL + sb * PANEL128 + (j % 4) * 32, 16, 1024),
-                          idP, j > 0);
-            mma_commit(BAR(C_P_FULL));
-            if (!mbar_wait(BAR(C_S_READY), kp & 1, ab)) { ok = false; break; }
-            ++kp;
-            tc_fence_after();
-            // X_rb += S^T_(rb,sb) dO_sb
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + ((k & 1) ? L::T_P1 : L::T_P0),
+                        sdesc_sw128(sK + (j / 4) * L::K_PANEL + rb * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sQ + (j / 4) * L::K_PANEL + sb * PANEL128 + (j % 4) * 32, 16, 1024),
+                        idP, j > 0);
+          // one barrier per P buffer: a buffer's next use waits for the epilogue's release of
+          // the previous one, so its barrier is never more than one phase ahead of the waiter
+          mma_commit(BAR((k & 1) ? C_P_FULL1 : C_P_FULL));
+        };
+        issue_p(0);
+        if (L::NP > 1) issue_p(1);
+        for (int k = 0; k < L::NP; ++k) {
+          const int rb = k < NB ? 0 : 1, sb = k < NB ? k : 1;
+          if (!mbar_wait(BAR(C_S_READY), kp & 1, ab)) { ok = false; break; }
+          ++kp;
+          tc_fence_after();
+          if (k + 2 < L::NP) issue_p(k + 2);
+          // X_rb += S^T_(rb,sb) dO_sb
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              mma_bf16_ss(tmem + L::T_X + NV * rb,
-                          sdesc_sw128(sS + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                          sdesc_sw128(sDO + sb * PANEL128 + j * 2048, 0, 1024), idX,
-                          (sb != rb) || (j > 0));
-            mma_commit(BAR(C_S_FREE));
-          }
+          for (int j = 0; j < 8; ++j)
+            mma_bf16_ss(tmem + L::T_X + NV * rb,
+                        sdesc_sw128(sS + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sDO + sb * PANEL128 + j * 2048, 0, 1024), idX,
+                        (sb != rb) || (j > 0));
+          mma_commit(BAR(C_S_FREE));
+        }
         if (!ok) break;
         mma_commit(BAR(C_X_FULL));
         // Y_b = K_b dW
@@ -217,7 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16, 1024),
                         sdesc_sw128(sDW + j * 2048, 0, 1024), idX, j > 0);
         mma_commit(BAR(C_Y_FULL));
-        // dW (already Gamma_C-scaled) += (Gamma Q)^T dO + K^T dZ
+        // dW (already Gamma_C-scaled) += Q^T (Gamma dO) + K^T dZ
         if (!mbar_wait(BAR(C_QS_READY), it & 1, ab)) break;
         tc_fence_after();
         for (int j = 0; j < C / 16; ++j)
@@ -259,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     epi_arrive(BAR(C_W_READY));
     int kp = 0;
+    int puse[2] = {0, 0};  // completed uses of each P buffer
     for (int it = 0; it < NC && ok; ++it) {
       const int c = NC - 1 - it;
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
@@ -271,46 +284,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(BAR(C_SCAN_FULL));
       }
       if (!mbar_wait(BAR(C_SCAN_FULL), it & 1, ab)) { ok = false; break; }
-      // ---- S^T blocks: S^T_rs = P^T_rs eta_r exp(L_s - L_r), s >= r
-      for (int rb = 0; rb < NB && ok; ++rb) {
+      // ---- S^T blocks: S^T_rs = P^T_rs eta_r exp(L_s - L_r), s >= r (block k in TMEM buffer k & 1)
+      for (int k = 0; k < L::NP && ok; ++k) {
+        const int rb = k < NB ? 0 : 1, sb = k < NB ? k : 1;
         const int r = 128 * rb + lrow;
         const float Lr = f_L[r], er = f_eta[r];
-        for (int sb = rb; sb < NB; ++sb) {
-          if (!mbar_wait(BAR(C_P_FULL), kp & 1, ab)) { ok = false; break; }
-          if (kp > 0 && !mbar_wait(BAR(C_S_FREE), (kp - 1) & 1, ab)) { ok = false; break; }
-          ++kp;
-          __syncwarp();
-          tc_fence_after();
-          const int s0 = 128 * sb + 64 * g;
+        if (!mbar_wait(BAR((k & 1) ? C_P_FULL1 : C_P_FULL), puse[k & 1] & 1, ab)) { ok = false; break; }
+        ++puse[k & 1];
+        if (kp > 0 && !mbar_wait(BAR(C_S_FREE), (kp - 1) & 1, ab)) { ok = false; break; }
+        ++kp;
+        __syncwarp();
+        tc_fence_after();
+        const int s0 = 128 * sb + 64 * g;
+        const uint32_t tp = (k & 1) ? L::T_P1 : L::T_P0;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            float v[32], w[32];
-            tmem_ld32(tmem + loff + L::T_P + 64 * g + 32 * half, v);
-            causal_weights_k(f_L, f_cT16, r, Lr, s0 + 32 * half, w);
-            tmem_wait_ld();
+        for (int half = 0; half < 2; ++half) {
+          float v[32], w[32];
+          tmem_ld32(tmem + loff + tp + 64 * g + 32 * half, v);
+          causal_weights_k(f_L, f_cT16, r, Lr, s0 + 32 * half, w);
+          tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= er * w[j];
-            st_row32(sS + g * PANEL128, lrow, 4 * half, v);
-          }
-          epi_arrive(BAR(C_S_READY));
+          for (int j = 0; j < 32; ++j) v[j] *= er * w[j];
+          st_row32(sS + g * PANEL128, lrow, 4 * half, v);
         }
+        epi_arrive(BAR(C_S_READY));
       }
       if (!ok) break;
-      // ---- scale Q rows by Gamma_s (all score MMAs are done) and the state by Gamma_C
+      // ---- scale dO rows by Gamma_s (X, the only other reader of dO, is done) and the state
+      // by Gamma_C
       if (!mbar_wait(BAR(C_X_FULL), it & 1, ab)) { ok = false; break; }
       for (int s = ew * 32 + lane; s < C; s += kEpiWarps * 32) {
         const float gs = f_gam[s];
-        for (int kp2 = 0; kp2 < L::KP; ++kp2)
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint32_t a = sQ + kp2 * L::K_PANEL + sw128_off(s, ch);
-            uint32_t w0, w1, w2, w3;
-            ld_shared_v4(a, w0, w1, w2, w3);
-            st_shared_v4(a, pack_bf16x2(bf16lo(w0) * gs, bf16hi(w0) * gs),
-                         pack_bf16x2(bf16lo(w1) * gs, bf16hi(w1) * gs),
-                         pack_bf16x2(bf16lo(w2) * gs, bf16hi(w2) * gs),
-                         pack_bf16x2(bf16lo(w3) * gs, bf16hi(w3) * gs));
-          }
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t a = sDO + sw128_off(s, ch);
+          uint32_t w0, w1, w2, w3;
+          ld_shared_v4(a, w0, w1, w2, w3);
+          st_shared_v4(a, pack_bf16x2(bf16lo(w0) * gs, bf16hi(w0) * gs),
+                       pack_bf16x2(bf16lo(w1) * gs, bf16hi(w1) * gs),
+                       pack_bf16x2(bf16lo(w2) * gs, bf16hi(w2) * gs),
+                       pack_bf16x2(bf16lo(w3) * gs, bf16hi(w3) * gs));
+        }
       }
       __syncwarp();
       tc_fence_after();
@@ -325,10 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       epi_arrive(BAR(C_QS_READY));
-      // ---- dG = -X - u Y ; dV = -dG ; dZ = dG (MSE)
+      // ---- dG = -X - u Y ; dZ = dG (MSE) is published first, dV = -dG stored after
       if (!mbar_wait(BAR(C_Y_FULL), it & 1, ab)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
+      float dg[NB][32];
+#pragma unroll
       for (int b = 0; b < NB; ++b) {
         const int r = 128 * b + lrow;
         float x[32], y[32];
@@ -337,14 +353,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         const float u = f_eta[r] * f_eLC[r];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          x[j] = -x[j] - u * y[j];  // dG
-          y[j] = -x[j];             // dV
-        }
-        st_global_bf16x32(p.dV + (tok0 + r) * D + NV * slice + 32 * g, y);
-        if (mse) st_row32(sS, r, 4 * g, x);
+        for (int j = 0; j < 32; ++j) dg[b][j] = -x[j] - u * y[j];
+        if (mse) st_row32(sS, r, 4 * g, dg[b]);
       }
       epi_arrive(BAR(C_DZ_READY));
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dg[b][j] = -dg[b][j];
+        st_global_bf16x32(p.dV + (tok0 + 128 * b + lrow) * D + NV * slice + 32 * g, dg[b]);
+      }
       // ---- adjoint at the end of chunk c-1 (or dW0)
       if (!mbar_wait(BAR(C_DW_FULL), it & 1, ab)) { ok = false; break; }
       __syncwarp();
