@@ -113,12 +113,12 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
  * Some callers cannot allocate device memory when they call the library: a host framework
  * that owns every byte of device memory through its own pool, or a plugin that is handed only
  * its input and output buffers. For them this variant takes the same arguments as
- * ttt_chunk_bwd minus the workspace, and keeps its scratch (the per-chunk adjoint states) in
- * a fixed array of TTT_NOALLOC_SCRATCH_BYTES that the library holds on every GPU it is loaded
+ * ttt_chunk_bwd minus the workspace, and keeps its scratch (the per-chunk adjoint states and
+ * the bf16 inner-loss gradient G of every token) in a fixed array of TTT_NOALLOC_SCRATCH_BYTES that the library holds on every GPU it is loaded
  * on, until the process exits. It allocates nothing and calls no allocating routine.
  *  - Only configs of the tensor-core backward are accepted (bf16, identity activation,
  *    dk == dv in {64, 128}, C in {128, 256}); others return TTT_ERR_UNSUPPORTED.
- *  - Configs needing more than the fixed scratch (B*H*(T/C)*dk*dv*2 bytes) return
+ *  - Configs needing more than the fixed scratch (B*H*(T/C)*dk*dv*2 + B*H*T*dv*2 bytes) return
  *    TTT_ERR_WORKSPACE with nothing launched; ttt_chunk_bwd serves those.
  *  - The first call on a device looks up the array's device address (with that device
  *    current); make that first call before any stream capture.

@@ -54,7 +54,7 @@ def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
 
 
 def test_noalloc_backward_refuses_configs_beyond_its_scratch():
-    big = abi_config(synth.TRAIN_1P45B)  # needs 32 MiB of scratch
+    big = abi_config(synth.TRAIN_1P45B)  # needs 96 MiB of scratch
     A = 4096  # never dereferenced: the size check comes first
     st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(big), A, A, A, A, A, A, A, A, None, A, A, A, A,
                                        A, None)

@@ -128,6 +128,70 @@ __device__ __forceinline__ void causal_weights_k(const float* L, const float* cT
   }
 }
 
+// -S for one query s (chunk-local) against 32 keys r0.. (r0 % 32 == 0), packed to bf16 pairs:
+//   S_sr = P_sr eta_r exp(L_s - L_r) = P_sr exp(L_s - L_{r16}) cF16_r,  r16 = r & ~15,
+// with one exponential per 16 keys. MASK: some keys lie after s and are zeroed.
+template <bool MASK>
+__device__ __forceinline__ void score_weights32(const float (&pv)[32], const float* Lv,
+                                                const float* cF16, int s, float Ls, int r0,
+                                                uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int g16 = 0; g16 < 2; ++g16) {
+    const int r16 = r0 + 16 * g16;
+    float a = -__expf(Ls - Lv[r16]);
+    if (MASK && s < r16) a = 0.f;
+    const float4* c4 = reinterpret_cast<const float4*>(cF16 + r16);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 cf = c4[k];
+      const int j = 16 * g16 + 4 * k;
+      float x0 = pv[j] * cf.x * a, x1 = pv[j + 1] * cf.y * a;
+      float x2 = pv[j + 2] * cf.z * a, x3 = pv[j + 3] * cf.w * a;
+      if (MASK) {
+        const int r = r16 + 4 * k;
+        if (r > s) x0 = 0.f;
+        if (r + 1 > s) x1 = 0.f;
+        if (r + 2 > s) x2 = 0.f;
+        if (r + 3 > s) x3 = 0.f;
+      }
+      pk[8 * g16 + 2 * k] = pack_bf16x2(x0, x1);
+      pk[8 * g16 + 2 * k + 1] = pack_bf16x2(x2, x3);
+    }
+  }
+}
+
+// -dP^T for one key r (chunk-local) against 32 queries s0.. (s0 % 32 == 0), packed to bf16:
+//   M^T_rs = eta_r exp(L_s - L_r) = eta_r exp(L_{s16} - L_r) cT16_s,  s16 = s & ~15,
+// for s >= r, with one exponential per 16 queries. MASK: some queries precede r.
+template <bool MASK>
+__device__ __forceinline__ void score_weights32_k(const float (&pv)[32], const float* Lv,
+                                                  const float* cT16, int r, float Lr, float er,
+                                                  int s0, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int g16 = 0; g16 < 2; ++g16) {
+    const int s16 = s0 + 16 * g16;
+    float a = -er * __expf(Lv[s16] - Lr);
+    if (MASK && s16 + 15 < r) a = 0.f;
+    const float4* c4 = reinterpret_cast<const float4*>(cT16 + s16);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 cf = c4[k];
+      const int j = 16 * g16 + 4 * k;
+      float x0 = pv[j] * cf.x * a, x1 = pv[j + 1] * cf.y * a;
+      float x2 = pv[j + 2] * cf.z * a, x3 = pv[j + 3] * cf.w * a;
+      if (MASK) {
+        const int s = s16 + 4 * k;
+        if (s < r) x0 = 0.f;
+        if (s + 1 < r) x1 = 0.f;
+        if (s + 2 < r) x2 = 0.f;
+        if (s + 3 < r) x3 = 0.f;
+      }
+      pk[8 * g16 + 2 * k] = pack_bf16x2(x0, x1);
+      pk[8 * g16 + 2 * k + 1] = pack_bf16x2(x2, x3);
+    }
+  }
+}
+
 // Bulk copy of `bytes` (multiple of 16, 16-byte aligned) from global to shared memory,
 // completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

@@ -14,14 +14,17 @@
 //   deta_r = sum_s dS_sr P_sr exp(L_s - L_r) - exp(L_C - L_r) K_r . (G_r dW^T)
 //   dbeta = deta * eta (1 - eta / 2)
 //
-// Three kernels:
+// Four kernels:
+//   g     : G = K W0 - V (MSE) or -V (IP) of every token from the saved chunk-start states,
+//           stored once (bf16) in the workspace.
 //   chain : one CTA per (batch, head, 64-wide value slice) walks the chunks backwards with
 //           dW (fp32) resident in TMEM, writing dV, dW0 and the bf16 adjoint at the end of
 //           every chunk (workspace). Columns of dW, X, Y, dG, dV are independent.
-//   dk    : one CTA per (batch, head, chunk, 128-key block): dK and dbeta of those keys.
 //   dq    : one CTA per (batch, head, chunk, 128-query block): dQ of those queries.
-// The two chunk-parallel kernels recompute G and the score blocks from the saved chunk-start
-// state and hold dP (bf16) in TMEM as the A operand of their last contraction.
+//   dk    : one CTA per (batch, head, chunk, 128-key block): dK and dbeta of those keys,
+//           with deta_r = (G_r . dG_r) / eta_r (see the dK kernel).
+// dq and dk rebuild the score-gradient blocks from G and dO and hold dP (bf16) in TMEM as the
+// A operand of their last contraction; they run two CTAs per SM.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -47,6 +50,7 @@ struct BwdParams {
   __nv_bfloat16* dV;          // chain: out; dk: in (dZ = -dV for MSE)
   float* dW0;
   __nv_bfloat16* dWs;         // [BH, NC, D, D] adjoint at the end of each chunk
+  __nv_bfloat16* G;           // [BH, T, D] inner-loss gradient G of every token
   __nv_bfloat16* dQ;
   __nv_bfloat16* dK;
   float* dbeta;
@@ -61,7 +65,8 @@ struct __align__(8) Bars {
 
 #define BAR(i) smem_u32(&bars->b[i])
 
-__device__ __forceinline__ void setup(Bars* bars, const int* counts, int n, uint32_t& tmem) {
+__device__ __forceinline__ void setup(Bars* bars, const int* counts, int n, uint32_t& tmem,
+                                      uint32_t ncols = kTmemCols) {
   const int warp = threadIdx.x / 32;
   if (threadIdx.x == 0) {
     for (int i = 0; i < n; ++i) mbar_init(BAR(i), counts[i]);
@@ -69,7 +74,7 @@ __device__ __forceinline__ void setup(Bars* bars, const int* counts, int n, uint
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_alloc(smem_u32(&bars->tmem_base), ncols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -78,13 +83,13 @@ __device__ __forceinline__ void setup(Bars* bars, const int* counts, int n, uint
   tmem = bars->tmem_base;
 }
 
-__device__ __forceinline__ void teardown(Bars* bars, uint32_t tmem) {
+__device__ __forceinline__ void teardown(Bars* bars, uint32_t tmem, uint32_t ncols = kTmemCols) {
   tc_fence_before();
   __syncthreads();
   if (bars->abort_flag) __nanosleep(100000);
   if (threadIdx.x / 32 == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, ncols);
   }
 }
 
@@ -389,171 +394,80 @@ __global__ void __launch_bounds__(kThreads, 1)
   teardown(bars, tmem);
 }
 
-// ================================================================================== dK
-template <int D, int NB>
-struct DkL {
-  static constexpr int C = 128 * NB, KP = D / 64;
+// =================================================================== chunk-parallel kernels
+// Three warps' worth of roles in 192 threads (producer, MMA issuer, four epilogue warps, one per
+// TMEM lane quadrant), at most ~100 KB of shared memory and 256 TMEM columns, so two CTAs share
+// an SM and each one's load and handshake latencies hide behind the other's work.
+constexpr int kSmallThreads = 192;
+constexpr int kSmallEpi = 4;
+
+// ------------------------------------------------------------------------------------ G
+// G = K W0 - V (MSE) or -V (IP) of one 128-token block with the chunk's saved state W0, stored
+// once (bf16) for the dQ and dK kernels.
+template <int D>
+struct GL {
+  static constexpr int KP = D / 64;
   static constexpr uint32_t BLK = KP * PANEL128;  // 128 rows x D
   static constexpr uint32_t WSZ = KP * D * 128;   // D rows x D
-  // the dW slot later receives a 128-row dV block, so it holds the larger of the two
-  static constexpr uint32_t DWSZ = WSZ > BLK ? WSZ : BLK;
-  static constexpr uint32_t OFF_K = 0, OFF_G = BLK, OFF_W0 = 2 * BLK, OFF_DW = 2 * BLK + WSZ,
-                            OFF_Q = OFF_DW + DWSZ, OFF_DO = OFF_Q + BLK, OFF_F = OFF_DO + BLK;
-  static constexpr uint32_t OFF_BAR = OFF_F + 8 * 256 * 4;
+  static constexpr uint32_t OFF_K = 0, OFF_W0 = BLK, OFF_V = BLK + WSZ, OFF_BAR = 2 * BLK + WSZ;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
-  static constexpr uint32_t T_ZDP = 0, T_DK = 128, T_DS = 256, T_P = 384;
 };
-enum { K_LD_FULL, K_Z_FULL, K_G_READY, K_H_FULL, K_H_SCALED, K_QDO_FULL, K_QDO_FREE, K_SP_FULL,
-       K_DP_READY, K_DP_FREE, K_DV_FULL, K_DK_FULL, K_PART, K_SCAN, K_H_DONE, K_NBARS };
+enum { G_LD, G_Z, G_NBARS };
 
-template <int D, int NB>
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_dk_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
-                  const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmW,
-                  const __grid_constant__ CUtensorMap tmDW, const BwdParams p) {
-  using L = DkL<D, NB>;
-  constexpr int C = L::C;
+template <int D>
+__global__ void __launch_bounds__(kSmallThreads, 2)
+    bwd_g_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmW,
+                 const __grid_constant__ CUtensorMap tmV, const BwdParams p) {
+  using L = GL<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sb0 = smem_u32(smem);
-  const uint32_t sK = sb0 + L::OFF_K, sG = sb0 + L::OFF_G, sW0 = sb0 + L::OFF_W0,
-                 sDW = sb0 + L::OFF_DW, sQ = sb0 + L::OFF_Q, sDO = sb0 + L::OFF_DO;
-  float* f = reinterpret_cast<float*>(smem + L::OFF_F);
-  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
-        *f_cT16 = f + 1280, *f_part = f + 1536;  // f_part[2][128]
+  const uint32_t sK = sb0 + L::OFF_K, sW0 = sb0 + L::OFF_W0, sV = sb0 + L::OFF_V;
   Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int rb = blockIdx.x % NB;
-  const int c = (blockIdx.x / NB) % p.NC;
-  const int bh = blockIdx.x / (NB * p.NC);
-  const int NC = p.NC;
   const bool mse = p.loss == 0;
-  const int counts[K_NBARS] = {1, 1, kEpiWarps, 1, kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1,
-                               kEpiWarps, 1, 1};
+  const int row0 = blockIdx.x * 128;                  // first token row in [B*H*T]
+  const int bh = row0 / p.T, c = (row0 % p.T) / (p.T / p.NC);
+  const int wrow = (bh * p.NC + c) * D;
+  const int counts[G_NBARS] = {1, 1};
   uint32_t tmem;
-  setup(bars, counts, K_NBARS, tmem);
+  setup(bars, counts, G_NBARS, tmem, 128);
   Abort ab{&bars->abort_flag, p.err};
-  const int tokc = bh * p.T + c * C;                 // first token of the chunk
-  const int wrow = (bh * NC + c) * D;                // first row of this chunk's state
-
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(BAR(K_LD_FULL), 2 * L::BLK + 2 * L::WSZ);
+      mbar_arrive_expect_tx(BAR(G_LD), mse ? 2 * L::BLK + L::WSZ : L::BLK);
 #pragma unroll
       for (int kp = 0; kp < L::KP; ++kp) {
-        tma_load_2d(sK + kp * PANEL128, &tmK, BAR(K_LD_FULL), 64 * kp, tokc + 128 * rb);
-        tma_load_2d(sG + kp * PANEL128, &tmV, BAR(K_LD_FULL), 64 * kp, tokc + 128 * rb);
-        tma_load_2d(sW0 + kp * D * 128, &tmW, BAR(K_LD_FULL), 64 * kp, wrow);
-        tma_load_2d(sDW + kp * D * 128, &tmDW, BAR(K_LD_FULL), 64 * kp, wrow);
-      }
-      int k = 0;
-      for (int sb = rb; sb < NB; ++sb, ++k) {
-        if (k > 0 && !mbar_wait(BAR(K_QDO_FREE), (k - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(BAR(K_QDO_FULL), 2 * L::BLK);
-#pragma unroll
-        for (int kp = 0; kp < L::KP; ++kp) {
-          tma_load_2d(sQ + kp * PANEL128, &tmQ, BAR(K_QDO_FULL), 64 * kp, tokc + 128 * sb);
-          tma_load_2d(sDO + kp * PANEL128, &tmDO, BAR(K_QDO_FULL), 64 * kp, tokc + 128 * sb);
+        tma_load_2d(sV + kp * PANEL128, &tmV, BAR(G_LD), 64 * kp, row0);
+        if (mse) {
+          tma_load_2d(sK + kp * PANEL128, &tmK, BAR(G_LD), 64 * kp, row0);
+          tma_load_2d(sW0 + kp * D * 128, &tmW, BAR(G_LD), 64 * kp, wrow);
         }
-      }
-      // dV (dZ = -dV) goes into the dW slot once the only MMA that reads dW (H) is done
-      if (mse && mbar_wait(BAR(K_H_DONE), 0, ab)) {
-        mbar_arrive_expect_tx(BAR(K_DV_FULL), L::BLK);
-#pragma unroll
-        for (int kp = 0; kp < L::KP; ++kp)
-          tma_load_2d(sDW + kp * PANEL128, &tmDV, BAR(K_DV_FULL), 64 * kp, tokc + 128 * rb);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && mse && mbar_wait(BAR(G_LD), 0, ab)) {
+      tc_fence_after();
       const uint32_t idZ = idesc_bf16(128, D, 0, 1);
-      const uint32_t idKK = idesc_bf16(128, D, 0, 0);
-      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
-      const uint32_t idQ = idesc_bf16(128, D, 0, 1);
-      const uint32_t idZW = idesc_bf16(128, D, 0, 0, 1);
-      do {
-        if (!mbar_wait(BAR(K_LD_FULL), 0, ab)) break;
-        tc_fence_after();
-        if (mse) {
-          // Z = K_rb W0
 #pragma unroll
-          for (int j = 0; j < D / 16; ++j)
-            mma_bf16_ss(tmem + L::T_ZDP, sdesc_sw128(sK + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                        sdesc_sw128(sW0 + j * 2048, D * 128, 1024), idZ, j > 0);
-          mma_commit(BAR(K_Z_FULL));
-        }
-        if (!mbar_wait(BAR(K_G_READY), 0, ab)) break;
-        tc_fence_after();
-        // H = G dW^T into the dK accumulator
-#pragma unroll
-        for (int j = 0; j < D / 16; ++j)
-          mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                      sdesc_sw128(sDW + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idKK, j > 0);
-        mma_commit(BAR(K_H_FULL));
-        mma_commit(BAR(K_H_DONE));
-        bool ok = true;
-        int k = 0;
-        for (int sb = rb; sb < NB; ++sb, ++k) {
-          if (!mbar_wait(BAR(K_QDO_FULL), k & 1, ab)) { ok = false; break; }
-          tc_fence_after();
-          // dS^T accumulator = G dO_sb^T ; P^T = K_rb Q_sb^T
-#pragma unroll
-          for (int j = 0; j < D / 16; ++j)
-            mma_bf16_ss(tmem + L::T_DS, sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                        sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
-#pragma unroll
-          for (int j = 0; j < D / 16; ++j)
-            mma_bf16_ss(tmem + L::T_P, sdesc_sw128(sK + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                        sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
-          mma_commit(BAR(K_SP_FULL));
-          if (!mbar_wait(BAR(K_DP_READY), k & 1, ab)) { ok = false; break; }
-          if (k == 0 && !mbar_wait(BAR(K_H_SCALED), 0, ab)) { ok = false; break; }
-          tc_fence_after();
-          // dK += dP^T Q_sb   (A = dP^T, bf16 in TMEM)
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            mma_bf16_ts(tmem + L::T_DK, tmem + L::T_ZDP + 8 * j,
-                        sdesc_sw128(sQ + j * 2048, PANEL128, 1024), idQ, 1);
-          mma_commit(BAR(K_QDO_FREE));
-          mma_commit(BAR(K_DP_FREE));
-        }
-        if (!ok) break;
-        if (mse) {
-          // dK += dZ W0^T with dZ = -dV
-          if (!mbar_wait(BAR(K_DV_FULL), 0, ab)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int j = 0; j < D / 16; ++j)
-            mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sDW + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                        sdesc_sw128(sW0 + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idZW, 1);
-        }
-        mma_commit(BAR(K_DK_FULL));
-      } while (0);
+      for (int j = 0; j < D / 16; ++j)
+        mma_bf16_ss(tmem, sdesc_sw128(sK + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                    sdesc_sw128(sW0 + j * 2048, D * 128, 1024), idZ, j > 0);
+      mma_commit(BAR(G_Z));
     }
   } else {
-    const int ew = warp - 2, g = ew / 4, q = warp & 3, lrow = q * 32 + lane;
+    const int q = warp & 3, lrow = q * 32 + lane;
     const uint32_t loff = (uint32_t)(q * 32) << 16;
-    const int r = 128 * rb + lrow;  // chunk-local key index
-    do {
-      if (ew == 0) {
-        chunk_scan_warp<C>(p.beta + tokc, p.gamma ? p.gamma + tokc : nullptr, p.lr_bias, f_eta,
-                           f_L, f_gam, f_eLC, f_cF16, f_cT16);
-        if (lane == 0) mbar_arrive(BAR(K_SCAN));
-      }
-      if (!mbar_wait(BAR(K_SCAN), 0, ab)) break;
-      if (!mbar_wait(BAR(K_LD_FULL), 0, ab)) break;
-      if (mse && !mbar_wait(BAR(K_Z_FULL), 0, ab)) break;
+    if (mbar_wait(BAR(G_LD), 0, ab) && (!mse || mbar_wait(BAR(G_Z), 0, ab))) {
       __syncwarp();
       tc_fence_after();
-      const float Lr = f_L[r], er = f_eta[r], eLCr = f_eLC[r];
-      // G = Z - V (MSE) or -V (IP), in place over V
-      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
         float v[32], z[32];
-        ld_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+        ld_row32(sV + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
         if (mse) {
-          tmem_ld32(tmem + loff + L::T_ZDP + 32 * cc, z);
+          tmem_ld32(tmem + loff + 32 * cc, z);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = z[j] - v[j];
@@ -561,103 +475,80 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = -v[j];
         }
-        st_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+        st_global_bf16x32(p.G + ((size_t)row0 + lrow) * D + 32 * cc, v);
       }
-      epi_arrive(BAR(K_G_READY));
-      // H = G dW^T: deta partial -exp(L_C - L_r) K_r . H_r and the dK term -u_r H_r
-      if (!mbar_wait(BAR(K_H_FULL), 0, ab)) break;
-      __syncwarp();
-      tc_fence_after();
-      float dot = 0.f;
-      const float ur = er * eLCr;
-      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
-        float h[32], kr[32];
-        tmem_ld32(tmem + loff + L::T_DK + 32 * cc, h);
-        ld_row32(sK + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), kr);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          dot += h[j] * kr[j];
-          h[j] *= -ur;
-        }
-        tmem_st32(tmem + loff + L::T_DK + 32 * cc, h);
-      }
-      tmem_wait_st();
-      epi_arrive(BAR(K_H_SCALED));
-      float deta = -eLCr * dot;
-      // score blocks: dP^T = dS^T M^T into TMEM (bf16), deta += sum_s dS^T P^T exp(L_s - L_r)
-      bool ok = true;
-      int k = 0;
-      for (int sb = rb; sb < NB; ++sb, ++k) {
-        if (!mbar_wait(BAR(K_SP_FULL), k & 1, ab)) { ok = false; break; }
-        if (k > 0 && !mbar_wait(BAR(K_DP_FREE), (k - 1) & 1, ab)) { ok = false; break; }
-        __syncwarp();
-        tc_fence_after();
-        const int s0 = 128 * sb + 64 * g;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float ds[32], pp[32], wt[32];
-          tmem_ld32(tmem + loff + L::T_DS + 64 * g + 32 * half, ds);
-          tmem_ld32(tmem + loff + L::T_P + 64 * g + 32 * half, pp);
-          causal_weights_k(f_L, f_cT16, r, Lr, s0 + 32 * half, wt);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float dsT = -ds[j];
-            deta += dsT * pp[j] * wt[j];
-            ds[j] = dsT * er * wt[j];  // dP^T
-          }
-          uint32_t w[16];
-          pack32(ds, w);
-          tmem_st16u(tmem + loff + L::T_ZDP + 32 * g + 16 * half, w);
-        }
-        tmem_wait_st();
-        epi_arrive(BAR(K_DP_READY));
-      }
-      if (!ok) break;
-      // dK out; dbeta from both warpgroups' partial sums
-      if (!mbar_wait(BAR(K_DK_FULL), 0, ab)) break;
-      __syncwarp();
-      tc_fence_after();
-      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
-        float v[32];
-        tmem_ld32(tmem + loff + L::T_DK + 32 * cc, v);
-        tmem_wait_ld();
-        st_global_bf16x32(p.dK + ((size_t)tokc + r) * D + 32 * cc, v);
-      }
-      f_part[g * 128 + lrow] = deta;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(K_PART));
-      if (!mbar_wait(BAR(K_PART), 0, ab)) break;
-      if (g == 0) {
-        const float d = f_part[lrow] + f_part[128 + lrow];
-        p.dbeta[(size_t)tokc + r] = d * er * (1.f - 0.5f * er);
-      }
-    } while (0);
+    }
   }
-  teardown(bars, tmem);
+  teardown(bars, tmem, 128);
 }
 
-// ================================================================================== dQ
+// In-place packing of one 128-key (or 128-query) score block held in TMEM by the thread's row:
+// the fp32 columns [64 pair, 64 pair + 64) become bf16 pairs at [32 pair, 32 pair + 32), read
+// before written by the same thread, so the packed block is contiguous for the MMA that reads
+// it as its A operand. kind: 0 every column masked, 1 none, 2 this warp's diagonal.
+template <typename F>
+__device__ __forceinline__ void pack_block_in_place(uint32_t tb, int q, bool diag, F&& weights) {
+#pragma unroll
+  for (int pair = 0; pair < 2; ++pair) {
+    int kind[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int idx = 2 * pair + h;
+      kind[h] = diag ? (idx == q ? 2 : weights.full(idx, q) ? 1 : 0) : 1;
+    }
+    float pv[2][32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (kind[h] != 0) tmem_ld32(tb + 64 * pair + 32 * h, pv[h]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t pk[16];
+      if (kind[h] == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+      } else {
+        weights(pv[h], 2 * pair + h, kind[h] == 2, pk);
+      }
+      tmem_st16u(tb + 32 * pair + 16 * h, pk);
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------------- dQ
+// dQ_s = Gamma_s dO_s W0^T + sum_{r <= s} dP_sr K_r with dP = -(dO G^T) * M, one CTA per
+// (batch, head, chunk, 128-query block); key blocks stream through one G and one K slot.
 template <int D, int NB>
 struct DqL {
   static constexpr int C = 128 * NB, KP = D / 64;
   static constexpr uint32_t BLK = KP * PANEL128;
   static constexpr uint32_t WSZ = KP * D * 128;
-  // per key block rb: K_rb at OFF_K + 2 rb BLK, V_rb (then G_rb) at OFF_K + (2 rb + 1) BLK
-  static constexpr uint32_t OFF_DO = 0, OFF_W0 = BLK, OFF_K = BLK + WSZ,
-                            OFF_F = BLK + WSZ + 2 * NB * BLK;
+  static constexpr uint32_t SLOT = BLK > WSZ ? BLK : WSZ;  // W0, then G blocks
+  static constexpr uint32_t OFF_DO = 0, OFF_GW = BLK, OFF_K = BLK + SLOT,
+                            OFF_F = 2 * BLK + SLOT;
   static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
-  static constexpr uint32_t T_DQ = 0, T_Z = 128, T_DS = 256, T_DP = 384;
+  static constexpr uint32_t T_DQ = 0, T_DS = D;
 };
-enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_KV_FULL, Q_KV_FULL1, Q_Z_FULL, Q_G_READY, Q_DS_FULL,
-       Q_DP_READY, Q_DP_FREE, Q_DQ_FULL, Q_SCAN, Q_NBARS };
+enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_G_FULL, Q_K_FULL, Q_DS_FULL, Q_DP_READY, Q_DP_DONE,
+       Q_DQ_FULL, Q_SCAN, Q_NBARS };
+
+// -dP for query s against 32 keys of key half idx: mask/decay weights of the forward's S.
+struct QWeights {
+  const float *L, *cF16;
+  int s, rbase;
+  float Ls;
+  __device__ bool full(int idx, int q) const { return idx < q; }
+  __device__ void operator()(const float (&pv)[32], int idx, bool mask, uint32_t (&pk)[16]) const {
+    if (mask) score_weights32<true>(pv, L, cF16, s, Ls, rbase + 32 * idx, pk);
+    else score_weights32<false>(pv, L, cF16, s, Ls, rbase + 32 * idx, pk);
+  }
+};
 
 template <int D, int NB>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kSmallThreads, 2)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmW,
-                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmG,
                   const BwdParams p) {
   using L = DqL<D, NB>;
   constexpr int C = L::C;
@@ -665,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sb0 = smem_u32(smem);
-  const uint32_t sDO = sb0 + L::OFF_DO, sW0 = sb0 + L::OFF_W0, sKV = sb0 + L::OFF_K;
+  const uint32_t sDO = sb0 + L::OFF_DO, sGW = sb0 + L::OFF_GW, sK = sb0 + L::OFF_K;
   float* f = reinterpret_cast<float*>(smem + L::OFF_F);
   float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
         *f_cT16 = f + 1280;
@@ -674,31 +565,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int sb = blockIdx.x % NB;
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
-  const int NC = p.NC;
-  const bool mse = p.loss == 0;
-  const int counts[Q_NBARS] = {1, 1, kEpiWarps, 1, 1, 1, kEpiWarps, 1, kEpiWarps, 1, 1, 1};
+  const int counts[Q_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1};
   uint32_t tmem;
-  setup(bars, counts, Q_NBARS, tmem);
+  setup(bars, counts, Q_NBARS, tmem, 256);
   Abort ab{&bars->abort_flag, p.err};
   const int tokc = bh * p.T + c * C;
-  const int wrow = (bh * NC + c) * D;
+  const int wrow = (bh * p.NC + c) * D;
 
   if (warp == 0) {
     if (lane == 0) {
       mbar_arrive_expect_tx(BAR(Q_LD0), L::BLK + L::WSZ);
+      mbar_arrive_expect_tx(BAR(Q_K_FULL), L::BLK);
 #pragma unroll
       for (int kp = 0; kp < L::KP; ++kp) {
         tma_load_2d(sDO + kp * PANEL128, &tmDO, BAR(Q_LD0), 64 * kp, tokc + 128 * sb);
-        tma_load_2d(sW0 + kp * D * 128, &tmW, BAR(Q_LD0), 64 * kp, wrow);
+        tma_load_2d(sGW + kp * D * 128, &tmW, BAR(Q_LD0), 64 * kp, wrow);
+        tma_load_2d(sK + kp * PANEL128, &tmK, BAR(Q_K_FULL), 64 * kp, tokc);
       }
       for (int rb = 0; rb <= sb; ++rb) {
-        const uint32_t bar = BAR(Q_KV_FULL + rb);
-        const uint32_t sK = sKV + 2 * rb * L::BLK, sG = sK + L::BLK;
-        mbar_arrive_expect_tx(bar, 2 * L::BLK);
+        // G_rb replaces W0 (read by dO W0^T) or G_{rb-1} (read by its dS MMA)
+        if (!mbar_wait(rb == 0 ? BAR(Q_DQ0) : BAR(Q_DS_FULL), rb == 0 ? 0 : (rb - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(BAR(Q_G_FULL), L::BLK);
 #pragma unroll
-        for (int kp = 0; kp < L::KP; ++kp) {
-          tma_load_2d(sK + kp * PANEL128, &tmK, bar, 64 * kp, tokc + 128 * rb);
-          tma_load_2d(sG + kp * PANEL128, &tmV, bar, 64 * kp, tokc + 128 * rb);
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sGW + kp * PANEL128, &tmG, BAR(Q_G_FULL), 64 * kp, tokc + 128 * rb);
+        if (rb > 0) {
+          // K_rb replaces K_{rb-1} once dQ += dP K_{rb-1} has read it
+          if (!mbar_wait(BAR(Q_DP_DONE), (rb - 1) & 1, ab)) break;
+          mbar_arrive_expect_tx(BAR(Q_K_FULL), L::BLK);
+#pragma unroll
+          for (int kp = 0; kp < L::KP; ++kp)
+            tma_load_2d(sK + kp * PANEL128, &tmK, BAR(Q_K_FULL), 64 * kp, tokc + 128 * rb);
         }
       }
     }
@@ -714,44 +611,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < D / 16; ++j)
           mma_bf16_ss(tmem + L::T_DQ, sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                      sdesc_sw128(sW0 + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idKK, j > 0);
+                      sdesc_sw128(sGW + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idKK, j > 0);
         mma_commit(BAR(Q_DQ0));
         bool ok = true;
         for (int rb = 0; rb <= sb; ++rb) {
-          const uint32_t sK = sKV + 2 * rb * L::BLK, sG = sK + L::BLK;
-          if (!mbar_wait(BAR(Q_KV_FULL + rb), 0, ab)) { ok = false; break; }
+          if (!mbar_wait(BAR(Q_G_FULL), rb & 1, ab)) { ok = false; break; }
+          // the score buffer holds dP_{rb-1} until dQ += dP K_{rb-1} is done
+          if (rb > 0 && !mbar_wait(BAR(Q_DP_DONE), (rb - 1) & 1, ab)) { ok = false; break; }
           tc_fence_after();
-          if (mse) {
-#pragma unroll
-            for (int j = 0; j < D / 16; ++j)
-              mma_bf16_ss(tmem + L::T_Z, sdesc_sw128(sK + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                          sdesc_sw128(sW0 + j * 2048, D * 128, 1024), idZ, j > 0);
-            mma_commit(BAR(Q_Z_FULL));
-          }
-          if (!mbar_wait(BAR(Q_G_READY), rb & 1, ab)) { ok = false; break; }
-          tc_fence_after();
-          // dS accumulator = dO_sb G_rb^T
+          // score accumulator = dO_sb G_rb^T
 #pragma unroll
           for (int j = 0; j < D / 16; ++j)
             mma_bf16_ss(tmem + L::T_DS, sdesc_sw128(sDO + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                        sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
+                        sdesc_sw128(sGW + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
           mma_commit(BAR(Q_DS_FULL));
           if (!mbar_wait(BAR(Q_DP_READY), rb & 1, ab)) { ok = false; break; }
+          if (!mbar_wait(BAR(Q_K_FULL), rb & 1, ab)) { ok = false; break; }
           if (rb == 0 && !mbar_wait(BAR(Q_DQ_SCALED), 0, ab)) { ok = false; break; }
           tc_fence_after();
           // dQ += dP K_rb   (A = dP, bf16 in TMEM)
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            mma_bf16_ts(tmem + L::T_DQ, tmem + L::T_DP + 8 * j,
+            mma_bf16_ts(tmem + L::T_DQ, tmem + L::T_DS + 8 * j,
                         sdesc_sw128(sK + j * 2048, PANEL128, 1024), idZ, 1);
-          mma_commit(BAR(Q_DP_FREE));
+          mma_commit(BAR(Q_DP_DONE));
         }
         if (!ok) break;
         mma_commit(BAR(Q_DQ_FULL));
       } while (0);
     }
   } else {
-    const int ew = warp - 2, g = ew / 4, q = warp & 3, lrow = q * 32 + lane;
+    const int ew = warp - 2, q = warp & 3, lrow = q * 32 + lane;
     const uint32_t loff = (uint32_t)(q * 32) << 16;
     const int s = 128 * sb + lrow;  // chunk-local query index
     do {
@@ -761,16 +651,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(BAR(Q_SCAN));
       }
       if (!mbar_wait(BAR(Q_SCAN), 0, ab)) break;
-      const float Ls = f_L[s];
       // dQ *= Gamma_s
       if (!mbar_wait(BAR(Q_DQ0), 0, ab)) break;
       __syncwarp();
       tc_fence_after();
-      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+      const float gs = f_gam[s];
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
         float v[32];
         tmem_ld32(tmem + loff + L::T_DQ + 32 * cc, v);
         tmem_wait_ld();
-        const float gs = f_gam[s];
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] *= gs;
         tmem_st32(tmem + loff + L::T_DQ + 32 * cc, v);
@@ -779,45 +669,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_arrive(BAR(Q_DQ_SCALED));
       bool ok = true;
       for (int rb = 0; rb <= sb; ++rb) {
-        const uint32_t sG = sKV + (2 * rb + 1) * L::BLK;
-        // G_rb = K_rb W0 - V_rb (MSE) or -V_rb (IP), rows of the key block
-        if (!mbar_wait(BAR(Q_KV_FULL + rb), 0, ab)) { ok = false; break; }
-        if (mse && !mbar_wait(BAR(Q_Z_FULL), rb & 1, ab)) { ok = false; break; }
-        __syncwarp();
-        tc_fence_after();
-        for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
-          float v[32], z[32];
-          ld_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
-          if (mse) {
-            tmem_ld32(tmem + loff + L::T_Z + 32 * cc, z);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = z[j] - v[j];
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = -v[j];
-          }
-          st_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
-        }
-        epi_arrive(BAR(Q_G_READY));
         // dP_sr = -acc * eta_r exp(L_s - L_r), r <= s
         if (!mbar_wait(BAR(Q_DS_FULL), rb & 1, ab)) { ok = false; break; }
-        if (rb > 0 && !mbar_wait(BAR(Q_DP_FREE), (rb - 1) & 1, ab)) { ok = false; break; }
         __syncwarp();
         tc_fence_after();
-        const int r0 = 128 * rb + 64 * g;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float v[32], m[32];
-          tmem_ld32(tmem + loff + L::T_DS + 64 * g + 32 * half, v);
-          causal_weights_q(f_L, f_cF16, s, Ls, r0 + 32 * half, m);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = -v[j] * m[j];
-          uint32_t w[16];
-          pack32(v, w);
-          tmem_st16u(tmem + loff + L::T_DP + 32 * g + 16 * half, w);
-        }
+        QWeights w{f_L, f_cF16, s, 128 * rb, f_L[s]};
+        pack_block_in_place(tmem + loff + L::T_DS, q, rb == sb, w);
         tmem_wait_st();
         epi_arrive(BAR(Q_DP_READY));
       }
@@ -825,7 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(BAR(Q_DQ_FULL), 0, ab)) break;
       __syncwarp();
       tc_fence_after();
-      for (int cc = g * (D / 64); cc < (g + 1) * (D / 64); ++cc) {
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
         float v[32];
         tmem_ld32(tmem + loff + L::T_DQ + 32 * cc, v);
         tmem_wait_ld();
@@ -833,7 +691,226 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } while (0);
   }
-  teardown(bars, tmem);
+  teardown(bars, tmem, 256);
+}
+
+// ----------------------------------------------------------------------------------- dK
+// dK_r = -u_r (G_r dW^T) + sum_{s >= r} dP^T_rs Q_s + dZ_r W0^T (dZ = -dV for MSE), and
+// dbeta_r = deta_r eta_r (1 - eta_r / 2) with deta_r = (G_r . dG_r) / eta_r = -(G_r . dV_r) / eta_r:
+// the score term sum_s dS_sr P_sr exp(L_s - L_r) equals -(G_r . X_r) / eta_r and the state term
+// -exp(L_C - L_r) K_r . (G_r dW^T) equals -(u_r / eta_r) G_r . Y_r, so the two together are
+// G_r . (-X_r - u_r Y_r) / eta_r. One CTA per (batch, head, chunk, 128-key block).
+template <int D, int NB>
+struct DkL {
+  static constexpr int C = 128 * NB, KP = D / 64;
+  static constexpr uint32_t BLK = KP * PANEL128;
+  static constexpr uint32_t WSZ = KP * D * 128;
+  static constexpr uint32_t SLOT = BLK > WSZ ? BLK : WSZ;  // dW, then Q blocks, then W0
+  static constexpr uint32_t OFF_G = 0, OFF_A = BLK, OFF_B = BLK + SLOT, OFF_F = 2 * BLK + SLOT;
+  static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
+  static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
+  static constexpr uint32_t T_DK = 0, T_DS = D;
+};
+enum { K_LD0, K_H, K_H_SCALED, K_DO_FULL, K_Q_FULL, K_DS_FULL, K_DP_READY, K_DK_STEP,
+       K_DVW_FULL, K_DK_FULL, K_SCAN, K_NBARS };
+
+// -dP^T for key r against 32 queries of query half idx.
+struct KWeights {
+  const float *L, *cT16;
+  int r, sbase;
+  float Lr, er;
+  __device__ bool full(int idx, int q) const { return idx > q; }
+  __device__ void operator()(const float (&pv)[32], int idx, bool mask, uint32_t (&pk)[16]) const {
+    if (mask) score_weights32_k<true>(pv, L, cT16, r, Lr, er, sbase + 32 * idx, pk);
+    else score_weights32_k<false>(pv, L, cT16, r, Lr, er, sbase + 32 * idx, pk);
+  }
+};
+
+template <int D, int NB>
+__global__ void __launch_bounds__(kSmallThreads, 2)
+    bwd_dk_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmDW,
+                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmW,
+                  const BwdParams p) {
+  using L = DkL<D, NB>;
+  constexpr int C = L::C;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb0 = smem_u32(smem);
+  const uint32_t sG = sb0 + L::OFF_G, sA = sb0 + L::OFF_A, sB = sb0 + L::OFF_B;
+  float* f = reinterpret_cast<float*>(smem + L::OFF_F);
+  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
+        *f_cT16 = f + 1280;
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int rb = blockIdx.x % NB;
+  const int c = (blockIdx.x / NB) % p.NC;
+  const int bh = blockIdx.x / (NB * p.NC);
+  const bool mse = p.loss == 0;
+  const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1};
+  uint32_t tmem;
+  setup(bars, counts, K_NBARS, tmem, 256);
+  Abort ab{&bars->abort_flag, p.err};
+  const int tokc = bh * p.T + c * C;
+  const int wrow = (bh * p.NC + c) * D;
+  const int nq = NB - rb;  // query blocks at or after this key block
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(BAR(K_LD0), L::BLK + L::WSZ);
+#pragma unroll
+      for (int kp = 0; kp < L::KP; ++kp) {
+        tma_load_2d(sG + kp * PANEL128, &tmG, BAR(K_LD0), 64 * kp, tokc + 128 * rb);
+        tma_load_2d(sA + kp * D * 128, &tmDW, BAR(K_LD0), 64 * kp, wrow);
+      }
+      bool ok = true;
+      for (int k = 0; k < nq && ok; ++k) {
+        const int sb = rb + k;
+        // dO_sb into slot B after the previous score MMA
+        if (k > 0 && !mbar_wait(BAR(K_DS_FULL), (k - 1) & 1, ab)) { ok = false; break; }
+        mbar_arrive_expect_tx(BAR(K_DO_FULL), L::BLK);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sB + kp * PANEL128, &tmDO, BAR(K_DO_FULL), 64 * kp, tokc + 128 * sb);
+        // Q_sb into slot A after G dW^T (first) or the previous dK step
+        if (!mbar_wait(k == 0 ? BAR(K_H) : BAR(K_DK_STEP), k == 0 ? 0 : (k - 1) & 1, ab)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(BAR(K_Q_FULL), L::BLK);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sA + kp * PANEL128, &tmQ, BAR(K_Q_FULL), 64 * kp, tokc + 128 * sb);
+      }
+      // dV into slot B and (MSE) W0 into slot A after the last score MMA and dK step
+      if (ok && mbar_wait(BAR(K_DS_FULL), (nq - 1) & 1, ab) &&
+          mbar_wait(BAR(K_DK_STEP), (nq - 1) & 1, ab)) {
+        mbar_arrive_expect_tx(BAR(K_DVW_FULL), L::BLK + (mse ? L::WSZ : 0));
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp) {
+          tma_load_2d(sB + kp * PANEL128, &tmDV, BAR(K_DVW_FULL), 64 * kp, tokc + 128 * rb);
+          if (mse) tma_load_2d(sA + kp * D * 128, &tmW, BAR(K_DVW_FULL), 64 * kp, wrow);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idKK = idesc_bf16(128, D, 0, 0);
+      const uint32_t idS = idesc_bf16(128, 128, 0, 0);
+      const uint32_t idQ = idesc_bf16(128, D, 0, 1);
+      const uint32_t idZW = idesc_bf16(128, D, 0, 0, 1);
+      do {
+        if (!mbar_wait(BAR(K_LD0), 0, ab)) break;
+        tc_fence_after();
+        // H = G dW^T into the dK accumulator (scaled by -u_r in the epilogue)
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j)
+          mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                      sdesc_sw128(sA + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idKK, j > 0);
+        mma_commit(BAR(K_H));
+        bool ok = true;
+        for (int k = 0; k < nq; ++k) {
+          if (!mbar_wait(BAR(K_DO_FULL), k & 1, ab)) { ok = false; break; }
+          if (k > 0 && !mbar_wait(BAR(K_DK_STEP), (k - 1) & 1, ab)) { ok = false; break; }
+          tc_fence_after();
+          // score accumulator = G dO_sb^T
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_DS, sdesc_sw128(sG + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sB + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024), idS, j > 0);
+          mma_commit(BAR(K_DS_FULL));
+          if (!mbar_wait(BAR(K_DP_READY), k & 1, ab)) { ok = false; break; }
+          if (!mbar_wait(BAR(K_Q_FULL), k & 1, ab)) { ok = false; break; }
+          if (k == 0 && !mbar_wait(BAR(K_H_SCALED), 0, ab)) { ok = false; break; }
+          tc_fence_after();
+          // dK += dP^T Q_sb   (A = dP^T, bf16 in TMEM)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            mma_bf16_ts(tmem + L::T_DK, tmem + L::T_DS + 8 * j,
+                        sdesc_sw128(sA + j * 2048, PANEL128, 1024), idQ, 1);
+          mma_commit(BAR(K_DK_STEP));
+        }
+        if (!ok) break;
+        if (mse) {
+          // dK += dZ W0^T with dZ = -dV (negated A)
+          if (!mbar_wait(BAR(K_DVW_FULL), 0, ab)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::T_DK, sdesc_sw128(sB + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sA + (j / 4) * D * 128 + (j % 4) * 32, 16, 1024), idZW, 1);
+        }
+        mma_commit(BAR(K_DK_FULL));
+      } while (0);
+    }
+  } else {
+    const int ew = warp - 2, q = warp & 3, lrow = q * 32 + lane;
+    const uint32_t loff = (uint32_t)(q * 32) << 16;
+    const int r = 128 * rb + lrow;  // chunk-local key index
+    do {
+      if (ew == 0) {
+        chunk_scan_warp<C>(p.beta + tokc, p.gamma ? p.gamma + tokc : nullptr, p.lr_bias, f_eta,
+                           f_L, f_gam, f_eLC, f_cF16, f_cT16);
+        if (lane == 0) mbar_arrive(BAR(K_SCAN));
+      }
+      if (!mbar_wait(BAR(K_SCAN), 0, ab)) break;
+      const float Lr = f_L[r], er = f_eta[r], nur = -er * f_eLC[r];
+      // dK accumulator = -u_r H_r
+      if (!mbar_wait(BAR(K_H), 0, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float h[32];
+        tmem_ld32(tmem + loff + L::T_DK + 32 * cc, h);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) h[j] *= nur;
+        tmem_st32(tmem + loff + L::T_DK + 32 * cc, h);
+      }
+      tmem_wait_st();
+      epi_arrive(BAR(K_H_SCALED));
+      bool ok = true;
+      for (int k = 0; k < nq; ++k) {
+        const int sb = rb + k;
+        // dP^T_rs = -acc * eta_r exp(L_s - L_r), s >= r
+        if (!mbar_wait(BAR(K_DS_FULL), k & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        KWeights w{f_L, f_cT16, r, 128 * sb, Lr, er};
+        pack_block_in_place(tmem + loff + L::T_DS, q, sb == rb, w);
+        tmem_wait_st();
+        epi_arrive(BAR(K_DP_READY));
+      }
+      if (!ok) break;
+      // dbeta_r = -(1 - eta_r / 2) G_r . dV_r
+      if (!mbar_wait(BAR(K_DVW_FULL), 0, ab)) break;
+      {
+        float dot = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float gv[32], dv[32];
+          ld_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), gv);
+          ld_row32(sB + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), dv);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dot += gv[j] * dv[j];
+        }
+        p.dbeta[(size_t)tokc + r] = -(1.f - 0.5f * er) * dot;
+      }
+      if (!mbar_wait(BAR(K_DK_FULL), 0, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float v[32];
+        tmem_ld32(tmem + loff + L::T_DK + 32 * cc, v);
+        tmem_wait_ld();
+        st_global_bf16x32(p.dK + ((size_t)tokc + r) * D + 32 * cc, v);
+      }
+    } while (0);
+  }
+  teardown(bars, tmem, 256);
 }
 
 #undef BAR
@@ -845,7 +922,8 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   const int BH = a.B * a.H, NC = a.T / a.C;
   const uint64_t wrows = (uint64_t)BH * NC * D;
   __nv_bfloat16* dWs = static_cast<__nv_bfloat16*>(a.ws);
-  CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tW, tDW;
+  __nv_bfloat16* G = dWs + wrows * D;
+  CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tG1, tW, tDW;
   if (!make_tmap_bf16(&tK, a.K, D, rows, D, 64, C) || !make_tmap_bf16(&tQ, a.Q, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tDO, a.dO, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tK1, a.K, D, rows, D, 64, 128) ||
@@ -853,6 +931,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       !make_tmap_bf16(&tQ1, a.Q, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tDO1, a.dO, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tDV1, a.dV, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tG1, G, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tW, a.W_chunks, D, wrows, D, 64, D) ||
       !make_tmap_bf16(&tDW, dWs, D, wrows, D, 64, D))
     return cudaErrorInvalidValue;
@@ -869,26 +948,31 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.dV = static_cast<__nv_bfloat16*>(a.dV);
   p.dW0 = a.dW0;
   p.dWs = dWs;
+  p.G = G;
   p.dQ = static_cast<__nv_bfloat16*>(a.dQ);
   p.dK = static_cast<__nv_bfloat16*>(a.dK);
   p.dbeta = a.dbeta;
   p.err = a.err;
 
+  const size_t sm_g = GL<D>::BYTES + 1024;
   const size_t sm_chain = ChainL<D, NB>::BYTES + 1024;
   const size_t sm_dk = DkL<D, NB>::BYTES + 1024;
   const size_t sm_dq = DqL<D, NB>::BYTES + 1024;
+  auto kg = bwd_g_kernel<D>;
   auto kc = bwd_chain_kernel<D, NB>;
   auto kk = bwd_dk_kernel<D, NB>;
   auto kq = bwd_dq_kernel<D, NB>;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chain)) ||
+  if ((e = cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_g)) ||
+      (e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_chain)) ||
       (e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dk)) ||
       (e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dq)))
     return e;
+  kg<<<(int)(rows / 128), kSmallThreads, sm_g, s>>>(tK1, tW, tV1, p);
   kc<<<BH * p.nslice, kThreads, sm_chain, s>>>(tK, tQ, tDO, p);
-  kq<<<BH * NC * NB, kThreads, sm_dq, s>>>(tDO1, tW, tK1, tV1, p);
-  kk<<<BH * NC * NB, kThreads, sm_dk, s>>>(tK1, tV1, tQ1, tDO1, tDV1, tW, tDW, p);
-  count_launches(3);
+  kq<<<BH * NC * NB, kSmallThreads, sm_dq, s>>>(tDO1, tW, tK1, tG1, p);
+  kk<<<BH * NC * NB, kSmallThreads, sm_dk, s>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, p);
+  count_launches(4);
   return cudaGetLastError();
 }
 
@@ -899,8 +983,9 @@ bool tc_bwd_supported(const LayerArgs& a) {
          (a.C == 128 || a.C == 256) && a.T % a.C == 0;
 }
 
+// [BH, NC, dk, dv] bf16 chunk-end adjoints, then [BH, T, dv] bf16 G
 size_t tc_bwd_workspace(const LayerArgs& a) {
-  return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2;
+  return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2 + (size_t)a.B * a.H * a.T * a.dv * 2;
 }
 
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s) {

@@ -18,9 +18,12 @@
 // score columns [64g, 64g+64) of each 128x128 score block), warp 10 computes the lr and decay
 // scans of the next chunk into the other of two buffers. Every wait is bounded.
 //
-// TMEM columns: [0,64) W (lanes = key features), [64, 64+64NB) Z blocks,
-// [64+64NB, 64+128NB) Y / Zq blocks, [64+128NB, +128) one 128x128 fp32 score block P, then
-// 64 columns of bf16 S (the A operand of S G, read by the MMA straight from TMEM).
+// TMEM columns: [0,64) W (lanes = key features; held pre-multiplied by the chunk's Gamma_C),
+// [64, 64+64NB) Z blocks, [64+64NB, 64+128NB) Y / Zq blocks, [64+128NB, +128) score buffer A.
+// With two 128-token blocks per chunk the Z columns double as score buffer B once G has been
+// formed, so the next score block's MMA runs while the epilogue masks the current one. The
+// epilogue writes S (bf16) in place over the fp32 scores it read; the S G MMA takes S straight
+// from TMEM.
 // Shared memory: K as two 128-row halves with their own full/free barriers, V double-buffered,
 // so the next chunk's loads start as soon as each buffer's last reader has finished.
 #include <cuda_bf16.h>
@@ -67,13 +70,16 @@ struct Layout {
   static constexpr uint32_t BYTES = OFF_BAR + 256;
   static constexpr uint32_t V_TX = C * 128;
   // TMEM columns
-  static constexpr uint32_t T_W = 0, T_Z = 64, T_Y = 64 + 64 * NB, T_P = 64 + 128 * NB,
-                            T_S = T_P + 128;
+  static constexpr uint32_t T_W = 0, T_Z = 64, T_Y = 64 + 64 * NB, T_PA = 64 + 128 * NB;
+  static constexpr int NP = NB * (NB + 1) / 2;  // causal score blocks per chunk
+  // score block k (order (0,0), (1,0), (1,1)) -> buffer: the middle one goes to the Z columns
+  __host__ __device__ static constexpr int buf(int k) { return (NB == 2 && k == 1) ? 1 : 0; }
+  __host__ __device__ static constexpr uint32_t tbuf(int x) { return x ? T_Z : T_PA; }
 };
 
 struct __align__(8) FwdBars {
   uint64_t k_full[2], k_free[2], v_full[2], v_free[2], q_full, q_free, z_full, g_ready, y_full,
-      y_scaled, p_full, s_ready, s_free, zq_full, y_free, w_full, w0_ready, scan_full[2],
+      y_scaled, p_full[2], s_ready[2], s_done[2], zq_full, y_free, w_full, w0_ready, scan_full[2],
       scan_free[2], bg_full[2];
   uint32_t tmem_base;
   int abort_flag;
@@ -114,9 +120,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(BAR(g_ready), kEpiWarps);
     mbar_init(BAR(y_full), 1);
     mbar_init(BAR(y_scaled), kEpiWarps);
-    mbar_init(BAR(p_full), 1);
-    mbar_init(BAR(s_ready), kEpiWarps);
-    mbar_init(BAR(s_free), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(p_full[i]), 1);
+      mbar_init(BAR(s_ready[i]), kEpiWarps);
+      mbar_init(BAR(s_done[i]), 1);
+    }
     mbar_init(BAR(zq_full), 1);
     mbar_init(BAR(y_free), kEpiWarps);
     mbar_init(BAR(w_full), 1);
@@ -196,43 +204,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idP = idesc_bf16(128, 128, 0, 0);  // K-major A and B
       const uint32_t idW = idesc_bf16(128, NV, 1, 1);   // MN-major A and B
       const uint32_t lboKt = D == 128 ? PANEL128 : 0;  // second 64-row block of K^T
-      int kq = 0, ks = 0;
+      int kq = 0;
+      int sd0 = 0, sd1 = 0;  // S G MMAs committed on s_done[x]
+      int sr0 = 0, sr1 = 0;  // s_ready[x] phases consumed
+      // a score buffer is rewritten only after the S G MMA that read it last has completed
+      auto buf_free = [&](int x) -> bool {
+        const int n = x ? sd1 : sd0;
+        return n == 0 || mbar_wait(BAR(s_done[x]), (n - 1) & 1, ab);
+      };
       for (int c = 0; c < NC; ++c) {
         const uint32_t sVc = sV + (c & 1) * C * 128;
         if (!mbar_wait(BAR(w0_ready), c & 1, ab)) break;
-        // Z_b = K_b W0
         bool ok = true;
-        for (int b = 0; b < NB; ++b) {
+        for (int b = 0; b < NB; ++b)
           if (!mbar_wait(BAR(k_full[b]), c & 1, ab)) { ok = false; break; }
-          tc_fence_after();
+        if (!ok || (NB == 2 && !buf_free(1))) break;  // Z columns = score buffer B
+        tc_fence_after();
+        // Z_b = K_b W0
+        for (int b = 0; b < NB; ++b) {
 #pragma unroll
           for (int j = 0; j < D / 16; ++j)
             mma_bf16_ss(tmem + L::T_Z + NV * b,
                         sdesc_sw128(sK + (b * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                         sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
         }
-        if (!ok) break;
         mma_commit(BAR(z_full));
         for (int h = 0; h < NB && ok; ++h) {
+          const int k0 = h * (h + 1) / 2;  // first score block of query half h
           if (!mbar_wait(BAR(q_full), kq & 1, ab)) { ok = false; break; }
           ++kq;
           if (h == 0 && c > 0 && !mbar_wait(BAR(y_free), (c - 1) & 1, ab)) { ok = false; break; }
           tc_fence_after();
+          // Y_h = Q_h W0
 #pragma unroll
           for (int j = 0; j < D / 16; ++j)
             mma_bf16_ss(tmem + L::T_Y + NV * h,
                         sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                         sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
           mma_commit(BAR(y_full));
+          // all score blocks of this query half first, so the epilogue never waits for one
           for (int b = 0; b <= h; ++b) {
+            const int x = L::buf(k0 + b);
+            if (!buf_free(x)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
             for (int j = 0; j < D / 16; ++j)
-              mma_bf16_ss(tmem + L::T_P,
+              mma_bf16_ss(tmem + L::tbuf(x),
                           sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                           sdesc_sw128(sK + (b * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
                           idP, j > 0);
-            mma_commit(BAR(p_full));
-            if (b == h) mma_commit(BAR(q_free));
+            mma_commit(BAR(p_full[x]));
             if (h == 0 && b == 0) {
               // state transition W += K^T (u * -G), W already scaled by Gamma_C
               if (!mbar_wait(BAR(g_ready), c & 1, ab)) { ok = false; break; }
@@ -243,18 +264,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             sdesc_sw128(sUG + j * 2048, 0, 1024), idW, 1);
               mma_commit(BAR(w_full));
             }
-            // release K half b after its last reader (P_{NB-1,b}; with one block also W)
+            if (b == h) mma_commit(BAR(q_free));
+            // K half b: its last reader is this block in the last query half (and W)
             if (h == NB - 1) mma_commit(BAR(k_free[b]));
-            if (!mbar_wait(BAR(s_ready), ks & 1, ab)) { ok = false; break; }
+          }
+          if (!ok) break;
+          for (int b = 0; b <= h; ++b) {
+            const int x = L::buf(k0 + b);
+            const int n = x ? sr1++ : sr0++;
+            if (!mbar_wait(BAR(s_ready[x]), n & 1, ab)) { ok = false; break; }
             if (b == 0 && !mbar_wait(BAR(y_scaled), (c * NB + h) & 1, ab)) { ok = false; break; }
-            ++ks;
             tc_fence_after();
-            // Zq_h += (-S_hb) G_b, S (bf16) read from TMEM
+            // Zq_h += (-S_hb) G_b; S (bf16) in TMEM, 32 packed columns per warpgroup
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              mma_bf16_ts(tmem + L::T_Y + NV * h, tmem + L::T_S + 8 * j,
+              mma_bf16_ts(tmem + L::T_Y + NV * h, tmem + L::tbuf(x) + 64 * (j / 4) + 8 * (j % 4),
                           sdesc_sw128(sVc + b * PANEL128 + j * 2048, 0, 1024), idZ, 1);
-            mma_commit(BAR(s_free));
+            mma_commit(BAR(s_done[x]));
+            if (x) ++sd1; else ++sd0;
           }
           if (ok) mma_commit(BAR(zq_full));
         }
@@ -284,8 +311,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool w_rows = q * 32 < D;   // this warp holds state rows
     const size_t wofs = (size_t)bh * D * D + (size_t)lrow * D + NV * slice + 32 * g;
     bool ok = true;
-    // initial state: fp32 into TMEM, bf16 operand copy, chunk-0 checkpoint
-    if (w_rows) {
+    // initial state: Gamma_C(0) W0 into TMEM, bf16 operand copy, chunk-0 checkpoint
+    if (!mbar_wait(BAR(scan_full[0]), 0, ab)) ok = false;
+    if (ok && w_rows) {
       float w[32];
       const float4* src = reinterpret_cast<const float4*>(p.W0 + wofs);
 #pragma unroll
@@ -293,18 +321,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float4 v = src[k];
         w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
       }
-      tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
-      tmem_wait_st();
       st_row32(sW0, lrow, 4 * g, w);
       if (p.W_chunks)
         st_global_bf16x32(p.W_chunks + (size_t)bh * NC * D * D + (size_t)lrow * D + NV * slice + 32 * g, w);
+      const float gam0 = f_scan[512 + C - 1];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) w[j] *= gam0;
+      tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
+      tmem_wait_st();
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(BAR(w0_ready));
 
-    int kp = 0;  // score blocks consumed
+    int puse0 = 0, puse1 = 0;  // score blocks consumed per buffer
     for (int c = 0; c < NC && ok; ++c) {
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
       // -------- this chunk's scan arrays (computed by warp 10)
@@ -314,39 +345,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* f_gam = f_eta + 512;
       const float* f_eLC = f_eta + 768;
       const float* f_cF16 = f_eta + 1024;
-      const float gamC = f_gam[C - 1];
 
-      // -------- train view: G = a(Z) act'(Z) in place over V, -u*G, state decay
+      // -------- train view: G = a(Z) act'(Z) in place over V, and -u*G
       const uint32_t sVc = sV + (c & 1) * C * 128;
       if (!mbar_wait(BAR(v_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
       if (!mbar_wait(BAR(z_full), c & 1, ab)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
-      for (int b = 0; b < NB; ++b) {
-        float z[32], v[32];
-        tmem_ld32(tmem + lane_off + L::T_Z + NV * b + 32 * g, z);
-        tmem_wait_ld();
-        const int row = 128 * b + lrow;
-        ld_row32(sVc, row, 4 * g, v);
-        const float un = -f_eta[row] * f_eLC[row];
+      {
+        // identity: both Z blocks in flight at once; SiLU needs the registers for its temporaries
+        constexpr int ZB = ACT == 0 ? NB : 1;
+        float z[ZB][32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float a = LOSS == 0 ? act_f<ACT>(z[j]) - v[j] : -v[j];
-          const float gg = a * act_d1<ACT>(z[j]);
-          v[j] = gg;
-          z[j] = un * gg;
+        for (int b0 = 0; b0 < NB; b0 += ZB) {
+#pragma unroll
+          for (int i = 0; i < ZB; ++i)
+            tmem_ld32(tmem + lane_off + L::T_Z + NV * (b0 + i) + 32 * g, z[i]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < ZB; ++i) {
+            float v[32];
+            const int row = 128 * (b0 + i) + lrow;
+            ld_row32(sVc, row, 4 * g, v);
+            const float un = -f_eta[row] * f_eLC[row];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float a = LOSS == 0 ? act_f<ACT>(z[i][j]) - v[j] : -v[j];
+              const float gg = a * act_d1<ACT>(z[i][j]);
+              v[j] = gg;
+              z[i][j] = un * gg;
+            }
+            st_row32(sVc, row, 4 * g, v);
+            st_row32(sUG, row, 4 * g, z[i]);
+          }
         }
-        st_row32(sVc, row, 4 * g, v);
-        st_row32(sUG, row, 4 * g, z);
-      }
-      if (w_rows) {
-        float w[32];
-        tmem_ld32(tmem + lane_off + L::T_W + 32 * g, w);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) w[j] *= gamC;
-        tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
-        tmem_wait_st();
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -354,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(BAR(g_ready));
 
       for (int h = 0; h < NB && ok; ++h) {
+        const int k0 = h * (h + 1) / 2;
         const int srow = 128 * h + lrow;  // chunk-local query index of this thread
         // Y_h *= Gamma_s
         if (!mbar_wait(BAR(y_full), (c * NB + h) & 1, ab)) { ok = false; break; }
@@ -375,19 +408,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         if (h == NB - 1) {
           // -------- state copy for the next chunk: after the transition MMA and after the
-          // last MMA that reads the current bf16 copy (Y of this block, complete above)
+          // last MMA that reads the current bf16 copy (Y of this block, complete above). The
+          // fp32 state goes back into TMEM already decayed by the next chunk's Gamma_C.
           if (!mbar_wait(BAR(w_full), c & 1, ab)) { ok = false; break; }
+          const bool more = c + 1 < NC;
+          if (more && !mbar_wait(BAR(scan_full[(c + 1) & 1]), ((c + 1) >> 1) & 1, ab)) {
+            ok = false;
+            break;
+          }
           __syncwarp();
           tc_fence_after();
           if (w_rows) {
             float w[32];
             tmem_ld32(tmem + lane_off + L::T_W + 32 * g, w);
             tmem_wait_ld();
-            if (c + 1 < NC) {
+            if (more) {
               st_row32(sW0, lrow, 4 * g, w);
               if (p.W_chunks)
                 st_global_bf16x32(p.W_chunks + ((size_t)bh * NC + c + 1) * D * D +
                                       (size_t)lrow * D + NV * slice + 32 * g, w);
+              const float gnext = f_scan[((c + 1) & 1) * 6 * 256 + 512 + C - 1];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) w[j] *= gnext;
+              tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
+              tmem_wait_st();
             } else if (p.W_final) {
               float4* dst = reinterpret_cast<float4*>(p.W_final + wofs);
 #pragma unroll
@@ -401,30 +445,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(BAR(w0_ready));
         }
 
+        // -------- score blocks of this query half: S = -(Q K^T) * weights, bf16 in place
         const float Ls = f_L[srow];
         for (int b = 0; b <= h; ++b) {
-          if (!mbar_wait(BAR(p_full), kp & 1, ab)) { ok = false; break; }
-          if (kp > 0 && !mbar_wait(BAR(s_free), (kp - 1) & 1, ab)) { ok = false; break; }
-          ++kp;
+          const int x = L::buf(k0 + b);
+          const int pu = x ? puse1++ : puse0++;
+          if (!mbar_wait(BAR(p_full[x]), pu & 1, ab)) { ok = false; break; }
           __syncwarp();
           tc_fence_after();
-          const int r0 = 128 * b + 64 * g;  // first key of this thread's 64 columns
+          const uint32_t tb = tmem + lane_off + L::tbuf(x) + 64 * g;
+          // this warp's 32 rows against each 32-key half: 0 all masked, 1 none, 2 the diagonal
+          int kind[2];
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
-            float sv[32], w[32];
-            tmem_ld32(tmem + lane_off + L::T_P + 64 * g + 32 * half, sv);
-            causal_weights_q(f_L, f_cF16, srow, Ls, r0 + 32 * half, w);
-            tmem_wait_ld();
+            const int idx = 2 * g + half;
+            kind[half] = b < h ? 1 : (idx < q ? 1 : (idx == q ? 2 : 0));
+          }
+          float pv[2][32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) sv[j] = -sv[j] * w[j];
+          for (int half = 0; half < 2; ++half)
+            if (kind[half] != 0) tmem_ld32(tb + 32 * half, pv[half]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int r0 = 128 * b + 64 * g + 32 * half;
             uint32_t pk[16];
-            pack32(sv, pk);
-            tmem_st16u(tmem + lane_off + L::T_S + 32 * g + 16 * half, pk);
+            if (kind[half] == 1)
+              score_weights32<false>(pv[half], f_L, f_cF16, srow, Ls, r0, pk);
+            else if (kind[half] == 2)
+              score_weights32<true>(pv[half], f_L, f_cF16, srow, Ls, r0, pk);
+            else
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pk[j] = 0u;
+            tmem_st16u(tb + 16 * half, pk);
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(s_ready));
+          if (lane == 0) mbar_arrive(BAR(s_ready[x]));
         }
         if (!ok) break;
         if (h == NB - 1) {
