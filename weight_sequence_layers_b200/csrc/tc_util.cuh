@@ -192,6 +192,73 @@ __device__ __forceinline__ void score_weights32_k(const float (&pv)[32], const f
   }
 }
 
+// Causal weights of a query row s against 32 keys of key half idx (r = rbase + 32 idx + j):
+// -S or -dP packed to bf16. A half is entirely unmasked when its keys precede the warp's rows.
+struct QWeights {
+  const float *L, *cF16;
+  int s, rbase;
+  float Ls;
+  __device__ bool full(int idx, int q) const { return idx < q; }
+  __device__ void operator()(const float (&pv)[32], int idx, bool mask, uint32_t (&pk)[16]) const {
+    if (mask) score_weights32<true>(pv, L, cF16, s, Ls, rbase + 32 * idx, pk);
+    else score_weights32<false>(pv, L, cF16, s, Ls, rbase + 32 * idx, pk);
+  }
+};
+// The same for a key row r against 32 queries of query half idx (s = sbase + 32 idx + j):
+// -S^T or -dP^T. A half is entirely unmasked when its queries follow the warp's rows.
+struct KWeights {
+  const float *L, *cT16;
+  int r, sbase;
+  float Lr, er;
+  __device__ bool full(int idx, int q) const { return idx > q; }
+  __device__ void operator()(const float (&pv)[32], int idx, bool mask, uint32_t (&pk)[16]) const {
+    if (mask) score_weights32_k<true>(pv, L, cT16, r, Lr, er, sbase + 32 * idx, pk);
+    else score_weights32_k<false>(pv, L, cT16, r, Lr, er, sbase + 32 * idx, pk);
+  }
+};
+
+// In-place packing of a 128-column fp32 score block held in TMEM by the thread's row (tb =
+// TMEM address of the row's column 0). Column pair p (64 columns [64p, 64p+64), halves
+// idx = 2p, 2p+1) becomes 32 bf16-pair columns at [OUT p, OUT p + 32); every column is read
+// before the same thread overwrites it. With OUT = 32 the packed block is contiguous (the MMA
+// reading it as A takes K-step j at 8 j); with OUT = 64 each warpgroup packs inside its own
+// 64 columns (K-step j at 64 (j / 4) + 8 (j % 4)). Halves are classified per warp (q = TMEM
+// lane quadrant = rows [32q, 32q+32) of the block): on a diagonal block a half is the warp's
+// own diagonal, entirely unmasked or entirely masked (written as zeros without a load).
+template <int OUT, typename F>
+__device__ __forceinline__ void pack_in_place(uint32_t tb, int p0, int p1, int q, bool diag,
+                                              const F& weights) {
+  for (int pair = p0; pair < p1; ++pair) {
+    int kind[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int idx = 2 * pair + h;
+      kind[h] = diag ? (idx == q ? 2 : weights.full(idx, q) ? 1 : 0) : 1;
+    }
+    float pv[2][32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+      if (kind[h] != 0) tmem_ld32(tb + 64 * pair + 32 * h, pv[h]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t pk[16];
+      if (kind[h] == 0) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[j] = 0u;
+      } else {
+        weights(pv[h], 2 * pair + h, kind[h] == 2, pk);
+      }
+      tmem_st16u(tb + OUT * pair + 16 * h, pk);
+    }
+  }
+}
+// TMEM column of K-step j (16 keys) of a block packed by pack_in_place<OUT>.
+template <int OUT>
+__host__ __device__ constexpr uint32_t packed_col(int j) {
+  return OUT == 32 ? 8 * j : 64 * (j / 4) + 8 * (j % 4);
+}
+
 // Bulk copy of `bytes` (multiple of 16, 16-byte aligned) from global to shared memory,
 // completing on `bar`.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

@@ -25,8 +25,13 @@
 //           with deta_r = (G_r . dG_r) / eta_r (see the dK kernel).
 // dq and dk rebuild the score-gradient blocks from G and dO and hold dP (bf16) in TMEM as the
 // A operand of their last contraction; they run two CTAs per SM.
+// The chain is serial over chunks and fills one SM per (head, slice); g and dq do not depend
+// on it, so they run on a second stream on the SMs the chain leaves free, and dk follows the
+// chain. The caller's stream forks into the two and joins them again at the end.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -108,20 +113,21 @@ struct ChainL {
   static constexpr uint32_t K_PANEL = C * 128;
   static constexpr uint32_t OFF_K = 0, OFF_Q = KP * K_PANEL, OFF_DO = 2 * KP * K_PANEL;
   static constexpr uint32_t OFF_DW = OFF_DO + C * 128;   // bf16 adjoint, MN-major [D][64]
-  static constexpr uint32_t OFF_S = OFF_DW + D * 128;    // S^T blocks, then dZ (C rows)
+  static constexpr uint32_t OFF_S = OFF_DW + D * 128;    // dZ (C rows x 64)
   static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;
   static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of 2 chunks
   static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t TX = 2 * KP * K_PANEL + C * 128;
-  // P^T blocks alternate between two TMEM buffers; Y reuses buffer 0 after the score loop
+  // P^T blocks alternate between two TMEM buffers, S^T packed in place (bf16) for the X MMA;
+  // Y reuses buffer 0 after the score loop
   static constexpr uint32_t T_DW = 0, T_X = 64, T_P0 = 64 + 64 * NB, T_P1 = T_P0 + 128,
                             T_Y = T_P0;
   static constexpr int NP = NB * (NB + 1) / 2;
 };
-enum { C_KV_FULL, C_KV_FREE, C_P_FULL, C_S_READY, C_S_FREE, C_X_FULL, C_W_READY, C_Y_FULL,
+enum { C_KV_FULL, C_KV_FREE, C_P_FULL, C_S_READY, C_XB0, C_X_FULL, C_W_READY, C_Y_FULL,
        C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_BG_FULL, C_BG_FULL1,
-       C_P_FULL1, C_NBARS };
+       C_P_FULL1, C_S_READY1, C_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -143,8 +149,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = blockIdx.x / p.nslice, slice = blockIdx.x % p.nslice;
   const int NC = p.NC;
   const bool mse = p.loss == 0;
+  // arrivals per barrier, in enum order
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
-                               kEpiWarps, 1, 1, 1};
+                               kEpiWarps, 1, 1, 1, kEpiWarps};
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   uint32_t tmem;
   setup(bars, counts, C_NBARS, tmem);
@@ -186,13 +193,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idX = idesc_bf16(128, NV, 0, 1);
       const uint32_t idW = idesc_bf16(128, NV, 1, 1);
       const uint32_t lboT = D == 128 ? L::K_PANEL : 0;
-      int kp = 0;
+      int sr0 = 0, sr1 = 0;  // S^T ready phases consumed per buffer
+      int xb0 = 0;           // X MMAs committed on buffer 0
       for (int it = 0; it < NC; ++it) {
         if (!mbar_wait(BAR(C_KV_FULL), it & 1, ab)) break;
         tc_fence_after();
         bool ok = true;
-        // score blocks in order k = (rb, sb), sb >= rb; P^T_k goes to TMEM buffer k & 1 and the
-        // next-but-one block is issued as soon as the epilogue has consumed this buffer
+        // score blocks in order k = (rb, sb), sb >= rb; P^T_k goes to TMEM buffer k & 1, where the
+        // epilogue packs S^T_k in place; block k+2 reuses the buffer once X has read block k
         auto issue_p = [&](int k) {
           const int rb = k < NB ? 0 : 1, sb = k < NB ? k : 1;  // NB <= 2
 #pragma unroll
@@ -209,22 +217,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (L::NP > 1) issue_p(1);
         for (int k = 0; k < L::NP; ++k) {
           const int rb = k < NB ? 0 : 1, sb = k < NB ? k : 1;
-          if (!mbar_wait(BAR(C_S_READY), kp & 1, ab)) { ok = false; break; }
-          ++kp;
+          const int x = k & 1;
+          const int n = x ? sr1++ : sr0++;
+          if (!mbar_wait(BAR(x ? C_S_READY1 : C_S_READY), n & 1, ab)) { ok = false; break; }
           tc_fence_after();
-          if (k + 2 < L::NP) issue_p(k + 2);
-          // X_rb += S^T_(rb,sb) dO_sb
+          // X_rb += S^T_(rb,sb) dO_sb, S^T (bf16) read from TMEM
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            mma_bf16_ss(tmem + L::T_X + NV * rb,
-                        sdesc_sw128(sS + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+            mma_bf16_ts(tmem + L::T_X + NV * rb,
+                        tmem + (x ? L::T_P1 : L::T_P0) + packed_col<64>(j),
                         sdesc_sw128(sDO + sb * PANEL128 + j * 2048, 0, 1024), idX,
                         (sb != rb) || (j > 0));
-          mma_commit(BAR(C_S_FREE));
+          if (x == 0) {
+            mma_commit(BAR(C_XB0));
+            ++xb0;
+          }
+          if (k + 2 < L::NP) {
+            if (!mbar_wait(BAR(C_XB0), (xb0 - 1) & 1, ab)) { ok = false; break; }
+            issue_p(k + 2);
+          }
         }
         if (!ok) break;
         mma_commit(BAR(C_X_FULL));
-        // Y_b = K_b dW
+        // Y_b = K_b dW into buffer 0, once the X MMA that read the last S^T there is done
+        if (!mbar_wait(BAR(C_XB0), (xb0 - 1) & 1, ab)) break;
         if (!mbar_wait(BAR(C_W_READY), it & 1, ab)) break;
         tc_fence_after();
         for (int b = 0; b < NB; ++b)
@@ -275,8 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       st_global_bf16x32(p.dWs + ((size_t)bh * NC + NC - 1) * D * D + wcol, w);
     }
     epi_arrive(BAR(C_W_READY));
-    int kp = 0;
-    int puse[2] = {0, 0};  // completed uses of each P buffer
+    int puse0 = 0, puse1 = 0;  // completed uses of each P buffer
     for (int it = 0; it < NC && ok; ++it) {
       const int c = NC - 1 - it;
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
@@ -289,30 +304,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(BAR(C_SCAN_FULL));
       }
       if (!mbar_wait(BAR(C_SCAN_FULL), it & 1, ab)) { ok = false; break; }
-      // ---- S^T blocks: S^T_rs = P^T_rs eta_r exp(L_s - L_r), s >= r (block k in TMEM buffer k & 1)
+      // ---- S^T blocks: S^T_rs = P^T_rs eta_r exp(L_s - L_r), s >= r, packed to bf16 in place
+      // (block k in TMEM buffer k & 1; warpgroup g packs query columns [64g, 64g+64))
       for (int k = 0; k < L::NP && ok; ++k) {
         const int rb = k < NB ? 0 : 1, sb = k < NB ? k : 1;
+        const int x = k & 1;
         const int r = 128 * rb + lrow;
-        const float Lr = f_L[r], er = f_eta[r];
-        if (!mbar_wait(BAR((k & 1) ? C_P_FULL1 : C_P_FULL), puse[k & 1] & 1, ab)) { ok = false; break; }
-        ++puse[k & 1];
-        if (kp > 0 && !mbar_wait(BAR(C_S_FREE), (kp - 1) & 1, ab)) { ok = false; break; }
-        ++kp;
+        const int pu = x ? puse1++ : puse0++;
+        if (!mbar_wait(BAR(x ? C_P_FULL1 : C_P_FULL), pu & 1, ab)) { ok = false; break; }
         __syncwarp();
         tc_fence_after();
-        const int s0 = 128 * sb + 64 * g;
-        const uint32_t tp = (k & 1) ? L::T_P1 : L::T_P0;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float v[32], w[32];
-          tmem_ld32(tmem + loff + tp + 64 * g + 32 * half, v);
-          causal_weights_k(f_L, f_cT16, r, Lr, s0 + 32 * half, w);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= er * w[j];
-          st_row32(sS + g * PANEL128, lrow, 4 * half, v);
-        }
-        epi_arrive(BAR(C_S_READY));
+        // KWeights yields -(P^T * eta_r ...); a negated eta makes it +S^T
+        const KWeights w{f_L, f_cT16, r, 128 * sb, f_L[r], -f_eta[r]};
+        pack_in_place<64>(tmem + loff + (x ? L::T_P1 : L::T_P0), g, g + 1, q, sb == rb, w);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(x ? C_S_READY1 : C_S_READY));
       }
       if (!ok) break;
       // ---- scale dO rows by Gamma_s (X, the only other reader of dO, is done) and the state
@@ -482,39 +490,6 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   teardown(bars, tmem, 128);
 }
 
-// In-place packing of one 128-key (or 128-query) score block held in TMEM by the thread's row:
-// the fp32 columns [64 pair, 64 pair + 64) become bf16 pairs at [32 pair, 32 pair + 32), read
-// before written by the same thread, so the packed block is contiguous for the MMA that reads
-// it as its A operand. kind: 0 every column masked, 1 none, 2 this warp's diagonal.
-template <typename F>
-__device__ __forceinline__ void pack_block_in_place(uint32_t tb, int q, bool diag, F&& weights) {
-#pragma unroll
-  for (int pair = 0; pair < 2; ++pair) {
-    int kind[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int idx = 2 * pair + h;
-      kind[h] = diag ? (idx == q ? 2 : weights.full(idx, q) ? 1 : 0) : 1;
-    }
-    float pv[2][32];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-      if (kind[h] != 0) tmem_ld32(tb + 64 * pair + 32 * h, pv[h]);
-    tmem_wait_ld();
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t pk[16];
-      if (kind[h] == 0) {
-#pragma unroll
-        for (int j = 0; j < 16; ++j) pk[j] = 0u;
-      } else {
-        weights(pv[h], 2 * pair + h, kind[h] == 2, pk);
-      }
-      tmem_st16u(tb + 32 * pair + 16 * h, pk);
-    }
-  }
-}
-
 // ----------------------------------------------------------------------------------- dQ
 // dQ_s = Gamma_s dO_s W0^T + sum_{r <= s} dP_sr K_r with dP = -(dO G^T) * M, one CTA per
 // (batch, head, chunk, 128-query block); key blocks stream through one G and one K slot.
@@ -532,18 +507,6 @@ struct DqL {
 };
 enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_G_FULL, Q_K_FULL, Q_DS_FULL, Q_DP_READY, Q_DP_DONE,
        Q_DQ_FULL, Q_SCAN, Q_NBARS };
-
-// -dP for query s against 32 keys of key half idx: mask/decay weights of the forward's S.
-struct QWeights {
-  const float *L, *cF16;
-  int s, rbase;
-  float Ls;
-  __device__ bool full(int idx, int q) const { return idx < q; }
-  __device__ void operator()(const float (&pv)[32], int idx, bool mask, uint32_t (&pk)[16]) const {
-    if (mask) score_weights32<true>(pv, L, cF16, s, Ls, rbase + 32 * idx, pk);
-    else score_weights32<false>(pv, L, cF16, s, Ls, rbase + 32 * idx, pk);
-  }
-};
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
@@ -632,7 +595,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
           // dQ += dP K_rb   (A = dP, bf16 in TMEM)
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            mma_bf16_ts(tmem + L::T_DQ, tmem + L::T_DS + 8 * j,
+            mma_bf16_ts(tmem + L::T_DQ, tmem + L::T_DS + packed_col<32>(j),
                         sdesc_sw128(sK + j * 2048, PANEL128, 1024), idZ, 1);
           mma_commit(BAR(Q_DP_DONE));
         }
@@ -673,8 +636,8 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         if (!mbar_wait(BAR(Q_DS_FULL), rb & 1, ab)) { ok = false; break; }
         __syncwarp();
         tc_fence_after();
-        QWeights w{f_L, f_cF16, s, 128 * rb, f_L[s]};
-        pack_block_in_place(tmem + loff + L::T_DS, q, rb == sb, w);
+        const QWeights w{f_L, f_cF16, s, 128 * rb, f_L[s]};
+        pack_in_place<32>(tmem + loff + L::T_DS, 0, 2, q, rb == sb, w);
         tmem_wait_st();
         epi_arrive(BAR(Q_DP_READY));
       }
@@ -713,18 +676,6 @@ struct DkL {
 };
 enum { K_LD0, K_H, K_H_SCALED, K_DO_FULL, K_Q_FULL, K_DS_FULL, K_DP_READY, K_DK_STEP,
        K_DVW_FULL, K_DK_FULL, K_SCAN, K_NBARS };
-
-// -dP^T for key r against 32 queries of query half idx.
-struct KWeights {
-  const float *L, *cT16;
-  int r, sbase;
-  float Lr, er;
-  __device__ bool full(int idx, int q) const { return idx > q; }
-  __device__ void operator()(const float (&pv)[32], int idx, bool mask, uint32_t (&pk)[16]) const {
-    if (mask) score_weights32_k<true>(pv, L, cT16, r, Lr, er, sbase + 32 * idx, pk);
-    else score_weights32_k<false>(pv, L, cT16, r, Lr, er, sbase + 32 * idx, pk);
-  }
-};
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
@@ -827,7 +778,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
           // dK += dP^T Q_sb   (A = dP^T, bf16 in TMEM)
 #pragma unroll
           for (int j = 0; j < 8; ++j)
-            mma_bf16_ts(tmem + L::T_DK, tmem + L::T_DS + 8 * j,
+            mma_bf16_ts(tmem + L::T_DK, tmem + L::T_DS + packed_col<32>(j),
                         sdesc_sw128(sA + j * 2048, PANEL128, 1024), idQ, 1);
           mma_commit(BAR(K_DK_STEP));
         }
@@ -878,8 +829,8 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         if (!mbar_wait(BAR(K_DS_FULL), k & 1, ab)) { ok = false; break; }
         __syncwarp();
         tc_fence_after();
-        KWeights w{f_L, f_cT16, r, 128 * sb, Lr, er};
-        pack_block_in_place(tmem + loff + L::T_DS, q, sb == rb, w);
+        const KWeights w{f_L, f_cT16, r, 128 * sb, Lr, er};
+        pack_in_place<32>(tmem + loff + L::T_DS, 0, 2, q, sb == rb, w);
         tmem_wait_st();
         epi_arrive(BAR(K_DP_READY));
       }
@@ -914,6 +865,38 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
 }
 
 #undef BAR
+
+// Per-device pair of internal streams (chain then dk at the higher priority; g then dq at the
+// lower) and the events that fork the caller's stream into them and join it again. The enqueue
+// sequence runs under one lock, so calls from several host threads keep their dependencies
+// (their GPU work then serialises through the shared streams).
+struct ForkSet {
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t e0 = nullptr, eg = nullptr, ehi = nullptr, elo = nullptr;
+};
+constexpr int kMaxDevices = 64;
+ForkSet g_fork[kMaxDevices];
+std::mutex g_fork_mu;
+
+ForkSet* fork_set() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  ForkSet& f = g_fork[dev];
+  if (!f.hi) {
+    int lo_pri = 0, hi_pri = 0;
+    if (cudaDeviceGetStreamPriorityRange(&lo_pri, &hi_pri) != cudaSuccess) return nullptr;
+    ForkSet n;
+    if (cudaStreamCreateWithPriority(&n.hi, cudaStreamNonBlocking, hi_pri) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&n.lo, cudaStreamNonBlocking, lo_pri) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.e0, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.eg, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.ehi, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.elo, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    f = n;
+  }
+  return &f;
+}
 
 template <int D, int NB>
 cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
@@ -968,10 +951,21 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       (e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dk)) ||
       (e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dq)))
     return e;
-  kg<<<(int)(rows / 128), kSmallThreads, sm_g, s>>>(tK1, tW, tV1, p);
-  kc<<<BH * p.nslice, kThreads, sm_chain, s>>>(tK, tQ, tDO, p);
-  kq<<<BH * NC * NB, kSmallThreads, sm_dq, s>>>(tDO1, tW, tK1, tG1, p);
-  kk<<<BH * NC * NB, kSmallThreads, sm_dk, s>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, p);
+  std::lock_guard<std::mutex> lk(g_fork_mu);
+  ForkSet* f = fork_set();
+  if (!f) return cudaErrorInitializationError;
+  if ((e = cudaEventRecord(f->e0, s)) || (e = cudaStreamWaitEvent(f->hi, f->e0, 0)) ||
+      (e = cudaStreamWaitEvent(f->lo, f->e0, 0)))
+    return e;
+  kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, p);
+  kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
+  if ((e = cudaEventRecord(f->eg, f->lo))) return e;
+  kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, p);
+  if ((e = cudaEventRecord(f->elo, f->lo)) || (e = cudaStreamWaitEvent(f->hi, f->eg, 0))) return e;
+  kk<<<BH * NC * NB, kSmallThreads, sm_dk, f->hi>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, p);
+  if ((e = cudaEventRecord(f->ehi, f->hi)) || (e = cudaStreamWaitEvent(s, f->ehi, 0)) ||
+      (e = cudaStreamWaitEvent(s, f->elo, 0)))
+    return e;
   count_launches(4);
   return cudaGetLastError();
 }

@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Zq_h += (-S_hb) G_b; S (bf16) in TMEM, 32 packed columns per warpgroup
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-              mma_bf16_ts(tmem + L::T_Y + NV * h, tmem + L::tbuf(x) + 64 * (j / 4) + 8 * (j % 4),
+              mma_bf16_ts(tmem + L::T_Y + NV * h, tmem + L::tbuf(x) + packed_col<64>(j),
                           sdesc_sw128(sVc + b * PANEL128 + j * 2048, 0, 1024), idZ, 1);
             mma_commit(BAR(s_done[x]));
             if (x) ++sd1; else ++sd0;
@@ -453,32 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(BAR(p_full[x]), pu & 1, ab)) { ok = false; break; }
           __syncwarp();
           tc_fence_after();
-          const uint32_t tb = tmem + lane_off + L::tbuf(x) + 64 * g;
-          // this warp's 32 rows against each 32-key half: 0 all masked, 1 none, 2 the diagonal
-          int kind[2];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int idx = 2 * g + half;
-            kind[half] = b < h ? 1 : (idx < q ? 1 : (idx == q ? 2 : 0));
-          }
-          float pv[2][32];
-#pragma unroll
-          for (int half = 0; half < 2; ++half)
-            if (kind[half] != 0) tmem_ld32(tb + 32 * half, pv[half]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int r0 = 128 * b + 64 * g + 32 * half;
-            uint32_t pk[16];
-            if (kind[half] == 1)
-              score_weights32<false>(pv[half], f_L, f_cF16, srow, Ls, r0, pk);
-            else if (kind[half] == 2)
-              score_weights32<true>(pv[half], f_L, f_cF16, srow, Ls, r0, pk);
-            else
-#pragma unroll
-              for (int j = 0; j < 16; ++j) pk[j] = 0u;
-            tmem_st16u(tb + 16 * half, pk);
-          }
+          const QWeights w{f_L, f_cF16, srow, 128 * b, Ls};
+          pack_in_place<64>(tmem + lane_off + L::tbuf(x), g, g + 1, q, b == h, w);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
