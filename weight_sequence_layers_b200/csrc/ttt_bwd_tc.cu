@@ -113,26 +113,27 @@ struct ChainL {
   static constexpr uint32_t K_PANEL = C * 128;
   static constexpr uint32_t OFF_K = 0, OFF_Q = KP * K_PANEL, OFF_DO = 2 * KP * K_PANEL;
   static constexpr uint32_t OFF_DW = OFF_DO + C * 128;   // bf16 adjoint, MN-major [D][64]
-  static constexpr uint32_t OFF_S = OFF_DW + D * 128;    // dZ (C rows x 64)
+  static constexpr uint32_t OFF_S = OFF_DW + D * 128;    // dV = -dG (C rows x 64)
   static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;
   static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of 2 chunks
   static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
-  static constexpr uint32_t TX = 2 * KP * K_PANEL + C * 128;
+  static constexpr uint32_t TX_K = KP * K_PANEL, TX_QD = KP * K_PANEL + C * 128;
   // P^T blocks alternate between two TMEM buffers, S^T packed in place (bf16) for the X MMA;
   // Y reuses buffer 0 after the score loop
   static constexpr uint32_t T_DW = 0, T_X = 64, T_P0 = 64 + 64 * NB, T_P1 = T_P0 + 128,
                             T_Y = T_P0;
   static constexpr int NP = NB * (NB + 1) / 2;
 };
-enum { C_KV_FULL, C_KV_FREE, C_P_FULL, C_S_READY, C_XB0, C_X_FULL, C_W_READY, C_Y_FULL,
+enum { C_K_FULL, C_K_FREE, C_P_FULL, C_S_READY, C_XB0, C_X_FULL, C_W_READY, C_Y_FULL,
        C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_BG_FULL, C_BG_FULL1,
-       C_P_FULL1, C_S_READY1, C_NBARS };
+       C_P_FULL1, C_S_READY1, C_QD_FULL, C_QD_FREE, C_ST_READ, C_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_chain_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                     const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+                     const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmDV,
+                     const __grid_constant__ CUtensorMap tmDW, const BwdParams p) {
   using L = ChainL<D, NB>;
   constexpr int C = L::C;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -151,7 +152,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool mse = p.loss == 0;
   // arrivals per barrier, in enum order
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
-                               kEpiWarps, 1, 1, 1, kEpiWarps};
+                               kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1};
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   uint32_t tmem;
   setup(bars, counts, C_NBARS, tmem);
@@ -173,14 +174,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < NC; ++it) {
         const int c = NC - 1 - it;
         const int row0 = bh * p.T + c * C;
-        if (it > 0 && !mbar_wait(BAR(C_KV_FREE), (it - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(BAR(C_KV_FULL), L::TX);
+        // Q and dO are free once dW += Q^T (Gamma dO) is done, K after dW += K^T dZ
+        if (it > 0 && !mbar_wait(BAR(C_QD_FREE), (it - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(BAR(C_QD_FULL), L::TX_QD);
 #pragma unroll
-        for (int kp = 0; kp < L::KP; ++kp) {
-          tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(C_KV_FULL), 64 * kp, row0);
-          tma_load_2d(sQ + kp * L::K_PANEL, &tmQ, BAR(C_KV_FULL), 64 * kp, row0);
-        }
-        tma_load_2d(sDO, &tmDO, BAR(C_KV_FULL), NV * slice, row0);
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sQ + kp * L::K_PANEL, &tmQ, BAR(C_QD_FULL), 64 * kp, row0);
+        tma_load_2d(sDO, &tmDO, BAR(C_QD_FULL), NV * slice, row0);
+        if (it > 0 && !mbar_wait(BAR(C_K_FREE), (it - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(BAR(C_K_FULL), L::TX_K);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(C_K_FULL), 64 * kp, row0);
         if (it + 1 < NC) {
           if (it > 0 && !mbar_wait(BAR(C_SCAN_FULL), (it - 1) & 1, ab)) break;
           load_bg(it + 1);
@@ -192,11 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idP = idesc_bf16(128, 128, 0, 0);
       const uint32_t idX = idesc_bf16(128, NV, 0, 1);
       const uint32_t idW = idesc_bf16(128, NV, 1, 1);
+      const uint32_t idWn = idesc_bf16(128, NV, 1, 1, 1);
       const uint32_t lboT = D == 128 ? L::K_PANEL : 0;
       int sr0 = 0, sr1 = 0;  // S^T ready phases consumed per buffer
       int xb0 = 0;           // X MMAs committed on buffer 0
       for (int it = 0; it < NC; ++it) {
-        if (!mbar_wait(BAR(C_KV_FULL), it & 1, ab)) break;
+        if (!mbar_wait(BAR(C_K_FULL), it & 1, ab) || !mbar_wait(BAR(C_QD_FULL), it & 1, ab)) break;
         tc_fence_after();
         bool ok = true;
         // score blocks in order k = (rb, sb), sb >= rb; P^T_k goes to TMEM buffer k & 1, where the
@@ -250,20 +256,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16, 1024),
                         sdesc_sw128(sDW + j * 2048, 0, 1024), idX, j > 0);
         mma_commit(BAR(C_Y_FULL));
-        // dW (already Gamma_C-scaled) += Q^T (Gamma dO) + K^T dZ
+        // dW (already Gamma_C-scaled) += Q^T (Gamma dO) + K^T dZ, dZ = -dV (negated A)
         if (!mbar_wait(BAR(C_QS_READY), it & 1, ab)) break;
         tc_fence_after();
         for (int j = 0; j < C / 16; ++j)
           mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sQ + j * 2048, lboT, 1024),
                       sdesc_sw128(sDO + j * 2048, 0, 1024), idW, 1);
+        mma_commit(BAR(C_QD_FREE));
         if (!mbar_wait(BAR(C_DZ_READY), it & 1, ab)) break;
         tc_fence_after();
         if (mse)
           for (int j = 0; j < C / 16; ++j)
             mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sK + j * 2048, lboT, 1024),
-                        sdesc_sw128(sS + j * 2048, 0, 1024), idW, 1);
+                        sdesc_sw128(sS + j * 2048, 0, 1024), idWn, 1);
         mma_commit(BAR(C_DW_FULL));
-        mma_commit(BAR(C_KV_FREE));
+        mma_commit(BAR(C_K_FREE));
       }
     }
   } else {
@@ -352,11 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_st();
       }
       epi_arrive(BAR(C_QS_READY));
-      // ---- dG = -X - u Y ; dZ = dG (MSE) is published first, dV = -dG stored after
+      // ---- dV = -dG = X + u Y into shared memory (the MMA reads it as -dZ for MSE), then one
+      // bulk store per 128-row block, once the previous chunk's stores have read the buffers
       if (!mbar_wait(BAR(C_Y_FULL), it & 1, ab)) { ok = false; break; }
+      if (it > 0 && !mbar_wait(BAR(C_ST_READ), (it - 1) & 1, ab)) { ok = false; break; }
       __syncwarp();
       tc_fence_after();
-      float dg[NB][32];
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         const int r = 128 * b + lrow;
@@ -366,15 +374,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         const float u = f_eta[r] * f_eLC[r];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dg[b][j] = -x[j] - u * y[j];
-        if (mse) st_row32(sS, r, 4 * g, dg[b]);
+        for (int j = 0; j < 32; ++j) x[j] += u * y[j];
+        st_row32(sS, r, 4 * g, x);
       }
       epi_arrive(BAR(C_DZ_READY));
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) dg[b][j] = -dg[b][j];
-        st_global_bf16x32(p.dV + (tok0 + 128 * b + lrow) * D + NV * slice + 32 * g, dg[b]);
+      if (ew == 0) {
+        // one lane issues the stores; the warp leaves together if the wait ran out
+        if (lane == 0) {
+          ok = mbar_wait(BAR(C_DZ_READY), it & 1, ab);
+          if (ok) {
+            for (int b = 0; b < NB; ++b)
+              tma_store_2d(&tmDV, sS + b * PANEL128, NV * slice, (int)tok0 + 128 * b);
+            bulk_commit();
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
       }
       // ---- adjoint at the end of chunk c-1 (or dW0)
       if (!mbar_wait(BAR(C_DW_FULL), it & 1, ab)) { ok = false; break; }
@@ -386,7 +400,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         if (c > 0) {
           st_row32(sDW, lrow, 4 * g, w);
-          st_global_bf16x32(p.dWs + ((size_t)bh * NC + c - 1) * D * D + wcol, w);
         } else {
           float4* dst = reinterpret_cast<float4*>(p.dW0 + (size_t)bh * D * D + wcol);
 #pragma unroll
@@ -395,9 +408,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       epi_arrive(BAR(C_W_READY));
+      if (ew == 0) {
+        if (lane == 0) {
+          ok = mbar_wait(BAR(C_W_READY), (it + 1) & 1, ab);
+          if (ok && c > 0) {
+            tma_store_2d(&tmDW, sDW, NV * slice, (bh * NC + c - 1) * D);
+            bulk_commit();
+          }
+          // the next chunk rewrites dV and the adjoint copy only after these stores read them
+          bulk_wait_read0();
+          if (ok) mbar_arrive(BAR(C_ST_READ));
+        }
+        if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C_SCAN_FREE));
     }
+    if (ew == 0 && lane == 0) bulk_wait0();
   }
   teardown(bars, tmem);
 }
@@ -957,7 +984,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   if ((e = cudaEventRecord(f->e0, s)) || (e = cudaStreamWaitEvent(f->hi, f->e0, 0)) ||
       (e = cudaStreamWaitEvent(f->lo, f->e0, 0)))
     return e;
-  kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, p);
+  kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, tDV1, tDW, p);
   kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
   if ((e = cudaEventRecord(f->eg, f->lo))) return e;
   kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, p);

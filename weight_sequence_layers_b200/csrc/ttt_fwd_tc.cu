@@ -80,7 +80,7 @@ struct Layout {
 struct __align__(8) FwdBars {
   uint64_t k_full[2], k_free[2], v_full[2], v_free[2], q_full, q_free, z_full, g_ready, y_full,
       y_scaled, p_full[2], s_ready[2], s_done[2], zq_full, y_free, w_full, w0_ready, scan_full[2],
-      scan_free[2], bg_full[2];
+      scan_free[2], bg_full[2], o_ready, st_free;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -88,7 +88,8 @@ struct __align__(8) FwdBars {
 template <int D, int NB, int ACT, int LOSS>
 __global__ void __launch_bounds__(kThreads, 1)
     ttt_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                      const __grid_constant__ CUtensorMap tmWc, const FwdParams p) {
   using L = Layout<D, NB>;
   constexpr int C = L::C;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -135,6 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(BAR(bg_full[0]), 1);
     mbar_init(BAR(bg_full[1]), 1);
+    mbar_init(BAR(o_ready), kEpiWarps);
+    mbar_init(BAR(st_free), 1);
     bars->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -348,6 +351,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // -------- train view: G = a(Z) act'(Z) in place over V, and -u*G
       const uint32_t sVc = sV + (c & 1) * C * 128;
+      if (ew == 0 && c > 0) {
+        // the previous chunk's bulk stores (O from the -u*G buffer, the state checkpoint from
+        // the bf16 state copy) must have read their sources before those are rewritten
+        if (lane == 0) {
+          bulk_wait_read0();
+          mbar_arrive(BAR(st_free));
+        }
+        __syncwarp();
+      }
+      if (c > 0 && !mbar_wait(BAR(st_free), (c - 1) & 1, ab)) { ok = false; break; }
       if (!mbar_wait(BAR(v_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
       if (!mbar_wait(BAR(z_full), c & 1, ab)) { ok = false; break; }
       __syncwarp();
@@ -424,9 +437,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_ld();
             if (more) {
               st_row32(sW0, lrow, 4 * g, w);
-              if (p.W_chunks)
-                st_global_bf16x32(p.W_chunks + ((size_t)bh * NC + c + 1) * D * D +
-                                      (size_t)lrow * D + NV * slice + 32 * g, w);
               const float gnext = f_scan[((c + 1) & 1) * 6 * 256 + 512 + C - 1];
 #pragma unroll
               for (int j = 0; j < 32; ++j) w[j] *= gnext;
@@ -443,6 +453,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(BAR(w0_ready));
+          if (ew == 0 && c + 1 < NC && p.W_chunks) {
+            // checkpoint of the next chunk's start state, one bulk store of the bf16 copy
+            if (lane == 0) {
+              ok = mbar_wait(BAR(w0_ready), (c + 1) & 1, ab);
+              if (ok) {
+                tma_store_2d(&tmWc, sW0, NV * slice, (bh * NC + c + 1) * D);
+                bulk_commit();
+              }
+            }
+            if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
+          }
         }
 
         // -------- score blocks of this query half: S = -(Q K^T) * weights, bf16 in place
@@ -470,12 +491,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         tc_fence_after();
         {
+          // staged in the -u*G buffer (free since the transition MMA completed), one bulk store
           float o[32];
           tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, o);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = act_f<ACT>(o[j]);
-          st_global_bf16x32(p.O + (tok0 + srow) * D + NV * slice + 32 * g, o);
+          st_row32(sUG, srow, 4 * g, o);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(o_ready));
+        if (ew == 0) {
+          if (lane == 0) {
+            ok = mbar_wait(BAR(o_ready), (c * NB + h) & 1, ab);
+            if (ok) {
+              tma_store_2d(&tmO, sUG + h * PANEL128, NV * slice, (int)tok0 + 128 * h);
+              bulk_commit();
+            }
+          }
+          if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
         }
       }
       if (!ok) break;
@@ -483,6 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(y_free));
     }
+    if (ew == 0 && lane == 0) bulk_wait0();
   }
 #undef BAR
   tc_fence_before();
@@ -498,11 +534,15 @@ template <int D, int NB, int ACT, int LOSS>
 cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   using L = Layout<D, NB>;
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
-  CUtensorMap tk, tq, tv;
+  CUtensorMap tk, tq, tv, to, twc;
+  const uint64_t wrows = (uint64_t)a.B * a.H * (a.T / a.C) * D;
   if (!make_tmap_bf16(&tk, a.K, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tq, a.Q, D, rows, D, 64, 128) ||
-      !make_tmap_bf16(&tv, a.V, D, rows, D, 64, L::C))
+      !make_tmap_bf16(&tv, a.V, D, rows, D, 64, L::C) ||
+      !make_tmap_bf16(&to, a.O, D, rows, D, 64, 128) ||
+      (a.W_chunks && !make_tmap_bf16(&twc, a.W_chunks, D, wrows, D, 64, D)))
     return cudaErrorInvalidValue;
+  if (!a.W_chunks) twc = to;  // never used
   FwdParams p{};
   p.BH = a.B * a.H;
   p.T = a.T;
@@ -520,7 +560,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   auto k = ttt_fwd_tc_kernel<D, NB, ACT, LOSS>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, p);
+  k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, to, twc, p);
   count_launches(1);
   return cudaGetLastError();
 }
