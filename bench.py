@@ -167,25 +167,26 @@ class Layer:
         self.O = torch.empty((B, H, T, dv), device=dev, dtype=sd)
         self.Wf = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
         self.Wc = torch.empty((B, H, T // C, dk, dv), device=dev, dtype=sd)
+        self.G = torch.empty((B, H, T, dv), device=dev, dtype=sd)  # saved by fwd for bwd
         self.dQ = torch.empty((B, H, T, dk), device=dev, dtype=sd)
         self.dK = torch.empty((B, H, T, dk), device=dev, dtype=sd)
         self.dV = torch.empty((B, H, T, dv), device=dev, dtype=sd)
         self.dbeta = torch.empty((B, H, T), device=dev, dtype=torch.float32)
         self.dW0 = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
-        self.nf = ttt.ttt_workspace_bytes(self.c, False)
-        self.nb = ttt.ttt_workspace_bytes(self.c, True)
+        self.nf = ttt.ttt_workspace_bytes(self.c, 0)
+        self.nb = ttt.ttt_workspace_bytes(self.c, 2)
         self.ws = torch.empty(max(self.nf, self.nb, 16), device=dev, dtype=torch.uint8)
 
     def fwd(self):
         i = self.inp
         self.ttt.ttt_chunk_fwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
-                               self.O, self.Wf, self.Wc, self.ws, self.nf)
+                               self.O, self.Wf, self.Wc, self.G, self.ws, self.nf)
 
     def bwd(self):
         i = self.inp
         self.ttt.ttt_chunk_bwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
-                               self.Wc, i["dO"], i["dW_T"], self.dQ, self.dK, self.dV, self.dbeta,
-                               self.dW0, self.ws, self.nb)
+                               self.Wc, self.G, i["dO"], i["dW_T"], self.dQ, self.dK, self.dV,
+                               self.dbeta, self.dW0, self.ws, self.nb)
 
 
 def time_steps(layer, steps, warmup, sampler=None):

@@ -81,33 +81,38 @@ typedef struct {
  *   beta, gamma, dbeta  [B, H, T]       float32   (gamma NULL = no decay, gamma == 1)
  *   W0, W_final, dW_final, dW0   [B, H, dk, dv]  float32, row index = key feature
  *   W_chunks            [B, H, T/C, dk, dv]  dtype: the state at the start of every chunk
+ *   G_saved             [B, H, T, dv]   dtype: G of every token, the value the token's write
+ *                       subtracts (W_t = gamma_t W_{t-1} - eta_t k_t^T g_t)
  */
 
-/* Bytes of workspace ttt_chunk_fwd (for_bwd = 0) or ttt_chunk_bwd (for_bwd = 1) needs for
- * this config; 0 if none. Returns (size_t)-1 if the config is invalid. */
+/* Bytes of workspace ttt_chunk_fwd (for_bwd = 0) or ttt_chunk_bwd needs for this config; 0 if
+ * none. for_bwd = 1: the backward without G_saved (it rebuilds G in the workspace); for_bwd = 2:
+ * the backward given G_saved. Returns (size_t)-1 if the config (or for_bwd) is invalid. */
 size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd);
 
 /* Forward of the chunkwise TTT layer.
  *  in : Q, K, V, beta, gamma (nullable), W0
  *  out: O; W_final (nullable) = state after the last token; W_chunks (nullable) = chunk-start
- *       states, needed by ttt_chunk_bwd.
+ *       states, needed by ttt_chunk_bwd; G_saved (nullable) = G of every token, which
+ *       ttt_chunk_bwd then reads instead of rebuilding it.
  * bf16 configs with dk == dv in {64, 128} and C in {128, 256} run on the tcgen05 kernel;
  * other shapes (dk, dv <= 128, C <= 256) and all float32 configs run on the SIMT kernels. */
 ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0, void* O,
-                         float* W_final, void* W_chunks, void* workspace, size_t workspace_bytes,
-                         void* stream);
+                         float* W_final, void* W_chunks, void* G_saved, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /* Analytic backward of the layer for the objective J = <dO, O> + <dW_final, W_final>.
  *  in : Q, K, V, beta, gamma (nullable), W0, W_chunks (from ttt_chunk_fwd, required),
- *       dO, dW_final (nullable = 0)
+ *       G_saved (from ttt_chunk_fwd, nullable: rebuilt from W_chunks when NULL; kernels that
+ *       rebuild G anyway may ignore it), dO, dW_final (nullable = 0)
  *  out: dQ, dK, dV, dbeta, dW0 (plain stores, not accumulated). If the caller shares W0
  *       across the batch it reduces dW0 over B itself. No gradient is returned for gamma. */
 ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0,
-                         const void* W_chunks, const void* dO, const float* dW_final, void* dQ,
-                         void* dK, void* dV, float* dbeta, float* dW0, void* workspace,
-                         size_t workspace_bytes, void* stream);
+                         const void* W_chunks, const void* G_saved, const void* dO,
+                         const float* dW_final, void* dQ, void* dK, void* dV, float* dbeta,
+                         float* dW0, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Backward without caller-provided scratch (no counterpart in the papers: a deployment aid).
  * Some callers cannot allocate device memory when they call the library: a host framework
@@ -118,8 +123,8 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
  * on, until the process exits. It allocates nothing and calls no allocating routine.
  *  - Only configs of the tensor-core backward are accepted (bf16, identity activation,
  *    dk == dv in {64, 128}, C in {128, 256}); others return TTT_ERR_UNSUPPORTED.
- *  - Configs needing more than the fixed scratch (B*H*(T/C)*dk*dv*2 + B*H*T*dv*2 bytes) return
- *    TTT_ERR_WORKSPACE with nothing launched; ttt_chunk_bwd serves those.
+ *  - Configs needing more than the fixed scratch (B*H*(T/C)*dk*dv*2 bytes, plus B*H*T*dv*2 when
+ *    G_saved is NULL) return TTT_ERR_WORKSPACE with nothing launched; ttt_chunk_bwd serves those.
  *  - The first call on a device looks up the array's device address (with that device
  *    current); make that first call before any stream capture.
  *  - Every call shares the one array and leaves its contents behind. Calls that overlap on
@@ -128,9 +133,9 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
 #define TTT_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                                  const float* beta, const float* gamma, const float* W0,
-                                 const void* W_chunks, const void* dO, const float* dW_final,
-                                 void* dQ, void* dK, void* dV, float* dbeta, float* dW0,
-                                 void* stream);
+                                 const void* W_chunks, const void* G_saved, const void* dO,
+                                 const float* dW_final, void* dQ, void* dK, void* dV,
+                                 float* dbeta, float* dW0, void* stream);
 
 /* Workspace bytes of inplace_ttt_fwd; (size_t)-1 for invalid sizes. */
 size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C);

@@ -21,23 +21,25 @@ def gpu_inputs(cfg, seed=None):
     return synth.ttt_inputs(cfg, device="cuda", seed=seed)
 
 
-def run_fwd(cfg, inp):
+def run_fwd(cfg, inp, save_g=True):
     c = abi_config(cfg)
     sd = synth.storage_dtype(cfg)
     B, H, T, dk, dv, C = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C
     O = torch.empty((B, H, T, dv), device="cuda", dtype=sd)
     Wf = torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32)
     Wc = torch.empty((B, H, T // C, dk, dv), device="cuda", dtype=sd)
-    n = ttt.ttt_workspace_bytes(c, False)
+    G = torch.empty((B, H, T, dv), device="cuda", dtype=sd) if save_g else None
+    n = ttt.ttt_workspace_bytes(c, 0)
     ws = torch.empty(max(n, 16), device="cuda", dtype=torch.uint8)
     ttt.ttt_chunk_fwd(c, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], inp["W0"], O, Wf,
-                      Wc, ws, n)
+                      Wc, G, ws, n)
     torch.cuda.synchronize()
     assert ttt.ttt_get_device_error() == ttt.OK
-    return dict(O=O, W_final=Wf, W_chunks=Wc)
+    return dict(O=O, W_final=Wf, W_chunks=Wc, G=G)
 
 
-def run_bwd(cfg, inp, W_chunks):
+def run_bwd(cfg, inp, W_chunks, G=None):
+    """The backward; G (from run_fwd) is passed as G_saved, else the library rebuilds it."""
     c = abi_config(cfg)
     sd = synth.storage_dtype(cfg)
     B, H, T, dk, dv = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv
@@ -46,14 +48,32 @@ def run_bwd(cfg, inp, W_chunks):
                dV=torch.empty((B, H, T, dv), device="cuda", dtype=sd),
                dbeta=torch.empty((B, H, T), device="cuda", dtype=torch.float32),
                dW0=torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32))
-    n = ttt.ttt_workspace_bytes(c, True)
+    n = ttt.ttt_workspace_bytes(c, 2 if G is not None else 1)
     ws = torch.empty(max(n, 16), device="cuda", dtype=torch.uint8)
     ttt.ttt_chunk_bwd(c, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], inp["W0"],
-                      W_chunks, inp["dO"], inp["dW_T"], out["dQ"], out["dK"], out["dV"],
+                      W_chunks, G, inp["dO"], inp["dW_T"], out["dQ"], out["dK"], out["dV"],
                       out["dbeta"], out["dW0"], ws, n)
     torch.cuda.synchronize()
     assert ttt.ttt_get_device_error() == ttt.OK
     return out
+
+
+def reference_g(cfg, inp, W_chunks):
+    """G of every token written out from its definition, g_t = a(z_t) act'(z_t) with z_t = k_t W0
+    of the token's chunk (a = act(z) - v for MSE, -v for IP), in fp64 from the oracle's states."""
+    K = inp["K"].double().cpu().numpy()
+    V = inp["V"].double().cpu().numpy()
+    Wc = np.asarray(W_chunks, dtype=np.float64)
+    B, H, T, dk = K.shape
+    C = cfg.C
+    z = np.einsum("bhcsi,bhcij->bhcsj", K.reshape(B, H, T // C, C, dk), Wc).reshape(B, H, T, -1)
+    if cfg.act == "silu":
+        sg = 1.0 / (1.0 + np.exp(-z))
+        act, d1 = z * sg, sg * (1.0 + z * (1.0 - sg))
+    else:
+        act, d1 = z, np.ones_like(z)
+    a = act - V if cfg.loss == "mse" else -V
+    return a * d1
 
 
 def oracle_fwd(cfg, inp):

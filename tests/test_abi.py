@@ -43,8 +43,13 @@ def _cfg(**kw):
 
 
 def test_workspace_query_validates_config():
-    assert ttt.ttt_workspace_bytes(_cfg(), False) == 0
-    assert ttt.ttt_workspace_bytes(_cfg(), True) > 0
+    assert ttt.ttt_workspace_bytes(_cfg(), 0) == 0
+    assert ttt.ttt_workspace_bytes(_cfg(), 1) > 0
+    # the tensor-core backward keeps G in its workspace only when the forward's G is not passed
+    tc = _cfg(dtype="bf16", dk=128, dv=128, C=256, T=512)
+    assert 0 < ttt.ttt_workspace_bytes(tc, 2) < ttt.ttt_workspace_bytes(tc, 1)
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_workspace_bytes(tc, 3)
     for bad in (dict(T=250), dict(C=0), dict(B=0), dict(dk=0)):
         with pytest.raises(ttt.TTTError):
             ttt.ttt_workspace_bytes(_cfg(**bad), False)
@@ -57,7 +62,8 @@ def test_workspace_query_validates_config():
 def test_unsupported_shapes_are_reported():
     cfg = _cfg(dk=256)
     assert ttt.lib.ttt_workspace_bytes(ctypes.byref(cfg), 0) == ctypes.c_size_t(-1).value
-    st = ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), *([16] * 3), 16, None, 16, 16, None, None, None, 0, None)
+    st = ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), *([16] * 3), 16, None, 16, 16, None, None, None,
+                               None, 0, None)
     assert st == ttt.ERR_UNSUPPORTED
 
 
@@ -65,25 +71,27 @@ def test_fwd_argument_errors_before_launch():
     cfg = _cfg()
     call = lambda *p: ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), *p, None)
     A = 4096  # a 16-byte aligned fake address: never dereferenced on these paths
-    assert call(None, A, A, A, None, A, A, None, None, None, 0) == ttt.ERR_INVALID_ARG
-    assert call(A, A, A, A, None, A, None, None, None, None, 0) == ttt.ERR_INVALID_ARG
-    assert call(A + 4, A, A, A, None, A, A, None, None, None, 0) == ttt.ERR_ALIGNMENT
-    assert call(A, A, A, A, A + 8, A, A, None, None, None, 0) == ttt.ERR_ALIGNMENT
+    assert call(None, A, A, A, None, A, A, None, None, None, None, 0) == ttt.ERR_INVALID_ARG
+    assert call(A, A, A, A, None, A, None, None, None, None, None, 0) == ttt.ERR_INVALID_ARG
+    assert call(A + 4, A, A, A, None, A, A, None, None, None, None, 0) == ttt.ERR_ALIGNMENT
+    assert call(A, A, A, A, A + 8, A, A, None, None, None, None, 0) == ttt.ERR_ALIGNMENT
+    assert call(A, A, A, A, None, A, A, None, None, A + 2, None, 0) == ttt.ERR_ALIGNMENT  # G_saved
     bad = _cfg(T=100)
-    assert ttt.lib.ttt_chunk_fwd(ctypes.byref(bad), A, A, A, A, None, A, A, None, None, None, 0,
+    assert ttt.lib.ttt_chunk_fwd(ctypes.byref(bad), A, A, A, A, None, A, A, None, None, None, None,
+                                 0, None) == ttt.ERR_INVALID_ARG
+    assert ttt.lib.ttt_chunk_fwd(None, A, A, A, A, None, A, A, None, None, None, None, 0,
                                  None) == ttt.ERR_INVALID_ARG
-    assert ttt.lib.ttt_chunk_fwd(None, A, A, A, A, None, A, A, None, None, None, 0, None) == ttt.ERR_INVALID_ARG
 
 
 def test_bwd_requires_chunk_states_and_workspace():
     cfg = _cfg()
     A = 4096
-    base = [A, A, A, A, None, A, A, A, None, A, A, A, A, A]
+    base = [A, A, A, A, None, A, A, None, A, None, A, A, A, A, A]  # G_saved NULL
     args = list(base)
     args[6] = None  # W_chunks
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *args, None, 0, None) == ttt.ERR_INVALID_ARG
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *base, None, 0, None) == ttt.ERR_WORKSPACE
-    need = ttt.ttt_workspace_bytes(cfg, True)
+    need = ttt.ttt_workspace_bytes(cfg, 1)
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *base, A, need - 1, None) == ttt.ERR_WORKSPACE
 
 
@@ -109,5 +117,6 @@ def test_valid_call_without_a_gpu_reports_cuda_error():
         pytest.skip("a GPU is present")
     cfg = _cfg()
     A = 4096
-    st = ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), A, A, A, A, None, A, A, None, None, None, 0, None)
+    st = ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), A, A, A, A, None, A, A, None, None, None, None, 0,
+                               None)
     assert st == ttt.ERR_CUDA

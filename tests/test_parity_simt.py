@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import synth
-from _runners import oracle_bwd, oracle_fwd, run_bwd, run_fwd
+from _runners import oracle_bwd, oracle_fwd, reference_g, run_bwd, run_fwd
 from _util import rel_err
 
 pytestmark = pytest.mark.gpu
@@ -43,9 +43,10 @@ def test_fp32_forward_backward(shape, loss, act, decay):
     inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(3))
     got = run_fwd(cfg, inp)
     ref = oracle_fwd(cfg, inp)
-    for k in ("O", "W_final", "W_chunks"):
+    ref["G"] = reference_g(cfg, inp, ref["W_chunks"])
+    for k in ("O", "W_final", "W_chunks", "G"):
         assert rel_err(got[k], ref[k]) <= F32_TOL, k
-    g = run_bwd(cfg, inp, got["W_chunks"])
+    g = run_bwd(cfg, inp, got["W_chunks"], got["G"] if decay else None)
     r = oracle_bwd(cfg, inp)
     for k in ("dQ", "dK", "dV", "dbeta", "dW0"):
         assert rel_err(g[k], r[k]) <= F32_TOL, k

@@ -24,14 +24,15 @@ SHAPES = [
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("loss", ["mse", "ip"])
 @pytest.mark.parametrize("decay", [False, True])
-def test_tc_backward_small(shape, loss, decay):
+@pytest.mark.parametrize("saved_g", [True, False], ids=["g_from_fwd", "g_rebuilt"])
+def test_tc_backward_small(shape, loss, decay, saved_g):
     B, H, T, d, C = shape
     cfg = synth.TRAIN_1P45B.replace(B=B, H=H, T=T, dk=d, dv=d, C=C, loss=loss, act="id",
                                     decay=decay, w0_std=1.0 / d)
     inp = synth.ttt_inputs(cfg, device="cuda", seed=5 * T + d)
     inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(9))
-    fwd = run_fwd(cfg, inp)
-    got = run_bwd(cfg, inp, fwd["W_chunks"])
+    fwd = run_fwd(cfg, inp, save_g=saved_g)
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
     ref = oracle_bwd(cfg, inp)
     for k in GRADS:
         assert rel_err(got[k], ref[k]) <= TOL, (k, rel_err(got[k], ref[k]))
@@ -41,7 +42,7 @@ def test_tc_backward_full_size_sampled_heads():
     cfg = synth.TRAIN_1P45B
     inp = synth.ttt_inputs(cfg, device="cuda")
     fwd = run_fwd(cfg, inp)
-    got = run_bwd(cfg, inp, fwd["W_chunks"])
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
     rng = np.random.default_rng(44)
     heads = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(2)]
     sub = head_slice(inp, heads)

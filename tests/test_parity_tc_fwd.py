@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import synth
-from _runners import head_slice, oracle_fwd, run_fwd
+from _runners import head_slice, oracle_fwd, reference_g, run_fwd
 from _util import rel_err
 
 pytestmark = pytest.mark.gpu
@@ -30,7 +30,8 @@ def test_tc_forward_small(shape, loss, act, decay):
     inp = synth.ttt_inputs(cfg, device="cuda", seed=7 * T + d)
     got = run_fwd(cfg, inp)
     ref = oracle_fwd(cfg, inp)
-    for k in ("O", "W_final", "W_chunks"):
+    ref["G"] = reference_g(cfg, inp, ref["W_chunks"])
+    for k in ("O", "W_final", "W_chunks", "G"):
         assert rel_err(got[k], ref[k]) <= TOL, (k, rel_err(got[k], ref[k]))
 
 
@@ -56,6 +57,7 @@ def test_tc_forward_full_size_sampled_heads(cfg):
     sub = head_slice(inp, heads)
     sub_cfg = cfg.replace(B=1, H=len(heads))
     ref = oracle_fwd(sub_cfg, sub)
-    for k in ("O", "W_final", "W_chunks"):
+    ref["G"] = reference_g(sub_cfg, sub, ref["W_chunks"])
+    for k in ("O", "W_final", "W_chunks", "G"):
         g = torch.stack([got[k][b, h] for b, h in heads]).unsqueeze(0)
         assert rel_err(g, ref[k]) <= TOL, (k, rel_err(g, ref[k]))

@@ -19,7 +19,7 @@ TOL = 2e-2
 GRADS = ("dQ", "dK", "dV", "dbeta", "dW0")
 
 
-def noalloc_bwd(cfg, inp, W_chunks):
+def noalloc_bwd(cfg, inp, W_chunks, G=None):
     c = abi_config(cfg)
     sd = synth.storage_dtype(cfg)
     B, H, T, dk, dv = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv
@@ -31,7 +31,7 @@ def noalloc_bwd(cfg, inp, W_chunks):
     st = ttt.lib.ttt_chunk_bwd_noalloc(
         ctypes.byref(c), inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(),
         inp["beta"].data_ptr(), inp["gamma"].data_ptr(), inp["W0"].data_ptr(), W_chunks.data_ptr(),
-        inp["dO"].data_ptr(), inp["dW_T"].data_ptr(), out["dQ"].data_ptr(), out["dK"].data_ptr(),
+        G.data_ptr() if G is not None else None, inp["dO"].data_ptr(), inp["dW_T"].data_ptr(), out["dQ"].data_ptr(), out["dK"].data_ptr(),
         out["dV"].data_ptr(), out["dbeta"].data_ptr(), out["dW0"].data_ptr(),
         torch.cuda.current_stream().cuda_stream)
     assert st == ttt.OK, ttt.status_string(st)
@@ -41,25 +41,26 @@ def noalloc_bwd(cfg, inp, W_chunks):
 
 
 def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
-    # scratch needed: 4 heads x 4 chunks x 128 x 128 x 2 bytes = 512 KiB (limit 8 MiB)
+    # scratch needed: 4 heads x 4 chunks x 128 x 128 x 2 bytes = 512 KiB, plus 1 MiB of G when the
+    # forward's G is not passed (limit 8 MiB); the first call passes it, the second does not
     cfg = synth.TRAIN_1P45B.replace(B=1, H=4, T=1024)
-    for seed in (21, 22):
+    for seed, saved_g in ((21, True), (22, False)):
         inp = synth.ttt_inputs(cfg, device="cuda", seed=seed)
         inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(seed))
-        fwd = run_fwd(cfg, inp)
-        ref = run_bwd(cfg, inp, fwd["W_chunks"])
-        got = noalloc_bwd(cfg, inp, fwd["W_chunks"])
+        fwd = run_fwd(cfg, inp, save_g=saved_g)
+        ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
+        got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
         for k in GRADS:
             assert rel_err(got[k], ref[k]) <= TOL, (seed, k)
 
 
 def test_noalloc_backward_refuses_configs_beyond_its_scratch():
-    big = abi_config(synth.TRAIN_1P45B)  # needs 96 MiB of scratch
+    big = abi_config(synth.TRAIN_1P45B)  # needs 32 MiB of scratch even with G passed in
     A = 4096  # never dereferenced: the size check comes first
-    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(big), A, A, A, A, A, A, A, A, None, A, A, A, A,
-                                       A, None)
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(big), A, A, A, A, A, A, A, A, A, None, A, A, A,
+                                       A, A, None)
     assert st == ttt.ERR_WORKSPACE
     silu = abi_config(synth.TRAIN_1P45B.replace(B=1, H=1, T=256, act="silu"))
-    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(silu), A, A, A, A, A, A, A, A, None, A, A, A,
-                                       A, A, None)
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(silu), A, A, A, A, A, A, A, None, A, None, A,
+                                       A, A, A, A, None)
     assert st == ttt.ERR_UNSUPPORTED

@@ -44,15 +44,15 @@ _p, _i, _u, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_flo
 _cfgp = ctypes.POINTER(ttt_config)
 _SIGS = {
     "ttt_workspace_bytes": ([_cfgp, _i], _sz),
-    "ttt_chunk_fwd": ([_cfgp] + [_p] * 10 + [_sz, _p], _i),
-    "ttt_chunk_bwd": ([_cfgp] + [_p] * 15 + [_sz, _p], _i),
+    "ttt_chunk_fwd": ([_cfgp] + [_p] * 11 + [_sz, _p], _i),
+    "ttt_chunk_bwd": ([_cfgp] + [_p] * 16 + [_sz, _p], _i),
     "inplace_ttt_workspace_bytes": ([_i] * 4, _sz),
     "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 5 + [_sz, _p], _i),
     "ttt_get_device_error": ([_p], _i),
     "ttt_selftest_bounded_wait": ([_u, _p], _i),
     "ttt_status_string": ([_i], ctypes.c_char_p),
     "ttt_kernel_launches": ([], ctypes.c_ulonglong),
-    "ttt_chunk_bwd_noalloc": ([_cfgp] + [_p] * 14 + [_p], _i),
+    "ttt_chunk_bwd_noalloc": ([_cfgp] + [_p] * 15 + [_p], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -97,40 +97,41 @@ def make_config(B, H, T, dk, dv, C, dtype="bf16", loss="mse", act="id", lr_bias=
                       LOSS.get(loss, loss), ACT.get(act, act), float(lr_bias))
 
 
-def ttt_workspace_bytes(cfg: ttt_config, for_bwd: bool) -> int:
-    n = _lib.ttt_workspace_bytes(ctypes.byref(cfg), int(bool(for_bwd)))
+def ttt_workspace_bytes(cfg: ttt_config, for_bwd: int) -> int:
+    """for_bwd: 0 forward, 1 backward without G_saved, 2 backward given G_saved."""
+    n = _lib.ttt_workspace_bytes(ctypes.byref(cfg), int(for_bwd))
     if n == ctypes.c_size_t(-1).value:
         raise TTTError(ERR_INVALID_ARG, "ttt_workspace_bytes")
     return n
 
 
-def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None,
+def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None, G_saved=None,
                   workspace=None, workspace_bytes=0, stream=None):
     st = _lib.ttt_chunk_fwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
-                            _ptr(W0), _ptr(O), _ptr(W_final), _ptr(W_chunks), _ptr(workspace),
-                            int(workspace_bytes), _stream(stream))
+                            _ptr(W0), _ptr(O), _ptr(W_final), _ptr(W_chunks), _ptr(G_saved),
+                            _ptr(workspace), int(workspace_bytes), _stream(stream))
     _check(st, "ttt_chunk_fwd")
 
 
-def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final, dQ, dK, dV, dbeta, dW0,
-                  workspace=None, workspace_bytes=0, stream=None):
+def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, dQ, dK, dV,
+                  dbeta, dW0, workspace=None, workspace_bytes=0, stream=None):
     st = _lib.ttt_chunk_bwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
-                            _ptr(W0), _ptr(W_chunks), _ptr(dO), _ptr(dW_final), _ptr(dQ), _ptr(dK),
-                            _ptr(dV), _ptr(dbeta), _ptr(dW0), _ptr(workspace),
-                            int(workspace_bytes), _stream(stream))
+                            _ptr(W0), _ptr(W_chunks), _ptr(G_saved), _ptr(dO), _ptr(dW_final),
+                            _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta), _ptr(dW0),
+                            _ptr(workspace), int(workspace_bytes), _stream(stream))
     _check(st, "ttt_chunk_bwd")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
-def ttt_chunk_bwd_noalloc(cfg, Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final, dQ, dK, dV, dbeta,
-                          dW0, stream=None):
+def ttt_chunk_bwd_noalloc(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, dQ, dK,
+                          dV, dbeta, dW0, stream=None):
     """ttt_chunk_bwd for callers that cannot allocate: scratch is the library's fixed array."""
     st = _lib.ttt_chunk_bwd_noalloc(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
-                                    _ptr(gamma), _ptr(W0), _ptr(W_chunks), _ptr(dO),
-                                    _ptr(dW_final), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta),
-                                    _ptr(dW0), _stream(stream))
+                                    _ptr(gamma), _ptr(W0), _ptr(W_chunks), _ptr(G_saved),
+                                    _ptr(dO), _ptr(dW_final), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                    _ptr(dbeta), _ptr(dW0), _stream(stream))
     _check(st, "ttt_chunk_bwd_noalloc")
 
 

@@ -175,8 +175,9 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
       default: return (size_t)-1;
     }
   }
+  if (for_bwd != 1 && for_bwd != 2) return (size_t)-1;
   switch (bwd_path(a)) {
-    case PATH_TC: return tc_bwd_workspace(a);
+    case PATH_TC: return tc_bwd_workspace(a, for_bwd == 2);
     case PATH_SIMT: return simt_bwd_workspace(a);
     default: return (size_t)-1;
   }
@@ -184,12 +185,12 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
 
 ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0, void* O,
-                         float* W_final, void* W_chunks, void* workspace, size_t workspace_bytes,
-                         void* stream) {
+                         float* W_final, void* W_chunks, void* G_saved, void* workspace,
+                         size_t workspace_bytes, void* stream) {
   ttt_status st = check_config(cfg);
   if (st != TTT_OK) return st;
   if (!Q || !K || !V || !beta || !W0 || !O) return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {Q, K, V, beta, gamma, W0, O, W_final, W_chunks, workspace};
+  const void* ptrs[] = {Q, K, V, beta, gamma, W0, O, W_final, W_chunks, G_saved, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a = args_of(cfg);
@@ -201,7 +202,8 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
   unsigned* err = error_word(&e);
   if (!err) return TTT_ERR_CUDA;
   a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.W0 = W0; a.O = O;
-  a.W_final = W_final; a.W_chunks = W_chunks; a.ws = workspace; a.ws_bytes = workspace_bytes;
+  a.W_final = W_final; a.W_chunks = W_chunks; a.G_saved = G_saved; a.ws = workspace;
+  a.ws_bytes = workspace_bytes;
   a.err = err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launch_status(path == PATH_TC ? tc_fwd(a, s) : simt_fwd(a, s));
@@ -209,27 +211,29 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
 
 ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0,
-                         const void* W_chunks, const void* dO, const float* dW_final, void* dQ,
-                         void* dK, void* dV, float* dbeta, float* dW0, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+                         const void* W_chunks, const void* G_saved, const void* dO,
+                         const float* dW_final, void* dQ, void* dK, void* dV, float* dbeta,
+                         float* dW0, void* workspace, size_t workspace_bytes, void* stream) {
   ttt_status st = check_config(cfg);
   if (st != TTT_OK) return st;
   if (!Q || !K || !V || !beta || !W0 || !W_chunks || !dO || !dQ || !dK || !dV || !dbeta || !dW0)
     return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final,
+  const void* ptrs[] = {Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final,
                         dQ, dK, dV, dbeta, dW0, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a = args_of(cfg);
   const Path path = bwd_path(a);
   if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
-  const size_t need = path == PATH_TC ? tc_bwd_workspace(a) : simt_bwd_workspace(a);
+  const size_t need =
+      path == PATH_TC ? tc_bwd_workspace(a, G_saved != nullptr) : simt_bwd_workspace(a);
   if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   cudaError_t e;
   unsigned* err = error_word(&e);
   if (!err) return TTT_ERR_CUDA;
   a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.W0 = W0; a.W_chunks =
       const_cast<void*>(W_chunks);
+  a.G_saved = const_cast<void*>(G_saved);
   a.dO = dO; a.dW_final = dW_final; a.dQ = dQ; a.dK = dK; a.dV = dV; a.dbeta = dbeta;
   a.dW0 = dW0; a.ws = workspace; a.ws_bytes = workspace_bytes; a.err = err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

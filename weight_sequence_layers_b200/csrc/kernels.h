@@ -14,6 +14,7 @@ struct LayerArgs {
   void* O;
   float* W_final;
   void* W_chunks;
+  void* G_saved;  // nullable: G of every token [B, H, T, dv]
   const void* dO;
   const float* dW_final;
   void *dQ, *dK, *dV;
@@ -35,7 +36,7 @@ bool tc_fwd_supported(const LayerArgs& a);
 size_t tc_fwd_workspace(const LayerArgs& a);
 cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s);
 bool tc_bwd_supported(const LayerArgs& a);
-size_t tc_bwd_workspace(const LayerArgs& a);
+size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved);
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
 
 // In-Place TTT.

@@ -42,26 +42,29 @@ using namespace tttk;
 
 extern "C" ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q, const void* K,
                                             const void* V, const float* beta, const float* gamma,
-                                            const float* W0, const void* W_chunks, const void* dO,
+                                            const float* W0, const void* W_chunks,
+                                            const void* G_saved, const void* dO,
                                             const float* dW_final, void* dQ, void* dK, void* dV,
                                             float* dbeta, float* dW0, void* stream) {
   if (ttt_workspace_bytes(cfg, 1) == (size_t)-1) return TTT_ERR_INVALID_ARG;
   if (!Q || !K || !V || !beta || !W0 || !W_chunks || !dO || !dQ || !dK || !dV || !dbeta || !dW0)
     return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {Q, K, V, beta, gamma, W0, W_chunks, dO, dW_final, dQ, dK, dV, dbeta, dW0};
+  const void* ptrs[] = {Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final,
+                        dQ, dK, dV, dbeta, dW0};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a{};
   a.B = cfg->B; a.H = cfg->H; a.T = cfg->T; a.dk = cfg->dk; a.dv = cfg->dv; a.C = cfg->C;
   a.dtype = cfg->dtype; a.loss = cfg->loss; a.act = cfg->act; a.lr_bias = cfg->lr_bias;
   if (!tc_bwd_supported(a)) return TTT_ERR_UNSUPPORTED;
-  const size_t need = tc_bwd_workspace(a);
+  const size_t need = tc_bwd_workspace(a, G_saved != nullptr);
   if (need > TTT_NOALLOC_SCRATCH_BYTES) return TTT_ERR_WORKSPACE;
   void* scratch = scratch_address();
   unsigned* err = current_error_word();
   if (!scratch || !err) return TTT_ERR_CUDA;
   a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.W0 = W0;
   a.W_chunks = const_cast<void*>(W_chunks);
+  a.G_saved = const_cast<void*>(G_saved);
   a.dO = dO; a.dW_final = dW_final; a.dQ = dQ; a.dK = dK; a.dV = dV; a.dbeta = dbeta;
   a.dW0 = dW0; a.ws = scratch; a.ws_bytes = TTT_NOALLOC_SCRATCH_BYTES; a.err = err;
   return tc_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;

@@ -932,7 +932,8 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   const int BH = a.B * a.H, NC = a.T / a.C;
   const uint64_t wrows = (uint64_t)BH * NC * D;
   __nv_bfloat16* dWs = static_cast<__nv_bfloat16*>(a.ws);
-  __nv_bfloat16* G = dWs + wrows * D;
+  const bool g_saved = a.G_saved != nullptr;
+  __nv_bfloat16* G = g_saved ? static_cast<__nv_bfloat16*>(a.G_saved) : dWs + wrows * D;
   CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tG1, tW, tDW;
   if (!make_tmap_bf16(&tK, a.K, D, rows, D, 64, C) || !make_tmap_bf16(&tQ, a.Q, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tDO, a.dO, D, rows, D, 64, C) ||
@@ -985,7 +986,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       (e = cudaStreamWaitEvent(f->lo, f->e0, 0)))
     return e;
   kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, tDV1, tDW, p);
-  kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
+  if (!g_saved) kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
   if ((e = cudaEventRecord(f->eg, f->lo))) return e;
   kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, p);
   if ((e = cudaEventRecord(f->elo, f->lo)) || (e = cudaStreamWaitEvent(f->hi, f->eg, 0))) return e;
@@ -993,7 +994,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   if ((e = cudaEventRecord(f->ehi, f->hi)) || (e = cudaStreamWaitEvent(s, f->ehi, 0)) ||
       (e = cudaStreamWaitEvent(s, f->elo, 0)))
     return e;
-  count_launches(4);
+  count_launches(g_saved ? 3 : 4);
   return cudaGetLastError();
 }
 
@@ -1004,9 +1005,10 @@ bool tc_bwd_supported(const LayerArgs& a) {
          (a.C == 128 || a.C == 256) && a.T % a.C == 0;
 }
 
-// [BH, NC, dk, dv] bf16 chunk-end adjoints, then [BH, T, dv] bf16 G
-size_t tc_bwd_workspace(const LayerArgs& a) {
-  return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2 + (size_t)a.B * a.H * a.T * a.dv * 2;
+// [BH, NC, dk, dv] bf16 chunk-end adjoints, then (without G from the forward) [BH, T, dv] bf16 G
+size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved) {
+  return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2 +
+         (g_saved ? 0 : (size_t)a.B * a.H * a.T * a.dv * 2);
 }
 
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s) {

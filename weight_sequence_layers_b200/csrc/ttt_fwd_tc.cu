@@ -51,6 +51,7 @@ struct FwdParams {
   __nv_bfloat16* O;       // [BH, T, D]
   float* W_final;         // nullable
   __nv_bfloat16* W_chunks;  // nullable, [BH, NC, D, D]
+  int save_g;               // store G of every token (bulk stores through tmG)
   unsigned* err;
 };
 
@@ -80,7 +81,7 @@ struct Layout {
 struct __align__(8) FwdBars {
   uint64_t k_full[2], k_free[2], v_full[2], v_free[2], q_full, q_free, z_full, g_ready, y_full,
       y_scaled, p_full[2], s_ready[2], s_done[2], zq_full, y_free, w_full, w0_ready, scan_full[2],
-      scan_free[2], bg_full[2], o_ready, st_free;
+      scan_free[2], bg_full[2], o_ready, st_free, g_read[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -89,7 +90,8 @@ template <int D, int NB, int ACT, int LOSS>
 __global__ void __launch_bounds__(kThreads, 1)
     ttt_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                      const __grid_constant__ CUtensorMap tmWc, const FwdParams p) {
+                      const __grid_constant__ CUtensorMap tmWc, const __grid_constant__ CUtensorMap tmG,
+                      const FwdParams p) {
   using L = Layout<D, NB>;
   constexpr int C = L::C;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -138,6 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(BAR(bg_full[1]), 1);
     mbar_init(BAR(o_ready), kEpiWarps);
     mbar_init(BAR(st_free), 1);
+    mbar_init(BAR(g_read[0]), 1);
+    mbar_init(BAR(g_read[1]), 1);
     bars->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -174,6 +178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // V slice of chunk c into buffer c & 1, free once chunk c-2's last S G MMA is done
         const int vb = c & 1;
         if (c >= 2 && !mbar_wait(BAR(v_free[vb]), ((c - 2) >> 1) & 1, ab)) goto done_prod;
+        // with G saved, the bulk store of chunk c-2's G (in place over its V) must have read it
+        if (c >= 2 && p.save_g && !mbar_wait(BAR(g_read[vb]), ((c - 2) >> 1) & 1, ab))
+          goto done_prod;
         mbar_arrive_expect_tx(BAR(v_full[vb]), L::V_TX);
         tma_load_2d(sV + vb * C * 128, &tmV, BAR(v_full[vb]), NV * slice, row0);
         for (int h = 0; h < NB; ++h) {
@@ -357,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           bulk_wait_read0();
           mbar_arrive(BAR(st_free));
+          mbar_arrive(BAR(g_read[(c - 1) & 1]));
         }
         __syncwarp();
       }
@@ -397,6 +405,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(g_ready));
+      if (ew == 0 && p.save_g) {
+        // G of the chunk's tokens, one bulk store per 128-row block of this value slice
+        if (lane == 0) {
+          ok = mbar_wait(BAR(g_ready), c & 1, ab);
+          if (ok) {
+            for (int b = 0; b < NB; ++b)
+              tma_store_2d(&tmG, sVc + b * PANEL128, NV * slice, (int)tok0 + 128 * b);
+            bulk_commit();
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
+      }
 
       for (int h = 0; h < NB && ok; ++h) {
         const int k0 = h * (h + 1) / 2;
@@ -534,15 +554,17 @@ template <int D, int NB, int ACT, int LOSS>
 cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   using L = Layout<D, NB>;
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
-  CUtensorMap tk, tq, tv, to, twc;
+  CUtensorMap tk, tq, tv, to, twc, tg;
   const uint64_t wrows = (uint64_t)a.B * a.H * (a.T / a.C) * D;
   if (!make_tmap_bf16(&tk, a.K, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tq, a.Q, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tv, a.V, D, rows, D, 64, L::C) ||
       !make_tmap_bf16(&to, a.O, D, rows, D, 64, 128) ||
-      (a.W_chunks && !make_tmap_bf16(&twc, a.W_chunks, D, wrows, D, 64, D)))
+      (a.W_chunks && !make_tmap_bf16(&twc, a.W_chunks, D, wrows, D, 64, D)) ||
+      (a.G_saved && !make_tmap_bf16(&tg, a.G_saved, D, rows, D, 64, 128)))
     return cudaErrorInvalidValue;
   if (!a.W_chunks) twc = to;  // never used
+  if (!a.G_saved) tg = to;    // never used
   FwdParams p{};
   p.BH = a.B * a.H;
   p.T = a.T;
@@ -555,12 +577,13 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.O = static_cast<__nv_bfloat16*>(a.O);
   p.W_final = a.W_final;
   p.W_chunks = static_cast<__nv_bfloat16*>(a.W_chunks);
+  p.save_g = a.G_saved != nullptr;
   p.err = a.err;
   const size_t smem = L::BYTES + 1024;
   auto k = ttt_fwd_tc_kernel<D, NB, ACT, LOSS>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, to, twc, p);
+  k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, to, twc, tg, p);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -64,7 +64,7 @@ template <typename TI>
 __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, const TI* K,
                                                        const TI* V, const float* beta,
                                                        const float* gamma, const float* W0,
-                                                       TI* O, float* Wf, TI* Wc) {
+                                                       TI* O, float* Wf, TI* Wc, TI* Gs) {
   extern __shared__ float smem[];
   const int bh = blockIdx.y, j0 = blockIdx.x * kNvs;
   const int nv = min(kNvs, d.dv - j0);
@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
       const float vv = ldf(V + v0 + (tc + s) * dv + j0 + j);
       const float a = d.loss == 0 ? actf(d.act, z) - vv : -vv;
       G[s * kNvs + j] = a * act1(d.act, z);
+      if (Gs) stf(&Gs[v0 + (tc + s) * dv + j0 + j], G[s * kNvs + j]);
     }
     __syncthreads();
     // query view, kRows queries at a time
@@ -329,13 +330,15 @@ cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
     auto k = simt_fwd_kernel<float>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<grid, 256, smem, s>>>(d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta,
-                              a.gamma, a.W0, (float*)a.O, a.W_final, (float*)a.W_chunks);
+                              a.gamma, a.W0, (float*)a.O, a.W_final, (float*)a.W_chunks,
+                              (float*)a.G_saved);
   } else {
     auto k = simt_fwd_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<grid, 256, smem, s>>>(d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K,
                               (const __nv_bfloat16*)a.V, a.beta, a.gamma, a.W0,
-                              (__nv_bfloat16*)a.O, a.W_final, (__nv_bfloat16*)a.W_chunks);
+                              (__nv_bfloat16*)a.O, a.W_final, (__nv_bfloat16*)a.W_chunks,
+                              (__nv_bfloat16*)a.G_saved);
   }
   count_launches(1);
   return cudaGetLastError();
