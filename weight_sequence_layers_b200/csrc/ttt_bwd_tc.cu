@@ -154,6 +154,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
                                kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1};
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDV);
+    tma_prefetch_desc(&tmDW);
+  }
   uint32_t tmem;
   setup(bars, counts, C_NBARS, tmem);
   Abort ab{&bars->abort_flag, p.err};
@@ -533,13 +540,13 @@ struct DqL {
   static constexpr uint32_t T_DQ = 0, T_DS = D;
 };
 enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_G_FULL, Q_K_FULL, Q_DS_FULL, Q_DP_READY, Q_DP_DONE,
-       Q_DQ_FULL, Q_SCAN, Q_NBARS };
+       Q_DQ_FULL, Q_SCAN, Q_ST, Q_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmW,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmG,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using L = DqL<D, NB>;
   constexpr int C = L::C;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -555,7 +562,14 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int sb = blockIdx.x % NB;
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
-  const int counts[Q_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1};
+  const int counts[Q_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, kSmallEpi};
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmG);
+    tma_prefetch_desc(&tmDQ);
+  }
   uint32_t tmem;
   setup(bars, counts, Q_NBARS, tmem, 256);
   Abort ab{&bars->abort_flag, p.err};
@@ -669,6 +683,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         epi_arrive(BAR(Q_DP_READY));
       }
       if (!ok) break;
+      // dQ staged in the dO slot (its last readers, the MMAs, are complete), one bulk store
       if (!mbar_wait(BAR(Q_DQ_FULL), 0, ab)) break;
       __syncwarp();
       tc_fence_after();
@@ -677,7 +692,15 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         float v[32];
         tmem_ld32(tmem + loff + L::T_DQ + 32 * cc, v);
         tmem_wait_ld();
-        st_global_bf16x32(p.dQ + ((size_t)tokc + s) * D + 32 * cc, v);
+        st_row32(sDO + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+      }
+      epi_arrive(BAR(Q_ST));
+      if (ew == 0 && lane == 0 && mbar_wait(BAR(Q_ST), 0, ab)) {
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_store_2d(&tmDQ, sDO + kp * PANEL128, 64 * kp, tokc + 128 * sb);
+        bulk_commit();
+        bulk_wait_read0();
       }
     } while (0);
   }
@@ -702,14 +725,14 @@ struct DkL {
   static constexpr uint32_t T_DK = 0, T_DS = D;
 };
 enum { K_LD0, K_H, K_H_SCALED, K_DO_FULL, K_Q_FULL, K_DS_FULL, K_DP_READY, K_DK_STEP,
-       K_DVW_FULL, K_DK_FULL, K_SCAN, K_NBARS };
+       K_DVW_FULL, K_DK_FULL, K_SCAN, K_ST, K_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
     bwd_dk_kernel(const __grid_constant__ CUtensorMap tmG, const __grid_constant__ CUtensorMap tmDW,
                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmDV, const __grid_constant__ CUtensorMap tmW,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDK, const BwdParams p) {
   using L = DkL<D, NB>;
   constexpr int C = L::C;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -726,7 +749,16 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
   const bool mse = p.loss == 0;
-  const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1};
+  const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1, kSmallEpi};
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmG);
+    tma_prefetch_desc(&tmDW);
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDV);
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmDK);
+  }
   uint32_t tmem;
   setup(bars, counts, K_NBARS, tmem, 256);
   Abort ab{&bars->abort_flag, p.err};
@@ -876,6 +908,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         }
         p.dbeta[(size_t)tokc + r] = -(1.f - 0.5f * er) * dot;
       }
+      // dK staged over this thread's own row of G (every reader of G is done), one bulk store
       if (!mbar_wait(BAR(K_DK_FULL), 0, ab)) break;
       __syncwarp();
       tc_fence_after();
@@ -884,7 +917,15 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         float v[32];
         tmem_ld32(tmem + loff + L::T_DK + 32 * cc, v);
         tmem_wait_ld();
-        st_global_bf16x32(p.dK + ((size_t)tokc + r) * D + 32 * cc, v);
+        st_row32(sG + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+      }
+      epi_arrive(BAR(K_ST));
+      if (ew == 0 && lane == 0 && mbar_wait(BAR(K_ST), 0, ab)) {
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_store_2d(&tmDK, sG + kp * PANEL128, 64 * kp, tokc + 128 * rb);
+        bulk_commit();
+        bulk_wait_read0();
       }
     } while (0);
   }
@@ -934,7 +975,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   __nv_bfloat16* dWs = static_cast<__nv_bfloat16*>(a.ws);
   const bool g_saved = a.G_saved != nullptr;
   __nv_bfloat16* G = g_saved ? static_cast<__nv_bfloat16*>(a.G_saved) : dWs + wrows * D;
-  CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tG1, tW, tDW;
+  CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tG1, tW, tDW, tDQ1, tDK1;
   if (!make_tmap_bf16(&tK, a.K, D, rows, D, 64, C) || !make_tmap_bf16(&tQ, a.Q, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tDO, a.dO, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tK1, a.K, D, rows, D, 64, 128) ||
@@ -942,6 +983,8 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       !make_tmap_bf16(&tQ1, a.Q, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tDO1, a.dO, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tDV1, a.dV, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tDQ1, a.dQ, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tDK1, a.dK, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tG1, G, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tW, a.W_chunks, D, wrows, D, 64, D) ||
       !make_tmap_bf16(&tDW, dWs, D, wrows, D, 64, D))
@@ -988,9 +1031,9 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, tDV1, tDW, p);
   if (!g_saved) kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
   if ((e = cudaEventRecord(f->eg, f->lo))) return e;
-  kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, p);
+  kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, tDQ1, p);
   if ((e = cudaEventRecord(f->elo, f->lo)) || (e = cudaStreamWaitEvent(f->hi, f->eg, 0))) return e;
-  kk<<<BH * NC * NB, kSmallThreads, sm_dk, f->hi>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, p);
+  kk<<<BH * NC * NB, kSmallThreads, sm_dk, f->hi>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, tDK1, p);
   if ((e = cudaEventRecord(f->ehi, f->hi)) || (e = cudaStreamWaitEvent(s, f->ehi, 0)) ||
       (e = cudaStreamWaitEvent(s, f->elo, 0)))
     return e;
