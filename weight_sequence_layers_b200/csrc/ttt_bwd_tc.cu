@@ -41,7 +41,7 @@ namespace tttk {
 namespace {
 
 constexpr int NV = 64;
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;  // chain: producer, MMA, 8 epilogue warps, scan warp
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t PANEL128 = 128 * 128;
@@ -63,7 +63,7 @@ struct BwdParams {
 };
 
 struct __align__(8) Bars {
-  uint64_t b[20];
+  uint64_t b[24];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -115,7 +115,7 @@ struct ChainL {
   static constexpr uint32_t OFF_DW = OFF_DO + C * 128;   // bf16 adjoint, MN-major [D][64]
   static constexpr uint32_t OFF_S = OFF_DW + D * 128;    // dV = -dG (C rows x 64)
   static constexpr uint32_t OFF_F = OFF_S + 2 * PANEL128;
-  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of 2 chunks
+  static constexpr uint32_t OFF_BG = OFF_F + 2 * 6 * 256 * 4;  // beta, gamma of 2 chunks
   static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t TX_K = KP * K_PANEL, TX_QD = KP * K_PANEL + C * 128;
@@ -127,7 +127,8 @@ struct ChainL {
 };
 enum { C_K_FULL, C_K_FREE, C_P_FULL, C_S_READY, C_XB0, C_X_FULL, C_W_READY, C_Y_FULL,
        C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_BG_FULL, C_BG_FULL1,
-       C_P_FULL1, C_S_READY1, C_QD_FULL, C_QD_FREE, C_ST_READ, C_NBARS };
+       C_P_FULL1, C_S_READY1, C_QD_FULL, C_QD_FREE, C_ST_READ, C_SCAN_FULL1, C_SCAN_FREE1,
+       C_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -142,9 +143,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sb0 = smem_u32(smem);
   const uint32_t sK = sb0 + L::OFF_K, sQ = sb0 + L::OFF_Q, sDO = sb0 + L::OFF_DO,
                  sDW = sb0 + L::OFF_DW, sS = sb0 + L::OFF_S;
-  float* f = reinterpret_cast<float*>(smem + L::OFF_F);
-  float *f_eta = f, *f_L = f + 256, *f_gam = f + 512, *f_eLC = f + 768, *f_cF16 = f + 1024,
-        *f_cT16 = f + 1280;
+  // scan arrays of buffer i (iteration it uses buffer it & 1): eta, L, Gamma, exp(L_C - L),
+  // cF16, cT16, each 256 floats
+  float* f_scan = reinterpret_cast<float*>(smem + L::OFF_F);
   Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / p.nslice, slice = blockIdx.x % p.nslice;
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool mse = p.loss == 0;
   // arrivals per barrier, in enum order
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
-                               kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1};
+                               kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1, 1, kEpiWarps};
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmK);
@@ -194,7 +195,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kp = 0; kp < L::KP; ++kp)
           tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(C_K_FULL), 64 * kp, row0);
         if (it + 1 < NC) {
-          if (it > 0 && !mbar_wait(BAR(C_SCAN_FULL), (it - 1) & 1, ab)) break;
+          // buffer (it + 1) & 1 was last read by the scan of iteration it - 1
+          if (it > 0 && !mbar_wait(BAR((it - 1) & 1 ? C_SCAN_FULL1 : C_SCAN_FULL), ((it - 1) >> 1) & 1, ab))
+            break;
           load_bg(it + 1);
         }
       }
@@ -280,6 +283,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(BAR(C_K_FREE));
       }
     }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ scans, one iteration ahead
+    for (int it = 0; it < NC; ++it) {
+      const int sb = it & 1;
+      if (it >= 2 && !mbar_wait(BAR(sb ? C_SCAN_FREE1 : C_SCAN_FREE), ((it - 2) >> 1) & 1, ab)) break;
+      if (!mbar_wait(BAR(C_BG_FULL + sb), (it >> 1) & 1, ab)) break;
+      const float* bg = f_bg + sb * 2 * C;
+      float* fs = f_scan + sb * 6 * 256;
+      chunk_scan_warp<C>(bg, p.gamma ? bg + C : nullptr, p.lr_bias, fs, fs + 256, fs + 512,
+                         fs + 768, fs + 1024, fs + 1280);
+      if (lane == 0) mbar_arrive(BAR(sb ? C_SCAN_FULL1 : C_SCAN_FULL));
+    }
   } else {
     const int ew = warp - 2, g = ew / 4, q = warp & 3, lrow = q * 32 + lane;
     const uint32_t loff = (uint32_t)(q * 32) << 16;
@@ -309,15 +324,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int it = 0; it < NC && ok; ++it) {
       const int c = NC - 1 - it;
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
-      if (ew == 0) {
-        if (it > 0 && !mbar_wait(BAR(C_SCAN_FREE), (it - 1) & 1, ab)) { ok = false; break; }
-        if (!mbar_wait(BAR(C_BG_FULL + (it & 1)), (it >> 1) & 1, ab)) { ok = false; break; }
-        const float* bg = f_bg + (it & 1) * 2 * C;
-        chunk_scan_warp<C>(bg, p.gamma ? bg + C : nullptr, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
-                           f_cF16, f_cT16);
-        if (lane == 0) mbar_arrive(BAR(C_SCAN_FULL));
-      }
-      if (!mbar_wait(BAR(C_SCAN_FULL), it & 1, ab)) { ok = false; break; }
+      // this iteration's scan arrays (computed by warp 10 one iteration ahead)
+      if (!mbar_wait(BAR(it & 1 ? C_SCAN_FULL1 : C_SCAN_FULL), (it >> 1) & 1, ab)) { ok = false; break; }
+      const float* f_eta = f_scan + (it & 1) * 6 * 256;
+      const float *f_L = f_eta + 256, *f_gam = f_eta + 512, *f_eLC = f_eta + 768,
+                  *f_cT16 = f_eta + 1280;
       // ---- S^T blocks: S^T_rs = P^T_rs eta_r exp(L_s - L_r), s >= r, packed to bf16 in place
       // (block k in TMEM buffer k & 1; warpgroup g packs query columns [64g, 64g+64))
       for (int k = 0; k < L::NP && ok; ++k) {
@@ -429,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C_SCAN_FREE));
+      if (lane == 0) mbar_arrive(BAR(it & 1 ? C_SCAN_FREE1 : C_SCAN_FREE));
     }
     if (ew == 0 && lane == 0) bulk_wait0();
   }
