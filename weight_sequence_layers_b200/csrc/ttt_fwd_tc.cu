@@ -13,9 +13,11 @@
 // evolve independently, so d_v = 128 runs as two CTAs per head. The fp32 state lives in TMEM
 // for the whole sequence; a bf16 copy in shared memory is the MMA operand of the next chunk.
 //
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner), warps 2-9 epilogue
+// Warp roles: warp 0 TMA producer; warp 1 issues the state-chain MMAs (Z = K W0 and the
+// transition) and owns TMEM; warp 11 issues the query-side MMAs (Y = Q W0, the score blocks and
+// S G), so the next chunk's Z never waits behind this chunk's score work; warps 2-9 epilogue
 // (two warpgroups; warpgroup g handles value columns [32g, 32g+32) of each 128-row block and
-// score columns [64g, 64g+64) of each 128x128 score block), warp 10 computes the lr and decay
+// score columns [64g, 64g+64) of each 128x128 score block); warp 10 computes the lr and decay
 // scans of the next chunk into the other of two buffers. Every wait is bounded.
 //
 // TMEM columns: [0,64) W (lanes = key features; held pre-multiplied by the chunk's Gamma_C),
@@ -37,7 +39,7 @@ namespace tttk {
 namespace {
 
 constexpr int NV = 64;             // value columns per CTA
-constexpr int kThreads = 352;      // 11 warps
+constexpr int kThreads = 384;      // 12 warps
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t PANEL128 = 128 * 128;  // 128 rows x 128 bytes
@@ -61,27 +63,26 @@ struct Layout {
   static constexpr int KP = D / 64;                      // 64-wide key-feature panels
   static constexpr uint32_t KH = KP * PANEL128;          // one 128-row half of K (or of Q)
   static constexpr uint32_t OFF_K = 0;                   // K half b, panel p at OFF_K + (b KP + p) PANEL128
-  static constexpr uint32_t OFF_Q = OFF_K + NB * KH;     // one 128-row half of Q
-  static constexpr uint32_t OFF_V = OFF_Q + KH;          // V slice of chunk c in buffer c & 1; G in place
-  static constexpr uint32_t OFF_UG = OFF_V + 2 * C * 128;
-  static constexpr uint32_t OFF_W0 = OFF_UG + C * 128;   // bf16 state, MN-major [D][64]
-  static constexpr uint32_t OFF_F = OFF_W0 + D * 128;    // scan arrays, 2 buffers x 6 x 256
+  static constexpr uint32_t OFF_Q = OFF_K + NB * KH;     // Q half h at OFF_Q + h KH
+  // two rotating buffers: chunk c's V (then G, in place) in buffer c & 1 and its -u G in the
+  // other one, which then receives V of chunk c + 1 once the transition MMA has read -u G
+  static constexpr uint32_t OFF_VG = OFF_Q + NB * KH;
+  static constexpr uint32_t OFF_W0 = OFF_VG + 2 * C * 128;  // bf16 state, MN-major [D][64]
+  static constexpr uint32_t OFF_F = OFF_W0 + D * 128;       // scan arrays, 2 buffers x 6 x 256
   static constexpr uint32_t OFF_BG = OFF_F + 2 * 6 * 256 * 4;  // beta, gamma of 2 chunks
   static constexpr uint32_t OFF_BAR = OFF_BG + 4 * C * 4;
-  static constexpr uint32_t BYTES = OFF_BAR + 256;
+  static constexpr uint32_t BYTES = OFF_BAR + 512;
   static constexpr uint32_t V_TX = C * 128;
   // TMEM columns
   static constexpr uint32_t T_W = 0, T_Z = 64, T_Y = 64 + 64 * NB, T_PA = 64 + 128 * NB;
-  static constexpr int NP = NB * (NB + 1) / 2;  // causal score blocks per chunk
-  // score block k (order (0,0), (1,0), (1,1)) -> buffer: the middle one goes to the Z columns
-  __host__ __device__ static constexpr int buf(int k) { return (NB == 2 && k == 1) ? 1 : 0; }
+  // score buffer x: A (x = 0) its own 128 columns, B (x = 1) the Z columns once G is formed
   __host__ __device__ static constexpr uint32_t tbuf(int x) { return x ? T_Z : T_PA; }
 };
 
 struct __align__(8) FwdBars {
-  uint64_t k_full[2], k_free[2], v_full[2], v_free[2], q_full, q_free, z_full, g_ready, y_full,
-      y_scaled, p_full[2], s_ready[2], s_done[2], zq_full, y_free, w_full, w0_ready, scan_full[2],
-      scan_free[2], bg_full[2], o_ready, st_free, g_read[2];
+  uint64_t k_full[2], k_free[2], q_full[2], q_free[2], v_full[2], z_full, g_ready, y_full[2],
+      y_scaled[2], p_full[2], s_ready[2], s_done[2], zq_full[2], y_free[2], w_full, w0_ready,
+      g_done, scan_full[2], scan_free[2], bg_full[2], st_free, g_read[2];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -89,17 +90,16 @@ struct __align__(8) FwdBars {
 template <int D, int NB, int ACT, int LOSS>
 __global__ void __launch_bounds__(kThreads, 1)
     ttt_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                      const __grid_constant__ CUtensorMap tmWc, const __grid_constant__ CUtensorMap tmG,
-                      const FwdParams p) {
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmWc,
+                      const __grid_constant__ CUtensorMap tmG, const FwdParams p) {
   using L = Layout<D, NB>;
   constexpr int C = L::C;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t sK = sbase + L::OFF_K, sQ = sbase + L::OFF_Q, sV = sbase + L::OFF_V,
-                 sUG = sbase + L::OFF_UG, sW0 = sbase + L::OFF_W0;
+  const uint32_t sK = sbase + L::OFF_K, sQ = sbase + L::OFF_Q, sVG = sbase + L::OFF_VG,
+                 sW0 = sbase + L::OFF_W0;
   // scan arrays of buffer i: eta, L (chunk-local log decay), Gamma = exp(L), exp(L_C - L),
   // cF16 = eta exp(L_{r16} - L), cT16 = exp(L - L_{r16})
   float* f_scan = reinterpret_cast<float*>(smem + L::OFF_F);
@@ -113,35 +113,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(k_full[i]), 1);
-      mbar_init(BAR(k_free[i]), 1);
+      mbar_init(BAR(k_free[i]), 2);  // both MMA issuers read K
+      mbar_init(BAR(q_full[i]), 1);
+      mbar_init(BAR(q_free[i]), 1);
       mbar_init(BAR(v_full[i]), 1);
-      mbar_init(BAR(v_free[i]), 1);
-    }
-    mbar_init(BAR(q_full), 1);
-    mbar_init(BAR(q_free), 1);
-    mbar_init(BAR(z_full), 1);
-    mbar_init(BAR(g_ready), kEpiWarps);
-    mbar_init(BAR(y_full), 1);
-    mbar_init(BAR(y_scaled), kEpiWarps);
-    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(y_full[i]), 1);
+      mbar_init(BAR(y_scaled[i]), kEpiWarps);
       mbar_init(BAR(p_full[i]), 1);
       mbar_init(BAR(s_ready[i]), kEpiWarps);
       mbar_init(BAR(s_done[i]), 1);
-    }
-    mbar_init(BAR(zq_full), 1);
-    mbar_init(BAR(y_free), kEpiWarps);
-    mbar_init(BAR(w_full), 1);
-    mbar_init(BAR(w0_ready), kEpiWarps);
-    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(zq_full[i]), 1);
+      mbar_init(BAR(y_free[i]), kEpiWarps);
       mbar_init(BAR(scan_full[i]), 1);
       mbar_init(BAR(scan_free[i]), kEpiWarps);
+      mbar_init(BAR(bg_full[i]), 1);
+      mbar_init(BAR(g_read[i]), 1);
     }
-    mbar_init(BAR(bg_full[0]), 1);
-    mbar_init(BAR(bg_full[1]), 1);
-    mbar_init(BAR(o_ready), kEpiWarps);
+    mbar_init(BAR(z_full), 1);
+    mbar_init(BAR(g_ready), kEpiWarps);
+    mbar_init(BAR(w_full), 1);
+    mbar_init(BAR(w0_ready), kEpiWarps);
+    mbar_init(BAR(g_done), 1);
     mbar_init(BAR(st_free), 1);
-    mbar_init(BAR(g_read[0]), 1);
-    mbar_init(BAR(g_read[1]), 1);
     bars->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -161,7 +154,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int qk = 0;  // Q half loads issued
       // beta, gamma of chunk c go to buffer c & 1 on bg_full[c & 1] (phase (c >> 1) & 1),
       // one chunk ahead of the scan that reads them
       auto load_bg = [&](int cc) {
@@ -173,62 +165,58 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.gamma) bulk_g2s(bg + C * 4, p.gamma + r0, C * 4, bar);
       };
       load_bg(0);
+      mbar_arrive_expect_tx(BAR(v_full[0]), L::V_TX);
+      tma_load_2d(sVG, &tmV, BAR(v_full[0]), NV * slice, bh * p.T);
       for (int c = 0; c < NC; ++c) {
         const int row0 = bh * p.T + c * C;
-        // V slice of chunk c into buffer c & 1, free once chunk c-2's last S G MMA is done
-        const int vb = c & 1;
-        if (c >= 2 && !mbar_wait(BAR(v_free[vb]), ((c - 2) >> 1) & 1, ab)) goto done_prod;
-        // with G saved, the bulk store of chunk c-2's G (in place over its V) must have read it
-        if (c >= 2 && p.save_g && !mbar_wait(BAR(g_read[vb]), ((c - 2) >> 1) & 1, ab))
-          goto done_prod;
-        mbar_arrive_expect_tx(BAR(v_full[vb]), L::V_TX);
-        tma_load_2d(sV + vb * C * 128, &tmV, BAR(v_full[vb]), NV * slice, row0);
+        // K halves of chunk c, each free once its last reader of chunk c-1 is done
         for (int h = 0; h < NB; ++h) {
-          // K half h of chunk c, free once its last reader of chunk c-1 is done
           if (c > 0 && !mbar_wait(BAR(k_free[h]), (c - 1) & 1, ab)) goto done_prod;
           mbar_arrive_expect_tx(BAR(k_full[h]), L::KH);
 #pragma unroll
           for (int kp = 0; kp < L::KP; ++kp)
             tma_load_2d(sK + (h * L::KP + kp) * PANEL128, &tmK, BAR(k_full[h]), 64 * kp,
                         row0 + 128 * h);
-          if (qk > 0 && !mbar_wait(BAR(q_free), (qk - 1) & 1, ab)) goto done_prod;
-          mbar_arrive_expect_tx(BAR(q_full), L::KH);
+        }
+        // both Q halves of chunk c
+        for (int h = 0; h < NB; ++h) {
+          if (c > 0 && !mbar_wait(BAR(q_free[h]), (c - 1) & 1, ab)) goto done_prod;
+          mbar_arrive_expect_tx(BAR(q_full[h]), L::KH);
 #pragma unroll
           for (int kp = 0; kp < L::KP; ++kp)
-            tma_load_2d(sQ + kp * PANEL128, &tmQ, BAR(q_full), 64 * kp, row0 + 128 * h);
-          ++qk;
-          if (h == 0 && c + 1 < NC) {
-            // buffer (c+1)&1 was last read by the scan of chunk c-1
-            if (c > 0 && !mbar_wait(BAR(scan_full[(c - 1) & 1]), ((c - 1) >> 1) & 1, ab))
-              goto done_prod;
-            load_bg(c + 1);
-          }
+            tma_load_2d(sQ + (h * L::KP + kp) * PANEL128, &tmQ, BAR(q_full[h]), 64 * kp,
+                        row0 + 128 * h);
+        }
+        if (c + 1 < NC) {
+          // buffer (c+1)&1 of beta/gamma was last read by the scan of chunk c-1
+          if (c > 0 && !mbar_wait(BAR(scan_full[(c - 1) & 1]), ((c - 1) >> 1) & 1, ab))
+            goto done_prod;
+          load_bg(c + 1);
+          // V of chunk c+1 into the buffer holding chunk c's -u G, once the transition MMA has
+          // read it (and, with G saved, once the bulk store of chunk c-1's G there has read it)
+          const int vb = (c + 1) & 1;
+          if (!mbar_wait(BAR(w_full), c & 1, ab)) goto done_prod;
+          if (c >= 1 && p.save_g && !mbar_wait(BAR(g_read[vb]), ((c - 1) >> 1) & 1, ab))
+            goto done_prod;
+          mbar_arrive_expect_tx(BAR(v_full[vb]), L::V_TX);
+          tma_load_2d(sVG + vb * C * 128, &tmV, BAR(v_full[vb]), NV * slice, row0 + C);
         }
       }
     done_prod:;
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------ state-chain MMAs: Z, transition
     if (lane == 0) {
       const uint32_t idZ = idesc_bf16(128, NV, 0, 1);   // K-major A, MN-major B
-      const uint32_t idP = idesc_bf16(128, 128, 0, 0);  // K-major A and B
       const uint32_t idW = idesc_bf16(128, NV, 1, 1);   // MN-major A and B
       const uint32_t lboKt = D == 128 ? PANEL128 : 0;  // second 64-row block of K^T
-      int kq = 0;
-      int sd0 = 0, sd1 = 0;  // S G MMAs committed on s_done[x]
-      int sr0 = 0, sr1 = 0;  // s_ready[x] phases consumed
-      // a score buffer is rewritten only after the S G MMA that read it last has completed
-      auto buf_free = [&](int x) -> bool {
-        const int n = x ? sd1 : sd0;
-        return n == 0 || mbar_wait(BAR(s_done[x]), (n - 1) & 1, ab);
-      };
       for (int c = 0; c < NC; ++c) {
-        const uint32_t sVc = sV + (c & 1) * C * 128;
-        if (!mbar_wait(BAR(w0_ready), c & 1, ab)) break;
-        bool ok = true;
-        for (int b = 0; b < NB; ++b)
-          if (!mbar_wait(BAR(k_full[b]), c & 1, ab)) { ok = false; break; }
-        if (!ok || (NB == 2 && !buf_free(1))) break;  // Z columns = score buffer B
+        const uint32_t sUG = sVG + ((c + 1) & 1) * C * 128;
+        bool ok = mbar_wait(BAR(w0_ready), c & 1, ab);
+        for (int b = 0; b < NB && ok; ++b) ok = mbar_wait(BAR(k_full[b]), c & 1, ab);
+        // with two blocks the Z columns are score buffer B, read last by S_00 G_0 of chunk c-1
+        if (ok && NB == 2 && c > 0) ok = mbar_wait(BAR(s_done[1]), (c - 1) & 1, ab);
+        if (!ok) break;
         tc_fence_after();
         // Z_b = K_b W0
         for (int b = 0; b < NB; ++b) {
@@ -239,64 +227,97 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
         }
         mma_commit(BAR(z_full));
+        if (!mbar_wait(BAR(g_ready), c & 1, ab)) break;
+        tc_fence_after();
+        // W += K^T (u * -G), W already scaled by Gamma_C
+        for (int j = 0; j < C / 16; ++j)
+          mma_bf16_ss(tmem + L::T_W, sdesc_sw128(sK + (j / 8) * L::KH + (j % 8) * 2048, lboKt, 1024),
+                      sdesc_sw128(sUG + j * 2048, 0, 1024), idW, 1);
+        mma_commit(BAR(w_full));
+        for (int b = 0; b < NB; ++b) mma_commit(BAR(k_free[b]));
+      }
+    }
+  } else if (warp == 11) {
+    // ------------------------------------------------- query-side MMAs: Y, scores, S G
+    // Score blocks of a chunk: with two query halves (1,0) goes to buffer A first, (0,0) to B
+    // (the Z columns) once G is formed, (1,1) to A once S_10 G_0 has read it; so the Z columns
+    // are free for the next chunk as soon as S_00 G_0 is done. With one half, (0,0) uses A.
+    if (lane == 0) {
+      const uint32_t idZ = idesc_bf16(128, NV, 0, 1);   // K-major A, MN-major B
+      const uint32_t idP = idesc_bf16(128, 128, 0, 0);  // K-major A and B
+      int sdA = 0, srA = 0;                             // buffer A: S G commits, s_ready phases
+      auto issue_y = [&](int h) {
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j)
+          mma_bf16_ss(tmem + L::T_Y + NV * h,
+                      sdesc_sw128(sQ + (h * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                      sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
+        mma_commit(BAR(y_full[h]));
+      };
+      auto issue_p = [&](int h, int b, int x) {
+#pragma unroll
+        for (int j = 0; j < D / 16; ++j)
+          mma_bf16_ss(tmem + L::tbuf(x),
+                      sdesc_sw128(sQ + (h * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                      sdesc_sw128(sK + (b * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
+                      idP, j > 0);
+        mma_commit(BAR(p_full[x]));
+      };
+      auto wait_a_free = [&]() -> bool {
+        return sdA == 0 || mbar_wait(BAR(s_done[0]), (sdA - 1) & 1, ab);
+      };
+      // Zq_h += (-S_hb) G_b; S (bf16) in TMEM, 32 packed columns per warpgroup
+      auto issue_sg = [&](int h, int b, int x, uint32_t sG, int ready_phase) -> bool {
+        if (!mbar_wait(BAR(s_ready[x]), ready_phase & 1, ab)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          mma_bf16_ts(tmem + L::T_Y + NV * h, tmem + L::tbuf(x) + packed_col<64>(j),
+                      sdesc_sw128(sG + b * PANEL128 + j * 2048, 0, 1024), idZ, 1);
+        mma_commit(BAR(s_done[x]));
+        if (x == 0) ++sdA;
+        return true;
+      };
+      for (int c = 0; c < NC; ++c) {
+        const uint32_t sG = sVG + (c & 1) * C * 128;
+        // Y_h = Q_h W0 with this chunk's bf16 state copy
+        bool ok = mbar_wait(BAR(w0_ready), c & 1, ab);
         for (int h = 0; h < NB && ok; ++h) {
-          const int k0 = h * (h + 1) / 2;  // first score block of query half h
-          if (!mbar_wait(BAR(q_full), kq & 1, ab)) { ok = false; break; }
-          ++kq;
-          if (h == 0 && c > 0 && !mbar_wait(BAR(y_free), (c - 1) & 1, ab)) { ok = false; break; }
-          tc_fence_after();
-          // Y_h = Q_h W0
-#pragma unroll
-          for (int j = 0; j < D / 16; ++j)
-            mma_bf16_ss(tmem + L::T_Y + NV * h,
-                        sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                        sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
-          mma_commit(BAR(y_full));
-          // all score blocks of this query half first, so the epilogue never waits for one
-          for (int b = 0; b <= h; ++b) {
-            const int x = L::buf(k0 + b);
-            if (!buf_free(x)) { ok = false; break; }
+          ok = mbar_wait(BAR(q_full[h]), c & 1, ab) &&
+               (c == 0 || mbar_wait(BAR(y_free[h]), (c - 1) & 1, ab));
+          if (ok) {
             tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < D / 16; ++j)
-              mma_bf16_ss(tmem + L::tbuf(x),
-                          sdesc_sw128(sQ + (j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                          sdesc_sw128(sK + (b * L::KP + j / 4) * PANEL128 + (j % 4) * 32, 16, 1024),
-                          idP, j > 0);
-            mma_commit(BAR(p_full[x]));
-            if (h == 0 && b == 0) {
-              // state transition W += K^T (u * -G), W already scaled by Gamma_C
-              if (!mbar_wait(BAR(g_ready), c & 1, ab)) { ok = false; break; }
-              tc_fence_after();
-              for (int j = 0; j < C / 16; ++j)
-                mma_bf16_ss(tmem + L::T_W,
-                            sdesc_sw128(sK + (j / 8) * L::KH + (j % 8) * 2048, lboKt, 1024),
-                            sdesc_sw128(sUG + j * 2048, 0, 1024), idW, 1);
-              mma_commit(BAR(w_full));
-            }
-            if (b == h) mma_commit(BAR(q_free));
-            // K half b: its last reader is this block in the last query half (and W)
-            if (h == NB - 1) mma_commit(BAR(k_free[b]));
+            issue_y(h);
           }
-          if (!ok) break;
-          for (int b = 0; b <= h; ++b) {
-            const int x = L::buf(k0 + b);
-            const int n = x ? sr1++ : sr0++;
-            if (!mbar_wait(BAR(s_ready[x]), n & 1, ab)) { ok = false; break; }
-            if (b == 0 && !mbar_wait(BAR(y_scaled), (c * NB + h) & 1, ab)) { ok = false; break; }
-            tc_fence_after();
-            // Zq_h += (-S_hb) G_b; S (bf16) in TMEM, 32 packed columns per warpgroup
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              mma_bf16_ts(tmem + L::T_Y + NV * h, tmem + L::tbuf(x) + packed_col<64>(j),
-                          sdesc_sw128(sVc + b * PANEL128 + j * 2048, 0, 1024), idZ, 1);
-            mma_commit(BAR(s_done[x]));
-            if (x) ++sd1; else ++sd0;
-          }
-          if (ok) mma_commit(BAR(zq_full));
         }
-        if (!ok) break;
-        mma_commit(BAR(v_free[c & 1]));
+        for (int b = 0; b < NB && ok; ++b) ok = mbar_wait(BAR(k_full[b]), c & 1, ab);
+        if (!ok || !wait_a_free()) break;
+        tc_fence_after();
+        if constexpr (NB == 1) {
+          issue_p(0, 0, 0);
+          mma_commit(BAR(q_free[0]));
+          mma_commit(BAR(k_free[0]));
+          if (!mbar_wait(BAR(y_scaled[0]), c & 1, ab) || !issue_sg(0, 0, 0, sG, srA++)) break;
+          mma_commit(BAR(zq_full[0]));
+        } else {
+          issue_p(1, 0, 0);                                    // (1,0) -> A
+          if (!mbar_wait(BAR(g_ready), c & 1, ab)) break;      // Z columns free of Z
+          tc_fence_after();
+          issue_p(0, 0, 1);                                    // (0,0) -> B
+          mma_commit(BAR(q_free[0]));
+          mma_commit(BAR(k_free[0]));
+          if (!mbar_wait(BAR(y_scaled[1]), c & 1, ab) || !issue_sg(1, 0, 0, sG, srA++)) break;
+          if (!wait_a_free()) break;
+          tc_fence_after();
+          issue_p(1, 1, 0);                                    // (1,1) -> A
+          mma_commit(BAR(q_free[1]));
+          mma_commit(BAR(k_free[1]));
+          if (!mbar_wait(BAR(y_scaled[0]), c & 1, ab) || !issue_sg(0, 0, 1, sG, c)) break;
+          mma_commit(BAR(zq_full[0]));
+          if (!issue_sg(1, 1, 0, sG, srA++)) break;
+          mma_commit(BAR(zq_full[1]));
+        }
+        mma_commit(BAR(g_done));  // G of chunk c (in its V buffer) fully read
       }
     }
   } else if (warp == 10) {
@@ -348,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int puse0 = 0, puse1 = 0;  // score blocks consumed per buffer
     for (int c = 0; c < NC && ok; ++c) {
       const size_t tok0 = (size_t)bh * p.T + (size_t)c * C;
+      const uint32_t sG = sVG + (c & 1) * C * 128, sUG = sVG + ((c + 1) & 1) * C * 128;
       // -------- this chunk's scan arrays (computed by warp 10)
       if (!mbar_wait(BAR(scan_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
       const float* f_eta = f_scan + (c & 1) * 6 * 256;
@@ -356,11 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* f_eLC = f_eta + 768;
       const float* f_cF16 = f_eta + 1024;
 
-      // -------- train view: G = a(Z) act'(Z) in place over V, and -u*G
-      const uint32_t sVc = sV + (c & 1) * C * 128;
+      // -------- train view: G = a(Z) act'(Z) in place over V, -u G into the other buffer
       if (ew == 0 && c > 0) {
-        // the previous chunk's bulk stores (O from the -u*G buffer, the state checkpoint from
-        // the bf16 state copy) must have read their sources before those are rewritten
+        // the previous chunk's bulk stores (the state checkpoint from the bf16 state copy, G)
+        // must have read their sources before those are rewritten
         if (lane == 0) {
           bulk_wait_read0();
           mbar_arrive(BAR(st_free));
@@ -369,6 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       if (c > 0 && !mbar_wait(BAR(st_free), (c - 1) & 1, ab)) { ok = false; break; }
+      // -u G goes over chunk c-1's G, which its last S G MMA must have read
+      if (c > 0 && !mbar_wait(BAR(g_done), (c - 1) & 1, ab)) { ok = false; break; }
       if (!mbar_wait(BAR(v_full[c & 1]), (c >> 1) & 1, ab)) { ok = false; break; }
       if (!mbar_wait(BAR(z_full), c & 1, ab)) { ok = false; break; }
       __syncwarp();
@@ -387,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < ZB; ++i) {
             float v[32];
             const int row = 128 * (b0 + i) + lrow;
-            ld_row32(sVc, row, 4 * g, v);
+            ld_row32(sG, row, 4 * g, v);
             const float un = -f_eta[row] * f_eLC[row];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -396,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               v[j] = gg;
               z[i][j] = un * gg;
             }
-            st_row32(sVc, row, 4 * g, v);
+            st_row32(sG, row, 4 * g, v);
             st_row32(sUG, row, 4 * g, z[i]);
           }
         }
@@ -411,132 +434,113 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = mbar_wait(BAR(g_ready), c & 1, ab);
           if (ok) {
             for (int b = 0; b < NB; ++b)
-              tma_store_2d(&tmG, sVc + b * PANEL128, NV * slice, (int)tok0 + 128 * b);
+              tma_store_2d(&tmG, sG + b * PANEL128, NV * slice, (int)tok0 + 128 * b);
             bulk_commit();
           }
         }
         if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
       }
 
-      for (int h = 0; h < NB && ok; ++h) {
-        const int k0 = h * (h + 1) / 2;
-        const int srow = 128 * h + lrow;  // chunk-local query index of this thread
-        // Y_h *= Gamma_s
-        if (!mbar_wait(BAR(y_full), (c * NB + h) & 1, ab)) { ok = false; break; }
+      // -------- state copy for the next chunk: after the transition MMA and after the last MMA
+      // that reads the current bf16 copy (Y of the last query half). The fp32 state goes back
+      // into TMEM already decayed by the next chunk's Gamma_C.
+      {
+        const bool more = c + 1 < NC;
+        if (!mbar_wait(BAR(w_full), c & 1, ab) || !mbar_wait(BAR(y_full[NB - 1]), c & 1, ab) ||
+            (more && !mbar_wait(BAR(scan_full[(c + 1) & 1]), ((c + 1) >> 1) & 1, ab))) {
+          ok = false;
+          break;
+        }
         __syncwarp();
         tc_fence_after();
-        {
-          float y[32];
-          tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
+        if (w_rows) {
+          float w[32];
+          tmem_ld32(tmem + lane_off + L::T_W + 32 * g, w);
           tmem_wait_ld();
-          const float gs = f_gam[srow];
+          if (more) {
+            st_row32(sW0, lrow, 4 * g, w);
+            const float gnext = f_scan[((c + 1) & 1) * 6 * 256 + 512 + C - 1];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] *= gs;
-          tmem_st32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
-          tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(y_scaled));
-
-        if (h == NB - 1) {
-          // -------- state copy for the next chunk: after the transition MMA and after the
-          // last MMA that reads the current bf16 copy (Y of this block, complete above). The
-          // fp32 state goes back into TMEM already decayed by the next chunk's Gamma_C.
-          if (!mbar_wait(BAR(w_full), c & 1, ab)) { ok = false; break; }
-          const bool more = c + 1 < NC;
-          if (more && !mbar_wait(BAR(scan_full[(c + 1) & 1]), ((c + 1) >> 1) & 1, ab)) {
-            ok = false;
-            break;
+            for (int j = 0; j < 32; ++j) w[j] *= gnext;
+            tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
+            tmem_wait_st();
+          } else if (p.W_final) {
+            float4* dst = reinterpret_cast<float4*>(p.W_final + wofs);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              dst[k] = make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
           }
-          __syncwarp();
-          tc_fence_after();
-          if (w_rows) {
-            float w[32];
-            tmem_ld32(tmem + lane_off + L::T_W + 32 * g, w);
-            tmem_wait_ld();
-            if (more) {
-              st_row32(sW0, lrow, 4 * g, w);
-              const float gnext = f_scan[((c + 1) & 1) * 6 * 256 + 512 + C - 1];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) w[j] *= gnext;
-              tmem_st32(tmem + lane_off + L::T_W + 32 * g, w);
-              tmem_wait_st();
-            } else if (p.W_final) {
-              float4* dst = reinterpret_cast<float4*>(p.W_final + wofs);
-#pragma unroll
-              for (int k = 0; k < 8; ++k)
-                dst[k] = make_float4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-            }
-          }
-          fence_proxy_async_smem();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(w0_ready));
-          if (ew == 0 && c + 1 < NC && p.W_chunks) {
-            // checkpoint of the next chunk's start state, one bulk store of the bf16 copy
-            if (lane == 0) {
-              ok = mbar_wait(BAR(w0_ready), (c + 1) & 1, ab);
-              if (ok) {
-                tma_store_2d(&tmWc, sW0, NV * slice, (bh * NC + c + 1) * D);
-                bulk_commit();
-              }
-            }
-            if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
-          }
-        }
-
-        // -------- score blocks of this query half: S = -(Q K^T) * weights, bf16 in place
-        const float Ls = f_L[srow];
-        for (int b = 0; b <= h; ++b) {
-          const int x = L::buf(k0 + b);
-          const int pu = x ? puse1++ : puse0++;
-          if (!mbar_wait(BAR(p_full[x]), pu & 1, ab)) { ok = false; break; }
-          __syncwarp();
-          tc_fence_after();
-          const QWeights w{f_L, f_cF16, srow, 128 * b, Ls};
-          pack_in_place<64>(tmem + lane_off + L::tbuf(x), g, g + 1, q, b == h, w);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(s_ready[x]));
-        }
-        if (!ok) break;
-        if (h == NB - 1) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(BAR(scan_free[c & 1]));
-        }
-        // -------- O_h = act(Zq_h)
-        if (!mbar_wait(BAR(zq_full), (c * NB + h) & 1, ab)) { ok = false; break; }
-        __syncwarp();
-        tc_fence_after();
-        {
-          // staged in the -u*G buffer (free since the transition MMA completed), one bulk store
-          float o[32];
-          tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = act_f<ACT>(o[j]);
-          st_row32(sUG, srow, 4 * g, o);
         }
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(o_ready));
-        if (ew == 0) {
+        if (lane == 0) mbar_arrive(BAR(w0_ready));
+        if (ew == 0 && more && p.W_chunks) {
+          // checkpoint of the next chunk's start state, one bulk store of the bf16 copy
           if (lane == 0) {
-            ok = mbar_wait(BAR(o_ready), (c * NB + h) & 1, ab);
+            ok = mbar_wait(BAR(w0_ready), (c + 1) & 1, ab);
             if (ok) {
-              tma_store_2d(&tmO, sUG + h * PANEL128, NV * slice, (int)tok0 + 128 * h);
+              tma_store_2d(&tmWc, sW0, NV * slice, (bh * NC + c + 1) * D);
               bulk_commit();
             }
           }
           if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
         }
       }
+
+      // -------- Y_h *= Gamma_s for both query halves
+      for (int h = 0; h < NB; ++h) {
+        if (!mbar_wait(BAR(y_full[h]), c & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        float y[32];
+        tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
+        tmem_wait_ld();
+        const float gs = f_gam[128 * h + lrow];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] *= gs;
+        tmem_st32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(y_scaled[h]));
+      }
       if (!ok) break;
-      tc_fence_before();
+      // -------- score blocks S = -(Q K^T) * weights, bf16 in place, in the order the query-side
+      // issuer produces them: (1,0) in A, (0,0) in B, (1,1) in A; or (0,0) in A
+      for (int k = 0; k < (NB == 2 ? 3 : 1); ++k) {
+        const int h = NB == 2 ? (k == 1 ? 0 : 1) : 0, b = NB == 2 ? (k == 2 ? 1 : 0) : 0;
+        const int x = (NB == 2 && k == 1) ? 1 : 0;
+        const int pu = x ? puse1++ : puse0++;
+        if (!mbar_wait(BAR(p_full[x]), pu & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        const int srow = 128 * h + lrow;
+        const QWeights w{f_L, f_cF16, srow, 128 * b, f_L[srow]};
+        pack_in_place<64>(tmem + lane_off + L::tbuf(x), g, g + 1, q, b == h, w);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(s_ready[x]));
+      }
+      if (!ok) break;
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(y_free));
+      if (lane == 0) mbar_arrive(BAR(scan_free[c & 1]));
+      // -------- O_h = act(Zq_h), straight from registers to global memory
+      for (int h = 0; h < NB; ++h) {
+        if (!mbar_wait(BAR(zq_full[h]), c & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        float o[32];
+        tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = act_f<ACT>(o[j]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(y_free[h]));
+        st_global_bf16x32(p.O + (tok0 + 128 * h + lrow) * D + NV * slice + 32 * g, o);
+      }
     }
     if (ew == 0 && lane == 0) bulk_wait0();
   }
@@ -554,17 +558,16 @@ template <int D, int NB, int ACT, int LOSS>
 cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   using L = Layout<D, NB>;
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
-  CUtensorMap tk, tq, tv, to, twc, tg;
+  CUtensorMap tk, tq, tv, twc, tg;
   const uint64_t wrows = (uint64_t)a.B * a.H * (a.T / a.C) * D;
   if (!make_tmap_bf16(&tk, a.K, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tq, a.Q, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tv, a.V, D, rows, D, 64, L::C) ||
-      !make_tmap_bf16(&to, a.O, D, rows, D, 64, 128) ||
       (a.W_chunks && !make_tmap_bf16(&twc, a.W_chunks, D, wrows, D, 64, D)) ||
       (a.G_saved && !make_tmap_bf16(&tg, a.G_saved, D, rows, D, 64, 128)))
     return cudaErrorInvalidValue;
-  if (!a.W_chunks) twc = to;  // never used
-  if (!a.G_saved) tg = to;    // never used
+  if (!a.W_chunks) twc = tk;  // never used
+  if (!a.G_saved) tg = tk;    // never used
   FwdParams p{};
   p.BH = a.B * a.H;
   p.T = a.T;
@@ -583,7 +586,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   auto k = ttt_fwd_tc_kernel<D, NB, ACT, LOSS>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, to, twc, tg, p);
+  k<<<p.BH * p.nslice, kThreads, smem, s>>>(tk, tq, tv, twc, tg, p);
   count_launches(1);
   return cudaGetLastError();
 }
