@@ -546,12 +546,13 @@ struct DqL {
   static constexpr uint32_t SLOT = BLK > WSZ ? BLK : WSZ;  // W0, then G blocks
   static constexpr uint32_t OFF_DO = 0, OFF_GW = BLK, OFF_K = BLK + SLOT,
                             OFF_F = 2 * BLK + SLOT;
-  static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
+  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of the chunk
+  static constexpr uint32_t OFF_BAR = OFF_BG + 2 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t T_DQ = 0, T_DS = D;
 };
 enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_G_FULL, Q_K_FULL, Q_DS_FULL, Q_DP_READY, Q_DP_DONE,
-       Q_DQ_FULL, Q_SCAN, Q_ST, Q_NBARS };
+       Q_DQ_FULL, Q_SCAN, Q_ST, Q_BG, Q_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
@@ -573,7 +574,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int sb = blockIdx.x % NB;
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
-  const int counts[Q_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, kSmallEpi};
+  const int counts[Q_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1};
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmDO);
     tma_prefetch_desc(&tmW);
@@ -587,8 +588,13 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int tokc = bh * p.T + c * C;
   const int wrow = (bh * p.NC + c) * D;
 
+  float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   if (warp == 0) {
     if (lane == 0) {
+      // beta and gamma of the chunk first: the scan they feed gates the first epilogue steps
+      mbar_arrive_expect_tx(BAR(Q_BG), (p.gamma ? 2 : 1) * C * 4);
+      bulk_g2s(smem_u32(f_bg), p.beta + tokc, C * 4, BAR(Q_BG));
+      if (p.gamma) bulk_g2s(smem_u32(f_bg + C), p.gamma + tokc, C * 4, BAR(Q_BG));
       mbar_arrive_expect_tx(BAR(Q_LD0), L::BLK + L::WSZ);
       mbar_arrive_expect_tx(BAR(Q_K_FULL), L::BLK);
 #pragma unroll
@@ -661,8 +667,9 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
     const int s = 128 * sb + lrow;  // chunk-local query index
     do {
       if (ew == 0) {
-        chunk_scan_warp<C>(p.beta + tokc, p.gamma ? p.gamma + tokc : nullptr, p.lr_bias, f_eta,
-                           f_L, f_gam, f_eLC, f_cF16, f_cT16);
+        if (!mbar_wait(BAR(Q_BG), 0, ab)) break;
+        chunk_scan_warp<C>(f_bg, p.gamma ? f_bg + C : nullptr, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
+                           f_cF16, f_cT16);
         if (lane == 0) mbar_arrive(BAR(Q_SCAN));
       }
       if (!mbar_wait(BAR(Q_SCAN), 0, ab)) break;
@@ -731,12 +738,13 @@ struct DkL {
   static constexpr uint32_t WSZ = KP * D * 128;
   static constexpr uint32_t SLOT = BLK > WSZ ? BLK : WSZ;  // dW, then Q blocks, then W0
   static constexpr uint32_t OFF_G = 0, OFF_A = BLK, OFF_B = BLK + SLOT, OFF_F = 2 * BLK + SLOT;
-  static constexpr uint32_t OFF_BAR = OFF_F + 6 * 256 * 4;
+  static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of the chunk
+  static constexpr uint32_t OFF_BAR = OFF_BG + 2 * C * 4;
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t T_DK = 0, T_DS = D;
 };
 enum { K_LD0, K_H, K_H_SCALED, K_DO_FULL, K_Q_FULL, K_DS_FULL, K_DP_READY, K_DK_STEP,
-       K_DVW_FULL, K_DK_FULL, K_SCAN, K_ST, K_NBARS };
+       K_DVW_FULL, K_DK_FULL, K_SCAN, K_ST, K_BG, K_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
@@ -760,7 +768,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
   const bool mse = p.loss == 0;
-  const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1, kSmallEpi};
+  const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1, kSmallEpi, 1};
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmG);
     tma_prefetch_desc(&tmDW);
@@ -777,8 +785,13 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int wrow = (bh * p.NC + c) * D;
   const int nq = NB - rb;  // query blocks at or after this key block
 
+  float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   if (warp == 0) {
     if (lane == 0) {
+      // beta and gamma of the chunk first: the scan they feed gates the first epilogue steps
+      mbar_arrive_expect_tx(BAR(K_BG), (p.gamma ? 2 : 1) * C * 4);
+      bulk_g2s(smem_u32(f_bg), p.beta + tokc, C * 4, BAR(K_BG));
+      if (p.gamma) bulk_g2s(smem_u32(f_bg + C), p.gamma + tokc, C * 4, BAR(K_BG));
       mbar_arrive_expect_tx(BAR(K_LD0), L::BLK + L::WSZ);
 #pragma unroll
       for (int kp = 0; kp < L::KP; ++kp) {
@@ -871,8 +884,9 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
     const int r = 128 * rb + lrow;  // chunk-local key index
     do {
       if (ew == 0) {
-        chunk_scan_warp<C>(p.beta + tokc, p.gamma ? p.gamma + tokc : nullptr, p.lr_bias, f_eta,
-                           f_L, f_gam, f_eLC, f_cF16, f_cT16);
+        if (!mbar_wait(BAR(K_BG), 0, ab)) break;
+        chunk_scan_warp<C>(f_bg, p.gamma ? f_bg + C : nullptr, p.lr_bias, f_eta, f_L, f_gam, f_eLC,
+                           f_cF16, f_cT16);
         if (lane == 0) mbar_arrive(BAR(K_SCAN));
       }
       if (!mbar_wait(BAR(K_SCAN), 0, ab)) break;
