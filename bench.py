@@ -185,8 +185,8 @@ class Layer:
     def bwd(self):
         i = self.inp
         self.ttt.ttt_chunk_bwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
-                               self.Wc, self.G, i["dO"], i["dW_T"], self.dQ, self.dK, self.dV,
-                               self.dbeta, self.dW0, self.ws, self.nb)
+                               self.Wc, self.G, i["dO"], i["dW_T"], None, None, self.dQ, self.dK,
+                               self.dV, self.dbeta, self.dW0, None, self.ws, self.nb)
 
 
 def time_steps(layer, steps, warmup, sampler=None):

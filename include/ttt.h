@@ -105,14 +105,21 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
 /* Analytic backward of the layer for the objective J = <dO, O> + <dW_final, W_final>.
  *  in : Q, K, V, beta, gamma (nullable), W0, W_chunks (from ttt_chunk_fwd, required),
  *       G_saved (from ttt_chunk_fwd, nullable: rebuilt from W_chunks when NULL; kernels that
- *       rebuild G anyway may ignore it), dO, dW_final (nullable = 0)
- *  out: dQ, dK, dV, dbeta, dW0 (plain stores, not accumulated). If the caller shares W0
- *       across the batch it reduces dW0 over B itself. No gradient is returned for gamma. */
+ *       rebuild G anyway may ignore it), dO, dW_final (nullable = 0);
+ *       O and W_final (the forward's outputs) are read only for dgamma (then O is required,
+ *       and W_final too when dW_final is non-NULL).
+ *  out: dQ, dK, dV, dbeta, dW0 (plain stores, not accumulated); dgamma (nullable; requires
+ *       gamma) = dJ/dgamma. If the caller shares W0 across the batch it reduces dW0 over B.
+ * The decay gradient follows from L_s = sum_{t<=s} log gamma_t (chunk-local): with Zq the
+ * readout before the activation and dG the adjoint of G,
+ *     dJ/dL_s = dZq_s . Zq_s - g_s . dG_s  (+ <W_end, dW_end> on the chunk's last token)
+ *     dgamma_t = (1 / gamma_t) sum_{s >= t in the chunk} dJ/dL_s. */
 ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0,
                          const void* W_chunks, const void* G_saved, const void* dO,
-                         const float* dW_final, void* dQ, void* dK, void* dV, float* dbeta,
-                         float* dW0, void* workspace, size_t workspace_bytes, void* stream);
+                         const float* dW_final, const void* O, const float* W_final, void* dQ,
+                         void* dK, void* dV, float* dbeta, float* dW0, float* dgamma,
+                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* Backward without caller-provided scratch (no counterpart in the papers: a deployment aid).
  * Some callers cannot allocate device memory when they call the library: a host framework
@@ -134,8 +141,9 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
 ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                                  const float* beta, const float* gamma, const float* W0,
                                  const void* W_chunks, const void* G_saved, const void* dO,
-                                 const float* dW_final, void* dQ, void* dK, void* dV,
-                                 float* dbeta, float* dW0, void* stream);
+                                 const float* dW_final, const void* O, const float* W_final,
+                                 void* dQ, void* dK, void* dV, float* dbeta, float* dW0,
+                                 float* dgamma, void* stream);
 
 /* Workspace bytes of inplace_ttt_fwd; (size_t)-1 for invalid sizes. */
 size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C);

@@ -48,7 +48,7 @@ def _load():
         p = ctypes.c_void_p
         lib.ttt_oracle_fwd_f64.argtypes = [i] * 8 + [d] + [p] * 9 + [i]
         lib.ttt_oracle_fwd_f32.argtypes = [i] * 8 + [d] + [p] * 9 + [i]
-        lib.ttt_oracle_bwd_f64.argtypes = [i] * 8 + [d] + [p] * 13 + [i]
+        lib.ttt_oracle_bwd_f64.argtypes = [i] * 8 + [d] + [p] * 14 + [i]
         for fn in (lib.ttt_oracle_fwd_f64, lib.ttt_oracle_fwd_f32, lib.ttt_oracle_bwd_f64):
             fn.restype = i
         _lib = lib
@@ -97,7 +97,7 @@ def ttt_fwd(Q, K, V, beta, gamma, W0, *, C: int, loss: str = "mse", act: str = "
 def ttt_bwd(Q, K, V, beta, gamma, W0, dO, dW_T=None, *, C: int, loss: str = "mse",
             act: str = "id", lr_bias: float, nthreads: int = 0):
     """Reverse-mode of the per-token loop for J = <dO,O> + <dW_T,W_final> (fp64).
-    Returns dict dQ, dK, dV, dbeta, dW0."""
+    Returns dict dQ, dK, dV, dbeta, dW0, and dgamma when gamma is given."""
     lib = _load()
     dt = np.float64
     q, k, v = _np(Q, dt), _np(K, dt), _np(V, dt)
@@ -110,11 +110,13 @@ def ttt_bwd(Q, K, V, beta, gamma, W0, dO, dW_T=None, *, C: int, loss: str = "mse
     out = dict(dQ=np.empty((B, H, T, dk)), dK=np.empty((B, H, T, dk)),
                dV=np.empty((B, H, T, dv)), dbeta=np.empty((B, H, T)),
                dW0=np.empty((B, H, dk, dv)))
+    if g_ is not None:
+        out["dgamma"] = np.empty((B, H, T))
     used = lib.ttt_oracle_bwd_f64(B, H, T, dk, dv, C, LOSS[loss], ACT[act], float(lr_bias),
                                   _ptr(q), _ptr(k), _ptr(v), _ptr(b_), _ptr(g_), _ptr(w0),
                                   _ptr(do), _ptr(dwt), _ptr(out["dQ"]), _ptr(out["dK"]),
                                   _ptr(out["dV"]), _ptr(out["dbeta"]), _ptr(out["dW0"]),
-                                  int(nthreads))
+                                  _ptr(out.get("dgamma")), int(nthreads))
     if used < 0:
         raise ValueError("oracle rejected the shape")
     return out

@@ -34,7 +34,8 @@
 //   - the query view applies the same activation: O = act(Zq).
 //
 // The backward is reverse-mode differentiation of the same per-token loop
-// for J = <dO, O> + <dW_T, W_final>, returning dQ, dK, dV, dbeta and dW0.
+// for J = <dO, O> + <dW_T, W_final>, returning dQ, dK, dV, dbeta and dW0, and
+// on request the decay gradient dgamma_s = <adjoint of W_s, W_{s-1}>.
 //
 // Pins (tests/test_oracle_pins.py): brute-force evaluation of the chunk dual
 // form printed on the page, the C = 1 delta rule and decayed Hebbian closed
@@ -132,9 +133,11 @@ void fwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
 template <typename R, typename In>
 void bwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* beta,
               const In* gamma, const In* w_init, const In* dO, const In* dW_T,
-              R* dq, R* dk_, R* dv_, R* dbeta, R* dw0) {
+              R* dq, R* dk_, R* dv_, R* dbeta, R* dw0, R* dgamma) {
   const int dk = sh.dk, dv = sh.dv, C = sh.C, NC = sh.T / sh.C;
   const size_t WS = (size_t)dk * dv;
+  // with dgamma, the state before every token of the chunk being swept (W_{s-1})
+  std::vector<R> Wprev(dgamma ? (size_t)C * WS : 0);
   // Forward: keep only the chunk-start weights.
   std::vector<R> Wc((size_t)NC * WS), W(WS), z(dv), g(dv);
   for (size_t e = 0; e < WS; ++e) W[e] = R(w_init[e]);
@@ -169,6 +172,7 @@ void bwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
       train_view<R, In>(sh, k + t * dk, v + t * dv, W0, zs, gs);
       const R eta = R(2) * sigmoid_(R(beta[t]) + R(sh.lr_bias));
       const R gam = gamma ? R(gamma[t]) : R(1);
+      if (dgamma) std::memcpy(Wprev.data() + (size_t)s * WS, Ws.data(), sizeof(R) * WS);
       for (int i = 0; i < dk; ++i) {
         const R eki = eta * R(k[t * dk + i]);
         R* wrow = Ws.data() + (size_t)i * dv;
@@ -218,6 +222,13 @@ void bwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
       }
       R deta = R(0);
       for (int j = 0; j < dv; ++j) deta -= kW[j] * gs[j];
+      // W_s = gam W_{s-1} - ...: dJ/dgam = <adjoint of W_s, W_{s-1}>
+      if (dgamma) {
+        const R* wp = Wprev.data() + (size_t)s * WS;
+        R acc = R(0);
+        for (size_t e = 0; e < WS; ++e) acc += Wh[e] * wp[e];
+        dgamma[t] = acc;
+      }
       for (size_t e = 0; e < WS; ++e) Wh[e] *= gam;
       // g = a * act'(z),  a = act(z) - v (MSE) or -v (IP),  z = k W0
       for (int j = 0; j < dv; ++j) {
@@ -299,11 +310,13 @@ int ttt_oracle_fwd_f32(int B, int H, int T, int dk, int dv, int C, int loss, int
 }
 
 // Backward, fp64: reverse-mode of the per-token loop for J = <dO, O> + <dW_T, W_final>.
-// dW_T may be NULL (zero). Outputs dQ,dK [B,H,T,dk], dV [B,H,T,dv], dbeta [B,H,T], dW0 [B,H,dk,dv].
+// dW_T may be NULL (zero). Outputs dQ,dK [B,H,T,dk], dV [B,H,T,dv], dbeta [B,H,T], dW0 [B,H,dk,dv],
+// and dgamma [B,H,T] when both gamma and dgamma are non-NULL.
 int ttt_oracle_bwd_f64(int B, int H, int T, int dk, int dv, int C, int loss, int act, double lr_bias,
                        const double* Q, const double* K, const double* V, const double* beta,
                        const double* gamma, const double* W0, const double* dO, const double* dW_T,
-                       double* dQ, double* dK, double* dV, double* dbeta, double* dW0, int nthreads) {
+                       double* dQ, double* dK, double* dV, double* dbeta, double* dW0,
+                       double* dgamma, int nthreads) {
   if (B <= 0 || H <= 0 || T <= 0 || dk <= 0 || dv <= 0 || C <= 0 || T % C) return -1;
   Shape sh{B, H, T, dk, dv, C, loss, act, lr_bias};
   const int used = set_threads(nthreads);
@@ -314,7 +327,8 @@ int ttt_oracle_bwd_f64(int B, int H, int T, int dk, int dv, int C, int loss, int
     bwd_head<double, double>(sh, Q + bh * tk, K + bh * tk, V + bh * tv, beta + (size_t)bh * T,
                              gamma ? gamma + (size_t)bh * T : nullptr, W0 + bh * ws, dO + bh * tv,
                              dW_T ? dW_T + bh * ws : nullptr, dQ + bh * tk, dK + bh * tk,
-                             dV + bh * tv, dbeta + (size_t)bh * T, dW0 + bh * ws);
+                             dV + bh * tv, dbeta + (size_t)bh * T, dW0 + bh * ws,
+                             gamma && dgamma ? dgamma + (size_t)bh * T : nullptr);
   }
   return used;
 }

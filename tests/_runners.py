@@ -38,8 +38,9 @@ def run_fwd(cfg, inp, save_g=True):
     return dict(O=O, W_final=Wf, W_chunks=Wc, G=G)
 
 
-def run_bwd(cfg, inp, W_chunks, G=None):
-    """The backward; G (from run_fwd) is passed as G_saved, else the library rebuilds it."""
+def run_bwd(cfg, inp, W_chunks, G=None, fwd=None):
+    """The backward; G (from run_fwd) is passed as G_saved, else the library rebuilds it. With
+    `fwd` (run_fwd's outputs) and a decay, the decay gradient is asked for too."""
     c = abi_config(cfg)
     sd = synth.storage_dtype(cfg)
     B, H, T, dk, dv = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv
@@ -48,11 +49,15 @@ def run_bwd(cfg, inp, W_chunks, G=None):
                dV=torch.empty((B, H, T, dv), device="cuda", dtype=sd),
                dbeta=torch.empty((B, H, T), device="cuda", dtype=torch.float32),
                dW0=torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32))
+    want_dg = fwd is not None and inp["gamma"] is not None
+    if want_dg:
+        out["dgamma"] = torch.empty((B, H, T), device="cuda", dtype=torch.float32)
     n = ttt.ttt_workspace_bytes(c, 2 if G is not None else 1)
     ws = torch.empty(max(n, 16), device="cuda", dtype=torch.uint8)
     ttt.ttt_chunk_bwd(c, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], inp["W0"],
-                      W_chunks, G, inp["dO"], inp["dW_T"], out["dQ"], out["dK"], out["dV"],
-                      out["dbeta"], out["dW0"], ws, n)
+                      W_chunks, G, inp["dO"], inp["dW_T"], fwd["O"] if want_dg else None,
+                      fwd["W_final"] if want_dg else None, out["dQ"], out["dK"], out["dV"],
+                      out["dbeta"], out["dW0"], out.get("dgamma"), ws, n)
     torch.cuda.synchronize()
     assert ttt.ttt_get_device_error() == ttt.OK
     return out

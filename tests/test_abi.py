@@ -86,13 +86,23 @@ def test_fwd_argument_errors_before_launch():
 def test_bwd_requires_chunk_states_and_workspace():
     cfg = _cfg()
     A = 4096
-    base = [A, A, A, A, None, A, A, None, A, None, A, A, A, A, A]  # G_saved NULL
+    # Q K V beta gamma W0 W_chunks G_saved dO dW_final O W_final dQ dK dV dbeta dW0 dgamma
+    base = [A, A, A, A, None, A, A, None, A, None, None, None, A, A, A, A, A, None]
     args = list(base)
     args[6] = None  # W_chunks
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *args, None, 0, None) == ttt.ERR_INVALID_ARG
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *base, None, 0, None) == ttt.ERR_WORKSPACE
     need = ttt.ttt_workspace_bytes(cfg, 1)
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *base, A, need - 1, None) == ttt.ERR_WORKSPACE
+    # the decay gradient needs gamma and the forward's O (and W_final with dW_final)
+    dg = list(base)
+    dg[17] = A  # dgamma without gamma
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *dg, A, need, None) == ttt.ERR_INVALID_ARG
+    dg[4] = A   # gamma, but no O
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *dg, A, need, None) == ttt.ERR_INVALID_ARG
+    dg[10] = A  # O; dW_final set without W_final
+    dg[9] = A
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *dg, A, need, None) == ttt.ERR_INVALID_ARG
 
 
 def test_inplace_argument_errors():

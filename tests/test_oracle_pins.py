@@ -263,8 +263,8 @@ def test_backward_matches_finite_differences(loss, act):
     kw = dict(C=C, loss=loss, act=act, lr_bias=-0.4)
     g = oracle.ttt_bwd(Q, K, V, beta, gamma, W0, dO, dWT, **kw)
     h = 1e-6
-    args = dict(Q=Q, K=K, V=V, beta=beta, W0=W0)
-    names = dict(Q="dQ", K="dK", V="dV", beta="dbeta", W0="dW0")
+    args = dict(Q=Q, K=K, V=V, beta=beta, gamma=gamma, W0=W0)
+    names = dict(Q="dQ", K="dK", V="dV", beta="dbeta", gamma="dgamma", W0="dW0")
     for name, x in args.items():
         fd = np.zeros_like(x)
         for idx in np.ndindex(x.shape):

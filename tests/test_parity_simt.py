@@ -46,9 +46,9 @@ def test_fp32_forward_backward(shape, loss, act, decay):
     ref["G"] = reference_g(cfg, inp, ref["W_chunks"])
     for k in ("O", "W_final", "W_chunks", "G"):
         assert rel_err(got[k], ref[k]) <= F32_TOL, k
-    g = run_bwd(cfg, inp, got["W_chunks"], got["G"] if decay else None)
+    g = run_bwd(cfg, inp, got["W_chunks"], got["G"] if decay else None, fwd=got)
     r = oracle_bwd(cfg, inp)
-    for k in ("dQ", "dK", "dV", "dbeta", "dW0"):
+    for k in ("dQ", "dK", "dV", "dbeta", "dW0") + (("dgamma",) if decay else ()):
         assert rel_err(g[k], r[k]) <= F32_TOL, k
 
 
@@ -61,7 +61,7 @@ def test_bf16_shapes_outside_the_tensor_core_envelope(loss, act):
     ref = oracle_fwd(cfg, inp)
     for k in ("O", "W_final"):
         assert rel_err(got[k], ref[k]) <= BF16_TOL, k
-    g = run_bwd(cfg, inp, got["W_chunks"])
+    g = run_bwd(cfg, inp, got["W_chunks"], fwd=got)
     r = oracle_bwd(cfg, inp)
-    for k in ("dQ", "dK", "dV", "dbeta", "dW0"):
+    for k in ("dQ", "dK", "dV", "dbeta", "dW0") + (("dgamma",) if inp["gamma"] is not None else ()):
         assert rel_err(g[k], r[k]) <= BF16_TOL, k

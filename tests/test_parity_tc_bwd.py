@@ -32,9 +32,9 @@ def test_tc_backward_small(shape, loss, decay, saved_g):
     inp = synth.ttt_inputs(cfg, device="cuda", seed=5 * T + d)
     inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(9))
     fwd = run_fwd(cfg, inp, save_g=saved_g)
-    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd=fwd)
     ref = oracle_bwd(cfg, inp)
-    for k in GRADS:
+    for k in GRADS + (("dgamma",) if decay else ()):
         assert rel_err(got[k], ref[k]) <= TOL, (k, rel_err(got[k], ref[k]))
 
 
@@ -42,11 +42,11 @@ def test_tc_backward_full_size_sampled_heads():
     cfg = synth.TRAIN_1P45B
     inp = synth.ttt_inputs(cfg, device="cuda")
     fwd = run_fwd(cfg, inp)
-    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd=fwd)
     rng = np.random.default_rng(44)
     heads = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(2)]
     sub = head_slice(inp, heads)
     ref = oracle_bwd(cfg.replace(B=1, H=len(heads)), sub)
-    for k in GRADS:
+    for k in GRADS + ("dgamma",):
         g = torch.stack([got[k][b, h] for b, h in heads]).unsqueeze(0)
         assert rel_err(g, ref[k]) <= TOL, (k, rel_err(g, ref[k]))

@@ -31,8 +31,9 @@ def noalloc_bwd(cfg, inp, W_chunks, G=None):
     st = ttt.lib.ttt_chunk_bwd_noalloc(
         ctypes.byref(c), inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(),
         inp["beta"].data_ptr(), inp["gamma"].data_ptr(), inp["W0"].data_ptr(), W_chunks.data_ptr(),
-        G.data_ptr() if G is not None else None, inp["dO"].data_ptr(), inp["dW_T"].data_ptr(), out["dQ"].data_ptr(), out["dK"].data_ptr(),
-        out["dV"].data_ptr(), out["dbeta"].data_ptr(), out["dW0"].data_ptr(),
+        G.data_ptr() if G is not None else None, inp["dO"].data_ptr(), inp["dW_T"].data_ptr(),
+        None, None, out["dQ"].data_ptr(), out["dK"].data_ptr(), out["dV"].data_ptr(),
+        out["dbeta"].data_ptr(), out["dW0"].data_ptr(), None,
         torch.cuda.current_stream().cuda_stream)
     assert st == ttt.OK, ttt.status_string(st)
     torch.cuda.synchronize()
@@ -57,10 +58,11 @@ def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
 def test_noalloc_backward_refuses_configs_beyond_its_scratch():
     big = abi_config(synth.TRAIN_1P45B)  # needs 32 MiB of scratch even with G passed in
     A = 4096  # never dereferenced: the size check comes first
-    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(big), A, A, A, A, A, A, A, A, A, None, A, A, A,
-                                       A, A, None)
+    # Q K V beta gamma W0 W_chunks G_saved dO dW_final O W_final dQ dK dV dbeta dW0 dgamma stream
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(big), A, A, A, A, A, A, A, A, A, None, None, None,
+                                       A, A, A, A, A, None, None)
     assert st == ttt.ERR_WORKSPACE
     silu = abi_config(synth.TRAIN_1P45B.replace(B=1, H=1, T=256, act="silu"))
-    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(silu), A, A, A, A, A, A, A, None, A, None, A,
-                                       A, A, A, A, None)
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(silu), A, A, A, A, A, A, A, None, A, None, None,
+                                       None, A, A, A, A, A, None, None)
     assert st == ttt.ERR_UNSUPPORTED

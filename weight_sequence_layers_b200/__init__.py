@@ -45,14 +45,14 @@ _cfgp = ctypes.POINTER(ttt_config)
 _SIGS = {
     "ttt_workspace_bytes": ([_cfgp, _i], _sz),
     "ttt_chunk_fwd": ([_cfgp] + [_p] * 11 + [_sz, _p], _i),
-    "ttt_chunk_bwd": ([_cfgp] + [_p] * 16 + [_sz, _p], _i),
+    "ttt_chunk_bwd": ([_cfgp] + [_p] * 19 + [_sz, _p], _i),
     "inplace_ttt_workspace_bytes": ([_i] * 4, _sz),
     "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 5 + [_sz, _p], _i),
     "ttt_get_device_error": ([_p], _i),
     "ttt_selftest_bounded_wait": ([_u, _p], _i),
     "ttt_status_string": ([_i], ctypes.c_char_p),
     "ttt_kernel_launches": ([], ctypes.c_ulonglong),
-    "ttt_chunk_bwd_noalloc": ([_cfgp] + [_p] * 15 + [_p], _i),
+    "ttt_chunk_bwd_noalloc": ([_cfgp] + [_p] * 18 + [_p], _i),
 }
 for _name, (_args, _ret) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -113,25 +113,27 @@ def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None,
     _check(st, "ttt_chunk_fwd")
 
 
-def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, dQ, dK, dV,
-                  dbeta, dW0, workspace=None, workspace_bytes=0, stream=None):
+def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, O, W_final, dQ,
+                  dK, dV, dbeta, dW0, dgamma, workspace=None, workspace_bytes=0, stream=None):
     st = _lib.ttt_chunk_bwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
                             _ptr(W0), _ptr(W_chunks), _ptr(G_saved), _ptr(dO), _ptr(dW_final),
-                            _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta), _ptr(dW0),
-                            _ptr(workspace), int(workspace_bytes), _stream(stream))
+                            _ptr(O), _ptr(W_final), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta),
+                            _ptr(dW0), _ptr(dgamma), _ptr(workspace), int(workspace_bytes),
+                            _stream(stream))
     _check(st, "ttt_chunk_bwd")
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
-def ttt_chunk_bwd_noalloc(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, dQ, dK,
-                          dV, dbeta, dW0, stream=None):
+def ttt_chunk_bwd_noalloc(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, O,
+                          W_final, dQ, dK, dV, dbeta, dW0, dgamma, stream=None):
     """ttt_chunk_bwd for callers that cannot allocate: scratch is the library's fixed array."""
     st = _lib.ttt_chunk_bwd_noalloc(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
                                     _ptr(gamma), _ptr(W0), _ptr(W_chunks), _ptr(G_saved),
-                                    _ptr(dO), _ptr(dW_final), _ptr(dQ), _ptr(dK), _ptr(dV),
-                                    _ptr(dbeta), _ptr(dW0), _stream(stream))
+                                    _ptr(dO), _ptr(dW_final), _ptr(O), _ptr(W_final), _ptr(dQ),
+                                    _ptr(dK), _ptr(dV), _ptr(dbeta), _ptr(dW0), _ptr(dgamma),
+                                    _stream(stream))
     _check(st, "ttt_chunk_bwd_noalloc")
 
 

@@ -212,14 +212,17 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
 ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0,
                          const void* W_chunks, const void* G_saved, const void* dO,
-                         const float* dW_final, void* dQ, void* dK, void* dV, float* dbeta,
-                         float* dW0, void* workspace, size_t workspace_bytes, void* stream) {
+                         const float* dW_final, const void* O, const float* W_final, void* dQ,
+                         void* dK, void* dV, float* dbeta, float* dW0, float* dgamma,
+                         void* workspace, size_t workspace_bytes, void* stream) {
   ttt_status st = check_config(cfg);
   if (st != TTT_OK) return st;
   if (!Q || !K || !V || !beta || !W0 || !W_chunks || !dO || !dQ || !dK || !dV || !dbeta || !dW0)
     return TTT_ERR_INVALID_ARG;
+  // the decay gradient needs the decay, the forward's O, and W_final when dW_final is set
+  if (dgamma && (!gamma || !O || (dW_final && !W_final))) return TTT_ERR_INVALID_ARG;
   const void* ptrs[] = {Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final,
-                        dQ, dK, dV, dbeta, dW0, workspace};
+                        O, W_final, dQ, dK, dV, dbeta, dW0, dgamma, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a = args_of(cfg);
@@ -236,6 +239,7 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
   a.G_saved = const_cast<void*>(G_saved);
   a.dO = dO; a.dW_final = dW_final; a.dQ = dQ; a.dK = dK; a.dV = dV; a.dbeta = dbeta;
   a.dW0 = dW0; a.ws = workspace; a.ws_bytes = workspace_bytes; a.err = err;
+  a.O_in = O; a.W_final_in = W_final; a.dgamma = dgamma;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launch_status(path == PATH_TC ? tc_bwd(a, s) : simt_bwd(a, s));
 }

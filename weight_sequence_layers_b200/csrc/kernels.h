@@ -17,6 +17,9 @@ struct LayerArgs {
   void* G_saved;  // nullable: G of every token [B, H, T, dv]
   const void* dO;
   const float* dW_final;
+  const void* O_in;        // forward output, read for dgamma
+  const float* W_final_in; // forward output, read for dgamma when dW_final is set
+  float* dgamma;           // nullable
   void *dQ, *dK, *dV;
   float *dbeta, *dW0;
   void* ws;

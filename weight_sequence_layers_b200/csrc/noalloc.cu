@@ -44,13 +44,16 @@ extern "C" ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q
                                             const void* V, const float* beta, const float* gamma,
                                             const float* W0, const void* W_chunks,
                                             const void* G_saved, const void* dO,
-                                            const float* dW_final, void* dQ, void* dK, void* dV,
-                                            float* dbeta, float* dW0, void* stream) {
+                                            const float* dW_final, const void* O,
+                                            const float* W_final, void* dQ, void* dK, void* dV,
+                                            float* dbeta, float* dW0, float* dgamma,
+                                            void* stream) {
   if (ttt_workspace_bytes(cfg, 1) == (size_t)-1) return TTT_ERR_INVALID_ARG;
   if (!Q || !K || !V || !beta || !W0 || !W_chunks || !dO || !dQ || !dK || !dV || !dbeta || !dW0)
     return TTT_ERR_INVALID_ARG;
+  if (dgamma && (!gamma || !O || (dW_final && !W_final))) return TTT_ERR_INVALID_ARG;
   const void* ptrs[] = {Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final,
-                        dQ, dK, dV, dbeta, dW0};
+                        O, W_final, dQ, dK, dV, dbeta, dW0, dgamma};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a{};
@@ -67,5 +70,6 @@ extern "C" ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q
   a.G_saved = const_cast<void*>(G_saved);
   a.dO = dO; a.dW_final = dW_final; a.dQ = dQ; a.dK = dK; a.dV = dV; a.dbeta = dbeta;
   a.dW0 = dW0; a.ws = scratch; a.ws_bytes = TTT_NOALLOC_SCRATCH_BYTES; a.err = err;
+  a.O_in = O; a.W_final_in = W_final; a.dgamma = dgamma;
   return tc_bwd(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }

@@ -957,6 +957,78 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   teardown(bars, tmem, 256);
 }
 
+// --------------------------------------------------------------------------------- dgamma
+// Decay gradient of one (batch, head, chunk), one thread per token. L_s = sum_{t<=s} log gamma_t
+// (chunk-local) enters through Gamma_s and the score weights of the readout and through u and
+// Gamma_C of the transition; with the identity readout (Zq = O, dZq = dO) and dG = -dV,
+//   dJ/dL_s = dO_s . O_s + g_s . dV_s  (+ <W_end, dW_end> on the chunk's last token)
+//   dgamma_t = (1 / gamma_t) sum_{s >= t in the chunk} dJ/dL_s.
+// W_end is the next chunk's saved start state (W_final after the last chunk) and dW_end the
+// adjoint the chain saved at the chunk end (dW_final after the last chunk).
+__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
+  return bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x) + bf16lo(a.y) * bf16lo(b.y) +
+         bf16hi(a.y) * bf16hi(b.y) + bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z) +
+         bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+}
+
+template <int D, int C>
+__global__ void __launch_bounds__(C)
+    bwd_dgamma_kernel(const __nv_bfloat16* O, const __nv_bfloat16* dO, const __nv_bfloat16* G,
+                      const __nv_bfloat16* dV, const __nv_bfloat16* Wc, const __nv_bfloat16* dWs,
+                      const float* W_final, const float* dW_final, const float* gamma,
+                      float* dgamma, int T, int NC) {
+  __shared__ float red[C / 32];
+  __shared__ float wsum;
+  const int c = blockIdx.x % NC, bh = blockIdx.x / NC;
+  const int s = threadIdx.x, lane = s & 31, wid = s >> 5;
+  const size_t row = (size_t)bh * T + (size_t)c * C + s;
+  float e = 0.f;
+  {
+    const uint4* o4 = reinterpret_cast<const uint4*>(O + row * D);
+    const uint4* do4 = reinterpret_cast<const uint4*>(dO + row * D);
+    const uint4* g4 = reinterpret_cast<const uint4*>(G + row * D);
+    const uint4* dv4 = reinterpret_cast<const uint4*>(dV + row * D);
+#pragma unroll 4
+    for (int k = 0; k < D / 8; ++k) e += dot8_bf16(o4[k], do4[k]) + dot8_bf16(g4[k], dv4[k]);
+  }
+  // <W_end, dW_end> over the D x D state
+  float w = 0.f;
+  if (c + 1 < NC) {
+    const uint4* a4 = reinterpret_cast<const uint4*>(Wc + ((size_t)bh * NC + c + 1) * D * D);
+    const uint4* b4 = reinterpret_cast<const uint4*>(dWs + ((size_t)bh * NC + c) * D * D);
+    for (int k = s; k < D * D / 8; k += C) w += dot8_bf16(a4[k], b4[k]);
+  } else if (dW_final) {
+    const float4* a4 = reinterpret_cast<const float4*>(W_final + (size_t)bh * D * D);
+    const float4* b4 = reinterpret_cast<const float4*>(dW_final + (size_t)bh * D * D);
+    for (int k = s; k < D * D / 4; k += C) {
+      const float4 a = a4[k], b = b4[k];
+      w += a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) w += __shfl_xor_sync(0xffffffffu, w, off);
+  if (lane == 0) red[wid] = w;
+  __syncthreads();
+  if (s == 0) {
+    float t = 0.f;
+    for (int i = 0; i < C / 32; ++i) t += red[i];
+    wsum = t;
+  }
+  __syncthreads();
+  // suffix sum of e over the chunk: inclusive scan from the last token backwards
+  float x = e;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_down_sync(0xffffffffu, x, off);
+    if (lane + off < 32) x += y;
+  }
+  if (lane == 0) red[wid] = x;  // sum of this warp's 32 tokens
+  __syncthreads();
+  float later = 0.f;
+  for (int i = wid + 1; i < C / 32; ++i) later += red[i];
+  dgamma[row] = (x + later + wsum) / gamma[row];
+}
+
 #undef BAR
 
 // Per-device pair of internal streams (chain then dk at the higher priority; g then dq at the
@@ -965,7 +1037,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
 // (their GPU work then serialises through the shared streams).
 struct ForkSet {
   cudaStream_t hi = nullptr, lo = nullptr;
-  cudaEvent_t e0 = nullptr, eg = nullptr, ehi = nullptr, elo = nullptr;
+  cudaEvent_t e0 = nullptr, eg = nullptr, ehi = nullptr, elo = nullptr, ech = nullptr;
 };
 constexpr int kMaxDevices = 64;
 ForkSet g_fork[kMaxDevices];
@@ -984,7 +1056,8 @@ ForkSet* fork_set() {
         cudaEventCreateWithFlags(&n.e0, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&n.eg, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&n.ehi, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&n.elo, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&n.elo, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&n.ech, cudaEventDisableTiming) != cudaSuccess)
       return nullptr;
     f = n;
   }
@@ -1054,15 +1127,26 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       (e = cudaStreamWaitEvent(f->lo, f->e0, 0)))
     return e;
   kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, tDV1, tDW, p);
+  if ((e = cudaEventRecord(f->ech, f->hi))) return e;
   if (!g_saved) kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
   if ((e = cudaEventRecord(f->eg, f->lo))) return e;
   kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, tDQ1, p);
+  int launched = g_saved ? 3 : 4;
+  if (a.dgamma) {
+    // after the chain (dV, the chunk-end adjoints), beside dK
+    if ((e = cudaStreamWaitEvent(f->lo, f->ech, 0))) return e;
+    bwd_dgamma_kernel<D, C><<<BH * NC, C, 0, f->lo>>>(
+        static_cast<const __nv_bfloat16*>(a.O_in), static_cast<const __nv_bfloat16*>(a.dO), G,
+        static_cast<const __nv_bfloat16*>(a.dV), static_cast<const __nv_bfloat16*>(a.W_chunks),
+        dWs, a.W_final_in, a.dW_final, a.gamma, a.dgamma, a.T, NC);
+    ++launched;
+  }
   if ((e = cudaEventRecord(f->elo, f->lo)) || (e = cudaStreamWaitEvent(f->hi, f->eg, 0))) return e;
   kk<<<BH * NC * NB, kSmallThreads, sm_dk, f->hi>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, tDK1, p);
   if ((e = cudaEventRecord(f->ehi, f->hi)) || (e = cudaStreamWaitEvent(s, f->ehi, 0)) ||
       (e = cudaStreamWaitEvent(s, f->elo, 0)))
     return e;
-  count_launches(g_saved ? 3 : 4);
+  count_launches(launched);
   return cudaGetLastError();
 }
 

@@ -146,9 +146,10 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
 }
 
 // Per-head float32 scratch of the backward (in units of floats): Wh, Wn, W0 (dk x dv each),
-// Z, G, dZq, Y, dG, dZ (C x dv each), S, dS (C x C each), eta, L, deta (C each).
+// Z, G, dZq, Y, dG, dZ, Zq (C x dv each), S, dS (C x C each), eta, L, deta, dL (C each), and
+// one float for the chunk-end term of the decay gradient.
 __host__ __device__ inline size_t bwd_head_floats(int C, int dk, int dv) {
-  return 3 * (size_t)dk * dv + 6 * (size_t)C * dv + 2 * (size_t)C * C + 3 * (size_t)C;
+  return 3 * (size_t)dk * dv + 7 * (size_t)C * dv + 2 * (size_t)C * C + 4 * (size_t)C + 1;
 }
 
 // Analytic backward of the chunk dual form, reverse over chunks; one block per head.
@@ -156,8 +157,8 @@ __host__ __device__ inline size_t bwd_head_floats(int C, int dk, int dv) {
 template <typename TI>
 __global__ void __launch_bounds__(512) simt_bwd_kernel(
     Dims d, const TI* Q, const TI* K, const TI* V, const float* beta, const float* gamma,
-    const TI* Wc, const TI* dO, const float* dWf, TI* dQ, TI* dK, TI* dV, float* dbeta,
-    float* dW0, float* ws) {
+    const TI* Wc, const TI* dO, const float* dWf, const float* Wfin, TI* dQ, TI* dK, TI* dV,
+    float* dbeta, float* dW0, float* dgamma, float* ws) {
   const int bh = blockIdx.x;
   const int dk = d.dk, dv = d.dv, C = d.C, NC = d.T / d.C;
   float* Wh = ws + (size_t)bh * bwd_head_floats(C, dk, dv);
@@ -174,6 +175,9 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
   float* eta = DS + C * C;
   float* L = eta + C;
   float* deta = L + C;
+  float* ZQ = deta + C;
+  float* dL = ZQ + C * dv;
+  float* wend = dL + C;  // <W_end, dW_end> of the chunk
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
   for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
     Wh[e] = dWf ? dWf[(size_t)bh * dk * dv + e] : 0.f;
@@ -221,6 +225,7 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       for (int i = 0; i < dk; ++i) y += ldf(Q + qk0 + (tc + s) * dk + i) * W0[i * dv + j];
       float zq = expf(L[s]) * y;
       for (int r = 0; r <= s; ++r) zq -= S[s * C + r] * G[r * dv + j];
+      ZQ[e] = zq;
       DZQ[e] = ldf(dO + v0 + (tc + s) * dv + j) * act1(d.act, zq);
     }
     __syncthreads();
@@ -286,6 +291,34 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
     }
     for (int r = threadIdx.x; r < C; r += blockDim.x)
       dbeta[(size_t)bh * d.T + tc + r] = deta[r] * eta[r] * (1.f - 0.5f * eta[r]);
+    if (dgamma) {
+      // dJ/dL_s = dZq_s . Zq_s - g_s . dG_s, plus <W_end, dW_end> on the last token; dgamma_t is
+      // the suffix sum over the chunk divided by gamma_t
+      for (int s2 = threadIdx.x; s2 < C; s2 += blockDim.x) {
+        float acc = 0.f;
+        for (int j = 0; j < dv; ++j)
+          acc += DZQ[s2 * dv + j] * ZQ[s2 * dv + j] - G[s2 * dv + j] * DG[s2 * dv + j];
+        dL[s2] = acc;
+      }
+      if (threadIdx.x == 0) *wend = 0.f;
+      __syncthreads();
+      float part = 0.f;
+      if (c + 1 < NC || dWf)
+        for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+          const float we = c + 1 < NC ? ldf(Wc + ((size_t)bh * NC + c + 1) * dk * dv + e)
+                                      : Wfin[(size_t)bh * dk * dv + e];
+          part += we * Wh[e];
+        }
+      atomicAdd(wend, part);
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        float acc = *wend;
+        for (int s2 = C - 1; s2 >= 0; --s2) {
+          acc += dL[s2];
+          dgamma[(size_t)bh * d.T + tc + s2] = acc / gamma[(size_t)bh * d.T + tc + s2];
+        }
+      }
+    }
     // dW at the chunk start = Gamma_C Wh + Q^T diag(Gamma) dZq + K^T dZ
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
       const int i = e / dv, j = e % dv;
@@ -349,14 +382,14 @@ cudaError_t simt_bwd(const LayerArgs& a, cudaStream_t s) {
   if (a.dtype == 0) {
     simt_bwd_kernel<float><<<a.B * a.H, 512, 0, s>>>(
         d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta, a.gamma,
-        (const float*)a.W_chunks, (const float*)a.dO, a.dW_final, (float*)a.dQ, (float*)a.dK,
-        (float*)a.dV, a.dbeta, a.dW0, (float*)a.ws);
+        (const float*)a.W_chunks, (const float*)a.dO, a.dW_final, a.W_final_in, (float*)a.dQ,
+        (float*)a.dK, (float*)a.dV, a.dbeta, a.dW0, a.dgamma, (float*)a.ws);
   } else {
     simt_bwd_kernel<__nv_bfloat16><<<a.B * a.H, 512, 0, s>>>(
         d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K, (const __nv_bfloat16*)a.V,
         a.beta, a.gamma, (const __nv_bfloat16*)a.W_chunks, (const __nv_bfloat16*)a.dO,
-        a.dW_final, (__nv_bfloat16*)a.dQ, (__nv_bfloat16*)a.dK, (__nv_bfloat16*)a.dV, a.dbeta,
-        a.dW0, (float*)a.ws);
+        a.dW_final, a.W_final_in, (__nv_bfloat16*)a.dQ, (__nv_bfloat16*)a.dK,
+        (__nv_bfloat16*)a.dV, a.dbeta, a.dW0, a.dgamma, (float*)a.ws);
   }
   count_launches(1);
   return cudaGetLastError();
