@@ -182,11 +182,32 @@ class Layer:
         self.ttt.ttt_chunk_fwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
                                self.O, self.Wf, self.Wc, self.G, self.ws, self.nf)
 
-    def bwd(self):
+    def bwd(self, dgamma=None):
         i = self.inp
         self.ttt.ttt_chunk_bwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
-                               self.Wc, self.G, i["dO"], i["dW_T"], None, None, self.dQ, self.dK,
-                               self.dV, self.dbeta, self.dW0, None, self.ws, self.nb)
+                               self.Wc, self.G, i["dO"], i["dW_T"],
+                               self.O if dgamma is not None else None,
+                               self.Wf if dgamma is not None else None, self.dQ, self.dK,
+                               self.dV, self.dbeta, self.dW0, dgamma, self.ws, self.nb)
+
+
+def time_bwd_dgamma(layer, steps=5, warmup=2):
+    """Device time of the backward that also returns the decay gradient (a separate line: the
+    workload's gradients do not include it)."""
+    if layer.inp["gamma"] is None:
+        return None
+    dg = torch.empty_like(layer.inp["gamma"])
+    layer.fwd()
+    for _ in range(warmup):
+        layer.bwd(dg)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        layer.bwd(dg)
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
 
 
 def time_steps(layer, steps, warmup, sampler=None):
@@ -427,6 +448,9 @@ def main():
         "kernels_ms": {"ttt_chunk_fwd": fwd_ms, "ttt_chunk_bwd": bwd_ms},
         "gpu_launches": launches, "clocks": clocks,
     }
+    dg_ms = time_bwd_dgamma(layer)
+    if dg_ms is not None:
+        out["kernels_ms"]["ttt_chunk_bwd_with_dgamma"] = dg_ms
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(layer, args.steps, args.warmup)
         e2e_ms = reduce_max(e2e_ms)
