@@ -191,6 +191,43 @@ class Layer:
                                self.dV, self.dbeta, self.dW0, dgamma, self.ws, self.nb)
 
 
+FP32_ALU_PEAK = 148 * 128 * 2 * 1.965e9  # flop/s
+
+
+def time_fwd_configs(ttt, peaks, steps=10, warmup=3):
+    """Forward throughput of the other workloads (tiny fp32, 410M-shaped, SiLU/inner product):
+    tokens/s and the fractions of the tensor-core and HBM rooflines, inputs resident in HBM."""
+    res = {}
+    for cfg in (synth.TINY_FP32, synth.FWD_410M, synth.SILU_IP_FWD):
+        layer = Layer(cfg, ttt, seed=cfg.seed)
+        for _ in range(warmup):
+            layer.fwd()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            layer.fwd()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / steps
+        w = layer_work(cfg)
+        flops = w["fwd_flops"] / (ms * 1e-3)
+        res[cfg.name] = {
+            "call": "ttt_chunk_fwd", "ms": ms, "tokens_per_s": cfg.B * cfg.T / (ms * 1e-3),
+            "dtype": cfg.dtype, "hbm_frac": w["fwd_bytes"] / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+        }
+        if cfg.dtype == "bf16":
+            res[cfg.name].update(path="tcgen05", tc_frac=flops / (peaks["bf16_tflops"] * 1e12))
+        else:
+            # fp32 runs on CUDA cores: 148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz
+            res[cfg.name].update(path="simt", alu_frac=flops / FP32_ALU_PEAK)
+        if cfg.name == synth.TINY_FP32.name:
+            res[cfg.name]["note"] = "latency-bound correctness workload (two heads)"
+        del layer
+        torch.cuda.empty_cache()
+    return res
+
+
 def time_bwd_dgamma(layer, steps=5, warmup=2):
     """Device time of the backward that also returns the decay gradient (a separate line: the
     workload's gradients do not include it)."""
@@ -370,6 +407,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-inplace", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the forward throughput of the other workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -458,6 +497,8 @@ def main():
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del layer
     torch.cuda.empty_cache()
+    if not args.no_configs:
+        out["other_configs"] = time_fwd_configs(ttt, peaks)
     if not args.no_inplace:
         icfg, ims = time_inplace(ttt, steps=3, warmup=1)
         fl, by = inplace_work(icfg)
