@@ -87,7 +87,9 @@ typedef struct {
 
 /* Bytes of workspace ttt_chunk_fwd (for_bwd = 0) or ttt_chunk_bwd needs for this config; 0 if
  * none. for_bwd = 1: the backward without G_saved (it rebuilds G in the workspace); for_bwd = 2:
- * the backward given G_saved. Returns (size_t)-1 if the config (or for_bwd) is invalid. */
+ * the backward given G_saved. The backward figure covers a call that asks for dgamma (on the
+ * tensor-core path that adds B*H*T*4 bytes, which calls without dgamma do not touch).
+ * Returns (size_t)-1 if the config (or for_bwd) is invalid. */
 size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd);
 
 /* Forward of the chunkwise TTT layer.
@@ -131,7 +133,8 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
  *  - Only configs of the tensor-core backward are accepted (bf16, identity activation,
  *    dk == dv in {64, 128}, C in {128, 256}); others return TTT_ERR_UNSUPPORTED.
  *  - Configs needing more than the fixed scratch (B*H*(T/C)*dk*dv*2 bytes, plus B*H*T*dv*2 when
- *    G_saved is NULL) return TTT_ERR_WORKSPACE with nothing launched; ttt_chunk_bwd serves those.
+ *    G_saved is NULL, plus B*H*T*4 when dgamma is non-NULL) return TTT_ERR_WORKSPACE with
+ *    nothing launched; ttt_chunk_bwd serves those.
  *  - The first call on a device looks up the array's device address (with that device
  *    current); make that first call before any stream capture.
  *  - Every call shares the one array and leaves its contents behind. Calls that overlap on

@@ -105,6 +105,17 @@ def test_bwd_requires_chunk_states_and_workspace():
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *dg, A, need, None) == ttt.ERR_INVALID_ARG
 
 
+def test_tc_bwd_workspace_covers_the_decay_gradient():
+    # the query's backward figure includes the float per token that only dgamma calls use
+    tc = _cfg(dtype="bf16", dk=128, dv=128, C=256, T=512)
+    need = ttt.ttt_workspace_bytes(tc, 2)
+    A = 4096
+    # Q K V beta gamma W0 W_chunks G_saved dO dW_final O W_final dQ dK dV dbeta dW0 dgamma
+    args = [A, A, A, A, A, A, A, A, A, None, A, None, A, A, A, A, A, A]
+    short = need - tc.B * tc.H * tc.T * 4
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(tc), *args, A, short, None) == ttt.ERR_WORKSPACE
+
+
 def test_inplace_argument_errors():
     A = 4096
     f = ttt.lib.inplace_ttt_fwd

@@ -16,10 +16,10 @@ from _util import rel_err
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-2
-GRADS = ("dQ", "dK", "dV", "dbeta", "dW0")
+GRADS = ("dQ", "dK", "dV", "dbeta", "dW0", "dgamma")
 
 
-def noalloc_bwd(cfg, inp, W_chunks, G=None):
+def noalloc_bwd(cfg, inp, W_chunks, G, fwd):
     c = abi_config(cfg)
     sd = synth.storage_dtype(cfg)
     B, H, T, dk, dv = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv
@@ -27,13 +27,15 @@ def noalloc_bwd(cfg, inp, W_chunks, G=None):
                dK=torch.full((B, H, T, dk), float("nan"), device="cuda", dtype=sd),
                dV=torch.full((B, H, T, dv), float("nan"), device="cuda", dtype=sd),
                dbeta=torch.full((B, H, T), float("nan"), device="cuda"),
-               dW0=torch.full((B, H, dk, dv), float("nan"), device="cuda"))
+               dW0=torch.full((B, H, dk, dv), float("nan"), device="cuda"),
+               dgamma=torch.full((B, H, T), float("nan"), device="cuda"))
     st = ttt.lib.ttt_chunk_bwd_noalloc(
         ctypes.byref(c), inp["Q"].data_ptr(), inp["K"].data_ptr(), inp["V"].data_ptr(),
         inp["beta"].data_ptr(), inp["gamma"].data_ptr(), inp["W0"].data_ptr(), W_chunks.data_ptr(),
         G.data_ptr() if G is not None else None, inp["dO"].data_ptr(), inp["dW_T"].data_ptr(),
-        None, None, out["dQ"].data_ptr(), out["dK"].data_ptr(), out["dV"].data_ptr(),
-        out["dbeta"].data_ptr(), out["dW0"].data_ptr(), None,
+        fwd["O"].data_ptr(), fwd["W_final"].data_ptr(), out["dQ"].data_ptr(),
+        out["dK"].data_ptr(), out["dV"].data_ptr(), out["dbeta"].data_ptr(),
+        out["dW0"].data_ptr(), out["dgamma"].data_ptr(),
         torch.cuda.current_stream().cuda_stream)
     assert st == ttt.OK, ttt.status_string(st)
     torch.cuda.synchronize()
@@ -43,14 +45,15 @@ def noalloc_bwd(cfg, inp, W_chunks, G=None):
 
 def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
     # scratch needed: 4 heads x 4 chunks x 128 x 128 x 2 bytes = 512 KiB, plus 1 MiB of G when the
-    # forward's G is not passed (limit 8 MiB); the first call passes it, the second does not
+    # forward's G is not passed, plus 16 KiB for dgamma (limit 8 MiB); the first call passes G,
+    # the second does not
     cfg = synth.TRAIN_1P45B.replace(B=1, H=4, T=1024)
     for seed, saved_g in ((21, True), (22, False)):
         inp = synth.ttt_inputs(cfg, device="cuda", seed=seed)
         inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(seed))
         fwd = run_fwd(cfg, inp, save_g=saved_g)
-        ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
-        got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G"])
+        ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd=fwd)
+        got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd)
         for k in GRADS:
             assert rel_err(got[k], ref[k]) <= TOL, (seed, k)
 

@@ -177,7 +177,7 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
   }
   if (for_bwd != 1 && for_bwd != 2) return (size_t)-1;
   switch (bwd_path(a)) {
-    case PATH_TC: return tc_bwd_workspace(a, for_bwd == 2);
+    case PATH_TC: return tc_bwd_workspace(a, for_bwd == 2, true);
     case PATH_SIMT: return simt_bwd_workspace(a);
     default: return (size_t)-1;
   }
@@ -229,7 +229,8 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
   const Path path = bwd_path(a);
   if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
   const size_t need =
-      path == PATH_TC ? tc_bwd_workspace(a, G_saved != nullptr) : simt_bwd_workspace(a);
+      path == PATH_TC ? tc_bwd_workspace(a, G_saved != nullptr, dgamma != nullptr)
+                     : simt_bwd_workspace(a);
   if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   cudaError_t e;
   unsigned* err = error_word(&e);

@@ -39,7 +39,7 @@ bool tc_fwd_supported(const LayerArgs& a);
 size_t tc_fwd_workspace(const LayerArgs& a);
 cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s);
 bool tc_bwd_supported(const LayerArgs& a);
-size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved);
+size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved, bool dgamma);
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
 
 // In-Place TTT.

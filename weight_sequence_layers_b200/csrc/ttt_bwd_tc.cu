@@ -59,6 +59,13 @@ struct BwdParams {
   __nv_bfloat16* dQ;
   __nv_bfloat16* dK;
   float* dbeta;
+  // decay gradient (dgamma non-null): dq writes dO_s . O_s into dgamma, dk writes g_s . dV_s
+  // (plus <W_end, dW_end> on the chunk's last token) into dgk, and a last pass turns their sum
+  // into suffix sums over the chunk
+  const __nv_bfloat16* Wc;    // [BH, NC, D, D] start state of each chunk
+  const float* W_final;       // [BH, D, D] state after the last chunk
+  float* dgamma;
+  float* dgk;                 // [BH, T] workspace
   unsigned* err;
 };
 
@@ -535,6 +542,21 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   teardown(bars, tmem, 128);
 }
 
+// --------------------------------------------------------------------------------- dgamma
+// Decay gradient. L_s = sum_{t<=s} log gamma_t (chunk-local) enters through Gamma_s and the
+// score weights of the readout and through u and Gamma_C of the transition; with the identity readout (Zq = O, dZq = dO) and dG = -dV,
+//   dJ/dL_s = dO_s . O_s + g_s . dV_s  (+ <W_end, dW_end> on the chunk's last token)
+//   dgamma_t = (1 / gamma_t) sum_{s >= t in the chunk} dJ/dL_s.
+// W_end is the next chunk's saved start state (W_final after the last chunk) and dW_end the
+// adjoint the chain saved at the chunk end (dW_final after the last chunk). The dQ kernel
+// writes the first dot, the dK kernel adds the second and the state term, and a last pass over
+// each chunk forms the suffix sums.
+__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
+  return bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x) + bf16lo(a.y) * bf16lo(b.y) +
+         bf16hi(a.y) * bf16hi(b.y) + bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z) +
+         bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+}
+
 // ----------------------------------------------------------------------------------- dQ
 // dQ_s = Gamma_s dO_s W0^T + sum_{r <= s} dP_sr K_r with dP = -(dO G^T) * M, one CTA per
 // (batch, head, chunk, 128-query block); key blocks stream through one G and one K slot.
@@ -552,13 +574,14 @@ struct DqL {
   static constexpr uint32_t T_DQ = 0, T_DS = D;
 };
 enum { Q_LD0, Q_DQ0, Q_DQ_SCALED, Q_G_FULL, Q_K_FULL, Q_DS_FULL, Q_DP_READY, Q_DP_DONE,
-       Q_DQ_FULL, Q_SCAN, Q_ST, Q_BG, Q_NBARS };
+       Q_DQ_FULL, Q_SCAN, Q_ST, Q_BG, Q_O_FULL, Q_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmW,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmG,
-                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const __grid_constant__ CUtensorMap tmO,
+                  const BwdParams p) {
   using L = DqL<D, NB>;
   constexpr int C = L::C;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -574,13 +597,14 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int sb = blockIdx.x % NB;
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
-  const int counts[Q_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1};
+  const int counts[Q_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1};
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmDO);
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmG);
     tma_prefetch_desc(&tmDQ);
+    if (p.dgamma) tma_prefetch_desc(&tmO);
   }
   uint32_t tmem;
   setup(bars, counts, Q_NBARS, tmem, 256);
@@ -618,6 +642,13 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
           for (int kp = 0; kp < L::KP; ++kp)
             tma_load_2d(sK + kp * PANEL128, &tmK, BAR(Q_K_FULL), 64 * kp, tokc + 128 * rb);
         }
+      }
+      // decay gradient: O_sb into the G slot once the last score MMA has read G_sb
+      if (p.dgamma && mbar_wait(BAR(Q_DS_FULL), sb & 1, ab)) {
+        mbar_arrive_expect_tx(BAR(Q_O_FULL), L::BLK);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sGW + kp * PANEL128, &tmO, BAR(Q_O_FULL), 64 * kp, tokc + 128 * sb);
       }
     }
   } else if (warp == 1) {
@@ -701,6 +732,20 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         epi_arrive(BAR(Q_DP_READY));
       }
       if (!ok) break;
+      if (p.dgamma) {
+        // dJ/dL_s starts as dO_s . O_s; the dK kernel adds the rest
+        if (!mbar_wait(BAR(Q_O_FULL), 0, ab)) break;
+        float dot = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float a[32], b[32];
+          ld_row32(sDO + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), a);
+          ld_row32(sGW + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), b);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dot += a[j] * b[j];
+        }
+        p.dgamma[(size_t)tokc + s] = dot;
+      }
       // dQ staged in the dO slot (its last readers, the MMAs, are complete), one bulk store
       if (!mbar_wait(BAR(Q_DQ_FULL), 0, ab)) break;
       __syncwarp();
@@ -740,11 +785,12 @@ struct DkL {
   static constexpr uint32_t OFF_G = 0, OFF_A = BLK, OFF_B = BLK + SLOT, OFF_F = 2 * BLK + SLOT;
   static constexpr uint32_t OFF_BG = OFF_F + 6 * 256 * 4;  // beta, gamma of the chunk
   static constexpr uint32_t OFF_BAR = OFF_BG + 2 * C * 4;
-  static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
+  static constexpr uint32_t OFF_RED = OFF_BAR + sizeof(Bars);  // 4 partial sums
+  static constexpr uint32_t BYTES = OFF_RED + 4 * 4;
   static constexpr uint32_t T_DK = 0, T_DS = D;
 };
 enum { K_LD0, K_H, K_H_SCALED, K_DO_FULL, K_Q_FULL, K_DS_FULL, K_DP_READY, K_DK_STEP,
-       K_DVW_FULL, K_DK_FULL, K_SCAN, K_ST, K_BG, K_NBARS };
+       K_DVW_FULL, K_DK_FULL, K_SCAN, K_ST, K_BG, K_WD, K_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
@@ -768,7 +814,8 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
   const bool mse = p.loss == 0;
-  const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1, kSmallEpi, 1};
+  const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1, kSmallEpi, 1,
+                               kSmallEpi};
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmG);
     tma_prefetch_desc(&tmDW);
@@ -921,6 +968,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
       if (!ok) break;
       // dbeta_r = -(1 - eta_r / 2) G_r . dV_r
       if (!mbar_wait(BAR(K_DVW_FULL), 0, ab)) break;
+      float e_r = 0.f;  // decay gradient: dJ/dL_r without the state term
       {
         float dot = 0.f;
 #pragma unroll
@@ -932,6 +980,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
           for (int j = 0; j < 32; ++j) dot += gv[j] * dv[j];
         }
         p.dbeta[(size_t)tokc + r] = -(1.f - 0.5f * er) * dot;
+        e_r = dot;
       }
       // dK staged over this thread's own row of G (every reader of G is done), one bulk store
       if (!mbar_wait(BAR(K_DK_FULL), 0, ab)) break;
@@ -952,71 +1001,55 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         bulk_commit();
         bulk_wait_read0();
       }
+      if (p.dgamma) {
+        if (rb == NB - 1) {
+          // <W_end, dW_end> joins dJ/dL of the chunk's last token: W_end is the next chunk's
+          // start state (W_final after the last chunk), dW_end the adjoint at this chunk's end
+          const int et = threadIdx.x - 64;
+          float w = 0.f;
+          if (c + 1 < p.NC) {
+            const uint4* a4 = reinterpret_cast<const uint4*>(p.Wc + (size_t)(wrow + D) * D);
+            const uint4* b4 = reinterpret_cast<const uint4*>(p.dWs + (size_t)wrow * D);
+#pragma unroll 4
+            for (int k = et; k < D * D / 8; k += 32 * kSmallEpi) w += dot8_bf16(a4[k], b4[k]);
+          } else if (p.dW_final) {
+            const float4* a4 = reinterpret_cast<const float4*>(p.W_final + (size_t)bh * D * D);
+            const float4* b4 = reinterpret_cast<const float4*>(p.dW_final + (size_t)bh * D * D);
+#pragma unroll 4
+            for (int k = et; k < D * D / 4; k += 32 * kSmallEpi) {
+              const float4 x = a4[k], y = b4[k];
+              w += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+            }
+          }
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) w += __shfl_xor_sync(0xffffffffu, w, off);
+          float* red = reinterpret_cast<float*>(smem + L::OFF_RED);
+          if (lane == 0) {
+            red[q] = w;
+            mbar_arrive(BAR(K_WD));  // release: red[q] is visible to the waiter
+          }
+          if (lrow == 127) {
+            if (!mbar_wait(BAR(K_WD), 0, ab)) break;
+            e_r += red[0] + red[1] + red[2] + red[3];
+          }
+        }
+        p.dgk[(size_t)tokc + r] = e_r;
+      }
     } while (0);
   }
   teardown(bars, tmem, 256);
 }
 
-// --------------------------------------------------------------------------------- dgamma
-// Decay gradient of one (batch, head, chunk), one thread per token. L_s = sum_{t<=s} log gamma_t
-// (chunk-local) enters through Gamma_s and the score weights of the readout and through u and
-// Gamma_C of the transition; with the identity readout (Zq = O, dZq = dO) and dG = -dV,
-//   dJ/dL_s = dO_s . O_s + g_s . dV_s  (+ <W_end, dW_end> on the chunk's last token)
-//   dgamma_t = (1 / gamma_t) sum_{s >= t in the chunk} dJ/dL_s.
-// W_end is the next chunk's saved start state (W_final after the last chunk) and dW_end the
-// adjoint the chain saved at the chunk end (dW_final after the last chunk).
-__device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b) {
-  return bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x) + bf16lo(a.y) * bf16lo(b.y) +
-         bf16hi(a.y) * bf16hi(b.y) + bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z) +
-         bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
-}
-
-template <int D, int C>
+// One CTA per (batch, head, chunk), one thread per token: dJ/dL_s = dgamma_s + dgk_s on entry.
+template <int C>
 __global__ void __launch_bounds__(C)
-    bwd_dgamma_kernel(const __nv_bfloat16* O, const __nv_bfloat16* dO, const __nv_bfloat16* G,
-                      const __nv_bfloat16* dV, const __nv_bfloat16* Wc, const __nv_bfloat16* dWs,
-                      const float* W_final, const float* dW_final, const float* gamma,
-                      float* dgamma, int T, int NC) {
+    bwd_dgamma_scan_kernel(const float* gamma, const float* dgk, float* dgamma, int T, int NC) {
   __shared__ float red[C / 32];
-  __shared__ float wsum;
   const int c = blockIdx.x % NC, bh = blockIdx.x / NC;
   const int s = threadIdx.x, lane = s & 31, wid = s >> 5;
   const size_t row = (size_t)bh * T + (size_t)c * C + s;
-  float e = 0.f;
-  {
-    const uint4* o4 = reinterpret_cast<const uint4*>(O + row * D);
-    const uint4* do4 = reinterpret_cast<const uint4*>(dO + row * D);
-    const uint4* g4 = reinterpret_cast<const uint4*>(G + row * D);
-    const uint4* dv4 = reinterpret_cast<const uint4*>(dV + row * D);
-#pragma unroll 4
-    for (int k = 0; k < D / 8; ++k) e += dot8_bf16(o4[k], do4[k]) + dot8_bf16(g4[k], dv4[k]);
-  }
-  // <W_end, dW_end> over the D x D state
-  float w = 0.f;
-  if (c + 1 < NC) {
-    const uint4* a4 = reinterpret_cast<const uint4*>(Wc + ((size_t)bh * NC + c + 1) * D * D);
-    const uint4* b4 = reinterpret_cast<const uint4*>(dWs + ((size_t)bh * NC + c) * D * D);
-    for (int k = s; k < D * D / 8; k += C) w += dot8_bf16(a4[k], b4[k]);
-  } else if (dW_final) {
-    const float4* a4 = reinterpret_cast<const float4*>(W_final + (size_t)bh * D * D);
-    const float4* b4 = reinterpret_cast<const float4*>(dW_final + (size_t)bh * D * D);
-    for (int k = s; k < D * D / 4; k += C) {
-      const float4 a = a4[k], b = b4[k];
-      w += a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) w += __shfl_xor_sync(0xffffffffu, w, off);
-  if (lane == 0) red[wid] = w;
-  __syncthreads();
-  if (s == 0) {
-    float t = 0.f;
-    for (int i = 0; i < C / 32; ++i) t += red[i];
-    wsum = t;
-  }
-  __syncthreads();
-  // suffix sum of e over the chunk: inclusive scan from the last token backwards
-  float x = e;
+  // suffix sum over the chunk: inclusive scan from the last token backwards
+  float x = dgamma[row] + dgk[row];
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const float y = __shfl_down_sync(0xffffffffu, x, off);
@@ -1026,7 +1059,7 @@ __global__ void __launch_bounds__(C)
   __syncthreads();
   float later = 0.f;
   for (int i = wid + 1; i < C / 32; ++i) later += red[i];
-  dgamma[row] = (x + later + wsum) / gamma[row];
+  dgamma[row] = (x + later) / gamma[row];
 }
 
 #undef BAR
@@ -1037,7 +1070,7 @@ __global__ void __launch_bounds__(C)
 // (their GPU work then serialises through the shared streams).
 struct ForkSet {
   cudaStream_t hi = nullptr, lo = nullptr;
-  cudaEvent_t e0 = nullptr, eg = nullptr, ehi = nullptr, elo = nullptr, ech = nullptr;
+  cudaEvent_t e0 = nullptr, eg = nullptr, ehi = nullptr, elo = nullptr;
 };
 constexpr int kMaxDevices = 64;
 ForkSet g_fork[kMaxDevices];
@@ -1056,8 +1089,7 @@ ForkSet* fork_set() {
         cudaEventCreateWithFlags(&n.e0, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&n.eg, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&n.ehi, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&n.elo, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&n.ech, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&n.elo, cudaEventDisableTiming) != cudaSuccess)
       return nullptr;
     f = n;
   }
@@ -1073,7 +1105,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   __nv_bfloat16* dWs = static_cast<__nv_bfloat16*>(a.ws);
   const bool g_saved = a.G_saved != nullptr;
   __nv_bfloat16* G = g_saved ? static_cast<__nv_bfloat16*>(a.G_saved) : dWs + wrows * D;
-  CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tG1, tW, tDW, tDQ1, tDK1;
+  CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tG1, tW, tDW, tDQ1, tDK1, tO1;
   if (!make_tmap_bf16(&tK, a.K, D, rows, D, 64, C) || !make_tmap_bf16(&tQ, a.Q, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tDO, a.dO, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tK1, a.K, D, rows, D, 64, 128) ||
@@ -1085,7 +1117,8 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       !make_tmap_bf16(&tDK1, a.dK, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tG1, G, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tW, a.W_chunks, D, wrows, D, 64, D) ||
-      !make_tmap_bf16(&tDW, dWs, D, wrows, D, 64, D))
+      !make_tmap_bf16(&tDW, dWs, D, wrows, D, 64, D) ||
+      !make_tmap_bf16(&tO1, a.dgamma ? a.O_in : a.dO, D, rows, D, 64, 128))
     return cudaErrorInvalidValue;
   BwdParams p{};
   p.BH = BH;
@@ -1104,6 +1137,10 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.dQ = static_cast<__nv_bfloat16*>(a.dQ);
   p.dK = static_cast<__nv_bfloat16*>(a.dK);
   p.dbeta = a.dbeta;
+  p.Wc = static_cast<const __nv_bfloat16*>(a.W_chunks);
+  p.W_final = a.W_final_in;
+  p.dgamma = a.dgamma;
+  p.dgk = reinterpret_cast<float*>(dWs + wrows * D + (g_saved ? 0 : rows * D));
   p.err = a.err;
 
   const size_t sm_g = GL<D>::BYTES + 1024;
@@ -1127,22 +1164,18 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       (e = cudaStreamWaitEvent(f->lo, f->e0, 0)))
     return e;
   kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, tDV1, tDW, p);
-  if ((e = cudaEventRecord(f->ech, f->hi))) return e;
   if (!g_saved) kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
   if ((e = cudaEventRecord(f->eg, f->lo))) return e;
-  kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, tDQ1, p);
+  kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, tDQ1, tO1, p);
   int launched = g_saved ? 3 : 4;
-  if (a.dgamma) {
-    // after the chain (dV, the chunk-end adjoints), beside dK
-    if ((e = cudaStreamWaitEvent(f->lo, f->ech, 0))) return e;
-    bwd_dgamma_kernel<D, C><<<BH * NC, C, 0, f->lo>>>(
-        static_cast<const __nv_bfloat16*>(a.O_in), static_cast<const __nv_bfloat16*>(a.dO), G,
-        static_cast<const __nv_bfloat16*>(a.dV), static_cast<const __nv_bfloat16*>(a.W_chunks),
-        dWs, a.W_final_in, a.dW_final, a.gamma, a.dgamma, a.T, NC);
-    ++launched;
-  }
   if ((e = cudaEventRecord(f->elo, f->lo)) || (e = cudaStreamWaitEvent(f->hi, f->eg, 0))) return e;
   kk<<<BH * NC * NB, kSmallThreads, sm_dk, f->hi>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, tDK1, p);
+  if (a.dgamma) {
+    // the per-token sums of dq and dk meet here
+    if ((e = cudaStreamWaitEvent(f->hi, f->elo, 0))) return e;
+    bwd_dgamma_scan_kernel<C><<<BH * NC, C, 0, f->hi>>>(a.gamma, p.dgk, a.dgamma, a.T, NC);
+    ++launched;
+  }
   if ((e = cudaEventRecord(f->ehi, f->hi)) || (e = cudaStreamWaitEvent(s, f->ehi, 0)) ||
       (e = cudaStreamWaitEvent(s, f->elo, 0)))
     return e;
@@ -1157,10 +1190,12 @@ bool tc_bwd_supported(const LayerArgs& a) {
          (a.C == 128 || a.C == 256) && a.T % a.C == 0;
 }
 
-// [BH, NC, dk, dv] bf16 chunk-end adjoints, then (without G from the forward) [BH, T, dv] bf16 G
-size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved) {
+// [BH, NC, dk, dv] bf16 chunk-end adjoints, then (without G from the forward) [BH, T, dv] bf16 G,
+// then (for the decay gradient) [BH, T] float32 per-token sums of the dK kernel
+size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved, bool dgamma) {
   return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2 +
-         (g_saved ? 0 : (size_t)a.B * a.H * a.T * a.dv * 2);
+         (g_saved ? 0 : (size_t)a.B * a.H * a.T * a.dv * 2) +
+         (dgamma ? (size_t)a.B * a.H * a.T * 4 : 0);
 }
 
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s) {
