@@ -46,9 +46,9 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         d, f, i = ctypes.c_double, ctypes.c_float, ctypes.c_int
         p = ctypes.c_void_p
-        lib.ttt_oracle_fwd_f64.argtypes = [i] * 8 + [d] + [p] * 9 + [i]
-        lib.ttt_oracle_fwd_f32.argtypes = [i] * 8 + [d] + [p] * 9 + [i]
-        lib.ttt_oracle_bwd_f64.argtypes = [i] * 8 + [d] + [p] * 14 + [i]
+        lib.ttt_oracle_fwd_f64.argtypes = [i] * 8 + [d, i] + [p] * 9 + [i]
+        lib.ttt_oracle_fwd_f32.argtypes = [i] * 8 + [d, i] + [p] * 9 + [i]
+        lib.ttt_oracle_bwd_f64.argtypes = [i] * 8 + [d, i] + [p] * 14 + [i]
         for fn in (lib.ttt_oracle_fwd_f64, lib.ttt_oracle_fwd_f32, lib.ttt_oracle_bwd_f64):
             fn.restype = i
         _lib = lib
@@ -68,11 +68,23 @@ def _ptr(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
 
+def _gvec(g, q):
+    """1 when gamma carries one decay per key feature ([B,H,T,dk]), 0 for [B,H,T] or None."""
+    if g is None:
+        return 0
+    if g.shape == q.shape:
+        return 1
+    if g.shape != q.shape[:3]:
+        raise ValueError("gamma must be [B,H,T] or [B,H,T,dk]")
+    return 0
+
+
 def ttt_fwd(Q, K, V, beta, gamma, W0, *, C: int, loss: str = "mse", act: str = "id",
             lr_bias: float, nthreads: int = 0, state: str = "f64"):
     """Per-token fast-weight evolution. Returns (O, W_final, W_chunks, threads_used).
 
-    Q, K: [B,H,T,dk]; V: [B,H,T,dv]; beta, gamma: [B,H,T] (gamma None = no decay);
+    Q, K: [B,H,T,dk]; V: [B,H,T,dv]; beta: [B,H,T]; gamma: [B,H,T] (scalar decay),
+    [B,H,T,dk] (per-feature decay of the rows of W) or None (no decay);
     W0: [B,H,dk,dv]. state="f64" (parity) or "f32" (fp32 state, timed baseline).
     """
     lib = _load()
@@ -87,7 +99,8 @@ def ttt_fwd(Q, K, V, beta, gamma, W0, *, C: int, loss: str = "mse", act: str = "
     wf = np.empty((B, H, dk, dv), dt)
     wc = np.empty((B, H, T // C, dk, dv), dt)
     fn = lib.ttt_oracle_fwd_f64 if state == "f64" else lib.ttt_oracle_fwd_f32
-    used = fn(B, H, T, dk, dv, C, LOSS[loss], ACT[act], float(lr_bias), _ptr(q), _ptr(k), _ptr(v),
+    used = fn(B, H, T, dk, dv, C, LOSS[loss], ACT[act], float(lr_bias), _gvec(g_, q), _ptr(q),
+              _ptr(k), _ptr(v),
               _ptr(b_), _ptr(g_), _ptr(w0), _ptr(o), _ptr(wf), _ptr(wc), int(nthreads))
     if used < 0:
         raise ValueError("oracle rejected the shape")
@@ -97,7 +110,7 @@ def ttt_fwd(Q, K, V, beta, gamma, W0, *, C: int, loss: str = "mse", act: str = "
 def ttt_bwd(Q, K, V, beta, gamma, W0, dO, dW_T=None, *, C: int, loss: str = "mse",
             act: str = "id", lr_bias: float, nthreads: int = 0):
     """Reverse-mode of the per-token loop for J = <dO,O> + <dW_T,W_final> (fp64).
-    Returns dict dQ, dK, dV, dbeta, dW0, and dgamma when gamma is given."""
+    Returns dict dQ, dK, dV, dbeta, dW0, and dgamma (shaped like gamma) when gamma is given."""
     lib = _load()
     dt = np.float64
     q, k, v = _np(Q, dt), _np(K, dt), _np(V, dt)
@@ -111,9 +124,9 @@ def ttt_bwd(Q, K, V, beta, gamma, W0, dO, dW_T=None, *, C: int, loss: str = "mse
                dV=np.empty((B, H, T, dv)), dbeta=np.empty((B, H, T)),
                dW0=np.empty((B, H, dk, dv)))
     if g_ is not None:
-        out["dgamma"] = np.empty((B, H, T))
+        out["dgamma"] = np.empty(g_.shape)
     used = lib.ttt_oracle_bwd_f64(B, H, T, dk, dv, C, LOSS[loss], ACT[act], float(lr_bias),
-                                  _ptr(q), _ptr(k), _ptr(v), _ptr(b_), _ptr(g_), _ptr(w0),
+                                  _gvec(g_, q), _ptr(q), _ptr(k), _ptr(v), _ptr(b_), _ptr(g_), _ptr(w0),
                                   _ptr(do), _ptr(dwt), _ptr(out["dQ"]), _ptr(out["dK"]),
                                   _ptr(out["dV"]), _ptr(out["dbeta"]), _ptr(out["dW0"]),
                                   _ptr(out.get("dgamma")), int(nthreads))

@@ -13,7 +13,9 @@
 //     "测试时训练与快速权重");
 //   * learning rate eta_t = 2*sigmoid(beta_t + b) (section "内部学习规则与
 //     学习率参数化");
-//   * scalar decay of past writes (section "权重衰减");
+//   * decay of past writes (section "权重衰减"): scalar (one gamma_t per token)
+//     or per feature (vector decay: gamma_t has one factor per key feature and
+//     scales the matching row of W, W_s = diag(gamma_s) W_{s-1} - ...);
 //   * Algorithm 1, three passes per chunk: train-view forward Vhat = act(K W0),
 //     train-view backward of the inner loss (MSE or inner product), query-view
 //     readout, with the chunk-start weight W0 used for every gradient in the
@@ -35,7 +37,8 @@
 //
 // The backward is reverse-mode differentiation of the same per-token loop
 // for J = <dO, O> + <dW_T, W_final>, returning dQ, dK, dV, dbeta and dW0, and
-// on request the decay gradient dgamma_s = <adjoint of W_s, W_{s-1}>.
+// on request the decay gradient dgamma_s = <adjoint of W_s, W_{s-1}> (per feature:
+// the same inner product restricted to row i of both).
 //
 // Pins (tests/test_oracle_pins.py): brute-force evaluation of the chunk dual
 // form printed on the page, the C = 1 delta rule and decayed Hebbian closed
@@ -77,7 +80,15 @@ template <typename R> inline R act_d2(int act, R z) {
 struct Shape {
   int B, H, T, dk, dv, C, loss, act;
   double lr_bias;
+  int gvec;  // gamma holds one factor per key feature: [B,H,T,dk] instead of [B,H,T]
 };
+
+// Decay of row (key feature) i of W at token t.
+template <typename R, typename In>
+inline R decay_at(const Shape& sh, const In* gamma, size_t t, int i) {
+  if (!gamma) return R(1);
+  return R(sh.gvec ? gamma[t * sh.dk + i] : gamma[t]);
+}
 
 // Train view of token t at the chunk-start weight W0: z = k W0, g = a * act'(z).
 template <typename R, typename In>
@@ -111,8 +122,8 @@ void fwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
       const In* qt = q + t * dk;
       train_view<R, In>(sh, kt, v + t * dv, W0.data(), z.data(), g.data());
       const R eta = R(2) * sigmoid_(R(beta[t]) + R(sh.lr_bias));
-      const R gam = gamma ? R(gamma[t]) : R(1);
       for (int i = 0; i < dk; ++i) {
+        const R gam = decay_at<R, In>(sh, gamma, t, i);
         const R eki = eta * R(kt[i]);
         R* wrow = W.data() + (size_t)i * dv;
         for (int j = 0; j < dv; ++j) wrow[j] = gam * wrow[j] - eki * g[j];
@@ -148,8 +159,8 @@ void bwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
       const size_t t = (size_t)c * C + s;
       train_view<R, In>(sh, k + t * dk, v + t * dv, W0, z.data(), g.data());
       const R eta = R(2) * sigmoid_(R(beta[t]) + R(sh.lr_bias));
-      const R gam = gamma ? R(gamma[t]) : R(1);
       for (int i = 0; i < dk; ++i) {
+        const R gam = decay_at<R, In>(sh, gamma, t, i);
         const R eki = eta * R(k[t * dk + i]);
         R* wrow = W.data() + (size_t)i * dv;
         for (int j = 0; j < dv; ++j) wrow[j] = gam * wrow[j] - eki * g[j];
@@ -171,9 +182,9 @@ void bwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
       R* gs = G.data() + (size_t)s * dv;
       train_view<R, In>(sh, k + t * dk, v + t * dv, W0, zs, gs);
       const R eta = R(2) * sigmoid_(R(beta[t]) + R(sh.lr_bias));
-      const R gam = gamma ? R(gamma[t]) : R(1);
       if (dgamma) std::memcpy(Wprev.data() + (size_t)s * WS, Ws.data(), sizeof(R) * WS);
       for (int i = 0; i < dk; ++i) {
+        const R gam = decay_at<R, In>(sh, gamma, t, i);
         const R eki = eta * R(k[t * dk + i]);
         R* wrow = Ws.data() + (size_t)i * dv;
         for (int j = 0; j < dv; ++j) wrow[j] = gam * wrow[j] - eki * gs[j];
@@ -201,7 +212,6 @@ void bwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
       const R* gs = G.data() + (size_t)s * dv;
       const R* dzq = DZQ.data() + (size_t)s * dv;
       const R eta = R(2) * sigmoid_(R(beta[t]) + R(sh.lr_bias));
-      const R gam = gamma ? R(gamma[t]) : R(1);
       // readout o_s = act(q_s W_s) adds to the adjoint of W_s
       for (int i = 0; i < dk; ++i) {
         const R qi = R(q[t * dk + i]);
@@ -222,14 +232,23 @@ void bwd_head(const Shape& sh, const In* q, const In* k, const In* v, const In* 
       }
       R deta = R(0);
       for (int j = 0; j < dv; ++j) deta -= kW[j] * gs[j];
-      // W_s = gam W_{s-1} - ...: dJ/dgam = <adjoint of W_s, W_{s-1}>
+      // W_s = diag(gam) W_{s-1} - ...: dJ/dgam_i = <row i of the adjoint of W_s, row i of
+      // W_{s-1}>, summed over the rows for a scalar decay
       if (dgamma) {
         const R* wp = Wprev.data() + (size_t)s * WS;
-        R acc = R(0);
-        for (size_t e = 0; e < WS; ++e) acc += Wh[e] * wp[e];
-        dgamma[t] = acc;
+        R tot = R(0);
+        for (int i = 0; i < dk; ++i) {
+          R acc = R(0);
+          for (int j = 0; j < dv; ++j) acc += Wh[(size_t)i * dv + j] * wp[(size_t)i * dv + j];
+          if (sh.gvec) dgamma[t * dk + i] = acc;
+          tot += acc;
+        }
+        if (!sh.gvec) dgamma[t] = tot;
       }
-      for (size_t e = 0; e < WS; ++e) Wh[e] *= gam;
+      for (int i = 0; i < dk; ++i) {
+        const R gam = decay_at<R, In>(sh, gamma, t, i);
+        for (int j = 0; j < dv; ++j) Wh[(size_t)i * dv + j] *= gam;
+      }
       // g = a * act'(z),  a = act(z) - v (MSE) or -v (IP),  z = k W0
       for (int j = 0; j < dv; ++j) {
         const R dg = -eta * kW[j];
@@ -276,7 +295,8 @@ int fwd_all(const Shape& sh, const In* Q, const In* K, const In* V, const In* be
 #pragma omp parallel for schedule(dynamic, 1)
   for (int bh = 0; bh < BH; ++bh) {
     fwd_head<R, In>(sh, Q + bh * tk, K + bh * tk, V + bh * tv, beta + (size_t)bh * sh.T,
-                    gamma ? gamma + (size_t)bh * sh.T : nullptr, W0 + bh * ws, O + bh * tv,
+                    gamma ? gamma + (size_t)bh * sh.T * (sh.gvec ? sh.dk : 1) : nullptr,
+                    W0 + bh * ws, O + bh * tv,
                     Wf ? Wf + bh * ws : nullptr, Wc ? Wc + (size_t)bh * NC * ws : nullptr);
   }
   return used;
@@ -286,49 +306,51 @@ int fwd_all(const Shape& sh, const In* Q, const In* K, const In* V, const In* be
 
 extern "C" {
 
-// Forward, fp64 state and arithmetic. Q,K [B,H,T,dk]; V,O [B,H,T,dv]; beta,gamma [B,H,T]
-// (gamma may be NULL: no decay); W0, W_final [B,H,dk,dv]; W_chunks [B,H,T/C,dk,dv] or NULL.
+// Forward, fp64 state and arithmetic. Q,K [B,H,T,dk]; V,O [B,H,T,dv]; beta [B,H,T]; gamma
+// [B,H,T], or [B,H,T,dk] with gamma_per_feature set (gamma may be NULL: no decay); W0, W_final
+// [B,H,dk,dv]; W_chunks [B,H,T/C,dk,dv] or NULL.
 // Returns the number of threads used, or -1 on a bad shape.
 int ttt_oracle_fwd_f64(int B, int H, int T, int dk, int dv, int C, int loss, int act, double lr_bias,
-                       const double* Q, const double* K, const double* V, const double* beta,
+                       int gamma_per_feature, const double* Q, const double* K, const double* V, const double* beta,
                        const double* gamma, const double* W0, double* O, double* W_final,
                        double* W_chunks, int nthreads) {
   if (B <= 0 || H <= 0 || T <= 0 || dk <= 0 || dv <= 0 || C <= 0 || T % C) return -1;
-  Shape sh{B, H, T, dk, dv, C, loss, act, lr_bias};
+  Shape sh{B, H, T, dk, dv, C, loss, act, lr_bias, gamma_per_feature != 0};
   return fwd_all<double, double>(sh, Q, K, V, beta, gamma, W0, O, W_final, W_chunks, nthreads);
 }
 
 // Forward with an fp32 state and fp32 arithmetic (the per-token fp32 state evolver; used as the
 // timed CPU baseline). Same layouts as above with float buffers.
 int ttt_oracle_fwd_f32(int B, int H, int T, int dk, int dv, int C, int loss, int act, double lr_bias,
-                       const float* Q, const float* K, const float* V, const float* beta,
+                       int gamma_per_feature, const float* Q, const float* K, const float* V, const float* beta,
                        const float* gamma, const float* W0, float* O, float* W_final,
                        float* W_chunks, int nthreads) {
   if (B <= 0 || H <= 0 || T <= 0 || dk <= 0 || dv <= 0 || C <= 0 || T % C) return -1;
-  Shape sh{B, H, T, dk, dv, C, loss, act, lr_bias};
+  Shape sh{B, H, T, dk, dv, C, loss, act, lr_bias, gamma_per_feature != 0};
   return fwd_all<float, float>(sh, Q, K, V, beta, gamma, W0, O, W_final, W_chunks, nthreads);
 }
 
 // Backward, fp64: reverse-mode of the per-token loop for J = <dO, O> + <dW_T, W_final>.
 // dW_T may be NULL (zero). Outputs dQ,dK [B,H,T,dk], dV [B,H,T,dv], dbeta [B,H,T], dW0 [B,H,dk,dv],
-// and dgamma [B,H,T] when both gamma and dgamma are non-NULL.
+// and dgamma (the shape of gamma) when both gamma and dgamma are non-NULL.
 int ttt_oracle_bwd_f64(int B, int H, int T, int dk, int dv, int C, int loss, int act, double lr_bias,
-                       const double* Q, const double* K, const double* V, const double* beta,
+                       int gamma_per_feature, const double* Q, const double* K, const double* V, const double* beta,
                        const double* gamma, const double* W0, const double* dO, const double* dW_T,
                        double* dQ, double* dK, double* dV, double* dbeta, double* dW0,
                        double* dgamma, int nthreads) {
   if (B <= 0 || H <= 0 || T <= 0 || dk <= 0 || dv <= 0 || C <= 0 || T % C) return -1;
-  Shape sh{B, H, T, dk, dv, C, loss, act, lr_bias};
+  Shape sh{B, H, T, dk, dv, C, loss, act, lr_bias, gamma_per_feature != 0};
   const int used = set_threads(nthreads);
   const int BH = B * H;
   const size_t tk = (size_t)T * dk, tv = (size_t)T * dv, ws = (size_t)dk * dv;
+  const size_t tg = (size_t)T * (gamma_per_feature ? dk : 1);
 #pragma omp parallel for schedule(dynamic, 1)
   for (int bh = 0; bh < BH; ++bh) {
     bwd_head<double, double>(sh, Q + bh * tk, K + bh * tk, V + bh * tv, beta + (size_t)bh * T,
-                             gamma ? gamma + (size_t)bh * T : nullptr, W0 + bh * ws, dO + bh * tv,
+                             gamma ? gamma + bh * tg : nullptr, W0 + bh * ws, dO + bh * tv,
                              dW_T ? dW_T + bh * ws : nullptr, dQ + bh * tk, dK + bh * tk,
                              dV + bh * tv, dbeta + (size_t)bh * T, dW0 + bh * ws,
-                             gamma && dgamma ? dgamma + (size_t)bh * T : nullptr);
+                             gamma && dgamma ? dgamma + bh * tg : nullptr);
   }
   return used;
 }

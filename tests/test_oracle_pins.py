@@ -13,6 +13,9 @@
 * streaming and column independence;
 * hand-worked golden values (tests/golden/scalar_chunk_worked.txt);
 * central finite differences for every backward output;
+* per-feature (vector) decay: its own brute-force dual form, the scalar decay
+  when all features share one factor, a zero factor clearing exactly one row
+  of W, and finite differences including the per-feature decay gradient;
 * In-Place TTT (page "In-Place Test-Time Training", section "核心方法和技术细节"):
   associativity of the update, plain GEMM when C = T or eta = 0, and the
   dual form with Z_i Z_j^T corrections.
@@ -277,6 +280,135 @@ def test_backward_matches_finite_differences(loss, act):
             fd[idx] = (jp - jm) / (2 * h)
         an = g[names[name]]
         err = np.abs(an - fd).max() / max(1e-12, np.abs(fd).max())
+        assert err < 1e-7, (name, err)
+
+
+# ------------------------------------------------------------ per-feature (vector) decay
+# Page "Modular TTT: Rethinking Test-Time Training as Composable Modules", section "权重衰减":
+# vector decay is a per-feature forgetting factor. Reading: gamma_t has one factor per key
+# feature and scales that row of W, W_t = diag(gamma_t) W_{t-1} - eta_t k_t^T g_t.
+
+
+def vector_gamma(rng, B, H, T, dk):
+    return sigmoid(2.0 + rng.standard_normal((B, H, T, dk)))
+
+
+def dual_form_vector(Q, K, V, beta, gamma, W0, C, loss, act, b):
+    """Chunk dual form with a per-feature decay, by brute force: with L_s the chunk-local
+    cumulative log-decay of every feature,
+        Zq_s  = (q_s * exp(L_s)) W0 - sum_{r<=s} eta_r (sum_i q_si k_ri exp(L_si - L_ri)) g_r
+        W_end = diag(exp(L_C)) W0 - sum_r eta_r (k_r * exp(L_C - L_r))^T g_r."""
+    B, H, T, dk = Q.shape
+    dv = V.shape[-1]
+    O = np.zeros((B, H, T, dv))
+    WF = np.zeros((B, H, dk, dv))
+    for bi in range(B):
+        for hi in range(H):
+            W = W0[bi, hi].copy()
+            for c in range(T // C):
+                sl = slice(c * C, (c + 1) * C)
+                q, k, v = Q[bi, hi, sl], K[bi, hi, sl], V[bi, hi, sl]
+                eta = 2 * sigmoid(beta[bi, hi, sl] + b)
+                L = np.cumsum(np.log(gamma[bi, hi, sl]), axis=0)  # [C, dk]
+                Z = k @ W
+                A = act_np(act, Z) - v if loss == "mse" else -v
+                G = A * dact_np(act, Z)
+                Zq = np.zeros((C, dv))
+                for s in range(C):
+                    acc = (q[s] * np.exp(L[s])) @ W
+                    for r in range(s + 1):
+                        p = float(np.sum(q[s] * k[r] * np.exp(L[s] - L[r])))
+                        acc = acc - eta[r] * p * G[r]
+                    Zq[s] = acc
+                O[bi, hi, sl] = act_np(act, Zq)
+                Wn = np.exp(L[-1])[:, None] * W
+                for r in range(C):
+                    Wn = Wn - eta[r] * np.outer(k[r] * np.exp(L[-1] - L[r]), G[r])
+                W = Wn
+            WF[bi, hi] = W
+    return O, WF
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+@pytest.mark.parametrize("C", [1, 2, 4, 8])
+def test_vector_decay_matches_its_dual_form(loss, act, C):
+    rng = np.random.default_rng(300 + C)
+    Q, K, V, beta, _, W0 = rand_inputs(rng, 1, 2, 16, 5, 3, decay=False)
+    gamma = vector_gamma(rng, 1, 2, 16, 5)
+    b = -0.7
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=C, loss=loss, act=act, lr_bias=b)
+    O2, WF2 = dual_form_vector(Q, K, V, beta, gamma, W0, C, loss, act, b)
+    np.testing.assert_allclose(O, O2, rtol=0, atol=1e-12 * max(1, np.abs(O2).max()))
+    np.testing.assert_allclose(WF, WF2, rtol=0, atol=1e-12 * max(1, np.abs(WF2).max()))
+
+
+def test_vector_decay_with_equal_features_is_the_scalar_decay():
+    rng = np.random.default_rng(310)
+    B, H, T, dk, dv = 1, 2, 16, 4, 3
+    Q, K, V, beta, gamma, W0 = rand_inputs(rng, B, H, T, dk, dv, decay=True)
+    gv = np.repeat(gamma[..., None], dk, axis=-1)
+    dO = rng.standard_normal((B, H, T, dv))
+    dWT = rng.standard_normal((B, H, dk, dv))
+    kw = dict(C=4, loss="mse", act="silu", lr_bias=-0.5)
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, **kw)
+    Ov, WFv, _, _ = oracle.ttt_fwd(Q, K, V, beta, gv, W0, **kw)
+    np.testing.assert_allclose(Ov, O, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(WFv, WF, rtol=0, atol=1e-13)
+    g = oracle.ttt_bwd(Q, K, V, beta, gamma, W0, dO, dWT, **kw)
+    gv_ = oracle.ttt_bwd(Q, K, V, beta, gv, W0, dO, dWT, **kw)
+    for k in ("dQ", "dK", "dV", "dbeta", "dW0"):
+        np.testing.assert_allclose(gv_[k], g[k], rtol=0, atol=1e-12)
+    # the scalar factor multiplies every row, so its gradient is the sum of the rows'
+    np.testing.assert_allclose(gv_["dgamma"].sum(-1), g["dgamma"], rtol=0, atol=1e-12)
+
+
+def test_vector_decay_zero_clears_exactly_one_row():
+    # gamma = 0 on key feature i0 at the last token: row i0 of W_final is that token's write
+    # alone, -eta k_{i0} g with g = k W0c - v (MSE, identity) at the last chunk's start state
+    rng = np.random.default_rng(320)
+    B, H, T, dk, dv, C, i0 = 1, 1, 12, 5, 3, 4, 2
+    Q, K, V, beta, _, W0 = rand_inputs(rng, B, H, T, dk, dv, decay=False)
+    gamma = vector_gamma(rng, B, H, T, dk)
+    gamma[0, 0, T - 1, i0] = 0.0
+    b = 0.2
+    _, WF, WC, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=C, loss="mse", act="id", lr_bias=b)
+    k, v = K[0, 0, T - 1], V[0, 0, T - 1]
+    eta = 2 * sigmoid(beta[0, 0, T - 1] + b)
+    g = k @ WC[0, 0, -1] - v
+    np.testing.assert_allclose(WF[0, 0, i0], -eta * k[i0] * g, rtol=0, atol=1e-13)
+    # with gamma = 1 there instead, the row keeps its history and differs
+    gamma[0, 0, T - 1, i0] = 1.0
+    _, WF1, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, C=C, loss="mse", act="id", lr_bias=b)
+    assert np.abs(WF1[0, 0, i0] - WF[0, 0, i0]).max() > 1e-3
+    others = [i for i in range(dk) if i != i0]
+    np.testing.assert_allclose(WF1[0, 0, others], WF[0, 0, others], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+def test_vector_decay_backward_matches_finite_differences(loss, act):
+    rng = np.random.default_rng(330 + 2 * list(dict.fromkeys(COMBOS)).index((loss, act)))
+    B, H, T, dk, dv, C = 1, 1, 12, 4, 3, 4
+    Q, K, V, beta, _, W0 = rand_inputs(rng, B, H, T, dk, dv, decay=False, w0_scale=0.5)
+    gamma = vector_gamma(rng, B, H, T, dk)
+    dO = rng.standard_normal((B, H, T, dv))
+    dWT = rng.standard_normal((B, H, dk, dv))
+    kw = dict(C=C, loss=loss, act=act, lr_bias=-0.4)
+    g = oracle.ttt_bwd(Q, K, V, beta, gamma, W0, dO, dWT, **kw)
+    assert g["dgamma"].shape == gamma.shape
+    h = 1e-6
+    args = dict(Q=Q, K=K, V=V, beta=beta, gamma=gamma, W0=W0)
+    names = dict(Q="dQ", K="dK", V="dV", beta="dbeta", gamma="dgamma", W0="dW0")
+    for name, x in args.items():
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            jp = _objective(Q, K, V, beta, gamma, W0, dO, dWT, kw)
+            x[idx] = old - h
+            jm = _objective(Q, K, V, beta, gamma, W0, dO, dWT, kw)
+            x[idx] = old
+            fd[idx] = (jp - jm) / (2 * h)
+        err = np.abs(g[names[name]] - fd).max() / max(1e-12, np.abs(fd).max())
         assert err < 1e-7, (name, err)
 
 
