@@ -82,8 +82,10 @@ def layer_work(cfg):
     fl_b = units * (12 * C * dk * dv + 2 * C * (C + 1) * (dk + dv))
     e = 2 if cfg.dtype == "bf16" else 4
     tok = B * H * T
-    by_f = tok * (2 * dk + dv) * e + tok * 4 * (2 if cfg.decay else 1) + 2 * B * H * dk * dv * 4 + tok * dv * e
-    by_b = (tok * (2 * dk + 2 * dv) * e + tok * 4 * (2 if cfg.decay else 1) + B * H * dk * dv * 4
+    # beta, and gamma: one float per token (scalar decay) or per token and key feature (vector)
+    bg = 4 * (1 + (dk if cfg.decay == "vector" else 1 if cfg.decay else 0))
+    by_f = tok * (2 * dk + dv) * e + tok * bg + 2 * B * H * dk * dv * 4 + tok * dv * e
+    by_b = (tok * (2 * dk + 2 * dv) * e + tok * bg + B * H * dk * dv * 4
             + tok * (2 * dk + dv) * e + tok * 4 + B * H * dk * dv * 4)
     return dict(fwd_flops=fl_f, bwd_flops=fl_b, fwd_bytes=by_f, bwd_bytes=by_b)
 
@@ -163,7 +165,8 @@ class Layer:
         B, H, T, dk, dv, C = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C
         sd = synth.storage_dtype(cfg)
         dev = "cuda"
-        self.c = ttt.make_config(B, H, T, dk, dv, C, cfg.dtype, cfg.loss, cfg.act, cfg.lr_bias)
+        self.c = ttt.make_config(B, H, T, dk, dv, C, cfg.dtype, cfg.loss, cfg.act, cfg.lr_bias,
+                                 "vector" if cfg.decay == "vector" else "scalar")
         self.O = torch.empty((B, H, T, dv), device=dev, dtype=sd)
         self.Wf = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
         self.Wc = torch.empty((B, H, T // C, dk, dv), device=dev, dtype=sd)
@@ -194,35 +197,66 @@ class Layer:
 FP32_ALU_PEAK = 148 * 128 * 2 * 1.965e9  # flop/s
 
 
-def time_fwd_configs(ttt, peaks, steps=10, warmup=3):
-    """Forward throughput of the other workloads (tiny fp32, 410M-shaped, SiLU/inner product):
-    tokens/s and the fractions of the tensor-core and HBM rooflines, inputs resident in HBM."""
+def _path(cfg, call):
+    """Which kernels serve the call for this workload (mirrors the library's dispatch)."""
+    tc_shape = cfg.dtype == "bf16" and cfg.decay != "vector" and cfg.dk == cfg.dv and \
+        cfg.dk in (64, 128) and cfg.C in (128, 256)
+    if call == "ttt_chunk_bwd":
+        tc_shape = tc_shape and cfg.act == "id"
+    return "tcgen05" if tc_shape else "simt"
+
+
+def _event_ms(fn, steps, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def time_other_configs(ttt, peaks):
+    """Throughput of the other workloads, inputs resident in HBM: the forward of the tiny fp32,
+    410M-shaped and SiLU/inner-product workloads, and forward+backward of the SiLU/inner-product
+    workload and of the 410M shape with a per-feature (vector) decay. Per call: device ms,
+    tokens/s and the fraction of the roofline of the kernels that serve it (tensor-core peak for
+    the tcgen05 kernels, fp32 CUDA-core peak for the SIMT kernels) and of HBM bandwidth."""
+    work = [(synth.TINY_FP32.name, synth.TINY_FP32, False),
+            (synth.FWD_410M.name, synth.FWD_410M, False),
+            (synth.SILU_IP_FWD.name, synth.SILU_IP_FWD, False),
+            ("silu-ip-fwd-bwd", synth.SILU_IP_FWD, True),
+            ("410m-ttt-linear-vector-decay-fwd-bwd", synth.FWD_410M.replace(decay="vector"), True)]
     res = {}
-    for cfg in (synth.TINY_FP32, synth.FWD_410M, synth.SILU_IP_FWD):
+    for name, cfg, with_bwd in work:
         layer = Layer(cfg, ttt, seed=cfg.seed)
-        for _ in range(warmup):
-            layer.fwd()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        for _ in range(steps):
-            layer.fwd()
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / steps
         w = layer_work(cfg)
-        flops = w["fwd_flops"] / (ms * 1e-3)
-        res[cfg.name] = {
-            "call": "ttt_chunk_fwd", "ms": ms, "tokens_per_s": cfg.B * cfg.T / (ms * 1e-3),
-            "dtype": cfg.dtype, "hbm_frac": w["fwd_bytes"] / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
-        }
-        if cfg.dtype == "bf16":
-            res[cfg.name].update(path="tcgen05", tc_frac=flops / (peaks["bf16_tflops"] * 1e12))
-        else:
-            # fp32 runs on CUDA cores: 148 SMs x 128 FMA lanes x 2 flops x 1.965 GHz
-            res[cfg.name].update(path="simt", alu_frac=flops / FP32_ALU_PEAK)
+        steps, warmup = (3, 1) if with_bwd else (10, 3)
+        entry = {"dtype": cfg.dtype, "decay": "vector" if cfg.decay == "vector" else "scalar"}
+        calls = [("ttt_chunk_fwd", layer.fwd, w["fwd_flops"], w["fwd_bytes"])]
+        if with_bwd:
+            layer.fwd()
+            calls.append(("ttt_chunk_bwd", layer.bwd, w["bwd_flops"], w["bwd_bytes"]))
+        total = 0.0
+        for call, fn, fl, by in calls:
+            ms = _event_ms(fn, steps, warmup)
+            total += ms
+            path = _path(cfg, call)
+            d = {"ms": ms, "path": path, "hbm_frac": by / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9)}
+            if path == "tcgen05":
+                d["tc_frac"] = fl / (ms * 1e-3) / (peaks["bf16_tflops"] * 1e12)
+            else:
+                # CUDA cores: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz
+                d["alu_frac"] = fl / (ms * 1e-3) / FP32_ALU_PEAK
+            entry[call] = d
+        entry["ms"] = total
+        entry["tokens_per_s"] = cfg.B * cfg.T / (total * 1e-3)
         if cfg.name == synth.TINY_FP32.name:
-            res[cfg.name]["note"] = "latency-bound correctness workload (two heads)"
+            entry["note"] = "latency-bound correctness workload (two heads)"
+        res[name] = entry
         del layer
         torch.cuda.empty_cache()
     return res
@@ -408,7 +442,7 @@ def main():
     ap.add_argument("--no-inplace", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
-                    help="skip the forward throughput of the other workloads")
+                    help="skip the throughput lines of the other workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -498,7 +532,7 @@ def main():
     del layer
     torch.cuda.empty_cache()
     if not args.no_configs:
-        out["other_configs"] = time_fwd_configs(ttt, peaks)
+        out["other_configs"] = time_other_configs(ttt, peaks)
     if not args.no_inplace:
         icfg, ims = time_inplace(ttt, steps=3, warmup=1)
         fl, by = inplace_work(icfg)

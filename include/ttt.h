@@ -11,8 +11,9 @@
  *    Linear), train-view backward of the inner loss (MSE or inner product), and the
  *    causal query-view readout O = Q W_start - Tril(Q Khat^T) dVhat, ending with the
  *    state transition W_end = W_start - Khat^T dVhat. The learning rate is
- *    eta_t = 2 sigmoid(beta_t + b) (section "内部学习规则与学习率参数化"); scalar
- *    decay shrinks past writes (section "权重衰减").
+ *    eta_t = 2 sigmoid(beta_t + b) (section "内部学习规则与学习率参数化"); a decay
+ *    shrinks past writes (section "权重衰减"): scalar, or per feature (vector decay, one
+ *    factor per key feature scaling that row of W).
  *  - In-Place TTT (page "In-Place Test-Time Training", section "核心方法和技术细节"):
  *    W_down of a gated MLP is the fast weight; per chunk O_i = Z_i W_i^T, then
  *    W_{i+1} = W_i + eta Vhat_i^T Z_i.
@@ -21,7 +22,8 @@
  * W0 = state at the chunk start, act = identity or SiLU):
  *     z_t  = k_t W0;   g_t = a_t * act'(z_t),  a_t = act(z_t) - v_t (MSE) or -v_t (IP)
  *     eta_t = 2 sigmoid(beta_t + lr_bias)
- *     W_t  = gamma_t W_{t-1} - eta_t k_t^T g_t          (gamma_t = 1 without decay)
+ *     W_t  = gamma_t W_{t-1} - eta_t k_t^T g_t          (gamma_t = 1 without decay;
+ *                                                       diag(gamma_t) for a vector decay)
  *     o_t  = act(q_t W_t)                              (the token reads its own write)
  * which the kernels evaluate in the chunk dual form.
  *
@@ -62,6 +64,7 @@ typedef enum {
 typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;    /* type of Q,K,V,O,dO,dQ,dK,dV     */
 typedef enum { TTT_LOSS_MSE = 0, TTT_LOSS_IP = 1 } ttt_loss;
 typedef enum { TTT_ACT_ID = 0, TTT_ACT_SILU = 1 } ttt_act;
+typedef enum { TTT_DECAY_SCALAR = 0, TTT_DECAY_VECTOR = 1 } ttt_decay;
 
 /* Shape and variant of one TTT layer call. */
 typedef struct {
@@ -73,12 +76,15 @@ typedef struct {
   int loss;        /* ttt_loss: MSE = 1/2||act(z)-v||^2, IP = -<act(z), v>               */
   int act;         /* ttt_act applied to both the train view and the query view         */
   float lr_bias;   /* b in eta_t = 2 sigmoid(beta_t + b)                                 */
+  int decay;       /* ttt_decay: layout of gamma (zero-initialised configs: scalar)      */
 } ttt_config;
 
 /* Layouts (all contiguous):
  *   Q, K, dQ, dK        [B, H, T, dk]   dtype
  *   V, O, dO, dV        [B, H, T, dv]   dtype
- *   beta, gamma, dbeta  [B, H, T]       float32   (gamma NULL = no decay, gamma == 1)
+ *   beta, dbeta         [B, H, T]       float32
+ *   gamma, dgamma       [B, H, T] (scalar decay) or [B, H, T, dk] (vector decay)  float32;
+ *                       gamma NULL = no decay (gamma == 1)
  *   W0, W_final, dW_final, dW0   [B, H, dk, dv]  float32, row index = key feature
  *   W_chunks            [B, H, T/C, dk, dv]  dtype: the state at the start of every chunk
  *   G_saved             [B, H, T, dv]   dtype: G of every token, the value the token's write
@@ -97,8 +103,9 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd);
  *  out: O; W_final (nullable) = state after the last token; W_chunks (nullable) = chunk-start
  *       states, needed by ttt_chunk_bwd; G_saved (nullable) = G of every token, which
  *       ttt_chunk_bwd then reads instead of rebuilding it.
- * bf16 configs with dk == dv in {64, 128} and C in {128, 256} run on the tcgen05 kernel;
- * other shapes (dk, dv <= 128, C <= 256) and all float32 configs run on the SIMT kernels. */
+ * bf16 configs with dk == dv in {64, 128}, C in {128, 256} and a scalar decay (or none) run on
+ * the tcgen05 kernel; other shapes (dk, dv <= 128, C <= 256), all float32 configs and the
+ * vector decay run on the SIMT kernels. */
 ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0, void* O,
                          float* W_final, void* W_chunks, void* G_saved, void* workspace,
@@ -115,7 +122,11 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
  * The decay gradient follows from L_s = sum_{t<=s} log gamma_t (chunk-local): with Zq the
  * readout before the activation and dG the adjoint of G,
  *     dJ/dL_s = dZq_s . Zq_s - g_s . dG_s  (+ <W_end, dW_end> on the chunk's last token)
- *     dgamma_t = (1 / gamma_t) sum_{s >= t in the chunk} dJ/dL_s. */
+ *     dgamma_t = (1 / gamma_t) sum_{s >= t in the chunk} dJ/dL_s.
+ * For a vector decay L_s has one entry per key feature i and, with dZ the adjoint of
+ * Z = K W0,
+ *     dJ/dL_si = q_si dQ_si - k_si (dK_si - (dZ_s W0^T)_i)  (+ row i of <W_end, dW_end>)
+ *     dgamma_ti = (1 / gamma_ti) sum_{s >= t in the chunk} dJ/dL_si. */
 ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0,
                          const void* W_chunks, const void* G_saved, const void* dO,

@@ -10,7 +10,8 @@ the CUDA path and the CPU oracle receive the tensors produced here.
 
 Layouts
     Q, K, V, O, dO : [B, H, T, d]   (d = d_k for Q/K, d_v for V/O/dO)
-    beta, gamma    : [B, H, T]      float32
+    beta           : [B, H, T]      float32
+    gamma          : [B, H, T] (scalar decay) or [B, H, T, d_k] (vector decay) float32
     W0, dW_T       : [B, H, d_k, d_v] float32
     In-Place: Z [T, d_ff] bf16, Vhat [T, d_model] bf16, W [d_model, d_ff] f32
 
@@ -39,7 +40,8 @@ class TTTConfig:
     dtype: str          # "f32" or "bf16": storage type of Q, K, V, O, dO, dQ, dK, dV
     loss: str           # "mse" or "ip"
     act: str            # "id" or "silu"
-    decay: bool         # scalar per-token decay gamma_t (False: gamma == 1, passed as NULL)
+    decay: bool | str   # True: scalar decay gamma_t [B,H,T]; "vector": one decay per key feature
+                        # [B,H,T,dk]; False: gamma == 1, passed as NULL
     w0_std: float       # std of the initial fast weight (0 -> zeros)
     normalize: str      # "qkv": L2-normalise rows of Q, K and V; "qk": of Q and K only
     lr_bias: float = LR_BIAS_ETA0_0P1
@@ -130,7 +132,12 @@ def ttt_inputs(cfg: TTTConfig, device="cpu", seed: int | None = None) -> dict:
     if cfg.normalize == "qkv":
         v = _l2_rows(v)
     beta = _randn((B, H, T), g, device)
-    gamma = torch.sigmoid(3.0 + 0.5 * _randn((B, H, T), g, device)) if cfg.decay else None
+    if cfg.decay == "vector":
+        gamma = torch.sigmoid(3.0 + 0.5 * _randn((B, H, T, dk), g, device))
+    elif cfg.decay:
+        gamma = torch.sigmoid(3.0 + 0.5 * _randn((B, H, T), g, device))
+    else:
+        gamma = None
     if cfg.w0_std > 0:
         w0 = cfg.w0_std * _randn((B, H, dk, dv), g, device)
     else:

@@ -14,7 +14,7 @@ def lr_bias32(cfg):
 
 def abi_config(cfg):
     return ttt.make_config(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C, cfg.dtype, cfg.loss, cfg.act,
-                           cfg.lr_bias)
+                           cfg.lr_bias, "vector" if cfg.decay == "vector" else "scalar")
 
 
 def gpu_inputs(cfg, seed=None):
@@ -51,7 +51,7 @@ def run_bwd(cfg, inp, W_chunks, G=None, fwd=None):
                dW0=torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32))
     want_dg = fwd is not None and inp["gamma"] is not None
     if want_dg:
-        out["dgamma"] = torch.empty((B, H, T), device="cuda", dtype=torch.float32)
+        out["dgamma"] = torch.empty(inp["gamma"].shape, device="cuda", dtype=torch.float32)
     n = ttt.ttt_workspace_bytes(c, 2 if G is not None else 1)
     ws = torch.empty(max(n, 16), device="cuda", dtype=torch.uint8)
     ttt.ttt_chunk_bwd(c, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], inp["W0"],

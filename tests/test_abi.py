@@ -105,6 +105,23 @@ def test_bwd_requires_chunk_states_and_workspace():
     assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *dg, A, need, None) == ttt.ERR_INVALID_ARG
 
 
+def test_decay_kind_is_checked_and_vector_decay_leaves_the_tensor_core_path():
+    bad = _cfg()
+    bad.decay = 2
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_workspace_bytes(bad, 0)
+    # a shape the tensor-core backward takes with a scalar decay needs its chunk-end adjoint
+    # scratch; with a vector decay the SIMT backward's per-head scratch is sized instead
+    tc = _cfg(dtype="bf16", dk=128, dv=128, C=256, T=512)
+    vec = _cfg(dtype="bf16", dk=128, dv=128, C=256, T=512, decay="vector")
+    assert ttt.ttt_workspace_bytes(vec, 1) != ttt.ttt_workspace_bytes(tc, 1)
+    # the fixed-scratch backward serves tensor-core configs only
+    A = 4096
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(vec), A, A, A, A, A, A, A, None, A, None, None,
+                                       None, A, A, A, A, A, None, None)
+    assert st == ttt.ERR_UNSUPPORTED
+
+
 def test_tc_bwd_workspace_covers_the_decay_gradient():
     # the query's backward figure includes the float per token that only dgamma calls use
     tc = _cfg(dtype="bf16", dk=128, dv=128, C=256, T=512)

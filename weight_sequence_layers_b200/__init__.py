@@ -25,6 +25,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ER
 F32, BF16 = 0, 1
 LOSS = {"mse": 0, "ip": 1}
 ACT = {"id": 0, "silu": 1}
+DECAY = {"scalar": 0, "vector": 1}
 
 
 class TTTError(RuntimeError):
@@ -37,7 +38,7 @@ class ttt_config(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("loss", ctypes.c_int), ("act", ctypes.c_int),
-                ("lr_bias", ctypes.c_float)]
+                ("lr_bias", ctypes.c_float), ("decay", ctypes.c_int)]
 
 
 _p, _i, _u, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_float, ctypes.c_size_t
@@ -92,9 +93,12 @@ def _check(status: int, where: str):
         raise TTTError(status, where)
 
 
-def make_config(B, H, T, dk, dv, C, dtype="bf16", loss="mse", act="id", lr_bias=0.0) -> ttt_config:
+def make_config(B, H, T, dk, dv, C, dtype="bf16", loss="mse", act="id", lr_bias=0.0,
+                decay="scalar") -> ttt_config:
+    """decay: "scalar" (gamma [B,H,T], or no gamma) or "vector" (gamma [B,H,T,dk])."""
     return ttt_config(B, H, T, dk, dv, C, F32 if dtype in ("f32", F32) else BF16,
-                      LOSS.get(loss, loss), ACT.get(act, act), float(lr_bias))
+                      LOSS.get(loss, loss), ACT.get(act, act), float(lr_bias),
+                      DECAY.get(decay, decay))
 
 
 def ttt_workspace_bytes(cfg: ttt_config, for_bwd: int) -> int:

@@ -53,6 +53,7 @@ ttt_status check_config(const ttt_config* c) {
   if (c->loss != TTT_LOSS_MSE && c->loss != TTT_LOSS_IP) return TTT_ERR_INVALID_ARG;
   if (c->act != TTT_ACT_ID && c->act != TTT_ACT_SILU) return TTT_ERR_INVALID_ARG;
   if (!isfinite(c->lr_bias)) return TTT_ERR_INVALID_ARG;
+  if (c->decay != TTT_DECAY_SCALAR && c->decay != TTT_DECAY_VECTOR) return TTT_ERR_INVALID_ARG;
   if ((long long)c->B * c->H * c->T * (c->dk > c->dv ? c->dk : c->dv) > (1ll << 40))
     return TTT_ERR_INVALID_ARG;
   return TTT_OK;
@@ -70,6 +71,7 @@ LayerArgs args_of(const ttt_config* c) {
   a.loss = c->loss;
   a.act = c->act;
   a.lr_bias = c->lr_bias;
+  a.gvec = c->decay == TTT_DECAY_VECTOR;
   return a;
 }
 

@@ -9,6 +9,7 @@ namespace tttk {
 struct LayerArgs {
   int B, H, T, dk, dv, C, dtype, loss, act;
   float lr_bias;
+  int gvec;  // gamma is [B, H, T, dk]: one decay per key feature
   const void *Q, *K, *V;
   const float *beta, *gamma, *W0;
   void* O;

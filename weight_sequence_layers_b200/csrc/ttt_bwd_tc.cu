@@ -1186,7 +1186,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool tc_bwd_supported(const LayerArgs& a) {
-  return a.dtype == 1 && a.act == 0 && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
+  return a.dtype == 1 && a.act == 0 && !a.gvec && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
          (a.C == 128 || a.C == 256) && a.T % a.C == 0;
 }
 

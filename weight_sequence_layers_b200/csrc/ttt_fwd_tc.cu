@@ -594,7 +594,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool tc_fwd_supported(const LayerArgs& a) {
-  return a.dtype == 1 && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
+  return a.dtype == 1 && !a.gvec && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
          (a.C == 128 || a.C == 256) && a.T % a.C == 0;
 }
 

@@ -9,7 +9,11 @@
 //     O  = act(diag(Gamma) Q W0 - S G)               (query view)
 //     W_end = Gamma_C W0 - K^T diag(u) G,  u_r = eta_r exp(L_C - L_r)
 // with eta = 2 sigmoid(beta + b) (section "内部学习规则与学习率参数化") and
-// L_s = sum_{t<=s} log gamma_t (section "权重衰减").
+// L_s = sum_{t<=s} log gamma_t (section "权重衰减"). With a per-feature (vector) decay, L_s has one
+// entry per key feature i and scales row i of W, so the decay enters inside the contractions over
+// the key features:
+//     S_sr = eta_r sum_i q_si k_ri exp(L_si - L_ri),   Gamma Q W0 -> (Q * exp(L)) W0,
+//     W_end = diag(exp(L_C)) W0 - sum_r eta_r (k_r * exp(L_C - L_r))^T g_r.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -42,21 +46,30 @@ __device__ __forceinline__ float act2(int act, float z) {
 }
 
 struct Dims {
-  int T, dk, dv, C, loss, act, has_gamma;
+  int T, dk, dv, C, loss, act, has_gamma, gvec;
   float lr_bias;
 };
 
-// eta_s and the chunk-local log-decay prefix L_s for the C tokens of chunk c of head bh.
+// Entries of the log-decay prefix per chunk position: one, or one per key feature.
+__host__ __device__ inline int lwidth(const Dims& d) { return d.gvec ? d.dk : 1; }
+
+// Prefix L at chunk position s for key feature i (the same for every i with a scalar decay).
+__device__ __forceinline__ float Lat(const Dims& d, const float* L, int s, int i) {
+  return d.gvec ? L[s * d.dk + i] : L[s];
+}
+
+// eta_s and the chunk-local log-decay prefix L for the C tokens of chunk c of head bh; L is
+// [C] for a scalar decay and [C][dk] for a per-feature decay.
 __device__ void chunk_scans(const Dims& d, const float* beta, const float* gamma, int bh, int c,
                             float* eta, float* L) {
   const size_t t0 = (size_t)bh * d.T + (size_t)c * d.C;
-  for (int s = threadIdx.x; s < d.C; s += blockDim.x) {
-    eta[s] = 2.f * sigm(beta[t0 + s] + d.lr_bias);
-    L[s] = d.has_gamma ? logf(gamma[t0 + s]) : 0.f;
-  }
+  const int w = lwidth(d);
+  for (int s = threadIdx.x; s < d.C; s += blockDim.x) eta[s] = 2.f * sigm(beta[t0 + s] + d.lr_bias);
+  for (int e = threadIdx.x; e < d.C * w; e += blockDim.x)
+    L[e] = d.has_gamma ? logf(gamma[t0 * w + e]) : 0.f;
   __syncthreads();
-  if (threadIdx.x == 0)
-    for (int s = 1; s < d.C; ++s) L[s] += L[s - 1];
+  for (int i = threadIdx.x; i < w; i += blockDim.x)
+    for (int s = 1; s < d.C; ++s) L[s * w + i] += L[(s - 1) * w + i];
   __syncthreads();
 }
 
@@ -73,7 +86,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
   float* G = Ws + dk * kNvs;         // [C][kNvs]
   float* S = G + C * kNvs;           // [kRows][C]
   float* eta = S + kRows * C;        // [C]
-  float* L = eta + C;                // [C]
+  float* L = eta + C;                // [C] or [C][dk]
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
   for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
     const int i = e / nv, j = e % nv;
@@ -109,8 +122,14 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
           const TI* qs = Q + qk0 + (tc + s) * dk;
           const TI* kr = K + qk0 + (tc + r) * dk;
           float p = 0.f;
-          for (int i = 0; i < dk; ++i) p += ldf(qs + i) * ldf(kr + i);
-          v = eta[r] * expf(L[s] - L[r]) * p;
+          if (d.gvec) {
+            for (int i = 0; i < dk; ++i)
+              p += ldf(qs + i) * ldf(kr + i) * expf(L[s * dk + i] - L[r * dk + i]);
+            v = eta[r] * p;
+          } else {
+            for (int i = 0; i < dk; ++i) p += ldf(qs + i) * ldf(kr + i);
+            v = eta[r] * expf(L[s] - L[r]) * p;
+          }
         }
         S[sr * C + r] = v;
       }
@@ -119,21 +138,26 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
         const int sr = e / nv, j = e % nv, s = s0 + sr;
         if (s >= C) continue;
         const TI* qs = Q + qk0 + (tc + s) * dk;
-        float y = 0.f;
-        for (int i = 0; i < dk; ++i) y += ldf(qs + i) * Ws[i * kNvs + j];
-        float acc = expf(L[s]) * y;
+        float acc = 0.f;
+        if (d.gvec) {
+          for (int i = 0; i < dk; ++i) acc += ldf(qs + i) * expf(L[s * dk + i]) * Ws[i * kNvs + j];
+        } else {
+          for (int i = 0; i < dk; ++i) acc += ldf(qs + i) * Ws[i * kNvs + j];
+          acc *= expf(L[s]);
+        }
         for (int r = 0; r <= s; ++r) acc -= S[sr * C + r] * G[r * kNvs + j];
         stf(&O[v0 + (tc + s) * dv + j0 + j], actf(d.act, acc));
       }
       __syncthreads();
     }
     // state transition
-    const float LC = L[C - 1];
     for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
       const int i = e / nv, j = e % nv;
+      const float LC = Lat(d, L, C - 1, i);
       float w = expf(LC) * Ws[i * kNvs + j];
       for (int r = 0; r < C; ++r)
-        w -= eta[r] * expf(LC - L[r]) * ldf(K + qk0 + (tc + r) * dk + i) * G[r * kNvs + j];
+        w -= eta[r] * expf(LC - Lat(d, L, r, i)) * ldf(K + qk0 + (tc + r) * dk + i) *
+             G[r * kNvs + j];
       Ws[i * kNvs + j] = w;
     }
     __syncthreads();
@@ -147,9 +171,11 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
 
 // Per-head float32 scratch of the backward (in units of floats): Wh, Wn, W0 (dk x dv each),
 // Z, G, dZq, Y, dG, dZ, Zq (C x dv each), S, dS (C x C each), eta, L, deta, dL (C each), and
-// one float for the chunk-end term of the decay gradient.
-__host__ __device__ inline size_t bwd_head_floats(int C, int dk, int dv) {
-  return 3 * (size_t)dk * dv + 7 * (size_t)C * dv + 2 * (size_t)C * C + 4 * (size_t)C + 1;
+// one float for the chunk-end term of the decay gradient; with a per-feature decay also the
+// prefix L and two parts of dJ/dL (C x dk each) and the chunk-end term per feature (dk).
+__host__ __device__ inline size_t bwd_head_floats(int C, int dk, int dv, bool gvec) {
+  return 3 * (size_t)dk * dv + 7 * (size_t)C * dv + 2 * (size_t)C * C + 4 * (size_t)C + 1 +
+         (gvec ? 3 * (size_t)C * dk + dk : 0);
 }
 
 // Analytic backward of the chunk dual form, reverse over chunks; one block per head.
@@ -161,7 +187,7 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
     float* dbeta, float* dW0, float* dgamma, float* ws) {
   const int bh = blockIdx.x;
   const int dk = d.dk, dv = d.dv, C = d.C, NC = d.T / d.C;
-  float* Wh = ws + (size_t)bh * bwd_head_floats(C, dk, dv);
+  float* Wh = ws + (size_t)bh * bwd_head_floats(C, dk, dv, d.gvec);
   float* Wn = Wh + dk * dv;
   float* W0 = Wn + dk * dv;  // float copy of the chunk-start state
   float* Z = W0 + dk * dv;
@@ -178,6 +204,10 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
   float* ZQ = deta + C;
   float* dL = ZQ + C * dv;
   float* wend = dL + C;  // <W_end, dW_end> of the chunk
+  float* dLq = wend + 1;       // per-feature decay: q_si dQ_si  [C][dk]
+  float* dLk = dLq + C * dk;   //                    -k_si (dK_si - (dZ_s W0^T)_i)  [C][dk]
+  float* wendv = dLk + C * dk; //                    row sums of W_end * dW_end  [dk]
+  if (d.gvec) L = wendv + dk;  //                    log-decay prefix  [C][dk]
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
   for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
     Wh[e] = dWf ? dWf[(size_t)bh * dk * dv + e] : 0.f;
@@ -187,7 +217,6 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
       W0[e] = ldf(Wc + ((size_t)bh * NC + c) * dk * dv + e);
     chunk_scans(d, beta, gamma, bh, c, eta, L);  // ends with __syncthreads
-    const float LC = L[C - 1];
     // Z = K W0, G
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
       const int s = e / dv, j = e % dv;
@@ -205,25 +234,29 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       if (r <= s) {
         float p = 0.f;
         for (int i = 0; i < dk; ++i)
-          p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i);
-        v = eta[r] * expf(L[s] - L[r]) * p;
+          p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i) *
+               (d.gvec ? expf(L[s * dk + i] - L[r * dk + i]) : 1.f);
+        v = eta[r] * p * (d.gvec ? 1.f : expf(L[s] - L[r]));
       }
       S[e] = v;
     }
-    // Y = K Wh
+    // Y_r = (k_r * exp(L_C - L_r)) Wh: the key's route into the chunk-end state
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
       const int r = e / dv, j = e % dv;
       float y = 0.f;
-      for (int i = 0; i < dk; ++i) y += ldf(K + qk0 + (tc + r) * dk + i) * Wh[i * dv + j];
-      Y[e] = y;
+      for (int i = 0; i < dk; ++i)
+        y += ldf(K + qk0 + (tc + r) * dk + i) * Wh[i * dv + j] *
+             (d.gvec ? expf(Lat(d, L, C - 1, i) - L[r * dk + i]) : 1.f);
+      Y[e] = d.gvec ? y : y * expf(L[C - 1] - L[r]);
     }
     __syncthreads();
     // dZq = dO * act'(Zq), Zq = Gamma Q W0 - S G
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
       const int s = e / dv, j = e % dv;
       float y = 0.f;
-      for (int i = 0; i < dk; ++i) y += ldf(Q + qk0 + (tc + s) * dk + i) * W0[i * dv + j];
-      float zq = expf(L[s]) * y;
+      for (int i = 0; i < dk; ++i)
+        y += ldf(Q + qk0 + (tc + s) * dk + i) * W0[i * dv + j] * (d.gvec ? expf(L[s * dk + i]) : 1.f);
+      float zq = d.gvec ? y : expf(L[s]) * y;
       for (int r = 0; r <= s; ++r) zq -= S[s * C + r] * G[r * dv + j];
       ZQ[e] = zq;
       DZQ[e] = ldf(dO + v0 + (tc + s) * dv + j) * act1(d.act, zq);
@@ -242,7 +275,7 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       const int r = e / dv, j = e % dv;
       float g = 0.f;
       for (int s = r; s < C; ++s) g -= S[s * C + r] * DZQ[s * dv + j];
-      g -= eta[r] * expf(LC - L[r]) * Y[e];
+      g -= eta[r] * Y[e];
       DG[e] = g;
     }
     __syncthreads();
@@ -253,7 +286,7 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       acc /= eta[r];
       float yg = 0.f;
       for (int j = 0; j < dv; ++j) yg += Y[r * dv + j] * G[r * dv + j];
-      deta[r] = acc - expf(LC - L[r]) * yg;
+      deta[r] = acc - yg;
     }
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
       const int r = e / dv, j = e % dv;
@@ -265,33 +298,60 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       stf(&dV[v0 + (tc + r) * dv + j], -da);
     }
     __syncthreads();
-    // dQ = diag(Gamma) dZq W0^T + (dS * M) K
+    // dQ = diag(Gamma) dZq W0^T + (dS * M) K   (decay of feature i inside, per feature)
     for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
       const int s = e / dk, i = e % dk;
+      const float Ls = Lat(d, L, s, i);
       float a1 = 0.f;
       for (int j = 0; j < dv; ++j) a1 += DZQ[s * dv + j] * W0[i * dv + j];
-      float acc = expf(L[s]) * a1;
+      float acc = expf(Ls) * a1;
       for (int r = 0; r <= s; ++r)
-        acc += DS[s * C + r] * eta[r] * expf(L[s] - L[r]) * ldf(K + qk0 + (tc + r) * dk + i);
+        acc += DS[s * C + r] * eta[r] * expf(Ls - Lat(d, L, r, i)) * ldf(K + qk0 + (tc + r) * dk + i);
       stf(&dQ[qk0 + (tc + s) * dk + i], acc);
+      if (d.gvec && dgamma) dLq[e] = ldf(Q + qk0 + (tc + s) * dk + i) * acc;
     }
     // dK = (dS * M)^T Q - diag(u) G Wh^T + dZ W0^T
     for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
       const int r = e / dk, i = e % dk;
+      const float Lr = Lat(d, L, r, i);
       float acc = 0.f;
       for (int s = r; s < C; ++s)
-        acc += DS[s * C + r] * eta[r] * expf(L[s] - L[r]) * ldf(Q + qk0 + (tc + s) * dk + i);
+        acc += DS[s * C + r] * eta[r] * expf(Lat(d, L, s, i) - Lr) * ldf(Q + qk0 + (tc + s) * dk + i);
       float gw = 0.f, zw = 0.f;
       for (int j = 0; j < dv; ++j) {
         gw += G[r * dv + j] * Wh[i * dv + j];
         zw += DZ[r * dv + j] * W0[i * dv + j];
       }
-      acc += -eta[r] * expf(LC - L[r]) * gw + zw;
-      stf(&dK[qk0 + (tc + r) * dk + i], acc);
+      acc += -eta[r] * expf(Lat(d, L, C - 1, i) - Lr) * gw;
+      if (d.gvec && dgamma) dLk[e] = -ldf(K + qk0 + (tc + r) * dk + i) * acc;
+      stf(&dK[qk0 + (tc + r) * dk + i], acc + zw);
     }
     for (int r = threadIdx.x; r < C; r += blockDim.x)
       dbeta[(size_t)bh * d.T + tc + r] = deta[r] * eta[r] * (1.f - 0.5f * eta[r]);
-    if (dgamma) {
+    if (dgamma && d.gvec) {
+      // per feature: dJ/dL_si = q_si dQ_si - k_si (dK_si - (dZ_s W0^T)_i), plus the row-i part
+      // of <W_end, dW_end> on the last token; dgamma_ti is the suffix sum over the chunk divided
+      // by gamma_ti
+      for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        float acc = 0.f;
+        if (c + 1 < NC || dWf)
+          for (int j = 0; j < dv; ++j) {
+            const float we = c + 1 < NC ? ldf(Wc + (((size_t)bh * NC + c + 1) * dk + i) * dv + j)
+                                        : Wfin[((size_t)bh * dk + i) * dv + j];
+            acc += we * Wh[i * dv + j];
+          }
+        wendv[i] = acc;
+      }
+      __syncthreads();
+      for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        float acc = wendv[i];
+        for (int s2 = C - 1; s2 >= 0; --s2) {
+          acc += dLq[s2 * dk + i] + dLk[s2 * dk + i];
+          const size_t ti = ((size_t)bh * d.T + tc + s2) * dk + i;
+          dgamma[ti] = acc / gamma[ti];
+        }
+      }
+    } else if (dgamma) {
       // dJ/dL_s = dZq_s . Zq_s - g_s . dG_s, plus <W_end, dW_end> on the last token; dgamma_t is
       // the suffix sum over the chunk divided by gamma_t
       for (int s2 = threadIdx.x; s2 < C; s2 += blockDim.x) {
@@ -322,9 +382,9 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
     // dW at the chunk start = Gamma_C Wh + Q^T diag(Gamma) dZq + K^T dZ
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
       const int i = e / dv, j = e % dv;
-      float acc = expf(LC) * Wh[e];
+      float acc = expf(Lat(d, L, C - 1, i)) * Wh[e];
       for (int s = 0; s < C; ++s)
-        acc += expf(L[s]) * ldf(Q + qk0 + (tc + s) * dk + i) * DZQ[s * dv + j] +
+        acc += expf(Lat(d, L, s, i)) * ldf(Q + qk0 + (tc + s) * dk + i) * DZQ[s * dv + j] +
                ldf(K + qk0 + (tc + s) * dk + i) * DZ[s * dv + j];
       Wn[e] = acc;
     }
@@ -336,11 +396,13 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
 }
 
 Dims dims_of(const LayerArgs& a) {
-  return Dims{a.T, a.dk, a.dv, a.C, a.loss, a.act, a.gamma != nullptr, a.lr_bias};
+  return Dims{a.T, a.dk, a.dv, a.C, a.loss, a.act, a.gamma != nullptr, a.gvec, a.lr_bias};
 }
 
 size_t fwd_smem_bytes(const LayerArgs& a) {
-  return sizeof(float) * ((size_t)a.dk * kNvs + (size_t)a.C * kNvs + (size_t)kRows * a.C + 2 * a.C);
+  const size_t lw = a.gvec ? a.dk : 1;
+  return sizeof(float) *
+         ((size_t)a.dk * kNvs + (size_t)a.C * kNvs + (size_t)kRows * a.C + a.C + a.C * lw);
 }
 
 }  // namespace
@@ -352,7 +414,7 @@ bool simt_supported(const LayerArgs& a) {
 size_t simt_fwd_workspace(const LayerArgs&) { return 0; }
 
 size_t simt_bwd_workspace(const LayerArgs& a) {
-  return sizeof(float) * bwd_head_floats(a.C, a.dk, a.dv) * a.B * a.H;
+  return sizeof(float) * bwd_head_floats(a.C, a.dk, a.dv, a.gvec) * a.B * a.H;
 }
 
 cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
