@@ -8,7 +8,9 @@ cpu_baseline / reference leg may import this package. The product library
   (fp64 state and arithmetic; ttt_fwd_f32 is the fp32-state build).
 * inplace_fwd follows In-Place TTT (page "In-Place Test-Time Training",
   section "核心方法和技术细节", the chunkwise apply-then-update rule
-  W^(i+1) = W^(i) + eta * Vhat_[i]^T Z_[i]) with fp64 numpy matmuls.
+  W^(i+1) = W^(i) + eta * Vhat_[i]^T Z_[i]) with fp64 numpy matmuls;
+  inplace_bwd is the reverse-mode of that loop (the pages print no backward),
+  inplace_bwd_dz_tokens evaluates sampled rows of its dZ at any size.
 
 Every function here is pinned by tests/test_oracle_pins.py; no function is
 "parity unpinned" except for absolute agreement with the authors' own
@@ -161,3 +163,66 @@ def inplace_fwd(Z, Vhat, W, *, C: int, lr: float, rows=None):
         o[i * C:(i + 1) * C] = zi @ w.T          # apply with the current fast weight
         w += lr * (vh[i * C:(i + 1) * C].T @ zi)  # then update it with this chunk
     return o, w
+
+
+def inplace_bwd(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, rows=None):
+    """Reverse-mode of inplace_fwd for J = sum_i <dO_i, O_i> + <dW_final, W_final> (fp64).
+
+    The chunks are walked backwards carrying Wh, the adjoint of the fast weight (dW_final, or
+    zero, after the last chunk). With W_i the weight chunk i applied:
+        O_i = Z_i W_i^T                  gives  dZ_i += dO_i W_i,           Wh += dO_i^T Z_i
+        W_{i+1} = W_i + lr Vhat_i^T Z_i  gives  dZ_i += lr Vhat_i Wh_{i+1},  dVhat_i = lr Z_i Wh_{i+1}^T
+    (Wh_{i+1} is the adjoint before chunk i's own O_i term is added). Returns dict dZ [T, d_ff],
+    dVhat [T, d_model] and dW [d_model, d_ff], the gradient with respect to the initial W.
+    `rows` restricts the computation to those rows of W (columns of Vhat and dO): dVhat[:, rows]
+    and dW[rows] are then exact, and dZ, a sum over every row, is not returned (None).
+    """
+    z = _np(Z, np.float64)
+    vh = _np(Vhat, np.float64)
+    w = _np(W, np.float64)
+    do = _np(dO, np.float64)
+    dwf = np.zeros_like(w) if dW_final is None else _np(dW_final, np.float64)
+    if rows is not None:
+        rows = np.asarray(rows)
+        vh, do, w, dwf = vh[:, rows], do[:, rows], w[rows], dwf[rows]
+    T = z.shape[0]
+    if T % C:
+        raise ValueError("T must be a multiple of C")
+    applied = []
+    cur = w.copy()
+    for i in range(T // C):
+        sl = slice(i * C, (i + 1) * C)
+        applied.append(cur.copy())
+        cur = cur + lr * (vh[sl].T @ z[sl])
+    wh = dwf.copy()
+    dz = np.zeros_like(z) if rows is None else None
+    dvh = np.zeros_like(vh)
+    for i in reversed(range(T // C)):
+        sl = slice(i * C, (i + 1) * C)
+        if dz is not None:
+            dz[sl] = do[sl] @ applied[i] + lr * (vh[sl] @ wh)
+        dvh[sl] = lr * (z[sl] @ wh.T)
+        wh = wh + do[sl].T @ z[sl]
+    return dict(dZ=dz, dVhat=dvh, dW=wh)
+
+
+def inplace_bwd_dz_tokens(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, tokens):
+    """Rows `tokens` of dZ from inplace_bwd, by expanding both sums (fp64): for token t of
+    chunk i, W_i = W + lr Vhat_{<i}^T Z_{<i} and Wh_{i+1} = dW_final + dO_{>i}^T Z_{>i} (<i: the
+    tokens of the chunks before i, >i: after it), so
+        dZ_t = dO_t W + lr (dO_t Vhat_{<i}^T) Z_{<i} + lr Vhat_t dW_final + lr (Vhat_t dO_{>i}^T) Z_{>i}.
+    Cheap for a few tokens at any size: no d_model x d_ff product is formed."""
+    z = _np(Z, np.float64)
+    vh = _np(Vhat, np.float64)
+    w = _np(W, np.float64)
+    do = _np(dO, np.float64)
+    out = np.empty((len(tokens), z.shape[1]))
+    for n, t in enumerate(tokens):
+        i = t // C
+        lo, hi = i * C, (i + 1) * C
+        row = do[t] @ w + lr * ((vh[:lo] @ do[t]) @ z[:lo])
+        if dW_final is not None:
+            row = row + lr * (vh[t] @ _np(dW_final, np.float64))
+        row = row + lr * ((do[hi:] @ vh[t]) @ z[hi:])
+        out[n] = row
+    return out

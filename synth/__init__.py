@@ -13,7 +13,7 @@ Layouts
     beta           : [B, H, T]      float32
     gamma          : [B, H, T] (scalar decay) or [B, H, T, d_k] (vector decay) float32
     W0, dW_T       : [B, H, d_k, d_v] float32
-    In-Place: Z [T, d_ff] bf16, Vhat [T, d_model] bf16, W [d_model, d_ff] f32
+    In-Place: Z [T, d_ff] bf16, Vhat [T, d_model] bf16, W [d_model, d_ff] f32, dO [T, d_model] bf16
 
 Distribution notation: N(mu, s) takes s as the standard deviation.
 """
@@ -153,7 +153,9 @@ def ttt_inputs(cfg: TTTConfig, device="cpu", seed: int | None = None) -> dict:
 
 def inplace_inputs(cfg: InPlaceConfig, device="cpu", seed: int | None = None) -> dict:
     """Draw one seeded In-Place TTT workload: Z = SiLU(N(0,1)) * N(0,1) [T, d_ff] bf16,
-    Vhat ~ N(0, 0.02) [T, d_model] bf16 and W_down ~ N(0, 0.02) [d_model, d_ff] float32."""
+    Vhat ~ N(0, 0.02) [T, d_model] bf16, W_down ~ N(0, 0.02) [d_model, d_ff] float32 and, for
+    the backward, an upstream gradient dO ~ N(0, 1) [T, d_model] bf16 (drawn last, so the
+    forward's tensors do not depend on it)."""
     seed = cfg.seed if seed is None else seed
     g = make_generator(seed, device)
     a = _randn((cfg.T, cfg.d_ff), g, device)
@@ -162,4 +164,5 @@ def inplace_inputs(cfg: InPlaceConfig, device="cpu", seed: int | None = None) ->
     z = z.to(torch.bfloat16)
     vhat = (0.02 * _randn((cfg.T, cfg.d_model), g, device)).to(torch.bfloat16)
     w = 0.02 * _randn((cfg.d_model, cfg.d_ff), g, device)
-    return dict(Z=z.contiguous(), Vhat=vhat.contiguous(), W=w.contiguous())
+    do = _randn((cfg.T, cfg.d_model), g, device).to(torch.bfloat16)
+    return dict(Z=z.contiguous(), Vhat=vhat.contiguous(), W=w.contiguous(), dO=do.contiguous())

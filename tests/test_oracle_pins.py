@@ -18,7 +18,9 @@
   of W, and finite differences including the per-feature decay gradient;
 * In-Place TTT (page "In-Place Test-Time Training", section "核心方法和技术细节"):
   associativity of the update, plain GEMM when C = T or eta = 0, and the
-  dual form with Z_i Z_j^T corrections.
+  dual form with Z_i Z_j^T corrections; its backward against finite
+  differences, the single-chunk closed form, and the row-subset and
+  sampled-token evaluations against the full one.
 """
 import itertools
 import math
@@ -471,3 +473,64 @@ def test_inplace_row_subset_is_exact():
     Os, WFs = oracle.inplace_fwd(Z, Vh, W, C=4, lr=0.1, rows=rows)
     np.testing.assert_array_equal(Os, O[:, rows])
     np.testing.assert_array_equal(WFs, WF[rows])
+
+
+def _inplace_objective(Z, Vh, W, dO, dWf, C, lr):
+    O, WF = oracle.inplace_fwd(Z, Vh, W, C=C, lr=lr)
+    return float((O * dO).sum() + (WF * dWf).sum())
+
+
+def test_inplace_backward_matches_finite_differences():
+    rng = np.random.default_rng(44)
+    T, d_ff, d_model, C, lr = 8, 5, 3, 2, 0.3
+    Z, Vh, W = _inplace_rand(rng, T, d_ff, d_model)
+    dO = rng.standard_normal((T, d_model))
+    dWf = rng.standard_normal((d_model, d_ff))
+    g = oracle.inplace_bwd(Z, Vh, W, dO, dWf, C=C, lr=lr)
+    h = 1e-6
+    for name, x, key in (("Z", Z, "dZ"), ("Vhat", Vh, "dVhat"), ("W", W, "dW")):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            jp = _inplace_objective(Z, Vh, W, dO, dWf, C, lr)
+            x[idx] = old - h
+            jm = _inplace_objective(Z, Vh, W, dO, dWf, C, lr)
+            x[idx] = old
+            fd[idx] = (jp - jm) / (2 * h)
+        err = np.abs(g[key] - fd).max() / np.abs(fd).max()
+        assert err < 1e-8, (name, err)
+
+
+def test_inplace_backward_single_chunk_closed_form():
+    # C = T: O = Z W^T, W_final = W + lr Vhat^T Z, so dZ = dO W + lr Vhat dWf,
+    # dVhat = lr Z dWf^T and dW = dWf + dO^T Z
+    rng = np.random.default_rng(45)
+    T, lr = 16, 0.07
+    Z, Vh, W = _inplace_rand(rng, T, 6, 4)
+    dO = rng.standard_normal((T, 4))
+    dWf = rng.standard_normal((4, 6))
+    g = oracle.inplace_bwd(Z, Vh, W, dO, dWf, C=T, lr=lr)
+    np.testing.assert_allclose(g["dZ"], dO @ W + lr * Vh @ dWf, atol=1e-12)
+    np.testing.assert_allclose(g["dVhat"], lr * Z @ dWf.T, atol=1e-12)
+    np.testing.assert_allclose(g["dW"], dWf + dO.T @ Z, atol=1e-12)
+
+
+def test_inplace_backward_row_subset_and_sampled_tokens_are_exact():
+    rng = np.random.default_rng(46)
+    T, d_ff, d_model, C, lr = 24, 7, 6, 4, 0.05
+    Z, Vh, W = _inplace_rand(rng, T, d_ff, d_model)
+    dO = rng.standard_normal((T, d_model))
+    dWf = rng.standard_normal((d_model, d_ff))
+    g = oracle.inplace_bwd(Z, Vh, W, dO, dWf, C=C, lr=lr)
+    rows = np.array([1, 4, 5])
+    gs = oracle.inplace_bwd(Z, Vh, W, dO, dWf, C=C, lr=lr, rows=rows)
+    assert gs["dZ"] is None
+    np.testing.assert_allclose(gs["dVhat"], g["dVhat"][:, rows], atol=1e-13)
+    np.testing.assert_allclose(gs["dW"], g["dW"][rows], atol=1e-13)
+    tokens = [0, 5, 13, 23]
+    dz = oracle.inplace_bwd_dz_tokens(Z, Vh, W, dO, dWf, C=C, lr=lr, tokens=tokens)
+    np.testing.assert_allclose(dz, g["dZ"][tokens], atol=1e-12)
+    dz0 = oracle.inplace_bwd_dz_tokens(Z, Vh, W, dO, None, C=C, lr=lr, tokens=tokens)
+    g0 = oracle.inplace_bwd(Z, Vh, W, dO, None, C=C, lr=lr)
+    np.testing.assert_allclose(dz0, g0["dZ"][tokens], atol=1e-12)
