@@ -159,18 +159,37 @@ ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q, const voi
                                  void* dQ, void* dK, void* dV, float* dbeta, float* dW0,
                                  float* dgamma, void* stream);
 
-/* Workspace bytes of inplace_ttt_fwd; (size_t)-1 for invalid sizes. */
+/* Workspace bytes of inplace_ttt_fwd and of inplace_ttt_bwd (the same figure);
+ * (size_t)-1 for invalid sizes. */
 size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C);
 
-/* In-Place TTT forward of the W_down fast weight (one sequence).
+/* In-Place TTT forward of the W_down fast weight (one sequence); page "In-Place Test-Time
+ * Training", section "核心方法和技术细节".
  *  Z     [T, d_ff]      bf16   (the gated-MLP activation phi(H W_gate^T) * (H W_up^T))
  *  Vhat  [T, d_model]   bf16   (the update target)
  *  W     [d_model, d_ff] float32, in: W_down at token 0, out: W_down after the last chunk
  *  O     [T, d_model]   bf16   out: O_i = Z_i W_i^T (apply, then update: no intra-chunk term)
+ *  W_chunks [T/C, d_model, d_ff] bf16, nullable; out: W_i, the weight chunk i applied (what
+ *        inplace_ttt_bwd reads; 2 bytes per weight per chunk)
  * Requirements: T % C == 0, C % 128 == 0, d_ff % 64 == 0, d_model % 128 == 0. */
 ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
-                           const void* Vhat, float* W, void* O, void* workspace,
+                           const void* Vhat, float* W, void* O, void* W_chunks, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* Backward of inplace_ttt_fwd (no counterpart on the page, which gives only the forward): the
+ * reverse-mode of the apply-then-update loop for J = sum_i <dO_i, O_i> + <dW_final, W_final>.
+ * With Wh the adjoint of the fast weight (dW_final, or 0, after the last chunk), chunk i from
+ * the last one down gives
+ *     dVhat_i = lr Z_i Wh_{i+1}^T,  dZ_i = dO_i W_i + lr Vhat_i Wh_{i+1},  Wh_i = Wh_{i+1} + dO_i^T Z_i.
+ *  in : Z, Vhat as in the forward; W_chunks from inplace_ttt_fwd (required); dO [T, d_model]
+ *       bf16; dW_final [d_model, d_ff] float32 (nullable = 0)
+ *  out: dZ [T, d_ff] bf16, dVhat [T, d_model] bf16, dW [d_model, d_ff] float32 = Wh_0, the
+ *       gradient of the initial W_down (plain stores)
+ * Requirements as inplace_ttt_fwd; workspace from inplace_ttt_workspace_bytes. */
+ttt_status inplace_ttt_bwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                           const void* Vhat, const void* W_chunks, const void* dO,
+                           const float* dW_final, void* dZ, void* dVhat, float* dW,
+                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then returns TTT_ERR_TIMEOUT if any kernel of this library on the
  * current device recorded a bounded wait that ran out since the last call (and clears the

@@ -8,7 +8,7 @@ import pytest
 import weight_sequence_layers_b200 as ttt
 
 FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_ttt_workspace_bytes",
-             "inplace_ttt_fwd", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "inplace_ttt_fwd", "inplace_ttt_bwd", "ttt_get_device_error", "ttt_selftest_bounded_wait",
              "ttt_status_string"}
 
 
@@ -136,17 +136,38 @@ def test_tc_bwd_workspace_covers_the_decay_gradient():
 def test_inplace_argument_errors():
     A = 4096
     f = ttt.lib.inplace_ttt_fwd
-    assert f(1000, 256, 256, 128, 1e-3, A, A, A, A, A, 1 << 30, None) == ttt.ERR_INVALID_ARG  # T % C
-    assert f(960, 256, 256, 96, 1e-3, A, A, A, A, A, 1 << 30, None) == ttt.ERR_UNSUPPORTED    # C % 128
-    assert f(1024, 250, 256, 128, 1e-3, A, A, A, A, A, 1 << 30, None) == ttt.ERR_UNSUPPORTED  # d_ff % 64
-    assert f(1024, 256, 256, 128, float("nan"), A, A, A, A, A, 1 << 30, None) == ttt.ERR_INVALID_ARG
-    assert f(1024, 256, 256, 128, 1e-3, None, A, A, A, A, 1 << 30, None) == ttt.ERR_INVALID_ARG
-    assert f(1024, 256, 256, 128, 1e-3, A, A, A + 4, A, A, 1 << 30, None) == ttt.ERR_ALIGNMENT
+    # T d_ff d_model C lr Z Vhat W O W_chunks workspace bytes stream
+    assert f(1000, 256, 256, 128, 1e-3, A, A, A, A, None, A, 1 << 30, None) == ttt.ERR_INVALID_ARG  # T % C
+    assert f(960, 256, 256, 96, 1e-3, A, A, A, A, None, A, 1 << 30, None) == ttt.ERR_UNSUPPORTED    # C % 128
+    assert f(1024, 250, 256, 128, 1e-3, A, A, A, A, None, A, 1 << 30, None) == ttt.ERR_UNSUPPORTED  # d_ff % 64
+    assert f(1024, 256, 256, 128, float("nan"), A, A, A, A, None, A, 1 << 30, None) == ttt.ERR_INVALID_ARG
+    assert f(1024, 256, 256, 128, 1e-3, None, A, A, A, None, A, 1 << 30, None) == ttt.ERR_INVALID_ARG
+    assert f(1024, 256, 256, 128, 1e-3, A, A, A + 4, A, None, A, 1 << 30, None) == ttt.ERR_ALIGNMENT
+    assert f(1024, 256, 256, 128, 1e-3, A, A, A, A, A + 8, A, 1 << 30, None) == ttt.ERR_ALIGNMENT
     need = ttt.inplace_ttt_workspace_bytes(1024, 256, 256, 128)
     assert need >= 2 * 256 * 256 * 2
-    assert f(1024, 256, 256, 128, 1e-3, A, A, A, A, A, need - 1, None) == ttt.ERR_WORKSPACE
+    assert f(1024, 256, 256, 128, 1e-3, A, A, A, A, None, A, need - 1, None) == ttt.ERR_WORKSPACE
     with pytest.raises(ttt.TTTError):
         ttt.inplace_ttt_workspace_bytes(1000, 256, 256, 128)
+
+
+def test_inplace_bwd_argument_errors():
+    A = 4096
+    b = ttt.lib.inplace_ttt_bwd
+    need = ttt.inplace_ttt_workspace_bytes(1024, 256, 256, 128)
+    # T d_ff d_model C lr Z Vhat W_chunks dO dW_final dZ dVhat dW workspace bytes stream
+    ok = [A, A, A, A, None, A, A, A, A, need, None]
+    assert b(1000, 256, 256, 128, 1e-3, *ok) == ttt.ERR_INVALID_ARG        # T % C
+    assert b(1024, 256, 192, 128, 1e-3, *ok) == ttt.ERR_UNSUPPORTED        # d_model % 128
+    args = list(ok)
+    args[2] = None                                                          # W_chunks is required
+    assert b(1024, 256, 256, 128, 1e-3, *args) == ttt.ERR_INVALID_ARG
+    args = list(ok)
+    args[4] = A + 4                                                         # dW_final misaligned
+    assert b(1024, 256, 256, 128, 1e-3, *args) == ttt.ERR_ALIGNMENT
+    args = list(ok)
+    args[9] = need - 1
+    assert b(1024, 256, 256, 128, 1e-3, *args) == ttt.ERR_WORKSPACE
 
 
 def test_valid_call_without_a_gpu_reports_cuda_error():

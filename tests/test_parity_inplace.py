@@ -14,15 +14,31 @@ O_TOL = 2e-2     # bf16 output
 W_TOL = 1e-4     # float32 state built from exact bf16 products
 
 
-def run(cfg, inp):
+def run(cfg, inp, save=False):
     W = inp["W"].clone()
     O = torch.empty((cfg.T, cfg.d_model), device="cuda", dtype=torch.bfloat16)
+    Wc = torch.empty((cfg.T // cfg.C, cfg.d_model, cfg.d_ff), device="cuda",
+                     dtype=torch.bfloat16) if save else None
     n = ttt.inplace_ttt_workspace_bytes(cfg.T, cfg.d_ff, cfg.d_model, cfg.C)
     ws = torch.empty(n, device="cuda", dtype=torch.uint8)
-    ttt.inplace_ttt_fwd(cfg.T, cfg.d_ff, cfg.d_model, cfg.C, cfg.lr, inp["Z"], inp["Vhat"], W, O, ws, n)
+    ttt.inplace_ttt_fwd(cfg.T, cfg.d_ff, cfg.d_model, cfg.C, cfg.lr, inp["Z"], inp["Vhat"], W, O, ws, n,
+                        W_chunks=Wc)
     torch.cuda.synchronize()
     assert ttt.ttt_get_device_error() == ttt.OK
-    return O, W
+    return (O, W, Wc) if save else (O, W)
+
+
+def run_bwd(cfg, inp, Wc, dWf):
+    dZ = torch.full((cfg.T, cfg.d_ff), float("nan"), device="cuda", dtype=torch.bfloat16)
+    dVh = torch.full((cfg.T, cfg.d_model), float("nan"), device="cuda", dtype=torch.bfloat16)
+    dW = torch.full((cfg.d_model, cfg.d_ff), float("nan"), device="cuda", dtype=torch.float32)
+    n = ttt.inplace_ttt_workspace_bytes(cfg.T, cfg.d_ff, cfg.d_model, cfg.C)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    ttt.inplace_ttt_bwd(cfg.T, cfg.d_ff, cfg.d_model, cfg.C, cfg.lr, inp["Z"], inp["Vhat"], Wc,
+                        inp["dO"], dWf, dZ, dVh, dW, ws, n)
+    torch.cuda.synchronize()
+    assert ttt.ttt_get_device_error() == ttt.OK
+    return dZ, dVh, dW
 
 
 SMALL = [
@@ -56,3 +72,54 @@ def test_inplace_full_size_sampled_rows():
     # associativity over all rows (page "In-Place Test-Time Training": the update is a sum)
     Wsum = inp["W"] + cfg.lr * (inp["Vhat"].float().T @ inp["Z"].float())
     assert rel_err(W, Wsum) <= 1e-3
+
+
+@pytest.mark.parametrize("T,d_ff,d_model,C,lr", SMALL)
+def test_inplace_forward_saves_the_applied_weights(T, d_ff, d_model, C, lr):
+    cfg = synth.INPLACE_QWEN4B.replace(T=T, d_ff=d_ff, d_model=d_model, C=C, lr=lr)
+    inp = synth.inplace_inputs(cfg, device="cuda", seed=T + d_ff)
+    O, W = run(cfg, inp)
+    O2, W2, Wc = run(cfg, inp, save=True)
+    # the saved states are the operands the apply tiles read: outputs identical either way
+    assert torch.equal(O, O2) and torch.equal(W, W2)
+    lr32 = float(np.float32(lr))
+    for i in range(T // C):
+        # W_i: the state after the first i chunks (the initial W for i = 0)
+        ref = inp["W"].double().cpu().numpy() if i == 0 else oracle.inplace_fwd(
+            inp["Z"][: i * C], inp["Vhat"][: i * C], inp["W"], C=C, lr=lr32)[1]
+        assert rel_err(Wc[i], ref) <= 4e-3, i  # bf16 rounding of an fp32 state
+
+
+@pytest.mark.parametrize("T,d_ff,d_model,C,lr", SMALL)
+@pytest.mark.parametrize("with_dwf", [False, True])
+def test_inplace_backward_small(T, d_ff, d_model, C, lr, with_dwf):
+    cfg = synth.INPLACE_QWEN4B.replace(T=T, d_ff=d_ff, d_model=d_model, C=C, lr=lr)
+    inp = synth.inplace_inputs(cfg, device="cuda", seed=T + d_ff + 1)
+    dWf = (0.1 * torch.randn((d_model, d_ff), device="cuda",
+                             generator=torch.Generator("cuda").manual_seed(6))) if with_dwf else None
+    _, _, Wc = run(cfg, inp, save=True)
+    dZ, dVh, dW = run_bwd(cfg, inp, Wc, dWf)
+    ref = oracle.inplace_bwd(inp["Z"], inp["Vhat"], inp["W"], inp["dO"], dWf, C=C,
+                             lr=float(np.float32(lr)))
+    assert rel_err(dZ, ref["dZ"]) <= O_TOL
+    assert rel_err(dVh, ref["dVhat"]) <= O_TOL
+    assert rel_err(dW, ref["dW"]) <= W_TOL
+
+
+def test_inplace_backward_full_size_sampled():
+    cfg = synth.INPLACE_QWEN4B
+    inp = synth.inplace_inputs(cfg, device="cuda")
+    _, _, Wc = run(cfg, inp, save=True)
+    dZ, dVh, dW = run_bwd(cfg, inp, Wc, None)
+    lr32 = float(np.float32(cfg.lr))
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(cfg.d_model, 16, replace=False))
+    ref = oracle.inplace_bwd(inp["Z"], inp["Vhat"], inp["W"], inp["dO"], None, C=cfg.C, lr=lr32,
+                             rows=rows)
+    assert rel_err(dVh[:, rows], ref["dVhat"]) <= O_TOL
+    assert rel_err(dW[rows], ref["dW"]) <= W_TOL
+    # tokens from the first, a middle and the last chunk
+    tokens = [3, 1000, cfg.T // 2 + 17, cfg.T - 5]
+    dz = oracle.inplace_bwd_dz_tokens(inp["Z"], inp["Vhat"], inp["W"], inp["dO"], None, C=cfg.C,
+                                      lr=lr32, tokens=tokens)
+    assert rel_err(dZ[tokens], dz) <= O_TOL

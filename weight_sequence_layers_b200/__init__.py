@@ -48,7 +48,8 @@ _SIGS = {
     "ttt_chunk_fwd": ([_cfgp] + [_p] * 11 + [_sz, _p], _i),
     "ttt_chunk_bwd": ([_cfgp] + [_p] * 19 + [_sz, _p], _i),
     "inplace_ttt_workspace_bytes": ([_i] * 4, _sz),
-    "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 5 + [_sz, _p], _i),
+    "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 6 + [_sz, _p], _i),
+    "inplace_ttt_bwd": ([_i] * 4 + [_f] + [_p] * 9 + [_sz, _p], _i),
     "ttt_get_device_error": ([_p], _i),
     "ttt_selftest_bounded_wait": ([_u, _p], _i),
     "ttt_status_string": ([_i], ctypes.c_char_p),
@@ -149,10 +150,19 @@ def inplace_ttt_workspace_bytes(T, d_ff, d_model, C) -> int:
 
 
 def inplace_ttt_fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace=None, workspace_bytes=0,
-                    stream=None):
+                    stream=None, W_chunks=None):
     st = _lib.inplace_ttt_fwd(T, d_ff, d_model, C, float(lr), _ptr(Z), _ptr(Vhat), _ptr(W),
-                              _ptr(O), _ptr(workspace), int(workspace_bytes), _stream(stream))
+                              _ptr(O), _ptr(W_chunks), _ptr(workspace), int(workspace_bytes),
+                              _stream(stream))
     _check(st, "inplace_ttt_fwd")
+
+
+def inplace_ttt_bwd(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW,
+                    workspace=None, workspace_bytes=0, stream=None):
+    st = _lib.inplace_ttt_bwd(T, d_ff, d_model, C, float(lr), _ptr(Z), _ptr(Vhat), _ptr(W_chunks),
+                              _ptr(dO), _ptr(dW_final), _ptr(dZ), _ptr(dVhat), _ptr(dW),
+                              _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "inplace_ttt_bwd")
 
 
 def ttt_get_device_error(stream=None) -> int:

@@ -254,16 +254,24 @@ size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C) {
   return inplace_workspace(T, d_ff, d_model, C);
 }
 
-ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
-                           const void* Vhat, float* W, void* O, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+namespace {
+ttt_status inplace_sizes(int T, int d_ff, int d_model, int C, float lr) {
   if (T < 1 || d_ff < 1 || d_model < 1 || C < 1 || T % C || !isfinite(lr))
     return TTT_ERR_INVALID_ARG;
   if (C % 128 || d_ff % 64 || d_model % 128) return TTT_ERR_UNSUPPORTED;
-  if ((long long)T * d_ff > (1ll << 40) || (long long)d_model * d_ff > (1ll << 40))
+  if ((long long)T * d_ff > (1ll << 40) || (long long)(T / C) * d_model * d_ff > (1ll << 40))
     return TTT_ERR_INVALID_ARG;
+  return TTT_OK;
+}
+}  // namespace
+
+ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                           const void* Vhat, float* W, void* O, void* W_chunks, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  const ttt_status st = inplace_sizes(T, d_ff, d_model, C, lr);
+  if (st != TTT_OK) return st;
   if (!Z || !Vhat || !W || !O) return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {Z, Vhat, W, O, workspace};
+  const void* ptrs[] = {Z, Vhat, W, O, W_chunks, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   const size_t need = inplace_workspace(T, d_ff, d_model, C);
@@ -271,8 +279,28 @@ ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const 
   cudaError_t e;
   unsigned* err = error_word(&e);
   if (!err) return TTT_ERR_CUDA;
-  return launch_status(inplace_run(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace, err,
-                                   static_cast<cudaStream_t>(stream)));
+  return launch_status(inplace_run(T, d_ff, d_model, C, lr, Z, Vhat, W, O, W_chunks, workspace,
+                                   err, static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status inplace_ttt_bwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                           const void* Vhat, const void* W_chunks, const void* dO,
+                           const float* dW_final, void* dZ, void* dVhat, float* dW,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  const ttt_status st = inplace_sizes(T, d_ff, d_model, C, lr);
+  if (st != TTT_OK) return st;
+  if (!Z || !Vhat || !W_chunks || !dO || !dZ || !dVhat || !dW) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const size_t need = inplace_workspace(T, d_ff, d_model, C);
+  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  return launch_status(inplace_bwd_run(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final,
+                                       dZ, dVhat, dW, workspace, err,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 ttt_status ttt_get_device_error(void* stream) {

@@ -1,16 +1,26 @@
-// In-Place TTT forward of the W_down fast weight on sm_100a tensor cores.
+// In-Place TTT forward and backward of the W_down fast weight on sm_100a tensor cores.
 //
-// Page "In-Place Test-Time Training", section "核心方法和技术细节": W_down of a gated MLP
-// is the fast weight; the sequence is cut into chunks of C tokens and every chunk first
-// applies the current weight, O_[i] = Z_[i] W^(i)T, then updates it with the chunk's
-// inner-product gradient, W^(i+1) = W^(i) + eta Vhat_[i]^T Z_[i].
+// Page "In-Place Test-Time Training", section "核心方法和技术细节": W_down of a gated MLP is
+// the fast weight; the sequence is cut into chunks of C tokens and every chunk first applies
+// the current weight, O_[i] = Z_[i] W^(i)T, then updates it with the chunk's inner-product
+// gradient, W^(i+1) = W^(i) + eta Vhat_[i]^T Z_[i].
 //
-// One launch per chunk i runs both GEMMs of that chunk from a shared dynamic tile queue:
-//   apply  tiles: O_i[128 tokens x 256 d_model] = Z_i (K-major) x Wb_i^T (K-major), K = d_ff
-//   update tiles: W[128 d_model x 256 d_ff] += eta * Vhat_i^T (MN-major) x Z_i (MN-major),
-//                 K = C; the epilogue keeps W in float32 and writes the bf16 copy Wb_{i+1}
-//                 that the next chunk's apply tiles read.
-// Apply tiles (long, K = d_ff) are handed out first, update tiles fill the remaining SMs.
+// The backward is the reverse-mode of that loop for J = sum_i <dO_i, O_i> + <dW_final, W_final>
+// (the page gives no backward). With Wh the adjoint of the fast weight (dW_final after the last
+// chunk), chunk i, from the last one down, needs
+//     dVhat_i = Z_i (eta Wh_{i+1})^T,  dZ_i = dO_i W_i + Vhat_i (eta Wh_{i+1}),
+//     Wh_i = Wh_{i+1} + dO_i^T Z_i     (Wh_0 is the gradient of the initial W).
+//
+// One launch per chunk runs every GEMM of that chunk from a shared dynamic tile queue. Tile
+// kinds, each an fp32 accumulator of 128 x 256 in TMEM:
+//   row tiles    [128 tokens x 256] = A (K-major) x B^T (K-major), A = Z_i, K = d_ff: the
+//                forward's O_i (B = bf16 W_i) and the backward's dVhat_i (B = bf16 eta Wh_{i+1});
+//   dz tiles     [128 tokens x 256 d_ff] = [dO_i | Vhat_i] (K-major, K = 2 d_model) x
+//                [W_i ; eta Wh_{i+1}] (MN-major): the backward's dZ_i;
+//   update tiles [128 d_model x 256 d_ff]: M += s X_i^T (MN-major) x Z_i (MN-major), K = C,
+//                with (M, X, s) = (W, Vhat, eta) forward and (Wh, dO, 1) backward; the epilogue
+//                keeps M in float32 and writes the scaled bf16 copy the next launch reads.
+// Long tiles (row, then dz) are handed out first, update tiles fill the remaining SMs.
 // Warp roles: warp 0 issues TMA loads into a 4-stage ring, warp 1 issues tcgen05.mma into
 // two TMEM accumulators of 128 x 256 fp32, warps 2-9 drain the accumulators (two warps per
 // TMEM lane quadrant, each taking 128 of the 256 columns).
@@ -32,33 +42,45 @@ constexpr uint32_t kTmemCols = 512;            // two 256-column accumulators
 
 struct Params {
   int chunk, C, d_ff, d_model;
-  int n_apply_n, n_upd_n, n_apply, n_total;
-  int kb_apply, kb_upd;
-  int wb_cur_row0, wb_next_row0;
-  float lr;
-  float* W;
-  __nv_bfloat16* Wb;
-  __nv_bfloat16* O;
+  int n_row_n, n_dz_n, n_upd_n;  // N tiles per 128-row block of each kind
+  int n_row, n_dz, n_total;      // tiles [0, n_row) row, [n_row, n_row + n_dz) dz, rest update
+  int kb_row, kb_dz, kb_dz_split, kb_upd;
+  int wb_cur_row0;               // first row of the bf16 copy this launch reads
+  int wb_next_row0;              // first row of the bf16 copy it writes (-1: none)
+  int wc_row0;                   // first row of W_i among the saved chunk states (dz tiles)
+  float acc_scale, copy_scale;   // update epilogue: M += acc_scale acc; copy = bf16(copy_scale M)
+  float* M;                      // float32 matrix of the update tiles (W, or its adjoint)
+  __nv_bfloat16* Mb;             // its bf16 copies
+  __nv_bfloat16* Orow;           // row-tile output [T, d_model]
+  __nv_bfloat16* Odz;            // dz-tile output [T, d_ff]
   int* counter;
   unsigned* err;
 };
 
+enum Kind { KIND_ROW = 0, KIND_DZ = 1, KIND_UPD = 2 };
+
 struct Tile {
-  int apply, m0, n0, nkb;
+  int kind, m0, n0, nkb;
 };
 
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
   Tile x;
-  if (t < p.n_apply) {
-    x.apply = 1;
-    x.m0 = (t / p.n_apply_n) * BM;  // token offset inside the chunk
-    x.n0 = (t % p.n_apply_n) * BN;  // d_model column
-    x.nkb = p.kb_apply;
+  if (t < p.n_row) {
+    x.kind = KIND_ROW;
+    x.m0 = (t / p.n_row_n) * BM;  // token offset inside the chunk
+    x.n0 = (t % p.n_row_n) * BN;  // d_model column
+    x.nkb = p.kb_row;
+  } else if (t < p.n_row + p.n_dz) {
+    const int u = t - p.n_row;
+    x.kind = KIND_DZ;
+    x.m0 = (u / p.n_dz_n) * BM;   // token offset inside the chunk
+    x.n0 = (u % p.n_dz_n) * BN;   // d_ff column
+    x.nkb = p.kb_dz;
   } else {
-    const int u = t - p.n_apply;
-    x.apply = 0;
-    x.m0 = (u / p.n_upd_n) * BM;    // d_model row
-    x.n0 = (u % p.n_upd_n) * BN;    // d_ff column
+    const int u = t - p.n_row - p.n_dz;
+    x.kind = KIND_UPD;
+    x.m0 = (u / p.n_upd_n) * BM;  // d_model row
+    x.n0 = (u % p.n_upd_n) * BN;  // d_ff column
     x.nkb = p.kb_upd;
   }
   return x;
@@ -73,10 +95,15 @@ struct __align__(8) Bars {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    inplace_chunk_kernel(const __grid_constant__ CUtensorMap tm_za,
-                         const __grid_constant__ CUtensorMap tm_zb,
-                         const __grid_constant__ CUtensorMap tm_wb,
-                         const __grid_constant__ CUtensorMap tm_vh, const Params p) {
+    inplace_chunk_kernel(const __grid_constant__ CUtensorMap tm_za,    // Z, K-major boxes
+                         const __grid_constant__ CUtensorMap tm_zb,    // Z, MN-major boxes
+                         const __grid_constant__ CUtensorMap tm_mb,    // bf16 copy, K-major
+                         const __grid_constant__ CUtensorMap tm_x,     // Vhat or dO, MN-major
+                         const __grid_constant__ CUtensorMap tm_do,    // dO, K-major
+                         const __grid_constant__ CUtensorMap tm_vk,    // Vhat, K-major
+                         const __grid_constant__ CUtensorMap tm_wc,    // saved W_i, MN-major
+                         const __grid_constant__ CUtensorMap tm_mbn,   // bf16 copy, MN-major
+                         const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -102,8 +129,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tm_za);
     tma_prefetch_desc(&tm_zb);
-    tma_prefetch_desc(&tm_wb);
-    tma_prefetch_desc(&tm_vh);
+    tma_prefetch_desc(&tm_mb);
+    tma_prefetch_desc(&tm_x);
+    if (p.n_dz) {
+      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_vk);
+      tma_prefetch_desc(&tm_wc);
+      tma_prefetch_desc(&tm_mbn);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
@@ -133,13 +166,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = smem_u32(&bars->full[s]);
           const uint32_t sa = stage0 + s * STAGE_BYTES, sb = sa + A_BYTES;
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          if (x.apply) {
+          if (x.kind == KIND_ROW) {
             tma_load_2d(sa, &tm_za, fb, kb * BK, row_base + x.m0);
-            tma_load_2d(sb, &tm_wb, fb, kb * BK, p.wb_cur_row0 + x.n0);
+            tma_load_2d(sb, &tm_mb, fb, kb * BK, p.wb_cur_row0 + x.n0);
+          } else if (x.kind == KIND_DZ) {
+            // K runs over [dO_i | Vhat_i] against [W_i ; eta Wh_{i+1}]
+            const bool first = kb < p.kb_dz_split;
+            const int k0 = (first ? kb : kb - p.kb_dz_split) * BK;
+            tma_load_2d(sa, first ? &tm_do : &tm_vk, fb, k0, row_base + x.m0);
+            const CUtensorMap* mb = first ? &tm_wc : &tm_mbn;
+            const int r0 = (first ? p.wc_row0 : p.wb_cur_row0) + k0;
+            for (int j = 0; j < 4; ++j) tma_load_2d(sb + 8192 * j, mb, fb, x.n0 + 64 * j, r0);
           } else {
             const int tok = row_base + kb * BK;
-            tma_load_2d(sa, &tm_vh, fb, x.m0, tok);
-            tma_load_2d(sa + 8192, &tm_vh, fb, x.m0 + 64, tok);
+            tma_load_2d(sa, &tm_x, fb, x.m0, tok);
+            tma_load_2d(sa + 8192, &tm_x, fb, x.m0 + 64, tok);
             for (int j = 0; j < 4; ++j) tma_load_2d(sb + 8192 * j, &tm_zb, fb, x.n0 + 64 * j, tok);
           }
           if (++s == STAGES) { s = 0; sph ^= 1; }
@@ -151,7 +192,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int r = 0, s = 0, acc = 0;
       uint32_t rph = 0, sph = 0, aph = 0;
-      const uint32_t id_apply = idesc_bf16(BM, BN, 0, 0);
+      const uint32_t id_row = idesc_bf16(BM, BN, 0, 0);
+      const uint32_t id_dz = idesc_bf16(BM, BN, 0, 1);
       const uint32_t id_upd = idesc_bf16(BM, BN, 1, 1);
       for (;;) {
         if (!mbar_wait(smem_u32(&bars->tile_full[r]), rph, ab)) break;
@@ -163,6 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(smem_u32(&bars->acc_empty[acc]), aph ^ 1, ab)) break;
         tc_fence_after();
         const uint32_t d = tmem + acc * BN;
+        const uint32_t id = x.kind == KIND_ROW ? id_row : x.kind == KIND_DZ ? id_dz : id_upd;
+        const bool a_kmaj = x.kind != KIND_UPD, b_kmaj = x.kind == KIND_ROW;
         bool ok = true;
         for (int kb = 0; kb < x.nkb; ++kb) {
           if (!mbar_wait(smem_u32(&bars->full[s]), sph, ab)) { ok = false; break; }
@@ -170,15 +214,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = stage0 + s * STAGE_BYTES, sb = sa + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            uint64_t ad, bd;
-            if (x.apply) {
-              ad = sdesc_sw128(sa + kk * 32, 16, 1024);
-              bd = sdesc_sw128(sb + kk * 32, 16, 1024);
-            } else {
-              ad = sdesc_sw128(sa + kk * 2048, 8192, 1024);
-              bd = sdesc_sw128(sb + kk * 2048, 8192, 1024);
-            }
-            mma_bf16_ss(d, ad, bd, x.apply ? id_apply : id_upd, (kb | kk) != 0);
+            const uint64_t ad = a_kmaj ? sdesc_sw128(sa + kk * 32, 16, 1024)
+                                       : sdesc_sw128(sa + kk * 2048, 8192, 1024);
+            const uint64_t bd = b_kmaj ? sdesc_sw128(sb + kk * 32, 16, 1024)
+                                       : sdesc_sw128(sb + kk * 2048, 8192, 1024);
+            mma_bf16_ss(d, ad, bd, id, (kb | kk) != 0);
           }
           mma_commit(smem_u32(&bars->empty[s]));
           if (++s == STAGES) { s = 0; sph ^= 1; }
@@ -212,10 +252,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
         tmem_wait_ld();
         const int col0 = x.n0 + cb * 32;
-        if (x.apply) {
-          if (col0 < p.d_model) {
-            uint4* dst = reinterpret_cast<uint4*>(
-                p.O + (size_t)(row_base + x.m0 + row) * p.d_model + col0);
+        if (x.kind != KIND_UPD) {
+          // bf16 rows of O_i / dVhat_i ([T, d_model]) or dZ_i ([T, d_ff])
+          const int ncol = x.kind == KIND_ROW ? p.d_model : p.d_ff;
+          __nv_bfloat16* out = x.kind == KIND_ROW ? p.Orow : p.Odz;
+          if (col0 < ncol) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(out + (size_t)(row_base + x.m0 + row) * ncol + col0);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]),
@@ -226,24 +269,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           const int m = x.m0 + row;
           if (col0 < p.d_ff && m < p.d_model) {
-            float4* w = reinterpret_cast<float4*>(p.W + (size_t)m * p.d_ff + col0);
-            uint4* wb =
-                reinterpret_cast<uint4*>(p.Wb + (size_t)(p.wb_next_row0 + m) * p.d_ff + col0);
+            float4* w = reinterpret_cast<float4*>(p.M + (size_t)m * p.d_ff + col0);
+            uint4* wb = p.wb_next_row0 < 0 ? nullptr
+                                           : reinterpret_cast<uint4*>(
+                                                 p.Mb + (size_t)(p.wb_next_row0 + m) * p.d_ff + col0);
+            const float s = p.acc_scale, cs = p.copy_scale;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               float4 a0 = w[2 * j], a1 = w[2 * j + 1];
-              a0.x += p.lr * v[8 * j + 0];
-              a0.y += p.lr * v[8 * j + 1];
-              a0.z += p.lr * v[8 * j + 2];
-              a0.w += p.lr * v[8 * j + 3];
-              a1.x += p.lr * v[8 * j + 4];
-              a1.y += p.lr * v[8 * j + 5];
-              a1.z += p.lr * v[8 * j + 6];
-              a1.w += p.lr * v[8 * j + 7];
+              a0.x += s * v[8 * j + 0];
+              a0.y += s * v[8 * j + 1];
+              a0.z += s * v[8 * j + 2];
+              a0.w += s * v[8 * j + 3];
+              a1.x += s * v[8 * j + 4];
+              a1.y += s * v[8 * j + 5];
+              a1.z += s * v[8 * j + 6];
+              a1.w += s * v[8 * j + 7];
               w[2 * j] = a0;
               w[2 * j + 1] = a1;
-              wb[j] = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
-                                 pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+              if (wb)
+                wb[j] = make_uint4(pack_bf16x2(cs * a0.x, cs * a0.y), pack_bf16x2(cs * a0.z, cs * a0.w),
+                                   pack_bf16x2(cs * a1.x, cs * a1.y), pack_bf16x2(cs * a1.z, cs * a1.w));
             }
           }
         }
@@ -264,17 +310,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// dst = bf16(scale * src) over n elements.
 __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
-                               size_t n) {
+                               size_t n, float scale) {
   for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
-    dst[i] = __float2bfloat16_rn(src[i]);
+    dst[i] = __float2bfloat16_rn(scale * src[i]);
 }
 
 constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(Bars) + 1024;
 
+struct Launch {
+  int sms;
+};
+
+cudaError_t prepare(Launch* l) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&l->sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(inplace_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)kSmemBytes);
+}
+
 }  // namespace
 
+// Two bf16 copies of a d_model x d_ff matrix (read by one launch, written for the next), then
+// one tile counter per chunk.
 size_t inplace_workspace(int T, int d_ff, int d_model, int C) {
   const size_t wb = 2 * (size_t)d_model * d_ff * 2;
   const size_t counters = ((size_t)(T / C) * sizeof(int) + 255) & ~size_t(255);
@@ -282,51 +345,124 @@ size_t inplace_workspace(int T, int d_ff, int d_model, int C) {
 }
 
 cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
-                        const void* Vhat, float* W, void* O, void* ws, unsigned* err,
-                        cudaStream_t s) {
-  __nv_bfloat16* Wb = static_cast<__nv_bfloat16*>(ws);
-  int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 2 * (size_t)d_model * d_ff * 2);
+                        const void* Vhat, float* W, void* O, void* W_chunks, void* ws,
+                        unsigned* err, cudaStream_t s) {
   const int NC = T / C;
+  // bf16 W_i: the caller's [NC, d_model, d_ff] chunk states when given, else two rotating copies
+  __nv_bfloat16* Wb = W_chunks ? static_cast<__nv_bfloat16*>(W_chunks)
+                               : static_cast<__nv_bfloat16*>(ws);
+  const size_t wb_rows = W_chunks ? (size_t)NC * d_model : 2 * (size_t)d_model;
+  int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 2 * (size_t)d_model * d_ff * 2);
   CUtensorMap tza, tzb, twb, tvh;
   if (!make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
       !make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
-      !make_tmap_bf16(&twb, Wb, d_ff, 2 * (size_t)d_model, d_ff, BK, BN) ||
+      !make_tmap_bf16(&twb, Wb, d_ff, wb_rows, d_ff, BK, BN) ||
       !make_tmap_bf16(&tvh, Vhat, d_model, T, d_model, 64, BK))
     return cudaErrorInvalidValue;
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  Launch l;
+  cudaError_t e = prepare(&l);
   if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(inplace_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemBytes);
-  if (e != cudaSuccess) return e;
-  const size_t nW = (size_t)d_model * d_ff;
-  to_bf16_kernel<<<sms * 4, 256, 0, s>>>(W, Wb, nW);
+  to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W, Wb, (size_t)d_model * d_ff, 1.f);
   e = cudaMemsetAsync(counters, 0, NC * sizeof(int), s);
   if (e != cudaSuccess) return e;
   Params p{};
   p.C = C;
   p.d_ff = d_ff;
   p.d_model = d_model;
-  p.n_apply_n = (d_model + BN - 1) / BN;
+  p.n_row_n = (d_model + BN - 1) / BN;
   p.n_upd_n = (d_ff + BN - 1) / BN;
-  p.n_apply = (C / BM) * p.n_apply_n;
-  p.n_total = p.n_apply + (d_model / BM) * p.n_upd_n;
-  p.kb_apply = d_ff / BK;
+  p.n_row = (C / BM) * p.n_row_n;
+  p.n_total = p.n_row + (d_model / BM) * p.n_upd_n;
+  p.kb_row = d_ff / BK;
   p.kb_upd = C / BK;
-  p.lr = lr;
-  p.W = W;
-  p.Wb = Wb;
-  p.O = static_cast<__nv_bfloat16*>(O);
+  p.acc_scale = lr;
+  p.copy_scale = 1.f;
+  p.M = W;
+  p.Mb = Wb;
+  p.Orow = static_cast<__nv_bfloat16*>(O);
   p.err = err;
-  const int grid = p.n_total < sms ? p.n_total : sms;
+  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
   for (int i = 0; i < NC; ++i) {
     p.chunk = i;
-    p.wb_cur_row0 = (i & 1) * d_model;
-    p.wb_next_row0 = ((i + 1) & 1) * d_model;
+    if (W_chunks) {
+      p.wb_cur_row0 = i * d_model;
+      p.wb_next_row0 = i + 1 < NC ? (i + 1) * d_model : -1;
+    } else {
+      p.wb_cur_row0 = (i & 1) * d_model;
+      p.wb_next_row0 = ((i + 1) & 1) * d_model;
+    }
     p.counter = counters + i;
-    inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, twb, tvh, p);
+    inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, twb, tvh, tza, tza, tzb, tzb,
+                                                            p);
+  }
+  count_launches(NC + 1);
+  return cudaGetLastError();
+}
+
+cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                            const void* Vhat, const void* W_chunks, const void* dO,
+                            const float* dW_final, void* dZ, void* dVhat, float* dW, void* ws,
+                            unsigned* err, cudaStream_t s) {
+  const int NC = T / C;
+  // bf16 eta Wh_{i+1}: two rotating copies
+  __nv_bfloat16* Mb = static_cast<__nv_bfloat16*>(ws);
+  int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 2 * (size_t)d_model * d_ff * 2);
+  CUtensorMap tza, tzb, tmb, tdx, tdo, tvk, twc, tmbn;
+  if (!make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
+      !make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
+      !make_tmap_bf16(&tmb, Mb, d_ff, 2 * (size_t)d_model, d_ff, BK, BN) ||
+      !make_tmap_bf16(&tdx, dO, d_model, T, d_model, 64, BK) ||
+      !make_tmap_bf16(&tdo, dO, d_model, T, d_model, BK, BM) ||
+      !make_tmap_bf16(&tvk, Vhat, d_model, T, d_model, BK, BM) ||
+      !make_tmap_bf16(&twc, W_chunks, d_ff, (size_t)NC * d_model, d_ff, 64, BK) ||
+      !make_tmap_bf16(&tmbn, Mb, d_ff, 2 * (size_t)d_model, d_ff, 64, BK))
+    return cudaErrorInvalidValue;
+  Launch l;
+  cudaError_t e = prepare(&l);
+  if (e != cudaSuccess) return e;
+  const size_t nW = (size_t)d_model * d_ff;
+  const int first = (NC - 1) & 1;  // copy slot the last chunk reads
+  if (dW_final) {
+    e = cudaMemcpyAsync(dW, dW_final, nW * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return e;
+    to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(dW_final, Mb + first * nW, nW, lr);
+  } else {
+    if ((e = cudaMemsetAsync(dW, 0, nW * sizeof(float), s)) != cudaSuccess ||
+        (e = cudaMemsetAsync(Mb + first * nW, 0, nW * 2, s)) != cudaSuccess)
+      return e;
+  }
+  e = cudaMemsetAsync(counters, 0, NC * sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  Params p{};
+  p.C = C;
+  p.d_ff = d_ff;
+  p.d_model = d_model;
+  p.n_row_n = (d_model + BN - 1) / BN;
+  p.n_dz_n = (d_ff + BN - 1) / BN;
+  p.n_upd_n = (d_ff + BN - 1) / BN;
+  p.n_row = (C / BM) * p.n_row_n;
+  p.n_dz = (C / BM) * p.n_dz_n;
+  p.n_total = p.n_row + p.n_dz + (d_model / BM) * p.n_upd_n;
+  p.kb_row = d_ff / BK;
+  p.kb_dz_split = d_model / BK;
+  p.kb_dz = 2 * p.kb_dz_split;
+  p.kb_upd = C / BK;
+  p.acc_scale = 1.f;
+  p.copy_scale = lr;
+  p.M = dW;
+  p.Mb = Mb;
+  p.Orow = static_cast<__nv_bfloat16*>(dVhat);
+  p.Odz = static_cast<__nv_bfloat16*>(dZ);
+  p.err = err;
+  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
+  for (int i = NC - 1; i >= 0; --i) {
+    p.chunk = i;
+    p.wb_cur_row0 = (i & 1) * d_model;
+    p.wb_next_row0 = i > 0 ? ((i - 1) & 1) * d_model : -1;
+    p.wc_row0 = i * d_model;
+    p.counter = counters + i;
+    inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, tmb, tdx, tdo, tvk, twc,
+                                                            tmbn, p);
   }
   count_launches(NC + 1);
   return cudaGetLastError();

@@ -46,8 +46,12 @@ cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
 // In-Place TTT.
 size_t inplace_workspace(int T, int d_ff, int d_model, int C);
 cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
-                        const void* Vhat, float* W, void* O, void* ws, unsigned* err,
-                        cudaStream_t s);
+                        const void* Vhat, float* W, void* O, void* W_chunks, void* ws,
+                        unsigned* err, cudaStream_t s);
+cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                            const void* Vhat, const void* W_chunks, const void* dO,
+                            const float* dW_final, void* dZ, void* dVhat, float* dW, void* ws,
+                            unsigned* err, cudaStream_t s);
 
 // Address of the current device's error word (looked up once per device); NULL on failure.
 unsigned* current_error_word();
