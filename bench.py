@@ -348,33 +348,48 @@ def time_e2e(layer, steps, warmup):
 
 
 def time_inplace(ttt, steps, warmup):
+    """Device ms of the In-Place forward (without and with the saved chunk weights) and of the
+    backward, each averaged over `steps` launches."""
     icfg = synth.INPLACE_QWEN4B
     inp = synth.inplace_inputs(icfg, device="cuda")
+    T, F, M, C = icfg.T, icfg.d_ff, icfg.d_model, icfg.C
     W = inp["W"].clone()
-    O = torch.empty((icfg.T, icfg.d_model), device="cuda", dtype=torch.bfloat16)
-    n = ttt.inplace_ttt_workspace_bytes(icfg.T, icfg.d_ff, icfg.d_model, icfg.C)
+    O = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+    Wc = torch.empty((T // C, M, F), device="cuda", dtype=torch.bfloat16)
+    dZ = torch.empty((T, F), device="cuda", dtype=torch.bfloat16)
+    dV = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+    dW = torch.empty((M, F), device="cuda", dtype=torch.float32)
+    n = ttt.inplace_ttt_workspace_bytes(T, F, M, C)
     ws = torch.empty(n, device="cuda", dtype=torch.uint8)
 
-    def run():
-        W.copy_(inp["W"])
-        ttt.inplace_ttt_fwd(icfg.T, icfg.d_ff, icfg.d_model, icfg.C, icfg.lr, inp["Z"], inp["Vhat"],
-                            W, O, ws, n)
+    def fwd(save):
+        ttt.inplace_ttt_fwd(T, F, M, C, icfg.lr, inp["Z"], inp["Vhat"], W, O, ws, n,
+                            W_chunks=Wc if save else None)
 
-    for _ in range(warmup):
-        run()
-    torch.cuda.synchronize()
-    evs = []
-    for _ in range(steps):
-        W.copy_(inp["W"])
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        ttt.inplace_ttt_fwd(icfg.T, icfg.d_ff, icfg.d_model, icfg.C, icfg.lr, inp["Z"], inp["Vhat"],
-                            W, O, ws, n)
-        b.record()
-        evs.append((a, b))
-    torch.cuda.synchronize()
-    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    return icfg, ms
+    def bwd(_):
+        ttt.inplace_ttt_bwd(T, F, M, C, icfg.lr, inp["Z"], inp["Vhat"], Wc, inp["dO"], None, dZ,
+                            dV, dW, ws, n)
+
+    def timed(fn, arg):
+        for _ in range(warmup):
+            W.copy_(inp["W"])
+            fn(arg)
+        torch.cuda.synchronize()
+        evs = []
+        for _ in range(steps):
+            W.copy_(inp["W"])
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn(arg)
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    ms = timed(fwd, False)
+    ms_save = timed(fwd, True)
+    ms_bwd = timed(bwd, None)
+    return icfg, ms, ms_save, ms_bwd
 
 
 # --------------------------------------------------------------------------- oracle legs
@@ -534,7 +549,7 @@ def main():
     if not args.no_configs:
         out["other_configs"] = time_other_configs(ttt, peaks)
     if not args.no_inplace:
-        icfg, ims = time_inplace(ttt, steps=3, warmup=1)
+        icfg, ims, ims_save, ims_bwd = time_inplace(ttt, steps=3, warmup=1)
         fl, by = inplace_work(icfg)
         tf = fl / (ims * 1e-3) / 1e12
         out["inplace"] = {"workload": icfg.name, "ms": ims, "tokens_per_s": icfg.T / (ims * 1e-3),
@@ -543,7 +558,18 @@ def main():
                                        "frac": tf / peaks["bf16_tflops_sustained"],
                                        "traffic": measured_traffic("inplace_chunk", icfg.name),
                                        "traffic_unit": "bytes per chunk launch",
-                                       "peak_source": peak_src}}
+                                       "peak_source": peak_src},
+                          "ms_saving_chunk_weights": ims_save}
+        # backward per token: dZ 4 d_model d_ff (K = 2 d_model), dVhat 2 d_ff d_model and the
+        # adjoint update 2 d_model d_ff flops: twice the forward's 4 d_ff d_model
+        tfb = 2 * fl / (ims_bwd * 1e-3) / 1e12
+        out["inplace_bwd"] = {"workload": icfg.name.replace("-fwd", "-bwd"), "ms": ims_bwd,
+                              "tokens_per_s": icfg.T / (ims_bwd * 1e-3),
+                              "roofline": {"bound": "tensor", "achieved": tfb,
+                                           "peak": peaks["bf16_tflops_sustained"],
+                                           "unit": "TFLOP/s",
+                                           "frac": tfb / peaks["bf16_tflops_sustained"],
+                                           "peak_source": peak_src}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg)
     if _dist is not None:
