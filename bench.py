@@ -170,7 +170,8 @@ class Layer:
         self.O = torch.empty((B, H, T, dv), device=dev, dtype=sd)
         self.Wf = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
         self.Wc = torch.empty((B, H, T // C, dk, dv), device=dev, dtype=sd)
-        self.G = torch.empty((B, H, T, dv), device=dev, dtype=sd)  # saved by fwd for bwd
+        # saved by fwd for bwd: G, and with SiLU also Zq (the readout before the activation)
+        self.G = torch.empty((2 if cfg.act == "silu" else 1, B, H, T, dv), device=dev, dtype=sd)
         self.dQ = torch.empty((B, H, T, dk), device=dev, dtype=sd)
         self.dK = torch.empty((B, H, T, dk), device=dev, dtype=sd)
         self.dV = torch.empty((B, H, T, dv), device=dev, dtype=sd)
@@ -198,11 +199,10 @@ FP32_ALU_PEAK = 148 * 128 * 2 * 1.965e9  # flop/s
 
 
 def _path(cfg, call):
-    """Which kernels serve the call for this workload (mirrors the library's dispatch)."""
+    """Which kernels serve the call for this workload (mirrors the library's dispatch; the bench
+    always hands the backward the forward's saved G, and Zq with SiLU)."""
     tc_shape = cfg.dtype == "bf16" and cfg.decay != "vector" and cfg.dk == cfg.dv and \
         cfg.dk in (64, 128) and cfg.C in (128, 256)
-    if call == "ttt_chunk_bwd":
-        tc_shape = tc_shape and cfg.act == "id"
     return "tcgen05" if tc_shape else "simt"
 
 

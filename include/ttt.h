@@ -88,7 +88,8 @@ typedef struct {
  *   W0, W_final, dW_final, dW0   [B, H, dk, dv]  float32, row index = key feature
  *   W_chunks            [B, H, T/C, dk, dv]  dtype: the state at the start of every chunk
  *   G_saved             [B, H, T, dv]   dtype: G of every token, the value the token's write
- *                       subtracts (W_t = gamma_t W_{t-1} - eta_t k_t^T g_t)
+ *                       subtracts (W_t = gamma_t W_{t-1} - eta_t k_t^T g_t); with SiLU
+ *                       [2, B, H, T, dv]: G, then Zq = q_t W_t, the readout before the activation
  */
 
 /* Bytes of workspace ttt_chunk_fwd (for_bwd = 0) or ttt_chunk_bwd needs for this config; 0 if
@@ -101,8 +102,8 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd);
 /* Forward of the chunkwise TTT layer.
  *  in : Q, K, V, beta, gamma (nullable), W0
  *  out: O; W_final (nullable) = state after the last token; W_chunks (nullable) = chunk-start
- *       states, needed by ttt_chunk_bwd; G_saved (nullable) = G of every token, which
- *       ttt_chunk_bwd then reads instead of rebuilding it.
+ *       states, needed by ttt_chunk_bwd; G_saved (nullable) = G of every token (and, with
+ *       SiLU, Zq), which ttt_chunk_bwd then reads instead of rebuilding it.
  * bf16 configs with dk == dv in {64, 128}, C in {128, 256} and a scalar decay (or none) run on
  * the tcgen05 kernel; other shapes (dk, dv <= 128, C <= 256), all float32 configs and the
  * vector decay run on the SIMT kernels. */
@@ -114,7 +115,8 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
 /* Analytic backward of the layer for the objective J = <dO, O> + <dW_final, W_final>.
  *  in : Q, K, V, beta, gamma (nullable), W0, W_chunks (from ttt_chunk_fwd, required),
  *       G_saved (from ttt_chunk_fwd, nullable: rebuilt from W_chunks when NULL; kernels that
- *       rebuild G anyway may ignore it), dO, dW_final (nullable = 0);
+ *       rebuild G anyway may ignore it; with SiLU the tensor-core backward needs it, for Zq,
+ *       and a call without it runs on the SIMT kernels), dO, dW_final (nullable = 0);
  *       O and W_final (the forward's outputs) are read only for dgamma (then O is required,
  *       and W_final too when dW_final is non-NULL).
  *  out: dQ, dK, dV, dbeta, dW0 (plain stores, not accumulated); dgamma (nullable; requires
@@ -141,11 +143,12 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
  * ttt_chunk_bwd minus the workspace, and keeps its scratch (the per-chunk adjoint states and
  * the bf16 inner-loss gradient G of every token) in a fixed array of TTT_NOALLOC_SCRATCH_BYTES that the library holds on every GPU it is loaded
  * on, until the process exits. It allocates nothing and calls no allocating routine.
- *  - Only configs of the tensor-core backward are accepted (bf16, identity activation,
- *    dk == dv in {64, 128}, C in {128, 256}); others return TTT_ERR_UNSUPPORTED.
+ *  - Only configs of the tensor-core backward are accepted (bf16, dk == dv in {64, 128},
+ *    C in {128, 256}, scalar or no decay; SiLU only with G_saved); others return
+ *    TTT_ERR_UNSUPPORTED.
  *  - Configs needing more than the fixed scratch (B*H*(T/C)*dk*dv*2 bytes, plus B*H*T*dv*2 when
- *    G_saved is NULL, plus B*H*T*4 when dgamma is non-NULL) return TTT_ERR_WORKSPACE with
- *    nothing launched; ttt_chunk_bwd serves those.
+ *    G_saved is NULL, plus B*H*T*4 when dgamma is non-NULL, plus 4*B*H*T*dv*2 with SiLU) return
+ *    TTT_ERR_WORKSPACE with nothing launched; ttt_chunk_bwd serves those.
  *  - The first call on a device looks up the array's device address (with that device
  *    current); make that first call before any stream capture.
  *  - Every call shares the one array and leaves its contents behind. Calls that overlap on

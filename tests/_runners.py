@@ -28,19 +28,22 @@ def run_fwd(cfg, inp, save_g=True):
     O = torch.empty((B, H, T, dv), device="cuda", dtype=sd)
     Wf = torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32)
     Wc = torch.empty((B, H, T // C, dk, dv), device="cuda", dtype=sd)
-    G = torch.empty((B, H, T, dv), device="cuda", dtype=sd) if save_g else None
+    # with SiLU the saved buffer holds G, then Zq (the readout before the activation)
+    planes = 2 if cfg.act == "silu" else 1
+    Gs = torch.empty((planes, B, H, T, dv), device="cuda", dtype=sd) if save_g else None
     n = ttt.ttt_workspace_bytes(c, 0)
     ws = torch.empty(max(n, 16), device="cuda", dtype=torch.uint8)
     ttt.ttt_chunk_fwd(c, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], inp["W0"], O, Wf,
-                      Wc, G, ws, n)
+                      Wc, Gs, ws, n)
     torch.cuda.synchronize()
     assert ttt.ttt_get_device_error() == ttt.OK
-    return dict(O=O, W_final=Wf, W_chunks=Wc, G=G)
+    return dict(O=O, W_final=Wf, W_chunks=Wc, G=None if Gs is None else Gs[0], G_saved=Gs,
+                Zq=Gs[1] if Gs is not None and planes == 2 else None)
 
 
 def run_bwd(cfg, inp, W_chunks, G=None, fwd=None):
-    """The backward; G (from run_fwd) is passed as G_saved, else the library rebuilds it. With
-    `fwd` (run_fwd's outputs) and a decay, the decay gradient is asked for too."""
+    """The backward; G (run_fwd's "G_saved") is passed as G_saved, else the library rebuilds it.
+    With `fwd` (run_fwd's outputs) and a decay, the decay gradient is asked for too."""
     c = abi_config(cfg)
     sd = synth.storage_dtype(cfg)
     B, H, T, dk, dv = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv

@@ -46,7 +46,7 @@ def test_fp32_forward_backward(shape, loss, act, decay):
     ref["G"] = reference_g(cfg, inp, ref["W_chunks"])
     for k in ("O", "W_final", "W_chunks", "G"):
         assert rel_err(got[k], ref[k]) <= F32_TOL, k
-    g = run_bwd(cfg, inp, got["W_chunks"], got["G"] if decay else None, fwd=got)
+    g = run_bwd(cfg, inp, got["W_chunks"], got["G_saved"] if decay else None, fwd=got)
     r = oracle_bwd(cfg, inp)
     for k in ("dQ", "dK", "dV", "dbeta", "dW0") + (("dgamma",) if decay else ()):
         assert rel_err(g[k], r[k]) <= F32_TOL, k
@@ -78,7 +78,7 @@ def test_vector_decay_on_tensor_core_shapes_runs_on_simt(loss, act):
     ref = oracle_fwd(cfg, inp)
     for k in ("O", "W_final", "W_chunks"):
         assert rel_err(got[k], ref[k]) <= BF16_TOL, k
-    g = run_bwd(cfg, inp, got["W_chunks"], got["G"], fwd=got)
+    g = run_bwd(cfg, inp, got["W_chunks"], got["G_saved"], fwd=got)
     r = oracle_bwd(cfg, inp)
     for k in ("dQ", "dK", "dV", "dbeta", "dW0", "dgamma"):
         assert rel_err(g[k], r[k]) <= BF16_TOL, k

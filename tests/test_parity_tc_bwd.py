@@ -1,5 +1,5 @@
-"""GPU parity of the tcgen05 backward (identity activation, MSE or inner-product loss) against
-the oracle's reverse-mode of the per-token loop."""
+"""GPU parity of the tcgen05 backward (identity or SiLU activation, MSE or inner-product loss)
+against the oracle's reverse-mode of the per-token loop."""
 import numpy as np
 import pytest
 import torch
@@ -32,7 +32,7 @@ def test_tc_backward_small(shape, loss, decay, saved_g):
     inp = synth.ttt_inputs(cfg, device="cuda", seed=5 * T + d)
     inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(9))
     fwd = run_fwd(cfg, inp, save_g=saved_g)
-    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd=fwd)
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
     ref = oracle_bwd(cfg, inp)
     for k in GRADS + (("dgamma",) if decay else ()):
         assert rel_err(got[k], ref[k]) <= TOL, (k, rel_err(got[k], ref[k]))
@@ -42,8 +42,39 @@ def test_tc_backward_full_size_sampled_heads():
     cfg = synth.TRAIN_1P45B
     inp = synth.ttt_inputs(cfg, device="cuda")
     fwd = run_fwd(cfg, inp)
-    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd=fwd)
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
     rng = np.random.default_rng(44)
+    heads = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(2)]
+    sub = head_slice(inp, heads)
+    ref = oracle_bwd(cfg.replace(B=1, H=len(heads)), sub)
+    for k in GRADS + ("dgamma",):
+        g = torch.stack([got[k][b, h] for b, h in heads]).unsqueeze(0)
+        assert rel_err(g, ref[k]) <= TOL, (k, rel_err(g, ref[k]))
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("loss", ["mse", "ip"])
+@pytest.mark.parametrize("decay", [False, True])
+def test_tc_backward_silu_small(shape, loss, decay):
+    # SiLU on the tensor cores reads Zq and G saved by the forward
+    B, H, T, d, C = shape
+    cfg = synth.SILU_IP_FWD.replace(B=B, H=H, T=T, dk=d, dv=d, C=C, loss=loss, act="silu",
+                                    decay=decay, w0_std=1.0 / d)
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=3 * T + d)
+    inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(10))
+    fwd = run_fwd(cfg, inp)
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
+    ref = oracle_bwd(cfg, inp)
+    for k in GRADS + (("dgamma",) if decay else ()):
+        assert rel_err(got[k], ref[k]) <= TOL, (k, rel_err(got[k], ref[k]))
+
+
+def test_tc_backward_silu_full_size_sampled_heads():
+    cfg = synth.SILU_IP_FWD
+    inp = synth.ttt_inputs(cfg, device="cuda")
+    fwd = run_fwd(cfg, inp)
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
+    rng = np.random.default_rng(45)
     heads = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(2)]
     sub = head_slice(inp, heads)
     ref = oracle_bwd(cfg.replace(B=1, H=len(heads)), sub)

@@ -52,8 +52,8 @@ def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
         inp = synth.ttt_inputs(cfg, device="cuda", seed=seed)
         inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(seed))
         fwd = run_fwd(cfg, inp, save_g=saved_g)
-        ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd=fwd)
-        got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G"], fwd)
+        ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
+        got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd)
         for k in GRADS:
             assert rel_err(got[k], ref[k]) <= TOL, (seed, k)
 

@@ -82,8 +82,10 @@ Path fwd_path(const LayerArgs& a) {
   if (simt_supported(a)) return PATH_SIMT;
   return PATH_NONE;
 }
-Path bwd_path(const LayerArgs& a) {
-  if (a.dtype == TTT_BF16 && tc_bwd_supported(a)) return PATH_TC;
+// The tensor-core backward with SiLU reads the forward's Zq, saved beside G.
+Path bwd_path(const LayerArgs& a, bool g_saved) {
+  if (a.dtype == TTT_BF16 && tc_bwd_supported(a) && (a.act == TTT_ACT_ID || g_saved))
+    return PATH_TC;
   if (simt_supported(a)) return PATH_SIMT;
   return PATH_NONE;
 }
@@ -178,7 +180,7 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
     }
   }
   if (for_bwd != 1 && for_bwd != 2) return (size_t)-1;
-  switch (bwd_path(a)) {
+  switch (bwd_path(a, for_bwd == 2)) {
     case PATH_TC: return tc_bwd_workspace(a, for_bwd == 2, true);
     case PATH_SIMT: return simt_bwd_workspace(a);
     default: return (size_t)-1;
@@ -228,7 +230,7 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a = args_of(cfg);
-  const Path path = bwd_path(a);
+  const Path path = bwd_path(a, G_saved != nullptr);
   if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
   const size_t need =
       path == PATH_TC ? tc_bwd_workspace(a, G_saved != nullptr, dgamma != nullptr)

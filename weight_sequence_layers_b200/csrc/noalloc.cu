@@ -60,7 +60,8 @@ extern "C" ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q
   a.B = cfg->B; a.H = cfg->H; a.T = cfg->T; a.dk = cfg->dk; a.dv = cfg->dv; a.C = cfg->C;
   a.dtype = cfg->dtype; a.loss = cfg->loss; a.act = cfg->act; a.lr_bias = cfg->lr_bias;
   a.gvec = cfg->decay == TTT_DECAY_VECTOR;
-  if (!tc_bwd_supported(a)) return TTT_ERR_UNSUPPORTED;
+  // SiLU on the tensor cores also needs the forward's saved G and Zq
+  if (!tc_bwd_supported(a) || (a.act == TTT_ACT_SILU && !G_saved)) return TTT_ERR_UNSUPPORTED;
   const size_t need = tc_bwd_workspace(a, G_saved != nullptr, dgamma != nullptr);
   if (need > TTT_NOALLOC_SCRATCH_BYTES) return TTT_ERR_WORKSPACE;
   void* scratch = scratch_address();

@@ -66,6 +66,13 @@ struct BwdParams {
   const float* W_final;       // [BH, D, D] state after the last chunk
   float* dgamma;
   float* dgk;                 // [BH, T] workspace
+  // SiLU: every kernel reads dZq = dO act'(Zq) where the identity path reads dO, the chain
+  // stores -dG (through the dV tensor map, into workspace) and the dK kernel turns it into
+  // dV = -dG F1 and dZ = dG F2 with F1 = act'(Z), F2 = a act''(Z) (+ act'(Z)^2 for MSE)
+  int silu;
+  __nv_bfloat16* F1;          // [BH, T, D]
+  __nv_bfloat16* F2;          // [BH, T, D]
+  __nv_bfloat16* dV_out;      // [BH, T, D] the dV output
   unsigned* err;
 };
 
@@ -135,7 +142,7 @@ struct ChainL {
 enum { C_K_FULL, C_K_FREE, C_P_FULL, C_S_READY, C_XB0, C_X_FULL, C_W_READY, C_Y_FULL,
        C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_BG_FULL, C_BG_FULL1,
        C_P_FULL1, C_S_READY1, C_QD_FULL, C_QD_FREE, C_ST_READ, C_SCAN_FULL1, C_SCAN_FREE1,
-       C_NBARS };
+       C_V_READ, C_F2_READY, C_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool mse = p.loss == 0;
   // arrivals per barrier, in enum order
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
-                               kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1, 1, kEpiWarps};
+                               kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1, 1, kEpiWarps, 1, kEpiWarps};
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmK);
@@ -280,9 +287,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sQ + j * 2048, lboT, 1024),
                       sdesc_sw128(sDO + j * 2048, 0, 1024), idW, 1);
         mma_commit(BAR(C_QD_FREE));
-        if (!mbar_wait(BAR(C_DZ_READY), it & 1, ab)) break;
+        // -dZ: -dV for MSE with the identity, -dG * F2 once the epilogue has scaled it (SiLU)
+        if (!mbar_wait(BAR(p.silu ? C_F2_READY : C_DZ_READY), it & 1, ab)) break;
         tc_fence_after();
-        if (mse)
+        if (mse || p.silu)
           for (int j = 0; j < C / 16; ++j)
             mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sK + j * 2048, lboT, 1024),
                         sdesc_sw128(sS + j * 2048, 0, 1024), idWn, 1);
@@ -411,9 +419,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int b = 0; b < NB; ++b)
               tma_store_2d(&tmDV, sS + b * PANEL128, NV * slice, (int)tok0 + 128 * b);
             bulk_commit();
+            if (p.silu) {
+              // -dG must be read out before the buffer is scaled in place
+              bulk_wait_read0();
+              mbar_arrive(BAR(C_V_READ));
+            }
           }
         }
         if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
+      }
+      if (p.silu) {
+        // -dZ = -dG * F2 in place, the operand of dW += K^T dZ
+        uint4 f2[NB][4];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.F2 + (tok0 + 128 * b + lrow) * D + NV * slice + 32 * g);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) f2[b][k] = src[k];
+        }
+        if (!mbar_wait(BAR(C_V_READ), it & 1, ab)) { ok = false; break; }
+        __syncwarp();
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          const int r = 128 * b + lrow;
+          float v[32];
+          ld_row32(sS, r, 4 * g, v);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t w[4] = {f2[b][k].x, f2[b][k].y, f2[b][k].z, f2[b][k].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              v[8 * k + 2 * h] *= bf16lo(w[h]);
+              v[8 * k + 2 * h + 1] *= bf16hi(w[h]);
+            }
+          }
+          st_row32(sS, r, 4 * g, v);
+        }
+        epi_arrive(BAR(C_F2_READY));
       }
       // ---- adjoint at the end of chunk c-1 (or dW0)
       if (!mbar_wait(BAR(C_DW_FULL), it & 1, ab)) { ok = false; break; }
@@ -487,6 +530,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const bool mse = p.loss == 0;
+  const bool zmma = mse || p.silu;                    // Z = K W0 is needed
   const int row0 = blockIdx.x * 128;                  // first token row in [B*H*T]
   const int bh = row0 / p.T, c = (row0 % p.T) / (p.T / p.NC);
   const int wrow = (bh * p.NC + c) * D;
@@ -496,18 +540,18 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   Abort ab{&bars->abort_flag, p.err};
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(BAR(G_LD), mse ? 2 * L::BLK + L::WSZ : L::BLK);
+      mbar_arrive_expect_tx(BAR(G_LD), zmma ? 2 * L::BLK + L::WSZ : L::BLK);
 #pragma unroll
       for (int kp = 0; kp < L::KP; ++kp) {
         tma_load_2d(sV + kp * PANEL128, &tmV, BAR(G_LD), 64 * kp, row0);
-        if (mse) {
+        if (zmma) {
           tma_load_2d(sK + kp * PANEL128, &tmK, BAR(G_LD), 64 * kp, row0);
           tma_load_2d(sW0 + kp * D * 128, &tmW, BAR(G_LD), 64 * kp, wrow);
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0 && mse && mbar_wait(BAR(G_LD), 0, ab)) {
+    if (lane == 0 && zmma && mbar_wait(BAR(G_LD), 0, ab)) {
       tc_fence_after();
       const uint32_t idZ = idesc_bf16(128, D, 0, 1);
 #pragma unroll
@@ -519,13 +563,31 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   } else {
     const int q = warp & 3, lrow = q * 32 + lane;
     const uint32_t loff = (uint32_t)(q * 32) << 16;
-    if (mbar_wait(BAR(G_LD), 0, ab) && (!mse || mbar_wait(BAR(G_Z), 0, ab))) {
+    if (mbar_wait(BAR(G_LD), 0, ab) && (!zmma || mbar_wait(BAR(G_Z), 0, ab))) {
       __syncwarp();
       tc_fence_after();
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         float v[32], z[32];
         ld_row32(sV + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+        if (p.silu) {
+          // F1 = act'(z), F2 = a act''(z) (+ act'(z)^2 for MSE), a = act(z) - v or -v
+          tmem_ld32(tmem + loff + 32 * cc, z);
+          tmem_wait_ld();
+          float f1[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float sg = 1.f / (1.f + __expf(-z[j]));
+            const float d1 = sg * (1.f + z[j] * (1.f - sg));
+            const float d2 = sg * (1.f - sg) * (2.f + z[j] * (1.f - 2.f * sg));
+            const float a = mse ? z[j] * sg - v[j] : -v[j];
+            f1[j] = d1;
+            v[j] = a * d2 + (mse ? d1 * d1 : 0.f);
+          }
+          st_global_bf16x32(p.F1 + ((size_t)row0 + lrow) * D + 32 * cc, f1);
+          st_global_bf16x32(p.F2 + ((size_t)row0 + lrow) * D + 32 * cc, v);
+          continue;
+        }
         if (mse) {
           tmem_ld32(tmem + loff + 32 * cc, z);
           tmem_wait_ld();
@@ -790,7 +852,7 @@ struct DkL {
   static constexpr uint32_t T_DK = 0, T_DS = D;
 };
 enum { K_LD0, K_H, K_H_SCALED, K_DO_FULL, K_Q_FULL, K_DS_FULL, K_DP_READY, K_DK_STEP,
-       K_DVW_FULL, K_DK_FULL, K_SCAN, K_ST, K_BG, K_WD, K_NBARS };
+       K_DVW_FULL, K_DK_FULL, K_SCAN, K_ST, K_BG, K_WD, K_DZ_SCALED, K_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kSmallThreads, 2)
@@ -814,8 +876,9 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
   const int c = (blockIdx.x / NB) % p.NC;
   const int bh = blockIdx.x / (NB * p.NC);
   const bool mse = p.loss == 0;
+  const bool zterm = mse || p.silu;  // dK += dZ W0^T is present
   const int counts[K_NBARS] = {1, 1, kSmallEpi, 1, 1, 1, kSmallEpi, 1, 1, 1, 1, kSmallEpi, 1,
-                               kSmallEpi};
+                               kSmallEpi, kSmallEpi};
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmG);
     tma_prefetch_desc(&tmDW);
@@ -867,11 +930,11 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
       // dV into slot B and (MSE) W0 into slot A after the last score MMA and dK step
       if (ok && mbar_wait(BAR(K_DS_FULL), (nq - 1) & 1, ab) &&
           mbar_wait(BAR(K_DK_STEP), (nq - 1) & 1, ab)) {
-        mbar_arrive_expect_tx(BAR(K_DVW_FULL), L::BLK + (mse ? L::WSZ : 0));
+        mbar_arrive_expect_tx(BAR(K_DVW_FULL), L::BLK + (zterm ? L::WSZ : 0));
 #pragma unroll
         for (int kp = 0; kp < L::KP; ++kp) {
           tma_load_2d(sB + kp * PANEL128, &tmDV, BAR(K_DVW_FULL), 64 * kp, tokc + 128 * rb);
-          if (mse) tma_load_2d(sA + kp * D * 128, &tmW, BAR(K_DVW_FULL), 64 * kp, wrow);
+          if (zterm) tma_load_2d(sA + kp * D * 128, &tmW, BAR(K_DVW_FULL), 64 * kp, wrow);
         }
       }
     }
@@ -913,9 +976,9 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
           mma_commit(BAR(K_DK_STEP));
         }
         if (!ok) break;
-        if (mse) {
-          // dK += dZ W0^T with dZ = -dV (negated A)
-          if (!mbar_wait(BAR(K_DVW_FULL), 0, ab)) break;
+        if (zterm) {
+          // dK += dZ W0^T with dZ = -dV (MSE, identity) or -(-dG F2) (SiLU): negated A
+          if (!mbar_wait(BAR(p.silu ? K_DZ_SCALED : K_DVW_FULL), 0, ab)) break;
           tc_fence_after();
 #pragma unroll
           for (int j = 0; j < D / 16; ++j)
@@ -981,6 +1044,33 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
         }
         p.dbeta[(size_t)tokc + r] = -(1.f - 0.5f * er) * dot;
         e_r = dot;
+      }
+      if (p.silu) {
+        // the row holds -dG: dV = -dG F1 goes out, -dG F2 (= -dZ) stays for the MMA
+        const size_t grow = ((size_t)tokc + r) * D;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          float v[32], o[32];
+          ld_row32(sB + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+          const uint4* f1 = reinterpret_cast<const uint4*>(p.F1 + grow + 32 * cc);
+          const uint4* f2 = reinterpret_cast<const uint4*>(p.F2 + grow + 32 * cc);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint4 a = f1[k], b = f2[k];
+            const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const int j = 8 * k + 2 * h;
+              o[j] = v[j] * bf16lo(wa[h]);
+              o[j + 1] = v[j + 1] * bf16hi(wa[h]);
+              v[j] *= bf16lo(wb[h]);
+              v[j + 1] *= bf16hi(wb[h]);
+            }
+          }
+          st_global_bf16x32(p.dV_out + grow + 32 * cc, o);
+          st_row32(sB + (cc / 2) * PANEL128, lrow, 4 * (cc % 2), v);
+        }
+        epi_arrive(BAR(K_DZ_SCALED));
       }
       // dK staged over this thread's own row of G (every reader of G is done), one bulk store
       if (!mbar_wait(BAR(K_DK_FULL), 0, ab)) break;
@@ -1062,6 +1152,29 @@ __global__ void __launch_bounds__(C)
   dgamma[row] = (x + later) / gamma[row];
 }
 
+// dZq = dO * act'(Zq) for SiLU, eight elements per step.
+__global__ void __launch_bounds__(256)
+    bwd_dzq_kernel(const __nv_bfloat16* dO, const __nv_bfloat16* Zq, __nv_bfloat16* dZq, size_t n8) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 a = reinterpret_cast<const uint4*>(dO)[i];
+    const uint4 z = reinterpret_cast<const uint4*>(Zq)[i];
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wz[4] = {z.x, z.y, z.z, z.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float zz[2] = {bf16lo(wz[h]), bf16hi(wz[h])}, d[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float sg = 1.f / (1.f + __expf(-zz[e]));
+        d[e] = sg * (1.f + zz[e] * (1.f - sg));
+      }
+      o[h] = pack_bf16x2(bf16lo(wa[h]) * d[0], bf16hi(wa[h]) * d[1]);
+    }
+    reinterpret_cast<uint4*>(dZq)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
 #undef BAR
 
 // Per-device pair of internal streams (chain then dk at the higher priority; g then dq at the
@@ -1102,23 +1215,41 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
   const int BH = a.B * a.H, NC = a.T / a.C;
   const uint64_t wrows = (uint64_t)BH * NC * D;
-  __nv_bfloat16* dWs = static_cast<__nv_bfloat16*>(a.ws);
   const bool g_saved = a.G_saved != nullptr;
-  __nv_bfloat16* G = g_saved ? static_cast<__nv_bfloat16*>(a.G_saved) : dWs + wrows * D;
+  const bool silu = a.act == 1;  // requires G_saved (its second plane is Zq)
+  const uint64_t plane = rows * D;
+  // workspace: chunk-end adjoints | G (without G_saved) | dK's dgamma terms | SiLU: dZq, F1,
+  // F2, -dG
+  __nv_bfloat16* dWs = static_cast<__nv_bfloat16*>(a.ws);
+  uint8_t* wp = reinterpret_cast<uint8_t*>(dWs + wrows * D);
+  __nv_bfloat16* G = g_saved ? static_cast<__nv_bfloat16*>(a.G_saved)
+                             : reinterpret_cast<__nv_bfloat16*>(wp);
+  if (!g_saved) wp += plane * 2;
+  float* dgk = a.dgamma ? reinterpret_cast<float*>(wp) : nullptr;
+  if (a.dgamma) wp += rows * 4;
+  __nv_bfloat16* dZq = silu ? reinterpret_cast<__nv_bfloat16*>(wp) : nullptr;
+  __nv_bfloat16* F1 = silu ? dZq + plane : nullptr;
+  __nv_bfloat16* F2 = silu ? F1 + plane : nullptr;
+  __nv_bfloat16* mdG = silu ? F2 + plane : nullptr;
+  const __nv_bfloat16* Zq = silu ? G + plane : nullptr;
+  // what the kernels read as dO, what the chain stores (and dK reads) as dV, and as O for dgamma
+  const void* dO_k = silu ? static_cast<const void*>(dZq) : a.dO;
+  const void* dV_k = silu ? static_cast<void*>(mdG) : a.dV;
+  const void* O_k = silu ? static_cast<const void*>(Zq) : a.O_in;
   CUtensorMap tK, tQ, tDO, tK1, tV1, tQ1, tDO1, tDV1, tG1, tW, tDW, tDQ1, tDK1, tO1;
   if (!make_tmap_bf16(&tK, a.K, D, rows, D, 64, C) || !make_tmap_bf16(&tQ, a.Q, D, rows, D, 64, C) ||
-      !make_tmap_bf16(&tDO, a.dO, D, rows, D, 64, C) ||
+      !make_tmap_bf16(&tDO, dO_k, D, rows, D, 64, C) ||
       !make_tmap_bf16(&tK1, a.K, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tV1, a.V, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tQ1, a.Q, D, rows, D, 64, 128) ||
-      !make_tmap_bf16(&tDO1, a.dO, D, rows, D, 64, 128) ||
-      !make_tmap_bf16(&tDV1, a.dV, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tDO1, dO_k, D, rows, D, 64, 128) ||
+      !make_tmap_bf16(&tDV1, dV_k, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tDQ1, a.dQ, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tDK1, a.dK, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tG1, G, D, rows, D, 64, 128) ||
       !make_tmap_bf16(&tW, a.W_chunks, D, wrows, D, 64, D) ||
       !make_tmap_bf16(&tDW, dWs, D, wrows, D, 64, D) ||
-      !make_tmap_bf16(&tO1, a.dgamma ? a.O_in : a.dO, D, rows, D, 64, 128))
+      !make_tmap_bf16(&tO1, a.dgamma ? O_k : dO_k, D, rows, D, 64, 128))
     return cudaErrorInvalidValue;
   BwdParams p{};
   p.BH = BH;
@@ -1140,7 +1271,11 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.Wc = static_cast<const __nv_bfloat16*>(a.W_chunks);
   p.W_final = a.W_final_in;
   p.dgamma = a.dgamma;
-  p.dgk = reinterpret_cast<float*>(dWs + wrows * D + (g_saved ? 0 : rows * D));
+  p.dgk = dgk;
+  p.silu = silu;
+  p.F1 = F1;
+  p.F2 = F2;
+  p.dV_out = static_cast<__nv_bfloat16*>(a.dV);
   p.err = a.err;
 
   const size_t sm_g = GL<D>::BYTES + 1024;
@@ -1160,14 +1295,25 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   std::lock_guard<std::mutex> lk(g_fork_mu);
   ForkSet* f = fork_set();
   if (!f) return cudaErrorInitializationError;
+  int launched = g_saved ? 3 : 4;
+  if (silu) {
+    // dZq before the fork: the chain, dQ and dK all read it
+    bwd_dzq_kernel<<<2048, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.dO), Zq, dZq,
+                                        plane / 8);
+    ++launched;
+  }
   if ((e = cudaEventRecord(f->e0, s)) || (e = cudaStreamWaitEvent(f->hi, f->e0, 0)) ||
       (e = cudaStreamWaitEvent(f->lo, f->e0, 0)))
     return e;
+  if (silu) {
+    // F1, F2 (the chain scales -dG by F2)
+    kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->hi>>>(tK1, tW, tV1, p);
+    ++launched;
+  }
   kc<<<BH * p.nslice, kThreads, sm_chain, f->hi>>>(tK, tQ, tDO, tDV1, tDW, p);
   if (!g_saved) kg<<<(int)(rows / 128), kSmallThreads, sm_g, f->lo>>>(tK1, tW, tV1, p);
   if ((e = cudaEventRecord(f->eg, f->lo))) return e;
   kq<<<BH * NC * NB, kSmallThreads, sm_dq, f->lo>>>(tDO1, tW, tK1, tG1, tDQ1, tO1, p);
-  int launched = g_saved ? 3 : 4;
   if ((e = cudaEventRecord(f->elo, f->lo)) || (e = cudaStreamWaitEvent(f->hi, f->eg, 0))) return e;
   kk<<<BH * NC * NB, kSmallThreads, sm_dk, f->hi>>>(tG1, tDW, tQ1, tDO1, tDV1, tW, tDK1, p);
   if (a.dgamma) {
@@ -1185,17 +1331,19 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// SiLU also needs the forward's saved G and Zq (checked where the path is chosen).
 bool tc_bwd_supported(const LayerArgs& a) {
-  return a.dtype == 1 && a.act == 0 && !a.gvec && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
+  return a.dtype == 1 && !a.gvec && a.dk == a.dv && (a.dk == 64 || a.dk == 128) &&
          (a.C == 128 || a.C == 256) && a.T % a.C == 0;
 }
 
 // [BH, NC, dk, dv] bf16 chunk-end adjoints, then (without G from the forward) [BH, T, dv] bf16 G,
-// then (for the decay gradient) [BH, T] float32 per-token sums of the dK kernel
+// then (for the decay gradient) [BH, T] float32 per-token sums of the dK kernel, then (SiLU)
+// four [BH, T, dv] bf16 planes: dZq, F1, F2 and -dG
 size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved, bool dgamma) {
-  return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2 +
-         (g_saved ? 0 : (size_t)a.B * a.H * a.T * a.dv * 2) +
-         (dgamma ? (size_t)a.B * a.H * a.T * 4 : 0);
+  const size_t plane = (size_t)a.B * a.H * a.T * a.dv * 2;
+  return (size_t)a.B * a.H * (a.T / a.C) * a.dk * a.dv * 2 + (g_saved ? 0 : plane) +
+         (dgamma ? (size_t)a.B * a.H * a.T * 4 : 0) + (a.act == 1 ? 4 * plane : 0);
 }
 
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s) {

@@ -54,6 +54,7 @@ struct FwdParams {
   float* W_final;         // nullable
   __nv_bfloat16* W_chunks;  // nullable, [BH, NC, D, D]
   int save_g;               // store G of every token (bulk stores through tmG)
+  __nv_bfloat16* Zq;        // nullable, [BH, T, D]: the SiLU readout before the activation
   unsigned* err;
 };
 
@@ -534,6 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float o[32];
         tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, o);
         tmem_wait_ld();
+        if (ACT == 1 && p.Zq)
+          st_global_bf16x32(p.Zq + (tok0 + 128 * h + lrow) * D + NV * slice + 32 * g, o);
 #pragma unroll
         for (int j = 0; j < 32; ++j) o[j] = act_f<ACT>(o[j]);
         tc_fence_before();
@@ -581,6 +584,8 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.W_final = a.W_final;
   p.W_chunks = static_cast<__nv_bfloat16*>(a.W_chunks);
   p.save_g = a.G_saved != nullptr;
+  // with SiLU the saved buffer has a second plane for Zq, which the backward needs for dZq
+  p.Zq = ACT == 1 && a.G_saved ? static_cast<__nv_bfloat16*>(a.G_saved) + rows * D : nullptr;
   p.err = a.err;
   const size_t smem = L::BYTES + 1024;
   auto k = ttt_fwd_tc_kernel<D, NB, ACT, LOSS>;

@@ -77,7 +77,8 @@ template <typename TI>
 __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, const TI* K,
                                                        const TI* V, const float* beta,
                                                        const float* gamma, const float* W0,
-                                                       TI* O, float* Wf, TI* Wc, TI* Gs) {
+                                                       TI* O, float* Wf, TI* Wc, TI* Gs,
+                                                       TI* Zs) {
   extern __shared__ float smem[];
   const int bh = blockIdx.y, j0 = blockIdx.x * kNvs;
   const int nv = min(kNvs, d.dv - j0);
@@ -146,6 +147,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
           acc *= expf(L[s]);
         }
         for (int r = 0; r <= s; ++r) acc -= S[sr * C + r] * G[r * kNvs + j];
+        if (Zs) stf(&Zs[v0 + (tc + s) * dv + j0 + j], acc);
         stf(&O[v0 + (tc + s) * dv + j0 + j], actf(d.act, acc));
       }
       __syncthreads();
@@ -399,6 +401,9 @@ Dims dims_of(const LayerArgs& a) {
   return Dims{a.T, a.dk, a.dv, a.C, a.loss, a.act, a.gamma != nullptr, a.gvec, a.lr_bias};
 }
 
+// Elements of one [B, H, T, dv] plane: with SiLU, Zq follows G in the saved buffer.
+size_t zq_plane(const LayerArgs& a) { return (size_t)a.B * a.H * a.T * a.dv; }
+
 size_t fwd_smem_bytes(const LayerArgs& a) {
   const size_t lw = a.gvec ? a.dk : 1;
   return sizeof(float) *
@@ -424,16 +429,18 @@ cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
   if (a.dtype == 0) {
     auto k = simt_fwd_kernel<float>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    float* gs = (float*)a.G_saved;
     k<<<grid, 256, smem, s>>>(d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta,
-                              a.gamma, a.W0, (float*)a.O, a.W_final, (float*)a.W_chunks,
-                              (float*)a.G_saved);
+                              a.gamma, a.W0, (float*)a.O, a.W_final, (float*)a.W_chunks, gs,
+                              gs && a.act ? gs + zq_plane(a) : nullptr);
   } else {
     auto k = simt_fwd_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    __nv_bfloat16* gs = (__nv_bfloat16*)a.G_saved;
     k<<<grid, 256, smem, s>>>(d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K,
                               (const __nv_bfloat16*)a.V, a.beta, a.gamma, a.W0,
-                              (__nv_bfloat16*)a.O, a.W_final, (__nv_bfloat16*)a.W_chunks,
-                              (__nv_bfloat16*)a.G_saved);
+                              (__nv_bfloat16*)a.O, a.W_final, (__nv_bfloat16*)a.W_chunks, gs,
+                              gs && a.act ? gs + zq_plane(a) : nullptr);
   }
   count_launches(1);
   return cudaGetLastError();
