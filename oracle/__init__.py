@@ -10,7 +10,9 @@ cpu_baseline / reference leg may import this package. The product library
   section "核心方法和技术细节", the chunkwise apply-then-update rule
   W^(i+1) = W^(i) + eta * Vhat_[i]^T Z_[i]) with fp64 numpy matmuls;
   inplace_bwd is the reverse-mode of that loop (the pages print no backward),
-  inplace_bwd_dz_tokens evaluates sampled rows of its dZ at any size.
+  inplace_bwd_dz_tokens evaluates sampled rows of its dZ at any size;
+  inplace_target is the NTP-aligned target Vhat = Conv1D(X0) W_target of the same
+  section, with its reverse-mode inplace_target_bwd.
 
 Every function here is pinned by tests/test_oracle_pins.py; no function is
 "parity unpinned" except for absolute agreement with the authors' own
@@ -226,3 +228,38 @@ def inplace_bwd_dz_tokens(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, t
         row = row + lr * ((do[hi:] @ vh[t]) @ z[hi:])
         out[n] = row
     return out
+
+
+def inplace_target(X0, conv_w, W_target):
+    """NTP-aligned target of In-Place TTT (page "In-Place Test-Time Training", section
+    "核心方法和技术细节": Vhat = Conv1D(X0) W_target, the convolution reading nearby future
+    tokens), in fp64. Reading: a depthwise convolution over the current and the next k - 1
+    tokens, Y_t = sum_{j<k} conv_w[j] * X0_{t+j} (per channel, zero past the last token), then
+    Vhat = Y W_target with row vectors.
+    X0: [T, d]; conv_w: [k, d]; W_target: [d, d_out]. Returns (Vhat [T, d_out], Y [T, d])."""
+    x = _np(X0, np.float64)
+    w = _np(conv_w, np.float64)
+    wt = _np(W_target, np.float64)
+    T = x.shape[0]
+    y = np.zeros_like(x)
+    for j in range(w.shape[0]):
+        y[: T - j] += w[j] * x[j:]
+    return y @ wt, y
+
+
+def inplace_target_bwd(X0, conv_w, W_target, dVhat):
+    """Reverse-mode of inplace_target for J = <dVhat, Vhat> (fp64): returns dict dX0 [T, d],
+    dconv_w [k, d] and dW_target [d, d_out]."""
+    x = _np(X0, np.float64)
+    w = _np(conv_w, np.float64)
+    wt = _np(W_target, np.float64)
+    dv = _np(dVhat, np.float64)
+    _, y = inplace_target(x, w, wt)
+    dy = dv @ wt.T
+    T = x.shape[0]
+    dx = np.zeros_like(x)
+    dw = np.zeros_like(w)
+    for j in range(w.shape[0]):
+        dx[j:] += w[j] * dy[: T - j]
+        dw[j] = (dy[: T - j] * x[j:]).sum(axis=0)
+    return dict(dX0=dx, dconv_w=dw, dW_target=y.T @ dv)

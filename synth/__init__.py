@@ -166,3 +166,22 @@ def inplace_inputs(cfg: InPlaceConfig, device="cpu", seed: int | None = None) ->
     w = 0.02 * _randn((cfg.d_model, cfg.d_ff), g, device)
     do = _randn((cfg.T, cfg.d_model), g, device).to(torch.bfloat16)
     return dict(Z=z.contiguous(), Vhat=vhat.contiguous(), W=w.contiguous(), dO=do.contiguous())
+
+
+def inplace_target_inputs(cfg: InPlaceConfig, k: int = 4, device="cpu", seed: int | None = None) -> dict:
+    """Draw the inputs of the NTP-aligned target Vhat = Conv1D(X0) W_target (page "In-Place
+    Test-Time Training", section "核心方法和技术细节"): token embeddings X0 ~ N(0, 0.02)
+    [T, d_model] bf16, depthwise taps conv_w ~ N(0, 1/k) [k, d_model] float32 over the current
+    and the next k - 1 tokens, W_target ~ N(0, 1/sqrt(d_model)) [d_model, d_model] bf16 (input
+    rows, output columns), and an upstream gradient dVhat ~ N(0, 1) [T, d_model] bf16. The
+    page gives no window size; k = 4 is this workload's choice. Seeded apart from
+    inplace_inputs (seed + 1000)."""
+    seed = (cfg.seed if seed is None else seed) + 1000
+    g = make_generator(seed, device)
+    d = cfg.d_model
+    x0 = (0.02 * _randn((cfg.T, d), g, device)).to(torch.bfloat16)
+    w = _randn((k, d), g, device) / math.sqrt(k)
+    wt = (_randn((d, d), g, device) / math.sqrt(d)).to(torch.bfloat16)
+    dv = _randn((cfg.T, d), g, device).to(torch.bfloat16)
+    return dict(X0=x0.contiguous(), conv_w=w.contiguous(), W_target=wt.contiguous(),
+                dVhat=dv.contiguous())

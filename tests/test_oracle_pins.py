@@ -20,7 +20,9 @@
   associativity of the update, plain GEMM when C = T or eta = 0, and the
   dual form with Z_i Z_j^T corrections; its backward against finite
   differences, the single-chunk closed form, and the row-subset and
-  sampled-token evaluations against the full one.
+  sampled-token evaluations against the full one; the NTP-aligned target
+  against shifted copies (one-hot taps) and a plain matmul (one tap), and
+  its backward against finite differences.
 """
 import itertools
 import math
@@ -534,3 +536,45 @@ def test_inplace_backward_row_subset_and_sampled_tokens_are_exact():
     dz0 = oracle.inplace_bwd_dz_tokens(Z, Vh, W, dO, None, C=C, lr=lr, tokens=tokens)
     g0 = oracle.inplace_bwd(Z, Vh, W, dO, None, C=C, lr=lr)
     np.testing.assert_allclose(dz0, g0["dZ"][tokens], atol=1e-12)
+
+
+def test_inplace_target_special_cases():
+    # one tap at offset j with weight 1 and W_target = I: Vhat is X0 shifted j tokens up
+    rng = np.random.default_rng(47)
+    T, d, k = 12, 5, 4
+    X0 = rng.standard_normal((T, d))
+    for j in range(k):
+        w = np.zeros((k, d))
+        w[j] = 1.0
+        V, _ = oracle.inplace_target(X0, w, np.eye(d))
+        want = np.zeros_like(X0)
+        want[: T - j] = X0[j:]
+        np.testing.assert_array_equal(V, want)
+    # a single tap (k = 1) makes it a per-channel scale followed by a plain matmul
+    w1 = rng.standard_normal((1, d))
+    Wt = rng.standard_normal((d, 3))
+    V, _ = oracle.inplace_target(X0, w1, Wt)
+    np.testing.assert_allclose(V, (X0 * w1[0]) @ Wt, atol=1e-12)
+
+
+def test_inplace_target_backward_matches_finite_differences():
+    rng = np.random.default_rng(48)
+    T, d, k, d_out = 7, 3, 3, 2
+    X0 = rng.standard_normal((T, d))
+    w = rng.standard_normal((k, d))
+    Wt = rng.standard_normal((d, d_out))
+    dV = rng.standard_normal((T, d_out))
+    g = oracle.inplace_target_bwd(X0, w, Wt, dV)
+    h = 1e-6
+    for name, x, key in (("X0", X0, "dX0"), ("w", w, "dconv_w"), ("Wt", Wt, "dW_target")):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            jp = float((oracle.inplace_target(X0, w, Wt)[0] * dV).sum())
+            x[idx] = old - h
+            jm = float((oracle.inplace_target(X0, w, Wt)[0] * dV).sum())
+            x[idx] = old
+            fd[idx] = (jp - jm) / (2 * h)
+        err = np.abs(g[key] - fd).max() / np.abs(fd).max()
+        assert err < 1e-8, (name, err)
