@@ -389,7 +389,14 @@ def time_inplace(ttt, steps, warmup):
     ms = timed(fwd, False)
     ms_save = timed(fwd, True)
     ms_bwd = timed(bwd, None)
-    return icfg, ms, ms_save, ms_bwd
+    # the NTP-aligned target Vhat = Conv1D(X0) W_target (4 taps) on the same sequence
+    tin = synth.inplace_target_inputs(icfg, k=4, device="cuda")
+    nt = ttt.inplace_ttt_target_workspace_bytes(T, M)
+    wst = torch.empty(nt, device="cuda", dtype=torch.uint8)
+    Vt = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+    ms_tgt = timed(lambda _: ttt.inplace_ttt_target(T, M, 4, tin["X0"], tin["conv_w"],
+                                                    tin["W_target"], Vt, wst, nt), None)
+    return icfg, ms, ms_save, ms_bwd, ms_tgt
 
 
 # --------------------------------------------------------------------------- oracle legs
@@ -549,7 +556,7 @@ def main():
     if not args.no_configs:
         out["other_configs"] = time_other_configs(ttt, peaks)
     if not args.no_inplace:
-        icfg, ims, ims_save, ims_bwd = time_inplace(ttt, steps=3, warmup=1)
+        icfg, ims, ims_save, ims_bwd, ims_tgt = time_inplace(ttt, steps=3, warmup=1)
         fl, by = inplace_work(icfg)
         tf = fl / (ims * 1e-3) / 1e12
         out["inplace"] = {"workload": icfg.name, "ms": ims, "tokens_per_s": icfg.T / (ims * 1e-3),
@@ -570,6 +577,15 @@ def main():
                                            "unit": "TFLOP/s",
                                            "frac": tfb / peaks["bf16_tflops_sustained"],
                                            "peak_source": peak_src}}
+        # NTP target: 2 T d_model^2 flops of projection (the 4-tap convolution is HBM work)
+        tft = 2 * icfg.T * icfg.d_model ** 2 / (ims_tgt * 1e-3) / 1e12
+        out["inplace_target"] = {"workload": "inplace-ttt-ntp-target-k4", "ms": ims_tgt,
+                                 "tokens_per_s": icfg.T / (ims_tgt * 1e-3),
+                                 "roofline": {"bound": "tensor", "achieved": tft,
+                                              "peak": peaks["bf16_tflops_sustained"],
+                                              "unit": "TFLOP/s",
+                                              "frac": tft / peaks["bf16_tflops_sustained"],
+                                              "peak_source": peak_src}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg)
     if _dist is not None:

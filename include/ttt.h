@@ -179,6 +179,24 @@ ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const 
                            const void* Vhat, float* W, void* O, void* W_chunks, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Workspace bytes of inplace_ttt_target; (size_t)-1 for invalid sizes. */
+size_t inplace_ttt_target_workspace_bytes(int T, int d_model);
+
+/* NTP-aligned update target of In-Place TTT (page "In-Place Test-Time Training", section
+ * "核心方法和技术细节": Vhat = Conv1D(X0) W_target, the convolution extracting nearby future
+ * tokens of the embeddings). Reading: a depthwise convolution over the current and the next
+ * k - 1 tokens, zero past the last token, then the projection with row vectors:
+ *     Y_t = sum_{j<k} conv_w[j] * X0_{t+j}   (per channel),   Vhat = Y W_target.
+ *  X0        [T, d_model]       bf16     token embeddings
+ *  conv_w    [k, d_model]       float32  tap j weights token t + j
+ *  W_target  [d_model, d_model] bf16     input rows, output columns
+ *  Vhat      [T, d_model]       bf16     out (the Vhat of inplace_ttt_fwd)
+ * Requirements: T % 128 == 0, d_model % 128 == 0, 1 <= k <= 8. Y is rounded to bf16 before
+ * the projection. */
+ttt_status inplace_ttt_target(int T, int d_model, int k, const void* X0, const float* conv_w,
+                              const void* W_target, void* Vhat, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* Backward of inplace_ttt_fwd (no counterpart on the page, which gives only the forward): the
  * reverse-mode of the apply-then-update loop for J = sum_i <dO_i, O_i> + <dW_final, W_final>.
  * With Wh the adjoint of the fast weight (dW_final, or 0, after the last chunk), chunk i from

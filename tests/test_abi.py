@@ -8,7 +8,7 @@ import pytest
 import weight_sequence_layers_b200 as ttt
 
 FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_ttt_workspace_bytes",
-             "inplace_ttt_fwd", "inplace_ttt_bwd", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "inplace_ttt_fwd", "inplace_ttt_bwd", "inplace_ttt_target", "inplace_ttt_target_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
              "ttt_status_string"}
 
 
@@ -179,3 +179,19 @@ def test_valid_call_without_a_gpu_reports_cuda_error():
     st = ttt.lib.ttt_chunk_fwd(ctypes.byref(cfg), A, A, A, A, None, A, A, None, None, None, None, 0,
                                None)
     assert st == ttt.ERR_CUDA
+
+
+def test_inplace_target_argument_errors():
+    A = 4096
+    f = ttt.lib.inplace_ttt_target
+    need = ttt.inplace_ttt_target_workspace_bytes(256, 128)
+    assert need >= 256 * 128 * 2
+    # T d_model k X0 conv_w W_target Vhat workspace bytes stream
+    assert f(256, 128, 0, A, A, A, A, A, need, None) == ttt.ERR_INVALID_ARG     # k < 1
+    assert f(256, 128, 9, A, A, A, A, A, need, None) == ttt.ERR_UNSUPPORTED     # k > 8
+    assert f(200, 128, 4, A, A, A, A, A, need, None) == ttt.ERR_UNSUPPORTED     # T % 128
+    assert f(256, 128, 4, None, A, A, A, A, need, None) == ttt.ERR_INVALID_ARG
+    assert f(256, 128, 4, A, A + 4, A, A, A, need, None) == ttt.ERR_ALIGNMENT
+    assert f(256, 128, 4, A, A, A, A, A, need - 1, None) == ttt.ERR_WORKSPACE
+    with pytest.raises(ttt.TTTError):
+        ttt.inplace_ttt_target_workspace_bytes(256, 100)

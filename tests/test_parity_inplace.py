@@ -123,3 +123,35 @@ def test_inplace_backward_full_size_sampled():
     dz = oracle.inplace_bwd_dz_tokens(inp["Z"], inp["Vhat"], inp["W"], inp["dO"], None, C=cfg.C,
                                       lr=lr32, tokens=tokens)
     assert rel_err(dZ[tokens], dz) <= O_TOL
+
+
+def run_target(T, d, k, tin):
+    V = torch.full((T, d), float("nan"), device="cuda", dtype=torch.bfloat16)
+    n = ttt.inplace_ttt_target_workspace_bytes(T, d)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    ttt.inplace_ttt_target(T, d, k, tin["X0"], tin["conv_w"], tin["W_target"], V, ws, n)
+    torch.cuda.synchronize()
+    assert ttt.ttt_get_device_error() == ttt.OK
+    return V
+
+
+@pytest.mark.parametrize("T,d,k", [(256, 128, 1), (512, 256, 4), (384, 384, 8), (128, 640, 3)])
+def test_inplace_target_small(T, d, k):
+    cfg = synth.INPLACE_QWEN4B.replace(T=T, d_model=d)
+    tin = synth.inplace_target_inputs(cfg, k=k, device="cuda", seed=T + d + k)
+    V = run_target(T, d, k, tin)
+    ref, _ = oracle.inplace_target(tin["X0"], tin["conv_w"], tin["W_target"])
+    assert rel_err(V, ref) <= O_TOL
+
+
+def test_inplace_target_full_size_sampled_tokens():
+    cfg = synth.INPLACE_QWEN4B
+    k = 4
+    tin = synth.inplace_target_inputs(cfg, k=k, device="cuda")
+    V = run_target(cfg.T, cfg.d_model, k, tin)
+    # Vhat_t needs X0 rows t .. t+k-1 only: slice windows around sampled tokens, and the tail
+    for t0 in (0, 4093, cfg.T // 2 + 5, cfg.T - 32):
+        m = min(32, cfg.T - t0)
+        hi = min(cfg.T, t0 + m + k - 1)
+        ref, _ = oracle.inplace_target(tin["X0"][t0:hi], tin["conv_w"], tin["W_target"])
+        assert rel_err(V[t0:t0 + m], ref[:m]) <= O_TOL, t0

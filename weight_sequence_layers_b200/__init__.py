@@ -50,6 +50,8 @@ _SIGS = {
     "inplace_ttt_workspace_bytes": ([_i] * 4, _sz),
     "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 6 + [_sz, _p], _i),
     "inplace_ttt_bwd": ([_i] * 4 + [_f] + [_p] * 9 + [_sz, _p], _i),
+    "inplace_ttt_target_workspace_bytes": ([_i] * 2, _sz),
+    "inplace_ttt_target": ([_i] * 3 + [_p] * 5 + [_sz, _p], _i),
     "ttt_get_device_error": ([_p], _i),
     "ttt_selftest_bounded_wait": ([_u, _p], _i),
     "ttt_status_string": ([_i], ctypes.c_char_p),
@@ -155,6 +157,20 @@ def inplace_ttt_fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace=None, work
                               _ptr(O), _ptr(W_chunks), _ptr(workspace), int(workspace_bytes),
                               _stream(stream))
     _check(st, "inplace_ttt_fwd")
+
+
+def inplace_ttt_target_workspace_bytes(T, d_model) -> int:
+    n = _lib.inplace_ttt_target_workspace_bytes(T, d_model)
+    if n == ctypes.c_size_t(-1).value:
+        raise TTTError(ERR_INVALID_ARG, "inplace_ttt_target_workspace_bytes")
+    return n
+
+
+def inplace_ttt_target(T, d_model, k, X0, conv_w, W_target, Vhat, workspace=None,
+                       workspace_bytes=0, stream=None):
+    st = _lib.inplace_ttt_target(T, d_model, k, _ptr(X0), _ptr(conv_w), _ptr(W_target), _ptr(Vhat),
+                                 _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "inplace_ttt_target")
 
 
 def inplace_ttt_bwd(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW,

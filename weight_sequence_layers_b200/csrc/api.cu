@@ -285,6 +285,31 @@ ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const 
                                    err, static_cast<cudaStream_t>(stream)));
 }
 
+size_t inplace_ttt_target_workspace_bytes(int T, int d_model) {
+  if (T < 1 || d_model < 1 || T % 128 || d_model % 128 || (long long)T * d_model > (1ll << 40))
+    return (size_t)-1;
+  return inplace_target_workspace(T, d_model);
+}
+
+ttt_status inplace_ttt_target(int T, int d_model, int k, const void* X0, const float* conv_w,
+                              const void* W_target, void* Vhat, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (T < 1 || d_model < 1 || k < 1 || (long long)T * d_model > (1ll << 40))
+    return TTT_ERR_INVALID_ARG;
+  if (T % 128 || d_model % 128 || k > 8) return TTT_ERR_UNSUPPORTED;
+  if (!X0 || !conv_w || !W_target || !Vhat) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {X0, conv_w, W_target, Vhat, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const size_t need = inplace_target_workspace(T, d_model);
+  if (!workspace || workspace_bytes < need) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  return launch_status(inplace_target_run(T, d_model, k, X0, conv_w, W_target, Vhat, workspace,
+                                          err, static_cast<cudaStream_t>(stream)));
+}
+
 ttt_status inplace_ttt_bwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
                            const void* Vhat, const void* W_chunks, const void* dO,
                            const float* dW_final, void* dZ, void* dVhat, float* dW,

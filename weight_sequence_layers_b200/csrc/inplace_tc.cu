@@ -320,6 +320,40 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
 
 constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(Bars) + 1024;
 
+// Depthwise convolution over the current and the next k - 1 tokens, zero past the last one:
+// Y[t, c] = sum_{j<k} w[j, c] X0[t + j, c]. One thread per 8 channels and a run of tokens;
+// a warp's loads of one token row are contiguous.
+constexpr int kMaxTaps = 8;
+__global__ void __launch_bounds__(128)
+    conv_future_kernel(const __nv_bfloat16* __restrict__ X0, const float* __restrict__ w,
+                       __nv_bfloat16* __restrict__ Y, int T, int d, int k, int run) {
+  const int c8 = blockIdx.x * blockDim.x + threadIdx.x;  // group of 8 channels
+  if (c8 * 8 >= d) return;
+  float wv[kMaxTaps][8];
+#pragma unroll
+  for (int j = 0; j < kMaxTaps; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) wv[j][e] = j < k ? w[(size_t)j * d + c8 * 8 + e] : 0.f;
+  const int t0 = blockIdx.y * run, t1 = min(T, t0 + run);
+  for (int t = t0; t < t1; ++t) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < kMaxTaps; ++j) {
+      if (j >= k || t + j >= T) break;
+      const uint4 x = *reinterpret_cast<const uint4*>(X0 + (size_t)(t + j) * d + c8 * 8);
+      const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        acc[2 * h] += wv[j][2 * h] * bf16lo(xw[h]);
+        acc[2 * h + 1] += wv[j][2 * h + 1] * bf16hi(xw[h]);
+      }
+    }
+    *reinterpret_cast<uint4*>(Y + (size_t)t * d + c8 * 8) =
+        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                   pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
 struct Launch {
   int sms;
 };
@@ -465,6 +499,46 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
                                                             tmbn, p);
   }
   count_launches(NC + 1);
+  return cudaGetLastError();
+}
+
+size_t inplace_target_workspace(int T, int d) { return (size_t)T * d * 2 + 256; }
+
+// Vhat = Conv1D(X0) W_target: the convolution into bf16 Y (workspace), then Y W_target as one
+// launch of dz-kind tiles (A = Y K-major, B = W_target [d rows, d cols] MN-major, K = d).
+cudaError_t inplace_target_run(int T, int d, int k, const void* X0, const float* conv_w,
+                               const void* W_target, void* Vhat, void* ws, unsigned* err,
+                               cudaStream_t s) {
+  __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(ws);
+  int* counter = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + (size_t)T * d * 2);
+  CUtensorMap ty, twt;
+  if (!make_tmap_bf16(&ty, Y, d, T, d, BK, BM) || !make_tmap_bf16(&twt, W_target, d, d, d, 64, BK))
+    return cudaErrorInvalidValue;
+  Launch l;
+  cudaError_t e = prepare(&l);
+  if (e != cudaSuccess) return e;
+  constexpr int kRun = 32;
+  conv_future_kernel<<<dim3((d / 8 + 127) / 128, (T + kRun - 1) / kRun), 128, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(X0), conv_w, Y, T, d, k, kRun);
+  e = cudaMemsetAsync(counter, 0, sizeof(int), s);
+  if (e != cudaSuccess) return e;
+  Params p{};
+  p.chunk = 0;
+  p.C = T;  // one "chunk": the whole sequence
+  p.d_ff = d;
+  p.d_model = d;
+  p.n_dz_n = (d + BN - 1) / BN;
+  p.n_dz = (T / BM) * p.n_dz_n;
+  p.n_total = p.n_dz;
+  p.kb_dz = d / BK;
+  p.kb_dz_split = p.kb_dz;  // every k-block from the first operand pair
+  p.wb_next_row0 = -1;
+  p.Odz = static_cast<__nv_bfloat16*>(Vhat);
+  p.counter = counter;
+  p.err = err;
+  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
+  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(ty, ty, ty, ty, ty, ty, twt, twt, p);
+  count_launches(2);
   return cudaGetLastError();
 }
 
