@@ -396,7 +396,16 @@ def time_inplace(ttt, steps, warmup):
     Vt = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
     ms_tgt = timed(lambda _: ttt.inplace_ttt_target(T, M, 4, tin["X0"], tin["conv_w"],
                                                     tin["W_target"], Vt, wst, nt), None)
-    return icfg, ms, ms_save, ms_bwd, ms_tgt
+    del wst
+    ntb = ttt.inplace_ttt_target_bwd_workspace_bytes(T, M, 4)
+    wsb = torch.empty(ntb, device="cuda", dtype=torch.uint8)
+    dX0 = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+    dcw = torch.empty((4, M), device="cuda", dtype=torch.float32)
+    dWt = torch.empty((M, M), device="cuda", dtype=torch.float32)
+    ms_tgt_bwd = timed(lambda _: ttt.inplace_ttt_target_bwd(T, M, 4, tin["X0"], tin["conv_w"],
+                                                            tin["W_target"], tin["dVhat"], dX0,
+                                                            dcw, dWt, wsb, ntb), None)
+    return icfg, ms, ms_save, ms_bwd, (ms_tgt, ms_tgt_bwd)
 
 
 # --------------------------------------------------------------------------- oracle legs
@@ -556,7 +565,7 @@ def main():
     if not args.no_configs:
         out["other_configs"] = time_other_configs(ttt, peaks)
     if not args.no_inplace:
-        icfg, ims, ims_save, ims_bwd, ims_tgt = time_inplace(ttt, steps=3, warmup=1)
+        icfg, ims, ims_save, ims_bwd, (ims_tgt, ims_tgt_bwd) = time_inplace(ttt, steps=3, warmup=1)
         fl, by = inplace_work(icfg)
         tf = fl / (ims * 1e-3) / 1e12
         out["inplace"] = {"workload": icfg.name, "ms": ims, "tokens_per_s": icfg.T / (ims * 1e-3),
@@ -586,6 +595,15 @@ def main():
                                               "unit": "TFLOP/s",
                                               "frac": tft / peaks["bf16_tflops_sustained"],
                                               "peak_source": peak_src}}
+        # its backward: dY = dVhat W_target^T and dW_target = Y^T dVhat, 4 T d_model^2 flops
+        tftb = 4 * icfg.T * icfg.d_model ** 2 / (ims_tgt_bwd * 1e-3) / 1e12
+        out["inplace_target_bwd"] = {"workload": "inplace-ttt-ntp-target-k4-bwd", "ms": ims_tgt_bwd,
+                                     "tokens_per_s": icfg.T / (ims_tgt_bwd * 1e-3),
+                                     "roofline": {"bound": "tensor", "achieved": tftb,
+                                                  "peak": peaks["bf16_tflops_sustained"],
+                                                  "unit": "TFLOP/s",
+                                                  "frac": tftb / peaks["bf16_tflops_sustained"],
+                                                  "peak_source": peak_src}}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(cfg)
     if _dist is not None:

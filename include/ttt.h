@@ -197,6 +197,20 @@ ttt_status inplace_ttt_target(int T, int d_model, int k, const void* X0, const f
                               const void* W_target, void* Vhat, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Workspace bytes of inplace_ttt_target_bwd; (size_t)-1 for invalid sizes. */
+size_t inplace_ttt_target_bwd_workspace_bytes(int T, int d_model, int k);
+
+/* Backward of inplace_ttt_target for J = <dVhat, Vhat> (the page gives only the forward):
+ *     dY = dVhat W_target^T,  dW_target = Y^T dVhat,
+ *     dX0_t = sum_{j<k, t-j>=0} conv_w[j] * dY_{t-j},  dconv_w[j] = sum_t dY_t * X0_{t+j}.
+ *  in : X0, conv_w, W_target as in the forward; dVhat [T, d_model] bf16
+ *  out: dX0 [T, d_model] bf16, dconv_w [k, d_model] float32, dW_target [d_model, d_model]
+ *       float32 (plain stores). Y is recomputed (in bf16); requirements as the forward. */
+ttt_status inplace_ttt_target_bwd(int T, int d_model, int k, const void* X0, const float* conv_w,
+                                  const void* W_target, const void* dVhat, void* dX0,
+                                  float* dconv_w, float* dW_target, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 /* Backward of inplace_ttt_fwd (no counterpart on the page, which gives only the forward): the
  * reverse-mode of the apply-then-update loop for J = sum_i <dO_i, O_i> + <dW_final, W_final>.
  * With Wh the adjoint of the fast weight (dW_final, or 0, after the last chunk), chunk i from

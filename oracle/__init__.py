@@ -247,13 +247,19 @@ def inplace_target(X0, conv_w, W_target):
     return y @ wt, y
 
 
-def inplace_target_bwd(X0, conv_w, W_target, dVhat):
+def inplace_target_bwd(X0, conv_w, W_target, dVhat, channels=None):
     """Reverse-mode of inplace_target for J = <dVhat, Vhat> (fp64): returns dict dX0 [T, d],
-    dconv_w [k, d] and dW_target [d, d_out]."""
+    dconv_w [k, d] and dW_target [d, d_out]. `channels` (index array into d) restricts all
+    three to those input channels (columns of dX0 and dconv_w, rows of dW_target); every
+    channel's gradients depend only on its own column of X0 and conv_w and its row of W_target,
+    so the restricted result is exact."""
     x = _np(X0, np.float64)
     w = _np(conv_w, np.float64)
     wt = _np(W_target, np.float64)
     dv = _np(dVhat, np.float64)
+    if channels is not None:
+        channels = np.asarray(channels)
+        x, w, wt = x[:, channels], w[:, channels], wt[channels]
     _, y = inplace_target(x, w, wt)
     dy = dv @ wt.T
     T = x.shape[0]

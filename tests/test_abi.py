@@ -8,7 +8,8 @@ import pytest
 import weight_sequence_layers_b200 as ttt
 
 FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_ttt_workspace_bytes",
-             "inplace_ttt_fwd", "inplace_ttt_bwd", "inplace_ttt_target", "inplace_ttt_target_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "inplace_ttt_fwd", "inplace_ttt_bwd", "inplace_ttt_target", "inplace_ttt_target_workspace_bytes",
+             "inplace_ttt_target_bwd", "inplace_ttt_target_bwd_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
              "ttt_status_string"}
 
 
@@ -195,3 +196,20 @@ def test_inplace_target_argument_errors():
     assert f(256, 128, 4, A, A, A, A, A, need - 1, None) == ttt.ERR_WORKSPACE
     with pytest.raises(ttt.TTTError):
         ttt.inplace_ttt_target_workspace_bytes(256, 100)
+
+
+def test_inplace_target_bwd_argument_errors():
+    A = 4096
+    f = ttt.lib.inplace_ttt_target_bwd
+    need = ttt.inplace_ttt_target_bwd_workspace_bytes(256, 128, 4)
+    # T d_model k X0 conv_w W_target dVhat dX0 dconv_w dW_target workspace bytes stream
+    ok = [A, A, A, A, A, A, A, A, need, None]
+    assert f(256, 128, 9, *ok) == ttt.ERR_UNSUPPORTED
+    args = list(ok)
+    args[5] = None  # dconv_w
+    assert f(256, 128, 4, *args) == ttt.ERR_INVALID_ARG
+    args = list(ok)
+    args[8] = need - 1
+    assert f(256, 128, 4, *args) == ttt.ERR_WORKSPACE
+    with pytest.raises(ttt.TTTError):
+        ttt.inplace_ttt_target_bwd_workspace_bytes(256, 128, 0)

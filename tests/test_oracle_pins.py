@@ -578,3 +578,18 @@ def test_inplace_target_backward_matches_finite_differences():
             fd[idx] = (jp - jm) / (2 * h)
         err = np.abs(g[key] - fd).max() / np.abs(fd).max()
         assert err < 1e-8, (name, err)
+
+
+def test_inplace_target_backward_channel_subset_is_exact():
+    rng = np.random.default_rng(49)
+    T, d, k = 10, 6, 3
+    X0 = rng.standard_normal((T, d))
+    w = rng.standard_normal((k, d))
+    Wt = rng.standard_normal((d, 4))
+    dV = rng.standard_normal((T, 4))
+    g = oracle.inplace_target_bwd(X0, w, Wt, dV)
+    ch = np.array([0, 2, 5])
+    gs = oracle.inplace_target_bwd(X0, w, Wt, dV, channels=ch)
+    np.testing.assert_allclose(gs["dX0"], g["dX0"][:, ch], atol=1e-13)
+    np.testing.assert_allclose(gs["dconv_w"], g["dconv_w"][:, ch], atol=1e-13)
+    np.testing.assert_allclose(gs["dW_target"], g["dW_target"][ch], atol=1e-13)

@@ -155,3 +155,39 @@ def test_inplace_target_full_size_sampled_tokens():
         hi = min(cfg.T, t0 + m + k - 1)
         ref, _ = oracle.inplace_target(tin["X0"][t0:hi], tin["conv_w"], tin["W_target"])
         assert rel_err(V[t0:t0 + m], ref[:m]) <= O_TOL, t0
+
+
+def run_target_bwd(T, d, k, tin):
+    dX0 = torch.full((T, d), float("nan"), device="cuda", dtype=torch.bfloat16)
+    dw = torch.full((k, d), float("nan"), device="cuda", dtype=torch.float32)
+    dWt = torch.full((d, d), float("nan"), device="cuda", dtype=torch.float32)
+    n = ttt.inplace_ttt_target_bwd_workspace_bytes(T, d, k)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    ttt.inplace_ttt_target_bwd(T, d, k, tin["X0"], tin["conv_w"], tin["W_target"], tin["dVhat"],
+                               dX0, dw, dWt, ws, n)
+    torch.cuda.synchronize()
+    assert ttt.ttt_get_device_error() == ttt.OK
+    return dict(dX0=dX0, dconv_w=dw, dW_target=dWt)
+
+
+@pytest.mark.parametrize("T,d,k", [(256, 128, 1), (512, 256, 4), (384, 384, 8), (128, 640, 3)])
+def test_inplace_target_backward_small(T, d, k):
+    cfg = synth.INPLACE_QWEN4B.replace(T=T, d_model=d)
+    tin = synth.inplace_target_inputs(cfg, k=k, device="cuda", seed=2 * T + d + k)
+    got = run_target_bwd(T, d, k, tin)
+    ref = oracle.inplace_target_bwd(tin["X0"], tin["conv_w"], tin["W_target"], tin["dVhat"])
+    for key in ("dX0", "dconv_w", "dW_target"):
+        assert rel_err(got[key], ref[key]) <= O_TOL, key
+
+
+def test_inplace_target_backward_full_size_sampled_channels():
+    cfg = synth.INPLACE_QWEN4B
+    k = 4
+    tin = synth.inplace_target_inputs(cfg, k=k, device="cuda")
+    got = run_target_bwd(cfg.T, cfg.d_model, k, tin)
+    ch = np.sort(np.random.default_rng(2).choice(cfg.d_model, 12, replace=False))
+    ref = oracle.inplace_target_bwd(tin["X0"], tin["conv_w"], tin["W_target"], tin["dVhat"],
+                                    channels=ch)
+    assert rel_err(got["dX0"][:, ch], ref["dX0"]) <= O_TOL
+    assert rel_err(got["dconv_w"][:, ch], ref["dconv_w"]) <= O_TOL
+    assert rel_err(got["dW_target"][ch], ref["dW_target"]) <= O_TOL

@@ -52,6 +52,8 @@ _SIGS = {
     "inplace_ttt_bwd": ([_i] * 4 + [_f] + [_p] * 9 + [_sz, _p], _i),
     "inplace_ttt_target_workspace_bytes": ([_i] * 2, _sz),
     "inplace_ttt_target": ([_i] * 3 + [_p] * 5 + [_sz, _p], _i),
+    "inplace_ttt_target_bwd_workspace_bytes": ([_i] * 3, _sz),
+    "inplace_ttt_target_bwd": ([_i] * 3 + [_p] * 8 + [_sz, _p], _i),
     "ttt_get_device_error": ([_p], _i),
     "ttt_selftest_bounded_wait": ([_u, _p], _i),
     "ttt_status_string": ([_i], ctypes.c_char_p),
@@ -171,6 +173,21 @@ def inplace_ttt_target(T, d_model, k, X0, conv_w, W_target, Vhat, workspace=None
     st = _lib.inplace_ttt_target(T, d_model, k, _ptr(X0), _ptr(conv_w), _ptr(W_target), _ptr(Vhat),
                                  _ptr(workspace), int(workspace_bytes), _stream(stream))
     _check(st, "inplace_ttt_target")
+
+
+def inplace_ttt_target_bwd_workspace_bytes(T, d_model, k) -> int:
+    n = _lib.inplace_ttt_target_bwd_workspace_bytes(T, d_model, k)
+    if n == ctypes.c_size_t(-1).value:
+        raise TTTError(ERR_INVALID_ARG, "inplace_ttt_target_bwd_workspace_bytes")
+    return n
+
+
+def inplace_ttt_target_bwd(T, d_model, k, X0, conv_w, W_target, dVhat, dX0, dconv_w, dW_target,
+                           workspace=None, workspace_bytes=0, stream=None):
+    st = _lib.inplace_ttt_target_bwd(T, d_model, k, _ptr(X0), _ptr(conv_w), _ptr(W_target),
+                                     _ptr(dVhat), _ptr(dX0), _ptr(dconv_w), _ptr(dW_target),
+                                     _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "inplace_ttt_target_bwd")
 
 
 def inplace_ttt_bwd(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW,

@@ -310,6 +310,35 @@ ttt_status inplace_ttt_target(int T, int d_model, int k, const void* X0, const f
                                           err, static_cast<cudaStream_t>(stream)));
 }
 
+size_t inplace_ttt_target_bwd_workspace_bytes(int T, int d_model, int k) {
+  if (T < 1 || d_model < 1 || k < 1 || k > 8 || T % 128 || d_model % 128 ||
+      (long long)T * d_model > (1ll << 40))
+    return (size_t)-1;
+  return inplace_target_bwd_workspace(T, d_model, k);
+}
+
+ttt_status inplace_ttt_target_bwd(int T, int d_model, int k, const void* X0, const float* conv_w,
+                                  const void* W_target, const void* dVhat, void* dX0,
+                                  float* dconv_w, float* dW_target, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (T < 1 || d_model < 1 || k < 1 || (long long)T * d_model > (1ll << 40))
+    return TTT_ERR_INVALID_ARG;
+  if (T % 128 || d_model % 128 || k > 8) return TTT_ERR_UNSUPPORTED;
+  if (!X0 || !conv_w || !W_target || !dVhat || !dX0 || !dconv_w || !dW_target)
+    return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {X0, conv_w, W_target, dVhat, dX0, dconv_w, dW_target, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < inplace_target_bwd_workspace(T, d_model, k))
+    return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  return launch_status(inplace_target_bwd_run(T, d_model, k, X0, conv_w, W_target, dVhat, dX0,
+                                              dconv_w, dW_target, workspace, err,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 ttt_status inplace_ttt_bwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
                            const void* Vhat, const void* W_chunks, const void* dO,
                            const float* dW_final, void* dZ, void* dVhat, float* dW,

@@ -354,6 +354,72 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+// Transposed convolution and the tap gradients of one run of tokens, 8 channels per thread:
+// dX0[t, c] = sum_{j<k, t-j>=0} w[j, c] dY[t-j, c]; part[run, j, c] = sum_{t in run, t+j<T}
+// dY[t, c] X0[t+j, c] (summed over the runs by conv_taps_reduce_kernel).
+__global__ void __launch_bounds__(128)
+    conv_future_bwd_kernel(const __nv_bfloat16* __restrict__ X0, const float* __restrict__ w,
+                           const __nv_bfloat16* __restrict__ dY, __nv_bfloat16* __restrict__ dX0,
+                           float* __restrict__ part, int T, int d, int k, int run) {
+  const int c8 = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c8 * 8 >= d) return;
+  float wv[kMaxTaps][8], pw[kMaxTaps][8];
+#pragma unroll
+  for (int j = 0; j < kMaxTaps; ++j)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      wv[j][e] = j < k ? w[(size_t)j * d + c8 * 8 + e] : 0.f;
+      pw[j][e] = 0.f;
+    }
+  const int t0 = blockIdx.y * run, t1 = min(T, t0 + run);
+  auto load8 = [&](const __nv_bfloat16* base, int t, float (&v)[8]) {
+    const uint4 x = *reinterpret_cast<const uint4*>(base + (size_t)t * d + c8 * 8);
+    const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      v[2 * h] = bf16lo(xw[h]);
+      v[2 * h + 1] = bf16hi(xw[h]);
+    }
+  };
+  for (int t = t0; t < t1; ++t) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, g[8], x[8];
+    load8(dY, t, g);
+#pragma unroll
+    for (int j = 0; j < kMaxTaps; ++j) {
+      if (j >= k) break;
+      if (t - j >= 0) {
+        float gj[8];
+        load8(dY, t - j, gj);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += wv[j][e] * gj[e];
+      }
+      if (t + j < T) {
+        load8(X0, t + j, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pw[j][e] += g[e] * x[e];
+      }
+    }
+    *reinterpret_cast<uint4*>(dX0 + (size_t)t * d + c8 * 8) =
+        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                   pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxTaps; ++j)
+    if (j < k)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[((size_t)blockIdx.y * k + j) * d + c8 * 8 + e] = pw[j][e];
+}
+
+// dconv_w[j, c] = sum over the runs of part[run, j, c], in a fixed order.
+__global__ void conv_taps_reduce_kernel(const float* __restrict__ part, float* __restrict__ dw,
+                                        int nrun, int kd) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= kd) return;
+  float s = 0.f;
+  for (int r = 0; r < nrun; ++r) s += part[(size_t)r * kd + i];
+  dw[i] = s;
+}
+
 struct Launch {
   int sms;
 };
@@ -502,6 +568,8 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   return cudaGetLastError();
 }
 
+constexpr int kConvRun = 32;  // tokens per thread in the convolution kernels
+
 size_t inplace_target_workspace(int T, int d) { return (size_t)T * d * 2 + 256; }
 
 // Vhat = Conv1D(X0) W_target: the convolution into bf16 Y (workspace), then Y W_target as one
@@ -517,9 +585,8 @@ cudaError_t inplace_target_run(int T, int d, int k, const void* X0, const float*
   Launch l;
   cudaError_t e = prepare(&l);
   if (e != cudaSuccess) return e;
-  constexpr int kRun = 32;
-  conv_future_kernel<<<dim3((d / 8 + 127) / 128, (T + kRun - 1) / kRun), 128, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(X0), conv_w, Y, T, d, k, kRun);
+  conv_future_kernel<<<dim3((d / 8 + 127) / 128, (T + kConvRun - 1) / kConvRun), 128, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(X0), conv_w, Y, T, d, k, kConvRun);
   e = cudaMemsetAsync(counter, 0, sizeof(int), s);
   if (e != cudaSuccess) return e;
   Params p{};
@@ -539,6 +606,69 @@ cudaError_t inplace_target_run(int T, int d, int k, const void* X0, const float*
   const int grid = p.n_total < l.sms ? p.n_total : l.sms;
   inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(ty, ty, ty, ty, ty, ty, twt, twt, p);
   count_launches(2);
+  return cudaGetLastError();
+}
+
+// Y (bf16), dY (bf16) and the per-run tap partial sums.
+size_t inplace_target_bwd_workspace(int T, int d, int k) {
+  const size_t nrun = (T + kConvRun - 1) / kConvRun;
+  return 2 * (size_t)T * d * 2 + nrun * k * d * 4 + 256;
+}
+
+// Backward of inplace_target_run for J = <dVhat, Vhat>: recompute Y; one launch of row tiles
+// dY = dVhat W_target^T (A = dVhat K-major, B = W_target [d rows, d cols] K-major over its
+// columns) and update tiles dW_target = Y^T dVhat (MN-major both, K = T); then the transposed
+// convolution (dX0) with the tap partials, and their reduction (dconv_w).
+cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const float* conv_w,
+                                   const void* W_target, const void* dVhat, void* dX0,
+                                   float* dconv_w, float* dW_target, void* ws, unsigned* err,
+                                   cudaStream_t s) {
+  const int nrun = (T + kConvRun - 1) / kConvRun;
+  __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* dY = Y + (size_t)T * d;
+  float* part = reinterpret_cast<float*>(dY + (size_t)T * d);
+  int* counter = reinterpret_cast<int*>(part + (size_t)nrun * k * d);
+  CUtensorMap tdv_k, tdv_n, twt_k, ty_n;
+  if (!make_tmap_bf16(&tdv_k, dVhat, d, T, d, BK, BM) ||
+      !make_tmap_bf16(&tdv_n, dVhat, d, T, d, 64, BK) ||
+      !make_tmap_bf16(&twt_k, W_target, d, d, d, BK, BN) ||
+      !make_tmap_bf16(&ty_n, Y, d, T, d, 64, BK))
+    return cudaErrorInvalidValue;
+  Launch l;
+  cudaError_t e = prepare(&l);
+  if (e != cudaSuccess) return e;
+  const dim3 cgrid((d / 8 + 127) / 128, nrun);
+  conv_future_kernel<<<cgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(X0), conv_w, Y, T,
+                                           d, k, kConvRun);
+  if ((e = cudaMemsetAsync(dW_target, 0, (size_t)d * d * sizeof(float), s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(counter, 0, sizeof(int), s)) != cudaSuccess)
+    return e;
+  Params p{};
+  p.chunk = 0;
+  p.C = T;
+  p.d_ff = d;
+  p.d_model = d;
+  p.n_row_n = (d + BN - 1) / BN;
+  p.n_upd_n = (d + BN - 1) / BN;
+  p.n_row = (T / BM) * p.n_row_n;
+  p.n_total = p.n_row + (d / BM) * p.n_upd_n;
+  p.kb_row = d / BK;
+  p.kb_upd = T / BK;
+  p.wb_next_row0 = -1;
+  p.acc_scale = 1.f;
+  p.copy_scale = 1.f;
+  p.M = dW_target;
+  p.Orow = dY;
+  p.counter = counter;
+  p.err = err;
+  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
+  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tdv_k, tdv_n, twt_k, ty_n, tdv_k, tdv_k,
+                                                          tdv_n, tdv_n, p);
+  conv_future_bwd_kernel<<<cgrid, 128, 0, s>>>(static_cast<const __nv_bfloat16*>(X0), conv_w, dY,
+                                               static_cast<__nv_bfloat16*>(dX0), part, T, d, k,
+                                               kConvRun);
+  conv_taps_reduce_kernel<<<(k * d + 255) / 256, 256, 0, s>>>(part, dconv_w, nrun, k * d);
+  count_launches(4);
   return cudaGetLastError();
 }
 

@@ -52,6 +52,11 @@ size_t inplace_target_workspace(int T, int d);
 cudaError_t inplace_target_run(int T, int d, int k, const void* X0, const float* conv_w,
                                const void* W_target, void* Vhat, void* ws, unsigned* err,
                                cudaStream_t s);
+size_t inplace_target_bwd_workspace(int T, int d, int k);
+cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const float* conv_w,
+                                   const void* W_target, const void* dVhat, void* dX0,
+                                   float* dconv_w, float* dW_target, void* ws, unsigned* err,
+                                   cudaStream_t s);
 cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
                             const void* Vhat, const void* W_chunks, const void* dO,
                             const float* dW_final, void* dZ, void* dVhat, float* dW, void* ws,
