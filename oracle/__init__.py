@@ -269,3 +269,95 @@ def inplace_target_bwd(X0, conv_w, W_target, dVhat, channels=None):
         dx[j:] += w[j] * dy[: T - j]
         dw[j] = (dy[: T - j] * x[j:]).sum(axis=0)
     return dict(dX0=dx, dconv_w=dw, dW_target=y.T @ dv)
+
+
+# --------------------------------------------------------------------------------- TTT-MLP
+def _act_t(act, z):
+    import torch
+    return z * torch.sigmoid(z) if act == "silu" else z
+
+
+def ttt_mlp_fwd(Q, K, V, beta, gamma, W1, W2, *, C: int, loss: str = "mse", act: str = "silu",
+                lr_bias: float, keep_graph: bool = False):
+    """TTT-MLP: the fast weight is a two-layer network vhat = act(k W1) W2 (page "Modular TTT:
+    Rethinking Test-Time Training as Composable Modules": TTT-MLP, the two-layer fast weight of
+    its throughput table; deeper learners factor an effective W = W1 W2), evolved per token in
+    fp64 on the CPU with plain PyTorch ops. Readings, as for the single Linear: both layers
+    decay by gamma_t and take one gradient step with eta_t = 2 sigmoid(beta_t + b); every
+    gradient of a chunk is taken at the chunk-start weights (W1_0, W2_0); the token reads its own
+    write, o_t = act(q_t W1_t) W2_t; MSE is 1/2 ||vhat - v||^2, IP is -<vhat, v>.
+    Per token t of a chunk:
+        z = k W1_0, a = act(z), vhat = a W2_0, g2 = vhat - v (MSE) or -v (IP),
+        g1 = (g2 W2_0^T) * act'(z),
+        W1 <- gamma W1 - eta k^T g1,   W2 <- gamma W2 - eta a^T g2,   o = act(q W1) W2.
+    Q, K: [B,H,T,dk]; V: [B,H,T,dv]; beta, gamma: [B,H,T] (gamma None: no decay);
+    W1: [B,H,dk,h]; W2: [B,H,h,dv]. Returns (O, W1_final, W2_final) as torch fp64 tensors
+    (with keep_graph, still attached to the autograd graph of the inputs)."""
+    import torch
+    t = lambda x: x if isinstance(x, torch.Tensor) and x.dtype == torch.float64 and x.device.type == "cpu" \
+        else torch.as_tensor(np.asarray(_np(x, np.float64)), dtype=torch.float64)
+    q, k, v, b, w1, w2 = t(Q), t(K), t(V), t(beta), t(W1), t(W2)
+    g = None if gamma is None else t(gamma)
+    B, H, T, _ = q.shape
+    if T % C:
+        raise ValueError("T must be a multiple of C")
+    outs, w1f, w2f = [], [], []
+    for bi in range(B):
+        ob, w1b, w2b = [], [], []
+        for hi in range(H):
+            A, Bw = w1[bi, hi], w2[bi, hi]
+            orows = []
+            for c in range(T // C):
+                A0, B0 = A, Bw
+                for s_ in range(C):
+                    tt = c * C + s_
+                    kt, qt, vt = k[bi, hi, tt], q[bi, hi, tt], v[bi, hi, tt]
+                    eta = 2 * torch.sigmoid(b[bi, hi, tt] + lr_bias)
+                    gam = 1.0 if g is None else g[bi, hi, tt]
+                    z = kt @ A0
+                    a = _act_t(act, z)
+                    vh = a @ B0
+                    g2 = vh - vt if loss == "mse" else -vt
+                    if act == "silu":
+                        sg = torch.sigmoid(z)
+                        d1 = sg * (1 + z * (1 - sg))
+                    else:
+                        d1 = torch.ones_like(z)
+                    g1 = (B0 @ g2) * d1
+                    A = gam * A - eta * torch.outer(kt, g1)
+                    Bw = gam * Bw - eta * torch.outer(a, g2)
+                    orows.append(_act_t(act, qt @ A) @ Bw)
+            ob.append(torch.stack(orows))
+            w1b.append(A)
+            w2b.append(Bw)
+        outs.append(torch.stack(ob))
+        w1f.append(torch.stack(w1b))
+        w2f.append(torch.stack(w2b))
+    O, W1f, W2f = torch.stack(outs), torch.stack(w1f), torch.stack(w2f)
+    if not keep_graph:
+        O, W1f, W2f = O.detach(), W1f.detach(), W2f.detach()
+    return O, W1f, W2f
+
+
+def ttt_mlp_bwd(Q, K, V, beta, gamma, W1, W2, dO, dW1_T=None, dW2_T=None, *, C: int,
+                loss: str = "mse", act: str = "silu", lr_bias: float):
+    """Gradients of J = <dO, O> + <dW1_T, W1_final> + <dW2_T, W2_final> through ttt_mlp_fwd's
+    per-token loop, by reverse-mode automatic differentiation of the fp64 CPU loop (a library
+    primitive standing in for the hand derivation). Returns numpy fp64 dQ, dK, dV, dbeta,
+    dW1 (initial W1), dW2 (initial W2), and dgamma when gamma is given."""
+    import torch
+    names = ["Q", "K", "V", "beta", "W1", "W2"] + (["gamma"] if gamma is not None else [])
+    vals = dict(Q=Q, K=K, V=V, beta=beta, W1=W1, W2=W2, gamma=gamma)
+    leaves = {n: torch.as_tensor(np.asarray(_np(vals[n], np.float64)), dtype=torch.float64).requires_grad_(True)
+              for n in names}
+    O, W1f, W2f = ttt_mlp_fwd(leaves["Q"], leaves["K"], leaves["V"], leaves["beta"],
+                              leaves.get("gamma"), leaves["W1"], leaves["W2"], C=C, loss=loss,
+                              act=act, lr_bias=lr_bias, keep_graph=True)
+    J = (O * torch.as_tensor(_np(dO, np.float64))).sum()
+    if dW1_T is not None:
+        J = J + (W1f * torch.as_tensor(_np(dW1_T, np.float64))).sum()
+    if dW2_T is not None:
+        J = J + (W2f * torch.as_tensor(_np(dW2_T, np.float64))).sum()
+    grads = torch.autograd.grad(J, [leaves[n] for n in names])
+    key = dict(Q="dQ", K="dK", V="dV", beta="dbeta", W1="dW1", W2="dW2", gamma="dgamma")
+    return {key[n]: gr.numpy() for n, gr in zip(names, grads)}

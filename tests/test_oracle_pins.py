@@ -13,6 +13,8 @@
 * streaming and column independence;
 * hand-worked golden values (tests/golden/scalar_chunk_worked.txt);
 * central finite differences for every backward output;
+* TTT-MLP (two-layer fast weight): its own brute-force chunk dual form, the
+  decay-only case without learning, and finite differences of its backward;
 * per-feature (vector) decay: its own brute-force dual form, the scalar decay
   when all features share one factor, a zero factor clearing exactly one row
   of W, and finite differences including the per-feature decay gradient;
@@ -593,3 +595,110 @@ def test_inplace_target_backward_channel_subset_is_exact():
     np.testing.assert_allclose(gs["dX0"], g["dX0"][:, ch], atol=1e-13)
     np.testing.assert_allclose(gs["dconv_w"], g["dconv_w"][:, ch], atol=1e-13)
     np.testing.assert_allclose(gs["dW_target"], g["dW_target"][ch], atol=1e-13)
+
+
+# ------------------------------------------------------------------------------- TTT-MLP
+
+
+def _mlp_rand(rng, B, H, T, dk, dv, hd, decay=True):
+    Q, K, V, beta, gamma, _ = rand_inputs(rng, B, H, T, dk, dv, decay=decay)
+    W1 = 0.4 * rng.standard_normal((B, H, dk, hd))
+    W2 = 0.4 * rng.standard_normal((B, H, hd, dv))
+    return Q, K, V, beta, gamma, W1, W2
+
+
+def mlp_dual_form(Q, K, V, beta, gamma, W1, W2, C, loss, act, b):
+    """Chunk dual form of the two-layer learner, by brute force: with A1 = act(K W1_0),
+    G2 = dl/dvhat, G1 = (G2 W2_0^T) * act'(K W1_0) and w_sr = eta_r exp(L_s - L_r), r <= s,
+        Zq1_s = Gamma_s q_s W1_0 - sum_r w_sr (q_s . k_r) G1_r,   Aq_s = act(Zq1_s),
+        o_s   = Gamma_s Aq_s W2_0 - sum_r w_sr (Aq_s . A1_r) G2_r,
+        W1_end = Gamma_C W1_0 - K^T diag(u) G1,  W2_end = Gamma_C W2_0 - A1^T diag(u) G2."""
+    B, H, T, dk = Q.shape
+    dv = V.shape[-1]
+    O = np.zeros((B, H, T, dv))
+    W1F, W2F = np.zeros_like(W1), np.zeros_like(W2)
+    for bi in range(B):
+        for hi in range(H):
+            A, Bw = W1[bi, hi].copy(), W2[bi, hi].copy()
+            for c in range(T // C):
+                sl = slice(c * C, (c + 1) * C)
+                q, k, v = Q[bi, hi, sl], K[bi, hi, sl], V[bi, hi, sl]
+                eta = 2 * sigmoid(beta[bi, hi, sl] + b)
+                L = np.cumsum(np.log(gamma[bi, hi, sl])) if gamma is not None else np.zeros(C)
+                Z1 = k @ A
+                A1 = act_np(act, Z1)
+                G2 = A1 @ Bw - v if loss == "mse" else -v
+                G1 = (G2 @ Bw.T) * dact_np(act, Z1)
+                for s_ in range(C):
+                    zq = math.exp(L[s_]) * (q[s_] @ A)
+                    for r in range(s_ + 1):
+                        zq = zq - eta[r] * math.exp(L[s_] - L[r]) * float(q[s_] @ k[r]) * G1[r]
+                    aq = act_np(act, zq)
+                    o = math.exp(L[s_]) * (aq @ Bw)
+                    for r in range(s_ + 1):
+                        o = o - eta[r] * math.exp(L[s_] - L[r]) * float(aq @ A1[r]) * G2[r]
+                    O[bi, hi, c * C + s_] = o
+                u = eta * np.exp(L[-1] - L)
+                A = math.exp(L[-1]) * A - k.T @ (u[:, None] * G1)
+                Bw = math.exp(L[-1]) * Bw - A1.T @ (u[:, None] * G2)
+            W1F[bi, hi], W2F[bi, hi] = A, Bw
+    return O, W1F, W2F
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+@pytest.mark.parametrize("C", [1, 2, 4])
+def test_ttt_mlp_matches_its_dual_form(loss, act, C):
+    rng = np.random.default_rng(500 + C)
+    Q, K, V, beta, gamma, W1, W2 = _mlp_rand(rng, 1, 2, 8, 3, 2, 5)
+    b = -0.6
+    O, W1F, W2F = oracle.ttt_mlp_fwd(Q, K, V, beta, gamma, W1, W2, C=C, loss=loss, act=act,
+                                     lr_bias=b)
+    O2, W1F2, W2F2 = mlp_dual_form(Q, K, V, beta, gamma, W1, W2, C, loss, act, b)
+    np.testing.assert_allclose(O.numpy(), O2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(W1F.numpy(), W1F2, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(W2F.numpy(), W2F2, rtol=0, atol=1e-12)
+
+
+def test_ttt_mlp_without_learning_only_decays():
+    # eta = 2 sigmoid(beta + b) -> 0: both layers only decay, o_t = act(c_t q_t W1) c_t W2 with
+    # c_t the product of every gamma up to t
+    rng = np.random.default_rng(510)
+    Q, K, V, beta, gamma, W1, W2 = _mlp_rand(rng, 1, 1, 8, 3, 2, 4)
+    O, W1F, W2F = oracle.ttt_mlp_fwd(Q, K, V, beta, gamma, W1, W2, C=4, loss="mse", act="silu",
+                                     lr_bias=-80.0)
+    cum = np.cumprod(gamma[0, 0])
+    for t in range(8):
+        want = act_np("silu", cum[t] * (Q[0, 0, t] @ W1[0, 0])) @ (cum[t] * W2[0, 0])
+        np.testing.assert_allclose(O[0, 0, t].numpy(), want, atol=1e-12)
+    np.testing.assert_allclose(W2F[0, 0].numpy(), cum[-1] * W2[0, 0], atol=1e-12)
+
+
+@pytest.mark.parametrize("loss,act", COMBOS)
+def test_ttt_mlp_backward_matches_finite_differences(loss, act):
+    rng = np.random.default_rng(520 + 2 * list(dict.fromkeys(COMBOS)).index((loss, act)))
+    B, H, T, dk, dv, hd, C = 1, 1, 6, 2, 2, 3, 3
+    Q, K, V, beta, gamma, W1, W2 = _mlp_rand(rng, B, H, T, dk, dv, hd)
+    dO = rng.standard_normal((B, H, T, dv))
+    dW1 = rng.standard_normal(W1.shape)
+    dW2 = rng.standard_normal(W2.shape)
+    kw = dict(C=C, loss=loss, act=act, lr_bias=-0.3)
+    g = oracle.ttt_mlp_bwd(Q, K, V, beta, gamma, W1, W2, dO, dW1, dW2, **kw)
+
+    def J():
+        O, A, Bw = oracle.ttt_mlp_fwd(Q, K, V, beta, gamma, W1, W2, **kw)
+        return float((O.numpy() * dO).sum() + (A.numpy() * dW1).sum() + (Bw.numpy() * dW2).sum())
+
+    h = 1e-6
+    for name, x, key in (("Q", Q, "dQ"), ("K", K, "dK"), ("V", V, "dV"), ("beta", beta, "dbeta"),
+                         ("gamma", gamma, "dgamma"), ("W1", W1, "dW1"), ("W2", W2, "dW2")):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            jp = J()
+            x[idx] = old - h
+            jm = J()
+            x[idx] = old
+            fd[idx] = (jp - jm) / (2 * h)
+        err = np.abs(g[key] - fd).max() / np.abs(fd).max()
+        assert err < 1e-7, (name, err)
