@@ -259,7 +259,46 @@ def time_other_configs(ttt, peaks):
         res[name] = entry
         del layer
         torch.cuda.empty_cache()
+    res[synth.TTT_MLP_410M.name] = time_mlp(ttt, peaks)
     return res
+
+
+def time_mlp(ttt, peaks):
+    """TTT-MLP (two-layer fast weight, SIMT kernels) forward and backward on the 410M layer
+    shape with hidden width 4 d: device ms, tokens/s and the fraction of the fp32 CUDA-core
+    peak. flops per chunk and head: the readout and training GEMMs of both layers (causal halves
+    of the C x C products), 2 C (3 dk h + 3 h dv) + C (C+1) (dk + dv + 2 h) forward and twice
+    that backward; recomputation not counted."""
+    cfg, hid = synth.TTT_MLP_410M, synth.TTT_MLP_HIDDEN
+    inp = synth.ttt_inputs(cfg, device="cuda")
+    w = synth.ttt_mlp_weights(cfg, hid, device="cuda")
+    c = ttt.make_config(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C, cfg.dtype, cfg.loss, cfg.act,
+                        cfg.lr_bias)
+    B, H, T, dk, dv, C = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C
+    O = torch.empty((B, H, T, dv), device="cuda", dtype=torch.bfloat16)
+    W1f, W2f = torch.empty_like(w["W1"]), torch.empty_like(w["W2"])
+    W1c = torch.empty((B, H, T // C, dk, hid), device="cuda")
+    W2c = torch.empty((B, H, T // C, hid, dv), device="cuda")
+    n = ttt.ttt_mlp_workspace_bytes(c, hid)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    g = [torch.empty_like(inp["Q"]), torch.empty_like(inp["K"]), torch.empty_like(inp["V"]),
+         torch.empty_like(inp["beta"]), torch.empty_like(w["W1"]), torch.empty_like(w["W2"])]
+    fwd = lambda: ttt.ttt_mlp_fwd(c, hid, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"],
+                                  w["W1"], w["W2"], O, W1f, W2f, W1c, W2c, ws, n)
+    bwd = lambda: ttt.ttt_mlp_bwd(c, hid, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"],
+                                  W1c, W2c, inp["dO"], None, None, *g, ws, n)
+    ms_f = _event_ms(fwd, 2, 1)
+    ms_b = _event_ms(bwd, 2, 1)
+    units = B * H * (T // C)
+    fl_f = units * (2 * C * (3 * dk * hid + 3 * hid * dv) + C * (C + 1) * (dk + dv + 2 * hid))
+    out = {"dtype": cfg.dtype, "hidden": hid, "decay": "scalar",
+           "ttt_mlp_fwd": {"ms": ms_f, "path": "simt", "alu_frac": fl_f / (ms_f * 1e-3) / FP32_ALU_PEAK},
+           "ttt_mlp_bwd": {"ms": ms_b, "path": "simt",
+                           "alu_frac": 2 * fl_f / (ms_b * 1e-3) / FP32_ALU_PEAK},
+           "ms": ms_f + ms_b, "tokens_per_s": B * T / ((ms_f + ms_b) * 1e-3)}
+    del ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def time_bwd_dgamma(layer, steps=5, warmup=2):

@@ -162,6 +162,34 @@ ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q, const voi
                                  void* dQ, void* dK, void* dV, float* dbeta, float* dW0,
                                  float* dgamma, void* stream);
 
+/* TTT-MLP: the fast weight is the two-layer network vhat = act(k W1) W2 (page "Modular TTT:
+ * Rethinking Test-Time Training as Composable Modules", TTT-MLP; cfg->act is the hidden
+ * activation, the output layer is linear). Per token t of a chunk, gradients at the chunk-start
+ * weights W1_0, W2_0:
+ *     z = k W1_0, a = act(z), g2 = a W2_0 - v (MSE) or -v (IP), g1 = (g2 W2_0^T) * act'(z)
+ *     W1_t = gamma_t W1_{t-1} - eta_t k^T g1,  W2_t = gamma_t W2_{t-1} - eta_t a^T g2
+ *     o_t  = act(q_t W1_t) W2_t
+ * evaluated in the chunk dual form on the SIMT kernels (float32 arithmetic).
+ * Layouts: Q, K, dQ, dK [B,H,T,dk] and V, O, dO, dV [B,H,T,dv] in cfg->dtype; beta, gamma, dbeta
+ * [B,H,T] float32 (gamma nullable; scalar decay only); W1 [B,H,dk,hidden], W2 [B,H,hidden,dv]
+ * float32, likewise W1_final, W2_final, dW1_final, dW2_final, dW1_0, dW2_0; W1_chunks
+ * [B,H,T/C,dk,hidden] and W2_chunks [B,H,T/C,hidden,dv] float32 (chunk-start weights, written by
+ * the forward when non-NULL, required by the backward). dk, dv <= 128, hidden <= 512, C <= 256. */
+size_t ttt_mlp_workspace_bytes(const ttt_config* cfg, int hidden);
+ttt_status ttt_mlp_fwd(const ttt_config* cfg, int hidden, const void* Q, const void* K,
+                       const void* V, const float* beta, const float* gamma, const float* W1_0,
+                       const float* W2_0, void* O, float* W1_final, float* W2_final,
+                       float* W1_chunks, float* W2_chunks, void* workspace,
+                       size_t workspace_bytes, void* stream);
+/* Backward for J = <dO, O> + <dW1_final, W1_final> + <dW2_final, W2_final> (dW*_final nullable
+ * = 0): dQ, dK, dV, dbeta and the gradients of the initial weights dW1_0, dW2_0. */
+ttt_status ttt_mlp_bwd(const ttt_config* cfg, int hidden, const void* Q, const void* K,
+                       const void* V, const float* beta, const float* gamma,
+                       const float* W1_chunks, const float* W2_chunks, const void* dO,
+                       const float* dW1_final, const float* dW2_final, void* dQ, void* dK,
+                       void* dV, float* dbeta, float* dW1_0, float* dW2_0, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
 /* Workspace bytes of inplace_ttt_fwd and of inplace_ttt_bwd (the same figure);
  * (size_t)-1 for invalid sizes. */
 size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C);

@@ -185,3 +185,25 @@ def inplace_target_inputs(cfg: InPlaceConfig, k: int = 4, device="cpu", seed: in
     dv = _randn((cfg.T, d), g, device).to(torch.bfloat16)
     return dict(X0=x0.contiguous(), conv_w=w.contiguous(), W_target=wt.contiguous(),
                 dVhat=dv.contiguous())
+
+
+# TTT-MLP workload: the 410M layer shape with a two-layer fast weight of hidden width 4 d,
+# SiLU between the layers, both layers initialised with std 0.02 (section "复现评估").
+TTT_MLP_410M = TTTConfig("410m-ttt-mlp-fwd-bwd", B=8, H=16, T=2048, dk=64, dv=64, C=256,
+                         dtype="bf16", loss="mse", act="silu", decay=True, w0_std=0.02,
+                         normalize="qk", backward=True, seed=6)
+TTT_MLP_HIDDEN = 256
+
+
+def ttt_mlp_weights(cfg: TTTConfig, hidden: int, device="cpu", seed: int | None = None) -> dict:
+    """Initial weights of the two-layer fast weight: W1 [B,H,dk,hidden] and W2 [B,H,hidden,dv]
+    ~ N(0, cfg.w0_std) float32, and upstream gradients of the final weights dW1_T, dW2_T
+    (zeros). Seeded apart from ttt_inputs (seed + 2000)."""
+    seed = (cfg.seed if seed is None else seed) + 2000
+    g = make_generator(seed, device)
+    B, H = cfg.B, cfg.H
+    w1 = cfg.w0_std * _randn((B, H, cfg.dk, hidden), g, device)
+    w2 = cfg.w0_std * _randn((B, H, hidden, cfg.dv), g, device)
+    z1 = torch.zeros_like(w1)
+    z2 = torch.zeros_like(w2)
+    return dict(W1=w1.contiguous(), W2=w2.contiguous(), dW1_T=z1, dW2_T=z2)

@@ -9,7 +9,8 @@ import weight_sequence_layers_b200 as ttt
 
 FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_ttt_workspace_bytes",
              "inplace_ttt_fwd", "inplace_ttt_bwd", "inplace_ttt_target", "inplace_ttt_target_workspace_bytes",
-             "inplace_ttt_target_bwd", "inplace_ttt_target_bwd_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "inplace_ttt_target_bwd", "inplace_ttt_target_bwd_workspace_bytes",
+             "ttt_mlp_fwd", "ttt_mlp_bwd", "ttt_mlp_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
              "ttt_status_string"}
 
 
@@ -213,3 +214,29 @@ def test_inplace_target_bwd_argument_errors():
     assert f(256, 128, 4, *args) == ttt.ERR_WORKSPACE
     with pytest.raises(ttt.TTTError):
         ttt.inplace_ttt_target_bwd_workspace_bytes(256, 128, 0)
+
+
+def test_ttt_mlp_argument_errors():
+    cfg = _cfg()
+    A = 4096
+    need = ttt.ttt_mlp_workspace_bytes(cfg, 96)
+    assert need > 0
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_mlp_workspace_bytes(cfg, 600)                     # hidden > 512
+    vec = _cfg(decay="vector")
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_mlp_workspace_bytes(vec, 96)                      # scalar decay only
+    f = ttt.lib.ttt_mlp_fwd
+    # cfg hidden Q K V beta gamma W1_0 W2_0 O W1_final W2_final W1_chunks W2_chunks ws bytes stream
+    ok = [A, A, A, A, None, A, A, A, None, None, None, None, A, need, None]
+    assert f(ctypes.byref(cfg), 0, *ok) == ttt.ERR_UNSUPPORTED
+    args = list(ok)
+    args[5] = None  # W1_0
+    assert f(ctypes.byref(cfg), 96, *args) == ttt.ERR_INVALID_ARG
+    args = list(ok)
+    args[13] = need - 1
+    assert f(ctypes.byref(cfg), 96, *args) == ttt.ERR_WORKSPACE
+    b = ttt.lib.ttt_mlp_bwd
+    # cfg hidden Q K V beta gamma W1c W2c dO dW1f dW2f dQ dK dV dbeta dW1 dW2 ws bytes stream
+    okb = [A, A, A, A, None, None, A, A, None, None, A, A, A, A, A, A, A, need, None]
+    assert b(ctypes.byref(cfg), 96, *okb) == ttt.ERR_INVALID_ARG  # W1_chunks is required

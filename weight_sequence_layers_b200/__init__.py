@@ -48,6 +48,9 @@ _SIGS = {
     "ttt_chunk_fwd": ([_cfgp] + [_p] * 11 + [_sz, _p], _i),
     "ttt_chunk_bwd": ([_cfgp] + [_p] * 19 + [_sz, _p], _i),
     "inplace_ttt_workspace_bytes": ([_i] * 4, _sz),
+    "ttt_mlp_workspace_bytes": ([_cfgp, _i], _sz),
+    "ttt_mlp_fwd": ([_cfgp, _i] + [_p] * 13 + [_sz, _p], _i),
+    "ttt_mlp_bwd": ([_cfgp, _i] + [_p] * 17 + [_sz, _p], _i),
     "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 6 + [_sz, _p], _i),
     "inplace_ttt_bwd": ([_i] * 4 + [_f] + [_p] * 9 + [_sz, _p], _i),
     "inplace_ttt_target_workspace_bytes": ([_i] * 2, _sz),
@@ -144,6 +147,31 @@ def ttt_chunk_bwd_noalloc(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, 
                                     _ptr(dK), _ptr(dV), _ptr(dbeta), _ptr(dW0), _ptr(dgamma),
                                     _stream(stream))
     _check(st, "ttt_chunk_bwd_noalloc")
+
+
+def ttt_mlp_workspace_bytes(cfg: ttt_config, hidden: int) -> int:
+    n = _lib.ttt_mlp_workspace_bytes(ctypes.byref(cfg), int(hidden))
+    if n == ctypes.c_size_t(-1).value:
+        raise TTTError(ERR_INVALID_ARG, "ttt_mlp_workspace_bytes")
+    return n
+
+
+def ttt_mlp_fwd(cfg, hidden, Q, K, V, beta, gamma, W1_0, W2_0, O, W1_final, W2_final, W1_chunks,
+                W2_chunks, workspace, workspace_bytes, stream=None):
+    st = _lib.ttt_mlp_fwd(ctypes.byref(cfg), int(hidden), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
+                          _ptr(gamma), _ptr(W1_0), _ptr(W2_0), _ptr(O), _ptr(W1_final),
+                          _ptr(W2_final), _ptr(W1_chunks), _ptr(W2_chunks), _ptr(workspace),
+                          int(workspace_bytes), _stream(stream))
+    _check(st, "ttt_mlp_fwd")
+
+
+def ttt_mlp_bwd(cfg, hidden, Q, K, V, beta, gamma, W1_chunks, W2_chunks, dO, dW1_final, dW2_final,
+                dQ, dK, dV, dbeta, dW1_0, dW2_0, workspace, workspace_bytes, stream=None):
+    st = _lib.ttt_mlp_bwd(ctypes.byref(cfg), int(hidden), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
+                          _ptr(gamma), _ptr(W1_chunks), _ptr(W2_chunks), _ptr(dO), _ptr(dW1_final),
+                          _ptr(dW2_final), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta), _ptr(dW1_0),
+                          _ptr(dW2_0), _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "ttt_mlp_bwd")
 
 
 def inplace_ttt_workspace_bytes(T, d_ff, d_model, C) -> int:

@@ -249,6 +249,57 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
   return launch_status(path == PATH_TC ? tc_bwd(a, s) : simt_bwd(a, s));
 }
 
+size_t ttt_mlp_workspace_bytes(const ttt_config* cfg, int hidden) {
+  if (check_config(cfg) != TTT_OK) return (size_t)-1;
+  const LayerArgs a = args_of(cfg);
+  if (!mlp_supported(a, hidden)) return (size_t)-1;
+  return mlp_workspace(a, hidden);
+}
+
+ttt_status ttt_mlp_fwd(const ttt_config* cfg, int hidden, const void* Q, const void* K,
+                       const void* V, const float* beta, const float* gamma, const float* W1_0,
+                       const float* W2_0, void* O, float* W1_final, float* W2_final,
+                       float* W1_chunks, float* W2_chunks, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  const ttt_status st = check_config(cfg);
+  if (st != TTT_OK) return st;
+  LayerArgs a = args_of(cfg);
+  if (!mlp_supported(a, hidden)) return TTT_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !beta || !W1_0 || !W2_0 || !O) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, beta, gamma, W1_0, W2_0, O, W1_final, W2_final, W1_chunks,
+                        W2_chunks, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < mlp_workspace(a, hidden)) return TTT_ERR_WORKSPACE;
+  a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.O = O; a.ws = workspace;
+  return launch_status(mlp_fwd(a, hidden, W1_0, W2_0, W1_final, W2_final, W1_chunks, W2_chunks,
+                               static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status ttt_mlp_bwd(const ttt_config* cfg, int hidden, const void* Q, const void* K,
+                       const void* V, const float* beta, const float* gamma,
+                       const float* W1_chunks, const float* W2_chunks, const void* dO,
+                       const float* dW1_final, const float* dW2_final, void* dQ, void* dK,
+                       void* dV, float* dbeta, float* dW1_0, float* dW2_0, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  const ttt_status st = check_config(cfg);
+  if (st != TTT_OK) return st;
+  LayerArgs a = args_of(cfg);
+  if (!mlp_supported(a, hidden)) return TTT_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !beta || !W1_chunks || !W2_chunks || !dO || !dQ || !dK || !dV || !dbeta ||
+      !dW1_0 || !dW2_0)
+    return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, beta, gamma, W1_chunks, W2_chunks, dO, dW1_final, dW2_final,
+                        dQ, dK, dV, dbeta, dW1_0, dW2_0, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < mlp_workspace(a, hidden)) return TTT_ERR_WORKSPACE;
+  a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.dO = dO; a.dQ = dQ; a.dK = dK;
+  a.dV = dV; a.dbeta = dbeta; a.ws = workspace;
+  return launch_status(mlp_bwd(a, hidden, W1_chunks, W2_chunks, dW1_final, dW2_final, dW1_0,
+                               dW2_0, static_cast<cudaStream_t>(stream)));
+}
+
 size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C) {
   if (T < 1 || d_ff < 1 || d_model < 1 || C < 1 || T % C || C % 128 || d_ff % 64 ||
       d_model % 128)

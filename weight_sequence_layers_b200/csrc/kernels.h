@@ -43,6 +43,15 @@ bool tc_bwd_supported(const LayerArgs& a);
 size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved, bool dgamma);
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
 
+// TTT-MLP (SIMT).
+bool mlp_supported(const LayerArgs& a, int hidden);
+size_t mlp_workspace(const LayerArgs& a, int hidden);
+cudaError_t mlp_fwd(const LayerArgs& a, int hidden, const float* W1_0, const float* W2_0,
+                    float* W1f, float* W2f, float* W1c, float* W2c, cudaStream_t s);
+cudaError_t mlp_bwd(const LayerArgs& a, int hidden, const float* W1c, const float* W2c,
+                    const float* dW1f, const float* dW2f, float* dW1_0, float* dW2_0,
+                    cudaStream_t s);
+
 // In-Place TTT.
 size_t inplace_workspace(int T, int d_ff, int d_model, int C);
 cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
