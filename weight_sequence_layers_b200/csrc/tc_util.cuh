@@ -9,8 +9,9 @@
 namespace tttk {
 namespace {
 
-// Sigmoid with the hardware exponential and reciprocal (bf16-level accuracy is enough here).
-__device__ __forceinline__ float sigm(float x) { return __frcp_rn(1.f + __expf(-x)); }
+// Sigmoid with the hardware exponential and the fast approximate division (bf16-level
+// accuracy is enough here; 1 + exp(-x) above 2^126 gives 0, the right limit).
+__device__ __forceinline__ float sigm(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 
 // Activation of the fast-weight network (ACT = 0 identity, 1 SiLU) and its derivative; a
 // compile-time choice so the identity path carries no transcendental at all.
@@ -26,6 +27,18 @@ __device__ __forceinline__ float act_d1(float z) {
     return s * (1.f + z * (1.f - s));
   }
   return 1.f;
+}
+// act(z) and act'(z) from one sigmoid.
+template <int ACT>
+__device__ __forceinline__ void act_both(float z, float& f, float& d1) {
+  if constexpr (ACT == 1) {
+    const float s = sigm(z);
+    f = z * s;
+    d1 = s * (1.f + z * (1.f - s));
+  } else {
+    f = z;
+    d1 = 1.f;
+  }
 }
 
 // Reads 32 bf16 (16-byte chunks c0..c0+3 of `row`) of a swizzled panel as floats.

@@ -577,7 +577,7 @@ __global__ void __launch_bounds__(kSmallThreads, 2)
           float f1[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const float sg = 1.f / (1.f + __expf(-z[j]));
+            const float sg = __fdividef(1.f, 1.f + __expf(-z[j]));
             const float d1 = sg * (1.f + z[j] * (1.f - sg));
             const float d2 = sg * (1.f - sg) * (2.f + z[j] * (1.f - 2.f * sg));
             const float a = mse ? z[j] * sg - v[j] : -v[j];
@@ -1166,7 +1166,7 @@ __global__ void __launch_bounds__(256)
       float zz[2] = {bf16lo(wz[h]), bf16hi(wz[h])}, d[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float sg = 1.f / (1.f + __expf(-zz[e]));
+        const float sg = __fdividef(1.f, 1.f + __expf(-zz[e]));
         d[e] = sg * (1.f + zz[e] * (1.f - sg));
       }
       o[h] = pack_bf16x2(bf16lo(wa[h]) * d[0], bf16hi(wa[h]) * d[1]);

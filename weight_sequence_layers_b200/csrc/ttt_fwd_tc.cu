@@ -398,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       tc_fence_after();
       {
-        // identity: both Z blocks in flight at once; SiLU needs the registers for its temporaries
-        constexpr int ZB = ACT == 0 ? NB : 1;
+        // both Z blocks in flight at once
+        constexpr int ZB = NB;
         float z[ZB][32];
 #pragma unroll
         for (int b0 = 0; b0 < NB; b0 += ZB) {
@@ -415,8 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float un = -f_eta[row] * f_eLC[row];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float a = LOSS == 0 ? act_f<ACT>(z[i][j]) - v[j] : -v[j];
-              const float gg = a * act_d1<ACT>(z[i][j]);
+              float fz, d1;
+              act_both<ACT>(z[i][j], fz, d1);
+              const float a = LOSS == 0 ? fz - v[j] : -v[j];
+              const float gg = a * d1;
               v[j] = gg;
               z[i][j] = un * gg;
             }
