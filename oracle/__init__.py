@@ -139,14 +139,17 @@ def ttt_bwd(Q, K, V, beta, gamma, W0, dO, dW_T=None, *, C: int, loss: str = "mse
     return out
 
 
-def inplace_fwd(Z, Vhat, W, *, C: int, lr: float, rows=None):
+def inplace_fwd(Z, Vhat, W, *, C: int, lr: float, rows=None, doc_starts=()):
     """In-Place TTT W_down forward, apply-then-update per chunk (fp64).
 
     Z: [T, d_ff]; Vhat: [T, d_model]; W: [d_model, d_ff] (the fast weight W_down).
     For chunk i: O_i = Z_i W_i^T, then W_{i+1} = W_i + lr * Vhat_i^T Z_i.
     `rows` (optional index array into d_model) restricts the computation to
     those rows of W (and columns of O and Vhat): the rows evolve independently,
-    so the restricted result is exact. Returns (O[:, rows], W_final[rows]).
+    so the restricted result is exact. `doc_starts`: chunk indices where a new
+    document begins (section "实践建议": the fast weight is reset at document
+    boundaries); its first chunk applies the initial W again. Returns
+    (O[:, rows], W_final[rows]).
     """
     z = _np(Z, np.float64)
     vh = _np(Vhat, np.float64)
@@ -155,19 +158,23 @@ def inplace_fwd(Z, Vhat, W, *, C: int, lr: float, rows=None):
         rows = np.asarray(rows)
         vh = vh[:, rows]
         w = w[rows]
+    w0 = w.copy()
     w = w.copy()
     T = z.shape[0]
     if T % C:
         raise ValueError("T must be a multiple of C")
     o = np.empty((T, w.shape[0]))
+    starts = set(doc_starts)
     for i in range(T // C):
+        if i in starts:
+            w = w0.copy()  # a new document starts from the initial fast weight
         zi = z[i * C:(i + 1) * C]
         o[i * C:(i + 1) * C] = zi @ w.T          # apply with the current fast weight
         w += lr * (vh[i * C:(i + 1) * C].T @ zi)  # then update it with this chunk
     return o, w
 
 
-def inplace_bwd(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, rows=None):
+def inplace_bwd(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, rows=None, doc_starts=()):
     """Reverse-mode of inplace_fwd for J = sum_i <dO_i, O_i> + <dW_final, W_final> (fp64).
 
     The chunks are walked backwards carrying Wh, the adjoint of the fast weight (dW_final, or
@@ -176,6 +183,8 @@ def inplace_bwd(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, rows=None):
         W_{i+1} = W_i + lr Vhat_i^T Z_i  gives  dZ_i += lr Vhat_i Wh_{i+1},  dVhat_i = lr Z_i Wh_{i+1}^T
     (Wh_{i+1} is the adjoint before chunk i's own O_i term is added). Returns dict dZ [T, d_ff],
     dVhat [T, d_model] and dW [d_model, d_ff], the gradient with respect to the initial W.
+    With `doc_starts` (see inplace_fwd) a document's first chunk applied the initial W, so the
+    adjoint reaching it joins dW and the previous document's end state gets no adjoint.
     `rows` restricts the computation to those rows of W (columns of Vhat and dO): dVhat[:, rows]
     and dW[rows] are then exact, and dZ, a sum over every row, is not returned (None).
     """
@@ -190,13 +199,17 @@ def inplace_bwd(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, rows=None):
     T = z.shape[0]
     if T % C:
         raise ValueError("T must be a multiple of C")
+    starts = set(doc_starts)
     applied = []
     cur = w.copy()
     for i in range(T // C):
         sl = slice(i * C, (i + 1) * C)
+        if i in starts:
+            cur = w.copy()
         applied.append(cur.copy())
         cur = cur + lr * (vh[sl].T @ z[sl])
     wh = dwf.copy()
+    dw = np.zeros_like(w)
     dz = np.zeros_like(z) if rows is None else None
     dvh = np.zeros_like(vh)
     for i in reversed(range(T // C)):
@@ -205,7 +218,10 @@ def inplace_bwd(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, rows=None):
             dz[sl] = do[sl] @ applied[i] + lr * (vh[sl] @ wh)
         dvh[sl] = lr * (z[sl] @ wh.T)
         wh = wh + do[sl].T @ z[sl]
-    return dict(dZ=dz, dVhat=dvh, dW=wh)
+        if i in starts or i == 0:
+            dw = dw + wh              # this document's start state is the initial W
+            wh = np.zeros_like(wh)    # the previous document's end state is discarded
+    return dict(dZ=dz, dVhat=dvh, dW=dw)
 
 
 def inplace_bwd_dz_tokens(Z, Vhat, W, dO, dW_final=None, *, C: int, lr: float, tokens):

@@ -22,7 +22,8 @@
   associativity of the update, plain GEMM when C = T or eta = 0, and the
   dual form with Z_i Z_j^T corrections; its backward against finite
   differences, the single-chunk closed form, and the row-subset and
-  sampled-token evaluations against the full one; the NTP-aligned target
+  sampled-token evaluations against the full one; document resets against
+  independent per-document calls and finite differences; the NTP-aligned target
   against shifted copies (one-hot taps) and a plain matmul (one tap), and
   its backward against finite differences.
 """
@@ -702,3 +703,57 @@ def test_ttt_mlp_backward_matches_finite_differences(loss, act):
             fd[idx] = (jp - jm) / (2 * h)
         err = np.abs(g[key] - fd).max() / np.abs(fd).max()
         assert err < 1e-7, (name, err)
+
+
+def test_inplace_document_resets():
+    rng = np.random.default_rng(50)
+    T, d_ff, d_model, C, lr = 24, 7, 5, 4, 0.05
+    Z, Vh, W = _inplace_rand(rng, T, d_ff, d_model)
+    # a reset at every chunk: each chunk applies the initial W; the final state holds the last
+    # chunk's update only
+    every = list(range(1, T // C))
+    O, WF = oracle.inplace_fwd(Z, Vh, W, C=C, lr=lr, doc_starts=every)
+    np.testing.assert_allclose(O, Z @ W.T, atol=1e-12)
+    np.testing.assert_allclose(WF, W + lr * Vh[-C:].T @ Z[-C:], atol=1e-12)
+    # a reset at chunk 3 == two independent calls, one per document
+    O2, WF2 = oracle.inplace_fwd(Z, Vh, W, C=C, lr=lr, doc_starts=[3])
+    Oa, _ = oracle.inplace_fwd(Z[:12], Vh[:12], W, C=C, lr=lr)
+    Ob, WFb = oracle.inplace_fwd(Z[12:], Vh[12:], W, C=C, lr=lr)
+    np.testing.assert_allclose(O2, np.concatenate([Oa, Ob]), atol=1e-12)
+    np.testing.assert_allclose(WF2, WFb, atol=1e-12)
+    # and the gradients: the initial W gets both documents' adjoints, each part its own
+    dO = rng.standard_normal((T, d_model))
+    dWf = rng.standard_normal((d_model, d_ff))
+    g = oracle.inplace_bwd(Z, Vh, W, dO, dWf, C=C, lr=lr, doc_starts=[3])
+    ga = oracle.inplace_bwd(Z[:12], Vh[:12], W, dO[:12], None, C=C, lr=lr)
+    gb = oracle.inplace_bwd(Z[12:], Vh[12:], W, dO[12:], dWf, C=C, lr=lr)
+    np.testing.assert_allclose(g["dZ"], np.concatenate([ga["dZ"], gb["dZ"]]), atol=1e-12)
+    np.testing.assert_allclose(g["dVhat"], np.concatenate([ga["dVhat"], gb["dVhat"]]), atol=1e-12)
+    np.testing.assert_allclose(g["dW"], ga["dW"] + gb["dW"], atol=1e-12)
+
+
+def test_inplace_backward_with_resets_matches_finite_differences():
+    rng = np.random.default_rng(51)
+    T, d_ff, d_model, C, lr = 8, 4, 3, 2, 0.3
+    Z, Vh, W = _inplace_rand(rng, T, d_ff, d_model)
+    dO = rng.standard_normal((T, d_model))
+    dWf = rng.standard_normal((d_model, d_ff))
+    starts = [2]
+    g = oracle.inplace_bwd(Z, Vh, W, dO, dWf, C=C, lr=lr, doc_starts=starts)
+
+    def J():
+        O, WF = oracle.inplace_fwd(Z, Vh, W, C=C, lr=lr, doc_starts=starts)
+        return float((O * dO).sum() + (WF * dWf).sum())
+
+    h = 1e-6
+    for x, key in ((Z, "dZ"), (Vh, "dVhat"), (W, "dW")):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            jp = J()
+            x[idx] = old - h
+            jm = J()
+            x[idx] = old
+            fd[idx] = (jp - jm) / (2 * h)
+        assert np.abs(g[key] - fd).max() / np.abs(fd).max() < 1e-8, key

@@ -100,3 +100,17 @@ def test_mlp_full_size_sampled_head():
         assert rel_err(f[k][b:b + 1, h:h + 1], rf[k]) <= BF16_TOL, k
     for k in ("dQ", "dK", "dV", "dbeta", "dW1", "dW2"):
         assert rel_err(g[k][b:b + 1, h:h + 1], rg[k]) <= BF16_TOL, k
+
+
+def test_mlp_single_chunk_fp32():
+    cfg = synth.TTT_MLP_410M.replace(B=1, H=1, T=32, dk=8, dv=8, C=32, dtype="f32", w0_std=0.2)
+    hidden = 16
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=33)
+    w = synth.ttt_mlp_weights(cfg, hidden, device="cuda", seed=33)
+    w["dW2_T"].normal_(generator=torch.Generator("cuda").manual_seed(3))
+    f, g = run_mlp(cfg, hidden, inp, w)
+    rf, rg = reference(cfg, inp, w)
+    for k in ("O", "W1_final", "W2_final"):
+        assert rel_err(f[k], rf[k]) <= F32_TOL, k
+    for k in ("dQ", "dK", "dV", "dbeta", "dW1", "dW2"):
+        assert rel_err(g[k], rg[k]) <= F32_TOL, k

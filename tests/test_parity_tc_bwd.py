@@ -5,7 +5,7 @@ import pytest
 import torch
 
 import synth
-from _runners import head_slice, oracle_bwd, run_bwd, run_fwd
+from _runners import head_slice, oracle_bwd, oracle_fwd, run_bwd, run_fwd
 from _util import rel_err
 
 pytestmark = pytest.mark.gpu
@@ -81,3 +81,22 @@ def test_tc_backward_silu_full_size_sampled_heads():
     for k in GRADS + ("dgamma",):
         g = torch.stack([got[k][b, h] for b, h in heads]).unsqueeze(0)
         assert rel_err(g, ref[k]) <= TOL, (k, rel_err(g, ref[k]))
+
+
+@pytest.mark.parametrize("d,C", [(64, 128), (64, 256), (128, 128), (128, 256)])
+@pytest.mark.parametrize("act", ["id", "silu"])
+def test_tc_single_chunk(d, C, act):
+    # T == C: the chain runs one iteration and the decay gradient's state term comes from
+    # W_final and dW_final
+    cfg = synth.SILU_IP_FWD.replace(B=1, H=2, T=C, dk=d, dv=d, C=C, loss="mse", act=act,
+                                    decay=True, w0_std=1.0 / d)
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=d + C)
+    inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(12))
+    fwd = run_fwd(cfg, inp)
+    ref_f = oracle_fwd(cfg, inp)
+    for k in ("O", "W_final", "W_chunks"):
+        assert rel_err(fwd[k], ref_f[k]) <= TOL, k
+    got = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
+    ref = oracle_bwd(cfg, inp)
+    for k in GRADS + ("dgamma",):
+        assert rel_err(got[k], ref[k]) <= TOL, (k, rel_err(got[k], ref[k]))
