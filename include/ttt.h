@@ -207,6 +207,26 @@ ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const 
                            const void* Vhat, float* W, void* O, void* W_chunks, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Document resets (page "In-Place Test-Time Training", section "实践建议": the fast weight is
+ * reset at document boundaries so that no information leaks across documents). Same as
+ * inplace_ttt_fwd / inplace_ttt_bwd with a HOST array doc_starts of n_docs chunk indices
+ * (strictly increasing, each in [1, T/C - 1]) where a new document begins: that chunk applies,
+ * and its update starts from, the initial W_down (the W passed in). W_final is the last
+ * document's end state; the backward's adjoint does not cross a boundary and dW sums the
+ * adjoints reaching every document start. Boundaries fall on chunk starts (pack or pad
+ * documents to multiples of C). Workspace from inplace_ttt_docs_workspace_bytes (one float32
+ * d_model x d_ff matrix more). A malformed list returns TTT_ERR_INVALID_ARG. */
+size_t inplace_ttt_docs_workspace_bytes(int T, int d_ff, int d_model, int C);
+ttt_status inplace_ttt_fwd_docs(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                                const void* Vhat, float* W, void* O, void* W_chunks,
+                                const int* doc_starts, int n_docs, void* workspace,
+                                size_t workspace_bytes, void* stream);
+ttt_status inplace_ttt_bwd_docs(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                                const void* Vhat, const void* W_chunks, const void* dO,
+                                const float* dW_final, void* dZ, void* dVhat, float* dW,
+                                const int* doc_starts, int n_docs, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
 /* Workspace bytes of inplace_ttt_target; (size_t)-1 for invalid sizes. */
 size_t inplace_ttt_target_workspace_bytes(int T, int d_model);
 

@@ -10,7 +10,8 @@ import weight_sequence_layers_b200 as ttt
 FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_ttt_workspace_bytes",
              "inplace_ttt_fwd", "inplace_ttt_bwd", "inplace_ttt_target", "inplace_ttt_target_workspace_bytes",
              "inplace_ttt_target_bwd", "inplace_ttt_target_bwd_workspace_bytes",
-             "ttt_mlp_fwd", "ttt_mlp_bwd", "ttt_mlp_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "ttt_mlp_fwd", "ttt_mlp_bwd", "ttt_mlp_workspace_bytes",
+             "inplace_ttt_fwd_docs", "inplace_ttt_bwd_docs", "inplace_ttt_docs_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
              "ttt_status_string"}
 
 
@@ -240,3 +241,18 @@ def test_ttt_mlp_argument_errors():
     # cfg hidden Q K V beta gamma W1c W2c dO dW1f dW2f dQ dK dV dbeta dW1 dW2 ws bytes stream
     okb = [A, A, A, A, None, None, A, A, None, None, A, A, A, A, A, A, A, need, None]
     assert b(ctypes.byref(cfg), 96, *okb) == ttt.ERR_INVALID_ARG  # W1_chunks is required
+
+
+def test_inplace_document_list_is_checked():
+    A = 4096
+    f = ttt.lib.inplace_ttt_fwd_docs
+    need = ttt.inplace_ttt_docs_workspace_bytes(1024, 256, 256, 128)
+    assert need > ttt.inplace_ttt_workspace_bytes(1024, 256, 256, 128)
+    # T d_ff d_model C lr Z Vhat W O W_chunks doc_starts n_docs workspace bytes stream
+    for bad in ([0], [8], [3, 3], [4, 2], [-1]):  # 8 chunks: starts must be in 1..7, increasing
+        arr = (ctypes.c_int * len(bad))(*bad)
+        assert f(1024, 256, 256, 128, 1e-3, A, A, A, A, None, arr, len(bad), A, need, None) == \
+            ttt.ERR_INVALID_ARG, bad
+    arr = (ctypes.c_int * 1)(3)
+    short = ttt.inplace_ttt_workspace_bytes(1024, 256, 256, 128)
+    assert f(1024, 256, 256, 128, 1e-3, A, A, A, A, None, arr, 1, A, short, None) == ttt.ERR_WORKSPACE

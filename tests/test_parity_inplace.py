@@ -191,3 +191,33 @@ def test_inplace_target_backward_full_size_sampled_channels():
     assert rel_err(got["dX0"][:, ch], ref["dX0"]) <= O_TOL
     assert rel_err(got["dconv_w"][:, ch], ref["dconv_w"]) <= O_TOL
     assert rel_err(got["dW_target"][ch], ref["dW_target"]) <= O_TOL
+
+
+@pytest.mark.parametrize("starts", [[2], [1, 3], [1, 2, 3]])
+def test_inplace_document_resets(starts):
+    cfg = synth.INPLACE_QWEN4B.replace(T=512, d_ff=256, d_model=256, C=128, lr=0.1)
+    inp = synth.inplace_inputs(cfg, device="cuda", seed=61)
+    T, F, M, C = cfg.T, cfg.d_ff, cfg.d_model, cfg.C
+    n = ttt.inplace_ttt_docs_workspace_bytes(T, F, M, C)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    W = inp["W"].clone()
+    O = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+    Wc = torch.empty((T // C, M, F), device="cuda", dtype=torch.bfloat16)
+    ttt.inplace_ttt_fwd_docs(T, F, M, C, cfg.lr, inp["Z"], inp["Vhat"], W, O, Wc, starts, ws, n)
+    dWf = 0.1 * torch.randn((M, F), device="cuda", generator=torch.Generator("cuda").manual_seed(7))
+    dZ = torch.empty((T, F), device="cuda", dtype=torch.bfloat16)
+    dVh = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+    dW = torch.empty((M, F), device="cuda")
+    ttt.inplace_ttt_bwd_docs(T, F, M, C, cfg.lr, inp["Z"], inp["Vhat"], Wc, inp["dO"], dWf, dZ, dVh,
+                             dW, starts, ws, n)
+    torch.cuda.synchronize()
+    assert ttt.ttt_get_device_error() == ttt.OK
+    lr32 = float(np.float32(cfg.lr))
+    Oref, Wref = oracle.inplace_fwd(inp["Z"], inp["Vhat"], inp["W"], C=C, lr=lr32, doc_starts=starts)
+    assert rel_err(O, Oref) <= O_TOL
+    assert rel_err(W, Wref) <= W_TOL
+    ref = oracle.inplace_bwd(inp["Z"], inp["Vhat"], inp["W"], inp["dO"], dWf, C=C, lr=lr32,
+                             doc_starts=starts)
+    assert rel_err(dZ, ref["dZ"]) <= O_TOL
+    assert rel_err(dVh, ref["dVhat"]) <= O_TOL
+    assert rel_err(dW, ref["dW"]) <= W_TOL

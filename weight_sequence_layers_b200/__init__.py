@@ -54,6 +54,9 @@ _SIGS = {
     "inplace_ttt_fwd": ([_i] * 4 + [_f] + [_p] * 6 + [_sz, _p], _i),
     "inplace_ttt_bwd": ([_i] * 4 + [_f] + [_p] * 9 + [_sz, _p], _i),
     "inplace_ttt_target_workspace_bytes": ([_i] * 2, _sz),
+    "inplace_ttt_docs_workspace_bytes": ([_i] * 4, _sz),
+    "inplace_ttt_fwd_docs": ([_i] * 4 + [_f] + [_p] * 6 + [_i, _p, _sz, _p], _i),
+    "inplace_ttt_bwd_docs": ([_i] * 4 + [_f] + [_p] * 9 + [_i, _p, _sz, _p], _i),
     "inplace_ttt_target": ([_i] * 3 + [_p] * 5 + [_sz, _p], _i),
     "inplace_ttt_target_bwd_workspace_bytes": ([_i] * 3, _sz),
     "inplace_ttt_target_bwd": ([_i] * 3 + [_p] * 8 + [_sz, _p], _i),
@@ -187,6 +190,37 @@ def inplace_ttt_fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace=None, work
                               _ptr(O), _ptr(W_chunks), _ptr(workspace), int(workspace_bytes),
                               _stream(stream))
     _check(st, "inplace_ttt_fwd")
+
+
+def _int_array(xs):
+    xs = [int(x) for x in xs]
+    return (ctypes.c_int * max(1, len(xs)))(*xs), len(xs)
+
+
+def inplace_ttt_docs_workspace_bytes(T, d_ff, d_model, C) -> int:
+    n = _lib.inplace_ttt_docs_workspace_bytes(T, d_ff, d_model, C)
+    if n == ctypes.c_size_t(-1).value:
+        raise TTTError(ERR_INVALID_ARG, "inplace_ttt_docs_workspace_bytes")
+    return n
+
+
+def inplace_ttt_fwd_docs(T, d_ff, d_model, C, lr, Z, Vhat, W, O, W_chunks, doc_starts, workspace,
+                         workspace_bytes, stream=None):
+    arr, n = _int_array(doc_starts)
+    st = _lib.inplace_ttt_fwd_docs(T, d_ff, d_model, C, float(lr), _ptr(Z), _ptr(Vhat), _ptr(W),
+                                   _ptr(O), _ptr(W_chunks), arr, n, _ptr(workspace),
+                                   int(workspace_bytes), _stream(stream))
+    _check(st, "inplace_ttt_fwd_docs")
+
+
+def inplace_ttt_bwd_docs(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW,
+                         doc_starts, workspace, workspace_bytes, stream=None):
+    arr, n = _int_array(doc_starts)
+    st = _lib.inplace_ttt_bwd_docs(T, d_ff, d_model, C, float(lr), _ptr(Z), _ptr(Vhat),
+                                   _ptr(W_chunks), _ptr(dO), _ptr(dW_final), _ptr(dZ), _ptr(dVhat),
+                                   _ptr(dW), arr, n, _ptr(workspace), int(workspace_bytes),
+                                   _stream(stream))
+    _check(st, "inplace_ttt_bwd_docs")
 
 
 def inplace_ttt_target_workspace_bytes(T, d_model) -> int:

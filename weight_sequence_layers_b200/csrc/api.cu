@@ -6,7 +6,10 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <memory>
+#include <new>
 #include <mutex>
+#include <vector>
 
 #include "../../include/ttt.h"
 #include "common.cuh"
@@ -304,7 +307,12 @@ size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C) {
   if (T < 1 || d_ff < 1 || d_model < 1 || C < 1 || T % C || C % 128 || d_ff % 64 ||
       d_model % 128)
     return (size_t)-1;
-  return inplace_workspace(T, d_ff, d_model, C);
+  return inplace_workspace(T, d_ff, d_model, C, false);
+}
+
+size_t inplace_ttt_docs_workspace_bytes(int T, int d_ff, int d_model, int C) {
+  if (inplace_ttt_workspace_bytes(T, d_ff, d_model, C) == (size_t)-1) return (size_t)-1;
+  return inplace_workspace(T, d_ff, d_model, C, true);
 }
 
 namespace {
@@ -316,24 +324,87 @@ ttt_status inplace_sizes(int T, int d_ff, int d_model, int C, float lr) {
     return TTT_ERR_INVALID_ARG;
   return TTT_OK;
 }
+
+// Chunk flags from a host list of document-start chunks (strictly increasing, each in
+// [1, NC - 1]); false if the list is malformed.
+bool doc_flags(const int* starts, int n, int NC, std::vector<bool>& flags) {
+  try {
+    flags.assign(NC, false);
+  } catch (...) {
+    return false;
+  }
+  if (n < 0 || (n > 0 && !starts)) return false;
+  for (int k = 0; k < n; ++k) {
+    if (starts[k] < 1 || starts[k] >= NC || (k > 0 && starts[k] <= starts[k - 1])) return false;
+    flags[starts[k]] = true;
+  }
+  return true;
+}
+
+ttt_status inplace_fwd_impl(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                            const void* Vhat, float* W, void* O, void* W_chunks,
+                            const int* doc_starts, int n_docs, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  const ttt_status st = inplace_sizes(T, d_ff, d_model, C, lr);
+  if (st != TTT_OK) return st;
+  if (!Z || !Vhat || !W || !O) return TTT_ERR_INVALID_ARG;
+  std::vector<bool> flags;
+  if (!doc_flags(doc_starts, n_docs, T / C, flags)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Z, Vhat, W, O, W_chunks, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const size_t need = inplace_workspace(T, d_ff, d_model, C, n_docs > 0);
+  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  std::unique_ptr<bool[]> reset(n_docs > 0 ? new (std::nothrow) bool[T / C] : nullptr);
+  if (n_docs > 0 && !reset) return TTT_ERR_INVALID_ARG;
+  for (int i = 0; reset && i < T / C; ++i) reset[i] = flags[i];
+  return launch_status(inplace_run(T, d_ff, d_model, C, lr, Z, Vhat, W, O, W_chunks, reset.get(),
+                                   workspace, err, static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status inplace_bwd_impl(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                            const void* Vhat, const void* W_chunks, const void* dO,
+                            const float* dW_final, void* dZ, void* dVhat, float* dW,
+                            const int* doc_starts, int n_docs, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  const ttt_status st = inplace_sizes(T, d_ff, d_model, C, lr);
+  if (st != TTT_OK) return st;
+  if (!Z || !Vhat || !W_chunks || !dO || !dZ || !dVhat || !dW) return TTT_ERR_INVALID_ARG;
+  std::vector<bool> flags;
+  if (!doc_flags(doc_starts, n_docs, T / C, flags)) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  const size_t need = inplace_workspace(T, d_ff, d_model, C, n_docs > 0);
+  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  std::unique_ptr<bool[]> reset(n_docs > 0 ? new (std::nothrow) bool[T / C] : nullptr);
+  if (n_docs > 0 && !reset) return TTT_ERR_INVALID_ARG;
+  for (int i = 0; reset && i < T / C; ++i) reset[i] = flags[i];
+  return launch_status(inplace_bwd_run(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final,
+                                       dZ, dVhat, dW, reset.get(), workspace, err,
+                                       static_cast<cudaStream_t>(stream)));
+}
 }  // namespace
 
 ttt_status inplace_ttt_fwd(int T, int d_ff, int d_model, int C, float lr, const void* Z,
                            const void* Vhat, float* W, void* O, void* W_chunks, void* workspace,
                            size_t workspace_bytes, void* stream) {
-  const ttt_status st = inplace_sizes(T, d_ff, d_model, C, lr);
-  if (st != TTT_OK) return st;
-  if (!Z || !Vhat || !W || !O) return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {Z, Vhat, W, O, W_chunks, workspace};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
-  const size_t need = inplace_workspace(T, d_ff, d_model, C);
-  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
-  cudaError_t e;
-  unsigned* err = error_word(&e);
-  if (!err) return TTT_ERR_CUDA;
-  return launch_status(inplace_run(T, d_ff, d_model, C, lr, Z, Vhat, W, O, W_chunks, workspace,
-                                   err, static_cast<cudaStream_t>(stream)));
+  return inplace_fwd_impl(T, d_ff, d_model, C, lr, Z, Vhat, W, O, W_chunks, nullptr, 0,
+                          workspace, workspace_bytes, stream);
+}
+
+ttt_status inplace_ttt_fwd_docs(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                                const void* Vhat, float* W, void* O, void* W_chunks,
+                                const int* doc_starts, int n_docs, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return inplace_fwd_impl(T, d_ff, d_model, C, lr, Z, Vhat, W, O, W_chunks, doc_starts, n_docs,
+                          workspace, workspace_bytes, stream);
 }
 
 size_t inplace_ttt_target_workspace_bytes(int T, int d_model) {
@@ -394,20 +465,17 @@ ttt_status inplace_ttt_bwd(int T, int d_ff, int d_model, int C, float lr, const 
                            const void* Vhat, const void* W_chunks, const void* dO,
                            const float* dW_final, void* dZ, void* dVhat, float* dW,
                            void* workspace, size_t workspace_bytes, void* stream) {
-  const ttt_status st = inplace_sizes(T, d_ff, d_model, C, lr);
-  if (st != TTT_OK) return st;
-  if (!Z || !Vhat || !W_chunks || !dO || !dZ || !dVhat || !dW) return TTT_ERR_INVALID_ARG;
-  const void* ptrs[] = {Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW, workspace};
-  for (const void* p : ptrs)
-    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
-  const size_t need = inplace_workspace(T, d_ff, d_model, C);
-  if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
-  cudaError_t e;
-  unsigned* err = error_word(&e);
-  if (!err) return TTT_ERR_CUDA;
-  return launch_status(inplace_bwd_run(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final,
-                                       dZ, dVhat, dW, workspace, err,
-                                       static_cast<cudaStream_t>(stream)));
+  return inplace_bwd_impl(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW,
+                          nullptr, 0, workspace, workspace_bytes, stream);
+}
+
+ttt_status inplace_ttt_bwd_docs(int T, int d_ff, int d_model, int C, float lr, const void* Z,
+                                const void* Vhat, const void* W_chunks, const void* dO,
+                                const float* dW_final, void* dZ, void* dVhat, float* dW,
+                                const int* doc_starts, int n_docs, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  return inplace_bwd_impl(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW,
+                          doc_starts, n_docs, workspace, workspace_bytes, stream);
 }
 
 ttt_status ttt_get_device_error(void* stream) {

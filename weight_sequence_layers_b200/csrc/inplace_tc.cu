@@ -320,6 +320,17 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
 
 constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(Bars) + 1024;
 
+// dst += src over n floats (n a multiple of 4).
+__global__ void add_kernel(float* __restrict__ dst, const float* __restrict__ src, size_t n4) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float4 a = reinterpret_cast<float4*>(dst)[i];
+    const float4 b = reinterpret_cast<const float4*>(src)[i];
+    a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    reinterpret_cast<float4*>(dst)[i] = a;
+  }
+}
+
 // Depthwise convolution over the current and the next k - 1 tokens, zero past the last one:
 // Y[t, c] = sum_{j<k} w[j, c] X0[t + j, c]. One thread per 8 channels and a run of tokens;
 // a warp's loads of one token row are contiguous.
@@ -437,22 +448,27 @@ cudaError_t prepare(Launch* l) {
 }  // namespace
 
 // Two bf16 copies of a d_model x d_ff matrix (read by one launch, written for the next), then
-// one tile counter per chunk.
-size_t inplace_workspace(int T, int d_ff, int d_model, int C) {
+// one tile counter per chunk; with document resets one float32 d_model x d_ff matrix more (the
+// initial W forward, the running adjoint backward).
+size_t inplace_workspace(int T, int d_ff, int d_model, int C, bool docs) {
   const size_t wb = 2 * (size_t)d_model * d_ff * 2;
   const size_t counters = ((size_t)(T / C) * sizeof(int) + 255) & ~size_t(255);
-  return wb + counters;
+  return wb + counters + (docs ? (size_t)d_model * d_ff * 4 : 0);
 }
 
 cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
-                        const void* Vhat, float* W, void* O, void* W_chunks, void* ws,
-                        unsigned* err, cudaStream_t s) {
+                        const void* Vhat, float* W, void* O, void* W_chunks, const bool* reset,
+                        void* ws, unsigned* err, cudaStream_t s) {
   const int NC = T / C;
+  const size_t nW = (size_t)d_model * d_ff;
   // bf16 W_i: the caller's [NC, d_model, d_ff] chunk states when given, else two rotating copies
   __nv_bfloat16* Wb = W_chunks ? static_cast<__nv_bfloat16*>(W_chunks)
                                : static_cast<__nv_bfloat16*>(ws);
   const size_t wb_rows = W_chunks ? (size_t)NC * d_model : 2 * (size_t)d_model;
   int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 2 * (size_t)d_model * d_ff * 2);
+  // with document resets: the initial W, kept after the counters
+  float* W0 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
+                                       inplace_workspace(T, d_ff, d_model, C, false));
   CUtensorMap tza, tzb, twb, tvh;
   if (!make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
       !make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
@@ -462,7 +478,10 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   Launch l;
   cudaError_t e = prepare(&l);
   if (e != cudaSuccess) return e;
-  to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W, Wb, (size_t)d_model * d_ff, 1.f);
+  to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W, Wb, nW, 1.f);
+  int launches = NC + 1;
+  if (reset && (e = cudaMemcpyAsync(W0, W, nW * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+    return e;
   e = cudaMemsetAsync(counters, 0, NC * sizeof(int), s);
   if (e != cudaSuccess) return e;
   Params p{};
@@ -492,18 +511,30 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
       p.wb_next_row0 = ((i + 1) & 1) * d_model;
     }
     p.counter = counters + i;
+    if (reset && i > 0 && reset[i]) {
+      // a new document: this chunk applies, and its update starts from, the initial W
+      if ((e = cudaMemcpyAsync(W, W0, nW * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+        return e;
+      to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W0, Wb + (size_t)p.wb_cur_row0 * d_ff, nW, 1.f);
+      ++launches;
+    }
     inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, twb, tvh, tza, tza, tzb, tzb,
                                                             p);
   }
-  count_launches(NC + 1);
+  count_launches(launches);
   return cudaGetLastError();
 }
 
 cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
                             const void* Vhat, const void* W_chunks, const void* dO,
-                            const float* dW_final, void* dZ, void* dVhat, float* dW, void* ws,
-                            unsigned* err, cudaStream_t s) {
+                            const float* dW_final, void* dZ, void* dVhat, float* dW,
+                            const bool* reset, void* ws, unsigned* err, cudaStream_t s) {
   const int NC = T / C;
+  // with document resets the running adjoint lives in the workspace and dW collects it at every
+  // document start; without, dW is the running adjoint itself
+  float* R = reset ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
+                                              inplace_workspace(T, d_ff, d_model, C, false))
+                   : dW;
   // bf16 eta Wh_{i+1}: two rotating copies
   __nv_bfloat16* Mb = static_cast<__nv_bfloat16*>(ws);
   int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 2 * (size_t)d_model * d_ff * 2);
@@ -522,15 +553,17 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   if (e != cudaSuccess) return e;
   const size_t nW = (size_t)d_model * d_ff;
   const int first = (NC - 1) & 1;  // copy slot the last chunk reads
+  int launches = NC + 1;
   if (dW_final) {
-    e = cudaMemcpyAsync(dW, dW_final, nW * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    e = cudaMemcpyAsync(R, dW_final, nW * sizeof(float), cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess) return e;
     to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(dW_final, Mb + first * nW, nW, lr);
   } else {
-    if ((e = cudaMemsetAsync(dW, 0, nW * sizeof(float), s)) != cudaSuccess ||
+    if ((e = cudaMemsetAsync(R, 0, nW * sizeof(float), s)) != cudaSuccess ||
         (e = cudaMemsetAsync(Mb + first * nW, 0, nW * 2, s)) != cudaSuccess)
       return e;
   }
+  if (reset && (e = cudaMemsetAsync(dW, 0, nW * sizeof(float), s)) != cudaSuccess) return e;
   e = cudaMemsetAsync(counters, 0, NC * sizeof(int), s);
   if (e != cudaSuccess) return e;
   Params p{};
@@ -549,7 +582,7 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   p.kb_upd = C / BK;
   p.acc_scale = 1.f;
   p.copy_scale = lr;
-  p.M = dW;
+  p.M = R;
   p.Mb = Mb;
   p.Orow = static_cast<__nv_bfloat16*>(dVhat);
   p.Odz = static_cast<__nv_bfloat16*>(dZ);
@@ -563,8 +596,18 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
     p.counter = counters + i;
     inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, tmb, tdx, tdo, tvk, twc,
                                                             tmbn, p);
+    if (reset && (i == 0 || reset[i])) {
+      // this document's first chunk applied the initial W: its adjoint joins dW, and the
+      // previous document's end state (and its bf16 copy) gets none
+      add_kernel<<<l.sms * 4, 256, 0, s>>>(dW, R, nW / 4);
+      ++launches;
+      if (i > 0 && ((e = cudaMemsetAsync(R, 0, nW * sizeof(float), s)) != cudaSuccess ||
+                    (e = cudaMemsetAsync(Mb + (size_t)p.wb_next_row0 * d_ff, 0, nW * 2, s)) !=
+                        cudaSuccess))
+        return e;
+    }
   }
-  count_launches(NC + 1);
+  count_launches(launches);
   return cudaGetLastError();
 }
 

@@ -53,10 +53,11 @@ cudaError_t mlp_bwd(const LayerArgs& a, int hidden, const float* W1c, const floa
                     cudaStream_t s);
 
 // In-Place TTT.
-size_t inplace_workspace(int T, int d_ff, int d_model, int C);
+// `reset` (nullable, host, NC entries): chunks that start a new document.
+size_t inplace_workspace(int T, int d_ff, int d_model, int C, bool docs);
 cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
-                        const void* Vhat, float* W, void* O, void* W_chunks, void* ws,
-                        unsigned* err, cudaStream_t s);
+                        const void* Vhat, float* W, void* O, void* W_chunks, const bool* reset,
+                        void* ws, unsigned* err, cudaStream_t s);
 size_t inplace_target_workspace(int T, int d);
 cudaError_t inplace_target_run(int T, int d, int k, const void* X0, const float* conv_w,
                                const void* W_target, void* Vhat, void* ws, unsigned* err,
@@ -68,8 +69,8 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
                                    cudaStream_t s);
 cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
                             const void* Vhat, const void* W_chunks, const void* dO,
-                            const float* dW_final, void* dZ, void* dVhat, float* dW, void* ws,
-                            unsigned* err, cudaStream_t s);
+                            const float* dW_final, void* dZ, void* dVhat, float* dW,
+                            const bool* reset, void* ws, unsigned* err, cudaStream_t s);
 
 // Address of the current device's error word (looked up once per device); NULL on failure.
 unsigned* current_error_word();
