@@ -247,18 +247,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(smem_u32(&bars->acc_full[acc]), aph, ab)) break;
       __syncwarp();
       tc_fence_after();
-      for (int cb = hcol * (BN / 64); cb < (hcol + 1) * (BN / 64); ++cb) {
-        float v[32];
-        tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
-        tmem_wait_ld();
-        const int col0 = x.n0 + cb * 32;
-        if (x.kind != KIND_UPD) {
-          // bf16 rows of O_i / dVhat_i ([T, d_model]) or dZ_i ([T, d_ff])
-          const int ncol = x.kind == KIND_ROW ? p.d_model : p.d_ff;
-          __nv_bfloat16* out = x.kind == KIND_ROW ? p.Orow : p.Odz;
+      const int cb0 = hcol * (BN / 64), cb1 = cb0 + BN / 64;
+      if (x.kind != KIND_UPD) {
+        // bf16 rows of O_i / dVhat_i ([T, d_model]) or dZ_i ([T, d_ff])
+        const int ncol = x.kind == KIND_ROW ? p.d_model : p.d_ff;
+        __nv_bfloat16* out = (x.kind == KIND_ROW ? p.Orow : p.Odz) +
+                             (size_t)(row_base + x.m0 + row) * ncol;
+        for (int cb = cb0; cb < cb1; ++cb) {
+          float v[32];
+          tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
+          tmem_wait_ld();
+          const int col0 = x.n0 + cb * 32;
           if (col0 < ncol) {
-            uint4* dst =
-                reinterpret_cast<uint4*>(out + (size_t)(row_base + x.m0 + row) * ncol + col0);
+            uint4* dst = reinterpret_cast<uint4*>(out + col0);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
               dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]),
@@ -266,30 +267,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                                   pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
                                   pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
           }
-        } else {
-          const int m = x.m0 + row;
-          if (col0 < p.d_ff && m < p.d_model) {
-            float4* w = reinterpret_cast<float4*>(p.M + (size_t)m * p.d_ff + col0);
-            uint4* wb = p.wb_next_row0 < 0 ? nullptr
-                                           : reinterpret_cast<uint4*>(
-                                                 p.Mb + (size_t)(p.wb_next_row0 + m) * p.d_ff + col0);
-            const float s = p.acc_scale, cs = p.copy_scale;
+        }
+      } else {
+        // fp32 read-modify-write of this thread's row of M and its scaled bf16 copy. The eight
+        // float4 loads of a 32-column step go out together, and the next step's loads are in
+        // flight while this step's results are stored.
+        const int m = x.m0 + row;
+        const bool rowok = m < p.d_model;
+        float* mrow = p.M + (size_t)m * p.d_ff;
+        __nv_bfloat16* brow =
+            p.wb_next_row0 < 0 ? nullptr : p.Mb + (size_t)(p.wb_next_row0 + m) * p.d_ff;
+        const float s = p.acc_scale, cs = p.copy_scale;
+        float4 wv[8];
+        auto load8 = [&](int cb) {
+          const int c0 = x.n0 + cb * 32;
+          if (rowok && c0 < p.d_ff) {
+            const float4* src = reinterpret_cast<const float4*>(mrow + c0);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float4 a0 = w[2 * j], a1 = w[2 * j + 1];
-              a0.x += s * v[8 * j + 0];
-              a0.y += s * v[8 * j + 1];
-              a0.z += s * v[8 * j + 2];
-              a0.w += s * v[8 * j + 3];
-              a1.x += s * v[8 * j + 4];
-              a1.y += s * v[8 * j + 5];
-              a1.z += s * v[8 * j + 6];
-              a1.w += s * v[8 * j + 7];
-              w[2 * j] = a0;
-              w[2 * j + 1] = a1;
-              if (wb)
-                wb[j] = make_uint4(pack_bf16x2(cs * a0.x, cs * a0.y), pack_bf16x2(cs * a0.z, cs * a0.w),
-                                   pack_bf16x2(cs * a1.x, cs * a1.y), pack_bf16x2(cs * a1.z, cs * a1.w));
+            for (int j = 0; j < 8; ++j) wv[j] = src[j];
+          }
+        };
+        load8(cb0);
+        for (int cb = cb0; cb < cb1; ++cb) {
+          float v[32];
+          tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
+          tmem_wait_ld();
+          const int col0 = x.n0 + cb * 32;
+          if (rowok && col0 < p.d_ff) {
+            float4 o[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              o[j] = make_float4(wv[j].x + s * v[4 * j], wv[j].y + s * v[4 * j + 1],
+                                 wv[j].z + s * v[4 * j + 2], wv[j].w + s * v[4 * j + 3]);
+            if (cb + 1 < cb1) load8(cb + 1);
+            float4* dst = reinterpret_cast<float4*>(mrow + col0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dst[j] = o[j];
+            if (brow) {
+              uint4* bd = reinterpret_cast<uint4*>(brow + col0);
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                bd[j] = make_uint4(pack_bf16x2(cs * o[2 * j].x, cs * o[2 * j].y),
+                                   pack_bf16x2(cs * o[2 * j].z, cs * o[2 * j].w),
+                                   pack_bf16x2(cs * o[2 * j + 1].x, cs * o[2 * j + 1].y),
+                                   pack_bf16x2(cs * o[2 * j + 1].z, cs * o[2 * j + 1].w));
             }
           }
         }
