@@ -38,6 +38,7 @@ constexpr uint32_t B_BYTES = BN * BK * 2;      // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
+constexpr int kXpose = 32 * 33;  // floats of one epilogue warp's padded 32 x 32 transpose tile
 constexpr uint32_t kTmemCols = 512;            // two 256-column accumulators
 
 struct Params {
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
+  float* xpose = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + sizeof(Bars));
   const uint32_t stage0 = smem_u32(smem);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   Abort ab{&bars->abort_flag, p.err};
@@ -269,50 +271,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // fp32 read-modify-write of this thread's row of M and its scaled bf16 copy. The eight
-        // float4 loads of a 32-column step go out together, and the next step's loads are in
-        // flight while this step's results are stored.
-        const int m = x.m0 + row;
-        const bool rowok = m < p.d_model;
-        float* mrow = p.M + (size_t)m * p.d_ff;
-        __nv_bfloat16* brow =
-            p.wb_next_row0 < 0 ? nullptr : p.Mb + (size_t)(p.wb_next_row0 + m) * p.d_ff;
+        // fp32 read-modify-write of M and its scaled bf16 copy. TMEM hands each thread one row;
+        // a padded shared tile transposes the warp's 32 x 32 block so that the lanes walk along
+        // a row and every global access is one coalesced 128-byte (bf16: 64-byte) request.
+        float* xt = xpose + (warp - 2) * kXpose;
+        const int mbase = x.m0 + q * 32;
         const float s = p.acc_scale, cs = p.copy_scale;
-        float4 wv[8];
-        auto load8 = [&](int cb) {
-          const int c0 = x.n0 + cb * 32;
-          if (rowok && c0 < p.d_ff) {
-            const float4* src = reinterpret_cast<const float4*>(mrow + c0);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) wv[j] = src[j];
-          }
-        };
-        load8(cb0);
         for (int cb = cb0; cb < cb1; ++cb) {
           float v[32];
           tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
           tmem_wait_ld();
-          const int col0 = x.n0 + cb * 32;
-          if (rowok && col0 < p.d_ff) {
-            float4 o[8];
+          const int col = x.n0 + cb * 32 + lane;
+          if (x.n0 + cb * 32 >= p.d_ff) continue;  // the same for every lane
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              o[j] = make_float4(wv[j].x + s * v[4 * j], wv[j].y + s * v[4 * j + 1],
-                                 wv[j].z + s * v[4 * j + 2], wv[j].w + s * v[4 * j + 3]);
-            if (cb + 1 < cb1) load8(cb + 1);
-            float4* dst = reinterpret_cast<float4*>(mrow + col0);
+          for (int j = 0; j < 32; ++j) xt[lane * 33 + j] = v[j];
+          __syncwarp();
+          const size_t ld = p.d_ff;
+#pragma unroll 1
+          for (int h = 0; h < 2; ++h) {
+            // rows mbase + 16 h .. + 15: sixteen coalesced loads in flight, then the stores
+            const int m0 = mbase + 16 * h;
+            float* mp = p.M + (size_t)m0 * ld + col;
+            float w[16];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) dst[j] = o[j];
-            if (brow) {
-              uint4* bd = reinterpret_cast<uint4*>(brow + col0);
+            for (int r = 0; r < 16; ++r) w[r] = m0 + r < p.d_model ? mp[r * ld] : 0.f;
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                bd[j] = make_uint4(pack_bf16x2(cs * o[2 * j].x, cs * o[2 * j].y),
-                                   pack_bf16x2(cs * o[2 * j].z, cs * o[2 * j].w),
-                                   pack_bf16x2(cs * o[2 * j + 1].x, cs * o[2 * j + 1].y),
-                                   pack_bf16x2(cs * o[2 * j + 1].z, cs * o[2 * j + 1].w));
+            for (int r = 0; r < 16; ++r) {
+              if (m0 + r < p.d_model) {
+                const float o = w[r] + s * xt[(16 * h + r) * 33 + lane];
+                mp[r * ld] = o;
+                if (p.wb_next_row0 >= 0)
+                  p.Mb[(size_t)(p.wb_next_row0 + m0 + r) * ld + col] = __float2bfloat16_rn(cs * o);
+              }
             }
           }
+          __syncwarp();  // the tile is rewritten by the next step
         }
       }
       tc_fence_before();
@@ -339,7 +332,8 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
     dst[i] = __float2bfloat16_rn(scale * src[i]);
 }
 
-constexpr size_t kSmemBytes = STAGES * STAGE_BYTES + sizeof(Bars) + 1024;
+constexpr size_t kSmemBytes =
+    STAGES * STAGE_BYTES + sizeof(Bars) + kEpiWarps * kXpose * sizeof(float) + 1024;
 
 // dst += src over n floats (n a multiple of 4).
 __global__ void add_kernel(float* __restrict__ dst, const float* __restrict__ src, size_t n4) {
