@@ -356,34 +356,59 @@ def time_steps(layer, steps, warmup, sampler=None):
     return total, fwd_ms, bwd_ms, launches
 
 
-def time_e2e(layer, steps, warmup):
+def time_e2e(layer, layer2, steps, warmup):
     """Same step through the binding with the inputs in pinned HOST memory: every step copies
-    the inputs host->device and the gradients device->host inside the timed region."""
-    i = layer.inp
+    its inputs host->device and its gradients device->host inside the timed region. The loop is
+    pipelined the way a training loop feeds a GPU: two device buffer sets (`layer`, `layer2`),
+    step n uploads into set n % 2 on one copy stream while step n - 1 computes, and downloads its
+    gradients on a second copy stream while step n + 1 computes, so both PCIe directions and the
+    kernels overlap. The timed region spans the first upload to the last download."""
     names_in = ["Q", "K", "V", "dO", "beta", "gamma", "W0"]
-    host_in = {k: i[k].to("cpu").pin_memory() for k in names_in if i[k] is not None}
-    outs = {"dQ": layer.dQ, "dK": layer.dK, "dV": layer.dV, "dbeta": layer.dbeta, "dW0": layer.dW0}
-    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
+    host_in = {k: layer.inp[k].to("cpu").pin_memory() for k in names_in if layer.inp[k] is not None}
+    out_names = ["dQ", "dK", "dV", "dbeta", "dW0"]
+    sets = (layer, layer2)
+    host_out = [{k: torch.empty(getattr(L, k).shape, dtype=getattr(L, k).dtype, pin_memory=True)
+                 for k in out_names} for L in sets]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out[0].values())
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in sets]
+    ev_done = [torch.cuda.Event() for _ in sets]
+    ev_out = [torch.cuda.Event() for _ in sets]
+    for e in ev_done + ev_out:
+        e.record(comp)
 
-    def step():
-        for k, t in host_in.items():
-            i[k].copy_(t, non_blocking=True)
-        layer.fwd()
-        layer.bwd()
-        for k, t in outs.items():
-            host_out[k].copy_(t, non_blocking=True)
+    def step(n):
+        b = n % 2
+        L = sets[b]
+        with torch.cuda.stream(up):
+            up.wait_event(ev_done[b])  # step n - 2 has finished reading this set's inputs
+            for k, t in host_in.items():
+                L.inp[k].copy_(t, non_blocking=True)
+            ev_in[b].record(up)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])     # step n - 2's gradients have left this set
+        L.fwd()
+        L.bwd()
+        ev_done[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[b])
+            for k in out_names:
+                host_out[b][k].copy_(getattr(L, k), non_blocking=True)
+            ev_out[b].record(down)
 
-    for _ in range(warmup):
-        step()
+    for n in range(warmup):
+        step(n)
     torch.cuda.synchronize()
     barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(steps):
-        step()
-    e.record()
+    s.record(comp)
+    up.wait_stream(comp)
+    for n in range(steps):
+        step(n)
+    comp.wait_stream(down)
+    e.record(comp)
     torch.cuda.synchronize()
     barrier()
     return s.elapsed_time(e), h2d, d2h
@@ -599,7 +624,9 @@ def main():
     if dg_ms is not None:
         out["kernels_ms"]["ttt_chunk_bwd_with_dgamma"] = dg_ms
     if not args.no_e2e:
-        e2e_ms, h2d, d2h = time_e2e(layer, args.steps, args.warmup)
+        layer2 = Layer(cfg, ttt, seed=cfg.seed + 100)  # second buffer set of the pipeline
+        e2e_ms, h2d, d2h = time_e2e(layer, layer2, args.steps, args.warmup)
+        del layer2
         e2e_ms = reduce_max(e2e_ms)
         out["e2e"] = {"value": tokens / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
