@@ -227,6 +227,21 @@ ttt_status inplace_ttt_bwd_docs(int T, int d_ff, int d_model, int C, float lr, c
                                 const int* doc_starts, int n_docs, void* workspace,
                                 size_t workspace_bytes, void* stream);
 
+/* Context-parallel building blocks (page "In-Place Test-Time Training", section "核心方法和技术
+ * 细节": the update is associative, so a sequence split across devices runs as a parallel scan):
+ * with the sequence cut into shards, shard g starts from W_0 + sum_{h<g} dW_h where
+ *     dW_h = lr Vhat_h^T Z_h     (inplace_ttt_delta: every chunk update of shard h, summed)
+ * and then runs inplace_ttt_fwd on its own tokens. The exchange of the dW_h between devices is
+ * the caller's (the Python binding's inplace_cp_fwd uses torch.distributed); ttt_add_f32 adds
+ * them on the device.
+ *  Z [T, d_ff], Vhat [T, d_model] bf16; dW [d_model, d_ff] float32 out (plain stores).
+ *  Requirements: T % 128 == 0, d_ff % 64 == 0, d_model % 128 == 0; workspace >= 256 bytes. */
+ttt_status inplace_ttt_delta(int T, int d_ff, int d_model, float lr, const void* Z,
+                             const void* Vhat, float* dW, void* workspace, size_t workspace_bytes,
+                             void* stream);
+/* dst[i] += src[i] over n float32 (device pointers, n % 4 == 0). */
+ttt_status ttt_add_f32(float* dst, const float* src, size_t n, void* stream);
+
 /* Workspace bytes of inplace_ttt_target; (size_t)-1 for invalid sizes. */
 size_t inplace_ttt_target_workspace_bytes(int T, int d_model);
 

@@ -1,6 +1,6 @@
-"""The multi-rank path of bench.py on CPU with the gloo backend (world size 2): ranks run
-independent replicas, the step time is the max over ranks and the throughput aggregates all
-ranks' tokens (weak scaling, no data-path collective)."""
+"""Multi-rank paths on CPU with the gloo backend (world size 2): bench.py's replicas (the step
+time is the max over ranks and the throughput aggregates all ranks' tokens; weak scaling, no
+data-path collective) and the exchange of the context-parallel In-Place forward."""
 import os
 import socket
 
@@ -53,3 +53,87 @@ def test_replica_timing_is_max_over_ranks_and_tokens_add_up():
     for ms, value in res.values():
         assert ms == pytest.approx(20.0 / 5)                    # slowest rank, per step
         assert value == pytest.approx(2 * 1000 / (4.0e-3))      # both ranks' tokens
+
+
+
+class _OracleOps:
+    """CPU stand-ins of the library calls of inplace_cp_fwd, written on the oracle, so the
+    exchange (all-gather and the exclusive prefix) is tested without a GPU."""
+
+    @staticmethod
+    def delta(T, d_ff, d_model, lr, Z, Vhat, dW, workspace, workspace_bytes):
+        import numpy as np
+        import torch
+        import oracle
+        W0 = np.zeros((d_model, d_ff))
+        # one chunk from zero: lr Vhat^T Z (float64 arrays straight to the oracle)
+        _, WF = oracle.inplace_fwd(Z.numpy(), Vhat.numpy(), W0, C=T, lr=lr)
+        dW.copy_(torch.from_numpy(WF))
+
+    @staticmethod
+    def add(dst, src):
+        dst.add_(src)
+
+    @staticmethod
+    def fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace, workspace_bytes):
+        import torch
+        import oracle
+        o, wf = oracle.inplace_fwd(Z.numpy(), Vhat.numpy(), W.numpy(), C=C, lr=lr)
+        O.copy_(torch.from_numpy(o))
+        W.copy_(torch.from_numpy(wf))
+
+
+def _cp_rank(rank, world, port, out):
+    import datetime
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import weight_sequence_layers_b200 as ttt
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        rng = np.random.default_rng(70)
+        T, d_ff, d_model, C, lr = 8 * world, 6, 5, 4, 0.1
+        Z = rng.standard_normal((T, d_ff))
+        Vh = rng.standard_normal((T, d_model))
+        W0 = rng.standard_normal((d_model, d_ff))
+        n = T // world
+        sl = slice(rank * n, (rank + 1) * n)
+        W = torch.from_numpy(W0.copy())
+        O = torch.empty((n, d_model), dtype=torch.float64)
+        ttt.inplace_cp_fwd(n, d_ff, d_model, C, lr, torch.from_numpy(Z[sl].copy()),
+                           torch.from_numpy(Vh[sl].copy()), W, O, None, 0, ops=_OracleOps)
+        out[rank] = (O.numpy().tolist(), W.numpy().tolist())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_inplace_context_parallel_scan_equals_one_sequence():
+    import numpy as np
+
+    import oracle
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_cp_rank, args=(r, world, port, out)) for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(90)
+            assert p.exitcode == 0
+        res = dict(out)
+    rng = np.random.default_rng(70)
+    T, d_ff, d_model, C, lr = 8 * world, 6, 5, 4, 0.1
+    Z = rng.standard_normal((T, d_ff))
+    Vh = rng.standard_normal((T, d_model))
+    W0 = rng.standard_normal((d_model, d_ff))
+    O, WF = oracle.inplace_fwd(Z, Vh, W0, C=C, lr=lr)
+    got = np.concatenate([np.array(res[r][0]) for r in range(world)])
+    np.testing.assert_allclose(got, O, atol=1e-12)
+    np.testing.assert_allclose(np.array(res[world - 1][1]), WF, atol=1e-12)

@@ -221,3 +221,36 @@ def test_inplace_document_resets(starts):
     assert rel_err(dZ, ref["dZ"]) <= O_TOL
     assert rel_err(dVh, ref["dVhat"]) <= O_TOL
     assert rel_err(dW, ref["dW"]) <= W_TOL
+
+
+def test_inplace_delta_and_single_rank_context_parallel():
+    import datetime
+    import os
+    import socket
+
+    import torch.distributed as dist
+    cfg = synth.INPLACE_QWEN4B.replace(T=512, d_ff=256, d_model=256, C=128, lr=0.1)
+    inp = synth.inplace_inputs(cfg, device="cuda", seed=71)
+    T, F, M, C = cfg.T, cfg.d_ff, cfg.d_model, cfg.C
+    n = ttt.inplace_ttt_workspace_bytes(T, F, M, C)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    dW = torch.empty((M, F), device="cuda")
+    ttt.inplace_ttt_delta(T, F, M, cfg.lr, inp["Z"], inp["Vhat"], dW, ws, n)
+    lr32 = float(np.float32(cfg.lr))
+    _, WF = oracle.inplace_fwd(inp["Z"], inp["Vhat"], np.zeros((M, F)), C=T, lr=lr32)
+    torch.cuda.synchronize()
+    assert rel_err(dW, WF) <= W_TOL
+    # one rank: the context-parallel forward is the plain forward
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        W = inp["W"].clone()
+        O = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+        ttt.inplace_cp_fwd(T, F, M, C, cfg.lr, inp["Z"], inp["Vhat"], W, O, ws, n)
+    finally:
+        dist.destroy_process_group()
+    O2, W2 = run(cfg, inp)
+    assert torch.equal(O, O2) and torch.equal(W, W2)

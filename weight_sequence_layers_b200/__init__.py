@@ -55,6 +55,8 @@ _SIGS = {
     "inplace_ttt_bwd": ([_i] * 4 + [_f] + [_p] * 9 + [_sz, _p], _i),
     "inplace_ttt_target_workspace_bytes": ([_i] * 2, _sz),
     "inplace_ttt_docs_workspace_bytes": ([_i] * 4, _sz),
+    "inplace_ttt_delta": ([_i] * 3 + [_f] + [_p] * 4 + [_sz, _p], _i),
+    "ttt_add_f32": ([_p, _p, _sz, _p], _i),
     "inplace_ttt_fwd_docs": ([_i] * 4 + [_f] + [_p] * 6 + [_i, _p, _sz, _p], _i),
     "inplace_ttt_bwd_docs": ([_i] * 4 + [_f] + [_p] * 9 + [_i, _p, _sz, _p], _i),
     "inplace_ttt_target": ([_i] * 3 + [_p] * 5 + [_sz, _p], _i),
@@ -275,3 +277,56 @@ def ttt_kernel_launches() -> int:
 
 # Raw C entry points (for callers that marshal pointers themselves).
 lib = _lib
+
+
+def inplace_ttt_delta(T, d_ff, d_model, lr, Z, Vhat, dW, workspace, workspace_bytes, stream=None):
+    """dW = lr Vhat^T Z over all T tokens (the summed chunk updates of one shard)."""
+    st = _lib.inplace_ttt_delta(T, d_ff, d_model, float(lr), _ptr(Z), _ptr(Vhat), _ptr(dW),
+                                _ptr(workspace), int(workspace_bytes), _stream(stream))
+    _check(st, "inplace_ttt_delta")
+
+
+def ttt_add_f32(dst, src, stream=None):
+    st = _lib.ttt_add_f32(_ptr(dst), _ptr(src), int(dst.numel()), _stream(stream))
+    _check(st, "ttt_add_f32")
+
+
+class _CudaOps:
+    """The library calls the context-parallel In-Place forward is made of."""
+
+    @staticmethod
+    def delta(T, d_ff, d_model, lr, Z, Vhat, dW, workspace, workspace_bytes):
+        inplace_ttt_delta(T, d_ff, d_model, lr, Z, Vhat, dW, workspace, workspace_bytes)
+
+    @staticmethod
+    def add(dst, src):
+        ttt_add_f32(dst, src)
+
+    @staticmethod
+    def fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace, workspace_bytes):
+        inplace_ttt_fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace, workspace_bytes)
+
+
+def inplace_cp_fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace, workspace_bytes,
+                   group=None, ops=None):
+    """Context-parallel In-Place forward (page "In-Place Test-Time Training", section "核心方法和
+    技术细节": the update is associative, so the chunk loop runs as a parallel scan across
+    devices). The sequence is split in order across the ranks of `group`; this rank holds its
+    T tokens (Z [T, d_ff], Vhat [T, d_model]), and W holds the initial W_down on every rank.
+    Each rank computes its shard's summed update dW_g = lr Vhat_g^T Z_g, the ranks exchange
+    them (all-gather), rank g adds dW_h for h < g to W and runs inplace_ttt_fwd on its tokens.
+    On return O holds this shard's outputs and W its end state (the last rank's W is the
+    sequence's final W_down). `ops` replaces the library calls (the CPU tests of the exchange
+    pass an implementation built on the oracle); by default they are the C ABI's."""
+    import torch
+    import torch.distributed as dist
+    ops = ops or _CudaOps
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    dW = torch.empty_like(W)
+    ops.delta(T, d_ff, d_model, lr, Z, Vhat, dW, workspace, workspace_bytes)
+    parts = [torch.empty_like(dW) for _ in range(world)]
+    dist.all_gather(parts, dW, group=group)
+    for h in range(rank):
+        ops.add(W, parts[h])
+    ops.fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace, workspace_bytes)

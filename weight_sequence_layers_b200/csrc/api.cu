@@ -407,6 +407,30 @@ ttt_status inplace_ttt_fwd_docs(int T, int d_ff, int d_model, int C, float lr, c
                           workspace, workspace_bytes, stream);
 }
 
+ttt_status inplace_ttt_delta(int T, int d_ff, int d_model, float lr, const void* Z,
+                             const void* Vhat, float* dW, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (T < 1 || d_ff < 1 || d_model < 1 || !isfinite(lr) || (long long)T * d_ff > (1ll << 40))
+    return TTT_ERR_INVALID_ARG;
+  if (T % 128 || d_ff % 64 || d_model % 128) return TTT_ERR_UNSUPPORTED;
+  if (!Z || !Vhat || !dW) return TTT_ERR_INVALID_ARG;
+  const void* ptrs[] = {Z, Vhat, dW, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < 256) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
+  return launch_status(inplace_delta_run(T, d_ff, d_model, lr, Z, Vhat, dW, workspace, err,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+ttt_status ttt_add_f32(float* dst, const float* src, size_t n, void* stream) {
+  if (!dst || !src || n % 4) return TTT_ERR_INVALID_ARG;
+  if (!aligned16(dst) || !aligned16(src)) return TTT_ERR_ALIGNMENT;
+  return launch_status(add_f32_run(dst, src, n, static_cast<cudaStream_t>(stream)));
+}
+
 size_t inplace_ttt_target_workspace_bytes(int T, int d_model) {
   if (T < 1 || d_model < 1 || T % 128 || d_model % 128 || (long long)T * d_model > (1ll << 40))
     return (size_t)-1;

@@ -730,4 +730,51 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
   return cudaGetLastError();
 }
 
+// dW = lr Vhat^T Z over all T tokens (the update of every chunk summed; the update is
+// associative): one launch of update tiles with K = T into the zeroed float32 dW.
+cudaError_t inplace_delta_run(int T, int d_ff, int d_model, float lr, const void* Z,
+                              const void* Vhat, float* dW, void* ws, unsigned* err,
+                              cudaStream_t s) {
+  int* counter = static_cast<int*>(ws);
+  CUtensorMap tzb, tvh;
+  if (!make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
+      !make_tmap_bf16(&tvh, Vhat, d_model, T, d_model, 64, BK))
+    return cudaErrorInvalidValue;
+  Launch l;
+  cudaError_t e = prepare(&l);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(dW, 0, (size_t)d_model * d_ff * sizeof(float), s)) != cudaSuccess ||
+      (e = cudaMemsetAsync(counter, 0, sizeof(int), s)) != cudaSuccess)
+    return e;
+  Params p{};
+  p.chunk = 0;
+  p.C = T;
+  p.d_ff = d_ff;
+  p.d_model = d_model;
+  p.n_upd_n = (d_ff + BN - 1) / BN;
+  p.n_total = (d_model / BM) * p.n_upd_n;
+  p.kb_upd = T / BK;
+  p.wb_next_row0 = -1;
+  p.acc_scale = lr;
+  p.copy_scale = 1.f;
+  p.M = dW;
+  p.counter = counter;
+  p.err = err;
+  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
+  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tzb, tzb, tzb, tvh, tzb, tzb, tzb, tzb, p);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t add_f32_run(float* dst, const float* src, size_t n, cudaStream_t s) {
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  add_kernel<<<sms * 4, 256, 0, s>>>(dst, src, n / 4);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
 }  // namespace tttk

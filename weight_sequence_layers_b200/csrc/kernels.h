@@ -67,6 +67,10 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
                                    const void* W_target, const void* dVhat, void* dX0,
                                    float* dconv_w, float* dW_target, void* ws, unsigned* err,
                                    cudaStream_t s);
+cudaError_t inplace_delta_run(int T, int d_ff, int d_model, float lr, const void* Z,
+                              const void* Vhat, float* dW, void* ws, unsigned* err,
+                              cudaStream_t s);
+cudaError_t add_f32_run(float* dst, const float* src, size_t n, cudaStream_t s);
 cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const void* Z,
                             const void* Vhat, const void* W_chunks, const void* dO,
                             const float* dW_final, void* dZ, void* dVhat, float* dW,
