@@ -11,7 +11,8 @@ FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_t
              "inplace_ttt_fwd", "inplace_ttt_bwd", "inplace_ttt_target", "inplace_ttt_target_workspace_bytes",
              "inplace_ttt_target_bwd", "inplace_ttt_target_bwd_workspace_bytes",
              "ttt_mlp_fwd", "ttt_mlp_bwd", "ttt_mlp_workspace_bytes",
-             "inplace_ttt_fwd_docs", "inplace_ttt_bwd_docs", "inplace_ttt_docs_workspace_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "inplace_ttt_fwd_docs", "inplace_ttt_bwd_docs", "inplace_ttt_docs_workspace_bytes",
+             "inplace_ttt_delta", "ttt_add_f32", "ttt_get_device_error", "ttt_selftest_bounded_wait",
              "ttt_status_string"}
 
 
@@ -256,3 +257,17 @@ def test_inplace_document_list_is_checked():
     arr = (ctypes.c_int * 1)(3)
     short = ttt.inplace_ttt_workspace_bytes(1024, 256, 256, 128)
     assert f(1024, 256, 256, 128, 1e-3, A, A, A, A, None, arr, 1, A, short, None) == ttt.ERR_WORKSPACE
+
+
+def test_context_parallel_calls_check_arguments():
+    A = 4096
+    d = ttt.lib.inplace_ttt_delta
+    # T d_ff d_model lr Z Vhat dW workspace bytes stream
+    assert d(200, 256, 256, 1e-3, A, A, A, A, 256, None) == ttt.ERR_UNSUPPORTED   # T % 128
+    assert d(256, 256, 256, float("nan"), A, A, A, A, 256, None) == ttt.ERR_INVALID_ARG
+    assert d(256, 256, 256, 1e-3, A, A, None, A, 256, None) == ttt.ERR_INVALID_ARG
+    assert d(256, 256, 256, 1e-3, A, A, A, A, 255, None) == ttt.ERR_WORKSPACE
+    a = ttt.lib.ttt_add_f32
+    assert a(A, A, 6, None) == ttt.ERR_INVALID_ARG      # n % 4
+    assert a(A + 4, A, 8, None) == ttt.ERR_ALIGNMENT
+    assert a(None, A, 8, None) == ttt.ERR_INVALID_ARG
