@@ -20,14 +20,6 @@ __device__ __forceinline__ float act_f(float z) {
   if constexpr (ACT == 1) return z * sigm(z);
   return z;
 }
-template <int ACT>
-__device__ __forceinline__ float act_d1(float z) {
-  if constexpr (ACT == 1) {
-    const float s = sigm(z);
-    return s * (1.f + z * (1.f - s));
-  }
-  return 1.f;
-}
 // act(z) and act'(z) from one sigmoid.
 template <int ACT>
 __device__ __forceinline__ void act_both(float z, float& f, float& d1) {
@@ -111,34 +103,6 @@ __device__ __forceinline__ void chunk_scan_warp(const float* beta, const float* 
     cT16[r] = __expf(Lr - L16);
   }
   __syncwarp();
-}
-
-// Causal decay weights of one query s against 32 consecutive keys r0..r0+31 (r0 % 16 == 0):
-//   w_j = [r <= s] eta_r exp(L_s - L_r) = [r <= s] exp(L_s - L_{r16}) * cF16_r.
-// One exponential per 16 keys, no division; the first factor is <= 1 whenever a key of the
-// group precedes s, the second is bounded by the decay of at most 15 tokens.
-__device__ __forceinline__ void causal_weights_q(const float* L, const float* cF16, int s, float Ls,
-                                                 int r0, float (&w)[32]) {
-#pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    const int r16 = r0 + 16 * g;
-    const float a = s >= r16 ? __expf(Ls - L[r16]) : 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) w[16 * g + j] = (r16 + j <= s) ? a * cF16[r16 + j] : 0.f;
-  }
-}
-
-// Causal decay weights of one key r against 32 consecutive queries s0..s0+31 (s0 % 16 == 0):
-//   w_j = [s >= r] exp(L_s - L_r) = [s >= r] exp(L_{s16} - L_r) * cT16_s.
-__device__ __forceinline__ void causal_weights_k(const float* L, const float* cT16, int r, float Lr,
-                                                 int s0, float (&w)[32]) {
-#pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    const int s16 = s0 + 16 * g;
-    const float b = s16 + 15 >= r ? __expf(L[s16] - Lr) : 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) w[16 * g + j] = (s16 + j >= r) ? b * cT16[s16 + j] : 0.f;
-  }
 }
 
 // -S for one query s (chunk-local) against 32 keys r0.. (r0 % 32 == 0), packed to bf16 pairs:
@@ -279,12 +243,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
-}
-
-// 32 consecutive floats -> 16 packed bf16 pairs (even index in the low half).
-__device__ __forceinline__ void pack32(const float (&x)[32], uint32_t (&w)[16]) {
-#pragma unroll
-  for (int j = 0; j < 16; ++j) w[j] = pack_bf16x2(x[2 * j], x[2 * j + 1]);
 }
 
 }  // namespace
