@@ -99,6 +99,10 @@ typedef struct {
  * Returns (size_t)-1 if the config (or for_bwd) is invalid. */
 size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd);
 
+/* Bytes of the G_saved buffer of this config (B*H*T*dv elements of cfg->dtype, twice that with
+ * SiLU, where Zq follows G); (size_t)-1 if the config is invalid. */
+size_t ttt_saved_bytes(const ttt_config* cfg);
+
 /* Forward of the chunkwise TTT layer.
  *  in : Q, K, V, beta, gamma (nullable), W0
  *  out: O; W_final (nullable) = state after the last token; W_chunks (nullable) = chunk-start

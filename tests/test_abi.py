@@ -12,7 +12,7 @@ FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_t
              "inplace_ttt_target_bwd", "inplace_ttt_target_bwd_workspace_bytes",
              "ttt_mlp_fwd", "ttt_mlp_bwd", "ttt_mlp_workspace_bytes",
              "inplace_ttt_fwd_docs", "inplace_ttt_bwd_docs", "inplace_ttt_docs_workspace_bytes",
-             "inplace_ttt_delta", "ttt_add_f32", "ttt_get_device_error", "ttt_selftest_bounded_wait",
+             "inplace_ttt_delta", "ttt_add_f32", "ttt_saved_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
              "ttt_status_string"}
 
 
@@ -271,3 +271,13 @@ def test_context_parallel_calls_check_arguments():
     assert a(A, A, 6, None) == ttt.ERR_INVALID_ARG      # n % 4
     assert a(A + 4, A, 8, None) == ttt.ERR_ALIGNMENT
     assert a(None, A, 8, None) == ttt.ERR_INVALID_ARG
+
+
+def test_saved_buffer_size():
+    cfg = _cfg(dtype="bf16", dk=128, dv=96, C=128, T=512)
+    assert ttt.ttt_saved_bytes(cfg) == 2 * 3 * 512 * 96 * 2
+    assert ttt.ttt_saved_bytes(_cfg(dtype="bf16", dk=128, dv=96, C=128, T=512, act="silu")) == \
+        2 * 2 * 3 * 512 * 96 * 2
+    assert ttt.ttt_saved_bytes(_cfg()) == 2 * 3 * 256 * 64 * 4
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_saved_bytes(_cfg(T=250))

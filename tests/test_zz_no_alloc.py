@@ -58,6 +58,18 @@ def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
             assert rel_err(got[k], ref[k]) <= TOL, (seed, k)
 
 
+def test_noalloc_backward_silu():
+    # SiLU reads Zq from G_saved; its scratch adds four bf16 planes (4 MiB here, limit 8 MiB)
+    cfg = synth.SILU_IP_FWD.replace(B=1, H=4, T=1024, loss="mse")
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=23)
+    inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(23))
+    fwd = run_fwd(cfg, inp)
+    ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
+    got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd)
+    for k in GRADS:
+        assert rel_err(got[k], ref[k]) <= TOL, k
+
+
 def test_noalloc_backward_refuses_configs_beyond_its_scratch():
     big = abi_config(synth.TRAIN_1P45B)  # needs 32 MiB of scratch even with G passed in
     A = 4096  # never dereferenced: the size check comes first

@@ -45,6 +45,7 @@ _p, _i, _u, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_flo
 _cfgp = ctypes.POINTER(ttt_config)
 _SIGS = {
     "ttt_workspace_bytes": ([_cfgp, _i], _sz),
+    "ttt_saved_bytes": ([_cfgp], _sz),
     "ttt_chunk_fwd": ([_cfgp] + [_p] * 11 + [_sz, _p], _i),
     "ttt_chunk_bwd": ([_cfgp] + [_p] * 19 + [_sz, _p], _i),
     "inplace_ttt_workspace_bytes": ([_i] * 4, _sz),
@@ -112,6 +113,14 @@ def make_config(B, H, T, dk, dv, C, dtype="bf16", loss="mse", act="id", lr_bias=
     return ttt_config(B, H, T, dk, dv, C, F32 if dtype in ("f32", F32) else BF16,
                       LOSS.get(loss, loss), ACT.get(act, act), float(lr_bias),
                       DECAY.get(decay, decay))
+
+
+def ttt_saved_bytes(cfg: ttt_config) -> int:
+    """Bytes of the forward's G_saved buffer (G, and Zq with SiLU)."""
+    n = _lib.ttt_saved_bytes(ctypes.byref(cfg))
+    if n == ctypes.c_size_t(-1).value:
+        raise TTTError(ERR_INVALID_ARG, "ttt_saved_bytes")
+    return n
 
 
 def ttt_workspace_bytes(cfg: ttt_config, for_bwd: int) -> int:

@@ -407,6 +407,12 @@ ttt_status inplace_ttt_fwd_docs(int T, int d_ff, int d_model, int C, float lr, c
                           workspace, workspace_bytes, stream);
 }
 
+size_t ttt_saved_bytes(const ttt_config* cfg) {
+  if (check_config(cfg) != TTT_OK) return (size_t)-1;
+  const size_t elem = cfg->dtype == TTT_BF16 ? 2 : 4;
+  return (size_t)cfg->B * cfg->H * cfg->T * cfg->dv * elem * (cfg->act == TTT_ACT_SILU ? 2 : 1);
+}
+
 ttt_status inplace_ttt_delta(int T, int d_ff, int d_model, float lr, const void* Z,
                              const void* Vhat, float* dW, void* workspace, size_t workspace_bytes,
                              void* stream) {
