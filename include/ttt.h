@@ -69,7 +69,7 @@ typedef enum { TTT_DECAY_SCALAR = 0, TTT_DECAY_VECTOR = 1 } ttt_decay;
 /* Shape and variant of one TTT layer call. */
 typedef struct {
   int B, H;        /* batch, heads                                                     */
-  int T;           /* tokens per sequence; T % C == 0                                    */
+  int T;           /* tokens per sequence; T % C == 0; B * H * T < 2^31                   */
   int dk, dv;      /* key/query width and value width of the fast weight (1..128)        */
   int C;           /* chunk size (semantic: gradients inside a chunk are taken at W0)    */
   int dtype;       /* ttt_dtype                                                         */

@@ -54,7 +54,8 @@ def test_workspace_query_validates_config():
     assert 0 < ttt.ttt_workspace_bytes(tc, 2) < ttt.ttt_workspace_bytes(tc, 1)
     with pytest.raises(ttt.TTTError):
         ttt.ttt_workspace_bytes(tc, 3)
-    for bad in (dict(T=250), dict(C=0), dict(B=0), dict(dk=0)):
+    for bad in (dict(T=250), dict(C=0), dict(B=0), dict(dk=0),
+                dict(B=1 << 14, H=1 << 10, T=1 << 7, C=128, dk=1, dv=1)):  # B*H*T = 2^31
         with pytest.raises(ttt.TTTError):
             ttt.ttt_workspace_bytes(_cfg(**bad), False)
     cfg = _cfg()

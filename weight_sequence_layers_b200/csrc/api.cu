@@ -59,6 +59,8 @@ ttt_status check_config(const ttt_config* c) {
   if (c->decay != TTT_DECAY_SCALAR && c->decay != TTT_DECAY_VECTOR) return TTT_ERR_INVALID_ARG;
   if ((long long)c->B * c->H * c->T * (c->dk > c->dv ? c->dk : c->dv) > (1ll << 40))
     return TTT_ERR_INVALID_ARG;
+  // token rows are addressed with 32-bit indices (and TMA coordinates) inside the kernels
+  if ((long long)c->B * c->H * c->T >= (1ll << 31)) return TTT_ERR_INVALID_ARG;
   return TTT_OK;
 }
 
