@@ -77,7 +77,7 @@ struct BwdParams {
 };
 
 struct __align__(8) Bars {
-  uint64_t b[24];
+  uint64_t b[26];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -134,15 +134,17 @@ struct ChainL {
   static constexpr uint32_t BYTES = OFF_BAR + sizeof(Bars);
   static constexpr uint32_t TX_K = KP * K_PANEL, TX_QD = KP * K_PANEL + C * 128;
   // P^T blocks alternate between two TMEM buffers, S^T packed in place (bf16) for the X MMA;
-  // Y reuses buffer 0 after the score loop
+  // Y_0 goes to the spare columns at the top, Y_1 to buffer 1 once X has read S^T_(0,1) there
   static constexpr uint32_t T_DW = 0, T_X = 64, T_P0 = 64 + 64 * NB, T_P1 = T_P0 + 128,
-                            T_Y = T_P0;
+                            T_Y0 = 448;
+  static_assert(T_P1 + 128 <= T_Y0, "TMEM columns");
+  __host__ __device__ static constexpr uint32_t t_y(int b) { return b ? T_P1 : T_Y0; }
   static constexpr int NP = NB * (NB + 1) / 2;
 };
 enum { C_K_FULL, C_K_FREE, C_P_FULL, C_S_READY, C_XB0, C_X_FULL, C_W_READY, C_Y_FULL,
        C_QS_READY, C_DZ_READY, C_DW_FULL, C_SCAN_FULL, C_SCAN_FREE, C_BG_FULL, C_BG_FULL1,
        C_P_FULL1, C_S_READY1, C_QD_FULL, C_QD_FREE, C_ST_READ, C_SCAN_FULL1, C_SCAN_FREE1,
-       C_V_READ, C_F2_READY, C_NBARS };
+       C_V_READ, C_F2_READY, C_XB1, C_NBARS };
 
 template <int D, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool mse = p.loss == 0;
   // arrivals per barrier, in enum order
   const int counts[C_NBARS] = {1, 1, 1, kEpiWarps, 1, 1, kEpiWarps, 1, kEpiWarps, kEpiWarps, 1, 1,
-                               kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1, 1, kEpiWarps, 1, kEpiWarps};
+                               kEpiWarps, 1, 1, 1, kEpiWarps, 1, 1, 1, 1, kEpiWarps, 1, kEpiWarps, 1};
   float* f_bg = reinterpret_cast<float*>(smem + L::OFF_BG);
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmK);
@@ -196,18 +198,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int it = 0; it < NC; ++it) {
         const int c = NC - 1 - it;
         const int row0 = bh * p.T + c * C;
-        // Q and dO are free once dW += Q^T (Gamma dO) is done, K after dW += K^T dZ
+        // K is free once dW += K^T dZ is done, Q and dO after dW += Q^T (Gamma dO)
+        if (it > 0 && !mbar_wait(BAR(C_K_FREE), (it - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(BAR(C_K_FULL), L::TX_K);
+#pragma unroll
+        for (int kp = 0; kp < L::KP; ++kp)
+          tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(C_K_FULL), 64 * kp, row0);
         if (it > 0 && !mbar_wait(BAR(C_QD_FREE), (it - 1) & 1, ab)) break;
         mbar_arrive_expect_tx(BAR(C_QD_FULL), L::TX_QD);
 #pragma unroll
         for (int kp = 0; kp < L::KP; ++kp)
           tma_load_2d(sQ + kp * L::K_PANEL, &tmQ, BAR(C_QD_FULL), 64 * kp, row0);
         tma_load_2d(sDO, &tmDO, BAR(C_QD_FULL), NV * slice, row0);
-        if (it > 0 && !mbar_wait(BAR(C_K_FREE), (it - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(BAR(C_K_FULL), L::TX_K);
+        // the next iteration's tiles into L2 now, so that its loads do not all reach HBM in
+        // the same burst at the end of this iteration
+        if (it + 1 < NC) {
 #pragma unroll
-        for (int kp = 0; kp < L::KP; ++kp)
-          tma_load_2d(sK + kp * L::K_PANEL, &tmK, BAR(C_K_FULL), 64 * kp, row0);
+          for (int kp = 0; kp < L::KP; ++kp) {
+            tma_prefetch_l2_2d(&tmK, 64 * kp, row0 - C);
+            tma_prefetch_l2_2d(&tmQ, 64 * kp, row0 - C);
+          }
+          tma_prefetch_l2_2d(&tmDO, NV * slice, row0 - C);
+        }
         if (it + 1 < NC) {
           // buffer (it + 1) & 1 was last read by the scan of iteration it - 1
           if (it > 0 && !mbar_wait(BAR((it - 1) & 1 ? C_SCAN_FULL1 : C_SCAN_FULL), ((it - 1) >> 1) & 1, ab))
@@ -243,8 +255,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the previous one, so its barrier is never more than one phase ahead of the waiter
           mma_commit(BAR((k & 1) ? C_P_FULL1 : C_P_FULL));
         };
+        // Y_b = K_b dW (dW: the adjoint copy written at the end of the previous iteration)
+        auto issue_y = [&](int b) {
+#pragma unroll
+          for (int j = 0; j < D / 16; ++j)
+            mma_bf16_ss(tmem + L::t_y(b),
+                        sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16, 1024),
+                        sdesc_sw128(sDW + j * 2048, 0, 1024), idX, j > 0);
+        };
         issue_p(0);
         if (L::NP > 1) issue_p(1);
+        if (!mbar_wait(BAR(C_W_READY), it & 1, ab)) break;
+        tc_fence_after();
+        issue_y(0);
+        if (NB == 1) mma_commit(BAR(C_Y_FULL));
         for (int k = 0; k < L::NP; ++k) {
           const int rb = k < NB ? 0 : 1, sb = k < NB ? k : 1;
           const int x = k & 1;
@@ -262,6 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(BAR(C_XB0));
             ++xb0;
           }
+          if (NB == 2 && k == 1) {
+            // Y_1 into buffer 1 once the X MMA has read S^T_(0,1) from it
+            mma_commit(BAR(C_XB1));
+            if (!mbar_wait(BAR(C_XB1), it & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+            issue_y(1);
+            mma_commit(BAR(C_Y_FULL));
+          }
           if (k + 2 < L::NP) {
             if (!mbar_wait(BAR(C_XB0), (xb0 - 1) & 1, ab)) { ok = false; break; }
             issue_p(k + 2);
@@ -269,24 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         mma_commit(BAR(C_X_FULL));
-        // Y_b = K_b dW into buffer 0, once the X MMA that read the last S^T there is done
-        if (!mbar_wait(BAR(C_XB0), (xb0 - 1) & 1, ab)) break;
-        if (!mbar_wait(BAR(C_W_READY), it & 1, ab)) break;
-        tc_fence_after();
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-          for (int j = 0; j < D / 16; ++j)
-            mma_bf16_ss(tmem + L::T_Y + NV * b,
-                        sdesc_sw128(sK + (j / 4) * L::K_PANEL + b * PANEL128 + (j % 4) * 32, 16, 1024),
-                        sdesc_sw128(sDW + j * 2048, 0, 1024), idX, j > 0);
-        mma_commit(BAR(C_Y_FULL));
-        // dW (already Gamma_C-scaled) += Q^T (Gamma dO) + K^T dZ, dZ = -dV (negated A)
-        if (!mbar_wait(BAR(C_QS_READY), it & 1, ab)) break;
-        tc_fence_after();
-        for (int j = 0; j < C / 16; ++j)
-          mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sQ + j * 2048, lboT, 1024),
-                      sdesc_sw128(sDO + j * 2048, 0, 1024), idW, 1);
-        mma_commit(BAR(C_QD_FREE));
+        // dW (scaled by Gamma_C in the dV step) += K^T dZ + Q^T (Gamma dO); dZ first, so that K
+        // is released for the next iteration's load as early as possible.
         // -dZ: -dV for MSE with the identity, -dG * F2 once the epilogue has scaled it (SiLU)
         if (!mbar_wait(BAR(p.silu ? C_F2_READY : C_DZ_READY), it & 1, ab)) break;
         tc_fence_after();
@@ -294,8 +310,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < C / 16; ++j)
             mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sK + j * 2048, lboT, 1024),
                         sdesc_sw128(sS + j * 2048, 0, 1024), idWn, 1);
-        mma_commit(BAR(C_DW_FULL));
         mma_commit(BAR(C_K_FREE));
+        if (!mbar_wait(BAR(C_QS_READY), it & 1, ab)) break;
+        tc_fence_after();
+        for (int j = 0; j < C / 16; ++j)
+          mma_bf16_ss(tmem + L::T_DW, sdesc_sw128(sQ + j * 2048, lboT, 1024),
+                      sdesc_sw128(sDO + j * 2048, 0, 1024), idW, 1);
+        mma_commit(BAR(C_QD_FREE));
+        mma_commit(BAR(C_DW_FULL));
       }
     }
   } else if (warp == 10) {
@@ -363,24 +385,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(BAR(x ? C_S_READY1 : C_S_READY));
       }
       if (!ok) break;
-      // ---- scale dO rows by Gamma_s (X, the only other reader of dO, is done) and the state
-      // by Gamma_C
-      if (!mbar_wait(BAR(C_X_FULL), it & 1, ab)) { ok = false; break; }
-      for (int s = ew * 32 + lane; s < C; s += kEpiWarps * 32) {
-        const float gs = f_gam[s];
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint32_t a = sDO + sw128_off(s, ch);
-          uint32_t w0, w1, w2, w3;
-          ld_shared_v4(a, w0, w1, w2, w3);
-          st_shared_v4(a, pack_bf16x2(bf16lo(w0) * gs, bf16hi(w0) * gs),
-                       pack_bf16x2(bf16lo(w1) * gs, bf16hi(w1) * gs),
-                       pack_bf16x2(bf16lo(w2) * gs, bf16hi(w2) * gs),
-                       pack_bf16x2(bf16lo(w3) * gs, bf16hi(w3) * gs));
-        }
+      // ---- dV = -dG = X + u Y into shared memory (the MMA reads it as -dZ for MSE), then one
+      // bulk store per 128-row block, once the previous chunk's stores have read the buffers;
+      // the state is decayed by Gamma_C here, before K^T dZ accumulates into it
+      if (!mbar_wait(BAR(C_X_FULL), it & 1, ab) || !mbar_wait(BAR(C_Y_FULL), it & 1, ab) ||
+          (it > 0 && !mbar_wait(BAR(C_ST_READ), (it - 1) & 1, ab))) {
+        ok = false;
+        break;
       }
       __syncwarp();
       tc_fence_after();
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const int r = 128 * b + lrow;
+        float x[32], y[32];
+        tmem_ld32(tmem + loff + L::T_X + NV * b + 32 * g, x);
+        tmem_ld32(tmem + loff + L::t_y(b) + 32 * g, y);
+        tmem_wait_ld();
+        const float u = f_eta[r] * f_eLC[r];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) x[j] += u * y[j];
+        st_row32(sS, r, 4 * g, x);
+      }
       if (w_rows) {
         float w[32];
         tmem_ld32(tmem + loff + L::T_DW + 32 * g, w);
@@ -390,25 +416,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 32; ++j) w[j] *= gC;
         tmem_st32(tmem + loff + L::T_DW + 32 * g, w);
         tmem_wait_st();
-      }
-      epi_arrive(BAR(C_QS_READY));
-      // ---- dV = -dG = X + u Y into shared memory (the MMA reads it as -dZ for MSE), then one
-      // bulk store per 128-row block, once the previous chunk's stores have read the buffers
-      if (!mbar_wait(BAR(C_Y_FULL), it & 1, ab)) { ok = false; break; }
-      if (it > 0 && !mbar_wait(BAR(C_ST_READ), (it - 1) & 1, ab)) { ok = false; break; }
-      __syncwarp();
-      tc_fence_after();
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const int r = 128 * b + lrow;
-        float x[32], y[32];
-        tmem_ld32(tmem + loff + L::T_X + NV * b + 32 * g, x);
-        tmem_ld32(tmem + loff + L::T_Y + NV * b + 32 * g, y);
-        tmem_wait_ld();
-        const float u = f_eta[r] * f_eLC[r];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) x[j] += u * y[j];
-        st_row32(sS, r, 4 * g, x);
       }
       epi_arrive(BAR(C_DZ_READY));
       if (ew == 0) {
@@ -458,6 +465,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         epi_arrive(BAR(C_F2_READY));
       }
+      // ---- dO rows scaled by Gamma_s for Q^T (Gamma dO); the X MMAs, its other readers, are done
+      for (int s = ew * 32 + lane; s < C; s += kEpiWarps * 32) {
+        const float gs = f_gam[s];
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t a = sDO + sw128_off(s, ch);
+          uint32_t w0, w1, w2, w3;
+          ld_shared_v4(a, w0, w1, w2, w3);
+          st_shared_v4(a, pack_bf16x2(bf16lo(w0) * gs, bf16hi(w0) * gs),
+                       pack_bf16x2(bf16lo(w1) * gs, bf16hi(w1) * gs),
+                       pack_bf16x2(bf16lo(w2) * gs, bf16hi(w2) * gs),
+                       pack_bf16x2(bf16lo(w3) * gs, bf16hi(w3) * gs));
+        }
+      }
+      epi_arrive(BAR(C_QS_READY));
       // ---- adjoint at the end of chunk c-1 (or dW0)
       if (!mbar_wait(BAR(C_DW_FULL), it & 1, ab)) { ok = false; break; }
       __syncwarp();

@@ -83,7 +83,7 @@ struct Layout {
 struct __align__(8) FwdBars {
   uint64_t k_full[2], k_free[2], q_full[2], q_free[2], v_full[2], z_full, g_ready, y_full[2],
       y_scaled[2], p_full[2], s_ready[2], s_done[2], zq_full[2], y_free[2], w_full, w0_ready,
-      g_done, scan_full[2], scan_free[2], bg_full[2], st_free, g_read[2];
+      g_done, scan_full[2], scan_free[2], bg_full[2], st_free, g_read[2], z_issued, t_issued;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(BAR(w0_ready), kEpiWarps);
     mbar_init(BAR(g_done), 1);
     mbar_init(BAR(st_free), 1);
+    mbar_init(BAR(z_issued), 1);
+    mbar_init(BAR(t_issued), 1);
     bars->abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
@@ -228,6 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sdesc_sw128(sW0 + j * 2048, 0, 1024), idZ, j > 0);
         }
         mma_commit(BAR(z_full));
+        // the query side issues this chunk's Y only now, so Z is first in the tensor pipe
+        mbar_arrive(BAR(z_issued));
         if (!mbar_wait(BAR(g_ready), c & 1, ab)) break;
         tc_fence_after();
         // W += K^T (u * -G), W already scaled by Gamma_C
@@ -236,6 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       sdesc_sw128(sUG + j * 2048, 0, 1024), idW, 1);
         mma_commit(BAR(w_full));
         for (int b = 0; b < NB; ++b) mma_commit(BAR(k_free[b]));
+        mbar_arrive(BAR(t_issued));
       }
     }
   } else if (warp == 11) {
@@ -281,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int c = 0; c < NC; ++c) {
         const uint32_t sG = sVG + (c & 1) * C * 128;
-        // Y_h = Q_h W0 with this chunk's bf16 state copy
-        bool ok = mbar_wait(BAR(w0_ready), c & 1, ab);
+        // Y_h = Q_h W0 with this chunk's bf16 state copy, behind Z in the tensor pipe
+        bool ok = mbar_wait(BAR(w0_ready), c & 1, ab) && mbar_wait(BAR(z_issued), c & 1, ab);
         for (int h = 0; h < NB && ok; ++h) {
           ok = mbar_wait(BAR(q_full[h]), c & 1, ab) &&
                (c == 0 || mbar_wait(BAR(y_free[h]), (c - 1) & 1, ab));
@@ -302,7 +307,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(BAR(zq_full[0]));
         } else {
           issue_p(1, 0, 0);                                    // (1,0) -> A
-          if (!mbar_wait(BAR(g_ready), c & 1, ab)) break;      // Z columns free of Z
+          // the Z columns are free once G is formed; waiting for the transition's issue as
+          // well keeps the state chain ahead of this block in the tensor pipe
+          if (!mbar_wait(BAR(t_issued), c & 1, ab)) break;
           tc_fence_after();
           issue_p(0, 0, 1);                                    // (0,0) -> B
           mma_commit(BAR(q_free[0]));
@@ -444,6 +451,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { ok = false; break; }
       }
 
+      // -------- Y_h *= Gamma_s for both query halves (while the transition MMA runs)
+      for (int h = 0; h < NB; ++h) {
+        if (!mbar_wait(BAR(y_full[h]), c & 1, ab)) { ok = false; break; }
+        __syncwarp();
+        tc_fence_after();
+        float y[32];
+        tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
+        tmem_wait_ld();
+        const float gs = f_gam[128 * h + lrow];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] *= gs;
+        tmem_st32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(y_scaled[h]));
+      }
+      if (!ok) break;
       // -------- state copy for the next chunk: after the transition MMA and after the last MMA
       // that reads the current bf16 copy (Y of the last query half). The fp32 state goes back
       // into TMEM already decayed by the next chunk's Gamma_C.
@@ -491,24 +516,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // -------- Y_h *= Gamma_s for both query halves
-      for (int h = 0; h < NB; ++h) {
-        if (!mbar_wait(BAR(y_full[h]), c & 1, ab)) { ok = false; break; }
-        __syncwarp();
-        tc_fence_after();
-        float y[32];
-        tmem_ld32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
-        tmem_wait_ld();
-        const float gs = f_gam[128 * h + lrow];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) y[j] *= gs;
-        tmem_st32(tmem + lane_off + L::T_Y + NV * h + 32 * g, y);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(y_scaled[h]));
-      }
-      if (!ok) break;
       // -------- score blocks S = -(Q K^T) * weights, bf16 in place, in the order the query-side
       // issuer produces them: (1,0) in A, (0,0) in B, (1,1) in A; or (0,0) in A
       for (int k = 0; k < (NB == 2 ? 3 : 1); ++k) {
