@@ -40,6 +40,14 @@
 namespace tttk {
 namespace {
 
+// Prefetch of one box of a 2-D tensor map into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
 constexpr int NV = 64;
 constexpr int kThreads = 352;  // chain: producer, MMA, 8 epilogue warps, scan warp
 constexpr int kEpiWarps = 8;
