@@ -181,10 +181,13 @@ class Layer:
         self.nb = ttt.ttt_workspace_bytes(self.c, 2)
         self.ws = torch.empty(max(self.nf, self.nb, 16), device=dev, dtype=torch.uint8)
 
-    def fwd(self):
+    def fwd(self, save=True):
+        """save=False is the inference forward (O and W_final only); a training step saves the
+        chunk-start states and G (and Zq with SiLU) for the backward."""
         i = self.inp
         self.ttt.ttt_chunk_fwd(self.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
-                               self.O, self.Wf, self.Wc, self.G, self.ws, self.nf)
+                               self.O, self.Wf, self.Wc if save else None,
+                               self.G if save else None, self.ws, self.nf)
 
     def bwd(self, dgamma=None):
         i = self.inp
@@ -236,7 +239,12 @@ def time_other_configs(ttt, peaks):
         w = layer_work(cfg)
         steps, warmup = (3, 1) if with_bwd else (10, 3)
         entry = {"dtype": cfg.dtype, "decay": "vector" if cfg.decay == "vector" else "scalar"}
-        calls = [("ttt_chunk_fwd", layer.fwd, w["fwd_flops"], w["fwd_bytes"])]
+        # a forward-only workload is timed as inference (nothing saved for a backward); the
+        # forward that saves the backward's inputs is reported beside it
+        calls = [("ttt_chunk_fwd", layer.fwd if with_bwd else (lambda: layer.fwd(save=False)),
+                  w["fwd_flops"], w["fwd_bytes"])]
+        if not with_bwd:
+            entry["ttt_chunk_fwd_saving_for_bwd_ms"] = _event_ms(layer.fwd, steps, warmup)
         if with_bwd:
             layer.fwd()
             calls.append(("ttt_chunk_bwd", layer.bwd, w["bwd_flops"], w["bwd_bytes"]))

@@ -21,13 +21,15 @@ def gpu_inputs(cfg, seed=None):
     return synth.ttt_inputs(cfg, device="cuda", seed=seed)
 
 
-def run_fwd(cfg, inp, save_g=True):
+def run_fwd(cfg, inp, save_g=True, save_w=True):
+    """The forward through the C ABI; save_w / save_g request the chunk-start states and G (with
+    SiLU also Zq) that a backward reads. With both off it is the inference forward."""
     c = abi_config(cfg)
     sd = synth.storage_dtype(cfg)
     B, H, T, dk, dv, C = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C
     O = torch.empty((B, H, T, dv), device="cuda", dtype=sd)
     Wf = torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32)
-    Wc = torch.empty((B, H, T // C, dk, dv), device="cuda", dtype=sd)
+    Wc = torch.empty((B, H, T // C, dk, dv), device="cuda", dtype=sd) if save_w else None
     # with SiLU the saved buffer holds G, then Zq (the readout before the activation)
     planes = 2 if cfg.act == "silu" else 1
     Gs = torch.empty((planes, B, H, T, dv), device="cuda", dtype=sd) if save_g else None

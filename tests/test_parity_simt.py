@@ -20,6 +20,10 @@ def test_tiny_fp32_workload_forward():
     ref = oracle_fwd(cfg, inp)
     for k in ("O", "W_final", "W_chunks"):
         assert rel_err(got[k], ref[k]) <= F32_TOL, k
+    # the inference forward (no chunk states, no G kept for a backward)
+    got = run_fwd(cfg, inp, save_g=False, save_w=False)
+    for k in ("O", "W_final"):
+        assert rel_err(got[k], ref[k]) <= F32_TOL, k
 
 
 SHAPES = [

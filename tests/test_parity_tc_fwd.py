@@ -61,3 +61,16 @@ def test_tc_forward_full_size_sampled_heads(cfg):
     for k in ("O", "W_final", "W_chunks", "G"):
         g = torch.stack([got[k][b, h] for b, h in heads]).unsqueeze(0)
         assert rel_err(g, ref[k]) <= TOL, (k, rel_err(g, ref[k]))
+
+
+@pytest.mark.parametrize("d,C,loss,act", [(64, 256, "mse", "id"), (128, 256, "ip", "silu"),
+                                          (128, 128, "mse", "silu"), (64, 128, "ip", "id")])
+def test_tc_inference_forward_without_saved_tensors(d, C, loss, act):
+    # the forward with no W_chunks and no G_saved (nothing kept for a backward) gives the same
+    # O and W_final as the oracle
+    cfg = synth.SILU_IP_FWD.replace(B=1, H=2, T=4 * C, dk=d, dv=d, C=C, loss=loss, act=act)
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=d + C)
+    got = run_fwd(cfg, inp, save_g=False, save_w=False)
+    ref = oracle_fwd(cfg, inp)
+    for k in ("O", "W_final"):
+        assert rel_err(got[k], ref[k]) <= TOL, k
