@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
   float* S = G + C * kNvs;           // [kRows][C]
   float* eta = S + kRows * C;        // [C]
   float* L = eta + C;                // [C] or [C][dk]
+  float* X = L + C * lwidth(d);      // [C + dk]: per-key factors of the transition
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
   for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
     const int i = e / nv, j = e % nv;
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
           float p = 0.f;
           if (d.gvec) {
             for (int i = 0; i < dk; ++i)
-              p += ldf(qs + i) * ldf(kr + i) * expf(L[s * dk + i] - L[r * dk + i]);
+              p += ldf(qs + i) * ldf(kr + i) * __expf(L[s * dk + i] - L[r * dk + i]);
             v = eta[r] * p;
           } else {
             for (int i = 0; i < dk; ++i) p += ldf(qs + i) * ldf(kr + i);
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
         const TI* qs = Q + qk0 + (tc + s) * dk;
         float acc = 0.f;
         if (d.gvec) {
-          for (int i = 0; i < dk; ++i) acc += ldf(qs + i) * expf(L[s * dk + i]) * Ws[i * kNvs + j];
+          for (int i = 0; i < dk; ++i) acc += ldf(qs + i) * __expf(L[s * dk + i]) * Ws[i * kNvs + j];
         } else {
           for (int i = 0; i < dk; ++i) acc += ldf(qs + i) * Ws[i * kNvs + j];
           acc *= expf(L[s]);
@@ -136,14 +137,28 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
       }
       __syncthreads();
     }
-    // state transition
+    // state transition; first the decayed, lr-weighted keys eta_r exp(L_C - L_r) k_r, one
+    // exponential per key (and feature): into X for a scalar decay, over L (no longer needed in
+    // this chunk) for a per-feature decay, with L_C kept in X
+    if (d.gvec) {
+      for (int i = threadIdx.x; i < dk; i += blockDim.x) X[i] = L[(C - 1) * dk + i];
+      __syncthreads();
+      for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+        const int r = e / dk, i = e % dk;
+        L[e] = eta[r] * expf(X[i] - L[e]) * ldf(K + qk0 + (tc + r) * dk + i);
+      }
+    } else {
+      for (int r = threadIdx.x; r < C; r += blockDim.x) X[r] = eta[r] * expf(L[C - 1] - L[r]);
+      if (threadIdx.x == 0) X[C] = L[C - 1];
+    }
+    __syncthreads();
     for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
       const int i = e / nv, j = e % nv;
-      const float LC = Lat(d, L, C - 1, i);
-      float w = expf(LC) * Ws[i * kNvs + j];
-      for (int r = 0; r < C; ++r)
-        w -= eta[r] * expf(LC - Lat(d, L, r, i)) * ldf(K + qk0 + (tc + r) * dk + i) *
-             G[r * kNvs + j];
+      float w = expf(d.gvec ? X[i] : X[C]) * Ws[i * kNvs + j];
+      if (d.gvec)
+        for (int r = 0; r < C; ++r) w -= L[r * dk + i] * G[r * kNvs + j];
+      else
+        for (int r = 0; r < C; ++r) w -= X[r] * ldf(K + qk0 + (tc + r) * dk + i) * G[r * kNvs + j];
       Ws[i * kNvs + j] = w;
     }
     __syncthreads();
@@ -156,12 +171,13 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
 }
 
 // Per-head float32 scratch of the backward (in units of floats): Wh, Wn, W0 (dk x dv each),
-// Z, G, dZq, Y, dG, dZ, Zq (C x dv each), S, dS (C x C each), eta, L, deta, dL (C each), and
-// one float for the chunk-end term of the decay gradient; with a per-feature decay also the
-// prefix L and two parts of dJ/dL (C x dk each) and the chunk-end term per feature (dk).
+// Z, G, dZq, Y, dG, dZ, Zq (C x dv each), S, dS (C x C each), eta, L, deta, dL (C each), one
+// float for the chunk-end term of the decay gradient, and the decay-scaled operands
+// q_s exp(L_s) and k_r exp(L_C - L_r) (C x dk each); with a per-feature decay also the prefix L
+// and two parts of dJ/dL (C x dk each) and the chunk-end term per feature (dk).
 __host__ __device__ inline size_t bwd_head_floats(int C, int dk, int dv, bool gvec) {
   return 3 * (size_t)dk * dv + 7 * (size_t)C * dv + 2 * (size_t)C * C + 4 * (size_t)C + 1 +
-         (gvec ? 3 * (size_t)C * dk + dk : 0);
+         2 * (size_t)C * dk + (gvec ? 3 * (size_t)C * dk + dk : 0);
 }
 
 // Analytic backward of the chunk dual form, reverse over chunks; one block per head.
@@ -190,7 +206,9 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
   float* ZQ = deta + C;
   float* dL = ZQ + C * dv;
   float* wend = dL + C;  // <W_end, dW_end> of the chunk
-  float* dLq = wend + 1;       // per-feature decay: q_si dQ_si  [C][dk]
+  float* QG = wend + 1;        // q_s exp(L_s)  [C][dk]
+  float* KC = QG + C * dk;     // k_r exp(L_C - L_r)  [C][dk]
+  float* dLq = KC + C * dk;    // per-feature decay: q_si dQ_si  [C][dk]
   float* dLk = dLq + C * dk;   //                    -k_si (dK_si - (dZ_s W0^T)_i)  [C][dk]
   float* wendv = dLk + C * dk; //                    row sums of W_end * dW_end  [dk]
   if (d.gvec) L = wendv + dk;  //                    log-decay prefix  [C][dk]
@@ -203,6 +221,15 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
     for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
       W0[e] = ldf(Wc + ((size_t)bh * NC + c) * dk * dv + e);
     chunk_scans(d, beta, gamma, bh, c, eta, L);  // ends with __syncthreads
+    // the decay-scaled operands of the readout, the chunk-end route of the keys and the dW
+    // update, one exponential per token and feature
+    for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+      const int s = e / dk, i = e % dk;
+      const float Ls = Lat(d, L, s, i);
+      QG[e] = ldf(Q + qk0 + (tc + s) * dk + i) * expf(Ls);
+      KC[e] = ldf(K + qk0 + (tc + s) * dk + i) * expf(Lat(d, L, C - 1, i) - Ls);
+    }
+    __syncthreads();
     // Z = K W0, G
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
       const int s = e / dv, j = e % dv;
@@ -219,9 +246,13 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       float v = 0.f;
       if (r <= s) {
         float p = 0.f;
-        for (int i = 0; i < dk; ++i)
-          p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i) *
-               (d.gvec ? expf(L[s * dk + i] - L[r * dk + i]) : 1.f);
+        if (d.gvec)
+          for (int i = 0; i < dk; ++i)
+            p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i) *
+                 __expf(L[s * dk + i] - L[r * dk + i]);
+        else
+          for (int i = 0; i < dk; ++i)
+            p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i);
         v = eta[r] * p * (d.gvec ? 1.f : expf(L[s] - L[r]));
       }
       S[e] = v;
@@ -230,19 +261,15 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
       const int r = e / dv, j = e % dv;
       float y = 0.f;
-      for (int i = 0; i < dk; ++i)
-        y += ldf(K + qk0 + (tc + r) * dk + i) * Wh[i * dv + j] *
-             (d.gvec ? expf(Lat(d, L, C - 1, i) - L[r * dk + i]) : 1.f);
-      Y[e] = d.gvec ? y : y * expf(L[C - 1] - L[r]);
+      for (int i = 0; i < dk; ++i) y += KC[r * dk + i] * Wh[i * dv + j];
+      Y[e] = y;
     }
     __syncthreads();
     // dZq = dO * act'(Zq), Zq = Gamma Q W0 - S G
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
       const int s = e / dv, j = e % dv;
-      float y = 0.f;
-      for (int i = 0; i < dk; ++i)
-        y += ldf(Q + qk0 + (tc + s) * dk + i) * W0[i * dv + j] * (d.gvec ? expf(L[s * dk + i]) : 1.f);
-      float zq = d.gvec ? y : expf(L[s]) * y;
+      float zq = 0.f;
+      for (int i = 0; i < dk; ++i) zq += QG[s * dk + i] * W0[i * dv + j];
       for (int r = 0; r <= s; ++r) zq -= S[s * C + r] * G[r * dv + j];
       ZQ[e] = zq;
       DZQ[e] = ldf(dO + v0 + (tc + s) * dv + j) * act1(d.act, zq);
@@ -284,6 +311,13 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       stf(&dV[v0 + (tc + r) * dv + j], -da);
     }
     __syncthreads();
+    // dS * eta_r (and exp(L_s - L_r) with a scalar decay) in place: the causal weights of the
+    // dQ and dK contractions; deta, the last reader of dS itself, is done
+    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
+      const int s = e / C, r = e % C;
+      if (r <= s) DS[e] *= eta[r] * (d.gvec ? 1.f : expf(L[s] - L[r]));
+    }
+    __syncthreads();
     // dQ = diag(Gamma) dZq W0^T + (dS * M) K   (decay of feature i inside, per feature)
     for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
       const int s = e / dk, i = e % dk;
@@ -291,8 +325,11 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       float a1 = 0.f;
       for (int j = 0; j < dv; ++j) a1 += DZQ[s * dv + j] * W0[i * dv + j];
       float acc = expf(Ls) * a1;
-      for (int r = 0; r <= s; ++r)
-        acc += DS[s * C + r] * eta[r] * expf(Ls - Lat(d, L, r, i)) * ldf(K + qk0 + (tc + r) * dk + i);
+      if (d.gvec)
+        for (int r = 0; r <= s; ++r)
+          acc += DS[s * C + r] * __expf(Ls - L[r * dk + i]) * ldf(K + qk0 + (tc + r) * dk + i);
+      else
+        for (int r = 0; r <= s; ++r) acc += DS[s * C + r] * ldf(K + qk0 + (tc + r) * dk + i);
       stf(&dQ[qk0 + (tc + s) * dk + i], acc);
       if (d.gvec && dgamma) dLq[e] = ldf(Q + qk0 + (tc + s) * dk + i) * acc;
     }
@@ -301,8 +338,11 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       const int r = e / dk, i = e % dk;
       const float Lr = Lat(d, L, r, i);
       float acc = 0.f;
-      for (int s = r; s < C; ++s)
-        acc += DS[s * C + r] * eta[r] * expf(Lat(d, L, s, i) - Lr) * ldf(Q + qk0 + (tc + s) * dk + i);
+      if (d.gvec)
+        for (int s = r; s < C; ++s)
+          acc += DS[s * C + r] * __expf(L[s * dk + i] - Lr) * ldf(Q + qk0 + (tc + s) * dk + i);
+      else
+        for (int s = r; s < C; ++s) acc += DS[s * C + r] * ldf(Q + qk0 + (tc + s) * dk + i);
       float gw = 0.f, zw = 0.f;
       for (int j = 0; j < dv; ++j) {
         gw += G[r * dv + j] * Wh[i * dv + j];
@@ -370,8 +410,7 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       const int i = e / dv, j = e % dv;
       float acc = expf(Lat(d, L, C - 1, i)) * Wh[e];
       for (int s = 0; s < C; ++s)
-        acc += expf(Lat(d, L, s, i)) * ldf(Q + qk0 + (tc + s) * dk + i) * DZQ[s * dv + j] +
-               ldf(K + qk0 + (tc + s) * dk + i) * DZ[s * dv + j];
+        acc += QG[s * dk + i] * DZQ[s * dv + j] + ldf(K + qk0 + (tc + s) * dk + i) * DZ[s * dv + j];
       Wn[e] = acc;
     }
     __syncthreads();
@@ -390,8 +429,8 @@ size_t zq_plane(const LayerArgs& a) { return (size_t)a.B * a.H * a.T * a.dv; }
 
 size_t fwd_smem_bytes(const LayerArgs& a) {
   const size_t lw = a.gvec ? a.dk : 1;
-  return sizeof(float) *
-         ((size_t)a.dk * kNvs + (size_t)a.C * kNvs + (size_t)kRows * a.C + a.C + a.C * lw);
+  return sizeof(float) * ((size_t)a.dk * kNvs + (size_t)a.C * kNvs + (size_t)kRows * a.C + a.C +
+                           a.C * lw + a.C + 1 + a.dk);
 }
 
 }  // namespace
