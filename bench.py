@@ -237,7 +237,7 @@ def time_other_configs(ttt, peaks):
     for name, cfg, with_bwd in work:
         layer = Layer(cfg, ttt, seed=cfg.seed)
         w = layer_work(cfg)
-        steps, warmup = (3, 1) if with_bwd else (10, 3)
+        steps, warmup = (3, 3) if with_bwd else (10, 3)
         entry = {"dtype": cfg.dtype, "decay": "vector" if cfg.decay == "vector" else "scalar"}
         # a forward-only workload is timed as inference (nothing saved for a backward); the
         # forward that saves the backward's inputs is reported beside it
@@ -312,7 +312,7 @@ def time_mlp(ttt, peaks):
     return out
 
 
-def time_bwd_dgamma(layer, steps=5, warmup=2):
+def time_bwd_dgamma(layer, steps=5, warmup=3):
     """Device time of the backward that also returns the decay gradient (a separate line: the
     workload's gradients do not include it)."""
     if layer.inp["gamma"] is None:
@@ -643,7 +643,7 @@ def main():
     if not args.no_configs:
         out["other_configs"] = time_other_configs(ttt, peaks)
     if not args.no_inplace:
-        icfg, ims, ims_save, ims_bwd, (ims_tgt, ims_tgt_bwd) = time_inplace(ttt, steps=3, warmup=1)
+        icfg, ims, ims_save, ims_bwd, (ims_tgt, ims_tgt_bwd) = time_inplace(ttt, steps=3, warmup=3)
         fl, by = inplace_work(icfg)
         tf = fl / (ims * 1e-3) / 1e12
         out["inplace"] = {"workload": icfg.name, "ms": ims, "tokens_per_s": icfg.T / (ims * 1e-3),
