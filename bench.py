@@ -296,8 +296,8 @@ def time_mlp(ttt, peaks):
                                   w["W1"], w["W2"], O, W1f, W2f, W1c, W2c, ws, n)
     bwd = lambda: ttt.ttt_mlp_bwd(c, hid, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"],
                                   W1c, W2c, inp["dO"], None, None, *g, ws, n)
-    ms_f = _event_ms(fwd, 2, 1)
-    ms_b = _event_ms(bwd, 2, 1)
+    ms_f = _event_ms(fwd, 2, 3)
+    ms_b = _event_ms(bwd, 2, 3)
     units = B * H * (T // C)
     fl_f = units * (2 * C * (3 * dk * hid + 3 * hid * dv) + C * (C + 1) * (dk + dv + 2 * hid))
     tc = peaks["bf16_tflops"] * 1e12

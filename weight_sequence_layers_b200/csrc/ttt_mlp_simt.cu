@@ -89,15 +89,21 @@ __device__ void mlp_chunk_forward(const MlpDims& d, const MlpScratch& S, const T
     const float v = ldf(Vh + (size_t)s * dv + j);
     S.G2[e] = d.loss == 0 ? vh - v : -v;
   }
-  for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-    const int s = e / C, r = e % C;
-    float v = 0.f;
-    if (r <= s) {
-      float p = 0.f;
-      for (int k = 0; k < dk; ++k) p += ldf(Qh + (size_t)s * dk + k) * ldf(Kh + (size_t)r * dk + k);
-      v = S.eta[r] * expf(S.L[s] - S.L[r]) * p;
-    }
-    S.S1[e] = v;
+  // S1: a warp per query row, its lanes over the key features (dk <= 128)
+  for (int s = threadIdx.x >> 5; s < C; s += blockDim.x >> 5) {
+    const int lane = threadIdx.x & 31;
+    warp_row_dots<0>(
+        (dk + 31) / 32, s + 1,
+        [&](int m) {
+          const int k = lane + 32 * m;
+          return k < dk ? ldf(Qh + (size_t)s * dk + k) : 0.f;
+        },
+        [&](int r, int m) {
+          const int k = lane + 32 * m;
+          return k < dk ? ldf(Kh + (size_t)r * dk + k) : 0.f;
+        },
+        [&](int r, float p) { S.S1[s * C + r] = S.eta[r] * expf(S.L[s] - S.L[r]) * p; });
+    for (int r = s + 1 + lane; r < C; r += 32) S.S1[s * C + r] = 0.f;
   }
   __syncthreads();
   for (int e = threadIdx.x; e < C * h; e += blockDim.x) {
@@ -118,15 +124,21 @@ __device__ void mlp_chunk_forward(const MlpDims& d, const MlpScratch& S, const T
     S.Aq[e] = actf(d.act, zq);
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-    const int s = e / C, r = e % C;
-    float v = 0.f;
-    if (r <= s) {
-      float p = 0.f;
-      for (int i = 0; i < h; ++i) p += S.Aq[s * h + i] * S.A1[r * h + i];
-      v = S.eta[r] * expf(S.L[s] - S.L[r]) * p;
-    }
-    S.S2[e] = v;
+  // S2: a warp per query row, its lanes over the hidden features (h <= 512)
+  for (int s = threadIdx.x >> 5; s < C; s += blockDim.x >> 5) {
+    const int lane = threadIdx.x & 31;
+    warp_row_dots<0>(
+        (h + 31) / 32, s + 1,
+        [&](int m) {
+          const int i = lane + 32 * m;
+          return i < h ? S.Aq[s * h + i] : 0.f;
+        },
+        [&](int r, int m) {
+          const int i = lane + 32 * m;
+          return i < h ? S.A1[r * h + i] : 0.f;
+        },
+        [&](int r, float p) { S.S2[s * C + r] = S.eta[r] * expf(S.L[s] - S.L[r]) * p; });
+    for (int r = s + 1 + lane; r < C; r += 32) S.S2[s * C + r] = 0.f;
   }
   __syncthreads();
 }
@@ -223,13 +235,21 @@ __global__ void __launch_bounds__(512)
       for (int i = 0; i < h; ++i) y += S.A1[r * h + i] * S.Wh2[i * dv + j];
       S.Ya[e] = y;
     }
-    // output layer: dS2 = -dO G2^T (causal)
-    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-      const int s = e / C, r = e % C;
-      float v = 0.f;
-      if (r <= s)
-        for (int j = 0; j < dv; ++j) v -= ldf(dOh + (size_t)s * dv + j) * S.G2[r * dv + j];
-      S.dS2[e] = v;
+    // output layer: dS2 = -dO G2^T (causal), a warp per row, its lanes over the value features
+    for (int s = threadIdx.x >> 5; s < C; s += blockDim.x >> 5) {
+      const int lane = threadIdx.x & 31;
+      warp_row_dots<0>(
+          (dv + 31) / 32, s + 1,
+          [&](int m) {
+            const int j = lane + 32 * m;
+            return j < dv ? ldf(dOh + (size_t)s * dv + j) : 0.f;
+          },
+          [&](int r, int m) {
+            const int j = lane + 32 * m;
+            return j < dv ? S.G2[r * dv + j] : 0.f;
+          },
+          [&](int r, float p) { S.dS2[s * C + r] = -p; });
+      for (int r = s + 1 + lane; r < C; r += 32) S.dS2[s * C + r] = 0.f;
     }
     __syncthreads();
     // dG2 (readout and transition parts), dAq -> dZq, dA1 (score and transition parts)
@@ -258,13 +278,21 @@ __global__ void __launch_bounds__(512)
       S.dA1[e] = a - S.eta[r] * expf(LC - S.L[r]) * gw;
     }
     __syncthreads();
-    // first layer: dS1 = -dZq G1^T (causal)
-    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-      const int s = e / C, r = e % C;
-      float v = 0.f;
-      if (r <= s)
-        for (int i = 0; i < h; ++i) v -= S.dZq[s * h + i] * S.G1[r * h + i];
-      S.dS1[e] = v;
+    // first layer: dS1 = -dZq G1^T (causal), a warp per row, its lanes over the hidden features
+    for (int s = threadIdx.x >> 5; s < C; s += blockDim.x >> 5) {
+      const int lane = threadIdx.x & 31;
+      warp_row_dots<0>(
+          (h + 31) / 32, s + 1,
+          [&](int m) {
+            const int i = lane + 32 * m;
+            return i < h ? S.dZq[s * h + i] : 0.f;
+          },
+          [&](int r, int m) {
+            const int i = lane + 32 * m;
+            return i < h ? S.G1[r * h + i] : 0.f;
+          },
+          [&](int r, float p) { S.dS1[s * C + r] = -p; });
+      for (int r = s + 1 + lane; r < C; r += 32) S.dS1[s * C + r] = 0.f;
     }
     __syncthreads();
     for (int e = threadIdx.x; e < C * h; e += blockDim.x) {

@@ -101,23 +101,36 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
     __syncthreads();
     // query view, kRows queries at a time
     for (int s0 = 0; s0 < C; s0 += kRows) {
-      for (int e = threadIdx.x; e < kRows * C; e += blockDim.x) {
-        const int sr = e / C, r = e % C, s = s0 + sr;
-        float v = 0.f;
-        if (r <= s && s < C) {
-          const TI* qs = Q + qk0 + (tc + s) * dk;
-          const TI* kr = K + qk0 + (tc + r) * dk;
-          float p = 0.f;
-          if (d.gvec) {
-            for (int i = 0; i < dk; ++i)
-              p += ldf(qs + i) * ldf(kr + i) * __expf(L[s * dk + i] - L[r * dk + i]);
-            v = eta[r] * p;
-          } else {
-            for (int i = 0; i < dk; ++i) p += ldf(qs + i) * ldf(kr + i);
-            v = eta[r] * expf(L[s] - L[r]) * p;
-          }
+      // a warp per query row, its lanes over the key features
+      for (int sr = threadIdx.x >> 5; sr < kRows; sr += blockDim.x >> 5) {
+        const int s = s0 + sr, lane = threadIdx.x & 31;
+        float* Srow = S + sr * C;
+        if (s >= C) {
+          for (int r = lane; r < C; r += 32) Srow[r] = 0.f;
+          continue;
         }
-        S[sr * C + r] = v;
+        float qv[4], lv[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const int i = lane + 32 * m;
+          qv[m] = i < dk ? ldf(Q + qk0 + (tc + s) * dk + i) : 0.f;
+          lv[m] = i < dk && d.gvec ? L[s * dk + i] : 0.f;
+        }
+        const TI* Kc = K + qk0 + tc * dk;
+        const float Ls = d.gvec ? 0.f : L[s];
+        const bool gv = d.gvec;
+        warp_row_dots<4>(
+            4, s + 1, [=](int m) { return qv[m]; },
+            [=](int r, int m) {
+              const int i = lane + 32 * m;
+              if (i >= dk) return 0.f;
+              const float kv = ldf(Kc + r * dk + i);
+              return gv ? kv * __expf(lv[m] - L[r * dk + i]) : kv;
+            },
+            [=](int r, float p) {
+              Srow[r] = gv ? eta[r] * p : eta[r] * expf(Ls - L[r]) * p;
+            });
+        for (int r = s + 1 + lane; r < C; r += 32) Srow[r] = 0.f;
       }
       __syncthreads();
       for (int e = threadIdx.x; e < kRows * nv; e += blockDim.x) {
@@ -240,22 +253,28 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       Z[e] = z;
       G[e] = a * act1(d.act, z);
     }
-    // S (causal, scaled)
-    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-      const int s = e / C, r = e % C;
-      float v = 0.f;
-      if (r <= s) {
-        float p = 0.f;
-        if (d.gvec)
-          for (int i = 0; i < dk; ++i)
-            p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i) *
-                 __expf(L[s * dk + i] - L[r * dk + i]);
-        else
-          for (int i = 0; i < dk; ++i)
-            p += ldf(Q + qk0 + (tc + s) * dk + i) * ldf(K + qk0 + (tc + r) * dk + i);
-        v = eta[r] * p * (d.gvec ? 1.f : expf(L[s] - L[r]));
+    // S (causal, scaled): a warp per query row, its lanes over the key features
+    for (int s = threadIdx.x >> 5; s < C; s += blockDim.x >> 5) {
+      const int lane = threadIdx.x & 31;
+      float qv[4], lv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int i = lane + 32 * m;
+        qv[m] = i < dk ? ldf(Q + qk0 + (tc + s) * dk + i) : 0.f;
+        lv[m] = i < dk && d.gvec ? L[s * dk + i] : 0.f;
       }
-      S[e] = v;
+      warp_row_dots<4>(
+          4, s + 1, [&](int m) { return qv[m]; },
+          [&](int r, int m) {
+            const int i = lane + 32 * m;
+            if (i >= dk) return 0.f;
+            const float kv = ldf(K + qk0 + (tc + r) * dk + i);
+            return d.gvec ? kv * __expf(lv[m] - L[r * dk + i]) : kv;
+          },
+          [&](int r, float p) {
+            S[s * C + r] = eta[r] * p * (d.gvec ? 1.f : expf(L[s] - L[r]));
+          });
+      for (int r = s + 1 + lane; r < C; r += 32) S[s * C + r] = 0.f;
     }
     // Y_r = (k_r * exp(L_C - L_r)) Wh: the key's route into the chunk-end state
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
@@ -275,13 +294,23 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       DZQ[e] = ldf(dO + v0 + (tc + s) * dv + j) * act1(d.act, zq);
     }
     __syncthreads();
-    // dS = -dZq G^T (causal)
-    for (int e = threadIdx.x; e < C * C; e += blockDim.x) {
-      const int s = e / C, r = e % C;
-      float v = 0.f;
-      if (r <= s)
-        for (int j = 0; j < dv; ++j) v -= DZQ[s * dv + j] * G[r * dv + j];
-      DS[e] = v;
+    // dS = -dZq G^T (causal): a warp per row, its lanes over the value features
+    for (int s = threadIdx.x >> 5; s < C; s += blockDim.x >> 5) {
+      const int lane = threadIdx.x & 31;
+      float av[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int j = lane + 32 * m;
+        av[m] = j < dv ? DZQ[s * dv + j] : 0.f;
+      }
+      warp_row_dots<4>(
+          4, s + 1, [&](int m) { return av[m]; },
+          [&](int r, int m) {
+            const int j = lane + 32 * m;
+            return j < dv ? G[r * dv + j] : 0.f;
+          },
+          [&](int r, float p) { DS[s * C + r] = -p; });
+      for (int r = s + 1 + lane; r < C; r += 32) DS[s * C + r] = 0.f;
     }
     // dG = -S^T dZq - diag(u) Y
     for (int e = threadIdx.x; e < C * dv; e += blockDim.x) {
