@@ -27,6 +27,7 @@ struct MlpDims {
 // Per-head scratch, in floats.
 struct MlpScratch {
   float *W1, *W2, *Wh1, *Wh2, *Wn1, *Wn2;                                     // weights
+  float *W1T, *W2T, *Wh1T;  // transposes of W1, W2, Wh1 (reads with lanes over the other index)
   float *Z1, *A1, *Bm, *G1, *Zq, *Aq, *dZq, *dA1, *dG1, *dB, *dZ1, *Yk;       // C x h
   float *G2, *dG2, *Ya;                                                       // C x dv
   float *S1, *S2, *dS1, *dS2;                                                 // C x C
@@ -35,7 +36,7 @@ struct MlpScratch {
 
 __host__ __device__ inline size_t mlp_head_floats(int C, int dk, int dv, int h) {
   const size_t nW = (size_t)dk * h + (size_t)h * dv;
-  return 3 * nW + 12 * (size_t)C * h + 3 * (size_t)C * dv + 4 * (size_t)C * C + 3 * (size_t)C;
+  return 4 * nW + (size_t)dk * h + 12 * (size_t)C * h + 3 * (size_t)C * dv + 4 * (size_t)C * C + 3 * (size_t)C;
 }
 
 __device__ MlpScratch carve(float* base, const MlpDims& d) {
@@ -46,6 +47,7 @@ __device__ MlpScratch carve(float* base, const MlpDims& d) {
   s.W1 = p; p += w1; s.W2 = p; p += w2;
   s.Wh1 = p; p += w1; s.Wh2 = p; p += w2;
   s.Wn1 = p; p += w1; s.Wn2 = p; p += w2;
+  s.W1T = p; p += w1; s.W2T = p; p += w2; s.Wh1T = p; p += w1;
   float** chs[] = {&s.Z1, &s.A1, &s.Bm, &s.G1, &s.Zq, &s.Aq, &s.dZq, &s.dA1, &s.dG1, &s.dB, &s.dZ1, &s.Yk};
   for (float** q : chs) { *q = p; p += ch; }
   s.G2 = p; p += cv; s.dG2 = p; p += cv; s.Ya = p; p += cv;
@@ -109,7 +111,7 @@ __device__ void mlp_chunk_forward(const MlpDims& d, const MlpScratch& S, const T
   for (int e = threadIdx.x; e < C * h; e += blockDim.x) {
     const int s = e / h, i = e % h;
     float b = 0.f;
-    for (int j = 0; j < dv; ++j) b += S.G2[s * dv + j] * S.W2[i * dv + j];
+    for (int j = 0; j < dv; ++j) b += S.G2[s * dv + j] * S.W2T[j * h + i];
     S.Bm[e] = b;
     S.G1[e] = b * act1(d.act, S.Z1[e]);
   }
@@ -153,7 +155,10 @@ __global__ void __launch_bounds__(512)
   const MlpScratch S = carve(ws + (size_t)bh * mlp_head_floats(C, dk, dv, h), d);
   const size_t n1 = (size_t)dk * h, n2 = (size_t)h * dv;
   for (size_t e = threadIdx.x; e < n1; e += blockDim.x) S.W1[e] = W1_0[bh * n1 + e];
-  for (size_t e = threadIdx.x; e < n2; e += blockDim.x) S.W2[e] = W2_0[bh * n2 + e];
+  for (size_t e = threadIdx.x; e < n2; e += blockDim.x) {
+    S.W2[e] = W2_0[bh * n2 + e];
+    S.W2T[(e % dv) * h + e / dv] = S.W2[e];
+  }
   __syncthreads();
   for (int c = 0; c < NC; ++c) {
     const size_t tok = (size_t)bh * d.T + (size_t)c * C;
@@ -191,7 +196,10 @@ __global__ void __launch_bounds__(512)
     }
     __syncthreads();
     for (size_t e = threadIdx.x; e < n1; e += blockDim.x) S.W1[e] = S.Wn1[e];
-    for (size_t e = threadIdx.x; e < n2; e += blockDim.x) S.W2[e] = S.Wn2[e];
+    for (size_t e = threadIdx.x; e < n2; e += blockDim.x) {
+      S.W2[e] = S.Wn2[e];
+      S.W2T[(e % dv) * h + e / dv] = S.Wn2[e];
+    }
     __syncthreads();
   }
   if (W1f)
@@ -212,13 +220,22 @@ __global__ void __launch_bounds__(512)
   const bool mse = d.loss == 0;
   const MlpScratch S = carve(ws + (size_t)bh * mlp_head_floats(C, dk, dv, h), d);
   const size_t n1 = (size_t)dk * h, n2 = (size_t)h * dv;
-  for (size_t e = threadIdx.x; e < n1; e += blockDim.x) S.Wh1[e] = dW1f ? dW1f[bh * n1 + e] : 0.f;
+  for (size_t e = threadIdx.x; e < n1; e += blockDim.x) {
+    S.Wh1[e] = dW1f ? dW1f[bh * n1 + e] : 0.f;
+    S.Wh1T[(e % h) * dk + e / h] = S.Wh1[e];
+  }
   for (size_t e = threadIdx.x; e < n2; e += blockDim.x) S.Wh2[e] = dW2f ? dW2f[bh * n2 + e] : 0.f;
   for (int c = NC - 1; c >= 0; --c) {
     const size_t tok = (size_t)bh * d.T + (size_t)c * C;
     const TI *Qh = Q + tok * dk, *Kh = K + tok * dk, *dOh = dO + tok * dv;
-    for (size_t e = threadIdx.x; e < n1; e += blockDim.x) S.W1[e] = W1c[((size_t)bh * NC + c) * n1 + e];
-    for (size_t e = threadIdx.x; e < n2; e += blockDim.x) S.W2[e] = W2c[((size_t)bh * NC + c) * n2 + e];
+    for (size_t e = threadIdx.x; e < n1; e += blockDim.x) {
+      S.W1[e] = W1c[((size_t)bh * NC + c) * n1 + e];
+      S.W1T[(e % h) * dk + e / h] = S.W1[e];
+    }
+    for (size_t e = threadIdx.x; e < n2; e += blockDim.x) {
+      S.W2[e] = W2c[((size_t)bh * NC + c) * n2 + e];
+      S.W2T[(e % dv) * h + e / dv] = S.W2[e];
+    }
     mlp_scans(d, beta, gamma, bh, c, S.eta, S.L);  // ends with a barrier
     mlp_chunk_forward(d, S, Qh, Kh, V + tok * dv);
     const float LC = S.L[C - 1];
@@ -262,7 +279,7 @@ __global__ void __launch_bounds__(512)
     for (int e = threadIdx.x; e < C * h; e += blockDim.x) {
       const int s = e / h, i = e % h;
       float a = 0.f;
-      for (int j = 0; j < dv; ++j) a += ldf(dOh + (size_t)s * dv + j) * S.W2[i * dv + j];
+      for (int j = 0; j < dv; ++j) a += ldf(dOh + (size_t)s * dv + j) * S.W2T[j * h + i];
       a *= expf(S.L[s]);
       for (int r = 0; r <= s; ++r)
         a += S.dS2[s * C + r] * S.eta[r] * expf(S.L[s] - S.L[r]) * S.A1[r * h + i];
@@ -304,7 +321,7 @@ __global__ void __launch_bounds__(512)
     for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
       const int s = e / dk, k = e % dk;
       float a = 0.f;
-      for (int i = 0; i < h; ++i) a += S.dZq[s * h + i] * S.W1[k * h + i];
+      for (int i = 0; i < h; ++i) a += S.dZq[s * h + i] * S.W1T[i * dk + k];
       a *= expf(S.L[s]);
       for (int r = 0; r <= s; ++r)
         a += S.dS1[s * C + r] * S.eta[r] * expf(S.L[s] - S.L[r]) * ldf(Kh + (size_t)r * dk + k);
@@ -341,7 +358,7 @@ __global__ void __launch_bounds__(512)
       const int r = e / h, i = e % h;
       float a = S.dA1[e];
       if (mse)
-        for (int j = 0; j < dv; ++j) a += S.dG2[r * dv + j] * S.W2[i * dv + j];
+        for (int j = 0; j < dv; ++j) a += S.dG2[r * dv + j] * S.W2T[j * h + i];
       S.dZ1[e] += a * act1(d.act, S.Z1[e]);
     }
     __syncthreads();
@@ -352,8 +369,8 @@ __global__ void __launch_bounds__(512)
         a += S.dS1[s * C + r] * S.eta[r] * expf(S.L[s] - S.L[r]) * ldf(Qh + (size_t)s * dk + k);
       float gw = 0.f, zw = 0.f;
       for (int i = 0; i < h; ++i) {
-        gw += S.G1[r * h + i] * S.Wh1[k * h + i];
-        zw += S.dZ1[r * h + i] * S.W1[k * h + i];
+        gw += S.G1[r * h + i] * S.Wh1T[i * dk + k];
+        zw += S.dZ1[r * h + i] * S.W1T[i * dk + k];
       }
       stf(dK + (tok + r) * dk + k, a - S.eta[r] * expf(LC - S.L[r]) * gw + zw);
     }
@@ -379,7 +396,10 @@ __global__ void __launch_bounds__(512)
       S.Wn2[e] = acc;
     }
     __syncthreads();
-    for (size_t e = threadIdx.x; e < n1; e += blockDim.x) S.Wh1[e] = S.Wn1[e];
+    for (size_t e = threadIdx.x; e < n1; e += blockDim.x) {
+      S.Wh1[e] = S.Wn1[e];
+      S.Wh1T[(e % h) * dk + e / h] = S.Wn1[e];
+    }
     for (size_t e = threadIdx.x; e < n2; e += blockDim.x) S.Wh2[e] = S.Wn2[e];
     __syncthreads();
   }

@@ -183,13 +183,15 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
     }
 }
 
-// Per-head float32 scratch of the backward (in units of floats): Wh, Wn, W0 (dk x dv each),
+// Per-head float32 scratch of the backward (in units of floats): Wh, Wn, W0 (dk x dv each) and
+// the transposes of W0 and Wh (dv x dk each, for contractions over the value features with
+// lanes over the key features),
 // Z, G, dZq, Y, dG, dZ, Zq (C x dv each), S, dS (C x C each), eta, L, deta, dL (C each), one
 // float for the chunk-end term of the decay gradient, and the decay-scaled operands
 // q_s exp(L_s) and k_r exp(L_C - L_r) (C x dk each); with a per-feature decay also the prefix L
 // and two parts of dJ/dL (C x dk each) and the chunk-end term per feature (dk).
 __host__ __device__ inline size_t bwd_head_floats(int C, int dk, int dv, bool gvec) {
-  return 3 * (size_t)dk * dv + 7 * (size_t)C * dv + 2 * (size_t)C * C + 4 * (size_t)C + 1 +
+  return 5 * (size_t)dk * dv + 7 * (size_t)C * dv + 2 * (size_t)C * C + 4 * (size_t)C + 1 +
          2 * (size_t)C * dk + (gvec ? 3 * (size_t)C * dk + dk : 0);
 }
 
@@ -205,7 +207,9 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
   float* Wh = ws + (size_t)bh * bwd_head_floats(C, dk, dv, d.gvec);
   float* Wn = Wh + dk * dv;
   float* W0 = Wn + dk * dv;  // float copy of the chunk-start state
-  float* Z = W0 + dk * dv;
+  float* W0T = W0 + dk * dv; // W0 transposed [dv][dk]
+  float* WhT = W0T + dk * dv; // Wh transposed [dv][dk]
+  float* Z = WhT + dk * dv;
   float* G = Z + C * dv;
   float* DZQ = G + C * dv;
   float* Y = DZQ + C * dv;
@@ -226,13 +230,17 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
   float* wendv = dLk + C * dk; //                    row sums of W_end * dW_end  [dk]
   if (d.gvec) L = wendv + dk;  //                    log-decay prefix  [C][dk]
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
-  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
+  for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
     Wh[e] = dWf ? dWf[(size_t)bh * dk * dv + e] : 0.f;
+    WhT[(e % dv) * dk + e / dv] = Wh[e];
+  }
   __syncthreads();
   for (int c = NC - 1; c >= 0; --c) {
     const size_t tc = (size_t)c * C;
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x)
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
       W0[e] = ldf(Wc + ((size_t)bh * NC + c) * dk * dv + e);
+      W0T[(e % dv) * dk + e / dv] = W0[e];
+    }
     chunk_scans(d, beta, gamma, bh, c, eta, L);  // ends with __syncthreads
     // the decay-scaled operands of the readout, the chunk-end route of the keys and the dW
     // update, one exponential per token and feature
@@ -352,7 +360,7 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       const int s = e / dk, i = e % dk;
       const float Ls = Lat(d, L, s, i);
       float a1 = 0.f;
-      for (int j = 0; j < dv; ++j) a1 += DZQ[s * dv + j] * W0[i * dv + j];
+      for (int j = 0; j < dv; ++j) a1 += DZQ[s * dv + j] * W0T[j * dk + i];
       float acc = expf(Ls) * a1;
       if (d.gvec)
         for (int r = 0; r <= s; ++r)
@@ -374,8 +382,8 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
         for (int s = r; s < C; ++s) acc += DS[s * C + r] * ldf(Q + qk0 + (tc + s) * dk + i);
       float gw = 0.f, zw = 0.f;
       for (int j = 0; j < dv; ++j) {
-        gw += G[r * dv + j] * Wh[i * dv + j];
-        zw += DZ[r * dv + j] * W0[i * dv + j];
+        gw += G[r * dv + j] * WhT[j * dk + i];
+        zw += DZ[r * dv + j] * W0T[j * dk + i];
       }
       acc += -eta[r] * expf(Lat(d, L, C - 1, i) - Lr) * gw;
       if (d.gvec && dgamma) dLk[e] = -ldf(K + qk0 + (tc + r) * dk + i) * acc;
@@ -443,7 +451,10 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
       Wn[e] = acc;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) Wh[e] = Wn[e];
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+      Wh[e] = Wn[e];
+      WhT[(e % dv) * dk + e / dv] = Wn[e];
+    }
     __syncthreads();
   }
   for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) dW0[(size_t)bh * dk * dv + e] = Wh[e];
