@@ -282,3 +282,23 @@ def test_saved_buffer_size():
     assert ttt.ttt_saved_bytes(_cfg()) == 2 * 3 * 256 * 64 * 4
     with pytest.raises(ttt.TTTError):
         ttt.ttt_saved_bytes(_cfg(T=250))
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    # the library takes dense device arrays; the binding refuses anything else before calling it
+    import torch
+    cfg = _cfg(B=1, H=1, T=64, dk=16, dv=16, C=16)
+    x = torch.zeros((1, 1, 64, 16))
+    beta, W0 = torch.zeros((1, 1, 64)), torch.zeros((1, 1, 16, 16))
+    n0 = ttt.ttt_kernel_launches()
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        ttt.ttt_chunk_fwd(cfg, x, x, x, beta, None, W0, x)
+    with pytest.raises(ValueError, match="contiguous"):
+        ttt.ttt_chunk_fwd(cfg, x.transpose(2, 3), x, x, beta, None, W0, x)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        ttt.ttt_add_f32(torch.zeros(8), torch.zeros(8))
+    Zt = torch.zeros((128, 256)).t()  # [T, d_ff] = [256, 128], column-major
+    Vh, W, O = (torch.zeros(s) for s in ((256, 128), (128, 128), (256, 128)))
+    with pytest.raises(ValueError, match="contiguous"):
+        ttt.inplace_ttt_fwd(256, 128, 128, 128, 1e-3, Zt, Vh, W, O)
+    assert ttt.ttt_kernel_launches() == n0

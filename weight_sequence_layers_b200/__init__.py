@@ -86,10 +86,24 @@ def status_string(status: int) -> str:
 
 
 def _ptr(t):
+    """Device address of a tensor argument; None and raw integer addresses pass through.
+
+    The library reads and writes every array argument as a dense row-major array on the
+    current CUDA device. A strided view, a host tensor or a tensor on another device would
+    give wrong results or a memory fault, so they are refused here, before any library call.
+    """
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous (dense row-major, no strided views)")
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors: the library takes device pointers")
+    import torch
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"tensor on {t.device}, but the library runs on the current device "
+                         f"cuda:{torch.cuda.current_device()}")
     return t.data_ptr()
 
 
