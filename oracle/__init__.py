@@ -43,19 +43,24 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def open_library(path: str):
+    """A build of ttt_oracle.cpp at `path`, with the C signatures of its entry points."""
+    lib = ctypes.CDLL(path)
+    d, i = ctypes.c_double, ctypes.c_int
+    p = ctypes.c_void_p
+    lib.ttt_oracle_fwd_f64.argtypes = [i] * 8 + [d, i] + [p] * 9 + [i]
+    lib.ttt_oracle_fwd_f32.argtypes = [i] * 8 + [d, i] + [p] * 9 + [i]
+    lib.ttt_oracle_bwd_f64.argtypes = [i] * 8 + [d, i] + [p] * 14 + [i]
+    for fn in (lib.ttt_oracle_fwd_f64, lib.ttt_oracle_fwd_f32, lib.ttt_oracle_bwd_f64):
+        fn.restype = i
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
         build()
-        lib = ctypes.CDLL(_LIB)
-        d, f, i = ctypes.c_double, ctypes.c_float, ctypes.c_int
-        p = ctypes.c_void_p
-        lib.ttt_oracle_fwd_f64.argtypes = [i] * 8 + [d, i] + [p] * 9 + [i]
-        lib.ttt_oracle_fwd_f32.argtypes = [i] * 8 + [d, i] + [p] * 9 + [i]
-        lib.ttt_oracle_bwd_f64.argtypes = [i] * 8 + [d, i] + [p] * 14 + [i]
-        for fn in (lib.ttt_oracle_fwd_f64, lib.ttt_oracle_fwd_f32, lib.ttt_oracle_bwd_f64):
-            fn.restype = i
-        _lib = lib
+        _lib = open_library(_LIB)
     return _lib
 
 
