@@ -1,6 +1,7 @@
 """The C-ABI library loads, exports every function include/ttt.h declares, and rejects bad
 arguments on the host before touching a GPU (these run without one)."""
 import ctypes
+import os
 import subprocess
 
 import pytest
@@ -302,3 +303,47 @@ def test_binding_refuses_host_and_strided_tensors():
     with pytest.raises(ValueError, match="contiguous"):
         ttt.inplace_ttt_fwd(256, 128, 128, 128, 1e-3, Zt, Vh, W, O)
     assert ttt.ttt_kernel_launches() == n0
+
+
+C_CLIENT = r"""
+#include "ttt.h"
+#include <stdio.h>
+#include <string.h>
+
+/* A plain C99 caller of the library: the header must compile as C, the entry points must
+   link, and argument errors must come back as statuses with nothing launched. */
+int main(void) {
+  ttt_config c = {2, 3, 256, 64, 64, 64, TTT_F32, TTT_LOSS_MSE, TTT_ACT_ID, -2.9f,
+                  TTT_DECAY_SCALAR};
+  char a[64];
+  void* p = (void*)(((unsigned long)a + 15) & ~15ul); /* aligned, never dereferenced */
+  int bad = 0;
+  bad |= strcmp(ttt_status_string(TTT_OK), "ok") != 0;
+  bad |= ttt_workspace_bytes(&c, 0) != 0;
+  bad |= ttt_workspace_bytes(&c, 1) == 0 || ttt_workspace_bytes(&c, 1) == (size_t)-1;
+  /* Q missing */
+  bad |= ttt_chunk_fwd(&c, NULL, p, p, (const float*)p, NULL, (const float*)p, p, NULL, NULL,
+                       NULL, NULL, 0, NULL) != TTT_ERR_INVALID_ARG;
+  /* misaligned K */
+  bad |= ttt_chunk_fwd(&c, p, (char*)p + 4, p, (const float*)p, NULL, (const float*)p, p, NULL,
+                       NULL, NULL, NULL, 0, NULL) != TTT_ERR_ALIGNMENT;
+  /* T not a multiple of C */
+  c.T = 250;
+  bad |= ttt_workspace_bytes(&c, 0) != (size_t)-1;
+  bad |= inplace_ttt_workspace_bytes(1000, 256, 256, 128) != (size_t)-1;
+  printf("%s\n", bad ? "FAIL" : "PASS");
+  return bad;
+}
+"""
+
+
+def test_header_compiles_and_links_as_plain_c(tmp_path):
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    pkg = os.path.dirname(ttt.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.dirname(ttt.HEADER), str(src), "-L", pkg, "-lttt",
+                    f"-Wl,-rpath,{pkg}", "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "PASS", r.stdout + r.stderr
