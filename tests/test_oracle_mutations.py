@@ -23,7 +23,8 @@ COMBOS = pins.COMBOS
 
 # --------------------------------------------------------------------------- pin batteries
 FWD_PINS = (
-    [("golden scalar chunks", pins.test_golden_scalar_worked_examples)]
+    [("golden scalar chunks", pins.test_golden_scalar_worked_examples),
+     ("golden vector-decay chunk", pins.test_golden_vector_decay_worked_example)]
     + [(f"dual form {l}/{a} C={C} decay={d}",
         lambda l=l, a=a, C=C, d=d: pins.test_oracle_matches_chunk_dual_form(l, a, C, d))
        for l, a in COMBOS for C in (1, 4) for d in (False, True)]

@@ -349,6 +349,33 @@ def test_vector_decay_matches_its_dual_form(loss, act, C):
     np.testing.assert_allclose(WF, WF2, rtol=0, atol=1e-12 * max(1, np.abs(WF2).max()))
 
 
+VECTOR_GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "vector_decay_worked.txt")
+
+
+def test_golden_vector_decay_worked_example():
+    """Hand-worked rationals of tests/golden/vector_decay_worked.txt, forward and backward."""
+    want = {}
+    with open(VECTOR_GOLDEN) as f:
+        for line in f:
+            if "|" in line and not line.startswith("#"):
+                name, vals = line.split("|")
+                want[name.strip()] = [float(x) for x in vals.split()]
+    assert len(want) == 8
+    Q = np.array([[1.0, 1.0], [1.0, 1.0]]).reshape(1, 1, 2, 2)
+    K = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 1, 2, 2)
+    V = np.array([0.0, 1.0]).reshape(1, 1, 2, 1)
+    beta = np.zeros((1, 1, 2))
+    gamma = np.array([[0.5, 1.0], [1.0, 0.5]]).reshape(1, 1, 2, 2)
+    W0 = np.array([1.0, 0.0]).reshape(1, 1, 2, 1)
+    kw = dict(C=2, loss="mse", act="id", lr_bias=0.0)
+    O, WF, _, _ = oracle.ttt_fwd(Q, K, V, beta, gamma, W0, **kw)
+    g = oracle.ttt_bwd(Q, K, V, beta, gamma, W0, np.array([0.0, 1.0]).reshape(1, 1, 2, 1), None,
+                       **kw)
+    got = dict(O=O, W_final=WF, **g)
+    for name, vals in want.items():
+        np.testing.assert_allclose(got[name].ravel(), vals, atol=1e-14, err_msg=name)
+
+
 def test_vector_decay_with_equal_features_is_the_scalar_decay():
     rng = np.random.default_rng(310)
     B, H, T, dk, dv = 1, 2, 16, 4, 3
