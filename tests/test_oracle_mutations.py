@@ -46,6 +46,7 @@ BWD_PINS = (
        for l, a in COMBOS]
 )
 INPLACE_PINS = [
+    ("golden In-Place and NTP target", pins.test_golden_inplace_and_target_worked_examples),
     ("associative update", pins.test_inplace_final_state_is_associative),
     ("plain GEMM cases", pins.test_inplace_single_chunk_and_zero_lr_are_plain_gemm),
     ("In-Place dual form", pins.test_inplace_dual_form),
@@ -56,7 +57,8 @@ INPLACE_PINS = [
     ("NTP target finite differences", pins.test_inplace_target_backward_matches_finite_differences),
 ]
 MLP_PINS = (
-    [(f"TTT-MLP dual form {l}/{a} C={C}",
+    [("golden TTT-MLP", pins.test_golden_ttt_mlp_worked_example)]
+    + [(f"TTT-MLP dual form {l}/{a} C={C}",
       lambda l=l, a=a, C=C: pins.test_ttt_mlp_matches_its_dual_form(l, a, C))
      for l, a in COMBOS for C in (2, 4)]
     + [("TTT-MLP without learning", pins.test_ttt_mlp_without_learning_only_decays)]

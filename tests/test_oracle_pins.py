@@ -11,7 +11,9 @@
   (section "内部学习规则与学习率参数化", the update matrix whose eigenvalues
   govern stability);
 * streaming and column independence;
-* hand-worked golden values (tests/golden/scalar_chunk_worked.txt);
+* hand-worked golden values (tests/golden/: a scalar chunk, a vector-decay chunk, a TTT-MLP
+  chunk, In-Place with and without a document reset, and the NTP target), forward and
+  backward;
 * central finite differences for every backward output;
 * TTT-MLP (two-layer fast weight): its own brute-force chunk dual form, the
   decay-only case without learning, and finite differences of its backward;
@@ -784,3 +786,59 @@ def test_inplace_backward_with_resets_matches_finite_differences():
             x[idx] = old
             fd[idx] = (jp - jm) / (2 * h)
         assert np.abs(g[key] - fd).max() / np.abs(fd).max() < 1e-8, key
+
+
+# ------------------------------------------------------------------ hand-worked fixtures
+def _worked_values(name):
+    want = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", name)) as f:
+        for line in f:
+            if "|" in line and not line.startswith("#"):
+                key, vals = line.split("|")
+                want[key.strip()] = [float(x) for x in vals.split()]
+    return want
+
+
+def test_golden_ttt_mlp_worked_example():
+    """Hand-worked integers of tests/golden/ttt_mlp_worked.txt, forward and backward."""
+    want = _worked_values("ttt_mlp_worked.txt")
+    assert len(want) == 9
+    col = lambda *v: np.array(v, dtype=float).reshape(1, 1, len(v), 1)
+    Q, K, V = col(1, 2), col(1, 1), col(1, 0)
+    beta = np.zeros((1, 1, 2))
+    W1, W2 = np.ones((1, 1, 1, 1)), np.full((1, 1, 1, 1), 2.0)
+    kw = dict(C=2, loss="mse", act="id", lr_bias=0.0)
+    O, W1f, W2f = oracle.ttt_mlp_fwd(Q, K, V, beta, None, W1, W2, **kw)
+    got = dict(O=O.numpy(), W1_final=W1f.numpy(), W2_final=W2f.numpy())
+    for key in got:
+        np.testing.assert_allclose(got[key].ravel(), want[key], atol=1e-12, err_msg=key)
+    g = oracle.ttt_mlp_bwd(Q, K, V, beta, None, W1, W2, col(0, 1), **kw)
+    for key in ("dQ", "dK", "dV", "dbeta", "dW1", "dW2"):
+        np.testing.assert_allclose(g[key].ravel(), want[key], atol=1e-12, err_msg=key)
+
+
+def test_golden_inplace_and_target_worked_examples():
+    """Hand-worked rationals of tests/golden/inplace_worked.txt: In-Place forward and backward
+    without and with a document reset, and the NTP target with its backward."""
+    want = _worked_values("inplace_worked.txt")
+    assert len(want) == 15
+    Z = np.array([[1.0, 0.0], [1.0, 1.0]])
+    Vh = np.array([[2.0], [4.0]])
+    W = np.array([[1.0, 2.0]])
+    dO = np.array([[0.0], [1.0]])
+    for tag, starts in (("inplace", ()), ("reset", (1,))):
+        O, Wf = oracle.inplace_fwd(Z, Vh, W, C=1, lr=0.5, doc_starts=starts)
+        g = oracle.inplace_bwd(Z, Vh, W, dO, None, C=1, lr=0.5, doc_starts=starts)
+        got = dict(O=O, W_final=Wf, **g)
+        for key in ("O", "W_final", "dZ", "dVhat", "dW"):
+            np.testing.assert_allclose(got[key].ravel(), want[f"{tag} {key}"], atol=1e-14,
+                                       err_msg=f"{tag} {key}")
+    X0 = np.array([[1.0], [2.0], [3.0]])
+    taps = np.array([[1.0], [2.0]])
+    Wt = np.array([[3.0]])
+    Vt, Y = oracle.inplace_target(X0, taps, Wt)
+    g = oracle.inplace_target_bwd(X0, taps, Wt, np.array([[1.0], [0.0], [1.0]]))
+    got = dict(Vhat=Vt, Y=Y, **g)
+    for key in ("Vhat", "Y", "dX0", "dconv_w", "dW_target"):
+        np.testing.assert_allclose(got[key].ravel(), want[f"target {key}"], atol=1e-14,
+                                   err_msg=f"target {key}")
