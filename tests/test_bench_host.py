@@ -209,3 +209,30 @@ def test_traffic_counters_are_dropped_once_a_source_changes(tmp_path, monkeypatc
     assert bench.measured_traffic("missing", "w") is None
     src.write_bytes(b"kernel v2")
     assert bench.measured_traffic("call", "w") is None
+
+
+def test_reference_arm_line():
+    # `bench.py --impl reference` times the oracle on the host cores; it needs no GPU
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+           "--warmup", "0"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "tokens/s" and line["higher_is_better"] is True
+    assert line["steps"] == 1 and line["warmup"] >= 3  # at least three warm-up steps, always
+    assert line["config"]["workload"] == synth.TRAIN_1P45B.name
+    assert line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+    # under torchrun only rank 0 runs it; the other ranks exit at once without output
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=120, cwd=root,
+                       env=dict(os.environ, RANK="1", WORLD_SIZE="2"))
+    assert r.returncode == 0 and r.stdout.strip() == ""
