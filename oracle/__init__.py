@@ -90,7 +90,10 @@ def _gvec(g, q):
 
 def ttt_fwd(Q, K, V, beta, gamma, W0, *, C: int, loss: str = "mse", act: str = "id",
             lr_bias: float, nthreads: int = 0, state: str = "f64"):
-    """Per-token fast-weight evolution. Returns (O, W_final, W_chunks, threads_used).
+    """Per-token fast-weight evolution of the chunkwise TTT layer (page "Modular TTT:
+    Rethinking Test-Time Training as Composable Modules", section "方法步骤详情", Algorithm 1,
+    with the learning rate of section "内部学习规则与学习率参数化" and the decay of section
+    "权重衰减"), run by ttt_oracle.cpp. Returns (O, W_final, W_chunks, threads_used).
 
     Q, K: [B,H,T,dk]; V: [B,H,T,dv]; beta: [B,H,T]; gamma: [B,H,T] (scalar decay),
     [B,H,T,dk] (per-feature decay of the rows of W) or None (no decay);
@@ -118,7 +121,9 @@ def ttt_fwd(Q, K, V, beta, gamma, W0, *, C: int, loss: str = "mse", act: str = "
 
 def ttt_bwd(Q, K, V, beta, gamma, W0, dO, dW_T=None, *, C: int, loss: str = "mse",
             act: str = "id", lr_bias: float, nthreads: int = 0):
-    """Reverse-mode of the per-token loop for J = <dO,O> + <dW_T,W_final> (fp64).
+    """Reverse-mode of ttt_fwd's per-token loop for J = <dO,O> + <dW_T,W_final> (fp64), run by
+    ttt_oracle.cpp. The page (section "技术新颖性") hand-derives analytic backward operators
+    without printing them; this is the plain reverse-mode of the forward it follows.
     Returns dict dQ, dK, dV, dbeta, dW0, and dgamma (shaped like gamma) when gamma is given."""
     lib = _load()
     dt = np.float64
