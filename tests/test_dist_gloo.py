@@ -1,6 +1,8 @@
-"""Multi-rank paths on CPU with the gloo backend (world size 2): bench.py's replicas (the step
-time is the max over ranks and the throughput aggregates all ranks' tokens; weak scaling, no
-data-path collective) and the exchange of the context-parallel In-Place forward."""
+"""Multi-rank paths on CPU with the gloo backend (world sizes 2 and 4): bench.py's replicas (the
+step time is the max over ranks and the throughput aggregates all ranks' tokens; weak scaling,
+no data-path collective), the exchange of the context-parallel In-Place forward, and what a
+rank sees when a peer fails before the exchange (an error from the collective within the
+process group's timeout, not a hang)."""
 import os
 import socket
 
@@ -35,8 +37,8 @@ def _rank_main(rank, world, port, out):
 
 
 @pytest.mark.timeout(120)
-def test_replica_timing_is_max_over_ranks_and_tokens_add_up():
-    world = 2
+@pytest.mark.parametrize("world", [2, 4])
+def test_replica_timing_is_max_over_ranks_and_tokens_add_up(world):
     ctx = mp.get_context("spawn")
     with ctx.Manager() as mgr:
         out = mgr.dict()
@@ -49,10 +51,10 @@ def test_replica_timing_is_max_over_ranks_and_tokens_add_up():
             p.join(90)
             assert p.exitcode == 0
         res = dict(out)
-    assert set(res) == {0, 1}
+    assert set(res) == set(range(world))
     for ms, value in res.values():
-        assert ms == pytest.approx(20.0 / 5)                    # slowest rank, per step
-        assert value == pytest.approx(2 * 1000 / (4.0e-3))      # both ranks' tokens
+        assert ms == pytest.approx(10.0 * world / 5)                       # slowest rank, per step
+        assert value == pytest.approx(world * 1000 / (ms * 1e-3))          # every rank's tokens
 
 
 
@@ -112,11 +114,11 @@ def _cp_rank(rank, world, port, out):
 
 
 @pytest.mark.timeout(120)
-def test_inplace_context_parallel_scan_equals_one_sequence():
+@pytest.mark.parametrize("world", [2, 4])
+def test_inplace_context_parallel_scan_equals_one_sequence(world):
     import numpy as np
 
     import oracle
-    world = 2
     ctx = mp.get_context("spawn")
     with ctx.Manager() as mgr:
         out = mgr.dict()
@@ -137,3 +139,47 @@ def test_inplace_context_parallel_scan_equals_one_sequence():
     got = np.concatenate([np.array(res[r][0]) for r in range(world)])
     np.testing.assert_allclose(got, O, atol=1e-12)
     np.testing.assert_allclose(np.array(res[world - 1][1]), WF, atol=1e-12)
+
+
+def _cp_rank_with_failed_peer(rank, world, port, out):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    import weight_sequence_layers_b200 as ttt
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=10))
+    if rank == world - 1:
+        os._exit(3)  # this rank fails between steps, before the exchange
+    n, d_ff, d_model, C = 4, 6, 5, 4
+    W = torch.zeros((d_model, d_ff), dtype=torch.float64)
+    O = torch.empty((n, d_model), dtype=torch.float64)
+    try:
+        ttt.inplace_cp_fwd(n, d_ff, d_model, C, 0.1, torch.ones((n, d_ff), dtype=torch.float64),
+                           torch.ones((n, d_model), dtype=torch.float64), W, O, None, 0,
+                           ops=_OracleOps)
+        out[rank] = "returned"
+    except Exception as e:  # the collective reports the lost peer
+        out[rank] = "raised " + type(e).__name__
+    os._exit(0)
+
+
+@pytest.mark.timeout(120)
+def test_context_parallel_exchange_fails_loudly_when_a_peer_is_gone():
+    world = 2
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_cp_rank_with_failed_peer, args=(r, world, port, out))
+                 for r in range(world)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(90)
+        codes = [p.exitcode for p in procs]
+        res = dict(out)
+    assert codes == [0, 3]
+    assert res.get(0, "").startswith("raised"), res
