@@ -14,7 +14,12 @@ FWD_NAMES = {"ttt_workspace_bytes", "ttt_chunk_fwd", "ttt_chunk_bwd", "inplace_t
              "ttt_mlp_fwd", "ttt_mlp_bwd", "ttt_mlp_workspace_bytes",
              "inplace_ttt_fwd_docs", "inplace_ttt_bwd_docs", "inplace_ttt_docs_workspace_bytes",
              "inplace_ttt_delta", "ttt_add_f32", "ttt_saved_bytes", "ttt_get_device_error", "ttt_selftest_bounded_wait",
-             "ttt_status_string"}
+             "ttt_status_string", "ttt_kernel_launches", "ttt_chunk_bwd_noalloc"}
+
+
+def test_binding_gives_every_declared_function_its_signature():
+    # ctypes would otherwise pass every argument as a C int
+    assert set(ttt.header_functions()) == set(ttt._SIGS)
 
 
 def test_header_declares_the_entry_points():

@@ -78,7 +78,10 @@ for _name, (_args, _ret) in _SIGS.items():
 def header_functions() -> list[str]:
     """Names of the functions include/ttt.h declares."""
     text = open(HEADER).read()
-    return re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(\w+)\s*\(", text, flags=re.M)
+    # a declaration starts in column 0 with its return type (one or more words, pointers
+    # included), then the name and "("; comments, macros and continuation lines do not
+    return re.findall(r"^(?!typedef\b)(?:[A-Za-z_]\w*[ \t\*]+)+([A-Za-z_]\w*)\s*\(", text,
+                      flags=re.M)
 
 
 def status_string(status: int) -> str:
