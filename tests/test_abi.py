@@ -352,3 +352,51 @@ def test_header_compiles_and_links_as_plain_c(tmp_path):
                     f"-Wl,-rpath,{pkg}", "-o", str(exe)], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "PASS", r.stdout + r.stderr
+
+
+def _declared_parameters():
+    """name -> list of parameter declarations, parsed from include/ttt.h."""
+    import re
+    text = open(ttt.HEADER).read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)  # drop comments
+    out = {}
+    for name in ttt.header_functions():
+        m = re.search(r"\b" + name + r"\s*\(([^)]*)\)\s*;", text)
+        assert m, name
+        params = [p.strip() for p in m.group(1).split(",")]
+        out[name] = [] if params == ["void"] else params
+    return out
+
+
+def _kind_of_declaration(p):
+    if "*" in p:
+        return "pointer"
+    words = p.split()[:-1]  # drop the parameter name
+    if words == ["size_t"]:
+        return "size_t"
+    if words == ["float"]:
+        return "float"
+    if words in (["int"], ["unsigned"], ["ttt_status"]):
+        return "int"
+    raise AssertionError(f"unexpected parameter {p!r}")
+
+
+def _kind_of_ctype(t):
+    if t in (ctypes.c_void_p,) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "pointer"
+    if t is ctypes.c_size_t:
+        return "size_t"
+    if t is ctypes.c_float:
+        return "float"
+    if t in (ctypes.c_int, ctypes.c_uint):
+        return "int"
+    raise AssertionError(f"unexpected ctypes type {t!r}")
+
+
+def test_binding_signatures_match_the_header():
+    # the number and kind (pointer, size_t, float, int) of every argument ctypes passes agree
+    # with the declaration; a mismatch would shift every later argument
+    for name, params in _declared_parameters().items():
+        argtypes, _ = ttt._SIGS[name]
+        assert [_kind_of_declaration(p) for p in params] == \
+            [_kind_of_ctype(t) for t in argtypes], name
