@@ -400,3 +400,14 @@ def test_binding_signatures_match_the_header():
         argtypes, _ = ttt._SIGS[name]
         assert [_kind_of_declaration(p) for p in params] == \
             [_kind_of_ctype(t) for t in argtypes], name
+
+
+def test_binding_return_types_match_the_header():
+    import re
+    text = open(ttt.HEADER).read()
+    want = {"size_t": ctypes.c_size_t, "ttt_status": ctypes.c_int, "const char*": ctypes.c_char_p,
+            "unsigned long long": ctypes.c_ulonglong}
+    for name in ttt.header_functions():
+        m = re.search(r"^([A-Za-z_][\w \t\*]*?)\s*\b" + name + r"\s*\(", text, flags=re.M)
+        ret = " ".join(m.group(1).replace("*", " * ").split()).replace(" *", "*")
+        assert ttt._SIGS[name][1] is want[ret], (name, ret)
