@@ -411,3 +411,30 @@ def test_binding_return_types_match_the_header():
         m = re.search(r"^([A-Za-z_][\w \t\*]*?)\s*\b" + name + r"\s*\(", text, flags=re.M)
         ret = " ".join(m.group(1).replace("*", " * ").split()).replace(" *", "*")
         assert ttt._SIGS[name][1] is want[ret], (name, ret)
+
+
+def test_config_struct_matches_the_header():
+    # field order and types of ttt_config in the binding are the header's, and so are the
+    # enum values the binding passes
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", open(ttt.HEADER).read(), flags=re.S)
+    body = re.search(r"typedef struct \{(.*?)\} ttt_config;", text, flags=re.S).group(1)
+    fields = []
+    for decl in body.split(";"):
+        words = decl.replace(",", " ").split()
+        if words:
+            fields += [(name, words[0]) for name in words[1:]]
+    ctype = {"int": ctypes.c_int, "float": ctypes.c_float}
+    assert [(n, ctype[t]) for n, t in fields] == list(ttt.ttt_config._fields_)
+    enums = dict(re.findall(r"\b(TTT_[A-Z0-9_]+)\s*=\s*(\d+)", text))
+    assert int(enums["TTT_F32"]) == ttt.F32 and int(enums["TTT_BF16"]) == ttt.BF16
+    assert {k: int(enums["TTT_LOSS_" + k.upper()]) for k in ttt.LOSS} == ttt.LOSS
+    assert {k: int(enums["TTT_ACT_" + k.upper()]) for k in ttt.ACT} == ttt.ACT
+    assert {k: int(enums["TTT_DECAY_" + k.upper()]) for k in ttt.DECAY} == ttt.DECAY
+    names = ["TTT_OK", "TTT_ERR_INVALID_ARG", "TTT_ERR_UNSUPPORTED", "TTT_ERR_ALIGNMENT",
+             "TTT_ERR_WORKSPACE", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT"]
+    assert [int(enums[n]) for n in names] == [ttt.OK, ttt.ERR_INVALID_ARG, ttt.ERR_UNSUPPORTED,
+                                             ttt.ERR_ALIGNMENT, ttt.ERR_WORKSPACE, ttt.ERR_CUDA,
+                                             ttt.ERR_TIMEOUT]
+    m = re.search(r"#define TTT_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert int(m.group(1)) << int(m.group(2)) == ttt.NOALLOC_SCRATCH_BYTES
