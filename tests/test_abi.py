@@ -438,3 +438,17 @@ def test_config_struct_matches_the_header():
                                              ttt.ERR_TIMEOUT]
     m = re.search(r"#define TTT_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
     assert int(m.group(1)) << int(m.group(2)) == ttt.NOALLOC_SCRATCH_BYTES
+
+
+@pytest.mark.parametrize("act", ["id", "silu"])
+@pytest.mark.parametrize("d,C", [(64, 256), (128, 128), (128, 256)])
+def test_tensor_core_backward_workspace_is_the_documented_sum(act, d, C):
+    # the bf16 chunk-end adjoints, G when the forward's G is not passed, a float per token for
+    # the decay gradient, and with SiLU four bf16 planes (include/ttt.h, ttt_chunk_bwd_noalloc)
+    B, H, T = 2, 3, 4 * C
+    cfg = _cfg(B=B, H=H, T=T, dk=d, dv=d, C=C, dtype="bf16", act=act)
+    adj, G, dg = B * H * (T // C) * d * d * 2, B * H * T * d * 2, B * H * T * 4
+    planes = 4 * B * H * T * d * 2 if act == "silu" else 0
+    assert ttt.ttt_workspace_bytes(cfg, 2) == adj + dg + planes
+    if act == "id":  # the SiLU backward without the forward's G and Zq runs on SIMT kernels
+        assert ttt.ttt_workspace_bytes(cfg, 1) == adj + G + dg
