@@ -150,6 +150,13 @@ def ttt_workspace_bytes(cfg: ttt_config, for_bwd: int) -> int:
 
 def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None, G_saved=None,
                   workspace=None, workspace_bytes=0, stream=None):
+    """Forward of the chunkwise TTT layer on the current device and stream.
+
+    Q, K [B,H,T,dk]; V, O [B,H,T,dv] in cfg's dtype; beta [B,H,T] and W0, W_final [B,H,dk,dv]
+    float32; gamma [B,H,T] or [B,H,T,dk] float32, or None (no decay). W_chunks [B,H,T/C,dk,dv]
+    in cfg's dtype
+    and G_saved (ttt_saved_bytes) are optional outputs that ttt_chunk_bwd reads. Workspace:
+    ttt_workspace_bytes(cfg, 0) bytes. Raises TTTError on a non-OK status."""
     st = _lib.ttt_chunk_fwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
                             _ptr(W0), _ptr(O), _ptr(W_final), _ptr(W_chunks), _ptr(G_saved),
                             _ptr(workspace), int(workspace_bytes), _stream(stream))
@@ -158,6 +165,12 @@ def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None,
 
 def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, O, W_final, dQ,
                   dK, dV, dbeta, dW0, dgamma, workspace=None, workspace_bytes=0, stream=None):
+    """Analytic backward of the layer for J = <dO, O> + <dW_final, W_final>.
+
+    Takes the forward's inputs, its W_chunks and (optionally) G_saved, dO and dW_final (or
+    None), and writes dQ, dK, dV, dbeta, dW0 and, when dgamma is given, the decay gradient
+    (which also needs the forward's O, and W_final when dW_final is given). Workspace:
+    ttt_workspace_bytes(cfg, 2 if G_saved is passed else 1) bytes."""
     st = _lib.ttt_chunk_bwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
                             _ptr(W0), _ptr(W_chunks), _ptr(G_saved), _ptr(dO), _ptr(dW_final),
                             _ptr(O), _ptr(W_final), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta),
@@ -189,6 +202,9 @@ def ttt_mlp_workspace_bytes(cfg: ttt_config, hidden: int) -> int:
 
 def ttt_mlp_fwd(cfg, hidden, Q, K, V, beta, gamma, W1_0, W2_0, O, W1_final, W2_final, W1_chunks,
                 W2_chunks, workspace, workspace_bytes, stream=None):
+    """TTT-MLP forward: the fast weight act(k W1) W2 with W1 [B,H,dk,hidden] and W2
+    [B,H,hidden,dv] float32; W1_chunks / W2_chunks keep the chunk-start weights for the
+    backward. Workspace: ttt_mlp_workspace_bytes(cfg, hidden)."""
     st = _lib.ttt_mlp_fwd(ctypes.byref(cfg), int(hidden), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
                           _ptr(gamma), _ptr(W1_0), _ptr(W2_0), _ptr(O), _ptr(W1_final),
                           _ptr(W2_final), _ptr(W1_chunks), _ptr(W2_chunks), _ptr(workspace),
@@ -198,6 +214,7 @@ def ttt_mlp_fwd(cfg, hidden, Q, K, V, beta, gamma, W1_0, W2_0, O, W1_final, W2_f
 
 def ttt_mlp_bwd(cfg, hidden, Q, K, V, beta, gamma, W1_chunks, W2_chunks, dO, dW1_final, dW2_final,
                 dQ, dK, dV, dbeta, dW1_0, dW2_0, workspace, workspace_bytes, stream=None):
+    """TTT-MLP backward for J = <dO, O> + <dW1_final, W1_final> + <dW2_final, W2_final>."""
     st = _lib.ttt_mlp_bwd(ctypes.byref(cfg), int(hidden), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
                           _ptr(gamma), _ptr(W1_chunks), _ptr(W2_chunks), _ptr(dO), _ptr(dW1_final),
                           _ptr(dW2_final), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta), _ptr(dW1_0),
@@ -214,6 +231,11 @@ def inplace_ttt_workspace_bytes(T, d_ff, d_model, C) -> int:
 
 def inplace_ttt_fwd(T, d_ff, d_model, C, lr, Z, Vhat, W, O, workspace=None, workspace_bytes=0,
                     stream=None, W_chunks=None):
+    """In-Place TTT forward: per chunk of C tokens O_i = Z_i W^T, then W += lr Vhat_i^T Z_i.
+
+    Z [T,d_ff] and Vhat [T,d_model] bf16; W [d_model,d_ff] float32 in/out; O [T,d_model] bf16;
+    W_chunks [T/C,d_model,d_ff] bf16 (optional) keeps the weight each chunk applied, for
+    inplace_ttt_bwd. Workspace: inplace_ttt_workspace_bytes(T, d_ff, d_model, C)."""
     st = _lib.inplace_ttt_fwd(T, d_ff, d_model, C, float(lr), _ptr(Z), _ptr(Vhat), _ptr(W),
                               _ptr(O), _ptr(W_chunks), _ptr(workspace), int(workspace_bytes),
                               _stream(stream))
@@ -282,6 +304,9 @@ def inplace_ttt_target_bwd(T, d_model, k, X0, conv_w, W_target, dVhat, dX0, dcon
 
 def inplace_ttt_bwd(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ, dVhat, dW,
                     workspace=None, workspace_bytes=0, stream=None):
+    """In-Place TTT backward for J = sum_i <dO_i, O_i> + <dW_final, W_final> (dW_final may
+    be None): writes dZ [T,d_ff] and dVhat [T,d_model] bf16 and dW, the float32 gradient of the
+    initial W, from the forward's W_chunks."""
     st = _lib.inplace_ttt_bwd(T, d_ff, d_model, C, float(lr), _ptr(Z), _ptr(Vhat), _ptr(W_chunks),
                               _ptr(dO), _ptr(dW_final), _ptr(dZ), _ptr(dVhat), _ptr(dW),
                               _ptr(workspace), int(workspace_bytes), _stream(stream))
