@@ -153,10 +153,10 @@ def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None,
     """Forward of the chunkwise TTT layer on the current device and stream.
 
     Q, K [B,H,T,dk]; V, O [B,H,T,dv] in cfg's dtype; beta [B,H,T] and W0, W_final [B,H,dk,dv]
-    float32; gamma [B,H,T] or [B,H,T,dk] float32, or None (no decay). W_chunks [B,H,T/C,dk,dv]
-    in cfg's dtype
-    and G_saved (ttt_saved_bytes) are optional outputs that ttt_chunk_bwd reads. Workspace:
-    ttt_workspace_bytes(cfg, 0) bytes. Raises TTTError on a non-OK status."""
+    float32; gamma [B,H,T] or [B,H,T,dk] float32, or None (no decay). W_chunks
+    [B,H,T/C,dk,dv] in cfg's dtype and G_saved (ttt_saved_bytes) are optional outputs that
+    ttt_chunk_bwd reads. Workspace: ttt_workspace_bytes(cfg, 0) bytes. Raises TTTError on a
+    non-OK status."""
     st = _lib.ttt_chunk_fwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
                             _ptr(W0), _ptr(O), _ptr(W_final), _ptr(W_chunks), _ptr(G_saved),
                             _ptr(workspace), int(workspace_bytes), _stream(stream))
