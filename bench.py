@@ -171,7 +171,8 @@ class Layer:
         self.Wf = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
         self.Wc = torch.empty((B, H, T // C, dk, dv), device=dev, dtype=sd)
         # saved by fwd for bwd: G, and with SiLU also Zq (the readout before the activation)
-        self.G = torch.empty((2 if cfg.act == "silu" else 1, B, H, T, dv), device=dev, dtype=sd)
+        planes = ttt.ttt_saved_bytes(self.c) // (B * H * T * dv * sd.itemsize)
+        self.G = torch.empty((planes, B, H, T, dv), device=dev, dtype=sd)
         self.dQ = torch.empty((B, H, T, dk), device=dev, dtype=sd)
         self.dK = torch.empty((B, H, T, dk), device=dev, dtype=sd)
         self.dV = torch.empty((B, H, T, dv), device=dev, dtype=sd)
@@ -538,6 +539,92 @@ def replica_throughput(local_ms: float, steps: int, tokens_per_rank: int, world:
     return ms, world * tokens_per_rank / (ms * 1e-3)
 
 
+# ---------------------------------------------------------------------- profiling cases
+PROFILE_CASES = {
+    # name: what it launches (one small call each, sized for an ncu capture of a few GB at most)
+    "train-1.45b-quarter": "the training step on a quarter of the 1.45B batch (B=1): the forward "
+                           "kernel and the chain, dQ and dK kernels of the backward",
+    "bwd-rebuild-g": "the backward without the forward's saved G (B=4, H=16, T=2048): the G "
+                     "kernel, then chain, dQ, dK",
+    "silu-bwd": "SiLU + MSE forward and backward (B=2, H=16, T=2048): the dZq and SiLU-factor "
+                "kernels, then chain, dQ, dK in SiLU mode",
+    "ntp-target": "the NTP target and its backward (T=32768, d_model=2560, k=4): the convolution "
+                  "kernels and the projection GEMMs",
+    "vector-decay": "vector decay forward and backward on the SIMT kernels (B=1, H=4, T=512, "
+                    "d=64, C=256)",
+    "ttt-mlp": "TTT-MLP forward and backward on the SIMT kernels (B=1, H=4, T=512, d=64, hidden "
+               "256, C=256)",
+}
+
+
+def run_case(name, ttt):
+    """One warm-up call and one call of a small workload that exercises the named kernels, for
+    profiling with ncu (-k selects the kernel). Prints one line when done."""
+    torch.cuda.set_device(0)
+    if name in ("train-1.45b-quarter", "bwd-rebuild-g", "silu-bwd"):
+        cfg = {"train-1.45b-quarter": synth.TRAIN_1P45B.replace(B=1),
+               "bwd-rebuild-g": synth.TRAIN_1P45B.replace(T=2048),
+               "silu-bwd": synth.SILU_IP_FWD.replace(B=2, T=2048, loss="mse")}[name]
+        layer = Layer(cfg, ttt, seed=cfg.seed)
+        for _ in range(2):
+            layer.fwd()
+            if name == "bwd-rebuild-g":
+                i = layer.inp
+                ttt.ttt_chunk_bwd(layer.c, i["Q"], i["K"], i["V"], i["beta"], i["gamma"], i["W0"],
+                                  layer.Wc, None, i["dO"], i["dW_T"], None, None, layer.dQ,
+                                  layer.dK, layer.dV, layer.dbeta, layer.dW0, None, layer.ws,
+                                  layer.ws.numel())
+            else:
+                layer.bwd()
+    elif name == "ntp-target":
+        icfg, k = synth.INPLACE_QWEN4B, 4
+        tin = synth.inplace_target_inputs(icfg, k, device="cuda")
+        T, d = icfg.T, icfg.d_model
+        Vh = torch.empty((T, d), device="cuda", dtype=torch.bfloat16)
+        n = ttt.inplace_ttt_target_workspace_bytes(T, d)
+        nb = ttt.inplace_ttt_target_bwd_workspace_bytes(T, d, k)
+        ws = torch.empty(max(n, nb, 16), device="cuda", dtype=torch.uint8)
+        dX0 = torch.empty_like(tin["X0"])
+        dcw = torch.empty_like(tin["conv_w"])
+        dWt = torch.empty((d, d), device="cuda")
+        for _ in range(2):
+            ttt.inplace_ttt_target(T, d, k, tin["X0"], tin["conv_w"], tin["W_target"], Vh, ws, n)
+            ttt.inplace_ttt_target_bwd(T, d, k, tin["X0"], tin["conv_w"], tin["W_target"],
+                                       tin["dVhat"], dX0, dcw, dWt, ws, nb)
+    elif name == "vector-decay":
+        cfg = synth.FWD_410M.replace(B=1, H=4, T=512, decay="vector")
+        layer = Layer(cfg, ttt, seed=cfg.seed)
+        for _ in range(2):
+            layer.fwd()
+            layer.bwd()
+    elif name == "ttt-mlp":
+        cfg, hid = synth.TTT_MLP_410M.replace(B=1, H=4, T=512), synth.TTT_MLP_HIDDEN
+        inp = synth.ttt_inputs(cfg, device="cuda")
+        w = synth.ttt_mlp_weights(cfg, hid, device="cuda")
+        c = ttt.make_config(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C, cfg.dtype, cfg.loss,
+                            cfg.act, cfg.lr_bias)
+        B, H, T, dk, dv, C = cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C
+        O = torch.empty((B, H, T, dv), device="cuda", dtype=torch.bfloat16)
+        W1f, W2f = torch.empty_like(w["W1"]), torch.empty_like(w["W2"])
+        W1c = torch.empty((B, H, T // C, dk, hid), device="cuda")
+        W2c = torch.empty((B, H, T // C, hid, dv), device="cuda")
+        n = ttt.ttt_mlp_workspace_bytes(c, hid)
+        ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+        g = [torch.empty_like(inp["Q"]), torch.empty_like(inp["K"]), torch.empty_like(inp["V"]),
+             torch.empty_like(inp["beta"]), torch.empty_like(w["W1"]), torch.empty_like(w["W2"])]
+        for _ in range(2):
+            ttt.ttt_mlp_fwd(c, hid, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"],
+                            w["W1"], w["W2"], O, W1f, W2f, W1c, W2c, ws, n)
+            ttt.ttt_mlp_bwd(c, hid, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], W1c,
+                            W2c, inp["dO"], None, None, *g, ws, n)
+    else:
+        raise SystemExit(f"unknown case {name}; one of {sorted(PROFILE_CASES)}")
+    torch.cuda.synchronize()
+    if ttt.ttt_get_device_error() != ttt.OK:
+        raise SystemExit("device error word set")
+    print(f"case {name} done")
+
+
 def main():
     global _dist
     ap = argparse.ArgumentParser()
@@ -550,7 +637,13 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the throughput lines of the other workloads")
+    ap.add_argument("--case", choices=sorted(PROFILE_CASES),
+                    help="run one small call of a kernel family for profiling, and exit")
     args = ap.parse_args()
+    if args.case:
+        import weight_sequence_layers_b200 as ttt
+        run_case(args.case, ttt)
+        return
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -646,10 +739,12 @@ def main():
         icfg, ims, ims_save, ims_bwd, (ims_tgt, ims_tgt_bwd) = time_inplace(ttt, steps=3, warmup=3)
         fl, by = inplace_work(icfg)
         tf = fl / (ims * 1e-3) / 1e12
+        # these calls are timed alone (a few launches of a few ms each, not a seconds-long
+        # loop under the power cap), so the burst figure of the measured GEMM is the peak
         out["inplace"] = {"workload": icfg.name, "ms": ims, "tokens_per_s": icfg.T / (ims * 1e-3),
                           "roofline": {"bound": "tensor", "achieved": tf,
-                                       "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                                       "frac": tf / peaks["bf16_tflops_sustained"],
+                                       "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                       "frac": tf / peaks["bf16_tflops"],
                                        "traffic": measured_traffic("inplace_chunk", icfg.name),
                                        "traffic_unit": "bytes per chunk launch",
                                        "peak_source": peak_src},
@@ -660,27 +755,27 @@ def main():
         out["inplace_bwd"] = {"workload": icfg.name.replace("-fwd", "-bwd"), "ms": ims_bwd,
                               "tokens_per_s": icfg.T / (ims_bwd * 1e-3),
                               "roofline": {"bound": "tensor", "achieved": tfb,
-                                           "peak": peaks["bf16_tflops_sustained"],
+                                           "peak": peaks["bf16_tflops"],
                                            "unit": "TFLOP/s",
-                                           "frac": tfb / peaks["bf16_tflops_sustained"],
+                                           "frac": tfb / peaks["bf16_tflops"],
                                            "peak_source": peak_src}}
         # NTP target: 2 T d_model^2 flops of projection (the 4-tap convolution is HBM work)
         tft = 2 * icfg.T * icfg.d_model ** 2 / (ims_tgt * 1e-3) / 1e12
         out["inplace_target"] = {"workload": "inplace-ttt-ntp-target-k4", "ms": ims_tgt,
                                  "tokens_per_s": icfg.T / (ims_tgt * 1e-3),
                                  "roofline": {"bound": "tensor", "achieved": tft,
-                                              "peak": peaks["bf16_tflops_sustained"],
+                                              "peak": peaks["bf16_tflops"],
                                               "unit": "TFLOP/s",
-                                              "frac": tft / peaks["bf16_tflops_sustained"],
+                                              "frac": tft / peaks["bf16_tflops"],
                                               "peak_source": peak_src}}
         # its backward: dY = dVhat W_target^T and dW_target = Y^T dVhat, 4 T d_model^2 flops
         tftb = 4 * icfg.T * icfg.d_model ** 2 / (ims_tgt_bwd * 1e-3) / 1e12
         out["inplace_target_bwd"] = {"workload": "inplace-ttt-ntp-target-k4-bwd", "ms": ims_tgt_bwd,
                                      "tokens_per_s": icfg.T / (ims_tgt_bwd * 1e-3),
                                      "roofline": {"bound": "tensor", "achieved": tftb,
-                                                  "peak": peaks["bf16_tflops_sustained"],
+                                                  "peak": peaks["bf16_tflops"],
                                                   "unit": "TFLOP/s",
-                                                  "frac": tftb / peaks["bf16_tflops_sustained"],
+                                                  "frac": tftb / peaks["bf16_tflops"],
                                                   "peak_source": peak_src}}
     # the pages' own number: context, not a target (no hardware stated, not re-runnable here)
     out["pages_claim"] = {"ratio": "2.2-3.3x the training throughput of the official TTT "

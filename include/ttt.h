@@ -36,8 +36,15 @@
  *    ready when the stream reaches that point.
  *  - Argument checks run on the host before anything is launched. On any error nothing
  *    is launched and no output is touched. Device pointers must be 16-byte aligned.
- *  - No exceptions cross the ABI; the library keeps no per-call state, so calls on
- *    different streams may overlap provided their buffers do not alias.
+ *  - No exceptions cross the ABI and the library keeps no per-call state: calls on different
+ *    streams may overlap provided their buffers do not alias, with one exception. The
+ *    tensor-core path of ttt_chunk_bwd forks the caller's stream onto two library-owned
+ *    streams of the current device (it runs its serial adjoint kernel beside a chunk-parallel
+ *    one) and joins them back into the caller's stream before returning; these streams and four
+ *    events are created by the first such call on each device and shared by every later call,
+ *    under a process-wide lock. Backward calls from different streams or host threads therefore
+ *    serialise on the GPU, and the first tensor-core backward on a device should come before
+ *    any stream capture.
  *  - Kernels never trap. Every wait inside a kernel is bounded; a wait that runs out
  *    sets a per-device error word and the kernel returns early (outputs then invalid).
  *    ttt_get_device_error() reports and clears it.
@@ -120,7 +127,8 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
  *  in : Q, K, V, beta, gamma (nullable), W0, W_chunks (from ttt_chunk_fwd, required),
  *       G_saved (from ttt_chunk_fwd, nullable: rebuilt from W_chunks when NULL; kernels that
  *       rebuild G anyway may ignore it; with SiLU the tensor-core backward needs it, for Zq,
- *       and a call without it runs on the SIMT kernels), dO, dW_final (nullable = 0);
+ *       and a SiLU call on a tensor-core shape without it returns TTT_ERR_UNSUPPORTED),
+ *       dO, dW_final (nullable = 0);
  *       O and W_final (the forward's outputs) are read only for dgamma (then O is required,
  *       and W_final too when dW_final is non-NULL).
  *  out: dQ, dK, dV, dbeta, dW0 (plain stores, not accumulated); dgamma (nullable; requires
@@ -145,8 +153,9 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
  * that owns every byte of device memory through its own pool, or a plugin that is handed only
  * its input and output buffers. For them this variant takes the same arguments as
  * ttt_chunk_bwd minus the workspace, and keeps its scratch (the per-chunk adjoint states and
- * the bf16 inner-loss gradient G of every token) in a fixed array of TTT_NOALLOC_SCRATCH_BYTES that the library holds on every GPU it is loaded
- * on, until the process exits. It allocates nothing and calls no allocating routine.
+ * the bf16 inner-loss gradient G of every token) in a fixed array of TTT_NOALLOC_SCRATCH_BYTES
+ * that the library holds on every GPU it is loaded on, until the process exits. It allocates no
+ * device memory and calls no allocating routine.
  *  - Only configs of the tensor-core backward are accepted (bf16, dk == dv in {64, 128},
  *    C in {128, 256}, scalar or no decay; SiLU only with G_saved); others return
  *    TTT_ERR_UNSUPPORTED.
@@ -154,7 +163,9 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
  *    G_saved is NULL, plus B*H*T*4 when dgamma is non-NULL, plus 4*B*H*T*dv*2 with SiLU) return
  *    TTT_ERR_WORKSPACE with nothing launched; ttt_chunk_bwd serves those.
  *  - The first call on a device looks up the array's device address (with that device
- *    current); make that first call before any stream capture.
+ *    current) and, unless a ttt_chunk_bwd call on the tensor cores ran there before, creates
+ *    the library's two fork streams and four events of that device (see the stream conventions
+ *    at the top): make that first call before any stream capture. Later calls create nothing.
  *  - Every call shares the one array and leaves its contents behind. Calls that overlap on
  *    the GPU (different streams, or different host threads) race on it: serialise them.
  *    Nothing in the array has to start at zero. */

@@ -30,8 +30,8 @@ def run_fwd(cfg, inp, save_g=True, save_w=True):
     O = torch.empty((B, H, T, dv), device="cuda", dtype=sd)
     Wf = torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32)
     Wc = torch.empty((B, H, T // C, dk, dv), device="cuda", dtype=sd) if save_w else None
-    # with SiLU the saved buffer holds G, then Zq (the readout before the activation)
-    planes = 2 if cfg.act == "silu" else 1
+    # the saved buffer holds G, then with SiLU Zq (the readout before the activation)
+    planes = ttt.ttt_saved_bytes(c) // (B * H * T * dv * sd.itemsize)
     Gs = torch.empty((planes, B, H, T, dv), device="cuda", dtype=sd) if save_g else None
     n = ttt.ttt_workspace_bytes(c, 0)
     ws = torch.empty(max(n, 16), device="cuda", dtype=torch.uint8)

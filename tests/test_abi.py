@@ -55,7 +55,8 @@ def _cfg(**kw):
 def test_workspace_query_validates_config():
     assert ttt.ttt_workspace_bytes(_cfg(), 0) == 0
     assert ttt.ttt_workspace_bytes(_cfg(), 1) > 0
-    # the tensor-core backward keeps G in its workspace only when the forward's G is not passed
+    # the tensor-core backward keeps G in its workspace only when the forward's saved tensors
+    # are not passed
     tc = _cfg(dtype="bf16", dk=128, dv=128, C=256, T=512)
     assert 0 < ttt.ttt_workspace_bytes(tc, 2) < ttt.ttt_workspace_bytes(tc, 1)
     with pytest.raises(ttt.TTTError):
@@ -131,6 +132,15 @@ def test_decay_kind_is_checked_and_vector_decay_leaves_the_tensor_core_path():
     st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(vec), A, A, A, A, A, A, A, None, A, None, None,
                                        None, A, A, A, A, A, None, None)
     assert st == ttt.ERR_UNSUPPORTED
+    # a valid config that no backward path serves (dk = dv = 256) is unsupported, not invalid;
+    # an invalid one is invalid
+    wide = _cfg(dtype="bf16", dk=256, dv=256, C=256, T=512)
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(wide), A, A, A, A, A, A, A, None, A, None, None,
+                                       None, A, A, A, A, A, None, None)
+    assert st == ttt.ERR_UNSUPPORTED
+    st = ttt.lib.ttt_chunk_bwd_noalloc(ctypes.byref(_cfg(T=250)), A, A, A, A, A, A, A, None, A, None,
+                                       None, None, A, A, A, A, A, None, None)
+    assert st == ttt.ERR_INVALID_ARG
 
 
 def test_tc_bwd_workspace_covers_the_decay_gradient():
@@ -450,5 +460,20 @@ def test_tensor_core_backward_workspace_is_the_documented_sum(act, d, C):
     adj, G, dg = B * H * (T // C) * d * d * 2, B * H * T * d * 2, B * H * T * 4
     planes = 4 * B * H * T * d * 2 if act == "silu" else 0
     assert ttt.ttt_workspace_bytes(cfg, 2) == adj + dg + planes
-    if act == "id":  # the SiLU backward without the forward's G and Zq runs on SIMT kernels
+    if act == "id":
         assert ttt.ttt_workspace_bytes(cfg, 1) == adj + G + dg
+    else:  # the SiLU backward without the forward's G and Zq is refused on these shapes
+        with pytest.raises(ttt.TTTError):
+            ttt.ttt_workspace_bytes(cfg, 1)
+
+
+def test_silu_tensor_core_backward_without_saved_tensors_is_refused():
+    # a SiLU backward on a tensor-core shape needs the forward's G and Zq; without them the call
+    # returns TTT_ERR_UNSUPPORTED before anything is launched (the pointers are never read)
+    cfg = _cfg(dtype="bf16", dk=128, dv=128, C=256, T=512, act="silu")
+    A = 4096
+    ws = ttt.ttt_workspace_bytes(cfg, 2)
+    args = [A] * 7 + [None, A, None, None, None] + [A] * 5 + [None]  # ... G_saved = NULL ...
+    assert ttt.lib.ttt_chunk_bwd(ctypes.byref(cfg), *args, A, ws, None) == ttt.ERR_UNSUPPORTED
+    # with G_saved the same call passes the host checks (it would launch; not run here)
+    assert ttt.ttt_workspace_bytes(cfg, 2) > 0

@@ -39,6 +39,9 @@ def test_tc_backward_small(shape, loss, decay, saved_g):
 
 
 def test_tc_backward_full_size_sampled_heads():
+    # The whole 16-chunk sequence of the 1.45B workload. The chunk-start states the backward
+    # rebuilds Z and G from are stored in bf16 (W_chunks has the storage dtype); the errors
+    # below show how much of the 2e-2 budget that and the bf16 operands use after 16 chunks.
     cfg = synth.TRAIN_1P45B
     inp = synth.ttt_inputs(cfg, device="cuda")
     fwd = run_fwd(cfg, inp)
@@ -47,9 +50,14 @@ def test_tc_backward_full_size_sampled_heads():
     heads = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(2)]
     sub = head_slice(inp, heads)
     ref = oracle_bwd(cfg.replace(B=1, H=len(heads)), sub)
+    errs = {}
     for k in GRADS + ("dgamma",):
         g = torch.stack([got[k][b, h] for b, h in heads]).unsqueeze(0)
-        assert rel_err(g, ref[k]) <= TOL, (k, rel_err(g, ref[k]))
+        errs[k] = rel_err(g, ref[k])
+    print("full-length backward errors (max|d| / max|ref|, budget 2e-2):",
+          {k: f"{v:.2e}" for k, v in errs.items()})
+    for k, v in errs.items():
+        assert v <= TOL, (k, v)
 
 
 @pytest.mark.parametrize("shape", SHAPES)

@@ -1,8 +1,9 @@
 """ttt_chunk_bwd_noalloc: the backward for callers that cannot allocate device memory when they
 call the library (a host framework that owns all device memory, a plugin handed only its
-buffers). It must give the same gradients as ttt_chunk_bwd with a caller workspace, on two
-calls in a row that share its fixed scratch array, and refuse configs whose scratch would not
-fit. This file is collected last on purpose."""
+buffers). It must give the same gradients as ttt_chunk_bwd with a caller workspace, bit for
+bit, on consecutive calls that share its fixed scratch array (each call finds the bytes the
+previous one left behind), and refuse configs whose scratch would not fit. This file is
+collected last on purpose."""
 import ctypes
 
 import pytest
@@ -43,31 +44,30 @@ def noalloc_bwd(cfg, inp, W_chunks, G, fwd):
     return out
 
 
-def test_noalloc_backward_matches_the_workspace_backward_on_two_calls():
-    # scratch needed: 4 heads x 4 chunks x 128 x 128 x 2 bytes = 512 KiB, plus 1 MiB of G when the
-    # forward's G is not passed, plus 16 KiB for dgamma (limit 8 MiB); the first call passes G,
-    # the second does not
-    cfg = synth.TRAIN_1P45B.replace(B=1, H=4, T=1024)
-    for seed, saved_g in ((21, True), (22, False)):
-        inp = synth.ttt_inputs(cfg, device="cuda", seed=seed)
-        inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(seed))
-        fwd = run_fwd(cfg, inp, save_g=saved_g)
-        ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
-        got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd)
-        for k in GRADS:
-            assert rel_err(got[k], ref[k]) <= TOL, (seed, k)
-
-
-def test_noalloc_backward_silu():
-    # SiLU reads Zq from G_saved; its scratch adds four bf16 planes (4 MiB here, limit 8 MiB)
-    cfg = synth.SILU_IP_FWD.replace(B=1, H=4, T=1024, loss="mse")
-    inp = synth.ttt_inputs(cfg, device="cuda", seed=23)
-    inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(23))
-    fwd = run_fwd(cfg, inp)
-    ref = run_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
-    got = noalloc_bwd(cfg, inp, fwd["W_chunks"], fwd["G_saved"], fwd)
+def _same(got, ref, where):
+    # the same kernels on the same inputs (no atomics): the results agree bit for bit
     for k in GRADS:
-        assert rel_err(got[k], ref[k]) <= TOL, k
+        assert torch.equal(got[k], ref[k]), (where, k, rel_err(got[k], ref[k]))
+        assert rel_err(got[k], ref[k]) <= TOL, (where, k)
+
+
+def test_noalloc_backward_matches_the_workspace_backward_call_after_call():
+    # Scratch needed (limit 8 MiB): 4 heads x 4 chunks x 128 x 128 x 2 bytes = 512 KiB of
+    # chunk-end adjoints, plus 1 MiB of G when the forward's saved tensors are not passed, plus
+    # 16 KiB for dgamma, plus 4 MiB of SiLU planes. The calls run in an order that makes each
+    # one start from the bytes an earlier call of another kind left behind: without the saved
+    # tensors (fills the G region), with them, SiLU (fills the four planes), then without them
+    # again, and the first one once more.
+    cfg = synth.TRAIN_1P45B.replace(B=1, H=4, T=1024)
+    silu = synth.SILU_IP_FWD.replace(B=1, H=4, T=1024, loss="mse")
+    plan = [(cfg, 21, False), (cfg, 22, True), (silu, 23, True), (cfg, 24, False), (cfg, 21, False)]
+    for c, seed, saved in plan:
+        inp = synth.ttt_inputs(c, device="cuda", seed=seed)
+        inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(seed))
+        fwd = run_fwd(c, inp, save_g=saved)
+        ref = run_bwd(c, inp, fwd["W_chunks"], fwd["G_saved"], fwd=fwd)
+        got = noalloc_bwd(c, inp, fwd["W_chunks"], fwd["G_saved"], fwd)
+        _same(got, ref, (c.name, seed, saved))
 
 
 def test_noalloc_backward_refuses_configs_beyond_its_scratch():

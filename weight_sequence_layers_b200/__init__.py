@@ -148,6 +148,18 @@ def ttt_workspace_bytes(cfg: ttt_config, for_bwd: int) -> int:
     return n
 
 
+def _check_size(t, nbytes: int, name: str):
+    """A buffer the library fills or reads for this config must hold nbytes; the C ABI cannot
+    tell, and a short buffer would be written past its end."""
+    if t is not None and not isinstance(t, int) and t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, the config needs "
+                         f"{nbytes}")
+
+
+def _chunks_bytes(cfg) -> int:
+    return cfg.B * cfg.H * (cfg.T // cfg.C) * cfg.dk * cfg.dv * (2 if cfg.dtype == BF16 else 4)
+
+
 def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None, G_saved=None,
                   workspace=None, workspace_bytes=0, stream=None):
     """Forward of the chunkwise TTT layer on the current device and stream.
@@ -157,6 +169,10 @@ def ttt_chunk_fwd(cfg, Q, K, V, beta, gamma, W0, O, W_final=None, W_chunks=None,
     [B,H,T/C,dk,dv] in cfg's dtype and G_saved (ttt_saved_bytes) are optional outputs that
     ttt_chunk_bwd reads. Workspace: ttt_workspace_bytes(cfg, 0) bytes. Raises TTTError on a
     non-OK status."""
+    if G_saved is not None:
+        _check_size(G_saved, ttt_saved_bytes(cfg), "G_saved")
+    if W_chunks is not None:
+        _check_size(W_chunks, _chunks_bytes(cfg), "W_chunks")
     st = _lib.ttt_chunk_fwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
                             _ptr(W0), _ptr(O), _ptr(W_final), _ptr(W_chunks), _ptr(G_saved),
                             _ptr(workspace), int(workspace_bytes), _stream(stream))
@@ -171,6 +187,8 @@ def ttt_chunk_bwd(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final
     None), and writes dQ, dK, dV, dbeta, dW0 and, when dgamma is given, the decay gradient
     (which also needs the forward's O, and W_final when dW_final is given). Workspace:
     ttt_workspace_bytes(cfg, 2 if G_saved is passed else 1) bytes."""
+    if G_saved is not None:
+        _check_size(G_saved, ttt_saved_bytes(cfg), "G_saved")
     st = _lib.ttt_chunk_bwd(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta), _ptr(gamma),
                             _ptr(W0), _ptr(W_chunks), _ptr(G_saved), _ptr(dO), _ptr(dW_final),
                             _ptr(O), _ptr(W_final), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(dbeta),
@@ -185,6 +203,8 @@ NOALLOC_SCRATCH_BYTES = 8 << 20
 def ttt_chunk_bwd_noalloc(cfg, Q, K, V, beta, gamma, W0, W_chunks, G_saved, dO, dW_final, O,
                           W_final, dQ, dK, dV, dbeta, dW0, dgamma, stream=None):
     """ttt_chunk_bwd for callers that cannot allocate: scratch is the library's fixed array."""
+    if G_saved is not None:
+        _check_size(G_saved, ttt_saved_bytes(cfg), "G_saved")
     st = _lib.ttt_chunk_bwd_noalloc(ctypes.byref(cfg), _ptr(Q), _ptr(K), _ptr(V), _ptr(beta),
                                     _ptr(gamma), _ptr(W0), _ptr(W_chunks), _ptr(G_saved),
                                     _ptr(dO), _ptr(dW_final), _ptr(O), _ptr(W_final), _ptr(dQ),

@@ -46,6 +46,8 @@ unsigned* error_word(cudaError_t* e) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+}  // namespace
+
 // Checks the config; returns TTT_OK or the first failure.
 ttt_status check_config(const ttt_config* c) {
   if (!c) return TTT_ERR_INVALID_ARG;
@@ -63,6 +65,8 @@ ttt_status check_config(const ttt_config* c) {
   if ((long long)c->B * c->H * c->T >= (1ll << 31)) return TTT_ERR_INVALID_ARG;
   return TTT_OK;
 }
+
+namespace {
 
 LayerArgs args_of(const ttt_config* c) {
   LayerArgs a{};
@@ -87,10 +91,12 @@ Path fwd_path(const LayerArgs& a) {
   if (simt_supported(a)) return PATH_SIMT;
   return PATH_NONE;
 }
-// The tensor-core backward with SiLU reads the forward's Zq, saved beside G.
+// The tensor-core backward with SiLU reads the forward's Zq, saved beside G. A SiLU call on a
+// tensor-core shape without it is refused rather than sent to the SIMT kernels, which would
+// take several hundred times longer for the same result.
 Path bwd_path(const LayerArgs& a, bool g_saved) {
-  if (a.dtype == TTT_BF16 && tc_bwd_supported(a) && (a.act == TTT_ACT_ID || g_saved))
-    return PATH_TC;
+  if (a.dtype == TTT_BF16 && tc_bwd_supported(a))
+    return a.act == TTT_ACT_ID || g_saved ? PATH_TC : PATH_NONE;
   if (simt_supported(a)) return PATH_SIMT;
   return PATH_NONE;
 }

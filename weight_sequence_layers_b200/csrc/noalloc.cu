@@ -10,6 +10,9 @@
 #include "kernels.h"
 
 namespace tttk {
+
+ttt_status check_config(const ttt_config* c);  // api.cu
+
 namespace {
 
 // The scratch of every ttt_chunk_bwd_noalloc call on this device. In host code this name is
@@ -48,7 +51,8 @@ extern "C" ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q
                                             const float* W_final, void* dQ, void* dK, void* dV,
                                             float* dbeta, float* dW0, float* dgamma,
                                             void* stream) {
-  if (ttt_workspace_bytes(cfg, 1) == (size_t)-1) return TTT_ERR_INVALID_ARG;
+  const ttt_status cs = check_config(cfg);
+  if (cs != TTT_OK) return cs;
   if (!Q || !K || !V || !beta || !W0 || !W_chunks || !dO || !dQ || !dK || !dV || !dbeta || !dW0)
     return TTT_ERR_INVALID_ARG;
   if (dgamma && (!gamma || !O || (dW_final && !W_final))) return TTT_ERR_INVALID_ARG;
