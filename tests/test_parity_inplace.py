@@ -135,7 +135,7 @@ def run_target(T, d, k, tin):
     return V
 
 
-@pytest.mark.parametrize("T,d,k", [(256, 128, 1), (512, 256, 4), (384, 384, 8), (128, 640, 3)])
+@pytest.mark.parametrize("T,d,k", [(256, 128, 1), (256, 128, 2), (512, 256, 4), (384, 384, 8), (128, 640, 3)])
 def test_inplace_target_small(T, d, k):
     cfg = synth.INPLACE_QWEN4B.replace(T=T, d_model=d)
     tin = synth.inplace_target_inputs(cfg, k=k, device="cuda", seed=T + d + k)
@@ -170,7 +170,7 @@ def run_target_bwd(T, d, k, tin):
     return dict(dX0=dX0, dconv_w=dw, dW_target=dWt)
 
 
-@pytest.mark.parametrize("T,d,k", [(256, 128, 1), (512, 256, 4), (384, 384, 8), (128, 640, 3)])
+@pytest.mark.parametrize("T,d,k", [(256, 128, 1), (256, 128, 2), (512, 256, 4), (384, 384, 8), (128, 640, 3)])
 def test_inplace_target_backward_small(T, d, k):
     cfg = synth.INPLACE_QWEN4B.replace(T=T, d_model=d)
     tin = synth.inplace_target_inputs(cfg, k=k, device="cuda", seed=2 * T + d + k)
