@@ -207,7 +207,10 @@ def _path(cfg, call):
     always hands the backward the forward's saved G, and Zq with SiLU)."""
     tc_shape = cfg.dtype == "bf16" and cfg.decay != "vector" and cfg.dk == cfg.dv and \
         cfg.dk in (64, 128) and cfg.C in (128, 256)
-    return "tcgen05" if tc_shape else "simt"
+    # the vector decay's forward (identity activation, d = 64) runs on the tensor cores too
+    tc_vec_fwd = call == "ttt_chunk_fwd" and cfg.dtype == "bf16" and cfg.decay == "vector" and \
+        cfg.act == "id" and cfg.dk == cfg.dv == 64 and cfg.C in (128, 256)
+    return "tcgen05" if tc_shape or tc_vec_fwd else "simt"
 
 
 def _event_ms(fn, steps, warmup):
@@ -550,8 +553,10 @@ PROFILE_CASES = {
                 "kernels, then chain, dQ, dK in SiLU mode",
     "ntp-target": "the NTP target and its backward (T=32768, d_model=2560, k=4): the convolution "
                   "kernels and the projection GEMMs",
-    "vector-decay": "vector decay forward and backward on the SIMT kernels (B=1, H=4, T=512, "
-                    "d=64, C=256)",
+    "vector-decay": "vector decay forward (tensor cores) and backward (SIMT kernels), B=1, H=4, "
+                    "T=512, d=64, C=256",
+    "vector-decay-fwd-410m": "the vector-decay forward on the 410M shape (B=8, H=16, T=2048, "
+                             "d=64, C=256): the state and readout kernels",
     "ttt-mlp": "TTT-MLP forward and backward on the SIMT kernels (B=1, H=4, T=512, d=64, hidden "
                "256, C=256)",
 }
@@ -597,6 +602,11 @@ def run_case(name, ttt):
         for _ in range(2):
             layer.fwd()
             layer.bwd()
+    elif name == "vector-decay-fwd-410m":
+        cfg = synth.FWD_410M.replace(decay="vector")
+        layer = Layer(cfg, ttt, seed=cfg.seed)
+        for _ in range(2):
+            layer.fwd()
     elif name == "ttt-mlp":
         cfg, hid = synth.TTT_MLP_410M.replace(B=1, H=4, T=512), synth.TTT_MLP_HIDDEN
         inp = synth.ttt_inputs(cfg, device="cuda")

@@ -65,7 +65,9 @@ typedef enum {
   TTT_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned                        */
   TTT_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than the query returned       */
   TTT_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed             */
-  TTT_ERR_TIMEOUT = 6       /* a bounded in-kernel wait ran out (device error word)     */
+  TTT_ERR_TIMEOUT = 6,      /* a bounded in-kernel wait ran out (device error word)     */
+  TTT_ERR_RANGE = 7         /* an input left the range a kernel supports (device error
+                               word), e.g. a vector decay too strong for the tensor cores */
 } ttt_status;
 
 typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;    /* type of Q,K,V,O,dO,dQ,dK,dV     */
@@ -116,8 +118,14 @@ size_t ttt_saved_bytes(const ttt_config* cfg);
  *       states, needed by ttt_chunk_bwd; G_saved (nullable) = G of every token (and, with
  *       SiLU, Zq), which ttt_chunk_bwd then reads instead of rebuilding it.
  * bf16 configs with dk == dv in {64, 128}, C in {128, 256} and a scalar decay (or none) run on
- * the tcgen05 kernel; other shapes (dk, dv <= 128, C <= 256), all float32 configs and the
- * vector decay run on the SIMT kernels. */
+ * the tcgen05 kernel. A vector decay with bf16, dk == dv == 64, C in {128, 256} and the
+ * identity activation runs on tcgen05 kernels too: its per-feature weights enter the Q K^T
+ * contraction as operands scaled against a reference token in the middle of each 128-query
+ * block, so each scaled factor spans at most 64 tokens of one feature's decay; a factor beyond
+ * exp(80) (a feature's decay product below e^-80 over 64 tokens) is clamped and reported as
+ * TTT_ERR_RANGE by ttt_get_device_error, and such inputs take the float32 config instead. Other
+ * shapes (dk, dv <= 128, C <= 256), all float32 configs and the other vector-decay configs run
+ * on the SIMT kernels. */
 ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
                          const float* beta, const float* gamma, const float* W0, void* O,
                          float* W_final, void* W_chunks, void* G_saved, void* workspace,
@@ -305,8 +313,9 @@ ttt_status inplace_ttt_bwd(int T, int d_ff, int d_model, int C, float lr, const 
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then returns TTT_ERR_TIMEOUT if any kernel of this library on the
- * current device recorded a bounded wait that ran out since the last call (and clears the
- * word), TTT_ERR_CUDA if the stream reports an error, else TTT_OK. */
+ * current device recorded a bounded wait that ran out since the last call, else TTT_ERR_RANGE
+ * if one recorded an input outside its range (and clears the word), TTT_ERR_CUDA if the stream
+ * reports an error, else TTT_OK. */
 ttt_status ttt_get_device_error(void* stream);
 
 /* Launches a one-warp kernel whose wait on an mbarrier that nothing completes is bounded

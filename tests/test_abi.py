@@ -41,7 +41,7 @@ def test_library_links_no_libcuda():
 
 
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert ttt.status_string(s)
     assert ttt.status_string(99) == "unknown status"
 
@@ -442,10 +442,10 @@ def test_config_struct_matches_the_header():
     assert {k: int(enums["TTT_ACT_" + k.upper()]) for k in ttt.ACT} == ttt.ACT
     assert {k: int(enums["TTT_DECAY_" + k.upper()]) for k in ttt.DECAY} == ttt.DECAY
     names = ["TTT_OK", "TTT_ERR_INVALID_ARG", "TTT_ERR_UNSUPPORTED", "TTT_ERR_ALIGNMENT",
-             "TTT_ERR_WORKSPACE", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT"]
+             "TTT_ERR_WORKSPACE", "TTT_ERR_CUDA", "TTT_ERR_TIMEOUT", "TTT_ERR_RANGE"]
     assert [int(enums[n]) for n in names] == [ttt.OK, ttt.ERR_INVALID_ARG, ttt.ERR_UNSUPPORTED,
                                              ttt.ERR_ALIGNMENT, ttt.ERR_WORKSPACE, ttt.ERR_CUDA,
-                                             ttt.ERR_TIMEOUT]
+                                             ttt.ERR_TIMEOUT, ttt.ERR_RANGE]
     m = re.search(r"#define TTT_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
     assert int(m.group(1)) << int(m.group(2)) == ttt.NOALLOC_SCRATCH_BYTES
 

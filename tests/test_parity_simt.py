@@ -72,9 +72,10 @@ def test_bf16_shapes_outside_the_tensor_core_envelope(loss, act):
 
 
 @pytest.mark.parametrize("loss,act", COMBOS)
-def test_vector_decay_on_tensor_core_shapes_runs_on_simt(loss, act):
-    # bf16, d = 64, C = 256 would take the tensor-core kernels with a scalar decay; a per-feature
-    # decay is served by the SIMT kernels, decay gradient included
+def test_vector_decay_on_tensor_core_shapes(loss, act):
+    # bf16, d = 64, C = 256 with a per-feature decay: the forward runs on the tensor cores with
+    # the identity activation and on the SIMT kernels with SiLU; the backward (decay gradient
+    # included) runs on the SIMT kernels
     cfg = synth.FWD_410M.replace(B=1, H=2, T=512, loss=loss, act=act, decay="vector", w0_std=0.05)
     inp = synth.ttt_inputs(cfg, device="cuda", seed=77)
     inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(4))

@@ -21,7 +21,8 @@ if not os.path.exists(LIB_PATH):
 
 _lib = ctypes.CDLL(LIB_PATH)
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(7)
+(OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT,
+ ERR_RANGE) = range(8)
 F32, BF16 = 0, 1
 LOSS = {"mse": 0, "ip": 1}
 ACT = {"id": 0, "silu": 1}
@@ -334,7 +335,7 @@ def inplace_ttt_bwd(T, d_ff, d_model, C, lr, Z, Vhat, W_chunks, dO, dW_final, dZ
 
 
 def ttt_get_device_error(stream=None) -> int:
-    """Returns the status (OK, ERR_TIMEOUT or ERR_CUDA) instead of raising."""
+    """Returns the status (OK, ERR_TIMEOUT, ERR_RANGE or ERR_CUDA) instead of raising."""
     return _lib.ttt_get_device_error(_stream(stream))
 
 

@@ -84,10 +84,13 @@ LayerArgs args_of(const ttt_config* c) {
   return a;
 }
 
-enum Path { PATH_NONE, PATH_SIMT, PATH_TC };
+enum Path { PATH_NONE, PATH_SIMT, PATH_TC, PATH_TC_VEC };
 
+// The vector decay's forward on the tensor cores needs the decay itself (gamma non-NULL), which
+// the workspace query does not see: it sizes for that case.
 Path fwd_path(const LayerArgs& a) {
   if (a.dtype == TTT_BF16 && tc_fwd_supported(a)) return PATH_TC;
+  if (a.dtype == TTT_BF16 && tc_vec_fwd_supported(a)) return PATH_TC_VEC;
   if (simt_supported(a)) return PATH_SIMT;
   return PATH_NONE;
 }
@@ -176,6 +179,7 @@ const char* ttt_status_string(ttt_status s) {
     case TTT_ERR_WORKSPACE: return "workspace missing or too small";
     case TTT_ERR_CUDA: return "CUDA error";
     case TTT_ERR_TIMEOUT: return "bounded in-kernel wait timed out";
+    case TTT_ERR_RANGE: return "input outside the range the kernel supports";
   }
   return "unknown status";
 }
@@ -184,8 +188,10 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
   if (check_config(cfg) != TTT_OK) return (size_t)-1;
   LayerArgs a = args_of(cfg);
   if (!for_bwd) {
+    a.gamma = reinterpret_cast<const float*>(16);  // a decay is given (never dereferenced)
     switch (fwd_path(a)) {
       case PATH_TC: return tc_fwd_workspace(a);
+      case PATH_TC_VEC: return tc_vec_fwd_workspace(a);
       case PATH_SIMT: return simt_fwd_workspace(a);
       default: return (size_t)-1;
     }
@@ -209,9 +215,12 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a = args_of(cfg);
+  a.gamma = gamma;
   const Path path = fwd_path(a);
   if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
-  const size_t need = path == PATH_TC ? tc_fwd_workspace(a) : simt_fwd_workspace(a);
+  const size_t need = path == PATH_TC       ? tc_fwd_workspace(a)
+                      : path == PATH_TC_VEC ? tc_vec_fwd_workspace(a)
+                                            : simt_fwd_workspace(a);
   if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   cudaError_t e;
   unsigned* err = error_word(&e);
@@ -221,7 +230,9 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
   a.ws_bytes = workspace_bytes;
   a.err = err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launch_status(path == PATH_TC ? tc_fwd(a, s) : simt_fwd(a, s));
+  return launch_status(path == PATH_TC       ? tc_fwd(a, s)
+                       : path == PATH_TC_VEC ? tc_vec_fwd(a, s)
+                                             : simt_fwd(a, s));
 }
 
 ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, const void* V,
@@ -528,7 +539,7 @@ ttt_status ttt_get_device_error(void* stream) {
     const unsigned zero = 0;
     if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
       return TTT_ERR_CUDA;
-    return TTT_ERR_TIMEOUT;
+    return (h & ERR_WAIT_TIMEOUT) ? TTT_ERR_TIMEOUT : TTT_ERR_RANGE;
   }
   return TTT_OK;
 }

@@ -21,8 +21,9 @@
 namespace tttk {
 
 // ------------------------------------------------------------------------------- errors
-// Error codes OR-ed into the per-device error word when a bounded wait runs out.
-enum : unsigned { ERR_WAIT_TIMEOUT = 1u };
+// Error codes OR-ed into the per-device error word: a bounded wait ran out, or an input value
+// left the range a kernel supports (a scaled operand factor beyond what it represents).
+enum : unsigned { ERR_WAIT_TIMEOUT = 1u, ERR_RANGE = 2u };
 
 // Wall-clock limit of one bounded wait (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s

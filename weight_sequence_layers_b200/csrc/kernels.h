@@ -39,6 +39,11 @@ cudaError_t simt_bwd(const LayerArgs& a, cudaStream_t s);
 bool tc_fwd_supported(const LayerArgs& a);
 size_t tc_fwd_workspace(const LayerArgs& a);
 cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s);
+// Vector (per-feature) decay, identity activation, d_k = d_v = 64: a serial state pass and a
+// chunk-parallel readout on the tensor cores.
+bool tc_vec_fwd_supported(const LayerArgs& a);
+size_t tc_vec_fwd_workspace(const LayerArgs& a);
+cudaError_t tc_vec_fwd(const LayerArgs& a, cudaStream_t s);
 bool tc_bwd_supported(const LayerArgs& a);
 size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved, bool dgamma);
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
