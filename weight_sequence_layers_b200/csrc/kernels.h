@@ -39,11 +39,27 @@ cudaError_t simt_bwd(const LayerArgs& a, cudaStream_t s);
 bool tc_fwd_supported(const LayerArgs& a);
 size_t tc_fwd_workspace(const LayerArgs& a);
 cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s);
-// Vector (per-feature) decay, identity activation, d_k = d_v = 64: a serial state pass and a
-// chunk-parallel readout on the tensor cores.
+// Vector (per-feature) decay, identity activation, d_k = d_v = 64: a chunk-parallel pass that
+// forms the decayed operands, a serial state pass and a chunk-parallel readout on the tensor
+// cores.
 bool tc_vec_fwd_supported(const LayerArgs& a);
 size_t tc_vec_fwd_workspace(const LayerArgs& a);
 cudaError_t tc_vec_fwd(const LayerArgs& a, cudaStream_t s);
+
+// The decayed operands of the vector decay, one chunk-parallel pass (chunk-local L, chunk
+// length C = 128 NB, query block qb with reference token m(qb) = 128 qb + 63).
+struct VecPrep {
+  void* Qt;   // bf16 [B H T, 64]: q_s exp(L_s - L_m(qb(s)))
+  void* Kh;   // bf16 [B H T, 64]: k_r exp(L_C - L_r)
+  void* Kt;   // bf16 [B H NC NV 128, 64]: k_r exp(L_m(qb) - L_r) for every qb >= kb(r),
+              // version v = qb (qb + 1) / 2 + kb(r), NV = NB (NB + 1) / 2
+  float* GC;  // float32 [B H NC, 64]: exp(L_C)
+  float* Em;  // float32 [B H NC NB, 64]: exp(L_m(qb))
+  float* Lf;  // nullable: float32 [B H T, 64], L itself
+};
+size_t vec_prep_bytes(const LayerArgs& a, bool with_L);
+VecPrep vec_prep_carve(const LayerArgs& a, void* base, bool with_L);
+cudaError_t vec_prep(const LayerArgs& a, const VecPrep& o, cudaStream_t s);
 bool tc_bwd_supported(const LayerArgs& a);
 size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved, bool dgamma);
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
