@@ -207,10 +207,10 @@ def _path(cfg, call):
     always hands the backward the forward's saved G, and Zq with SiLU)."""
     tc_shape = cfg.dtype == "bf16" and cfg.decay != "vector" and cfg.dk == cfg.dv and \
         cfg.dk in (64, 128) and cfg.C in (128, 256)
-    # the vector decay's forward (identity activation, d = 64) runs on the tensor cores too
-    tc_vec_fwd = call == "ttt_chunk_fwd" and cfg.dtype == "bf16" and cfg.decay == "vector" and \
-        cfg.act == "id" and cfg.dk == cfg.dv == 64 and cfg.C in (128, 256)
-    return "tcgen05" if tc_shape or tc_vec_fwd else "simt"
+    # the vector decay (identity activation, d = 64) runs on the tensor cores too
+    tc_vec = cfg.dtype == "bf16" and cfg.decay == "vector" and cfg.act == "id" and \
+        cfg.dk == cfg.dv == 64 and cfg.C in (128, 256)
+    return "tcgen05" if tc_shape or tc_vec else "simt"
 
 
 def _event_ms(fn, steps, warmup):
@@ -236,6 +236,7 @@ def time_other_configs(ttt, peaks):
             (synth.FWD_410M.name, synth.FWD_410M, False),
             (synth.SILU_IP_FWD.name, synth.SILU_IP_FWD, False),
             ("silu-ip-fwd-bwd", synth.SILU_IP_FWD, True),
+            ("410m-ttt-linear-fwd-bwd", synth.FWD_410M, True),
             ("410m-ttt-linear-vector-decay-fwd-bwd", synth.FWD_410M.replace(decay="vector"), True)]
     res = {}
     for name, cfg, with_bwd in work:
@@ -267,11 +268,19 @@ def time_other_configs(ttt, peaks):
             entry[call] = d
         entry["ms"] = total
         entry["tokens_per_s"] = cfg.B * cfg.T / (total * 1e-3)
+        if with_bwd and cfg.decay:
+            # training the decay too: the backward that also returns its gradient
+            dg_ms = time_bwd_dgamma(layer, steps, warmup)
+            entry["ttt_chunk_bwd_with_dgamma_ms"] = dg_ms
+            entry["ms_with_dgamma"] = entry["ttt_chunk_fwd"]["ms"] + dg_ms
         if cfg.name == synth.TINY_FP32.name:
             entry["note"] = "latency-bound correctness workload (two heads)"
         res[name] = entry
         del layer
         torch.cuda.empty_cache()
+    vec, sca = res["410m-ttt-linear-vector-decay-fwd-bwd"], res["410m-ttt-linear-fwd-bwd"]
+    # the per-feature decay's cost over the scalar decay, both training the decay
+    vec["vs_scalar_decay"] = vec["ms_with_dgamma"] / sca["ms_with_dgamma"]
     res[synth.TTT_MLP_410M.name] = time_mlp(ttt, peaks)
     return res
 
@@ -557,6 +566,8 @@ PROFILE_CASES = {
                     "T=512, d=64, C=256",
     "vector-decay-fwd-410m": "the vector-decay forward on the 410M shape (B=8, H=16, T=2048, "
                              "d=64, C=256): the state and readout kernels",
+    "vector-decay-410m": "the vector-decay forward and backward (decay gradient included) on "
+                         "the 410M shape",
     "ttt-mlp": "TTT-MLP forward and backward on the SIMT kernels (B=1, H=4, T=512, d=64, hidden "
                "256, C=256)",
 }
@@ -607,6 +618,13 @@ def run_case(name, ttt):
         layer = Layer(cfg, ttt, seed=cfg.seed)
         for _ in range(2):
             layer.fwd()
+    elif name == "vector-decay-410m":
+        cfg = synth.FWD_410M.replace(decay="vector")
+        layer = Layer(cfg, ttt, seed=cfg.seed)
+        dg = torch.empty_like(layer.inp["gamma"])
+        for _ in range(2):
+            layer.fwd()
+            layer.bwd(dg)
     elif name == "ttt-mlp":
         cfg, hid = synth.TTT_MLP_410M.replace(B=1, H=4, T=512), synth.TTT_MLP_HIDDEN
         inp = synth.ttt_inputs(cfg, device="cuda")

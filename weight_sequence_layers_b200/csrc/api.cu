@@ -100,6 +100,7 @@ Path fwd_path(const LayerArgs& a) {
 Path bwd_path(const LayerArgs& a, bool g_saved) {
   if (a.dtype == TTT_BF16 && tc_bwd_supported(a))
     return a.act == TTT_ACT_ID || g_saved ? PATH_TC : PATH_NONE;
+  if (a.dtype == TTT_BF16 && tc_vec_fwd_supported(a)) return PATH_TC_VEC;
   if (simt_supported(a)) return PATH_SIMT;
   return PATH_NONE;
 }
@@ -197,8 +198,10 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
     }
   }
   if (for_bwd != 1 && for_bwd != 2) return (size_t)-1;
+  a.gamma = reinterpret_cast<const float*>(16);  // as above
   switch (bwd_path(a, for_bwd == 2)) {
     case PATH_TC: return tc_bwd_workspace(a, for_bwd == 2, true);
+    case PATH_TC_VEC: return tc_vec_bwd_workspace(a);
     case PATH_SIMT: return simt_bwd_workspace(a);
     default: return (size_t)-1;
   }
@@ -252,11 +255,13 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
   LayerArgs a = args_of(cfg);
+  a.gamma = gamma;
   const Path path = bwd_path(a, G_saved != nullptr);
   if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
   const size_t need =
-      path == PATH_TC ? tc_bwd_workspace(a, G_saved != nullptr, dgamma != nullptr)
-                     : simt_bwd_workspace(a);
+      path == PATH_TC       ? tc_bwd_workspace(a, G_saved != nullptr, dgamma != nullptr)
+      : path == PATH_TC_VEC ? tc_vec_bwd_workspace(a)
+                            : simt_bwd_workspace(a);
   if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   cudaError_t e;
   unsigned* err = error_word(&e);
@@ -268,7 +273,9 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
   a.dW0 = dW0; a.ws = workspace; a.ws_bytes = workspace_bytes; a.err = err;
   a.O_in = O; a.W_final_in = W_final; a.dgamma = dgamma;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return launch_status(path == PATH_TC ? tc_bwd(a, s) : simt_bwd(a, s));
+  return launch_status(path == PATH_TC       ? tc_bwd(a, s)
+                       : path == PATH_TC_VEC ? tc_vec_bwd(a, s)
+                                             : simt_bwd(a, s));
 }
 
 size_t ttt_mlp_workspace_bytes(const ttt_config* cfg, int hidden) {
