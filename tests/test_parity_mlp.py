@@ -1,5 +1,7 @@
-"""GPU parity of the TTT-MLP SIMT kernels (two-layer fast weight act(k W1) W2) against the
-oracle's fp64 per-token loop and its autograd backward."""
+"""GPU parity of TTT-MLP (two-layer fast weight act(k W1) W2) against the oracle's fp64
+per-token loop and its autograd backward: the SIMT kernels (float32, and bf16 shapes outside
+the tensor-core envelope) and the batched tcgen05 GEMM program (bf16, d = 64, hidden 128 or 256,
+C = 128 or 256)."""
 import numpy as np
 import pytest
 import torch
@@ -114,3 +116,23 @@ def test_mlp_single_chunk_fp32():
         assert rel_err(f[k], rf[k]) <= F32_TOL, k
     for k in ("dQ", "dK", "dV", "dbeta", "dW1", "dW2"):
         assert rel_err(g[k], rg[k]) <= F32_TOL, k
+
+
+TC_CASES = [(256, 128, 128, loss, act, decay) for loss, act in COMBOS for decay in (False, True)]
+TC_CASES += [(512, 256, 256, "mse", "silu", True), (512, 256, 256, "ip", "id", False)]
+
+
+@pytest.mark.parametrize("T,C,hidden,loss,act,decay", TC_CASES)
+def test_mlp_tensor_core_shapes(T, C, hidden, loss, act, decay):
+    cfg = synth.TTT_MLP_410M.replace(B=1, H=2, T=T, C=C, loss=loss, act=act, decay=decay,
+                                     w0_std=0.05)
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=T + C + hidden)
+    w = synth.ttt_mlp_weights(cfg, hidden, device="cuda", seed=T + hidden)
+    w["dW1_T"].normal_(generator=torch.Generator("cuda").manual_seed(5))
+    w["dW2_T"].normal_(generator=torch.Generator("cuda").manual_seed(6))
+    f, g = run_mlp(cfg, hidden, inp, w)
+    rf, rg = reference(cfg, inp, w)
+    for k in ("O", "W1_final", "W2_final"):
+        assert rel_err(f[k], rf[k]) <= BF16_TOL, (k, rel_err(f[k], rf[k]))
+    for k in ("dQ", "dK", "dV", "dbeta", "dW1", "dW2"):
+        assert rel_err(g[k], rg[k]) <= BF16_TOL, (k, rel_err(g[k], rg[k]))

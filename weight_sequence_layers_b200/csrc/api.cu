@@ -165,6 +165,21 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t r
   return r == CUDA_SUCCESS;
 }
 
+bool make_tmap3_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                     uint64_t batch, uint64_t row_stride_elems, uint64_t batch_stride_elems,
+                     uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {inner, rows, batch};
+  cuuint64_t strides[2] = {row_stride_elems * 2, batch_stride_elems * 2};
+  cuuint32_t box[3] = {box_inner, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 }  // namespace tttk
 
 using namespace tttk;
@@ -282,7 +297,10 @@ size_t ttt_mlp_workspace_bytes(const ttt_config* cfg, int hidden) {
   if (check_config(cfg) != TTT_OK) return (size_t)-1;
   const LayerArgs a = args_of(cfg);
   if (!mlp_supported(a, hidden)) return (size_t)-1;
-  return mlp_workspace(a, hidden);
+  const size_t simt = mlp_workspace(a, hidden);
+  if (!mlp_tc_supported(a, hidden)) return simt;
+  const size_t tc = mlp_tc_fwd_workspace(a, hidden);
+  return tc > simt ? tc : simt;
 }
 
 ttt_status ttt_mlp_fwd(const ttt_config* cfg, int hidden, const void* Q, const void* K,
@@ -299,10 +317,19 @@ ttt_status ttt_mlp_fwd(const ttt_config* cfg, int hidden, const void* Q, const v
                         W2_chunks, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
-  if (!workspace || workspace_bytes < mlp_workspace(a, hidden)) return TTT_ERR_WORKSPACE;
+  const bool tc = mlp_tc_supported(a, hidden);
+  const size_t need = tc ? mlp_tc_fwd_workspace(a, hidden) : mlp_workspace(a, hidden);
+  if (!workspace || workspace_bytes < need) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
   a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.O = O; a.ws = workspace;
-  return launch_status(mlp_fwd(a, hidden, W1_0, W2_0, W1_final, W2_final, W1_chunks, W2_chunks,
-                               static_cast<cudaStream_t>(stream)));
+  a.err = err;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(tc ? mlp_tc_fwd(a, hidden, W1_0, W2_0, W1_final, W2_final, W1_chunks,
+                                       W2_chunks, s)
+                          : mlp_fwd(a, hidden, W1_0, W2_0, W1_final, W2_final, W1_chunks,
+                                    W2_chunks, s));
 }
 
 ttt_status ttt_mlp_bwd(const ttt_config* cfg, int hidden, const void* Q, const void* K,

@@ -67,6 +67,13 @@ bool tc_bwd_supported(const LayerArgs& a);
 size_t tc_bwd_workspace(const LayerArgs& a, bool g_saved, bool dgamma);
 cudaError_t tc_bwd(const LayerArgs& a, cudaStream_t s);
 
+// TTT-MLP on the tensor cores (bf16, d = 64, hidden 128 or 256, C = 128 or 256): a program of
+// batched tcgen05 GEMMs with fused epilogues.
+bool mlp_tc_supported(const LayerArgs& a, int hidden);
+size_t mlp_tc_fwd_workspace(const LayerArgs& a, int hidden);
+cudaError_t mlp_tc_fwd(const LayerArgs& a, int hidden, const float* W1_0, const float* W2_0,
+                       float* W1f, float* W2f, float* W1c, float* W2c, cudaStream_t s);
+
 // TTT-MLP (SIMT).
 bool mlp_supported(const LayerArgs& a, int hidden);
 size_t mlp_workspace(const LayerArgs& a, int hidden);
@@ -110,5 +117,9 @@ void count_launches(int n);
 // `row_stride_elems` apart; box = {box_inner (64), box_rows}. Returns false on failure.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_rows);
+// 3-D bf16 tensor map (inner, rows, batch) with 128-byte swizzle; box = {box_inner, box_rows, 1}.
+bool make_tmap3_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                     uint64_t batch, uint64_t row_stride_elems, uint64_t batch_stride_elems,
+                     uint32_t box_inner, uint32_t box_rows);
 
 }  // namespace tttk
