@@ -286,9 +286,9 @@ def time_other_configs(ttt, peaks):
 
 
 def time_mlp(ttt, peaks):
-    """TTT-MLP (two-layer fast weight, SIMT kernels) forward and backward on the 410M layer
-    shape with hidden width 4 d: device ms, tokens/s and the fraction of the fp32 CUDA-core
-    peak. flops per chunk and head: the readout and training GEMMs of both layers (causal halves
+    """TTT-MLP (two-layer fast weight; a program of batched tcgen05 GEMMs on this shape) forward
+    and backward on the 410M layer shape with hidden width 4 d: device ms, tokens/s and the
+    fraction of the bf16 tensor-core peak. flops per chunk and head: the readout and training GEMMs of both layers (causal halves
     of the C x C products), 2 C (3 dk h + 3 h dv) + C (C+1) (dk + dv + 2 h) forward and twice
     that backward; recomputation not counted."""
     cfg, hid = synth.TTT_MLP_410M, synth.TTT_MLP_HIDDEN
@@ -309,16 +309,15 @@ def time_mlp(ttt, peaks):
                                   w["W1"], w["W2"], O, W1f, W2f, W1c, W2c, ws, n)
     bwd = lambda: ttt.ttt_mlp_bwd(c, hid, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"],
                                   W1c, W2c, inp["dO"], None, None, *g, ws, n)
-    ms_f = _event_ms(fwd, 2, 3)
-    ms_b = _event_ms(bwd, 2, 3)
+    ms_f = _event_ms(fwd, 10, 3)
+    ms_b = _event_ms(bwd, 10, 3)
     units = B * H * (T // C)
     fl_f = units * (2 * C * (3 * dk * hid + 3 * hid * dv) + C * (C + 1) * (dk + dv + 2 * hid))
     tc = peaks["bf16_tflops"] * 1e12
     out = {"dtype": cfg.dtype, "hidden": hid, "decay": "scalar",
-           "ttt_mlp_fwd": {"ms": ms_f, "path": "simt", "tc_frac": fl_f / (ms_f * 1e-3) / tc,
-                           "alu_frac": fl_f / (ms_f * 1e-3) / FP32_ALU_PEAK},
-           "ttt_mlp_bwd": {"ms": ms_b, "path": "simt", "tc_frac": 2 * fl_f / (ms_b * 1e-3) / tc,
-                           "alu_frac": 2 * fl_f / (ms_b * 1e-3) / FP32_ALU_PEAK},
+           "ttt_mlp_fwd": {"ms": ms_f, "path": "tcgen05", "tc_frac": fl_f / (ms_f * 1e-3) / tc},
+           "ttt_mlp_bwd": {"ms": ms_b, "path": "tcgen05",
+                           "tc_frac": 2 * fl_f / (ms_b * 1e-3) / tc},
            "ms": ms_f + ms_b, "tokens_per_s": B * T / ((ms_f + ms_b) * 1e-3)}
     del ws
     torch.cuda.empty_cache()
@@ -568,8 +567,10 @@ PROFILE_CASES = {
                              "d=64, C=256): the state and readout kernels",
     "vector-decay-410m": "the vector-decay forward and backward (decay gradient included) on "
                          "the 410M shape",
-    "ttt-mlp": "TTT-MLP forward and backward on the SIMT kernels (B=1, H=4, T=512, d=64, hidden "
-               "256, C=256)",
+    "ttt-mlp": "TTT-MLP forward and backward (tcgen05 GEMM program; B=1, H=4, T=512, d=64, "
+               "hidden 256, C=256)",
+    "ttt-mlp-410m": "TTT-MLP forward and backward on the 410M shape (B=8, H=16, T=2048, d=64, "
+                    "hidden 256, C=256)",
 }
 
 
@@ -625,8 +626,10 @@ def run_case(name, ttt):
         for _ in range(2):
             layer.fwd()
             layer.bwd(dg)
-    elif name == "ttt-mlp":
-        cfg, hid = synth.TTT_MLP_410M.replace(B=1, H=4, T=512), synth.TTT_MLP_HIDDEN
+    elif name in ("ttt-mlp", "ttt-mlp-410m"):
+        cfg, hid = synth.TTT_MLP_410M, synth.TTT_MLP_HIDDEN
+        if name == "ttt-mlp":
+            cfg = cfg.replace(B=1, H=4, T=512)
         inp = synth.ttt_inputs(cfg, device="cuda")
         w = synth.ttt_mlp_weights(cfg, hid, device="cuda")
         c = ttt.make_config(cfg.B, cfg.H, cfg.T, cfg.dk, cfg.dv, cfg.C, cfg.dtype, cfg.loss,

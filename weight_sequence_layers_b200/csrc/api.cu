@@ -299,7 +299,8 @@ size_t ttt_mlp_workspace_bytes(const ttt_config* cfg, int hidden) {
   if (!mlp_supported(a, hidden)) return (size_t)-1;
   const size_t simt = mlp_workspace(a, hidden);
   if (!mlp_tc_supported(a, hidden)) return simt;
-  const size_t tc = mlp_tc_fwd_workspace(a, hidden);
+  const size_t f = mlp_tc_fwd_workspace(a, hidden), b = mlp_tc_bwd_workspace(a, hidden);
+  const size_t tc = f > b ? f : b;
   return tc > simt ? tc : simt;
 }
 
@@ -349,11 +350,19 @@ ttt_status ttt_mlp_bwd(const ttt_config* cfg, int hidden, const void* Q, const v
                         dQ, dK, dV, dbeta, dW1_0, dW2_0, workspace};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTT_ERR_ALIGNMENT;
-  if (!workspace || workspace_bytes < mlp_workspace(a, hidden)) return TTT_ERR_WORKSPACE;
+  const bool tc = mlp_tc_supported(a, hidden);
+  const size_t need = tc ? mlp_tc_bwd_workspace(a, hidden) : mlp_workspace(a, hidden);
+  if (!workspace || workspace_bytes < need) return TTT_ERR_WORKSPACE;
+  cudaError_t e;
+  unsigned* err = error_word(&e);
+  if (!err) return TTT_ERR_CUDA;
   a.Q = Q; a.K = K; a.V = V; a.beta = beta; a.gamma = gamma; a.dO = dO; a.dQ = dQ; a.dK = dK;
-  a.dV = dV; a.dbeta = dbeta; a.ws = workspace;
-  return launch_status(mlp_bwd(a, hidden, W1_chunks, W2_chunks, dW1_final, dW2_final, dW1_0,
-                               dW2_0, static_cast<cudaStream_t>(stream)));
+  a.dV = dV; a.dbeta = dbeta; a.ws = workspace; a.err = err;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(tc ? mlp_tc_bwd(a, hidden, W1_chunks, W2_chunks, dW1_final, dW2_final,
+                                       dW1_0, dW2_0, s)
+                          : mlp_bwd(a, hidden, W1_chunks, W2_chunks, dW1_final, dW2_final,
+                                    dW1_0, dW2_0, s));
 }
 
 size_t inplace_ttt_workspace_bytes(int T, int d_ff, int d_model, int C) {

@@ -73,6 +73,10 @@ bool mlp_tc_supported(const LayerArgs& a, int hidden);
 size_t mlp_tc_fwd_workspace(const LayerArgs& a, int hidden);
 cudaError_t mlp_tc_fwd(const LayerArgs& a, int hidden, const float* W1_0, const float* W2_0,
                        float* W1f, float* W2f, float* W1c, float* W2c, cudaStream_t s);
+size_t mlp_tc_bwd_workspace(const LayerArgs& a, int hidden);
+cudaError_t mlp_tc_bwd(const LayerArgs& a, int hidden, const float* W1c, const float* W2c,
+                       const float* dW1f, const float* dW2f, float* dW1_0, float* dW2_0,
+                       cudaStream_t s);
 
 // TTT-MLP (SIMT).
 bool mlp_supported(const LayerArgs& a, int hidden);
