@@ -31,14 +31,11 @@ constexpr int D = 64;  // d_k = d_v
 
 struct MCtx {
   int T, C, NC, h;
-  float lr_bias;
   int loss;
-  const float* beta;
+  const float* Eb;  // [BH, T] eta_t = 2 sigmoid(beta_t + b)
   const float* Lb;  // [BH, T] chunk-local L (zeros without a decay)
 };
-__device__ __forceinline__ float eta_at(const MCtx& x, size_t tok) {
-  return 2.f * sigm(__ldg(x.beta + tok) + x.lr_bias);
-}
+__device__ __forceinline__ float eta_at(const MCtx& x, size_t tok) { return __ldg(x.Eb + tok); }
 // u_r = eta_r exp(L_C - L_r) of token tok of the chunk starting at tok0
 __device__ __forceinline__ float u_at(const MCtx& x, size_t tok0, size_t tok) {
   return eta_at(x, tok) * __expf(__ldg(x.Lb + tok0 + x.C - 1) - __ldg(x.Lb + tok));
@@ -251,11 +248,16 @@ struct EpiScore {
     return {tok0, s, __ldg(x.Lb + tok0 + s)};
   }
   __device__ void chunk(St& st, int col0, float (&v)[32]) const {
+    if (col0 <= st.s) {  // else every key of the group follows the query: zeros
+      float e[32], l[32];
+      ld_f32x32(x.Eb + st.tok0 + col0, e);
+      ld_f32x32(x.Lb + st.tok0 + col0, l);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int r = col0 + j;
-      v[j] = r <= st.s ? -eta_at(x, st.tok0 + r) * __expf(st.Ls - __ldg(x.Lb + st.tok0 + r)) * v[j]
-                       : 0.f;
+      for (int j = 0; j < 32; ++j)
+        v[j] = col0 + j <= st.s ? -e[j] * __expf(st.Ls - l[j]) * v[j] : 0.f;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.f;
     }
     st_global_bf16x32(S + (st.tok0 + st.s) * x.C + col0, v);
   }
@@ -298,15 +300,18 @@ struct EpiOut {
 };
 
 // ------------------------------------------------------------------------- helpers
-// Chunk-local L of every token (one block per chunk, a warp scan), Qhat = Gamma_s q_s and, when
-// given, Gamma_s dO_s.
+// Chunk-local L of every token (one block per chunk, a warp scan), eta, Qhat = Gamma_s q_s and,
+// when given, Gamma_s dO_s.
 __global__ void __launch_bounds__(256) mlp_scan_kernel(int C, const float* gamma,
+                                                       const float* beta, float lr_bias,
                                                        const __nv_bfloat16* Q, float* Lb,
-                                                       __nv_bfloat16* Qh,
+                                                       float* Eb, __nv_bfloat16* Qh,
                                                        const __nv_bfloat16* dO = nullptr,
                                                        __nv_bfloat16* dOh = nullptr) {
   __shared__ float sL[256];
   const size_t tok0 = (size_t)blockIdx.x * C;
+  for (int t = threadIdx.x; t < C; t += blockDim.x)
+    Eb[tok0 + t] = 2.f * sigm(__ldg(beta + tok0 + t) + lr_bias);
   if (threadIdx.x < 32) {
     const int lane = threadIdx.x, per = C / 32;
     float s = 0.f;
@@ -343,23 +348,49 @@ __global__ void __launch_bounds__(256) mlp_scan_kernel(int C, const float* gamma
   if (dO) scale(dO, dOh);
 }
 
-// Chunk-0 weights: the masters and operand copies from W1_0 [64, h] and W2_0 [h, 64].
-__global__ void mlp_init_kernel(int h, int NC, const float* W1_0, const float* W2_0, float* W1Tm,
-                                float* W2m, __nv_bfloat16* W1Tc, __nv_bfloat16* W2c,
-                                __nv_bfloat16* W2Tc, float* W1c, float* W2c_out) {
-  const size_t b = blockIdx.x, n = (size_t)h * D;
+// dst[c][r] = src[r][c] for an R x Cc float32 matrix (R, Cc multiples of 32; src NULL: zeros),
+// through 32 x 32 shared-memory tiles, one block of 256 threads; float or bf16 destinations.
+__device__ __forceinline__ void put(float* p, float v) { *p = v; }
+__device__ __forceinline__ void put(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+template <typename TA, typename TB>
+__device__ void transpose_to(const float* src, int R, int Cc, TA* dst, TB* dst2,
+                             float (*tile)[33]) {
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r0 = 0; r0 < R; r0 += 32)
+    for (int c0 = 0; c0 < Cc; c0 += 32) {
+      for (int k = ty; k < 32; k += 8)
+        tile[k][tx] = src ? src[(size_t)(r0 + k) * Cc + c0 + tx] : 0.f;
+      __syncthreads();
+      for (int k = ty; k < 32; k += 8) {
+        const size_t o = (size_t)(c0 + k) * R + r0 + tx;
+        put(dst + o, tile[tx][k]);
+        if (dst2) put(dst2 + o, tile[tx][k]);
+      }
+      __syncthreads();
+    }
+}
+// element-wise copies of an n-element float32 array (src NULL: zeros)
+template <typename TA, typename TB>
+__device__ void copy_to(const float* src, size_t n, TA* dst, TB* dst2) {
   for (size_t e = threadIdx.x; e < n; e += blockDim.x) {
-    const int i = (int)(e / D), k = (int)(e % D);  // row i of the [h, 64] matrices
-    const float w1 = W1_0[b * n + (size_t)k * h + i];
-    const float w2 = W2_0[b * n + e];
-    W1Tm[b * n + e] = w1;
-    W2m[b * n + e] = w2;
-    W1Tc[b * NC * n + e] = __float2bfloat16_rn(w1);
-    W2c[b * NC * n + e] = __float2bfloat16_rn(w2);
-    W2Tc[b * NC * n + (size_t)k * h + i] = __float2bfloat16_rn(w2);
-    if (W1c) W1c[b * NC * n + (size_t)k * h + i] = w1;
-    if (W2c_out) W2c_out[b * NC * n + e] = w2;
+    const float v = src ? src[e] : 0.f;
+    if (dst) put(dst + e, v);
+    if (dst2) put(dst2 + e, v);
   }
+}
+
+// Chunk-0 weights: the masters and operand copies from W1_0 [64, h] and W2_0 [h, 64].
+__global__ void __launch_bounds__(256)
+    mlp_init_kernel(int h, int NC, const float* W1_0, const float* W2_0, float* W1Tm, float* W2m,
+                    __nv_bfloat16* W1Tc, __nv_bfloat16* W2c, __nv_bfloat16* W2Tc, float* W1c,
+                    float* W2c_out) {
+  __shared__ float tile[32][33];
+  const size_t b = blockIdx.x, n = (size_t)h * D;
+  transpose_to(W1_0 + b * n, D, h, W1Tm + b * n, W1Tc + b * NC * n, tile);
+  transpose_to(W2_0 + b * n, h, D, W2Tc + b * NC * n, (float*)nullptr, tile);
+  copy_to(W2_0 + b * n, n, W2m + b * n, W2c + b * NC * n);
+  copy_to(W1_0 + b * n, n, W1c ? W1c + b * NC * n : nullptr, (float*)nullptr);
+  copy_to(W2_0 + b * n, n, W2c_out ? W2c_out + b * NC * n : nullptr, (float*)nullptr);
 }
 
 // ---------------------------------------------------------------------------- host side
@@ -392,7 +423,7 @@ bg::Prob prob1(int K, int a_k0, int a_row, int b_k0, int b_row) {
 }
 
 struct FwdBufs {
-  float *Lb, *W1Tm, *W2m, *Zs;
+  float *Lb, *Eb, *W1Tm, *W2m, *Zs;
   __nv_bfloat16 *Qh, *W1Tc, *W2c, *W2Tc, *A1, *A1T, *G2, *uG2, *G1T, *uG1T, *S1, *Aq, *Ahq, *S2;
 };
 
@@ -410,6 +441,7 @@ size_t carve_fwd(const LayerArgs& a, int h, void* base, FwdBufs* f) {
   };
   FwdBufs b{};
   b.Lb = (float*)take(rows * 4);
+  b.Eb = (float*)take(rows * 4);
   b.W1Tm = (float*)take(BH * h * D * 4);
   b.W2m = (float*)take(BH * h * D * 4);
   b.Zs = (float*)take(BH * C * h * 4);
@@ -440,9 +472,9 @@ cudaError_t mlp_tc_fwd_impl(const LayerArgs& a, int h, const float* W1_0, const 
   const auto* Q = static_cast<const __nv_bfloat16*>(a.Q);
   const auto* K = static_cast<const __nv_bfloat16*>(a.K);
   const auto* V = static_cast<const __nv_bfloat16*>(a.V);
-  MCtx x{T, C, NC, h, a.lr_bias, a.loss, a.beta, f.Lb};
+  MCtx x{T, C, NC, h, a.loss, f.Eb, f.Lb};
   cudaError_t e;
-  mlp_scan_kernel<<<BH * NC, 256, 0, s>>>(C, a.gamma, Q, f.Lb, f.Qh);
+  mlp_scan_kernel<<<BH * NC, 256, 0, s>>>(C, a.gamma, a.beta, a.lr_bias, Q, f.Lb, f.Eb, f.Qh);
   mlp_init_kernel<<<BH, 256, 0, s>>>(h, NC, W1_0, W2_0, f.W1Tm, f.W2m, f.W1Tc, f.W2c, f.W2Tc,
                                       W1c, W2c_out);
   count_launches(2);
@@ -673,10 +705,15 @@ struct EpiScoreT {
     return {tok0, r, -eta_at(x, tok0 + r), __ldg(x.Lb + tok0 + r)};
   }
   __device__ void chunk(St& st, int col0, float (&v)[32]) const {
+    if (col0 + 31 >= st.r) {  // else every query of the group precedes the key: zeros
+      float l[32];
+      ld_f32x32(x.Lb + st.tok0 + col0, l);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int s = col0 + j;
-      v[j] = s >= st.r ? st.ne * __expf(__ldg(x.Lb + st.tok0 + s) - st.Lr) * v[j] : 0.f;
+      for (int j = 0; j < 32; ++j)
+        v[j] = col0 + j >= st.r ? st.ne * __expf(l[j] - st.Lr) * v[j] : 0.f;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.f;
     }
     st_global_bf16x32(S + (st.tok0 + st.r) * x.C + col0, v);
   }
@@ -728,14 +765,19 @@ struct EpiDST {
     return {tok0, r, eta_at(x, tok0 + r), __ldg(x.Lb + tok0 + r), 0.f};
   }
   __device__ void chunk(St& st, int col0, float (&v)[32]) const {
-    float sn[32];
-    ld_bf16x32(StN + (st.tok0 + st.r) * x.C + col0, sn);
+    if (col0 + 31 >= st.r) {
+      float sn[32], l[32];
+      ld_bf16x32(StN + (st.tok0 + st.r) * x.C + col0, sn);
+      ld_f32x32(x.Lb + st.tok0 + col0, l);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int s = col0 + j;
-      const float ds = s >= st.r ? -v[j] : 0.f;
-      st.acc -= ds * sn[j];
-      v[j] = st.eta * __expf(__ldg(x.Lb + st.tok0 + s) - st.Lr) * ds;
+      for (int j = 0; j < 32; ++j) {
+        const float ds = col0 + j >= st.r ? -v[j] : 0.f;
+        st.acc -= ds * sn[j];
+        v[j] = st.eta * __expf(l[j] - st.Lr) * ds;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.f;
     }
     st_global_bf16x32(DT + (st.tok0 + st.r) * x.C + col0, v);
   }
@@ -975,37 +1017,29 @@ struct EpiAdj {
 
 // Per-chunk bf16 operand copies of the saved float32 chunk weights W1c [64, h], W2c [h, 64]:
 // W1^T, W1, W2, W2^T; and the adjoint masters from dW1_final, dW2_final (or zero).
-__global__ void mlp_bwd_init_kernel(int h, int NC, const float* W1c, const float* W2c,
-                                    const float* dW1f, const float* dW2f,
-                                    __nv_bfloat16* W1T, __nv_bfloat16* W1, __nv_bfloat16* W2,
-                                    __nv_bfloat16* W2T, float* Wh1m, float* Wh2m,
-                                    __nv_bfloat16* Wh1T_b, __nv_bfloat16* Wh1_b,
-                                    __nv_bfloat16* Wh2_b, __nv_bfloat16* Wh2T_b) {
+__global__ void __launch_bounds__(256)
+    mlp_bwd_init_kernel(int h, int NC, const float* W1c, const float* W2c, const float* dW1f,
+                        const float* dW2f, __nv_bfloat16* W1T, __nv_bfloat16* W1,
+                        __nv_bfloat16* W2, __nv_bfloat16* W2T, float* Wh1m, float* Wh2m,
+                        __nv_bfloat16* Wh1T_b, __nv_bfloat16* Wh1_b, __nv_bfloat16* Wh2_b,
+                        __nv_bfloat16* Wh2T_b) {
+  __shared__ float tile[32][33];
   const size_t bc = blockIdx.x, n = (size_t)h * D;
-  for (size_t e = threadIdx.x; e < n; e += blockDim.x) {
-    const int i = (int)(e / D), k = (int)(e % D);
-    const float w1 = W1c[bc * n + (size_t)k * h + i];
-    const float w2 = W2c[bc * n + e];
-    W1T[bc * n + e] = __float2bfloat16_rn(w1);
-    W1[bc * n + (size_t)k * h + i] = __float2bfloat16_rn(w1);
-    W2[bc * n + e] = __float2bfloat16_rn(w2);
-    W2T[bc * n + (size_t)k * h + i] = __float2bfloat16_rn(w2);
-    if (bc % NC == 0) {
-      const size_t b = bc / NC;
-      const float a1 = dW1f ? dW1f[b * n + (size_t)k * h + i] : 0.f;
-      const float a2 = dW2f ? dW2f[b * n + e] : 0.f;
-      Wh1m[b * n + e] = a1;
-      Wh2m[b * n + e] = a2;
-      Wh1T_b[b * n + e] = __float2bfloat16_rn(a1);
-      Wh1_b[b * n + (size_t)k * h + i] = __float2bfloat16_rn(a1);
-      Wh2_b[b * n + e] = __float2bfloat16_rn(a2);
-      Wh2T_b[b * n + (size_t)k * h + i] = __float2bfloat16_rn(a2);
-    }
+  transpose_to(W1c + bc * n, D, h, W1T + bc * n, (float*)nullptr, tile);
+  transpose_to(W2c + bc * n, h, D, W2T + bc * n, (float*)nullptr, tile);
+  copy_to(W1c + bc * n, n, W1 + bc * n, (float*)nullptr);
+  copy_to(W2c + bc * n, n, W2 + bc * n, (float*)nullptr);
+  if (bc % NC == 0) {
+    const size_t b = bc / NC;
+    transpose_to(dW1f ? dW1f + b * n : nullptr, D, h, Wh1m + b * n, Wh1T_b + b * n, tile);
+    transpose_to(dW2f ? dW2f + b * n : nullptr, h, D, Wh2T_b + b * n, (float*)nullptr, tile);
+    copy_to(dW1f ? dW1f + b * n : nullptr, n, Wh1_b + b * n, (float*)nullptr);
+    copy_to(dW2f ? dW2f + b * n : nullptr, n, Wh2m + b * n, Wh2_b + b * n);
   }
 }
 
 struct BwdBufs {
-  float *Lb, *Z1, *dG2s, *dKs, *deta, *dZ1a, *dA1, *Ya, *ykg, *yag, *Wh1m, *Wh2m;
+  float *Lb, *Eb, *Z1, *dG2s, *dKs, *deta, *dZ1a, *dA1, *Ya, *ykg, *yag, *Wh1m, *Wh2m;
   __nv_bfloat16 *Qh, *dOh, *W1T, *W1, *W2, *W2T, *A1, *Bm, *G1, *uG1n, *Aq, *dAct, *dZq, *dZqh,
       *dA1s, *dG1s, *A1T, *G1T, *AqT, *AhqT, *dZqT, *G2, *uG2n, *S1n, *S1nT, *S2nT, *D2T, *D2,
       *D1T, *D1, *dB, *dBT, *dG2, *dZ1, *dZ1T, *Wh1T_b, *Wh1_b, *Wh2_b, *Wh2T_b;
@@ -1024,6 +1058,7 @@ size_t carve_bwd(const LayerArgs& a, int h, void* base, BwdBufs* f) {
   auto f32 = [&](size_t n) { return (float*)take(n * 4); };
   BwdBufs b{};
   b.Lb = f32(rows);
+  b.Eb = f32(rows);
   b.deta = f32(rows);
   b.Qh = bf(rows * D);
   b.dOh = bf(rows * D);
@@ -1079,9 +1114,10 @@ cudaError_t mlp_tc_bwd_impl(const LayerArgs& a, int h, const float* W1c, const f
   const auto* K = static_cast<const __nv_bfloat16*>(a.K);
   const auto* V = static_cast<const __nv_bfloat16*>(a.V);
   const auto* dO = static_cast<const __nv_bfloat16*>(a.dO);
-  const MCtx x{T, C, NC, h, a.lr_bias, a.loss, a.beta, f.Lb};
+  const MCtx x{T, C, NC, h, a.loss, f.Eb, f.Lb};
   cudaError_t e;
-  mlp_scan_kernel<<<NB, 256, 0, s>>>(C, a.gamma, Q, f.Lb, f.Qh, dO, f.dOh);
+  mlp_scan_kernel<<<NB, 256, 0, s>>>(C, a.gamma, a.beta, a.lr_bias, Q, f.Lb, f.Eb, f.Qh, dO,
+                                     f.dOh);
   mlp_bwd_init_kernel<<<NB, 256, 0, s>>>(h, NC, W1c, W2c, dW1f, dW2f, f.W1T, f.W1, f.W2, f.W2T,
                                           f.Wh1m, f.Wh2m, f.Wh1T_b, f.Wh1_b, f.Wh2_b, f.Wh2T_b);
   count_launches(2);
