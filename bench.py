@@ -171,7 +171,7 @@ class Layer:
         self.Wf = torch.empty((B, H, dk, dv), device=dev, dtype=torch.float32)
         self.Wc = torch.empty((B, H, T // C, dk, dv), device=dev, dtype=sd)
         # saved by fwd for bwd: G, and with SiLU also Zq (the readout before the activation)
-        planes = ttt.ttt_saved_bytes(self.c) // (B * H * T * dv * sd.itemsize)
+        planes = -(-ttt.ttt_saved_bytes(self.c) // (B * H * T * dv * sd.itemsize))
         self.G = torch.empty((planes, B, H, T, dv), device=dev, dtype=sd)
         self.dQ = torch.empty((B, H, T, dk), device=dev, dtype=sd)
         self.dK = torch.empty((B, H, T, dk), device=dev, dtype=sd)

@@ -109,7 +109,11 @@ typedef struct {
 size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd);
 
 /* Bytes of the G_saved buffer of this config (B*H*T*dv elements of cfg->dtype, twice that with
- * SiLU, where Zq follows G); (size_t)-1 if the config is invalid. */
+ * SiLU, where Zq follows G); on the vector-decay tensor-core path (bf16, vector decay, identity,
+ * dk == dv == 64, C in {128, 256}) G is followed by the decayed operands the forward forms
+ * (q and k scaled per feature, the log decay L of every token) and the effective query R, so
+ * that the backward need not form them again: B*H*T*64*2 bytes for G, then that library-defined
+ * region. (size_t)-1 if the config is invalid. */
 size_t ttt_saved_bytes(const ttt_config* cfg);
 
 /* Forward of the chunkwise TTT layer.
@@ -135,7 +139,8 @@ ttt_status ttt_chunk_fwd(const ttt_config* cfg, const void* Q, const void* K, co
  *  in : Q, K, V, beta, gamma (nullable), W0, W_chunks (from ttt_chunk_fwd, required),
  *       G_saved (from ttt_chunk_fwd, nullable: rebuilt from W_chunks when NULL; kernels that
  *       rebuild G anyway may ignore it; with SiLU the tensor-core backward needs it, for Zq,
- *       and a SiLU call on a tensor-core shape without it returns TTT_ERR_UNSUPPORTED),
+ *       and a SiLU call on a tensor-core shape without it returns TTT_ERR_UNSUPPORTED; on the
+ *       vector-decay tensor-core path it supplies the forward's decayed operands and R),
  *       dO, dW_final (nullable = 0);
  *       O and W_final (the forward's outputs) are read only for dgamma (then O is required,
  *       and W_final too when dW_final is non-NULL).
@@ -192,7 +197,9 @@ ttt_status ttt_chunk_bwd_noalloc(const ttt_config* cfg, const void* Q, const voi
  *     z = k W1_0, a = act(z), g2 = a W2_0 - v (MSE) or -v (IP), g1 = (g2 W2_0^T) * act'(z)
  *     W1_t = gamma_t W1_{t-1} - eta_t k^T g1,  W2_t = gamma_t W2_{t-1} - eta_t a^T g2
  *     o_t  = act(q_t W1_t) W2_t
- * evaluated in the chunk dual form on the SIMT kernels (float32 arithmetic).
+ * evaluated in the chunk dual form. bf16 configs with dk == dv == 64, hidden in {128, 256} and
+ * C in {128, 256} run as a program of batched tcgen05 GEMMs with fused epilogues (fp32
+ * accumulation and fp32 master weights); the others on the SIMT kernels (float32 arithmetic).
  * Layouts: Q, K, dQ, dK [B,H,T,dk] and V, O, dO, dV [B,H,T,dv] in cfg->dtype; beta, gamma, dbeta
  * [B,H,T] float32 (gamma nullable; scalar decay only); W1 [B,H,dk,hidden], W2 [B,H,hidden,dv]
  * float32, likewise W1_final, W2_final, dW1_final, dW2_final, dW1_0, dW2_0; W1_chunks

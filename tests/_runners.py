@@ -30,8 +30,9 @@ def run_fwd(cfg, inp, save_g=True, save_w=True):
     O = torch.empty((B, H, T, dv), device="cuda", dtype=sd)
     Wf = torch.empty((B, H, dk, dv), device="cuda", dtype=torch.float32)
     Wc = torch.empty((B, H, T // C, dk, dv), device="cuda", dtype=sd) if save_w else None
-    # the saved buffer holds G, then with SiLU Zq (the readout before the activation)
-    planes = ttt.ttt_saved_bytes(c) // (B * H * T * dv * sd.itemsize)
+    # the saved buffer holds G, then with SiLU Zq (the readout before the activation); with a
+    # vector decay on the tensor cores more follows (whole [B, H, T, dv] planes, rounded up)
+    planes = -(-ttt.ttt_saved_bytes(c) // (B * H * T * dv * sd.itemsize))
     Gs = torch.empty((planes, B, H, T, dv), device="cuda", dtype=sd) if save_g else None
     n = ttt.ttt_workspace_bytes(c, 0)
     ws = torch.empty(max(n, 16), device="cuda", dtype=torch.uint8)
@@ -40,7 +41,7 @@ def run_fwd(cfg, inp, save_g=True, save_w=True):
     torch.cuda.synchronize()
     assert ttt.ttt_get_device_error() == ttt.OK
     return dict(O=O, W_final=Wf, W_chunks=Wc, G=None if Gs is None else Gs[0], G_saved=Gs,
-                Zq=Gs[1] if Gs is not None and planes == 2 else None)
+                Zq=Gs[1] if Gs is not None and cfg.act == "silu" else None)
 
 
 def run_bwd(cfg, inp, W_chunks, G=None, fwd=None):

@@ -296,6 +296,13 @@ def test_saved_buffer_size():
     assert ttt.ttt_saved_bytes(_cfg(dtype="bf16", dk=128, dv=96, C=128, T=512, act="silu")) == \
         2 * 2 * 3 * 512 * 96 * 2
     assert ttt.ttt_saved_bytes(_cfg()) == 2 * 3 * 256 * 64 * 4
+    # vector decay on the tensor cores: G first, then the forward's decayed operands and R
+    vec = _cfg(dtype="bf16", dk=64, dv=64, C=256, T=512, decay="vector")
+    g_plane = 2 * 3 * 512 * 64 * 2
+    assert ttt.ttt_saved_bytes(vec) > 4 * g_plane
+    # (the vector decay outside that path keeps G alone)
+    assert ttt.ttt_saved_bytes(_cfg(dtype="bf16", dk=64, dv=64, C=64, T=512, decay="vector")) == \
+        2 * 3 * 512 * 64 * 2
     with pytest.raises(ttt.TTTError):
         ttt.ttt_saved_bytes(_cfg(T=250))
 

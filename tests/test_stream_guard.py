@@ -37,14 +37,17 @@ def _cut(inp, a, b):
 
 
 CASES = [
-    # (workload, overrides): identity and SiLU on the tensor cores, float32 on SIMT
+    # (workload, overrides): identity and SiLU on the tensor cores, float32 on SIMT, and the
+    # per-feature decay on the tensor cores
     (synth.TRAIN_1P45B, dict(B=1, H=2, T=1024)),
     (synth.SILU_IP_FWD, dict(B=1, H=2, T=1024, loss="mse")),
     (synth.TINY_FP32, dict(B=1, H=2, T=512)),
+    (synth.FWD_410M, dict(B=1, H=2, T=1024, decay="vector", w0_std=0.05)),
 ]
+IDS = ["tc-id", "tc-silu", "simt-f32", "tc-vector"]
 
 
-@pytest.mark.parametrize("base,kw", CASES, ids=["tc-id", "tc-silu", "simt-f32"])
+@pytest.mark.parametrize("base,kw", CASES, ids=IDS)
 def test_two_calls_with_the_state_carried_equal_one_call(base, kw):
     cfg = base.replace(**kw)
     T1 = cfg.T // 2
@@ -91,7 +94,7 @@ def _intact(buf):
     return bool((buf[:PAD] == PATTERN).all()) and bool((buf[-PAD:] == PATTERN).all())
 
 
-@pytest.mark.parametrize("base,kw", CASES, ids=["tc-id", "tc-silu", "simt-f32"])
+@pytest.mark.parametrize("base,kw", CASES, ids=IDS)
 def test_no_output_is_written_past_its_ends(base, kw):
     cfg = base.replace(**kw)
     inp = synth.ttt_inputs(cfg, device="cuda", seed=103)
@@ -107,7 +110,8 @@ def test_no_output_is_written_past_its_ends(base, kw):
     O = out("O", (B, H, T, dv), sd)
     Wf = out("W_final", (B, H, dk, dv), torch.float32)
     Wc = out("W_chunks", (B, H, T // C, dk, dv), sd)
-    Gs = out("G_saved", (ttt.ttt_saved_bytes(c) // (B * H * T * dv * sd.itemsize), B, H, T, dv), sd)
+    Gs = out("G_saved", (-(-ttt.ttt_saved_bytes(c) // (B * H * T * dv * sd.itemsize)), B, H, T, dv),
+             sd)
     n = ttt.ttt_workspace_bytes(c, 0)
     ws = out("ws_fwd", (max(n, 16),), torch.uint8)
     ttt.ttt_chunk_fwd(c, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], inp["W0"], O, Wf,

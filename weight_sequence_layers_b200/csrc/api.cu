@@ -216,7 +216,7 @@ size_t ttt_workspace_bytes(const ttt_config* cfg, int for_bwd) {
   a.gamma = reinterpret_cast<const float*>(16);  // as above
   switch (bwd_path(a, for_bwd == 2)) {
     case PATH_TC: return tc_bwd_workspace(a, for_bwd == 2, true);
-    case PATH_TC_VEC: return tc_vec_bwd_workspace(a);
+    case PATH_TC_VEC: return tc_vec_bwd_workspace(a, for_bwd == 2);
     case PATH_SIMT: return simt_bwd_workspace(a);
     default: return (size_t)-1;
   }
@@ -275,7 +275,7 @@ ttt_status ttt_chunk_bwd(const ttt_config* cfg, const void* Q, const void* K, co
   if (path == PATH_NONE) return TTT_ERR_UNSUPPORTED;
   const size_t need =
       path == PATH_TC       ? tc_bwd_workspace(a, G_saved != nullptr, dgamma != nullptr)
-      : path == PATH_TC_VEC ? tc_vec_bwd_workspace(a)
+      : path == PATH_TC_VEC ? tc_vec_bwd_workspace(a, G_saved != nullptr)
                             : simt_bwd_workspace(a);
   if (need && (!workspace || workspace_bytes < need)) return TTT_ERR_WORKSPACE;
   cudaError_t e;
@@ -471,6 +471,9 @@ ttt_status inplace_ttt_fwd_docs(int T, int d_ff, int d_model, int C, float lr, c
 
 size_t ttt_saved_bytes(const ttt_config* cfg) {
   if (check_config(cfg) != TTT_OK) return (size_t)-1;
+  LayerArgs a = args_of(cfg);
+  a.gamma = reinterpret_cast<const float*>(16);  // a decay is given (never dereferenced)
+  if (fwd_path(a) == PATH_TC_VEC) return tc_vec_saved_bytes(a);
   const size_t elem = cfg->dtype == TTT_BF16 ? 2 : 4;
   return (size_t)cfg->B * cfg->H * cfg->T * cfg->dv * elem * (cfg->act == TTT_ACT_SILU ? 2 : 1);
 }

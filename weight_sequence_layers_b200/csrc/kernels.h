@@ -45,8 +45,10 @@ cudaError_t tc_fwd(const LayerArgs& a, cudaStream_t s);
 bool tc_vec_fwd_supported(const LayerArgs& a);
 size_t tc_vec_fwd_workspace(const LayerArgs& a);
 cudaError_t tc_vec_fwd(const LayerArgs& a, cudaStream_t s);
-// Its backward (same shapes; reads the forward's W_chunks, not G_saved).
-size_t tc_vec_bwd_workspace(const LayerArgs& a);
+// Its backward (same shapes; reads the forward's W_chunks and, when given, its saved buffer:
+// G, the decayed operands with L, and R).
+size_t tc_vec_bwd_workspace(const LayerArgs& a, bool g_saved);
+size_t tc_vec_saved_bytes(const LayerArgs& a);
 cudaError_t tc_vec_bwd(const LayerArgs& a, cudaStream_t s);
 
 // The decayed operands of the vector decay, one chunk-parallel pass (chunk-local L, chunk

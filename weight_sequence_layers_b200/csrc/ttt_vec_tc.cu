@@ -52,6 +52,7 @@ struct VecParams {
   __nv_bfloat16* Wc;    // [BH, NC, 64, 64]
   __nv_bfloat16* O;
   int save_g;
+  int save_r;  // the readout also stores R (for the backward)
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -566,7 +567,8 @@ __global__ void __launch_bounds__(kVoThreads, 2)
         if (mbar_wait(UB(U_PD0), 0, ab)) load(sB, &tmV, U_B2, tokc);
         if (qb == 1 && mbar_wait(UB(U_PD1), 0, ab)) load(sC, &tmV, U_C2, tokc + 128);
         if (LOSS == 0 && mbar_wait(UB(U_SK), 0, ab)) load_w(U_D2);
-      } else if (mbar_wait(UB(U_R), 0, ab)) {
+      }
+      if ((MODE == 1 || p.save_r) && mbar_wait(UB(U_R), 0, ab)) {
         tma_store_2d(&tmR, sA, 0, tokc + 128 * qb);
         bulk_commit();
         bulk_wait0();
@@ -1677,17 +1679,36 @@ cudaError_t launch_prep(const LayerArgs& a, const VecPrep& o, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// The forward's saved buffer on this path: G [B H T, 64], then the decayed operands with L,
+// then R [B H T, 64] (bf16).
+struct SavedVec {
+  VecPrep pr;
+  __nv_bfloat16* R;
+};
+size_t g_plane(const LayerArgs& a) { return align_up((size_t)a.B * a.H * a.T * VD * 2); }
+SavedVec saved_vec(const LayerArgs& a) {
+  SavedVec v{};
+  if (!a.G_saved) return v;
+  uint8_t* base = static_cast<uint8_t*>(a.G_saved) + g_plane(a);
+  v.pr = vec_prep_carve(a, base, true);
+  v.R = reinterpret_cast<__nv_bfloat16*>(base + vec_prep_bytes(a, true));
+  return v;
+}
+
 template <int NB, int LOSS>
 cudaError_t launch_vec(const LayerArgs& a, cudaStream_t s) {
   constexpr int C = 128 * NB, NV = NB * (NB + 1) / 2;
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
   const int BH = a.B * a.H, NC = a.T / C;
-  // workspace: the decayed operands, then (without W_chunks) the chunk-start states
-  const VecPrep pr = vec_prep_carve(a, a.ws, false);
+  // workspace: the decayed operands, then (without W_chunks) the chunk-start states; with
+  // G_saved the decayed operands (L included) and R go to the saved buffer after G instead,
+  // for the backward
+  const SavedVec sv = saved_vec(a);
+  const VecPrep pr = a.G_saved ? sv.pr : vec_prep_carve(a, a.ws, false);
   __nv_bfloat16* Wc = static_cast<__nv_bfloat16*>(
       a.W_chunks ? a.W_chunks
                  : static_cast<void*>(static_cast<uint8_t*>(a.ws) + vec_prep_bytes(a, false)));
-  CUtensorMap tK, tKh, tV, tVc, tQt, tKt, tW, tG;
+  CUtensorMap tK, tKh, tV, tVc, tQt, tKt, tW, tG, tR;
   if (!make_tmap_bf16(&tK, a.K, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tKh, pr.Kh, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tVc, a.V, VD, rows, VD, 64, C) ||
@@ -1695,9 +1716,10 @@ cudaError_t launch_vec(const LayerArgs& a, cudaStream_t s) {
       !make_tmap_bf16(&tQt, pr.Qt, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tKt, pr.Kt, VD, (uint64_t)BH * NC * NV * 128, VD, 64, 128) ||
       !make_tmap_bf16(&tW, Wc, VD, (uint64_t)BH * NC * VD, VD, 64, VD) ||
-      (a.G_saved && !make_tmap_bf16(&tG, a.G_saved, VD, rows, VD, 64, C)))
+      (a.G_saved && !make_tmap_bf16(&tG, a.G_saved, VD, rows, VD, 64, C)) ||
+      (a.G_saved && !make_tmap_bf16(&tR, sv.R, VD, rows, VD, 64, 128)))
     return cudaErrorInvalidValue;
-  if (!a.G_saved) tG = tK;  // never used
+  if (!a.G_saved) tG = tR = tK;  // never used
   VecParams p{};
   p.BH = BH;
   p.T = a.T;
@@ -1711,6 +1733,7 @@ cudaError_t launch_vec(const LayerArgs& a, cudaStream_t s) {
   p.Wc = Wc;
   p.O = static_cast<__nv_bfloat16*>(a.O);
   p.save_g = a.G_saved != nullptr;
+  p.save_r = a.G_saved != nullptr;
   const size_t sm_s = vs_bytes<NB>() + 1024, sm_o = vo_bytes() + 1024;
   auto ks = fwd_vstate_kernel<NB, LOSS>;
   auto ko = fwd_vout_kernel<NB, LOSS, 0>;
@@ -1720,7 +1743,7 @@ cudaError_t launch_vec(const LayerArgs& a, cudaStream_t s) {
     return e;
   if ((e = launch_prep<NB>(a, pr, s))) return e;
   ks<<<BH, kVsThreads, sm_s, s>>>(tK, tKh, tVc, tG, p, a.err);
-  ko<<<BH * NC * NB, kVoThreads, sm_o, s>>>(tQt, tKt, tK, tV, tW, tQt, p, a.err);
+  ko<<<BH * NC * NB, kVoThreads, sm_o, s>>>(tQt, tKt, tK, tV, tW, tR, p, a.err);
   count_launches(2);
   return cudaGetLastError();
 }
@@ -1731,14 +1754,18 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
   constexpr int C = 128 * NB, NV = NB * (NB + 1) / 2;
   const uint64_t rows = (uint64_t)a.B * a.H * a.T;
   const int BH = a.B * a.H, NC = a.T / C;
-  const VecPrep pr = vec_prep_carve(a, a.ws, true);
-  uint8_t* b = static_cast<uint8_t*>(a.ws) + vec_prep_bytes(a, true);
+  // the decayed operands and R: from the forward's saved buffer when given, else formed here
+  const bool saved = a.G_saved != nullptr;
+  const SavedVec sv = saved_vec(a);
+  const VecPrep pr = saved ? sv.pr : vec_prep_carve(a, a.ws, true);
+  uint8_t* b = static_cast<uint8_t*>(a.ws) + (saved ? 0 : vec_prep_bytes(a, true));
   auto take = [&](size_t n) {
     uint8_t* r = b;
     b += align_up(n);
     return r;
   };
-  __nv_bfloat16* R = reinterpret_cast<__nv_bfloat16*>(take(rows * VD * 2));
+  __nv_bfloat16* R =
+      saved ? sv.R : reinterpret_cast<__nv_bfloat16*>(take(rows * VD * 2));
   __nv_bfloat16* Lam = reinterpret_cast<__nv_bfloat16*>(take((size_t)BH * NC * VD * VD * 2));
   float* wl = reinterpret_cast<float*>(take((size_t)BH * NC * 2 * VD * 4));
   float* colk = reinterpret_cast<float*>(take((size_t)BH * NC * NB * 4 * VD * 4));
@@ -1803,12 +1830,15 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
       (e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_k)) ||
       (e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_q)))
     return e;
-  if ((e = launch_prep<NB>(a, pr, s))) return e;
-  kr<<<BH * NC * NB, kVoThreads, sm_r, s>>>(tQt, tKt, tK, tK, tK, tR, vp, a.err);
+  if (!saved) {
+    if ((e = launch_prep<NB>(a, pr, s))) return e;
+    kr<<<BH * NC * NB, kVoThreads, sm_r, s>>>(tQt, tKt, tK, tK, tK, tR, vp, a.err);
+    count_launches(1);
+  }
   kb<<<BH, kVsThreads, sm_b, s>>>(tK, tKh, tR, tdO, bp, a.err);
   kk<<<BH * NC * NB, kVoThreads, sm_k, s>>>(tK, tKh, tV, tKt, tQt, tdO, tW, tLam, gp, a.err);
   kq<<<BH * NC * NB, kVoThreads, sm_q, s>>>(tK, tV, tKt, tdO, tW, gp, a.err);
-  count_launches(4);
+  count_launches(3);
   if (dg) {
     DgParams dp{};
     dp.NB = NB;
@@ -1876,12 +1906,16 @@ cudaError_t tc_vec_fwd(const LayerArgs& a, cudaStream_t s) {
   return a.loss == 0 ? launch_vec<2, 0>(a, s) : launch_vec<2, 1>(a, s);
 }
 
-size_t tc_vec_bwd_workspace(const LayerArgs& a) {
+size_t tc_vec_bwd_workspace(const LayerArgs& a, bool g_saved) {
   const size_t rows = (size_t)a.B * a.H * a.T, BH = (size_t)a.B * a.H, NC = a.T / a.C;
   const size_t NB = a.C / 128;
-  return vec_prep_bytes(a, true) + align_up(rows * VD * 2) + align_up(BH * NC * VD * VD * 2) +
-         align_up(BH * NC * 2 * VD * 4) + align_up(BH * NC * NB * 4 * VD * 4) +
-         2 * align_up(rows * VD * 4);
+  return (g_saved ? 0 : vec_prep_bytes(a, true) + align_up(rows * VD * 2)) +
+         align_up(BH * NC * VD * VD * 2) + align_up(BH * NC * 2 * VD * 4) +
+         align_up(BH * NC * NB * 4 * VD * 4) + 2 * align_up(rows * VD * 4);
+}
+
+size_t tc_vec_saved_bytes(const LayerArgs& a) {
+  return g_plane(a) + vec_prep_bytes(a, true) + align_up((size_t)a.B * a.H * a.T * VD * 2);
 }
 
 cudaError_t tc_vec_bwd(const LayerArgs& a, cudaStream_t s) {
