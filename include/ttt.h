@@ -86,6 +86,10 @@ typedef struct {
   int act;         /* ttt_act applied to both the train view and the query view         */
   float lr_bias;   /* b in eta_t = 2 sigmoid(beta_t + b)                                 */
   int decay;       /* ttt_decay: layout of gamma (zero-initialised configs: scalar)      */
+  int w0_shared;   /* 0: W0 (and W1_0, W2_0 of TTT-MLP) holds one initial state per sequence
+                      and head, [B, H, ...]; 1: one per head, [H, ...], shared by the B
+                      sequences. W_final, W_chunks and dW0 stay per sequence either way; a
+                      caller that shares W0 sums dW0 over B. Zero-initialised configs: 0.  */
 } ttt_config;
 
 /* Layouts (all contiguous):

@@ -290,6 +290,16 @@ def test_context_parallel_calls_check_arguments():
     assert a(None, A, 8, None) == ttt.ERR_INVALID_ARG
 
 
+def test_shared_initial_state_flag_is_validated():
+    c = _cfg()
+    c.w0_shared = 1
+    assert ttt.ttt_workspace_bytes(c, 0) == 0
+    c.w0_shared = 2
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_workspace_bytes(c, 0)
+    assert _cfg(w0_shared=True).w0_shared == 1
+
+
 def test_saved_buffer_size():
     cfg = _cfg(dtype="bf16", dk=128, dv=96, C=128, T=512)
     assert ttt.ttt_saved_bytes(cfg) == 2 * 3 * 512 * 96 * 2
@@ -336,7 +346,7 @@ C_CLIENT = r"""
    link, and argument errors must come back as statuses with nothing launched. */
 int main(void) {
   ttt_config c = {2, 3, 256, 64, 64, 64, TTT_F32, TTT_LOSS_MSE, TTT_ACT_ID, -2.9f,
-                  TTT_DECAY_SCALAR};
+                  TTT_DECAY_SCALAR, 0};
   char a[64];
   void* p = (void*)(((unsigned long)a + 15) & ~15ul); /* aligned, never dereferenced */
   int bad = 0;

@@ -39,7 +39,8 @@ class ttt_config(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("C", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("loss", ctypes.c_int), ("act", ctypes.c_int),
-                ("lr_bias", ctypes.c_float), ("decay", ctypes.c_int)]
+                ("lr_bias", ctypes.c_float), ("decay", ctypes.c_int),
+                ("w0_shared", ctypes.c_int)]
 
 
 _p, _i, _u, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_float, ctypes.c_size_t
@@ -126,11 +127,13 @@ def _check(status: int, where: str):
 
 
 def make_config(B, H, T, dk, dv, C, dtype="bf16", loss="mse", act="id", lr_bias=0.0,
-                decay="scalar") -> ttt_config:
-    """decay: "scalar" (gamma [B,H,T], or no gamma) or "vector" (gamma [B,H,T,dk])."""
+                decay="scalar", w0_shared=False) -> ttt_config:
+    """decay: "scalar" (gamma [B,H,T], or no gamma) or "vector" (gamma [B,H,T,dk]).
+    w0_shared: W0 (W1_0, W2_0 for TTT-MLP) is [H, ...], one initial state per head shared by
+    the batch, instead of [B, H, ...]."""
     return ttt_config(B, H, T, dk, dv, C, F32 if dtype in ("f32", F32) else BF16,
                       LOSS.get(loss, loss), ACT.get(act, act), float(lr_bias),
-                      DECAY.get(decay, decay))
+                      DECAY.get(decay, decay), int(bool(w0_shared)))
 
 
 def ttt_saved_bytes(cfg: ttt_config) -> int:

@@ -59,6 +59,7 @@ ttt_status check_config(const ttt_config* c) {
   if (c->act != TTT_ACT_ID && c->act != TTT_ACT_SILU) return TTT_ERR_INVALID_ARG;
   if (!isfinite(c->lr_bias)) return TTT_ERR_INVALID_ARG;
   if (c->decay != TTT_DECAY_SCALAR && c->decay != TTT_DECAY_VECTOR) return TTT_ERR_INVALID_ARG;
+  if (c->w0_shared != 0 && c->w0_shared != 1) return TTT_ERR_INVALID_ARG;
   if ((long long)c->B * c->H * c->T * (c->dk > c->dv ? c->dk : c->dv) > (1ll << 40))
     return TTT_ERR_INVALID_ARG;
   // token rows are addressed with 32-bit indices (and TMA coordinates) inside the kernels
@@ -81,6 +82,7 @@ LayerArgs args_of(const ttt_config* c) {
   a.act = c->act;
   a.lr_bias = c->lr_bias;
   a.gvec = c->decay == TTT_DECAY_VECTOR;
+  a.w0_mod = c->w0_shared ? c->H : c->B * c->H;
   return a;
 }
 

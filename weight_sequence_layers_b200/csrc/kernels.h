@@ -10,6 +10,7 @@ struct LayerArgs {
   int B, H, T, dk, dv, C, dtype, loss, act;
   float lr_bias;
   int gvec;  // gamma is [B, H, T, dk]: one decay per key feature
+  int w0_mod;  // the initial state of (batch, head) bh is block bh % w0_mod of W0 (H: shared)
   const void *Q, *K, *V;
   const float *beta, *gamma, *W0;
   void* O;

@@ -49,7 +49,8 @@ struct FwdParams {
   float lr_bias;
   const float* beta;
   const float* gamma;     // nullable
-  const float* W0;        // [BH, D, D] fp32
+  const float* W0;        // [BH, D, D] fp32 (or [H, D, D]: block bh % w0_mod)
+  int w0_mod;
   __nv_bfloat16* O;       // [BH, T, D]
   float* W_final;         // nullable
   __nv_bfloat16* W_chunks;  // nullable, [BH, NC, D, D]
@@ -348,13 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lrow = q * 32 + lane;   // TMEM lane = row inside a 128-row block
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const bool w_rows = q * 32 < D;   // this warp holds state rows
+    // this thread's 32 state entries: in W_final (per sequence) and in W0 (maybe shared)
     const size_t wofs = (size_t)bh * D * D + (size_t)lrow * D + NV * slice + 32 * g;
+    const size_t w0ofs = (size_t)(bh % p.w0_mod) * D * D + (size_t)lrow * D + NV * slice + 32 * g;
     bool ok = true;
     // initial state: Gamma_C(0) W0 into TMEM, bf16 operand copy, chunk-0 checkpoint
     if (!mbar_wait(BAR(scan_full[0]), 0, ab)) ok = false;
     if (ok && w_rows) {
       float w[32];
-      const float4* src = reinterpret_cast<const float4*>(p.W0 + wofs);
+      const float4* src = reinterpret_cast<const float4*>(p.W0 + w0ofs);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float4 v = src[k];
@@ -589,6 +592,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
   p.beta = a.beta;
   p.gamma = a.gamma;
   p.W0 = a.W0;
+  p.w0_mod = a.w0_mod;
   p.O = static_cast<__nv_bfloat16*>(a.O);
   p.W_final = a.W_final;
   p.W_chunks = static_cast<__nv_bfloat16*>(a.W_chunks);

@@ -22,6 +22,7 @@ namespace {
 struct MlpDims {
   int T, dk, dv, h, C, loss, act, has_gamma;
   float lr_bias;
+  int w0_mod;
 };
 
 // Per-head scratch, in floats.
@@ -154,9 +155,10 @@ __global__ void __launch_bounds__(512)
   const int C = d.C, dk = d.dk, dv = d.dv, h = d.h, NC = d.T / d.C;
   const MlpScratch S = carve(ws + (size_t)bh * mlp_head_floats(C, dk, dv, h), d);
   const size_t n1 = (size_t)dk * h, n2 = (size_t)h * dv;
-  for (size_t e = threadIdx.x; e < n1; e += blockDim.x) S.W1[e] = W1_0[bh * n1 + e];
+  const size_t b0 = (size_t)(bh % d.w0_mod);
+  for (size_t e = threadIdx.x; e < n1; e += blockDim.x) S.W1[e] = W1_0[b0 * n1 + e];
   for (size_t e = threadIdx.x; e < n2; e += blockDim.x) {
-    S.W2[e] = W2_0[bh * n2 + e];
+    S.W2[e] = W2_0[b0 * n2 + e];
     S.W2T[(e % dv) * h + e / dv] = S.W2[e];
   }
   __syncthreads();
@@ -408,7 +410,8 @@ __global__ void __launch_bounds__(512)
 }
 
 MlpDims mlp_dims(const LayerArgs& a, int hidden) {
-  return MlpDims{a.T, a.dk, a.dv, hidden, a.C, a.loss, a.act, a.gamma != nullptr, a.lr_bias};
+  return MlpDims{a.T, a.dk, a.dv, hidden, a.C, a.loss, a.act, a.gamma != nullptr, a.lr_bias,
+                 a.w0_mod};
 }
 
 }  // namespace

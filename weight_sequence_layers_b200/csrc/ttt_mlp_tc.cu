@@ -380,17 +380,18 @@ __device__ void copy_to(const float* src, size_t n, TA* dst, TB* dst2) {
 }
 
 // Chunk-0 weights: the masters and operand copies from W1_0 [64, h] and W2_0 [h, 64].
+// (initial weights of head b are block b % w0_mod of W1_0 / W2_0)
 __global__ void __launch_bounds__(256)
-    mlp_init_kernel(int h, int NC, const float* W1_0, const float* W2_0, float* W1Tm, float* W2m,
-                    __nv_bfloat16* W1Tc, __nv_bfloat16* W2c, __nv_bfloat16* W2Tc, float* W1c,
-                    float* W2c_out) {
+    mlp_init_kernel(int h, int NC, int w0_mod, const float* W1_0, const float* W2_0, float* W1Tm,
+                    float* W2m, __nv_bfloat16* W1Tc, __nv_bfloat16* W2c, __nv_bfloat16* W2Tc,
+                    float* W1c, float* W2c_out) {
   __shared__ float tile[32][33];
-  const size_t b = blockIdx.x, n = (size_t)h * D;
-  transpose_to(W1_0 + b * n, D, h, W1Tm + b * n, W1Tc + b * NC * n, tile);
-  transpose_to(W2_0 + b * n, h, D, W2Tc + b * NC * n, (float*)nullptr, tile);
-  copy_to(W2_0 + b * n, n, W2m + b * n, W2c + b * NC * n);
-  copy_to(W1_0 + b * n, n, W1c ? W1c + b * NC * n : nullptr, (float*)nullptr);
-  copy_to(W2_0 + b * n, n, W2c_out ? W2c_out + b * NC * n : nullptr, (float*)nullptr);
+  const size_t b = blockIdx.x, n = (size_t)h * D, b0 = b % w0_mod;
+  transpose_to(W1_0 + b0 * n, D, h, W1Tm + b * n, W1Tc + b * NC * n, tile);
+  transpose_to(W2_0 + b0 * n, h, D, W2Tc + b * NC * n, (float*)nullptr, tile);
+  copy_to(W2_0 + b0 * n, n, W2m + b * n, W2c + b * NC * n);
+  copy_to(W1_0 + b0 * n, n, W1c ? W1c + b * NC * n : nullptr, (float*)nullptr);
+  copy_to(W2_0 + b0 * n, n, W2c_out ? W2c_out + b * NC * n : nullptr, (float*)nullptr);
 }
 
 // ---------------------------------------------------------------------------- host side
@@ -475,8 +476,8 @@ cudaError_t mlp_tc_fwd_impl(const LayerArgs& a, int h, const float* W1_0, const 
   MCtx x{T, C, NC, h, a.loss, f.Eb, f.Lb};
   cudaError_t e;
   mlp_scan_kernel<<<BH * NC, 256, 0, s>>>(C, a.gamma, a.beta, a.lr_bias, Q, f.Lb, f.Eb, f.Qh);
-  mlp_init_kernel<<<BH, 256, 0, s>>>(h, NC, W1_0, W2_0, f.W1Tm, f.W2m, f.W1Tc, f.W2c, f.W2Tc,
-                                      W1c, W2c_out);
+  mlp_init_kernel<<<BH, 256, 0, s>>>(h, NC, a.w0_mod, W1_0, W2_0, f.W1Tm, f.W2m, f.W1Tc, f.W2c,
+                                      f.W2Tc, W1c, W2c_out);
   count_launches(2);
   if ((e = cudaGetLastError())) return e;
   // maps that do not move with the chunk

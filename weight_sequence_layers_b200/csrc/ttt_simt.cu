@@ -32,6 +32,7 @@ constexpr int kMaxD = 128;
 struct Dims {
   int T, dk, dv, C, loss, act, has_gamma, gvec;
   float lr_bias;
+  int w0_mod;
 };
 
 // Entries of the log-decay prefix per chunk position: one, or one per key feature.
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
   for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
     const int i = e / nv, j = e % nv;
-    Ws[i * kNvs + j] = W0[(size_t)bh * dk * dv + (size_t)i * dv + j0 + j];
+    Ws[i * kNvs + j] = W0[(size_t)(bh % d.w0_mod) * dk * dv + (size_t)i * dv + j0 + j];
   }
   __syncthreads();
   for (int c = 0; c < NC; ++c) {
@@ -461,7 +462,8 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
 }
 
 Dims dims_of(const LayerArgs& a) {
-  return Dims{a.T, a.dk, a.dv, a.C, a.loss, a.act, a.gamma != nullptr, a.gvec, a.lr_bias};
+  return Dims{a.T, a.dk, a.dv, a.C, a.loss, a.act, a.gamma != nullptr, a.gvec, a.lr_bias,
+              a.w0_mod};
 }
 
 // Elements of one [B, H, T, dv] plane: with SiLU, Zq follows G in the saved buffer.

@@ -45,7 +45,8 @@ struct VecParams {
   int BH, T, NC;
   float lr_bias;
   const float* beta;
-  const float* W0;      // [BH, 64, 64]
+  const float* W0;      // [BH, 64, 64] (or [H, 64, 64]: block bh % w0_mod)
+  int w0_mod;
   const float* GC;      // [BH, NC, 64] exp(L_C)
   const float* Em;      // [BH, NC, NB, 64] exp(L_m)
   float* W_final;       // nullable
@@ -322,7 +323,8 @@ __global__ void __launch_bounds__(kVsThreads, 1)
     if (w_rows) {
       // chunk 0: the bf16 operand copy of W0, its checkpoint, diag(Gamma_C(0)) W0 into TMEM
       float w[32];
-      const float4* src = reinterpret_cast<const float4*>(p.W0 + ((size_t)bh * VD + lrow) * VD + col);
+      const float4* src =
+          reinterpret_cast<const float4*>(p.W0 + ((size_t)(bh % p.w0_mod) * VD + lrow) * VD + col);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const float4 v = src[k];
@@ -1727,6 +1729,7 @@ cudaError_t launch_vec(const LayerArgs& a, cudaStream_t s) {
   p.lr_bias = a.lr_bias;
   p.beta = a.beta;
   p.W0 = a.W0;
+  p.w0_mod = a.w0_mod;
   p.GC = pr.GC;
   p.Em = pr.Em;
   p.W_final = a.W_final;
