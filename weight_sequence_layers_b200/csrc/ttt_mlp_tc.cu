@@ -34,6 +34,11 @@ struct MCtx {
   int loss;
   const float* Eb;  // [BH, T] eta_t = 2 sigmoid(beta_t + b)
   const float* Lb;  // [BH, T] chunk-local L (zeros without a decay)
+  // with g(t) the first token of t's 32-token group: Cr_t = eta_t exp(L_g(t) - L_t) and
+  // Cf_t = exp(L_t - L_g(t)), so that a score weight eta_r exp(L_s - L_r) over a group of 32
+  // keys (or queries) costs one exponential per row and group
+  const float* Cr;
+  const float* Cf;
 };
 __device__ __forceinline__ float eta_at(const MCtx& x, size_t tok) { return __ldg(x.Eb + tok); }
 // u_r = eta_r exp(L_C - L_r) of token tok of the chunk starting at tok0
@@ -249,12 +254,11 @@ struct EpiScore {
   }
   __device__ void chunk(St& st, int col0, float (&v)[32]) const {
     if (col0 <= st.s) {  // else every key of the group follows the query: zeros
-      float e[32], l[32];
-      ld_f32x32(x.Eb + st.tok0 + col0, e);
-      ld_f32x32(x.Lb + st.tok0 + col0, l);
+      float c[32];
+      ld_f32x32(x.Cr + st.tok0 + col0, c);
+      const float rho = -__expf(st.Ls - __ldg(x.Lb + st.tok0 + col0));
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        v[j] = col0 + j <= st.s ? -e[j] * __expf(st.Ls - l[j]) * v[j] : 0.f;
+      for (int j = 0; j < 32; ++j) v[j] = col0 + j <= st.s ? rho * c[j] * v[j] : 0.f;
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -305,7 +309,8 @@ struct EpiOut {
 __global__ void __launch_bounds__(256) mlp_scan_kernel(int C, const float* gamma,
                                                        const float* beta, float lr_bias,
                                                        const __nv_bfloat16* Q, float* Lb,
-                                                       float* Eb, __nv_bfloat16* Qh,
+                                                       float* Eb, float* Cr, float* Cf,
+                                                       __nv_bfloat16* Qh,
                                                        const __nv_bfloat16* dO = nullptr,
                                                        __nv_bfloat16* dOh = nullptr) {
   __shared__ float sL[256];
@@ -330,7 +335,12 @@ __global__ void __launch_bounds__(256) mlp_scan_kernel(int C, const float* gamma
     for (int k = 0; k < per; ++k) sL[lane * per + k] = excl + loc[k];
   }
   __syncthreads();
-  for (int t = threadIdx.x; t < C; t += blockDim.x) Lb[tok0 + t] = sL[t];
+  for (int t = threadIdx.x; t < C; t += blockDim.x) {
+    Lb[tok0 + t] = sL[t];
+    const float e = sL[t] - sL[t & ~31];
+    Cr[tok0 + t] = 2.f * sigm(__ldg(beta + tok0 + t) + lr_bias) * __expf(-e);
+    Cf[tok0 + t] = __expf(e);
+  }
   auto scale = [&](const __nv_bfloat16* src, __nv_bfloat16* dst) {
     for (int e = threadIdx.x; e < C * D / 8; e += blockDim.x) {
       const int t = e / (D / 8), q8 = e % (D / 8);
@@ -424,7 +434,7 @@ bg::Prob prob1(int K, int a_k0, int a_row, int b_k0, int b_row) {
 }
 
 struct FwdBufs {
-  float *Lb, *Eb, *W1Tm, *W2m, *Zs;
+  float *Lb, *Eb, *Cr, *Cf, *W1Tm, *W2m, *Zs;
   __nv_bfloat16 *Qh, *W1Tc, *W2c, *W2Tc, *A1, *A1T, *G2, *uG2, *G1T, *uG1T, *S1, *Aq, *Ahq, *S2;
 };
 
@@ -443,6 +453,8 @@ size_t carve_fwd(const LayerArgs& a, int h, void* base, FwdBufs* f) {
   FwdBufs b{};
   b.Lb = (float*)take(rows * 4);
   b.Eb = (float*)take(rows * 4);
+  b.Cr = (float*)take(rows * 4);
+  b.Cf = (float*)take(rows * 4);
   b.W1Tm = (float*)take(BH * h * D * 4);
   b.W2m = (float*)take(BH * h * D * 4);
   b.Zs = (float*)take(BH * C * h * 4);
@@ -473,9 +485,10 @@ cudaError_t mlp_tc_fwd_impl(const LayerArgs& a, int h, const float* W1_0, const 
   const auto* Q = static_cast<const __nv_bfloat16*>(a.Q);
   const auto* K = static_cast<const __nv_bfloat16*>(a.K);
   const auto* V = static_cast<const __nv_bfloat16*>(a.V);
-  MCtx x{T, C, NC, h, a.loss, f.Eb, f.Lb};
+  MCtx x{T, C, NC, h, a.loss, f.Eb, f.Lb, f.Cr, f.Cf};
   cudaError_t e;
-  mlp_scan_kernel<<<BH * NC, 256, 0, s>>>(C, a.gamma, a.beta, a.lr_bias, Q, f.Lb, f.Eb, f.Qh);
+  mlp_scan_kernel<<<BH * NC, 256, 0, s>>>(C, a.gamma, a.beta, a.lr_bias, Q, f.Lb, f.Eb, f.Cr, f.Cf,
+                                          f.Qh);
   mlp_init_kernel<<<BH, 256, 0, s>>>(h, NC, a.w0_mod, W1_0, W2_0, f.W1Tm, f.W2m, f.W1Tc, f.W2c,
                                       f.W2Tc, W1c, W2c_out);
   count_launches(2);
@@ -707,11 +720,11 @@ struct EpiScoreT {
   }
   __device__ void chunk(St& st, int col0, float (&v)[32]) const {
     if (col0 + 31 >= st.r) {  // else every query of the group precedes the key: zeros
-      float l[32];
-      ld_f32x32(x.Lb + st.tok0 + col0, l);
+      float c[32];
+      ld_f32x32(x.Cf + st.tok0 + col0, c);
+      const float rho = st.ne * __expf(__ldg(x.Lb + st.tok0 + col0) - st.Lr);
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        v[j] = col0 + j >= st.r ? st.ne * __expf(l[j] - st.Lr) * v[j] : 0.f;
+      for (int j = 0; j < 32; ++j) v[j] = col0 + j >= st.r ? rho * c[j] * v[j] : 0.f;
     } else {
 #pragma unroll
       for (int j = 0; j < 32; ++j) v[j] = 0.f;
@@ -767,14 +780,15 @@ struct EpiDST {
   }
   __device__ void chunk(St& st, int col0, float (&v)[32]) const {
     if (col0 + 31 >= st.r) {
-      float sn[32], l[32];
+      float sn[32], c[32];
       ld_bf16x32(StN + (st.tok0 + st.r) * x.C + col0, sn);
-      ld_f32x32(x.Lb + st.tok0 + col0, l);
+      ld_f32x32(x.Cf + st.tok0 + col0, c);
+      const float rho = st.eta * __expf(__ldg(x.Lb + st.tok0 + col0) - st.Lr);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float ds = col0 + j >= st.r ? -v[j] : 0.f;
         st.acc -= ds * sn[j];
-        v[j] = st.eta * __expf(l[j] - st.Lr) * ds;
+        v[j] = rho * c[j] * ds;
       }
     } else {
 #pragma unroll
@@ -1040,7 +1054,7 @@ __global__ void __launch_bounds__(256)
 }
 
 struct BwdBufs {
-  float *Lb, *Eb, *Z1, *dG2s, *dKs, *deta, *dZ1a, *dA1, *Ya, *ykg, *yag, *Wh1m, *Wh2m;
+  float *Lb, *Eb, *Cr, *Cf, *Z1, *dG2s, *dKs, *deta, *dZ1a, *dA1, *Ya, *ykg, *yag, *Wh1m, *Wh2m;
   __nv_bfloat16 *Qh, *dOh, *W1T, *W1, *W2, *W2T, *A1, *Bm, *G1, *uG1n, *Aq, *dAct, *dZq, *dZqh,
       *dA1s, *dG1s, *A1T, *G1T, *AqT, *AhqT, *dZqT, *G2, *uG2n, *S1n, *S1nT, *S2nT, *D2T, *D2,
       *D1T, *D1, *dB, *dBT, *dG2, *dZ1, *dZ1T, *Wh1T_b, *Wh1_b, *Wh2_b, *Wh2T_b;
@@ -1060,6 +1074,8 @@ size_t carve_bwd(const LayerArgs& a, int h, void* base, BwdBufs* f) {
   BwdBufs b{};
   b.Lb = f32(rows);
   b.Eb = f32(rows);
+  b.Cr = f32(rows);
+  b.Cf = f32(rows);
   b.deta = f32(rows);
   b.Qh = bf(rows * D);
   b.dOh = bf(rows * D);
@@ -1115,10 +1131,10 @@ cudaError_t mlp_tc_bwd_impl(const LayerArgs& a, int h, const float* W1c, const f
   const auto* K = static_cast<const __nv_bfloat16*>(a.K);
   const auto* V = static_cast<const __nv_bfloat16*>(a.V);
   const auto* dO = static_cast<const __nv_bfloat16*>(a.dO);
-  const MCtx x{T, C, NC, h, a.loss, f.Eb, f.Lb};
+  const MCtx x{T, C, NC, h, a.loss, f.Eb, f.Lb, f.Cr, f.Cf};
   cudaError_t e;
-  mlp_scan_kernel<<<NB, 256, 0, s>>>(C, a.gamma, a.beta, a.lr_bias, Q, f.Lb, f.Eb, f.Qh, dO,
-                                     f.dOh);
+  mlp_scan_kernel<<<NB, 256, 0, s>>>(C, a.gamma, a.beta, a.lr_bias, Q, f.Lb, f.Eb, f.Cr, f.Cf,
+                                     f.Qh, dO, f.dOh);
   mlp_bwd_init_kernel<<<NB, 256, 0, s>>>(h, NC, W1c, W2c, dW1f, dW2f, f.W1T, f.W1, f.W2, f.W2T,
                                           f.Wh1m, f.Wh2m, f.Wh1T_b, f.Wh1_b, f.Wh2_b, f.Wh2T_b);
   count_launches(2);
