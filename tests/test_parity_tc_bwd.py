@@ -108,3 +108,25 @@ def test_tc_single_chunk(d, C, act):
     ref = oracle_bwd(cfg, inp)
     for k in GRADS + ("dgamma",):
         assert rel_err(got[k], ref[k]) <= TOL, (k, rel_err(got[k], ref[k]))
+
+
+def test_silu_backward_without_saved_zq_is_refused():
+    # the SiLU backward on a tensor-core shape reads the forward's Zq from G_saved; called
+    # without it on real device tensors it returns TTT_ERR_UNSUPPORTED and touches no output
+    import weight_sequence_layers_b200 as ttt
+    from _runners import abi_config
+    cfg = synth.SILU_IP_FWD.replace(B=1, H=2, T=512, loss="mse")
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=71)
+    fwd = run_fwd(cfg, inp)
+    c = abi_config(cfg)
+    n = ttt.ttt_workspace_bytes(c, 2)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    outs = [torch.full_like(inp[k], float("nan")) for k in ("Q", "K", "V", "beta")]
+    dW0 = torch.full_like(inp["W0"], float("nan"))
+    with pytest.raises(ttt.TTTError) as e:
+        ttt.ttt_chunk_bwd(c, inp["Q"], inp["K"], inp["V"], inp["beta"], inp["gamma"], inp["W0"],
+                          fwd["W_chunks"], None, inp["dO"], None, None, None, *outs, dW0, None,
+                          ws, n)
+    assert e.value.status == ttt.ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert all(torch.isnan(t.float()).all() for t in outs + [dW0])
