@@ -62,6 +62,8 @@ struct VecPrep {
   float* GC;  // float32 [B H NC, 64]: exp(L_C)
   float* Em;  // float32 [B H NC NB, 64]: exp(L_m(qb))
   float* Lf;  // nullable: float32 [B H T, 64], L itself
+  void* Qt2;  // nullable (C = 256, with L): bf16 [B H NC 128, 64], the second query block's
+              // q_s exp(L_s - L_m(0)) (the backward's key side refers both blocks to m(0))
 };
 size_t vec_prep_bytes(const LayerArgs& a, bool with_L);
 VecPrep vec_prep_carve(const LayerArgs& a, void* base, bool with_L);

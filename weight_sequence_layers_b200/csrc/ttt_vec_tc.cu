@@ -74,6 +74,7 @@ struct PrepParams {
   const __nv_bfloat16* Q;
   const __nv_bfloat16* K;
   __nv_bfloat16 *Qt, *Kh, *Kt;
+  __nv_bfloat16* Qt2;  // nullable (C = 256): second-block queries against the first reference
   float *GC, *Em, *Lf;
   unsigned* err;
 };
@@ -166,6 +167,11 @@ __global__ void __launch_bounds__(kPrepThreads) vec_prep_kernel(const PrepParams
           scale4(kv[t], make_float4(m.x - L.x, m.y - L.y, m.z - L.z, m.w - L.w), range);
     }
     if (p.Lf) reinterpret_cast<float4*>(p.Lf + r0 * VD)[o + fq] = L;
+    if (NB == 2 && kb == 1 && p.Qt2) {  // exponents <= 0: the reference precedes the token
+      const float4 m = Lm[0];
+      reinterpret_cast<uint2*>(p.Qt2 + (bc * 128 + tr) * VD)[fq] =
+          scale4(qv[t], make_float4(L.x - m.x, L.y - m.y, L.z - m.z, L.w - m.w), range);
+    }
   }
   if (seg == 0) {
     reinterpret_cast<float4*>(p.GC + bc * VD)[fq] =
@@ -1004,6 +1010,7 @@ struct VgParams {
   const float* Lf;        // [BH, T, 64] chunk-local L
   const float* Em;        // [BH, NC, NB, 64]
   const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
   __nv_bfloat16 *dQ, *dK, *dV;
   float* dbeta;
   float* dLk;             // nullable: -k * (dK - dG W0^T), [BH, T, 64]
@@ -1012,69 +1019,85 @@ struct VgParams {
 };
 
 // ------------------------------------------------------------- key side: dK, dV, dbeta
-// One CTA per (batch, head, chunk, 128-key block kb), one per SM. Shared memory (16 KB panels):
-//   0: K_kb      1: Khat_kb, then dG (bf16)      2: V_kb, then G (bf16, in place)
-//   3 + 3 qi: ktilde (qb, kb)   4 + 3 qi: qtilde_qb   5 + 3 qi: dO_qb
-// for the query blocks qb = kb + qi; W0 and Lambda (64 x 64 bf16) after them.
-// TMEM (512 columns): [0,64) G then (eta dS^T) qtilde of qi = 0; [64,128) X then the same of
-// qi = 1; [128,256) P^T then G Lambda^T and dG W0^T; [256,384) G dO^T, then eta dS^T packed to
-// bf16 in its first 64 columns; [384,448) packed S^T; [448,512) dG accumulator (from eta X).
-template <int NB>
+// One CTA per (batch, head, chunk, 128-key block kb), two per SM. Every query block qb >= kb
+// is taken in two halves of 64 queries, with both operands referred to the key block's
+// reference token m(kb): ktilde (kb, kb) for the keys and, for the queries, qtilde (qb = kb) or
+// the prep pass's second-block copy against m(0) (qb = kb + 1, kb = 0), so one accumulator
+// holds (eta dS^T) qtilde' over all query blocks and dK^S = exp(L_m(kb) - L) * that.
+// Shared memory (16 KB panels unless stated): K (MSE: the G product; then a query-half slot),
+// V (then G, bf16, in place), Khat (then dG, bf16), W0 and Lambda (8 KB each), ktilde (kb, kb),
+// a query-half slot (qtilde' half, then dO half, 8 KB each). Query halves alternate between the
+// two slots. TMEM (256 columns): [0,64) G (MSE), then the dK^S accumulator; [64,128) X, then
+// eta X and the dG accumulator; [128,192) P^T of a half, S^T packed over it; [192,256) G dO^T
+// of a half, eta dS^T packed over it; after the last half G Lambda^T and dG W0^T go to
+// [128,192) and [192,256).
 struct KgL {
-  static constexpr uint32_t OFF_W = (3 + 3 * NB) * PANEL;
-  static constexpr uint32_t OFF_L = OFF_W + VD * 128;
-  static constexpr uint32_t OFF_F = OFF_L + VD * 128;  // L_m[NB][64], L_C[64]
-  static constexpr uint32_t OFF_BAR = OFF_F + (NB + 1) * VD * 4;
-  static constexpr uint32_t T_G = 0, T_X = 64, T_P = 128, T_DS = 256, T_S = 384, T_DG = 448;
+  static constexpr uint32_t OFF_K = 0, OFF_V = PANEL, OFF_KH = 2 * PANEL, OFF_KT = 3 * PANEL,
+                            OFF_HA = 4 * PANEL, OFF_W = 5 * PANEL, OFF_L = OFF_W + VD * 128;
+  static constexpr uint32_t HALF = 64 * 128;               // 64 rows x 64 bf16
+  static constexpr uint32_t OFF_F = OFF_L + VD * 128;      // L_m(kb)[64], L_C[64]
+  static constexpr uint32_t OFF_BAR = OFF_F + 2 * VD * 4;
+  static constexpr uint32_t T_DKS = 0, T_DG = 64, T_P = 128, T_DS = 192;
 };
-enum { K_LDA, K_LDQ0, K_LDQ1, K_GA, K_GRDY, K_PS0, K_PS1, K_PK0, K_PK1, K_DK0, K_DK1, K_GL,
-       K_DGRDY, K_DGW, K_F, K_NBARS };
+enum { K_LDA, K_LDH0, K_LDH1, K_GA, K_GRDY, K_PS, K_PK, K_ST0, K_ST1, K_GL, K_DGRDY, K_DGW, K_F,
+       K_NBARS };
 struct __align__(8) KgBars {
   uint64_t b[K_NBARS];
   uint32_t tmem_base;
   int abort_flag;
 };
-template <int NB>
-constexpr uint32_t kg_bytes() { return KgL<NB>::OFF_BAR + sizeof(KgBars); }
+constexpr uint32_t kg_bytes() { return KgL::OFF_BAR + sizeof(KgBars); }
+
+__device__ __forceinline__ void ldg_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint4 u = __ldg(s4 + k);
+    v[8 * k] = bf16lo(u.x); v[8 * k + 1] = bf16hi(u.x);
+    v[8 * k + 2] = bf16lo(u.y); v[8 * k + 3] = bf16hi(u.y);
+    v[8 * k + 4] = bf16lo(u.z); v[8 * k + 5] = bf16hi(u.z);
+    v[8 * k + 6] = bf16lo(u.w); v[8 * k + 7] = bf16hi(u.w);
+  }
+}
 
 template <int NB, int LOSS>
-__global__ void __launch_bounds__(kVoThreads, 1)
+__global__ void __launch_bounds__(kVoThreads, 2)
     bwd_vkey_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKh,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
-                    const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmdO,
-                    const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmLam,
-                    const VgParams p, unsigned* err) {
+                    const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQ2h,
+                    const __grid_constant__ CUtensorMap tmdOh, const __grid_constant__ CUtensorMap tmW,
+                    const __grid_constant__ CUtensorMap tmLam, const VgParams p, unsigned* err) {
   constexpr int C = 128 * NB, NV = NB * (NB + 1) / 2;
-  using L = KgL<NB>;
+  using L = KgL;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const uint32_t sb = smem_u32(smem);
-  const uint32_t sK = sb, sKH = sb + PANEL, sV = sb + 2 * PANEL, sW = sb + L::OFF_W,
-                 sL = sb + L::OFF_L;
-  auto sKT = [&](int qi) { return sb + (3 + 3 * qi) * PANEL; };
-  auto sQT = [&](int qi) { return sb + (4 + 3 * qi) * PANEL; };
-  auto sDO = [&](int qi) { return sb + (5 + 3 * qi) * PANEL; };
+  const uint32_t sK = sb + L::OFF_K, sV = sb + L::OFF_V, sKH = sb + L::OFF_KH,
+                 sKT = sb + L::OFF_KT, sW = sb + L::OFF_W, sL = sb + L::OFF_L;
+  // query half h lives in slot h & 1: the half slot, or the K panel once K is no longer read
+  auto sQh = [&](int h) { return (h & 1) ? sK : sb + L::OFF_HA; };
+  auto sDOh = [&](int h) { return sQh(h) + L::HALF; };
   float* f_Lm = reinterpret_cast<float*>(smem + L::OFF_F);
-  float* f_LC = f_Lm + NB * VD;
+  float* f_LC = f_Lm + VD;
   KgBars* bars = reinterpret_cast<KgBars*>(smem + L::OFF_BAR);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int per_c = p.BH * NB;
   const int c = p.NC - 1 - (int)blockIdx.x / per_c;
   const int rem = (int)blockIdx.x % per_c;
   const int bh = rem / NB, kb = rem % NB;
-  const int NQ = NB - kb;
+  const int NH = 2 * (NB - kb);  // query halves at or after this key block
   const int tokc = bh * p.T + c * C;
   const int bc = bh * p.NC + c;
   Abort ab{&bars->abort_flag, err};
 #define KB(i) smem_u32(&bars->b[i])
   if (threadIdx.x == 0) {
     for (int i = 0; i < K_NBARS; ++i)
-      mbar_init(KB(i), (i == K_GRDY || i == K_PK0 || i == K_PK1 || i == K_DGRDY || i == K_F) ? 4 : 1);
+      mbar_init(KB(i), (i == K_GRDY || i == K_PK || i == K_DGRDY || i == K_F) ? 4 : 1);
     bars->abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(&bars->tmem_base), 512);
+    tmem_alloc(smem_u32(&bars->tmem_base), 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -1085,73 +1108,81 @@ __global__ void __launch_bounds__(kVoThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       const int tk = tokc + 128 * kb;
-      mbar_arrive_expect_tx(KB(K_LDA), 3 * PANEL + 2 * VD * 128);
-      tma_load_2d(sK, &tmK, KB(K_LDA), 0, tk);
+      mbar_arrive_expect_tx(KB(K_LDA), (LOSS == 0 ? 4 : 3) * PANEL + 2 * VD * 128);
+      if (LOSS == 0) tma_load_2d(sK, &tmK, KB(K_LDA), 0, tk);
       tma_load_2d(sKH, &tmKh, KB(K_LDA), 0, tk);
       tma_load_2d(sV, &tmV, KB(K_LDA), 0, tk);
+      tma_load_2d(sKT, &tmKt, KB(K_LDA), 0, (bc * NV + kb * (kb + 1) / 2 + kb) * 128);
       tma_load_2d(sW, &tmW, KB(K_LDA), 0, bc * VD);
       tma_load_2d(sL, &tmLam, KB(K_LDA), 0, bc * VD);
-      for (int qi = 0; qi < NQ; ++qi) {
-        const int qb = kb + qi, bar = qi == 0 ? K_LDQ0 : K_LDQ1;
-        mbar_arrive_expect_tx(KB(bar), 3 * PANEL);
-        tma_load_2d(sKT(qi), &tmKt, KB(bar), 0, (bc * NV + qb * (qb + 1) / 2 + kb) * 128);
-        tma_load_2d(sQT(qi), &tmQt, KB(bar), 0, tokc + 128 * qb);
-        tma_load_2d(sDO(qi), &tmdO, KB(bar), 0, tokc + 128 * qb);
+      for (int h = 0; h < NH; ++h) {
+        const int qb = kb + (h >> 1), half = h & 1, bar = (h & 1) ? K_LDH1 : K_LDH0;
+        // the slot is free once the half two before it has been multiplied (or, for the K
+        // panel's first use, once G = K W0 has read K)
+        if (h >= 2 && !mbar_wait(KB((h & 1) ? K_ST1 : K_ST0), ((h - 2) >> 1) & 1, ab)) break;
+        if (h == 1 && LOSS == 0 && !mbar_wait(KB(K_GA), 0, ab)) break;
+        mbar_arrive_expect_tx(KB(bar), 2 * L::HALF);
+        if (qb == kb)
+          tma_load_2d(sQh(h), &tmQh, KB(bar), 0, tokc + 128 * qb + 64 * half);
+        else
+          tma_load_2d(sQh(h), &tmQ2h, KB(bar), 0, bc * 128 + 64 * half);
+        tma_load_2d(sDOh(h), &tmdOh, KB(bar), 0, tokc + 128 * qb + 64 * half);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idKM = idesc_bf16(128, VD, 0, 1);   // K-major A, MN-major B, N = 64
-      const uint32_t idPP = idesc_bf16(128, 128, 0, 0);  // both K-major, N = 128
-      const uint32_t idKK = idesc_bf16(128, VD, 0, 0);   // both K-major, N = 64
+      const uint32_t idKM = idesc_bf16(128, VD, 0, 1);  // K-major A, MN-major B, N = 64
+      const uint32_t idKK = idesc_bf16(128, VD, 0, 0);  // both K-major, N = 64
       do {
         if (!mbar_wait(KB(K_LDA), 0, ab)) break;
         tc_fence_after();
         if constexpr (LOSS == 0) {
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
-            mma_bf16_ss(tmem + L::T_G, sdesc_sw128(sK + jj * 32, 16, 1024),
+            mma_bf16_ss(tmem + L::T_DKS, sdesc_sw128(sK + jj * 32, 16, 1024),
                         sdesc_sw128(sW + jj * 2048, 0, 1024), idKM, jj > 0);
         }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj)
-          mma_bf16_ss(tmem + L::T_X, sdesc_sw128(sKH + jj * 32, 16, 1024),
+          mma_bf16_ss(tmem + L::T_DG, sdesc_sw128(sKH + jj * 32, 16, 1024),
                       sdesc_sw128(sL + jj * 2048, 0, 1024), idKM, jj > 0);
         mma_commit(KB(K_GA));
+        if (!mbar_wait(KB(K_GRDY), 0, ab)) break;
         bool ok = true;
-        for (int qi = 0; qi < NQ && ok; ++qi) {
-          if (!(ok = mbar_wait(KB(qi == 0 ? K_LDQ0 : K_LDQ1), 0, ab))) break;
-          // P^T and G dO^T of the previous query block have been read out and S^T packed
-          if (qi > 0 && !(ok = mbar_wait(KB(K_PK0), 0, ab))) break;
-          if (qi == 0 && !(ok = mbar_wait(KB(K_GRDY), 0, ab))) break;
+        for (int h = 0; h < NH && ok; ++h) {
+          if (!(ok = mbar_wait(KB((h & 1) ? K_LDH1 : K_LDH0), (h >> 1) & 1, ab))) break;
+          // the previous half's products, which read the packed columns, are complete
+          if (h > 0 && !(ok = mbar_wait(KB(((h - 1) & 1) ? K_ST1 : K_ST0), ((h - 1) >> 1) & 1, ab)))
+            break;
           tc_fence_after();
+          const uint32_t sQ = sQh(h), sD = sDOh(h);
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
-            mma_bf16_ss(tmem + L::T_P, sdesc_sw128(sKT(qi) + jj * 32, 16, 1024),
-                        sdesc_sw128(sQT(qi) + jj * 32, 16, 1024), idPP, jj > 0);
+            mma_bf16_ss(tmem + L::T_P, sdesc_sw128(sKT + jj * 32, 16, 1024),
+                        sdesc_sw128(sQ + jj * 32, 16, 1024), idKK, jj > 0);
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
             mma_bf16_ss(tmem + L::T_DS, sdesc_sw128(sV + jj * 32, 16, 1024),
-                        sdesc_sw128(sDO(qi) + jj * 32, 16, 1024), idPP, jj > 0);
-          mma_commit(KB(qi == 0 ? K_PS0 : K_PS1));
-          if (!(ok = mbar_wait(KB(qi == 0 ? K_PK0 : K_PK1), 0, ab))) break;
+                        sdesc_sw128(sD + jj * 32, 16, 1024), idKK, jj > 0);
+          mma_commit(KB(K_PS));
+          if (!(ok = mbar_wait(KB(K_PK), h & 1, ab))) break;
           tc_fence_after();
-          // dG accumulator += S^T dO (A: the packed S^T in TMEM, K = 128 queries)
+          // dG accumulator += S^T dO and dK^S accumulator += (eta dS^T) qtilde' (A packed in
+          // TMEM, K = the half's 64 queries)
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj)
-            mma_bf16_ts(tmem + L::T_DG, tmem + L::T_S + 8 * jj, sdesc_sw128(sDO(qi) + jj * 2048, 0, 1024),
+          for (int jj = 0; jj < 4; ++jj)
+            mma_bf16_ts(tmem + L::T_DG, tmem + L::T_P + 8 * jj, sdesc_sw128(sD + jj * 2048, 0, 1024),
                         idKM, 1);
-          // (eta dS^T) qtilde: A = eta dS^T packed in TMEM (K = 128 queries)
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj)
-            mma_bf16_ts(tmem + (qi == 0 ? L::T_G : L::T_X), tmem + L::T_DS + 8 * jj,
-                        sdesc_sw128(sQT(qi) + jj * 2048, 0, 1024), idKM, jj > 0);
-          mma_commit(KB(qi == 0 ? K_DK0 : K_DK1));
-          // the next block's G dO^T overwrites the packed operand just read
-          if (qi + 1 < NQ && !(ok = mbar_wait(KB(K_DK0), 0, ab))) break;
+          for (int jj = 0; jj < 4; ++jj)
+            mma_bf16_ts(tmem + L::T_DKS, tmem + L::T_DS + 8 * jj,
+                        sdesc_sw128(sQ + jj * 2048, 0, 1024), idKM, h > 0 || jj > 0);
+          mma_commit(KB((h & 1) ? K_ST1 : K_ST0));
         }
         if (!ok) break;
-        // G Lambda^T over the score columns (read out by now)
+        if (!mbar_wait(KB(((NH - 1) & 1) ? K_ST1 : K_ST0), ((NH - 1) >> 1) & 1, ab)) break;
+        tc_fence_after();
+        // G Lambda^T over the score columns (all read out by now)
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj)
           mma_bf16_ss(tmem + L::T_P, sdesc_sw128(sV + jj * 32, 16, 1024),
@@ -1162,7 +1193,7 @@ __global__ void __launch_bounds__(kVoThreads, 1)
           tc_fence_after();
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
-            mma_bf16_ss(tmem + L::T_P + 64, sdesc_sw128(sKH + jj * 32, 16, 1024),
+            mma_bf16_ss(tmem + L::T_DS, sdesc_sw128(sKH + jj * 32, 16, 1024),
                         sdesc_sw128(sW + jj * 32, 16, 1024), idKK, jj > 0);
           mma_commit(KB(K_DGW));
         }
@@ -1177,12 +1208,11 @@ __global__ void __launch_bounds__(kVoThreads, 1)
     const float sg = sigm(__ldg(p.beta + tr) + p.lr_bias), eta = 2.f * sg;
     float deta = 0.f;
     do {
-      // L at each query block's reference token and at the chunk's last token
+      // L at the key block's reference token and at the chunk's last token
       {
         const int t = threadIdx.x - 64;
         if (t < VD) {
-          for (int qb = kb; qb < NB; ++qb)
-            f_Lm[qb * VD + t] = __ldg(p.Lf + ((size_t)tokc + 128 * qb + 63) * VD + t);
+          f_Lm[t] = __ldg(p.Lf + ((size_t)tokc + 128 * kb + 63) * VD + t);
           f_LC[t] = __ldg(p.Lf + ((size_t)tokc + C - 1) * VD + t);
         }
         __syncwarp();
@@ -1198,7 +1228,7 @@ __global__ void __launch_bounds__(kVoThreads, 1)
         ld_row32(sV, lrow, 4 * h, gv);
         if constexpr (LOSS == 0) {
           float z[32];
-          tmem_ld32(tmem + loff + L::T_G + 32 * h, z);
+          tmem_ld32(tmem + loff + L::T_DKS + 32 * h, z);
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) gv[k] = z[k] - gv[k];
@@ -1206,7 +1236,7 @@ __global__ void __launch_bounds__(kVoThreads, 1)
 #pragma unroll
           for (int k = 0; k < 32; ++k) gv[k] = -gv[k];
         }
-        tmem_ld32(tmem + loff + L::T_X + 32 * h, xv);
+        tmem_ld32(tmem + loff + L::T_DG + 32 * h, xv);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
@@ -1221,34 +1251,34 @@ __global__ void __launch_bounds__(kVoThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(KB(K_GRDY));
-      // -------- per query block: S^T = eta P^T and eta dS^T (s >= r), deta's dS . P term
+      // -------- per query half: S^T = eta P^T and eta dS^T (s >= r), packed in place
       bool ok = true;
-      for (int qi = 0; qi < NQ; ++qi) {
-        const bool diag = qi == 0;  // qb == kb
-        if (!mbar_wait(KB(qi == 0 ? K_PS0 : K_PS1), 0, ab) ||
-            (qi > 0 && !mbar_wait(KB(K_DK0), 0, ab))) {
+      for (int h = 0; h < NH; ++h) {
+        const bool diag = (h >> 1) == 0;  // qb == kb
+        if (!mbar_wait(KB(K_PS), h & 1, ab)) {
           ok = false;
           break;
         }
         __syncwarp();
         tc_fence_after();
-        // packing in place: group idx is read (columns [32 idx, 32 idx + 32)) before its packed
-        // form is written to columns [16 idx, 16 idx + 16), which earlier groups have vacated
+        // group g (32 queries) of the half is group G = 2 (h & 1) + g of the 128-query block;
+        // it is read (columns [32 g, 32 g + 32)) before its packed form goes to [16 g, 16 g + 16)
 #pragma unroll 1
-        for (int idx = 0; idx < 4; ++idx) {
+        for (int g = 0; g < 2; ++g) {
+          const int G = 2 * (h & 1) + g;
           uint32_t pk[16], pa[16];
-          if (diag && idx < q) {
-            // every query of this column group precedes every key of the warp: masked
+          if (diag && G < q) {
+            // every query of the group precedes every key of the warp: masked
 #pragma unroll
             for (int k = 0; k < 16; ++k) pk[k] = pa[k] = 0u;
           } else {
             float pv[32], dv[32];
-            tmem_ld32(tmem + loff + L::T_P + 32 * idx, pv);
-            tmem_ld32(tmem + loff + L::T_DS + 32 * idx, dv);
+            tmem_ld32(tmem + loff + L::T_P + 32 * g, pv);
+            tmem_ld32(tmem + loff + L::T_DS + 32 * g, dv);
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 32; ++k) {
-              const bool keep = !diag || idx > q || 32 * idx + k >= lrow;
+              const bool keep = !diag || G > q || 32 * G + k >= lrow;
               const float ds = keep ? -dv[k] : 0.f;
               const float pp = keep ? pv[k] : 0.f;
               deta += ds * pp;
@@ -1261,17 +1291,17 @@ __global__ void __launch_bounds__(kVoThreads, 1)
               pa[k] = pack_bf16x2(dv[2 * k], dv[2 * k + 1]);
             }
           }
-          tmem_st16u(tmem + loff + L::T_S + 16 * idx, pk);
-          tmem_st16u(tmem + loff + L::T_DS + 16 * idx, pa);
+          tmem_st16u(tmem + loff + L::T_P + 16 * g, pk);
+          tmem_st16u(tmem + loff + L::T_DS + 16 * g, pa);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(KB(qi == 0 ? K_PK0 : K_PK1));
+        if (lane == 0) mbar_arrive(KB(K_PK));
       }
       if (!ok) break;
       // -------- dG, dV; dG (bf16) for dG W0^T
-      if (!mbar_wait(KB(NQ == 1 ? K_DK0 : K_DK1), 0, ab)) break;
+      if (!mbar_wait(KB(((NH - 1) & 1) ? K_ST1 : K_ST0), ((NH - 1) >> 1) & 1, ab)) break;
       __syncwarp();
       tc_fence_after();
 #pragma unroll 1
@@ -1300,10 +1330,10 @@ __global__ void __launch_bounds__(kVoThreads, 1)
       tc_fence_after();
       bool range = false;
       const float* Lr = p.Lf + tr * VD;
+      const __nv_bfloat16* kr = p.K + tr * VD;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        float dk[32], kv[32], Lv[32], t32[32];
-        ld_row32(sK, lrow, 4 * h, kv);
+        float dk[32], t32[32], Lv[32];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const float4 v = __ldg(reinterpret_cast<const float4*>(Lr + 32 * h) + k);
@@ -1315,27 +1345,27 @@ __global__ void __launch_bounds__(kVoThreads, 1)
 #pragma unroll
         for (int k = 0; k < 32; ++k) dk[k] = -eta * __expf(LC[k] - Lv[k]) * t32[k];
         if (p.colk) {
+          ldg_bf16x32(kr + 32 * h, t32);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) t32[k] = kv[k] * dk[k];
+          for (int k = 0; k < 32; ++k) t32[k] *= dk[k];
           colsum32(t32, lane);
           p.colk[(((size_t)bc * NB + kb) * 4 + q) * VD + 32 * h + lane] = t32[0];
         }
-        for (int qi = 0; qi < NQ; ++qi) {
-          const float* Lm = f_Lm + (kb + qi) * VD + 32 * h;
-          tmem_ld32(tmem + loff + (qi == 0 ? L::T_G : L::T_X) + 32 * h, t32);
-          tmem_wait_ld();
+        tmem_ld32(tmem + loff + L::T_DKS + 32 * h, t32);
+        tmem_wait_ld();
+        const float* Lm = f_Lm + 32 * h;
 #pragma unroll
-          for (int k = 0; k < 32; ++k) dk[k] += clamped_exp(Lm[k] - Lv[k], range) * t32[k];
-        }
+        for (int k = 0; k < 32; ++k) dk[k] += clamped_exp(Lm[k] - Lv[k], range) * t32[k];
         if (p.dLk) {
+          ldg_bf16x32(kr + 32 * h, t32);
           float4* dst = reinterpret_cast<float4*>(p.dLk + tr * VD + 32 * h);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(-kv[4 * k] * dk[4 * k], -kv[4 * k + 1] * dk[4 * k + 1],
-                                 -kv[4 * k + 2] * dk[4 * k + 2], -kv[4 * k + 3] * dk[4 * k + 3]);
+            dst[k] = make_float4(-t32[4 * k] * dk[4 * k], -t32[4 * k + 1] * dk[4 * k + 1],
+                                 -t32[4 * k + 2] * dk[4 * k + 2], -t32[4 * k + 3] * dk[4 * k + 3]);
         }
         if constexpr (LOSS == 0) {
-          tmem_ld32(tmem + loff + L::T_P + 64 + 32 * h, t32);  // dG W0^T
+          tmem_ld32(tmem + loff + L::T_DS + 32 * h, t32);  // dG W0^T
           tmem_wait_ld();
 #pragma unroll
           for (int k = 0; k < 32; ++k) dk[k] += t32[k];
@@ -1352,7 +1382,7 @@ __global__ void __launch_bounds__(kVoThreads, 1)
   if (bars->abort_flag) __nanosleep(100000);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -1675,6 +1705,7 @@ cudaError_t launch_prep(const LayerArgs& a, const VecPrep& o, cudaStream_t s) {
   p.GC = o.GC;
   p.Em = o.Em;
   p.Lf = o.Lf;
+  p.Qt2 = static_cast<__nv_bfloat16*>(o.Qt2);
   p.err = a.err;
   vec_prep_kernel<NB><<<a.B * a.H * p.NC * 2, kPrepThreads, 0, s>>>(p);
   count_launches(1);
@@ -1775,7 +1806,7 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
   float* dLq = reinterpret_cast<float*>(take(rows * VD * 4));
   float* dLk = reinterpret_cast<float*>(take(rows * VD * 4));
   const bool dg = a.dgamma != nullptr;
-  CUtensorMap tK, tKh, tV, tR, tdO, tQt, tKt, tW, tLam;
+  CUtensorMap tK, tKh, tV, tR, tdO, tQt, tKt, tW, tLam, tQh, tQ2h, tdOh;
   if (!make_tmap_bf16(&tK, a.K, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tKh, pr.Kh, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tV, a.V, VD, rows, VD, 64, 128) ||
@@ -1784,8 +1815,12 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
       !make_tmap_bf16(&tQt, pr.Qt, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tKt, pr.Kt, VD, (uint64_t)BH * NC * NV * 128, VD, 64, 128) ||
       !make_tmap_bf16(&tW, a.W_chunks, VD, (uint64_t)BH * NC * VD, VD, 64, VD) ||
-      !make_tmap_bf16(&tLam, Lam, VD, (uint64_t)BH * NC * VD, VD, 64, VD))
+      !make_tmap_bf16(&tLam, Lam, VD, (uint64_t)BH * NC * VD, VD, 64, VD) ||
+      !make_tmap_bf16(&tQh, pr.Qt, VD, rows, VD, 64, 64) ||
+      !make_tmap_bf16(&tdOh, a.dO, VD, rows, VD, 64, 64) ||
+      (NB == 2 && !make_tmap_bf16(&tQ2h, pr.Qt2, VD, (uint64_t)BH * NC * 128, VD, 64, 64)))
     return cudaErrorInvalidValue;
+  if (NB == 1) tQ2h = tQh;  // never used
   VecParams vp{};
   vp.BH = BH;
   vp.T = a.T;
@@ -1814,6 +1849,7 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
   gp.Lf = pr.Lf;
   gp.Em = pr.Em;
   gp.Q = static_cast<const __nv_bfloat16*>(a.Q);
+  gp.K = static_cast<const __nv_bfloat16*>(a.K);
   gp.dQ = static_cast<__nv_bfloat16*>(a.dQ);
   gp.dK = static_cast<__nv_bfloat16*>(a.dK);
   gp.dV = static_cast<__nv_bfloat16*>(a.dV);
@@ -1821,7 +1857,7 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
   gp.dLk = dg ? dLk : nullptr;
   gp.dLq = dg ? dLq : nullptr;
   gp.colk = dg ? colk : nullptr;
-  const size_t sm_r = vo_bytes() + 1024, sm_b = vb_bytes<NB>() + 1024, sm_k = kg_bytes<NB>() + 1024,
+  const size_t sm_r = vo_bytes() + 1024, sm_b = vb_bytes<NB>() + 1024, sm_k = kg_bytes() + 1024,
                sm_q = qg_bytes() + 1024;
   auto kr = fwd_vout_kernel<NB, LOSS, 1>;
   auto kb = bwd_vstate_kernel<NB, LOSS>;
@@ -1839,7 +1875,8 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
     count_launches(1);
   }
   kb<<<BH, kVsThreads, sm_b, s>>>(tK, tKh, tR, tdO, bp, a.err);
-  kk<<<BH * NC * NB, kVoThreads, sm_k, s>>>(tK, tKh, tV, tKt, tQt, tdO, tW, tLam, gp, a.err);
+  kk<<<BH * NC * NB, kVoThreads, sm_k, s>>>(tK, tKh, tV, tKt, tQh, tQ2h, tdOh, tW, tLam, gp,
+                                            a.err);
   kq<<<BH * NC * NB, kVoThreads, sm_q, s>>>(tK, tV, tKt, tdO, tW, gp, a.err);
   count_launches(3);
   if (dg) {
@@ -1867,7 +1904,7 @@ size_t vec_prep_bytes(const LayerArgs& a, bool with_L) {
              + align_up(BH * NC * NV * 128 * VD * 2)    // Kt
              + align_up(BH * NC * VD * 4)               // GC
              + align_up(BH * NC * NB * VD * 4);         // Em
-  if (with_L) n += align_up(rows * VD * 4);
+  if (with_L) n += align_up(rows * VD * 4) + (NB == 2 ? align_up(BH * NC * 128 * VD * 2) : 0);
   return n;
 }
 
@@ -1887,6 +1924,7 @@ VecPrep vec_prep_carve(const LayerArgs& a, void* base, bool with_L) {
   o.Em = reinterpret_cast<float*>(b);
   b += align_up(BH * NC * NB * VD * 4);
   o.Lf = with_L ? reinterpret_cast<float*>(b) : nullptr;
+  if (with_L && NB == 2) o.Qt2 = b + align_up(rows * VD * 4);
   return o;
 }
 
