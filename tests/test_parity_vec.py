@@ -100,6 +100,10 @@ def test_vector_decay_backward_small(B, H, T, C, loss):
     g2 = run_bwd(cfg, inp, got["W_chunks"])
     for k in GRADS[:-1]:
         assert rel_err(g2[k], g[k]) <= 1e-6, k
+    # given the forward's saved buffer (G, the decayed operands, R) instead of forming them
+    g3 = run_bwd(cfg, inp, got["W_chunks"], got["G_saved"], fwd=got)
+    for k in GRADS:
+        assert rel_err(g3[k], r[k]) <= TOL, ("saved", k, rel_err(g3[k], r[k]))
 
 
 def test_vector_decay_backward_without_final_state_gradient():
@@ -119,7 +123,7 @@ def test_vector_decay_backward_full_size_sampled_heads(loss):
     inp = synth.ttt_inputs(cfg, device="cuda", seed=47)
     inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(48))
     got = run_fwd(cfg, inp)
-    g = run_bwd(cfg, inp, got["W_chunks"], fwd=got)
+    g = run_bwd(cfg, inp, got["W_chunks"], got["G_saved"], fwd=got)
     rng = np.random.default_rng(49)
     heads = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(2)]
     sub = head_slice(inp, heads)

@@ -1060,7 +1060,8 @@ __device__ __forceinline__ void ldg_bf16x32(const __nv_bfloat16* src, float (&v)
   }
 }
 
-template <int NB, int LOSS>
+// SG: the tmV operand is the forward's saved G (bf16), so G is neither recomputed nor negated.
+template <int NB, int LOSS, bool SG>
 __global__ void __launch_bounds__(kVoThreads, 2)
     bwd_vkey_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKh,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKt,
@@ -1108,8 +1109,9 @@ __global__ void __launch_bounds__(kVoThreads, 2)
   if (warp == 0) {
     if (lane == 0) {
       const int tk = tokc + 128 * kb;
-      mbar_arrive_expect_tx(KB(K_LDA), (LOSS == 0 ? 4 : 3) * PANEL + 2 * VD * 128);
-      if (LOSS == 0) tma_load_2d(sK, &tmK, KB(K_LDA), 0, tk);
+      constexpr bool kmma = LOSS == 0 && !SG;  // G = K W0 - V by MMA
+      mbar_arrive_expect_tx(KB(K_LDA), (kmma ? 4 : 3) * PANEL + 2 * VD * 128);
+      if (kmma) tma_load_2d(sK, &tmK, KB(K_LDA), 0, tk);
       tma_load_2d(sKH, &tmKh, KB(K_LDA), 0, tk);
       tma_load_2d(sV, &tmV, KB(K_LDA), 0, tk);
       tma_load_2d(sKT, &tmKt, KB(K_LDA), 0, (bc * NV + kb * (kb + 1) / 2 + kb) * 128);
@@ -1120,7 +1122,7 @@ __global__ void __launch_bounds__(kVoThreads, 2)
         // the slot is free once the half two before it has been multiplied (or, for the K
         // panel's first use, once G = K W0 has read K)
         if (h >= 2 && !mbar_wait(KB((h & 1) ? K_ST1 : K_ST0), ((h - 2) >> 1) & 1, ab)) break;
-        if (h == 1 && LOSS == 0 && !mbar_wait(KB(K_GA), 0, ab)) break;
+        if (h == 1 && kmma && !mbar_wait(KB(K_GA), 0, ab)) break;
         mbar_arrive_expect_tx(KB(bar), 2 * L::HALF);
         if (qb == kb)
           tma_load_2d(sQh(h), &tmQh, KB(bar), 0, tokc + 128 * qb + 64 * half);
@@ -1136,7 +1138,7 @@ __global__ void __launch_bounds__(kVoThreads, 2)
       do {
         if (!mbar_wait(KB(K_LDA), 0, ab)) break;
         tc_fence_after();
-        if constexpr (LOSS == 0) {
+        if constexpr (LOSS == 0 && !SG) {
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj)
             mma_bf16_ss(tmem + L::T_DKS, sdesc_sw128(sK + jj * 32, 16, 1024),
@@ -1226,7 +1228,9 @@ __global__ void __launch_bounds__(kVoThreads, 2)
       for (int h = 0; h < 2; ++h) {
         float gv[32], xv[32];
         ld_row32(sV, lrow, 4 * h, gv);
-        if constexpr (LOSS == 0) {
+        if constexpr (SG) {
+          // G as saved
+        } else if constexpr (LOSS == 0) {
           float z[32];
           tmem_ld32(tmem + loff + L::T_DKS + 32 * h, z);
           tmem_wait_ld();
@@ -1243,7 +1247,7 @@ __global__ void __launch_bounds__(kVoThreads, 2)
           deta -= xv[k] * gv[k];
           xv[k] *= eta;
         }
-        st_row32(sV, lrow, 4 * h, gv);
+        if (!SG) st_row32(sV, lrow, 4 * h, gv);
         tmem_st32(tmem + loff + L::T_DG + 32 * h, xv);
       }
       tmem_wait_st();
@@ -1406,7 +1410,8 @@ struct __align__(8) QgBars {
 };
 constexpr uint32_t qg_bytes() { return QgL::OFF_BAR + sizeof(QgBars); }
 
-template <int NB, int LOSS>
+// SG: the tmV operand is the forward's saved G (bf16), so G is neither recomputed nor negated.
+template <int NB, int LOSS, bool SG>
 __global__ void __launch_bounds__(kVoThreads, 2)
     bwd_vquery_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmKt, const __grid_constant__ CUtensorMap tmdO,
@@ -1450,15 +1455,16 @@ __global__ void __launch_bounds__(kVoThreads, 2)
   if (warp == 0) {
     if (lane == 0) {
       const int nk = qb + 1;
-      mbar_arrive_expect_tx(QB(Q_LDA), (LOSS == 0 ? 2 : 1) * nk * PANEL + PANEL + VD * 128);
+      constexpr bool kmma = LOSS == 0 && !SG;  // G = K W0 - V by MMA
+      mbar_arrive_expect_tx(QB(Q_LDA), (kmma ? 2 : 1) * nk * PANEL + PANEL + VD * 128);
       for (int kb = 0; kb < nk; ++kb) {
-        if (LOSS == 0) tma_load_2d(sKb(kb), &tmK, QB(Q_LDA), 0, tokc + 128 * kb);
+        if (kmma) tma_load_2d(sKb(kb), &tmK, QB(Q_LDA), 0, tokc + 128 * kb);
         tma_load_2d(sVb(kb), &tmV, QB(Q_LDA), 0, tokc + 128 * kb);
       }
       tma_load_2d(sDO, &tmdO, QB(Q_LDA), 0, tokc + 128 * qb);
       tma_load_2d(sW, &tmW, QB(Q_LDA), 0, bc * VD);
       // ktilde over the K slots once K W0 is done
-      if (LOSS == 1 || mbar_wait(QB(Q_GF), 0, ab)) {
+      if (!kmma || mbar_wait(QB(Q_GF), 0, ab)) {
         mbar_arrive_expect_tx(QB(Q_KT), nk * PANEL);
         for (int kb = 0; kb < nk; ++kb)
           tma_load_2d(sKb(kb), &tmKt, QB(Q_KT), 0, (bc * NV + qb * (qb + 1) / 2 + kb) * 128);
@@ -1472,7 +1478,7 @@ __global__ void __launch_bounds__(kVoThreads, 2)
       do {
         if (!mbar_wait(QB(Q_LDA), 0, ab)) break;
         tc_fence_after();
-        if constexpr (LOSS == 0) {
+        if constexpr (LOSS == 0 && !SG) {
           for (int kb = 0; kb <= qb; ++kb) {
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj)
@@ -1528,12 +1534,12 @@ __global__ void __launch_bounds__(kVoThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(QB(Q_F));
       if (!mbar_wait(QB(Q_F), 0, ab) || !mbar_wait(QB(Q_LDA), 0, ab) ||
-          (LOSS == 0 && !mbar_wait(QB(Q_GF), 0, ab)))
+          (LOSS == 0 && !SG && !mbar_wait(QB(Q_GF), 0, ab)))
         break;
       __syncwarp();
       tc_fence_after();
-      // G_kb (bf16, over V_kb) for every key block up to this one
-      for (int kb = 0; kb <= qb; ++kb) {
+      // G_kb (bf16, over V_kb) for every key block up to this one (as saved: nothing to do)
+      for (int kb = 0; kb <= qb && !SG; ++kb) {
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           float gv[32];
@@ -1806,10 +1812,11 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
   float* dLq = reinterpret_cast<float*>(take(rows * VD * 4));
   float* dLk = reinterpret_cast<float*>(take(rows * VD * 4));
   const bool dg = a.dgamma != nullptr;
+  // (with the saved buffer, the gradient kernels take its G through tV instead of V)
   CUtensorMap tK, tKh, tV, tR, tdO, tQt, tKt, tW, tLam, tQh, tQ2h, tdOh;
   if (!make_tmap_bf16(&tK, a.K, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tKh, pr.Kh, VD, rows, VD, 64, 128) ||
-      !make_tmap_bf16(&tV, a.V, VD, rows, VD, 64, 128) ||
+      !make_tmap_bf16(&tV, saved ? a.G_saved : a.V, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tR, R, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tdO, a.dO, VD, rows, VD, 64, 128) ||
       !make_tmap_bf16(&tQt, pr.Qt, VD, rows, VD, 64, 128) ||
@@ -1861,8 +1868,9 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
                sm_q = qg_bytes() + 1024;
   auto kr = fwd_vout_kernel<NB, LOSS, 1>;
   auto kb = bwd_vstate_kernel<NB, LOSS>;
-  auto kk = bwd_vkey_kernel<NB, LOSS>;
-  auto kq = bwd_vquery_kernel<NB, LOSS>;
+  const bool sg = saved;
+  auto kk = sg ? bwd_vkey_kernel<NB, LOSS, true> : bwd_vkey_kernel<NB, LOSS, false>;
+  auto kq = sg ? bwd_vquery_kernel<NB, LOSS, true> : bwd_vquery_kernel<NB, LOSS, false>;
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(kr, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_r)) ||
       (e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_b)) ||
