@@ -119,7 +119,9 @@ def test_mlp_single_chunk_fp32():
 
 
 TC_CASES = [(256, 128, 128, loss, act, decay) for loss, act in COMBOS for decay in (False, True)]
-TC_CASES += [(512, 256, 256, "mse", "silu", True), (512, 256, 256, "ip", "id", False)]
+TC_CASES += [(512, 256, 256, "mse", "silu", True), (512, 256, 256, "ip", "id", False),
+             (512, 128, 256, "mse", "silu", True), (512, 256, 128, "ip", "silu", True),
+             (256, 256, 256, "mse", "id", True)]  # (one chunk)
 
 
 @pytest.mark.parametrize("T,C,hidden,loss,act,decay", TC_CASES)

@@ -133,3 +133,23 @@ def test_vector_decay_backward_full_size_sampled_heads(loss):
         err = rel_err(got_k, r[k])
         print(f"{loss} {k}: rel err {err:.2e} (bound {TOL:.0e}, margin {TOL / max(err, 1e-30):.1f}x)")
         assert err <= TOL, (k, err)
+
+
+@pytest.mark.parametrize("loss", ["mse", "ip"])
+def test_vector_decay_of_ones_equals_no_decay(loss):
+    # gamma = 1 on every feature: the per-feature path (scaled operands, its own kernels) must
+    # give what the scalar-decay kernels give without a decay
+    cfg = _cfg(B=1, H=2, T=512, C=256, loss=loss)
+    inp = synth.ttt_inputs(cfg, device="cuda", seed=14)
+    inp["gamma"] = torch.ones_like(inp["gamma"])
+    inp["dW_T"].normal_(generator=torch.Generator("cuda").manual_seed(15))
+    vec = run_fwd(cfg, inp)
+    gv = run_bwd(cfg, inp, vec["W_chunks"], vec["G_saved"], fwd=vec)
+    sc_cfg = cfg.replace(decay=False)
+    sc_inp = dict(inp, gamma=None)
+    sc = run_fwd(sc_cfg, sc_inp)
+    gs = run_bwd(sc_cfg, sc_inp, sc["W_chunks"], sc["G_saved"])
+    assert rel_err(vec["O"], sc["O"]) <= 1e-2
+    assert rel_err(vec["W_final"], sc["W_final"]) <= 1e-2
+    for k in GRADS[:-1]:
+        assert rel_err(gv[k], gs[k]) <= 1e-2, (k, rel_err(gv[k], gs[k]))
