@@ -20,7 +20,9 @@
 //   update tiles [128 d_model x 256 d_ff]: M += s X_i^T (MN-major) x Z_i (MN-major), K = C,
 //                with (M, X, s) = (W, Vhat, eta) forward and (Wh, dO, 1) backward; the epilogue
 //                keeps M in float32 and writes the scaled bf16 copy the next launch reads.
-// Long tiles (row, then dz) are handed out first, update tiles fill the remaining SMs.
+// Long tiles (row, then dz) are handed out first, update tiles fill the remaining SMs. When
+// the producer takes an update tile it prefetches the tile's float32 block of M into L2, so
+// the epilogue's read-modify-write, issued after the tile's K steps, reads from L2.
 // Warp roles: warp 0 issues TMA loads into a 4-stage ring, warp 1 issues tcgen05.mma into
 // two TMEM accumulators of 128 x 256 fp32, warps 2-9 drain the accumulators (two warps per
 // TMEM lane quadrant, each taking 128 of the 256 columns).
@@ -59,6 +61,16 @@ struct Params {
 };
 
 enum Kind { KIND_ROW = 0, KIND_DZ = 1, KIND_UPD = 2 };
+
+constexpr int MBOX = 64;  // float32 columns of M per L2 prefetch box (box: 128 rows x 64)
+
+// Prefetch of one box of a 2-D tensor map into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
 
 struct Tile {
   int kind, m0, n0, nkb;
@@ -104,6 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                          const __grid_constant__ CUtensorMap tm_vk,    // Vhat, K-major
                          const __grid_constant__ CUtensorMap tm_wc,    // saved W_i, MN-major
                          const __grid_constant__ CUtensorMap tm_mbn,   // bf16 copy, MN-major
+                         const __grid_constant__ CUtensorMap tm_mf,    // float32 M (prefetch)
                          const Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -133,6 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_zb);
     tma_prefetch_desc(&tm_mb);
     tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_mf);
     if (p.n_dz) {
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_vk);
@@ -162,6 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (++r == RING) { r = 0; rph ^= 1; }
         if (t >= p.n_total) break;
         const Tile x = decode(p, t);
+        if (x.kind == KIND_UPD)
+          for (int j = 0; j < BN / MBOX; ++j) tma_prefetch_l2_2d(&tm_mf, x.n0 + MBOX * j, x.m0);
         bool ok = true;
         for (int kb = 0; kb < x.nkb && ok; ++kb) {
           if (!mbar_wait(smem_u32(&bars->empty[s]), sph ^ 1, ab)) { ok = false; break; }
@@ -287,22 +303,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j) xt[lane * 33 + j] = v[j];
           __syncwarp();
           const size_t ld = p.d_ff;
-#pragma unroll 1
-          for (int h = 0; h < 2; ++h) {
-            // rows mbase + 16 h .. + 15: sixteen coalesced loads in flight, then the stores
-            const int m0 = mbase + 16 * h;
-            float* mp = p.M + (size_t)m0 * ld + col;
-            float w[16];
+          // rows mbase .. mbase + 31 (d_model is a multiple of 128: all inside M): all 32
+          // coalesced loads in flight, then the stores, walking one row pointer each
+          float* mp = p.M + (size_t)mbase * ld + col;
+          float w[32];
+          {
+            const float* lp = mp;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) w[r] = m0 + r < p.d_model ? mp[r * ld] : 0.f;
+            for (int r = 0; r < 32; ++r, lp += ld) w[r] = *lp;
+          }
+          __nv_bfloat16* bp =
+              p.wb_next_row0 >= 0 ? p.Mb + (size_t)(p.wb_next_row0 + mbase) * ld + col : nullptr;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-              if (m0 + r < p.d_model) {
-                const float o = w[r] + s * xt[(16 * h + r) * 33 + lane];
-                mp[r * ld] = o;
-                if (p.wb_next_row0 >= 0)
-                  p.Mb[(size_t)(p.wb_next_row0 + m0 + r) * ld + col] = __float2bfloat16_rn(cs * o);
-              }
+          for (int r = 0; r < 32; ++r, mp += ld) {
+            const float o = w[r] + s * xt[r * 33 + lane];
+            *mp = o;
+            if (bp) {
+              *bp = __float2bfloat16_rn(cs * o);
+              bp += ld;
             }
           }
           __syncwarp();  // the tile is rewritten by the next step
@@ -650,11 +668,12 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   // with document resets: the initial W, kept after the counters
   float* W0 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) +
                                        inplace_workspace(T, d_ff, d_model, C, false));
-  CUtensorMap tza, tzb, twb, tvh;
+  CUtensorMap tza, tzb, twb, tvh, tmf;
   if (!make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
       !make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
       !make_tmap_bf16(&twb, Wb, d_ff, wb_rows, d_ff, BK, BN) ||
-      !make_tmap_bf16(&tvh, Vhat, d_model, T, d_model, 64, BK))
+      !make_tmap_bf16(&tvh, Vhat, d_model, T, d_model, 64, BK) ||
+      !make_tmap_f32(&tmf, W, d_ff, d_model, d_ff, MBOX, BM))
     return cudaErrorInvalidValue;
   Launch l;
   cudaError_t e = prepare(&l);
@@ -700,7 +719,7 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
       ++launches;
     }
     inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, twb, tvh, tza, tza, tzb, tzb,
-                                                            p);
+                                                            tmf, p);
   }
   count_launches(launches);
   return cudaGetLastError();
@@ -719,8 +738,9 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   // bf16 eta Wh_{i+1}: two rotating copies
   __nv_bfloat16* Mb = static_cast<__nv_bfloat16*>(ws);
   int* counters = reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + 2 * (size_t)d_model * d_ff * 2);
-  CUtensorMap tza, tzb, tmb, tdx, tdo, tvk, twc, tmbn;
-  if (!make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
+  CUtensorMap tza, tzb, tmb, tdx, tdo, tvk, twc, tmbn, tmf;
+  if (!make_tmap_f32(&tmf, R, d_ff, d_model, d_ff, MBOX, BM) ||
+      !make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
       !make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
       !make_tmap_bf16(&tmb, Mb, d_ff, 2 * (size_t)d_model, d_ff, BK, BN) ||
       !make_tmap_bf16(&tdx, dO, d_model, T, d_model, 64, BK) ||
@@ -776,7 +796,7 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
     p.wc_row0 = i * d_model;
     p.counter = counters + i;
     inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, tmb, tdx, tdo, tvk, twc,
-                                                            tmbn, p);
+                                                            tmbn, tmf, p);
     if (reset && (i == 0 || reset[i])) {
       // this document's first chunk applied the initial W: its adjoint joins dW, and the
       // previous document's end state (and its bf16 copy) gets none
@@ -826,7 +846,7 @@ cudaError_t inplace_target_run(int T, int d, int k, const void* X0, const float*
   p.counter = counter;
   p.err = err;
   const int grid = p.n_total < l.sms ? p.n_total : l.sms;
-  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(ty, ty, ty, ty, ty, ty, twt, twt, p);
+  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(ty, ty, ty, ty, ty, ty, twt, twt, ty, p);
   count_launches(2);
   return cudaGetLastError();
 }
@@ -850,8 +870,9 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
   __nv_bfloat16* dY = Y + (size_t)T * d;
   float* part = reinterpret_cast<float*>(dY + (size_t)T * d);
   int* counter = reinterpret_cast<int*>(part + (size_t)nrun * k * d);
-  CUtensorMap tdv_k, tdv_n, twt_k, ty_n;
-  if (!make_tmap_bf16(&tdv_k, dVhat, d, T, d, BK, BM) ||
+  CUtensorMap tdv_k, tdv_n, twt_k, ty_n, tmf;
+  if (!make_tmap_f32(&tmf, dW_target, d, d, d, MBOX, BM) ||
+      !make_tmap_bf16(&tdv_k, dVhat, d, T, d, BK, BM) ||
       !make_tmap_bf16(&tdv_n, dVhat, d, T, d, 64, BK) ||
       !make_tmap_bf16(&twt_k, W_target, d, d, d, BK, BN) ||
       !make_tmap_bf16(&ty_n, Y, d, T, d, 64, BK))
@@ -884,7 +905,7 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
   p.err = err;
   const int grid = p.n_total < l.sms ? p.n_total : l.sms;
   inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tdv_k, tdv_n, twt_k, ty_n, tdv_k, tdv_k,
-                                                          tdv_n, tdv_n, p);
+                                                          tdv_n, tdv_n, tmf, p);
   if ((e = conv_bwd_launch(static_cast<const __nv_bfloat16*>(X0), conv_w, dY,
                            static_cast<__nv_bfloat16*>(dX0), part, dconv_w, T, d, k, s)))
     return e;
@@ -898,9 +919,10 @@ cudaError_t inplace_delta_run(int T, int d_ff, int d_model, float lr, const void
                               const void* Vhat, float* dW, void* ws, unsigned* err,
                               cudaStream_t s) {
   int* counter = static_cast<int*>(ws);
-  CUtensorMap tzb, tvh;
+  CUtensorMap tzb, tvh, tmf;
   if (!make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
-      !make_tmap_bf16(&tvh, Vhat, d_model, T, d_model, 64, BK))
+      !make_tmap_bf16(&tvh, Vhat, d_model, T, d_model, 64, BK) ||
+      !make_tmap_f32(&tmf, dW, d_ff, d_model, d_ff, MBOX, BM))
     return cudaErrorInvalidValue;
   Launch l;
   cudaError_t e = prepare(&l);
@@ -923,7 +945,8 @@ cudaError_t inplace_delta_run(int T, int d_ff, int d_model, float lr, const void
   p.counter = counter;
   p.err = err;
   const int grid = p.n_total < l.sms ? p.n_total : l.sms;
-  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tzb, tzb, tzb, tvh, tzb, tzb, tzb, tzb, p);
+  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tzb, tzb, tzb, tvh, tzb, tzb, tzb, tzb, tmf,
+                                                          p);
   count_launches(1);
   return cudaGetLastError();
 }

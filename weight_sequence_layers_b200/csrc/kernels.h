@@ -126,6 +126,9 @@ void count_launches(int n);
 // `row_stride_elems` apart; box = {box_inner (64), box_rows}. Returns false on failure.
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                     uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_rows);
+// 2-D float32 tensor map without swizzle (row-major boxes of box_rows x box_inner floats).
+bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                   uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_rows);
 // 3-D bf16 tensor map (inner, rows, batch) with 128-byte swizzle; box = {box_inner, box_rows, 1}.
 bool make_tmap3_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                      uint64_t batch, uint64_t row_stride_elems, uint64_t batch_stride_elems,
