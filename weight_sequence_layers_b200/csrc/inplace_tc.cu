@@ -76,23 +76,25 @@ struct Tile {
   int kind, m0, n0, nkb;
 };
 
+// Tile t of a launch whose tiles are TM rows high (128 for one CTA, 256 for a CTA pair).
+template <int TM = BM>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
   Tile x;
   if (t < p.n_row) {
     x.kind = KIND_ROW;
-    x.m0 = (t / p.n_row_n) * BM;  // token offset inside the chunk
+    x.m0 = (t / p.n_row_n) * TM;  // token offset inside the chunk
     x.n0 = (t % p.n_row_n) * BN;  // d_model column
     x.nkb = p.kb_row;
   } else if (t < p.n_row + p.n_dz) {
     const int u = t - p.n_row;
     x.kind = KIND_DZ;
-    x.m0 = (u / p.n_dz_n) * BM;   // token offset inside the chunk
+    x.m0 = (u / p.n_dz_n) * TM;   // token offset inside the chunk
     x.n0 = (u % p.n_dz_n) * BN;   // d_ff column
     x.nkb = p.kb_dz;
   } else {
     const int u = t - p.n_row - p.n_dz;
     x.kind = KIND_UPD;
-    x.m0 = (u / p.n_upd_n) * BM;  // d_model row
+    x.m0 = (u / p.n_upd_n) * TM;  // d_model row
     x.n0 = (u % p.n_upd_n) * BN;  // d_ff column
     x.nkb = p.kb_upd;
   }
@@ -289,29 +291,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         // fp32 read-modify-write of M and its scaled bf16 copy. TMEM hands each thread one row;
         // a padded shared tile transposes the warp's 32 x 32 block so that the lanes walk along
-        // a row and every global access is one coalesced 128-byte (bf16: 64-byte) request.
+        // a row and every global access is one coalesced 128-byte (bf16: 64-byte) request. The
+        // 32 row loads of the next column block are issued before the current block's stores,
+        // so that a warp keeps up to 64 loads (of the block of M prefetched into L2) in flight.
         float* xt = xpose + (warp - 2) * kXpose;
         const int mbase = x.m0 + q * 32;
         const float s = p.acc_scale, cs = p.copy_scale;
-        for (int cb = cb0; cb < cb1; ++cb) {
+        const size_t ld = p.d_ff;
+        auto valid = [&](int cb) { return x.n0 + cb * 32 < p.d_ff; };  // the same for every lane
+        auto load_block = [&](int cb, float (&w)[32]) {
+          const float* lp = p.M + (size_t)mbase * ld + x.n0 + cb * 32 + lane;
+#pragma unroll
+          for (int r = 0; r < 32; ++r, lp += ld) w[r] = __ldcg(lp);
+        };
+        auto stage_acc = [&](int cb) {  // this block of the accumulator into the transpose tile
           float v[32];
           tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
           tmem_wait_ld();
-          const int col = x.n0 + cb * 32 + lane;
-          if (x.n0 + cb * 32 >= p.d_ff) continue;  // the same for every lane
 #pragma unroll
           for (int j = 0; j < 32; ++j) xt[lane * 33 + j] = v[j];
           __syncwarp();
-          const size_t ld = p.d_ff;
-          // rows mbase .. mbase + 31 (d_model is a multiple of 128: all inside M): all 32
-          // coalesced loads in flight, then the stores, walking one row pointer each
+        };
+        auto store_block = [&](int cb, const float (&w)[32]) {
+          const int col = x.n0 + cb * 32 + lane;
           float* mp = p.M + (size_t)mbase * ld + col;
-          float w[32];
-          {
-            const float* lp = mp;
-#pragma unroll
-            for (int r = 0; r < 32; ++r, lp += ld) w[r] = *lp;
-          }
           __nv_bfloat16* bp =
               p.wb_next_row0 >= 0 ? p.Mb + (size_t)(p.wb_next_row0 + mbase) * ld + col : nullptr;
 #pragma unroll
@@ -323,7 +326,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               bp += ld;
             }
           }
-          __syncwarp();  // the tile is rewritten by the next step
+        };
+        // rows mbase .. mbase + 31 (d_model is a multiple of 128: all inside M)
+        float wa[32], wb[32];
+        if (valid(cb0)) load_block(cb0, wa);
+#pragma unroll
+        for (int i = 0; i < BN / 64; i += 2) {
+          const int cb = cb0 + i;
+          stage_acc(cb);
+          if (valid(cb + 1)) load_block(cb + 1, wb);
+          if (valid(cb)) store_block(cb, wa);
+          __syncwarp();  // the transpose tile is rewritten by the next block
+          stage_acc(cb + 1);
+          if (i + 2 < BN / 64 && valid(cb + 2)) load_block(cb + 2, wa);
+          if (valid(cb + 1)) store_block(cb + 1, wb);
+          __syncwarp();
         }
       }
       tc_fence_before();
@@ -340,6 +357,407 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// ============================================================================= CTA pairs
+// The same tile program on 2-CTA clusters with tcgen05.mma.cta_group::2: a tile is 256 rows
+// x 256 columns, each CTA of the pair holds 128 rows of A and 128 of the 256 columns of B in
+// its shared memory and receives its 128 rows x 256 columns of the accumulator in its own
+// TMEM. Per K step an SM thus loads 32 KB instead of 48 KB for the same flops, which is what
+// bounds the single-CTA tiles (operand traffic from L2). The leader CTA (rank 0) takes tiles
+// from the queue and hands each index to its peer through distributed shared memory; both
+// CTAs load their halves with TMA (no multicast), completing on the leader's stage barrier;
+// the leader's one MMA thread issues the pair MMAs and its commits arrive on the stage and
+// accumulator barriers of both CTAs; both CTAs drain their own accumulator rows, and the peer
+// signals the leader's accumulator-free and tile-free barriers remotely.
+constexpr int PTM = 2 * BM;                     // rows of a pair tile
+constexpr int P_STAGES = 6;
+constexpr uint32_t PA_BYTES = BM * BK * 2;      // 16 KB: this CTA's 128 rows of A
+constexpr uint32_t PB_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's 128 columns of B
+constexpr uint32_t P_STAGE = PA_BYTES + PB_BYTES;
+constexpr int kPairTileReaders = 2 * (1 + kEpiWarps);  // leader MMA + epilogue, peer producer +
+                                                       // epilogue
+
+struct __align__(8) PairBars {
+  uint64_t full[P_STAGES], empty[P_STAGES], acc_full[2], acc_empty[2], tile_full[RING],
+      tile_empty[RING];
+  int ring[RING];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr size_t kPairSmemBytes =
+    P_STAGES * P_STAGE + sizeof(PairBars) + kEpiWarps * kXpose * sizeof(float) + 1024;
+static_assert(kPairSmemBytes <= 232448, "shared memory of one CTA");
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared-memory word in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+// Arrive (release at cluster scope) on an mbarrier given by its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait with acquire at cluster scope (for what the other CTA of the pair wrote).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const Abort& ab) {
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*ab.flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *ab.flag = 1;
+        atomicOr(ab.err, ERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// 2-D TMA load into this CTA's shared memory whose completion counts on `bar_cluster`, an
+// mbarrier of either CTA of the pair (here always the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* m,
+                                                 uint32_t bar_cluster, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrives once on the mbarrier at this shared-memory offset in both CTAs of the pair when
+// every pair MMA issued so far by this thread has completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  const uint16_t both = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar), "h"(both)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    inplace_pair_kernel(const __grid_constant__ CUtensorMap tm_za,    // Z, K-major, 128 rows
+                        const __grid_constant__ CUtensorMap tm_zb,    // Z, MN-major boxes
+                        const __grid_constant__ CUtensorMap tm_mb,    // bf16 copy, K-major, 128 rows
+                        const __grid_constant__ CUtensorMap tm_x,     // Vhat or dO, MN-major
+                        const __grid_constant__ CUtensorMap tm_do,    // dO, K-major
+                        const __grid_constant__ CUtensorMap tm_vk,    // Vhat, K-major
+                        const __grid_constant__ CUtensorMap tm_wc,    // saved W_i, MN-major
+                        const __grid_constant__ CUtensorMap tm_mbn,   // bf16 copy, MN-major
+                        const __grid_constant__ CUtensorMap tm_mf,    // float32 M (prefetch)
+                        const Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  PairBars* bars = reinterpret_cast<PairBars*>(smem + P_STAGES * P_STAGE);
+  float* xpose = reinterpret_cast<float*>(smem + P_STAGES * P_STAGE + sizeof(PairBars));
+  const uint32_t stage0 = smem_u32(smem);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int half = (int)rank * BM;  // this CTA's first row (and first B column) of a pair tile
+  Abort ab{&bars->abort_flag, p.err};
+#define PB(x) smem_u32(&bars->x)
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(PB(full[s]), 1);
+      mbar_init(PB(empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(PB(acc_full[a]), 1);
+      mbar_init(PB(acc_empty[a]), 2 * kEpiWarps);
+    }
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(PB(tile_full[r]), 1);
+      mbar_init(PB(tile_empty[r]), kPairTileReaders);
+    }
+    bars->abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_za);
+    tma_prefetch_desc(&tm_zb);
+    tma_prefetch_desc(&tm_mb);
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_mf);
+    if (p.n_dz) {
+      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_vk);
+      tma_prefetch_desc(&tm_wc);
+      tma_prefetch_desc(&tm_mbn);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(PB(tmem_base), kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const int row_base = p.chunk * p.C;  // first token of this chunk
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      int r = 0, s = 0;
+      uint32_t rph = 0, sph = 0;
+      for (;;) {
+        int t;
+        if (leader) {
+          if (!mbar_wait_cluster(PB(tile_empty[r]), rph ^ 1, ab)) break;
+          t = atomicAdd(p.counter, 1);
+          bars->ring[r] = t;
+          st_cluster_u32(peer_addr(PB(ring[r]), 1), t);
+          mbar_arrive(PB(tile_full[r]));
+          mbar_arrive_cluster(peer_addr(PB(tile_full[r]), 1));
+        } else {
+          if (!mbar_wait_cluster(PB(tile_full[r]), rph, ab)) break;
+          t = bars->ring[r];
+          mbar_arrive_cluster(peer_addr(PB(tile_empty[r]), 0));
+        }
+        if (++r == RING) { r = 0; rph ^= 1; }
+        if (t >= p.n_total) break;
+        const Tile x = decode<PTM>(p, t);
+        const int m0 = x.m0 + half, nb = x.n0 + half;  // this CTA's rows of A, columns of B
+        if (x.kind == KIND_UPD && m0 < p.d_model)
+          for (int j = 0; j < BN / MBOX; ++j) tma_prefetch_l2_2d(&tm_mf, x.n0 + MBOX * j, m0);
+        bool ok = true;
+        for (int kb = 0; kb < x.nkb && ok; ++kb) {
+          if (!mbar_wait(PB(empty[s]), sph ^ 1, ab)) { ok = false; break; }
+          // both halves of the stage complete on the leader's barrier
+          if (leader) mbar_arrive_expect_tx(PB(full[s]), 2 * P_STAGE);
+          const uint32_t fb = peer_addr(PB(full[s]), 0);
+          const uint32_t sa = stage0 + s * P_STAGE, sb = sa + PA_BYTES;
+          if (x.kind == KIND_ROW) {
+            tma_load_2d_pair(sa, &tm_za, fb, kb * BK, row_base + m0);
+            tma_load_2d_pair(sb, &tm_mb, fb, kb * BK, p.wb_cur_row0 + nb);
+          } else if (x.kind == KIND_DZ) {
+            // K runs over [dO_i | Vhat_i] against [W_i ; eta Wh_{i+1}]
+            const bool first = kb < p.kb_dz_split;
+            const int k0 = (first ? kb : kb - p.kb_dz_split) * BK;
+            tma_load_2d_pair(sa, first ? &tm_do : &tm_vk, fb, k0, row_base + m0);
+            const CUtensorMap* mb = first ? &tm_wc : &tm_mbn;
+            const int r0 = (first ? p.wc_row0 : p.wb_cur_row0) + k0;
+            for (int j = 0; j < 2; ++j) tma_load_2d_pair(sb + 8192 * j, mb, fb, nb + 64 * j, r0);
+          } else {
+            const int tok = row_base + kb * BK;
+            tma_load_2d_pair(sa, &tm_x, fb, m0, tok);
+            tma_load_2d_pair(sa + 8192, &tm_x, fb, m0 + 64, tok);
+            for (int j = 0; j < 2; ++j) tma_load_2d_pair(sb + 8192 * j, &tm_zb, fb, nb + 64 * j, tok);
+          }
+          if (++s == P_STAGES) { s = 0; sph ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issue (the leader's thread)
+    if (lane == 0 && leader) {
+      int r = 0, s = 0, acc = 0;
+      uint32_t rph = 0, sph = 0, aph = 0;
+      const uint32_t id_row = idesc_bf16(PTM, BN, 0, 0);
+      const uint32_t id_dz = idesc_bf16(PTM, BN, 0, 1);
+      const uint32_t id_upd = idesc_bf16(PTM, BN, 1, 1);
+      for (;;) {
+        if (!mbar_wait(PB(tile_full[r]), rph, ab)) break;
+        const int t = bars->ring[r];
+        mbar_arrive(PB(tile_empty[r]));
+        if (++r == RING) { r = 0; rph ^= 1; }
+        if (t >= p.n_total) break;
+        const Tile x = decode<PTM>(p, t);
+        // both CTAs' epilogues have drained this accumulator
+        if (!mbar_wait_cluster(PB(acc_empty[acc]), aph ^ 1, ab)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + acc * BN;
+        const uint32_t id = x.kind == KIND_ROW ? id_row : x.kind == KIND_DZ ? id_dz : id_upd;
+        const bool a_kmaj = x.kind != KIND_UPD, b_kmaj = x.kind == KIND_ROW;
+        bool ok = true;
+        for (int kb = 0; kb < x.nkb; ++kb) {
+          if (!mbar_wait(PB(full[s]), sph, ab)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = stage0 + s * P_STAGE, sb = sa + PA_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = a_kmaj ? sdesc_sw128(sa + kk * 32, 16, 1024)
+                                       : sdesc_sw128(sa + kk * 2048, 8192, 1024);
+            const uint64_t bd = b_kmaj ? sdesc_sw128(sb + kk * 32, 16, 1024)
+                                       : sdesc_sw128(sb + kk * 2048, 8192, 1024);
+            mma_bf16_pair(d, ad, bd, id, (kb | kk) != 0);
+          }
+          mma_commit_pair(PB(empty[s]));  // the stage is free in both CTAs
+          if (++s == P_STAGES) { s = 0; sph ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit_pair(PB(acc_full[acc]));
+        if (++acc == 2) { acc = 0; aph ^= 1; }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue (both CTAs)
+    // Warp w drains TMEM lanes 32*(w%4) .. +31 (thread = one row of this CTA's half) and
+    // columns [128 h, 128 h + 128) with h = (w - 2) / 4, as in the single-CTA kernel.
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int hcol = (warp - 2) / 4;
+    int r = 0, acc = 0;
+    uint32_t rph = 0, aph = 0;
+    for (;;) {
+      if (!mbar_wait_cluster(PB(tile_full[r]), rph, ab)) break;
+      const int t = bars->ring[r];
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(PB(tile_empty[r]));
+        else
+          mbar_arrive_cluster(peer_addr(PB(tile_empty[r]), 0));
+      }
+      if (++r == RING) { r = 0; rph ^= 1; }
+      if (t >= p.n_total) break;
+      const Tile x = decode<PTM>(p, t);
+      const int m0 = x.m0 + half;
+      if (!mbar_wait(PB(acc_full[acc]), aph, ab)) break;
+      __syncwarp();
+      tc_fence_after();
+      const int cb0 = hcol * (BN / 64), cb1 = cb0 + BN / 64;
+      if (x.kind != KIND_UPD) {
+        // bf16 rows of O_i / dVhat_i ([T, d_model]) or dZ_i ([T, d_ff]); rows past the chunk
+        // (a pair tile reaching beyond C) are not written
+        const int ncol = x.kind == KIND_ROW ? p.d_model : p.d_ff;
+        const bool row_ok = m0 + row < p.C;
+        __nv_bfloat16* out = (x.kind == KIND_ROW ? p.Orow : p.Odz) +
+                             (size_t)(row_base + (row_ok ? m0 + row : 0)) * ncol;
+        for (int cb = cb0; cb < cb1; ++cb) {
+          float v[32];
+          tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
+          tmem_wait_ld();
+          const int col0 = x.n0 + cb * 32;
+          if (row_ok && col0 < ncol) {
+            uint4* dst = reinterpret_cast<uint4*>(out + col0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]),
+                                  pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
+                                  pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
+                                  pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
+          }
+        }
+      } else {
+        // fp32 read-modify-write of M and its scaled bf16 copy, as in the single-CTA kernel;
+        // a warp whose 32 rows lie past d_model (the upper half of the last pair tile when
+        // d_model is not a multiple of 256) touches no memory
+        float* xt = xpose + (warp - 2) * kXpose;
+        const int mbase = m0 + q * 32;
+        const bool rows_ok = mbase < p.d_model;  // d_model is a multiple of 128
+        const float s = p.acc_scale, cs = p.copy_scale;
+        const size_t ld = p.d_ff;
+        auto valid = [&](int cb) { return rows_ok && x.n0 + cb * 32 < p.d_ff; };
+        auto load_block = [&](int cb, float (&w)[32]) {
+          const float* lp = p.M + (size_t)mbase * ld + x.n0 + cb * 32 + lane;
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr, lp += ld) w[rr] = __ldcg(lp);
+        };
+        auto stage_acc = [&](int cb) {
+          float v[32];
+          tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) xt[lane * 33 + j] = v[j];
+          __syncwarp();
+        };
+        auto store_block = [&](int cb, const float (&w)[32]) {
+          const int col = x.n0 + cb * 32 + lane;
+          float* mp = p.M + (size_t)mbase * ld + col;
+          __nv_bfloat16* bp =
+              p.wb_next_row0 >= 0 ? p.Mb + (size_t)(p.wb_next_row0 + mbase) * ld + col : nullptr;
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr, mp += ld) {
+            const float o = w[rr] + s * xt[rr * 33 + lane];
+            *mp = o;
+            if (bp) {
+              *bp = __float2bfloat16_rn(cs * o);
+              bp += ld;
+            }
+          }
+        };
+        float wa[32], wb[32];
+        if (valid(cb0)) load_block(cb0, wa);
+#pragma unroll
+        for (int i = 0; i < BN / 64; i += 2) {
+          const int cb = cb0 + i;
+          stage_acc(cb);
+          if (valid(cb + 1)) load_block(cb + 1, wb);
+          if (valid(cb)) store_block(cb, wa);
+          __syncwarp();
+          stage_acc(cb + 1);
+          if (i + 2 < BN / 64 && valid(cb + 2)) load_block(cb + 2, wa);
+          if (valid(cb + 1)) store_block(cb + 1, wb);
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (leader)
+          mbar_arrive(PB(acc_empty[acc]));
+        else
+          mbar_arrive_cluster(peer_addr(PB(acc_empty[acc]), 0));
+      }
+      if (++acc == 2) { acc = 0; aph ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();  // no MMA of the leader still writes the peer's TMEM
+  if (bars->abort_flag) __nanosleep(100000);  // let any load issued before the abort land
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kTmemCols);
+  }
+#undef PB
 }
 
 // dst = bf16(scale * src) over n elements.
@@ -632,6 +1050,7 @@ cudaError_t conv_bwd_launch(const __nv_bfloat16* X0, const float* w, const __nv_
 
 struct Launch {
   int sms;
+  int pairs;  // CTA pairs that fit on the device at once
 };
 
 cudaError_t prepare(Launch* l) {
@@ -640,8 +1059,43 @@ cudaError_t prepare(Launch* l) {
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&l->sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(inplace_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)kSmemBytes);
+  e = cudaFuncSetAttribute(inplace_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(inplace_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kPairSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (l->sms / 2));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, inplace_pair_kernel, &cfg) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = l->sms / 2;
+  }
+  l->pairs = n;
+  return cudaSuccess;
+}
+
+// Tile counts of a pair launch: row and dz tiles over `rows` token rows, update tiles over the
+// d_model rows of M, each 256 rows high (the N counts are set by the caller).
+void pair_tiles(Params& p, int row_rows, int dz_rows, int upd_rows) {
+  auto blocks = [](int rows) { return (rows + PTM - 1) / PTM; };
+  p.n_row = row_rows ? blocks(row_rows) * p.n_row_n : 0;
+  p.n_dz = dz_rows ? blocks(dz_rows) * p.n_dz_n : 0;
+  p.n_total = p.n_row + p.n_dz + (upd_rows ? blocks(upd_rows) * p.n_upd_n : 0);
+}
+
+// One launch of the tile program on CTA pairs (grid: the co-resident pairs, at most one per
+// tile).
+void launch_pairs(const Launch& l, const Params& p, cudaStream_t s, const CUtensorMap& za,
+                  const CUtensorMap& zb, const CUtensorMap& mb, const CUtensorMap& x,
+                  const CUtensorMap& dO, const CUtensorMap& vk, const CUtensorMap& wc,
+                  const CUtensorMap& mbn, const CUtensorMap& mf) {
+  const int pairs = p.n_total < l.pairs ? p.n_total : l.pairs;
+  inplace_pair_kernel<<<2 * pairs, kThreads, kPairSmemBytes, s>>>(za, zb, mb, x, dO, vk, wc, mbn,
+                                                                  mf, p);
 }
 
 }  // namespace
@@ -671,7 +1125,7 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   CUtensorMap tza, tzb, twb, tvh, tmf;
   if (!make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
       !make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
-      !make_tmap_bf16(&twb, Wb, d_ff, wb_rows, d_ff, BK, BN) ||
+      !make_tmap_bf16(&twb, Wb, d_ff, wb_rows, d_ff, BK, BN / 2) ||
       !make_tmap_bf16(&tvh, Vhat, d_model, T, d_model, 64, BK) ||
       !make_tmap_f32(&tmf, W, d_ff, d_model, d_ff, MBOX, BM))
     return cudaErrorInvalidValue;
@@ -690,8 +1144,7 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   p.d_model = d_model;
   p.n_row_n = (d_model + BN - 1) / BN;
   p.n_upd_n = (d_ff + BN - 1) / BN;
-  p.n_row = (C / BM) * p.n_row_n;
-  p.n_total = p.n_row + (d_model / BM) * p.n_upd_n;
+  pair_tiles(p, C, 0, d_model);
   p.kb_row = d_ff / BK;
   p.kb_upd = C / BK;
   p.acc_scale = lr;
@@ -700,7 +1153,6 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   p.Mb = Wb;
   p.Orow = static_cast<__nv_bfloat16*>(O);
   p.err = err;
-  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
   for (int i = 0; i < NC; ++i) {
     p.chunk = i;
     if (W_chunks) {
@@ -718,8 +1170,7 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
       to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W0, Wb + (size_t)p.wb_cur_row0 * d_ff, nW, 1.f);
       ++launches;
     }
-    inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, twb, tvh, tza, tza, tzb, tzb,
-                                                            tmf, p);
+    launch_pairs(l, p, s, tza, tzb, twb, tvh, tza, tza, tzb, tzb, tmf);
   }
   count_launches(launches);
   return cudaGetLastError();
@@ -742,7 +1193,7 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   if (!make_tmap_f32(&tmf, R, d_ff, d_model, d_ff, MBOX, BM) ||
       !make_tmap_bf16(&tza, Z, d_ff, T, d_ff, BK, BM) ||
       !make_tmap_bf16(&tzb, Z, d_ff, T, d_ff, 64, BK) ||
-      !make_tmap_bf16(&tmb, Mb, d_ff, 2 * (size_t)d_model, d_ff, BK, BN) ||
+      !make_tmap_bf16(&tmb, Mb, d_ff, 2 * (size_t)d_model, d_ff, BK, BN / 2) ||
       !make_tmap_bf16(&tdx, dO, d_model, T, d_model, 64, BK) ||
       !make_tmap_bf16(&tdo, dO, d_model, T, d_model, BK, BM) ||
       !make_tmap_bf16(&tvk, Vhat, d_model, T, d_model, BK, BM) ||
@@ -774,9 +1225,7 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   p.n_row_n = (d_model + BN - 1) / BN;
   p.n_dz_n = (d_ff + BN - 1) / BN;
   p.n_upd_n = (d_ff + BN - 1) / BN;
-  p.n_row = (C / BM) * p.n_row_n;
-  p.n_dz = (C / BM) * p.n_dz_n;
-  p.n_total = p.n_row + p.n_dz + (d_model / BM) * p.n_upd_n;
+  pair_tiles(p, C, C, d_model);
   p.kb_row = d_ff / BK;
   p.kb_dz_split = d_model / BK;
   p.kb_dz = 2 * p.kb_dz_split;
@@ -788,15 +1237,13 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   p.Orow = static_cast<__nv_bfloat16*>(dVhat);
   p.Odz = static_cast<__nv_bfloat16*>(dZ);
   p.err = err;
-  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
   for (int i = NC - 1; i >= 0; --i) {
     p.chunk = i;
     p.wb_cur_row0 = (i & 1) * d_model;
     p.wb_next_row0 = i > 0 ? ((i - 1) & 1) * d_model : -1;
     p.wc_row0 = i * d_model;
     p.counter = counters + i;
-    inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tza, tzb, tmb, tdx, tdo, tvk, twc,
-                                                            tmbn, tmf, p);
+    launch_pairs(l, p, s, tza, tzb, tmb, tdx, tdo, tvk, twc, tmbn, tmf);
     if (reset && (i == 0 || reset[i])) {
       // this document's first chunk applied the initial W: its adjoint joins dW, and the
       // previous document's end state (and its bf16 copy) gets none
@@ -837,16 +1284,14 @@ cudaError_t inplace_target_run(int T, int d, int k, const void* X0, const float*
   p.d_ff = d;
   p.d_model = d;
   p.n_dz_n = (d + BN - 1) / BN;
-  p.n_dz = (T / BM) * p.n_dz_n;
-  p.n_total = p.n_dz;
+  pair_tiles(p, 0, T, 0);
   p.kb_dz = d / BK;
   p.kb_dz_split = p.kb_dz;  // every k-block from the first operand pair
   p.wb_next_row0 = -1;
   p.Odz = static_cast<__nv_bfloat16*>(Vhat);
   p.counter = counter;
   p.err = err;
-  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
-  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(ty, ty, ty, ty, ty, ty, twt, twt, ty, p);
+  launch_pairs(l, p, s, ty, ty, ty, ty, ty, ty, twt, twt, ty);
   count_launches(2);
   return cudaGetLastError();
 }
@@ -874,7 +1319,7 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
   if (!make_tmap_f32(&tmf, dW_target, d, d, d, MBOX, BM) ||
       !make_tmap_bf16(&tdv_k, dVhat, d, T, d, BK, BM) ||
       !make_tmap_bf16(&tdv_n, dVhat, d, T, d, 64, BK) ||
-      !make_tmap_bf16(&twt_k, W_target, d, d, d, BK, BN) ||
+      !make_tmap_bf16(&twt_k, W_target, d, d, d, BK, BN / 2) ||
       !make_tmap_bf16(&ty_n, Y, d, T, d, 64, BK))
     return cudaErrorInvalidValue;
   Launch l;
@@ -892,8 +1337,7 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
   p.d_model = d;
   p.n_row_n = (d + BN - 1) / BN;
   p.n_upd_n = (d + BN - 1) / BN;
-  p.n_row = (T / BM) * p.n_row_n;
-  p.n_total = p.n_row + (d / BM) * p.n_upd_n;
+  pair_tiles(p, T, 0, d);
   p.kb_row = d / BK;
   p.kb_upd = T / BK;
   p.wb_next_row0 = -1;
@@ -903,9 +1347,7 @@ cudaError_t inplace_target_bwd_run(int T, int d, int k, const void* X0, const fl
   p.Orow = dY;
   p.counter = counter;
   p.err = err;
-  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
-  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tdv_k, tdv_n, twt_k, ty_n, tdv_k, tdv_k,
-                                                          tdv_n, tdv_n, tmf, p);
+  launch_pairs(l, p, s, tdv_k, tdv_n, twt_k, ty_n, tdv_k, tdv_k, tdv_n, tdv_n, tmf);
   if ((e = conv_bwd_launch(static_cast<const __nv_bfloat16*>(X0), conv_w, dY,
                            static_cast<__nv_bfloat16*>(dX0), part, dconv_w, T, d, k, s)))
     return e;
@@ -936,7 +1378,7 @@ cudaError_t inplace_delta_run(int T, int d_ff, int d_model, float lr, const void
   p.d_ff = d_ff;
   p.d_model = d_model;
   p.n_upd_n = (d_ff + BN - 1) / BN;
-  p.n_total = (d_model / BM) * p.n_upd_n;
+  pair_tiles(p, 0, 0, d_model);
   p.kb_upd = T / BK;
   p.wb_next_row0 = -1;
   p.acc_scale = lr;
@@ -944,9 +1386,7 @@ cudaError_t inplace_delta_run(int T, int d_ff, int d_model, float lr, const void
   p.M = dW;
   p.counter = counter;
   p.err = err;
-  const int grid = p.n_total < l.sms ? p.n_total : l.sms;
-  inplace_chunk_kernel<<<grid, kThreads, kSmemBytes, s>>>(tzb, tzb, tzb, tvh, tzb, tzb, tzb, tzb, tmf,
-                                                          p);
+  launch_pairs(l, p, s, tzb, tzb, tzb, tvh, tzb, tzb, tzb, tzb, tmf);
   count_launches(1);
   return cudaGetLastError();
 }
