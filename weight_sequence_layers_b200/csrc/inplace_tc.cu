@@ -11,21 +11,28 @@
 //     dVhat_i = Z_i (eta Wh_{i+1})^T,  dZ_i = dO_i W_i + Vhat_i (eta Wh_{i+1}),
 //     Wh_i = Wh_{i+1} + dO_i^T Z_i     (Wh_0 is the gradient of the initial W).
 //
-// One launch per chunk runs every GEMM of that chunk from a shared dynamic tile queue. Tile
-// kinds, each an fp32 accumulator of 128 x 256 in TMEM:
-//   row tiles    [128 tokens x 256] = A (K-major) x B^T (K-major), A = Z_i, K = d_ff: the
+// One launch per chunk runs every GEMM of that chunk from a shared dynamic tile queue, on
+// 2-CTA clusters with tcgen05.mma.cta_group::2. A tile is 256 rows x 256 columns: each CTA of
+// the pair holds 128 rows of A and 128 of the 256 columns of B in its shared memory (32 KB per
+// K step of 64) and receives its 128 rows x 256 columns of the fp32 accumulator in its own
+// TMEM. Tile kinds:
+//   row tiles    [256 tokens x 256] = A (K-major) x B^T (K-major), A = Z_i, K = d_ff: the
 //                forward's O_i (B = bf16 W_i) and the backward's dVhat_i (B = bf16 eta Wh_{i+1});
-//   dz tiles     [128 tokens x 256 d_ff] = [dO_i | Vhat_i] (K-major, K = 2 d_model) x
+//   dz tiles     [256 tokens x 256 d_ff] = [dO_i | Vhat_i] (K-major, K = 2 d_model) x
 //                [W_i ; eta Wh_{i+1}] (MN-major): the backward's dZ_i;
-//   update tiles [128 d_model x 256 d_ff]: M += s X_i^T (MN-major) x Z_i (MN-major), K = C,
+//   update tiles [256 d_model x 256 d_ff]: M += s X_i^T (MN-major) x Z_i (MN-major), K = C,
 //                with (M, X, s) = (W, Vhat, eta) forward and (Wh, dO, 1) backward; the epilogue
 //                keeps M in float32 and writes the scaled bf16 copy the next launch reads.
 // Long tiles (row, then dz) are handed out first, update tiles fill the remaining SMs. When
-// the producer takes an update tile it prefetches the tile's float32 block of M into L2, so
-// the epilogue's read-modify-write, issued after the tile's K steps, reads from L2.
-// Warp roles: warp 0 issues TMA loads into a 4-stage ring, warp 1 issues tcgen05.mma into
-// two TMEM accumulators of 128 x 256 fp32, warps 2-9 drain the accumulators (two warps per
-// TMEM lane quadrant, each taking 128 of the 256 columns).
+// a CTA takes an update tile it prefetches its float32 block of M into L2, so the epilogue's
+// read-modify-write, issued after the tile's K steps, reads from L2.
+// Warp roles in each CTA: warp 0 issues TMA loads into a 6-stage ring, warp 1 of the leader CTA
+// (rank 0) issues the pair MMAs into two TMEM accumulators of 128 x 256 fp32 per CTA, warps 2-9
+// drain this CTA's accumulator rows (two warps per TMEM lane quadrant, each taking 128 of the
+// 256 columns). The leader takes tiles from the queue and hands each index to its peer through
+// distributed shared memory; both CTAs' loads (no multicast) complete on the leader's stage
+// barrier; the MMA commits arrive on the stage and accumulator barriers of both CTAs; the peer
+// signals the leader's accumulator-free and tile-free barriers remotely. Every wait is bounded.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -34,10 +41,7 @@
 namespace tttk {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, RING = 4;
-constexpr uint32_t A_BYTES = BM * BK * 2;      // 16 KB
-constexpr uint32_t B_BYTES = BN * BK * 2;      // 32 KB
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BM = 128, BN = 256, BK = 64, RING = 4;  // BM: rows of one CTA's half tile
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kXpose = 32 * 33;  // floats of one epilogue warp's padded 32 x 32 transpose tile
@@ -45,7 +49,7 @@ constexpr uint32_t kTmemCols = 512;            // two 256-column accumulators
 
 struct Params {
   int chunk, C, d_ff, d_model;
-  int n_row_n, n_dz_n, n_upd_n;  // N tiles per 128-row block of each kind
+  int n_row_n, n_dz_n, n_upd_n;  // N tiles per 256-row block of each kind
   int n_row, n_dz, n_total;      // tiles [0, n_row) row, [n_row, n_row + n_dz) dz, rest update
   int kb_row, kb_dz, kb_dz_split, kb_upd;
   int wb_cur_row0;               // first row of the bf16 copy this launch reads
@@ -76,8 +80,8 @@ struct Tile {
   int kind, m0, n0, nkb;
 };
 
-// Tile t of a launch whose tiles are TM rows high (128 for one CTA, 256 for a CTA pair).
-template <int TM = BM>
+// Tile t of a launch whose tiles are TM rows high (256: a CTA pair).
+template <int TM>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
   Tile x;
   if (t < p.n_row) {
@@ -101,275 +105,8 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
   return x;
 }
 
-struct __align__(8) Bars {
-  uint64_t full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], tile_full[RING],
-      tile_empty[RING];
-  int ring[RING];
-  uint32_t tmem_base;
-  int abort_flag;
-};
-
-__global__ void __launch_bounds__(kThreads, 1)
-    inplace_chunk_kernel(const __grid_constant__ CUtensorMap tm_za,    // Z, K-major boxes
-                         const __grid_constant__ CUtensorMap tm_zb,    // Z, MN-major boxes
-                         const __grid_constant__ CUtensorMap tm_mb,    // bf16 copy, K-major
-                         const __grid_constant__ CUtensorMap tm_x,     // Vhat or dO, MN-major
-                         const __grid_constant__ CUtensorMap tm_do,    // dO, K-major
-                         const __grid_constant__ CUtensorMap tm_vk,    // Vhat, K-major
-                         const __grid_constant__ CUtensorMap tm_wc,    // saved W_i, MN-major
-                         const __grid_constant__ CUtensorMap tm_mbn,   // bf16 copy, MN-major
-                         const __grid_constant__ CUtensorMap tm_mf,    // float32 M (prefetch)
-                         const Params p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES);
-  float* xpose = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + sizeof(Bars));
-  const uint32_t stage0 = smem_u32(smem);
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  Abort ab{&bars->abort_flag, p.err};
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&bars->full[s]), 1);
-      mbar_init(smem_u32(&bars->empty[s]), 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(smem_u32(&bars->acc_full[a]), 1);
-      mbar_init(smem_u32(&bars->acc_empty[a]), kEpiWarps);
-    }
-    for (int r = 0; r < RING; ++r) {
-      mbar_init(smem_u32(&bars->tile_full[r]), 1);
-      mbar_init(smem_u32(&bars->tile_empty[r]), 1 + kEpiWarps);
-    }
-    bars->abort_flag = 0;
-    fence_barrier_init();
-    tma_prefetch_desc(&tm_za);
-    tma_prefetch_desc(&tm_zb);
-    tma_prefetch_desc(&tm_mb);
-    tma_prefetch_desc(&tm_x);
-    tma_prefetch_desc(&tm_mf);
-    if (p.n_dz) {
-      tma_prefetch_desc(&tm_do);
-      tma_prefetch_desc(&tm_vk);
-      tma_prefetch_desc(&tm_wc);
-      tma_prefetch_desc(&tm_mbn);
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = bars->tmem_base;
-  const int row_base = p.chunk * p.C;  // first token of this chunk
-
-  if (warp == 0) {
-    if (lane == 0) {
-      int r = 0, s = 0;
-      uint32_t rph = 0, sph = 0;
-      for (;;) {
-        if (!mbar_wait(smem_u32(&bars->tile_empty[r]), rph ^ 1, ab)) break;
-        const int t = atomicAdd(p.counter, 1);
-        bars->ring[r] = t;
-        mbar_arrive(smem_u32(&bars->tile_full[r]));
-        if (++r == RING) { r = 0; rph ^= 1; }
-        if (t >= p.n_total) break;
-        const Tile x = decode(p, t);
-        if (x.kind == KIND_UPD)
-          for (int j = 0; j < BN / MBOX; ++j) tma_prefetch_l2_2d(&tm_mf, x.n0 + MBOX * j, x.m0);
-        bool ok = true;
-        for (int kb = 0; kb < x.nkb && ok; ++kb) {
-          if (!mbar_wait(smem_u32(&bars->empty[s]), sph ^ 1, ab)) { ok = false; break; }
-          const uint32_t fb = smem_u32(&bars->full[s]);
-          const uint32_t sa = stage0 + s * STAGE_BYTES, sb = sa + A_BYTES;
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          if (x.kind == KIND_ROW) {
-            tma_load_2d(sa, &tm_za, fb, kb * BK, row_base + x.m0);
-            tma_load_2d(sb, &tm_mb, fb, kb * BK, p.wb_cur_row0 + x.n0);
-          } else if (x.kind == KIND_DZ) {
-            // K runs over [dO_i | Vhat_i] against [W_i ; eta Wh_{i+1}]
-            const bool first = kb < p.kb_dz_split;
-            const int k0 = (first ? kb : kb - p.kb_dz_split) * BK;
-            tma_load_2d(sa, first ? &tm_do : &tm_vk, fb, k0, row_base + x.m0);
-            const CUtensorMap* mb = first ? &tm_wc : &tm_mbn;
-            const int r0 = (first ? p.wc_row0 : p.wb_cur_row0) + k0;
-            for (int j = 0; j < 4; ++j) tma_load_2d(sb + 8192 * j, mb, fb, x.n0 + 64 * j, r0);
-          } else {
-            const int tok = row_base + kb * BK;
-            tma_load_2d(sa, &tm_x, fb, x.m0, tok);
-            tma_load_2d(sa + 8192, &tm_x, fb, x.m0 + 64, tok);
-            for (int j = 0; j < 4; ++j) tma_load_2d(sb + 8192 * j, &tm_zb, fb, x.n0 + 64 * j, tok);
-          }
-          if (++s == STAGES) { s = 0; sph ^= 1; }
-        }
-        if (!ok) break;
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      int r = 0, s = 0, acc = 0;
-      uint32_t rph = 0, sph = 0, aph = 0;
-      const uint32_t id_row = idesc_bf16(BM, BN, 0, 0);
-      const uint32_t id_dz = idesc_bf16(BM, BN, 0, 1);
-      const uint32_t id_upd = idesc_bf16(BM, BN, 1, 1);
-      for (;;) {
-        if (!mbar_wait(smem_u32(&bars->tile_full[r]), rph, ab)) break;
-        const int t = bars->ring[r];
-        mbar_arrive(smem_u32(&bars->tile_empty[r]));
-        if (++r == RING) { r = 0; rph ^= 1; }
-        if (t >= p.n_total) break;
-        const Tile x = decode(p, t);
-        if (!mbar_wait(smem_u32(&bars->acc_empty[acc]), aph ^ 1, ab)) break;
-        tc_fence_after();
-        const uint32_t d = tmem + acc * BN;
-        const uint32_t id = x.kind == KIND_ROW ? id_row : x.kind == KIND_DZ ? id_dz : id_upd;
-        const bool a_kmaj = x.kind != KIND_UPD, b_kmaj = x.kind == KIND_ROW;
-        bool ok = true;
-        for (int kb = 0; kb < x.nkb; ++kb) {
-          if (!mbar_wait(smem_u32(&bars->full[s]), sph, ab)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sa = stage0 + s * STAGE_BYTES, sb = sa + A_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = a_kmaj ? sdesc_sw128(sa + kk * 32, 16, 1024)
-                                       : sdesc_sw128(sa + kk * 2048, 8192, 1024);
-            const uint64_t bd = b_kmaj ? sdesc_sw128(sb + kk * 32, 16, 1024)
-                                       : sdesc_sw128(sb + kk * 2048, 8192, 1024);
-            mma_bf16_ss(d, ad, bd, id, (kb | kk) != 0);
-          }
-          mma_commit(smem_u32(&bars->empty[s]));
-          if (++s == STAGES) { s = 0; sph ^= 1; }
-        }
-        if (!ok) break;
-        mma_commit(smem_u32(&bars->acc_full[acc]));
-        if (++acc == 2) { acc = 0; aph ^= 1; }
-      }
-    }
-  } else {
-    // Epilogue: warp w drains TMEM lanes 32*(w%4) .. +31 (thread = one accumulator row) and
-    // columns [128 h, 128 h + 128) with h = (w - 2) / 4.
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int hcol = (warp - 2) / 4;
-    int r = 0, acc = 0;
-    uint32_t rph = 0, aph = 0;
-    for (;;) {
-      if (!mbar_wait(smem_u32(&bars->tile_full[r]), rph, ab)) break;
-      const int t = bars->ring[r];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->tile_empty[r]));
-      if (++r == RING) { r = 0; rph ^= 1; }
-      if (t >= p.n_total) break;
-      const Tile x = decode(p, t);
-      if (!mbar_wait(smem_u32(&bars->acc_full[acc]), aph, ab)) break;
-      __syncwarp();
-      tc_fence_after();
-      const int cb0 = hcol * (BN / 64), cb1 = cb0 + BN / 64;
-      if (x.kind != KIND_UPD) {
-        // bf16 rows of O_i / dVhat_i ([T, d_model]) or dZ_i ([T, d_ff])
-        const int ncol = x.kind == KIND_ROW ? p.d_model : p.d_ff;
-        __nv_bfloat16* out = (x.kind == KIND_ROW ? p.Orow : p.Odz) +
-                             (size_t)(row_base + x.m0 + row) * ncol;
-        for (int cb = cb0; cb < cb1; ++cb) {
-          float v[32];
-          tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
-          tmem_wait_ld();
-          const int col0 = x.n0 + cb * 32;
-          if (col0 < ncol) {
-            uint4* dst = reinterpret_cast<uint4*>(out + col0);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              dst[j] = make_uint4(pack_bf16x2(v[8 * j], v[8 * j + 1]),
-                                  pack_bf16x2(v[8 * j + 2], v[8 * j + 3]),
-                                  pack_bf16x2(v[8 * j + 4], v[8 * j + 5]),
-                                  pack_bf16x2(v[8 * j + 6], v[8 * j + 7]));
-          }
-        }
-      } else {
-        // fp32 read-modify-write of M and its scaled bf16 copy. TMEM hands each thread one row;
-        // a padded shared tile transposes the warp's 32 x 32 block so that the lanes walk along
-        // a row and every global access is one coalesced 128-byte (bf16: 64-byte) request. The
-        // 32 row loads of the next column block are issued before the current block's stores,
-        // so that a warp keeps up to 64 loads (of the block of M prefetched into L2) in flight.
-        float* xt = xpose + (warp - 2) * kXpose;
-        const int mbase = x.m0 + q * 32;
-        const float s = p.acc_scale, cs = p.copy_scale;
-        const size_t ld = p.d_ff;
-        auto valid = [&](int cb) { return x.n0 + cb * 32 < p.d_ff; };  // the same for every lane
-        auto load_block = [&](int cb, float (&w)[32]) {
-          const float* lp = p.M + (size_t)mbase * ld + x.n0 + cb * 32 + lane;
-#pragma unroll
-          for (int r = 0; r < 32; ++r, lp += ld) w[r] = __ldcg(lp);
-        };
-        auto stage_acc = [&](int cb) {  // this block of the accumulator into the transpose tile
-          float v[32];
-          tmem_ld32(tmem_addr(tmem, q * 32, acc * BN + cb * 32), v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) xt[lane * 33 + j] = v[j];
-          __syncwarp();
-        };
-        auto store_block = [&](int cb, const float (&w)[32]) {
-          const int col = x.n0 + cb * 32 + lane;
-          float* mp = p.M + (size_t)mbase * ld + col;
-          __nv_bfloat16* bp =
-              p.wb_next_row0 >= 0 ? p.Mb + (size_t)(p.wb_next_row0 + mbase) * ld + col : nullptr;
-#pragma unroll
-          for (int r = 0; r < 32; ++r, mp += ld) {
-            const float o = w[r] + s * xt[r * 33 + lane];
-            *mp = o;
-            if (bp) {
-              *bp = __float2bfloat16_rn(cs * o);
-              bp += ld;
-            }
-          }
-        };
-        // rows mbase .. mbase + 31 (d_model is a multiple of 128: all inside M)
-        float wa[32], wb[32];
-        if (valid(cb0)) load_block(cb0, wa);
-#pragma unroll
-        for (int i = 0; i < BN / 64; i += 2) {
-          const int cb = cb0 + i;
-          stage_acc(cb);
-          if (valid(cb + 1)) load_block(cb + 1, wb);
-          if (valid(cb)) store_block(cb, wa);
-          __syncwarp();  // the transpose tile is rewritten by the next block
-          stage_acc(cb + 1);
-          if (i + 2 < BN / 64 && valid(cb + 2)) load_block(cb + 2, wa);
-          if (valid(cb + 1)) store_block(cb + 1, wb);
-          __syncwarp();
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->acc_empty[acc]));
-      if (++acc == 2) { acc = 0; aph ^= 1; }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (bars->abort_flag) __nanosleep(100000);  // let any load issued before the abort land
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
-  }
-}
 
 // ============================================================================= CTA pairs
-// The same tile program on 2-CTA clusters with tcgen05.mma.cta_group::2: a tile is 256 rows
-// x 256 columns, each CTA of the pair holds 128 rows of A and 128 of the 256 columns of B in
-// its shared memory and receives its 128 rows x 256 columns of the accumulator in its own
-// TMEM. Per K step an SM thus loads 32 KB instead of 48 KB for the same flops, which is what
-// bounds the single-CTA tiles (operand traffic from L2). The leader CTA (rank 0) takes tiles
-// from the queue and hands each index to its peer through distributed shared memory; both
-// CTAs load their halves with TMA (no multicast), completing on the leader's stage barrier;
-// the leader's one MMA thread issues the pair MMAs and its commits arrive on the stage and
-// accumulator barriers of both CTAs; both CTAs drain their own accumulator rows, and the peer
-// signals the leader's accumulator-free and tile-free barriers remotely.
 constexpr int PTM = 2 * BM;                     // rows of a pair tile
 constexpr int P_STAGES = 6;
 constexpr uint32_t PA_BYTES = BM * BK * 2;      // 16 KB: this CTA's 128 rows of A
@@ -768,8 +505,6 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
     dst[i] = __float2bfloat16_rn(scale * src[i]);
 }
 
-constexpr size_t kSmemBytes =
-    STAGES * STAGE_BYTES + sizeof(Bars) + kEpiWarps * kXpose * sizeof(float) + 1024;
 
 // dst += src over n floats (n a multiple of 4).
 __global__ void add_kernel(float* __restrict__ dst, const float* __restrict__ src, size_t n4) {
@@ -1058,9 +793,6 @@ cudaError_t prepare(Launch* l) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&l->sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(inplace_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(inplace_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kPairSmemBytes);
