@@ -62,7 +62,65 @@ struct Params {
   __nv_bfloat16* Odz;            // dz-tile output [T, d_ff]
   int* counter;
   unsigned* err;
+  // One launch over every chunk of the forward (persistent = 1): tile t belongs to chunk
+  // t / tiles_per_chunk; chunk i reads bf16 copy i (wb_saved) or i & 1 and writes the next one.
+  // done[0][i][b] / done[1][i][b] count the epilogue warps (16 per tile) that finished an update
+  // tile / a row tile of chunk i touching the 256 rows b of M; a tile of chunk i waits for the
+  // counts of chunk i - 1 it depends on.
+  int persistent, nchunk, tiles_per_chunk, n_mblk, wb_saved;
+  int* done;
 };
+
+constexpr int kTileWarps = 16;  // epilogue warps of a CTA pair: completion arrivals per tile
+
+// Chunk context of tile t: the chunk, its first token and the bf16 copies it reads and writes.
+struct TileCtx {
+  int chunk, u, row_base, wb_cur, wb_next;
+};
+__device__ __forceinline__ TileCtx ctx_of(const Params& p, int t) {
+  TileCtx c;
+  if (p.persistent) {
+    c.chunk = t / p.tiles_per_chunk;
+    c.u = t - c.chunk * p.tiles_per_chunk;
+    if (p.wb_saved) {
+      c.wb_cur = c.chunk * p.d_model;
+      c.wb_next = c.chunk + 1 < p.nchunk ? (c.chunk + 1) * p.d_model : -1;
+    } else {
+      c.wb_cur = (c.chunk & 1) * p.d_model;
+      c.wb_next = ((c.chunk + 1) & 1) * p.d_model;
+    }
+  } else {
+    c.chunk = p.chunk;
+    c.u = t;
+    c.wb_cur = p.wb_cur_row0;
+    c.wb_next = p.wb_next_row0;
+  }
+  c.row_base = c.chunk * p.C;
+  return c;
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* a) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
+  return v;
+}
+// Bounded wait until *a >= target (a count other CTAs raise); false on timeout or abort.
+__device__ __forceinline__ bool wait_count(const int* a, int target, const Abort& ab) {
+  if (ld_acquire_gpu(a) >= target) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(a) >= target) return true;
+    if ((it & 15u) == 0) {
+      if (*ab.flag) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *ab.flag = 1;
+        atomicOr(ab.err, ERR_WAIT_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
 
 enum Kind { KIND_ROW = 0, KIND_DZ = 1, KIND_UPD = 2 };
 
@@ -275,7 +333,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync_all();  // both CTAs' barriers initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const int row_base = p.chunk * p.C;  // first token of this chunk
 
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer (both CTAs)
@@ -298,11 +355,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         if (++r == RING) { r = 0; rph ^= 1; }
         if (t >= p.n_total) break;
-        const Tile x = decode<PTM>(p, t);
+        const TileCtx cx = ctx_of(p, t);
+        const Tile x = decode<PTM>(p, cx.u);
+        const int row_base = cx.row_base;
         const int m0 = x.m0 + half, nb = x.n0 + half;  // this CTA's rows of A, columns of B
+        bool ok = true;
+        if (p.persistent && cx.chunk > 0) {
+          // a row tile reads the bf16 rows [n0, n0 + 256) of W that the previous chunk's
+          // update tiles wrote; an update tile rewrites rows [m0, m0 + 256) of W after the
+          // previous chunk's update tiles, and of the bf16 copy the previous chunk's row tiles
+          // read (the copies rotate)
+          const int* done_upd = p.done + (size_t)(cx.chunk - 1) * p.n_mblk;
+          const int* done_row = p.done + ((size_t)p.nchunk + cx.chunk - 1) * p.n_mblk;
+          const int n_tok = p.n_row / p.n_row_n;  // row tiles per 256 rows of W
+          if (x.kind == KIND_ROW)
+            ok = wait_count(done_upd + x.n0 / PTM, kTileWarps * p.n_upd_n, ab);
+          else
+            ok = wait_count(done_upd + x.m0 / PTM, kTileWarps * p.n_upd_n, ab) &&
+                 wait_count(done_row + x.m0 / PTM, kTileWarps * n_tok, ab);
+          // what those tiles stored (generic proxy) is read next by TMA (async proxy)
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+          if (!ok) break;
+        }
         if (x.kind == KIND_UPD && m0 < p.d_model)
           for (int j = 0; j < BN / MBOX; ++j) tma_prefetch_l2_2d(&tm_mf, x.n0 + MBOX * j, m0);
-        bool ok = true;
         for (int kb = 0; kb < x.nkb && ok; ++kb) {
           if (!mbar_wait(PB(empty[s]), sph ^ 1, ab)) { ok = false; break; }
           // both halves of the stage complete on the leader's barrier
@@ -311,14 +387,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t sa = stage0 + s * P_STAGE, sb = sa + PA_BYTES;
           if (x.kind == KIND_ROW) {
             tma_load_2d_pair(sa, &tm_za, fb, kb * BK, row_base + m0);
-            tma_load_2d_pair(sb, &tm_mb, fb, kb * BK, p.wb_cur_row0 + nb);
+            tma_load_2d_pair(sb, &tm_mb, fb, kb * BK, cx.wb_cur + nb);
           } else if (x.kind == KIND_DZ) {
             // K runs over [dO_i | Vhat_i] against [W_i ; eta Wh_{i+1}]
             const bool first = kb < p.kb_dz_split;
             const int k0 = (first ? kb : kb - p.kb_dz_split) * BK;
             tma_load_2d_pair(sa, first ? &tm_do : &tm_vk, fb, k0, row_base + m0);
             const CUtensorMap* mb = first ? &tm_wc : &tm_mbn;
-            const int r0 = (first ? p.wc_row0 : p.wb_cur_row0) + k0;
+            const int r0 = (first ? p.wc_row0 : cx.wb_cur) + k0;
             for (int j = 0; j < 2; ++j) tma_load_2d_pair(sb + 8192 * j, mb, fb, nb + 64 * j, r0);
           } else {
             const int tok = row_base + kb * BK;
@@ -345,7 +421,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_arrive(PB(tile_empty[r]));
         if (++r == RING) { r = 0; rph ^= 1; }
         if (t >= p.n_total) break;
-        const Tile x = decode<PTM>(p, t);
+        const Tile x = decode<PTM>(p, ctx_of(p, t).u);
         // both CTAs' epilogues have drained this accumulator
         if (!mbar_wait_cluster(PB(acc_empty[acc]), aph ^ 1, ab)) break;
         tc_fence_after();
@@ -394,7 +470,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (++r == RING) { r = 0; rph ^= 1; }
       if (t >= p.n_total) break;
-      const Tile x = decode<PTM>(p, t);
+      const TileCtx cx = ctx_of(p, t);
+      const Tile x = decode<PTM>(p, cx.u);
+      const int row_base = cx.row_base;
       const int m0 = x.m0 + half;
       if (!mbar_wait(PB(acc_full[acc]), aph, ab)) break;
       __syncwarp();
@@ -449,7 +527,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const int col = x.n0 + cb * 32 + lane;
           float* mp = p.M + (size_t)mbase * ld + col;
           __nv_bfloat16* bp =
-              p.wb_next_row0 >= 0 ? p.Mb + (size_t)(p.wb_next_row0 + mbase) * ld + col : nullptr;
+              cx.wb_next >= 0 ? p.Mb + (size_t)(cx.wb_next + mbase) * ld + col : nullptr;
 #pragma unroll
           for (int rr = 0; rr < 32; ++rr, mp += ld) {
             const float o = w[rr] + s * xt[rr * 33 + lane];
@@ -482,6 +560,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           mbar_arrive(PB(acc_empty[acc]));
         else
           mbar_arrive_cluster(peer_addr(PB(acc_empty[acc]), 0));
+        if (p.persistent) {
+          // this warp's stores (the whole warp's, ordered by the __syncwarp) before the count
+          __threadfence();
+          const int blk = (x.kind == KIND_UPD ? x.m0 : x.n0) / PTM;
+          atomicAdd(p.done + ((size_t)(x.kind == KIND_UPD ? 0 : p.nchunk) + cx.chunk) * p.n_mblk + blk,
+                    1);
+        }
       }
       if (++acc == 2) { acc = 0; aph ^= 1; }
     }
@@ -832,12 +917,14 @@ void launch_pairs(const Launch& l, const Params& p, cudaStream_t s, const CUtens
 
 }  // namespace
 
-// Two bf16 copies of a d_model x d_ff matrix (read by one launch, written for the next), then
-// one tile counter per chunk; with document resets one float32 d_model x d_ff matrix more (the
+// Two bf16 copies of a d_model x d_ff matrix (read by one chunk, written for the next), then
+// one tile counter per chunk and the persistent forward's completion counts (two per chunk and
+// 256 rows of the matrix); with document resets one float32 d_model x d_ff matrix more (the
 // initial W forward, the running adjoint backward).
 size_t inplace_workspace(int T, int d_ff, int d_model, int C, bool docs) {
   const size_t wb = 2 * (size_t)d_model * d_ff * 2;
-  const size_t counters = ((size_t)(T / C) * sizeof(int) + 255) & ~size_t(255);
+  const size_t nc = (size_t)(T / C), n_mblk = ((size_t)d_model + PTM - 1) / PTM;
+  const size_t counters = ((nc + 2 * nc * n_mblk) * sizeof(int) + 255) & ~size_t(255);
   return wb + counters + (docs ? (size_t)d_model * d_ff * 4 : 0);
 }
 
@@ -865,10 +952,10 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   cudaError_t e = prepare(&l);
   if (e != cudaSuccess) return e;
   to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W, Wb, nW, 1.f);
-  int launches = NC + 1;
   if (reset && (e = cudaMemcpyAsync(W0, W, nW * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
     return e;
-  e = cudaMemsetAsync(counters, 0, NC * sizeof(int), s);
+  const int n_mblk = (d_model + PTM - 1) / PTM;
+  e = cudaMemsetAsync(counters, 0, ((size_t)NC + 2 * (size_t)NC * n_mblk) * sizeof(int), s);
   if (e != cudaSuccess) return e;
   Params p{};
   p.C = C;
@@ -885,6 +972,21 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   p.Mb = Wb;
   p.Orow = static_cast<__nv_bfloat16*>(O);
   p.err = err;
+  if (!reset) {
+    // one launch over all chunks; each tile waits for the previous chunk's tiles it depends on
+    p.persistent = 1;
+    p.nchunk = NC;
+    p.tiles_per_chunk = p.n_total;
+    p.n_total = NC * p.tiles_per_chunk;
+    p.n_mblk = n_mblk;
+    p.wb_saved = W_chunks != nullptr;
+    p.done = counters + NC;
+    p.counter = counters;
+    launch_pairs(l, p, s, tza, tzb, twb, tvh, tza, tza, tzb, tzb, tmf);
+    count_launches(2);
+    return cudaGetLastError();
+  }
+  int launches = NC + 1;
   for (int i = 0; i < NC; ++i) {
     p.chunk = i;
     if (W_chunks) {
