@@ -561,6 +561,11 @@ PROFILE_CASES = {
                 "kernels, then chain, dQ, dK in SiLU mode",
     "ntp-target": "the NTP target and its backward (T=32768, d_model=2560, k=4): the convolution "
                   "kernels and the projection GEMMs",
+    "inplace-fwd": "the In-Place forward (T=32768, d_ff=9728, d_model=2560, C=1024): one "
+                   "persistent launch of the CTA-pair tile kernel over all 32 chunks",
+    "inplace-fwd-8k": "the same forward on the first 8192 tokens (8 chunks), for captures with "
+                      "many passes",
+    "inplace-bwd-8k": "the In-Place backward on the first 8192 tokens (8 chunk launches)",
     "vector-decay": "vector decay forward (tensor cores) and backward (SIMT kernels), B=1, H=4, "
                     "T=512, d=64, C=256",
     "vector-decay-fwd-410m": "the vector-decay forward on the 410M shape (B=8, H=16, T=2048, "
@@ -608,6 +613,27 @@ def run_case(name, ttt):
             ttt.inplace_ttt_target(T, d, k, tin["X0"], tin["conv_w"], tin["W_target"], Vh, ws, n)
             ttt.inplace_ttt_target_bwd(T, d, k, tin["X0"], tin["conv_w"], tin["W_target"],
                                        tin["dVhat"], dX0, dcw, dWt, ws, nb)
+    elif name in ("inplace-fwd", "inplace-fwd-8k", "inplace-bwd-8k"):
+        icfg = synth.INPLACE_QWEN4B
+        if name.endswith("-8k"):
+            icfg = icfg.replace(T=8192)
+        inp = synth.inplace_inputs(icfg, device="cuda")
+        T, F, M, C = icfg.T, icfg.d_ff, icfg.d_model, icfg.C
+        W = inp["W"].clone()
+        O = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+        n = ttt.inplace_ttt_workspace_bytes(T, F, M, C)
+        ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+        bwd = name == "inplace-bwd-8k"
+        Wc = torch.empty((T // C, M, F), device="cuda", dtype=torch.bfloat16) if bwd else None
+        for _ in range(2):
+            W.copy_(inp["W"])
+            ttt.inplace_ttt_fwd(T, F, M, C, icfg.lr, inp["Z"], inp["Vhat"], W, O, ws, n, W_chunks=Wc)
+            if bwd:
+                dZ = torch.empty((T, F), device="cuda", dtype=torch.bfloat16)
+                dV = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+                dW = torch.empty((M, F), device="cuda")
+                ttt.inplace_ttt_bwd(T, F, M, C, icfg.lr, inp["Z"], inp["Vhat"], Wc, inp["dO"], None,
+                                    dZ, dV, dW, ws, n)
     elif name == "vector-decay":
         cfg = synth.FWD_410M.replace(B=1, H=4, T=512, decay="vector")
         layer = Layer(cfg, ttt, seed=cfg.seed)
@@ -776,8 +802,8 @@ def main():
                           "roofline": {"bound": "tensor", "achieved": tf,
                                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                        "frac": tf / peaks["bf16_tflops"],
-                                       "traffic": measured_traffic("inplace_chunk", icfg.name),
-                                       "traffic_unit": "bytes per chunk launch",
+                                       "traffic": measured_traffic("inplace_ttt_fwd", icfg.name),
+                                       "traffic_unit": "bytes per call (one launch)",
                                        "peak_source": peak_src},
                           "ms_saving_chunk_weights": ims_save}
         # backward per token: dZ 4 d_model d_ff (K = 2 d_model), dVhat 2 d_ff d_model and the

@@ -99,6 +99,9 @@ __device__ __forceinline__ TileCtx ctx_of(const Params& p, int t) {
   return c;
 }
 
+__device__ __forceinline__ void red_release_add(int* a) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(a) : "memory");
+}
 __device__ __forceinline__ int ld_acquire_gpu(const int* a) {
   int v;
   asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(a) : "memory");
@@ -561,11 +564,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         else
           mbar_arrive_cluster(peer_addr(PB(acc_empty[acc]), 0));
         if (p.persistent) {
-          // this warp's stores (the whole warp's, ordered by the __syncwarp) before the count
-          __threadfence();
+          // the count is raised with release semantics after this warp's stores (the whole
+          // warp's, ordered before this thread's by the __syncwarp)
           const int blk = (x.kind == KIND_UPD ? x.m0 : x.n0) / PTM;
-          atomicAdd(p.done + ((size_t)(x.kind == KIND_UPD ? 0 : p.nchunk) + cx.chunk) * p.n_mblk + blk,
-                    1);
+          red_release_add(p.done + ((size_t)(x.kind == KIND_UPD ? 0 : p.nchunk) + cx.chunk) *
+                                       p.n_mblk + blk);
         }
       }
       if (++acc == 2) { acc = 0; aph ^= 1; }
