@@ -29,7 +29,8 @@
 // Warp roles in each CTA: warp 0 issues TMA loads into a 6-stage ring, warp 1 of the leader CTA
 // (rank 0) issues the pair MMAs into two TMEM accumulators of 128 x 256 fp32 per CTA, warps 2-9
 // drain this CTA's accumulator rows (two warps per TMEM lane quadrant, each taking 128 of the
-// 256 columns). The leader takes tiles from the queue and hands each index to its peer through
+// 256 columns), warp 10 publishes each finished tile to the tiles of the next chunk that depend
+// on it (the persistent forward). The leader takes tiles from the queue and hands each index to its peer through
 // distributed shared memory; both CTAs' loads (no multicast) complete on the leader's stage
 // barrier; the MMA commits arrive on the stage and accumulator barriers of both CTAs; the peer
 // signals the leader's accumulator-free and tile-free barriers remotely. Every wait is bounded.
@@ -42,7 +43,7 @@ namespace tttk {
 namespace {
 
 constexpr int BM = 128, BN = 256, BK = 64, RING = 4;  // BM: rows of one CTA's half tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;  // producer, MMA, 8 epilogue warps, completion signaller
 constexpr int kEpiWarps = 8;
 constexpr int kXpose = 32 * 33;  // floats of one epilogue warp's padded 32 x 32 transpose tile
 constexpr uint32_t kTmemCols = 512;            // two 256-column accumulators
@@ -71,7 +72,7 @@ struct Params {
   int* done;
 };
 
-constexpr int kTileWarps = 16;  // epilogue warps of a CTA pair: completion arrivals per tile
+constexpr int kTileWarps = 2;  // completion arrivals per pair tile (one per CTA)
 
 // Chunk context of tile t: the chunk, its first token and the bf16 copies it reads and writes.
 struct TileCtx {
@@ -173,12 +174,12 @@ constexpr int P_STAGES = 6;
 constexpr uint32_t PA_BYTES = BM * BK * 2;      // 16 KB: this CTA's 128 rows of A
 constexpr uint32_t PB_BYTES = (BN / 2) * BK * 2;  // 16 KB: this CTA's 128 columns of B
 constexpr uint32_t P_STAGE = PA_BYTES + PB_BYTES;
-constexpr int kPairTileReaders = 2 * (1 + kEpiWarps);  // leader MMA + epilogue, peer producer +
-                                                       // epilogue
+constexpr int kPairTileReaders = 2 * (2 + kEpiWarps);  // leader MMA, peer producer, and in each
+                                                       // CTA the epilogue and the signaller
 
 struct __align__(8) PairBars {
   uint64_t full[P_STAGES], empty[P_STAGES], acc_full[2], acc_empty[2], tile_full[RING],
-      tile_empty[RING];
+      tile_empty[RING], tile_done[2];
   int ring[RING];
   uint32_t tmem_base;
   int abort_flag;
@@ -309,6 +310,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(PB(acc_full[a]), 1);
       mbar_init(PB(acc_empty[a]), 2 * kEpiWarps);
+      mbar_init(PB(tile_done[a]), kEpiWarps);
     }
     for (int r = 0; r < RING; ++r) {
       mbar_init(PB(tile_full[r]), 1);
@@ -452,6 +454,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (++acc == 2) { acc = 0; aph ^= 1; }
       }
     }
+  } else if (warp == 2 + kEpiWarps) {
+    // ------------------------------------------ completion signaller (both CTAs, one thread)
+    // After the eight epilogue warps of this CTA have stored a tile (tile_done), raise the
+    // tile's completion count with release semantics at GPU scope; the epilogue warps never wait
+    // for their stores to become visible.
+    if (lane == 0) {
+      int r = 0, acc = 0;
+      uint32_t rph = 0, aph = 0;
+      for (;;) {
+        if (!mbar_wait_cluster(PB(tile_full[r]), rph, ab)) break;
+        const int t = bars->ring[r];
+        if (leader)
+          mbar_arrive(PB(tile_empty[r]));
+        else
+          mbar_arrive_cluster(peer_addr(PB(tile_empty[r]), 0));
+        if (++r == RING) { r = 0; rph ^= 1; }
+        if (t >= p.n_total) break;
+        const TileCtx cx = ctx_of(p, t);
+        const Tile x = decode<PTM>(p, cx.u);
+        if (!mbar_wait(PB(tile_done[acc]), aph, ab)) break;
+        if (p.persistent) {
+          const int blk = (x.kind == KIND_UPD ? x.m0 : x.n0) / PTM;
+          red_release_add(p.done + ((size_t)(x.kind == KIND_UPD ? 0 : p.nchunk) + cx.chunk) *
+                                       p.n_mblk + blk);
+        }
+        if (++acc == 2) { acc = 0; aph ^= 1; }
+      }
+    }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     // Warp w drains TMEM lanes 32*(w%4) .. +31 (thread = one row of this CTA's half) and
@@ -563,13 +593,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           mbar_arrive(PB(acc_empty[acc]));
         else
           mbar_arrive_cluster(peer_addr(PB(acc_empty[acc]), 0));
-        if (p.persistent) {
-          // the count is raised with release semantics after this warp's stores (the whole
-          // warp's, ordered before this thread's by the __syncwarp)
-          const int blk = (x.kind == KIND_UPD ? x.m0 : x.n0) / PTM;
-          red_release_add(p.done + ((size_t)(x.kind == KIND_UPD ? 0 : p.nchunk) + cx.chunk) *
-                                       p.n_mblk + blk);
-        }
+        // this warp's stores of the tile (the whole warp's, ordered before this thread's by the
+        // __syncwarp) are done: the signaller publishes them with the tile's completion count
+        mbar_arrive(PB(tile_done[acc]));
       }
       if (++acc == 2) { acc = 0; aph ^= 1; }
     }
