@@ -47,6 +47,8 @@ SMALL = [
     (384, 320, 384, 128, 0.05),    # ragged N tiles on both GEMMs
     (1024, 512, 128, 256, 0.02),
     (128, 64, 128, 128, 0.1),      # one chunk: a plain GEMM
+    (4096, 512, 256, 128, 0.05),   # 32 chunks: the forward's cross-chunk dependency counts
+    (2048, 448, 640, 256, 0.05),   # 8 chunks, d_model = 2.5 pair tiles: a half-empty pair tile
 ]
 
 
