@@ -26,11 +26,14 @@
 // Long tiles (row, then dz) are handed out first, update tiles fill the remaining SMs. When
 // a CTA takes an update tile it prefetches its float32 block of M into L2, so the epilogue's
 // read-modify-write, issued after the tile's K steps, reads from L2.
+// Without document resets the forward and the backward are each ONE persistent launch over all
+// chunks, a tile waiting (bounded) for the tiles of the previously processed chunk it depends
+// on, through per-block completion counts in the workspace.
 // Warp roles in each CTA: warp 0 issues TMA loads into a 6-stage ring, warp 1 of the leader CTA
 // (rank 0) issues the pair MMAs into two TMEM accumulators of 128 x 256 fp32 per CTA, warps 2-9
 // drain this CTA's accumulator rows (two warps per TMEM lane quadrant, each taking 128 of the
 // 256 columns), warp 10 publishes each finished tile to the tiles of the next chunk that depend
-// on it (the persistent forward). The leader takes tiles from the queue and hands each index to its peer through
+// on it. The leader takes tiles from the queue and hands each index to its peer through
 // distributed shared memory; both CTAs' loads (no multicast) complete on the leader's stage
 // barrier; the MMA commits arrive on the stage and accumulator barriers of both CTAs; the peer
 // signals the leader's accumulator-free and tile-free barriers remotely. Every wait is bounded.
@@ -63,24 +66,48 @@ struct Params {
   __nv_bfloat16* Odz;            // dz-tile output [T, d_ff]
   int* counter;
   unsigned* err;
-  // One launch over every chunk of the forward (persistent = 1): tile t belongs to chunk
-  // t / tiles_per_chunk; chunk i reads bf16 copy i (wb_saved) or i & 1 and writes the next one.
-  // done[0][i][b] / done[1][i][b] count the epilogue warps (16 per tile) that finished an update
-  // tile / a row tile of chunk i touching the 256 rows b of M; a tile of chunk i waits for the
-  // counts of chunk i - 1 it depends on.
-  int persistent, nchunk, tiles_per_chunk, n_mblk, wb_saved;
+  // One launch over every chunk: persistent = 1 the forward (tile t belongs to chunk
+  // t / tiles_per_chunk, which reads bf16 copy i (wb_saved) or i & 1 and writes the next one),
+  // persistent = 2 the backward (chunk NC - 1 - t / tiles_per_chunk, reading copy i & 1 and
+  // writing (i - 1) & 1, its dz tiles the saved W_i). Completion counts (kTileWarps per tile),
+  // per chunk i and 256-wide block: done + UR: update tiles by row block of M; + RD: row tiles
+  // by their block of M's rows; + UC: update tiles by column block (backward); + DZ: dz tiles by
+  // column block (backward). A tile waits for the counts of the chunk processed before it.
+  int persistent, nchunk, tiles_per_chunk, n_mblk, n_nblk, wb_saved, upd_col_major;
   int* done;
 };
+
+// Offsets of the completion-count arrays in Params::done.
+__host__ __device__ __forceinline__ size_t done_ur(const Params& p, int i) {
+  return (size_t)i * p.n_mblk;
+}
+__host__ __device__ __forceinline__ size_t done_rd(const Params& p, int i) {
+  return ((size_t)p.nchunk + i) * p.n_mblk;
+}
+__host__ __device__ __forceinline__ size_t done_uc(const Params& p, int i) {
+  return 2 * (size_t)p.nchunk * p.n_mblk + (size_t)i * p.n_nblk;
+}
+__host__ __device__ __forceinline__ size_t done_dz(const Params& p, int i) {
+  return 2 * (size_t)p.nchunk * p.n_mblk + ((size_t)p.nchunk + i) * p.n_nblk;
+}
 
 constexpr int kTileWarps = 2;  // completion arrivals per pair tile (one per CTA)
 
 // Chunk context of tile t: the chunk, its first token and the bf16 copies it reads and writes.
 struct TileCtx {
-  int chunk, u, row_base, wb_cur, wb_next;
+  int chunk, u, row_base, wb_cur, wb_next, wc;
 };
 __device__ __forceinline__ TileCtx ctx_of(const Params& p, int t) {
   TileCtx c;
-  if (p.persistent) {
+  c.wc = p.wc_row0;
+  if (p.persistent == 2) {
+    const int k = t / p.tiles_per_chunk;
+    c.chunk = p.nchunk - 1 - k;
+    c.u = t - k * p.tiles_per_chunk;
+    c.wb_cur = (c.chunk & 1) * p.d_model;
+    c.wb_next = c.chunk > 0 ? ((c.chunk - 1) & 1) * p.d_model : -1;
+    c.wc = c.chunk * p.d_model;
+  } else if (p.persistent) {
     c.chunk = t / p.tiles_per_chunk;
     c.u = t - c.chunk * p.tiles_per_chunk;
     if (p.wb_saved) {
@@ -160,8 +187,16 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
   } else {
     const int u = t - p.n_row - p.n_dz;
     x.kind = KIND_UPD;
-    x.m0 = (u / p.n_upd_n) * TM;  // d_model row
-    x.n0 = (u % p.n_upd_n) * BN;  // d_ff column
+    if (p.upd_col_major) {
+      // the backward: the column blocks of the adjoint copy complete one after another, which
+      // is the order the next chunk's dz tiles need them in
+      const int n_m = (p.d_model + TM - 1) / TM;
+      x.m0 = (u % n_m) * TM;
+      x.n0 = (u / n_m) * BN;
+    } else {
+      x.m0 = (u / p.n_upd_n) * TM;  // d_model row
+      x.n0 = (u % p.n_upd_n) * BN;  // d_ff column
+    }
     x.nkb = p.kb_upd;
   }
   return x;
@@ -365,19 +400,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int row_base = cx.row_base;
         const int m0 = x.m0 + half, nb = x.n0 + half;  // this CTA's rows of A, columns of B
         bool ok = true;
-        if (p.persistent && cx.chunk > 0) {
-          // a row tile reads the bf16 rows [n0, n0 + 256) of W that the previous chunk's
-          // update tiles wrote; an update tile rewrites rows [m0, m0 + 256) of W after the
-          // previous chunk's update tiles, and of the bf16 copy the previous chunk's row tiles
-          // read (the copies rotate)
-          const int* done_upd = p.done + (size_t)(cx.chunk - 1) * p.n_mblk;
-          const int* done_row = p.done + ((size_t)p.nchunk + cx.chunk - 1) * p.n_mblk;
-          const int n_tok = p.n_row / p.n_row_n;  // row tiles per 256 rows of W
-          if (x.kind == KIND_ROW)
-            ok = wait_count(done_upd + x.n0 / PTM, kTileWarps * p.n_upd_n, ab);
-          else
-            ok = wait_count(done_upd + x.m0 / PTM, kTileWarps * p.n_upd_n, ab) &&
-                 wait_count(done_row + x.m0 / PTM, kTileWarps * n_tok, ab);
+        // the chunk processed just before this one (forward: i - 1, backward: i + 1)
+        const int prev = p.persistent == 2 ? cx.chunk + 1 : cx.chunk - 1;
+        if (p.persistent && prev >= 0 && prev < p.nchunk) {
+          const int n_tok = p.n_row / p.n_row_n;        // row (and dz) tiles per column block
+          const int n_m = (p.d_model + PTM - 1) / PTM;  // update tiles per column block
+          const int* d = p.done;
+          if (p.persistent == 1) {
+            // forward: a row tile reads the bf16 rows [n0, n0 + 256) of W that the previous
+            // chunk's update tiles wrote; an update tile rewrites rows [m0, m0 + 256) of W after
+            // the previous chunk's update tiles, and of the bf16 copy the previous chunk's row
+            // tiles read (the copies rotate)
+            if (x.kind == KIND_ROW)
+              ok = wait_count(d + done_ur(p, prev) + x.n0 / PTM, kTileWarps * p.n_upd_n, ab);
+            else
+              ok = wait_count(d + done_ur(p, prev) + x.m0 / PTM, kTileWarps * p.n_upd_n, ab) &&
+                   wait_count(d + done_rd(p, prev) + x.m0 / PTM, kTileWarps * n_tok, ab);
+          } else {
+            // backward: a row tile reads rows [n0, n0 + 256) of the adjoint copy, a dz tile
+            // every row of its columns [n0, n0 + 256), both written by the previous chunk's
+            // update tiles; an update tile rewrites its block of the adjoint after the previous
+            // chunk's update tiles of those rows, and of the copy the previous chunk's row tiles
+            // (its rows) and dz tiles (its columns) read
+            if (x.kind == KIND_ROW)
+              ok = wait_count(d + done_ur(p, prev) + x.n0 / PTM, kTileWarps * p.n_upd_n, ab);
+            else if (x.kind == KIND_DZ)
+              ok = wait_count(d + done_uc(p, prev) + x.n0 / BN, kTileWarps * n_m, ab);
+            else
+              ok = wait_count(d + done_ur(p, prev) + x.m0 / PTM, kTileWarps * p.n_upd_n, ab) &&
+                   wait_count(d + done_rd(p, prev) + x.m0 / PTM, kTileWarps * n_tok, ab) &&
+                   wait_count(d + done_dz(p, prev) + x.n0 / BN, kTileWarps * n_tok, ab);
+          }
           // what those tiles stored (generic proxy) is read next by TMA (async proxy)
           asm volatile("fence.proxy.async.global;" ::: "memory");
           if (!ok) break;
@@ -399,7 +452,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const int k0 = (first ? kb : kb - p.kb_dz_split) * BK;
             tma_load_2d_pair(sa, first ? &tm_do : &tm_vk, fb, k0, row_base + m0);
             const CUtensorMap* mb = first ? &tm_wc : &tm_mbn;
-            const int r0 = (first ? p.wc_row0 : cx.wb_cur) + k0;
+            const int r0 = (first ? cx.wc : cx.wb_cur) + k0;
             for (int j = 0; j < 2; ++j) tma_load_2d_pair(sb + 8192 * j, mb, fb, nb + 64 * j, r0);
           } else {
             const int tok = row_base + kb * BK;
@@ -475,9 +528,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const Tile x = decode<PTM>(p, cx.u);
         if (!mbar_wait(PB(tile_done[acc]), aph, ab)) break;
         if (p.persistent) {
-          const int blk = (x.kind == KIND_UPD ? x.m0 : x.n0) / PTM;
-          red_release_add(p.done + ((size_t)(x.kind == KIND_UPD ? 0 : p.nchunk) + cx.chunk) *
-                                       p.n_mblk + blk);
+          int* d = p.done;
+          if (x.kind == KIND_UPD) {
+            red_release_add(d + done_ur(p, cx.chunk) + x.m0 / PTM);
+            if (p.persistent == 2) red_release_add(d + done_uc(p, cx.chunk) + x.n0 / BN);
+          } else if (x.kind == KIND_ROW) {
+            red_release_add(d + done_rd(p, cx.chunk) + x.n0 / PTM);
+          } else {
+            red_release_add(d + done_dz(p, cx.chunk) + x.n0 / BN);
+          }
         }
         if (++acc == 2) { acc = 0; aph ^= 1; }
       }
@@ -947,13 +1006,14 @@ void launch_pairs(const Launch& l, const Params& p, cudaStream_t s, const CUtens
 }  // namespace
 
 // Two bf16 copies of a d_model x d_ff matrix (read by one chunk, written for the next), then
-// one tile counter per chunk and the persistent forward's completion counts (two per chunk and
-// 256 rows of the matrix); with document resets one float32 d_model x d_ff matrix more (the
-// initial W forward, the running adjoint backward).
+// one tile counter per chunk and the persistent launches' completion counts (two per chunk and
+// 256 rows of the matrix, two per chunk and 256 of its columns); with document resets one
+// float32 d_model x d_ff matrix more (the initial W forward, the running adjoint backward).
 size_t inplace_workspace(int T, int d_ff, int d_model, int C, bool docs) {
   const size_t wb = 2 * (size_t)d_model * d_ff * 2;
-  const size_t nc = (size_t)(T / C), n_mblk = ((size_t)d_model + PTM - 1) / PTM;
-  const size_t counters = ((nc + 2 * nc * n_mblk) * sizeof(int) + 255) & ~size_t(255);
+  const size_t nc = (size_t)(T / C), n_mblk = ((size_t)d_model + PTM - 1) / PTM,
+               n_nblk = ((size_t)d_ff + BN - 1) / BN;
+  const size_t counters = ((nc + 2 * nc * (n_mblk + n_nblk)) * sizeof(int) + 255) & ~size_t(255);
   return wb + counters + (docs ? (size_t)d_model * d_ff * 4 : 0);
 }
 
@@ -983,8 +1043,9 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W, Wb, nW, 1.f);
   if (reset && (e = cudaMemcpyAsync(W0, W, nW * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
     return e;
-  const int n_mblk = (d_model + PTM - 1) / PTM;
-  e = cudaMemsetAsync(counters, 0, ((size_t)NC + 2 * (size_t)NC * n_mblk) * sizeof(int), s);
+  const int n_mblk = (d_model + PTM - 1) / PTM, n_nblk = (d_ff + BN - 1) / BN;
+  e = cudaMemsetAsync(counters, 0, ((size_t)NC + 2 * (size_t)NC * (n_mblk + n_nblk)) * sizeof(int),
+                      s);
   if (e != cudaSuccess) return e;
   Params p{};
   p.C = C;
@@ -1008,6 +1069,7 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
     p.tiles_per_chunk = p.n_total;
     p.n_total = NC * p.tiles_per_chunk;
     p.n_mblk = n_mblk;
+    p.n_nblk = n_nblk;
     p.wb_saved = W_chunks != nullptr;
     p.done = counters + NC;
     p.counter = counters;
@@ -1079,7 +1141,9 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
       return e;
   }
   if (reset && (e = cudaMemsetAsync(dW, 0, nW * sizeof(float), s)) != cudaSuccess) return e;
-  e = cudaMemsetAsync(counters, 0, NC * sizeof(int), s);
+  const int n_mblk = (d_model + PTM - 1) / PTM, n_nblk = (d_ff + BN - 1) / BN;
+  e = cudaMemsetAsync(counters, 0, ((size_t)NC + 2 * (size_t)NC * (n_mblk + n_nblk)) * sizeof(int),
+                      s);
   if (e != cudaSuccess) return e;
   Params p{};
   p.C = C;
@@ -1100,6 +1164,22 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   p.Orow = static_cast<__nv_bfloat16*>(dVhat);
   p.Odz = static_cast<__nv_bfloat16*>(dZ);
   p.err = err;
+  if (!reset) {
+    // one launch over all chunks, from the last one; each tile waits for the tiles of the chunk
+    // after it that it depends on
+    p.persistent = 2;
+    p.upd_col_major = 1;
+    p.nchunk = NC;
+    p.tiles_per_chunk = p.n_total;
+    p.n_total = NC * p.tiles_per_chunk;
+    p.n_mblk = n_mblk;
+    p.n_nblk = n_nblk;
+    p.done = counters + NC;
+    p.counter = counters;
+    launch_pairs(l, p, s, tza, tzb, tmb, tdx, tdo, tvk, twc, tmbn, tmf);
+    count_launches(dW_final ? 2 : 1);
+    return cudaGetLastError();
+  }
   for (int i = NC - 1; i >= 0; --i) {
     p.chunk = i;
     p.wb_cur_row0 = (i & 1) * d_model;
