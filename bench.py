@@ -565,7 +565,8 @@ PROFILE_CASES = {
                    "persistent launch of the CTA-pair tile kernel over all 32 chunks",
     "inplace-fwd-8k": "the same forward on the first 8192 tokens (8 chunks), for captures with "
                       "many passes",
-    "inplace-bwd-8k": "the In-Place backward on the first 8192 tokens (8 chunk launches)",
+    "inplace-bwd-8k": "the In-Place forward and backward on the first 8192 tokens (8 chunks, one "
+                      "persistent launch each)",
     "vector-decay": "vector decay forward (tensor cores) and backward (SIMT kernels), B=1, H=4, "
                     "T=512, d=64, C=256",
     "vector-decay-fwd-410m": "the vector-decay forward on the 410M shape (B=8, H=16, T=2048, "
