@@ -559,6 +559,10 @@ PROFILE_CASES = {
                      "kernel, then chain, dQ, dK",
     "silu-bwd": "SiLU + MSE forward and backward (B=2, H=16, T=2048): the dZq and SiLU-factor "
                 "kernels, then chain, dQ, dK in SiLU mode",
+    "fwd-410m": "the 410M-shaped inference forward (B=8, H=16, T=2048, d=64, C=256): the "
+                "tensor-core forward kernel at d = 64",
+    "silu-ip-fwd": "the single-SiLU, inner-product inference forward (B=4, H=16, T=4096, d=128, "
+                   "C=256): the tensor-core forward kernel in SiLU mode",
     "ntp-target": "the NTP target and its backward (T=32768, d_model=2560, k=4): the convolution "
                   "kernels and the projection GEMMs",
     "inplace-fwd": "the In-Place forward (T=32768, d_ff=9728, d_model=2560, C=1024): one "
@@ -599,6 +603,11 @@ def run_case(name, ttt):
                                   layer.ws.numel())
             else:
                 layer.bwd()
+    elif name in ("fwd-410m", "silu-ip-fwd"):
+        cfg = synth.FWD_410M if name == "fwd-410m" else synth.SILU_IP_FWD
+        layer = Layer(cfg, ttt, seed=cfg.seed)
+        for _ in range(2):
+            layer.fwd(save=False)
     elif name == "ntp-target":
         icfg, k = synth.INPLACE_QWEN4B, 4
         tin = synth.inplace_target_inputs(icfg, k, device="cuda")
