@@ -1661,9 +1661,13 @@ __global__ void __launch_bounds__(kPrepThreads) vec_dgamma_kernel(const DgParams
   const size_t r0 = bc * C + seg * SEG;
   const float4* dq = reinterpret_cast<const float4*>(p.dLq + r0 * VD) + fq;
   const float4* dk = reinterpret_cast<const float4*>(p.dLk + r0 * VD) + fq;
-  float4 d[SEG];
+  // every load of the thread (its slice of dLq, dLk and gamma) in flight before any arithmetic
+  const float4* g = reinterpret_cast<const float4*>(p.gamma + r0 * VD) + fq;
+  float4 d[SEG], gv[SEG];
 #pragma unroll
   for (int t = 0; t < SEG; ++t) d[t] = add4(__ldg(dq + t * (VD / 4)), __ldg(dk + t * (VD / 4)));
+#pragma unroll
+  for (int t = 0; t < SEG; ++t) gv[t] = __ldg(g + t * (VD / 4));
   float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int t = 0; t < SEG; ++t) s = add4(s, d[t]);
@@ -1684,15 +1688,12 @@ __global__ void __launch_bounds__(kPrepThreads) vec_dgamma_kernel(const DgParams
 #pragma unroll
   for (int k = kPrepSeg - 1; k >= 0; --k)
     if (k > seg) acc = add4(acc, tot[k][f]);
-  const float4* g = reinterpret_cast<const float4*>(p.gamma + r0 * VD) + fq;
-  float4 gv[SEG];
-#pragma unroll
-  for (int t = 0; t < SEG; ++t) gv[t] = __ldg(g + t * (VD / 4));
   float4* out = reinterpret_cast<float4*>(p.dgamma + r0 * VD) + fq;
 #pragma unroll
   for (int t = SEG - 1; t >= 0; --t) {
     acc = add4(acc, d[t]);
-    out[t * (VD / 4)] = make_float4(acc.x / gv[t].x, acc.y / gv[t].y, acc.z / gv[t].z, acc.w / gv[t].w);
+    out[t * (VD / 4)] = make_float4(__fdividef(acc.x, gv[t].x), __fdividef(acc.y, gv[t].y),
+                                    __fdividef(acc.z, gv[t].z), __fdividef(acc.w, gv[t].w));
   }
 }
 
