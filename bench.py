@@ -87,7 +87,11 @@ def layer_work(cfg):
     by_f = tok * (2 * dk + dv) * e + tok * bg + 2 * B * H * dk * dv * 4 + tok * dv * e
     by_b = (tok * (2 * dk + 2 * dv) * e + tok * bg + B * H * dk * dv * 4
             + tok * (2 * dk + dv) * e + tok * 4 + B * H * dk * dv * 4)
-    return dict(fwd_flops=fl_f, bwd_flops=fl_b, fwd_bytes=by_f, bwd_bytes=by_b)
+    # secondary count: the C x C products taken dense (no causal halving)
+    dense = units * (6 * C * dk * dv + 2 * C * C * (dk + dv)) + \
+        units * (12 * C * dk * dv + 4 * C * C * (dk + dv))
+    return dict(fwd_flops=fl_f, bwd_flops=fl_b, fwd_bytes=by_f, bwd_bytes=by_b,
+                step_flops_dense=dense)
 
 
 def inplace_work(icfg):
@@ -778,6 +782,10 @@ def main():
                 "peak_source": peak_src}
     step_flops = work["fwd_flops"] + work["bwd_flops"]
     tc_frac = step_flops / (ms_step * 1e-3) / (peaks["bf16_tflops"] * 1e12)
+    # secondary: the step against HBM (algorithmic bytes of both calls), and the tensor-core
+    # fraction with the C x C products counted dense
+    hbm_step = (work["fwd_bytes"] + work["bwd_bytes"]) / (ms_step * 1e-3) / (peaks["hbm_gbs"] * 1e9)
+    tc_dense = work["step_flops_dense"] / (ms_step * 1e-3) / (peaks["bf16_tflops"] * 1e12)
 
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -785,6 +793,7 @@ def main():
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": config, "roofline": roofline,
         "tc_frac_of_bf16_peak": tc_frac,
+        "secondary": {"hbm_frac_of_step": hbm_step, "tc_frac_dense_count": tc_dense},
         "kernels_ms": {"ttt_chunk_fwd": fwd_ms, "ttt_chunk_bwd": bwd_ms},
         "gpu_launches": launches, "clocks": clocks,
     }
