@@ -24,6 +24,7 @@ namespace tttk {
 namespace {
 
 constexpr int kNvs = 32;        // value columns per forward block
+constexpr int kNvsNarrow = 8;   // ... when the grid would be small (few heads): 4x the blocks
 constexpr int kRows = 32;       // query rows per score tile in the forward
 constexpr int kMaxC = 256;
 constexpr int kMaxD = 128;
@@ -53,12 +54,31 @@ __device__ void chunk_scans(const Dims& d, const float* beta, const float* gamma
   for (int e = threadIdx.x; e < d.C * w; e += blockDim.x)
     L[e] = d.has_gamma ? logf(gamma[t0 * w + e]) : 0.f;
   __syncthreads();
-  for (int i = threadIdx.x; i < w; i += blockDim.x)
-    for (int s = 1; s < d.C; ++s) L[s * w + i] += L[(s - 1) * w + i];
+  if (w == 1) {
+    // scalar decay: one warp, each lane a run of C / 32 positions, then a shuffle scan
+    if (threadIdx.x < 32) {
+      const int lane = threadIdx.x, per = (d.C + 31) / 32, s0 = lane * per;
+      float run = 0.f;
+      for (int s = s0; s < min(s0 + per, d.C); ++s) run += L[s];
+      float incl = run;
+      for (int off = 1; off < 32; off <<= 1) {
+        const float o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      float acc = incl - run;  // sum of the runs before this lane's
+      for (int s = s0; s < min(s0 + per, d.C); ++s) {
+        acc += L[s];
+        L[s] = acc;
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < w; i += blockDim.x)
+      for (int s = 1; s < d.C; ++s) L[s * w + i] += L[(s - 1) * w + i];
+  }
   __syncthreads();
 }
 
-template <typename TI>
+template <typename TI, int kNvs>
 __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, const TI* K,
                                                        const TI* V, const float* beta,
                                                        const float* gamma, const float* W0,
@@ -469,10 +489,17 @@ Dims dims_of(const LayerArgs& a) {
 // Elements of one [B, H, T, dv] plane: with SiLU, Zq follows G in the saved buffer.
 size_t zq_plane(const LayerArgs& a) { return (size_t)a.B * a.H * a.T * a.dv; }
 
-size_t fwd_smem_bytes(const LayerArgs& a) {
+size_t fwd_smem_bytes(const LayerArgs& a, int nvs = kNvs) {
   const size_t lw = a.gvec ? a.dk : 1;
-  return sizeof(float) * ((size_t)a.dk * kNvs + (size_t)a.C * kNvs + (size_t)kRows * a.C + a.C +
+  return sizeof(float) * ((size_t)a.dk * nvs + (size_t)a.C * nvs + (size_t)kRows * a.C + a.C +
                            a.C * lw + a.C + 1 + a.dk);
+}
+
+// Value columns per forward block: narrower slices when the wide ones would leave most SMs idle
+// (each block recomputes the chunk's scores, so narrow slices trade that for parallelism).
+int fwd_nvs(const LayerArgs& a) {
+  const long blocks = (long)((a.dv + kNvs - 1) / kNvs) * a.B * a.H;
+  return blocks < 64 ? kNvsNarrow : kNvs;
 }
 
 }  // namespace
@@ -487,19 +514,19 @@ size_t simt_bwd_workspace(const LayerArgs& a) {
   return sizeof(float) * bwd_head_floats(a.C, a.dk, a.dv, a.gvec) * a.B * a.H;
 }
 
-cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
-  const Dims d = dims_of(a);
-  const size_t smem = fwd_smem_bytes(a);
-  dim3 grid((a.dv + kNvs - 1) / kNvs, a.B * a.H);
+template <int NVS>
+void simt_fwd_launch(const LayerArgs& a, const Dims& d, cudaStream_t s) {
+  const size_t smem = fwd_smem_bytes(a, NVS);
+  dim3 grid((a.dv + NVS - 1) / NVS, a.B * a.H);
   if (a.dtype == 0) {
-    auto k = simt_fwd_kernel<float>;
+    auto k = simt_fwd_kernel<float, NVS>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     float* gs = (float*)a.G_saved;
     k<<<grid, 256, smem, s>>>(d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta,
                               a.gamma, a.W0, (float*)a.O, a.W_final, (float*)a.W_chunks, gs,
                               gs && a.act ? gs + zq_plane(a) : nullptr);
   } else {
-    auto k = simt_fwd_kernel<__nv_bfloat16>;
+    auto k = simt_fwd_kernel<__nv_bfloat16, NVS>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     __nv_bfloat16* gs = (__nv_bfloat16*)a.G_saved;
     k<<<grid, 256, smem, s>>>(d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K,
@@ -507,6 +534,14 @@ cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
                               (__nv_bfloat16*)a.O, a.W_final, (__nv_bfloat16*)a.W_chunks, gs,
                               gs && a.act ? gs + zq_plane(a) : nullptr);
   }
+}
+
+cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
+  const Dims d = dims_of(a);
+  if (fwd_nvs(a) == kNvsNarrow)
+    simt_fwd_launch<kNvsNarrow>(a, d, s);
+  else
+    simt_fwd_launch<kNvs>(a, d, s);
   count_launches(1);
   return cudaGetLastError();
 }
