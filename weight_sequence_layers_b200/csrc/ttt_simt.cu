@@ -78,7 +78,9 @@ __device__ void chunk_scans(const Dims& d, const float* beta, const float* gamma
   __syncthreads();
 }
 
-template <typename TI, int kNvs>
+// STG: the chunk's keys and queries are staged in shared memory (float32, rows padded to dk + 1
+// so that the column walks of the element loops do not collide in one bank).
+template <typename TI, int kNvs, bool STG>
 __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, const TI* K,
                                                        const TI* V, const float* beta,
                                                        const float* gamma, const float* W0,
@@ -94,6 +96,9 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
   float* eta = S + kRows * C;        // [C]
   float* L = eta + C;                // [C] or [C][dk]
   float* X = L + C * lwidth(d);      // [C + dk]: per-key factors of the transition
+  const int ldk = dk + 1;
+  float* Ks = X + C + dk;            // [C][dk + 1] (STG)
+  float* Qs = Ks + C * ldk;          // [C][dk + 1] (STG)
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
   for (int e = threadIdx.x; e < dk * nv; e += blockDim.x) {
     const int i = e / nv, j = e % nv;
@@ -106,14 +111,28 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
         const int i = e / nv, j = e % nv;
         stf(&Wc[(((size_t)bh * NC + c) * dk + i) * dv + j0 + j], Ws[i * kNvs + j]);
       }
-    chunk_scans(d, beta, gamma, bh, c, eta, L);
     const size_t tc = (size_t)c * C;
+    if constexpr (STG)
+      for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
+        const int s = e / dk, i = e % dk;
+        Ks[s * ldk + i] = ldf(K + qk0 + (tc + s) * dk + i);
+        Qs[s * ldk + i] = ldf(Q + qk0 + (tc + s) * dk + i);
+      }
+    // key r / query s of the chunk, feature i
+    auto kat = [&](int r, int i) -> float {
+      if constexpr (STG) return Ks[r * ldk + i];
+      else return ldf(K + qk0 + (tc + r) * dk + i);
+    };
+    auto qat = [&](int s, int i) -> float {
+      if constexpr (STG) return Qs[s * ldk + i];
+      else return ldf(Q + qk0 + (tc + s) * dk + i);
+    };
+    chunk_scans(d, beta, gamma, bh, c, eta, L);  // ends with a block barrier
     // train view: G = a(Z) * act'(Z), Z = K W0
     for (int e = threadIdx.x; e < C * nv; e += blockDim.x) {
       const int s = e / nv, j = e % nv;
-      const TI* kr = K + qk0 + (tc + s) * dk;
       float z = 0.f;
-      for (int i = 0; i < dk; ++i) z += ldf(kr + i) * Ws[i * kNvs + j];
+      for (int i = 0; i < dk; ++i) z += kat(s, i) * Ws[i * kNvs + j];
       const float vv = ldf(V + v0 + (tc + s) * dv + j0 + j);
       const float a = d.loss == 0 ? actf(d.act, z) - vv : -vv;
       G[s * kNvs + j] = a * act1(d.act, z);
@@ -122,6 +141,43 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
     __syncthreads();
     // query view, kRows queries at a time
     for (int s0 = 0; s0 < C; s0 += kRows) {
+      if (STG && !d.gvec) {
+        // scalar decay with the chunk staged: the score tile as a register-tiled product, each
+        // thread two query rows x four keys (keys r = kc + ncp u, so a warp's key rows fall in
+        // distinct banks), then the decay, eta and the causal mask
+        const int ncp = (C + 3) / 4;
+        for (int pi = threadIdx.x; pi < (kRows / 2) * ncp; pi += blockDim.x) {
+          const int rp = pi / ncp, kc = pi % ncp, sa = s0 + 2 * rp;
+          float acc[2][4] = {};
+          if (sa < C && kc <= sa + 1) {
+            const float* qa = Qs + sa * ldk;
+            const float* qb = Qs + min(sa + 1, C - 1) * ldk;
+            const float* kr[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) kr[u] = Ks + min(kc + ncp * u, C - 1) * ldk;
+#pragma unroll 4
+            for (int i = 0; i < dk; ++i) {
+              const float a0 = qa[i], a1 = qb[i];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const float b = kr[u][i];
+                acc[0][u] += a0 * b;
+                acc[1][u] += a1 * b;
+              }
+            }
+          }
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int s = sa + v;
+            float* Srow = S + (2 * rp + v) * C;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int r = kc + ncp * u;
+              if (r < C) Srow[r] = s < C && r <= s ? eta[r] * expf(L[s] - L[r]) * acc[v][u] : 0.f;
+            }
+          }
+        }
+      } else
       // a warp per query row, its lanes over the key features
       for (int sr = threadIdx.x >> 5; sr < kRows; sr += blockDim.x >> 5) {
         const int s = s0 + sr, lane = threadIdx.x & 31;
@@ -134,10 +190,9 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
           const int i = lane + 32 * m;
-          qv[m] = i < dk ? ldf(Q + qk0 + (tc + s) * dk + i) : 0.f;
+          qv[m] = i < dk ? qat(s, i) : 0.f;
           lv[m] = i < dk && d.gvec ? L[s * dk + i] : 0.f;
         }
-        const TI* Kc = K + qk0 + tc * dk;
         const float Ls = d.gvec ? 0.f : L[s];
         const bool gv = d.gvec;
         warp_row_dots<4>(
@@ -145,7 +200,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
             [=](int r, int m) {
               const int i = lane + 32 * m;
               if (i >= dk) return 0.f;
-              const float kv = ldf(Kc + r * dk + i);
+              const float kv = kat(r, i);
               return gv ? kv * __expf(lv[m] - L[r * dk + i]) : kv;
             },
             [=](int r, float p) {
@@ -157,12 +212,11 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
       for (int e = threadIdx.x; e < kRows * nv; e += blockDim.x) {
         const int sr = e / nv, j = e % nv, s = s0 + sr;
         if (s >= C) continue;
-        const TI* qs = Q + qk0 + (tc + s) * dk;
         float acc = 0.f;
         if (d.gvec) {
-          for (int i = 0; i < dk; ++i) acc += ldf(qs + i) * __expf(L[s * dk + i]) * Ws[i * kNvs + j];
+          for (int i = 0; i < dk; ++i) acc += qat(s, i) * __expf(L[s * dk + i]) * Ws[i * kNvs + j];
         } else {
-          for (int i = 0; i < dk; ++i) acc += ldf(qs + i) * Ws[i * kNvs + j];
+          for (int i = 0; i < dk; ++i) acc += qat(s, i) * Ws[i * kNvs + j];
           acc *= expf(L[s]);
         }
         for (int r = 0; r <= s; ++r) acc -= S[sr * C + r] * G[r * kNvs + j];
@@ -179,7 +233,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
       __syncthreads();
       for (int e = threadIdx.x; e < C * dk; e += blockDim.x) {
         const int r = e / dk, i = e % dk;
-        L[e] = eta[r] * expf(X[i] - L[e]) * ldf(K + qk0 + (tc + r) * dk + i);
+        L[e] = eta[r] * expf(X[i] - L[e]) * kat(r, i);
       }
     } else {
       for (int r = threadIdx.x; r < C; r += blockDim.x) X[r] = eta[r] * expf(L[C - 1] - L[r]);
@@ -192,7 +246,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Dims d, const TI* Q, cons
       if (d.gvec)
         for (int r = 0; r < C; ++r) w -= L[r * dk + i] * G[r * kNvs + j];
       else
-        for (int r = 0; r < C; ++r) w -= X[r] * ldf(K + qk0 + (tc + r) * dk + i) * G[r * kNvs + j];
+        for (int r = 0; r < C; ++r) w -= X[r] * kat(r, i) * G[r * kNvs + j];
       Ws[i * kNvs + j] = w;
     }
     __syncthreads();
@@ -489,11 +543,12 @@ Dims dims_of(const LayerArgs& a) {
 // Elements of one [B, H, T, dv] plane: with SiLU, Zq follows G in the saved buffer.
 size_t zq_plane(const LayerArgs& a) { return (size_t)a.B * a.H * a.T * a.dv; }
 
-size_t fwd_smem_bytes(const LayerArgs& a, int nvs = kNvs) {
+size_t fwd_smem_bytes(const LayerArgs& a, int nvs = kNvs, bool stg = false) {
   const size_t lw = a.gvec ? a.dk : 1;
   return sizeof(float) * ((size_t)a.dk * nvs + (size_t)a.C * nvs + (size_t)kRows * a.C + a.C +
-                           a.C * lw + a.C + 1 + a.dk);
+                           a.C * lw + a.C + 1 + a.dk + (stg ? 2 * (size_t)a.C * (a.dk + 1) : 0));
 }
+constexpr size_t kFwdStageMaxSmem = 160 * 1024;  // stage the chunk's keys and queries up to this
 
 // Value columns per forward block: narrower slices when the wide ones would leave most SMs idle
 // (each block recomputes the chunk's scores, so narrow slices trade that for parallelism).
@@ -514,19 +569,19 @@ size_t simt_bwd_workspace(const LayerArgs& a) {
   return sizeof(float) * bwd_head_floats(a.C, a.dk, a.dv, a.gvec) * a.B * a.H;
 }
 
-template <int NVS>
+template <int NVS, bool STG>
 void simt_fwd_launch(const LayerArgs& a, const Dims& d, cudaStream_t s) {
-  const size_t smem = fwd_smem_bytes(a, NVS);
+  const size_t smem = fwd_smem_bytes(a, NVS, STG);
   dim3 grid((a.dv + NVS - 1) / NVS, a.B * a.H);
   if (a.dtype == 0) {
-    auto k = simt_fwd_kernel<float, NVS>;
+    auto k = simt_fwd_kernel<float, NVS, STG>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     float* gs = (float*)a.G_saved;
     k<<<grid, 256, smem, s>>>(d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta,
                               a.gamma, a.W0, (float*)a.O, a.W_final, (float*)a.W_chunks, gs,
                               gs && a.act ? gs + zq_plane(a) : nullptr);
   } else {
-    auto k = simt_fwd_kernel<__nv_bfloat16, NVS>;
+    auto k = simt_fwd_kernel<__nv_bfloat16, NVS, STG>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     __nv_bfloat16* gs = (__nv_bfloat16*)a.G_saved;
     k<<<grid, 256, smem, s>>>(d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K,
@@ -538,10 +593,12 @@ void simt_fwd_launch(const LayerArgs& a, const Dims& d, cudaStream_t s) {
 
 cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
   const Dims d = dims_of(a);
-  if (fwd_nvs(a) == kNvsNarrow)
-    simt_fwd_launch<kNvsNarrow>(a, d, s);
+  const int nvs = fwd_nvs(a);
+  const bool stg = fwd_smem_bytes(a, nvs, true) <= kFwdStageMaxSmem;
+  if (nvs == kNvsNarrow)
+    stg ? simt_fwd_launch<kNvsNarrow, true>(a, d, s) : simt_fwd_launch<kNvsNarrow, false>(a, d, s);
   else
-    simt_fwd_launch<kNvs>(a, d, s);
+    stg ? simt_fwd_launch<kNvs, true>(a, d, s) : simt_fwd_launch<kNvs, false>(a, d, s);
   count_launches(1);
   return cudaGetLastError();
 }
