@@ -17,6 +17,8 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include <algorithm>
+
 #include "kernels.h"
 #include "simt_util.cuh"
 
@@ -34,6 +36,7 @@ struct Dims {
   int T, dk, dv, C, loss, act, has_gamma, gvec;
   float lr_bias;
   int w0_mod;
+  int smem_floats;  // backward: dynamic shared memory (floats) its scratch arrays may move into
 };
 
 // Entries of the log-decay prefix per chunk position: one, or one per key feature.
@@ -304,6 +307,46 @@ __global__ void __launch_bounds__(512) simt_bwd_kernel(
   float* dLk = dLq + C * dk;   //                    -k_si (dK_si - (dZ_s W0^T)_i)  [C][dk]
   float* wendv = dLk + C * dk; //                    row sums of W_end * dW_end  [dk]
   if (d.gvec) L = wendv + dk;  //                    log-decay prefix  [C][dk]
+  {
+    // The arrays the loops read most move into shared memory, as many as fit (the smallest and
+    // most-read first); the rest stay in the head's global scratch. Every access goes through
+    // these pointers, so either place serves.
+    extern __shared__ float sm[];
+    size_t used = 0;
+    auto place = [&](float*& a, size_t n) {
+      if (used + n <= (size_t)d.smem_floats) {
+        a = sm + used;
+        used += n;
+      }
+    };
+    const size_t kv = (size_t)dk * dv, cv = (size_t)C * dv, ck = (size_t)C * dk;
+    place(eta, C);
+    place(L, d.gvec ? ck : C);
+    place(deta, C);
+    place(dL, C);
+    place(wend, 1);
+    place(S, (size_t)C * C);
+    place(DS, (size_t)C * C);
+    place(W0, kv);
+    place(W0T, kv);
+    place(Wh, kv);
+    place(WhT, kv);
+    place(G, cv);
+    place(DZQ, cv);
+    place(QG, ck);
+    place(KC, ck);
+    place(Y, cv);
+    place(DG, cv);
+    place(DZ, cv);
+    place(Wn, kv);
+    place(Z, cv);
+    place(ZQ, cv);
+    if (d.gvec) {
+      place(dLq, ck);
+      place(dLk, ck);
+      place(wendv, dk);
+    }
+  }
   const size_t qk0 = (size_t)bh * d.T * dk, v0 = (size_t)bh * d.T * dv;
   for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
     Wh[e] = dWf ? dWf[(size_t)bh * dk * dv + e] : 0.f;
@@ -604,14 +647,22 @@ cudaError_t simt_fwd(const LayerArgs& a, cudaStream_t s) {
 }
 
 cudaError_t simt_bwd(const LayerArgs& a, cudaStream_t s) {
-  const Dims d = dims_of(a);
+  Dims d = dims_of(a);
+  // as much of the head's scratch as fits in shared memory (up to 200 KB)
+  const size_t hf = bwd_head_floats(a.C, a.dk, a.dv, a.gvec);
+  d.smem_floats = (int)std::min<size_t>(hf, 200 * 1024 / sizeof(float));
+  const size_t smem = (size_t)d.smem_floats * sizeof(float);
   if (a.dtype == 0) {
-    simt_bwd_kernel<float><<<a.B * a.H, 512, 0, s>>>(
+    auto k = simt_bwd_kernel<float>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<a.B * a.H, 512, smem, s>>>(
         d, (const float*)a.Q, (const float*)a.K, (const float*)a.V, a.beta, a.gamma,
         (const float*)a.W_chunks, (const float*)a.dO, a.dW_final, a.W_final_in, (float*)a.dQ,
         (float*)a.dK, (float*)a.dV, a.dbeta, a.dW0, a.dgamma, (float*)a.ws);
   } else {
-    simt_bwd_kernel<__nv_bfloat16><<<a.B * a.H, 512, 0, s>>>(
+    auto k = simt_bwd_kernel<__nv_bfloat16>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<a.B * a.H, 512, smem, s>>>(
         d, (const __nv_bfloat16*)a.Q, (const __nv_bfloat16*)a.K, (const __nv_bfloat16*)a.V,
         a.beta, a.gamma, (const __nv_bfloat16*)a.W_chunks, (const __nv_bfloat16*)a.dO,
         a.dW_final, a.W_final_in, (__nv_bfloat16*)a.dQ, (__nv_bfloat16*)a.dK,
