@@ -1048,16 +1048,16 @@ struct __align__(8) KgBars {
 };
 constexpr uint32_t kg_bytes() { return KgL::OFF_BAR + sizeof(KgBars); }
 
-__device__ __forceinline__ void ldg_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
-  const uint4* s4 = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint4 u = __ldg(s4 + k);
-    v[8 * k] = bf16lo(u.x); v[8 * k + 1] = bf16hi(u.x);
-    v[8 * k + 2] = bf16lo(u.y); v[8 * k + 3] = bf16hi(u.y);
-    v[8 * k + 4] = bf16lo(u.z); v[8 * k + 5] = bf16hi(u.z);
-    v[8 * k + 6] = bf16lo(u.w); v[8 * k + 7] = bf16hi(u.w);
-  }
+__device__ __forceinline__ void prefetch_l2(const void* a) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+}
+__device__ __forceinline__ void prefetch_l1(const void* a) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(a));
+}
+// Eight bf16 of u (x, y, z, w in order) as float32.
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
 }
 
 // SG: the tmV operand is the forward's saved G (bf16), so G is neither recomputed nor negated.
@@ -1207,6 +1207,12 @@ __global__ void __launch_bounds__(kVoThreads, 2)
     const int lrow = q * 32 + lane;
     const uint32_t loff = (uint32_t)(q * 32) << 16;
     const size_t tr = (size_t)tokc + 128 * kb + lrow;
+    // this key's rows of L (two 128-byte lines) and k (one), read by the last phase: into L2 now
+    const float* Lr = p.Lf + tr * VD;
+    const __nv_bfloat16* kr = p.K + tr * VD;
+    prefetch_l2(Lr);
+    prefetch_l2(Lr + 32);
+    if (p.colk || p.dLk) prefetch_l2(kr);
     const float sg = sigm(__ldg(p.beta + tr) + p.lr_bias), eta = 2.f * sg;
     float deta = 0.f;
     do {
@@ -1327,21 +1333,38 @@ __global__ void __launch_bounds__(kVoThreads, 2)
         if (lane == 0) mbar_arrive(KB(K_DGRDY));
       }
       // -------- dK
+      // the first half's L and k go out before the last products are waited for, the second
+      // half's into L1, so no tensor-memory read below waits on global memory
+      float4 Lq[8];
+      uint4 kq[4];
+      const bool want_k = p.colk || p.dLk;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) Lq[k] = __ldg(reinterpret_cast<const float4*>(Lr) + k);
+      if (want_k) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) kq[k] = __ldg(reinterpret_cast<const uint4*>(kr) + k);
+      }
+      prefetch_l1(Lr + 32);
       if (!mbar_wait(KB(K_F), 0, ab) || !mbar_wait(KB(K_GL), 0, ab) ||
           (LOSS == 0 && !mbar_wait(KB(K_DGW), 0, ab)))
         break;
       __syncwarp();
       tc_fence_after();
       bool range = false;
-      const float* Lr = p.Lf + tr * VD;
-      const __nv_bfloat16* kr = p.K + tr * VD;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         float dk[32], t32[32], Lv[32];
+        if (h == 1) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) Lq[k] = __ldg(reinterpret_cast<const float4*>(Lr + 32) + k);
+          if (want_k) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) kq[k] = __ldg(reinterpret_cast<const uint4*>(kr + 32) + k);
+          }
+        }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(Lr + 32 * h) + k);
-          Lv[4 * k] = v.x; Lv[4 * k + 1] = v.y; Lv[4 * k + 2] = v.z; Lv[4 * k + 3] = v.w;
+          Lv[4 * k] = Lq[k].x; Lv[4 * k + 1] = Lq[k].y; Lv[4 * k + 2] = Lq[k].z; Lv[4 * k + 3] = Lq[k].w;
         }
         tmem_ld32(tmem + loff + L::T_P + 32 * h, t32);  // G Lambda^T
         tmem_wait_ld();
@@ -1349,7 +1372,8 @@ __global__ void __launch_bounds__(kVoThreads, 2)
 #pragma unroll
         for (int k = 0; k < 32; ++k) dk[k] = -eta * __expf(LC[k] - Lv[k]) * t32[k];
         if (p.colk) {
-          ldg_bf16x32(kr + 32 * h, t32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) unpack_bf16x8(kq[k], t32 + 8 * k);
 #pragma unroll
           for (int k = 0; k < 32; ++k) t32[k] *= dk[k];
           colsum32(t32, lane);
@@ -1361,7 +1385,8 @@ __global__ void __launch_bounds__(kVoThreads, 2)
 #pragma unroll
         for (int k = 0; k < 32; ++k) dk[k] += clamped_exp(Lm[k] - Lv[k], range) * t32[k];
         if (p.dLk) {
-          ldg_bf16x32(kr + 32 * h, t32);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) unpack_bf16x8(kq[k], t32 + 8 * k);
           float4* dst = reinterpret_cast<float4*>(p.dLk + tr * VD + 32 * h);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
@@ -1523,6 +1548,11 @@ __global__ void __launch_bounds__(kVoThreads, 2)
     const uint32_t loff = (uint32_t)(q * 32) << 16;
     const int s = 128 * qb + lrow;
     const size_t ts = (size_t)tokc + s;
+    // this query's rows of L (two 128-byte lines) and q (one), read by the last phase: into L2 now
+    const float* Ls = p.Lf + ts * VD;
+    prefetch_l2(Ls);
+    prefetch_l2(Ls + 32);
+    if (p.dLq) prefetch_l2(p.Q + ts * VD);
     do {
       for (int t = threadIdx.x - 64; t < 128 * (qb + 1); t += 128)
         f_neta[t] = -eta_of(p.beta, (size_t)tokc + t, p.lr_bias);
@@ -1592,19 +1622,38 @@ __global__ void __launch_bounds__(kVoThreads, 2)
       }
       if (!ok) break;
       // -------- dQ = exp(L_s - L_m) * accumulator; q * dQ for the decay gradient
+      // the first half's L and q go out before the accumulator is waited for, the second half's
+      // into L1
+      float4 Lq[8];
+      uint4 qq[4];
+      const uint4* q4 = reinterpret_cast<const uint4*>(p.Q + ts * VD);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) Lq[k] = __ldg(reinterpret_cast<const float4*>(Ls) + k);
+      if (p.dLq) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qq[k] = __ldg(q4 + k);
+      }
+      prefetch_l1(Ls + 32);
       if (!mbar_wait(QB(Q_DQ), 0, ab)) break;
       __syncwarp();
       tc_fence_after();
       bool range = false;
-      const float* Ls = p.Lf + ts * VD;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         float a[32];
+        if (h == 1) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) Lq[k] = __ldg(reinterpret_cast<const float4*>(Ls + 32) + k);
+          if (p.dLq) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) qq[k] = __ldg(q4 + 4 + k);
+          }
+        }
         tmem_ld32(tmem + loff + L::T_DQ + 32 * h, a);
         tmem_wait_ld();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-          const float4 v = __ldg(reinterpret_cast<const float4*>(Ls + 32 * h) + k);
+          const float4 v = Lq[k];
           a[4 * k] *= clamped_exp(v.x - f_Lm[32 * h + 4 * k], range);
           a[4 * k + 1] *= clamped_exp(v.y - f_Lm[32 * h + 4 * k + 1], range);
           a[4 * k + 2] *= clamped_exp(v.z - f_Lm[32 * h + 4 * k + 2], range);
@@ -1612,11 +1661,10 @@ __global__ void __launch_bounds__(kVoThreads, 2)
         }
         st_global_bf16x32(p.dQ + ts * VD + 32 * h, a);
         if (p.dLq) {
-          const uint4* q4 = reinterpret_cast<const uint4*>(p.Q + ts * VD + 32 * h);
           float4* dst = reinterpret_cast<float4*>(p.dLq + ts * VD + 32 * h);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint4 u = __ldg(q4 + k);
+            const uint4 u = qq[k];
             dst[2 * k] = make_float4(bf16lo(u.x) * a[8 * k], bf16hi(u.x) * a[8 * k + 1],
                                      bf16lo(u.y) * a[8 * k + 2], bf16hi(u.y) * a[8 * k + 3]);
             dst[2 * k + 1] = make_float4(bf16lo(u.z) * a[8 * k + 4], bf16hi(u.z) * a[8 * k + 5],
