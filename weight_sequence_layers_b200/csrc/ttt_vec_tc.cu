@@ -1054,6 +1054,49 @@ __device__ __forceinline__ void prefetch_l2(const void* a) {
 __device__ __forceinline__ void prefetch_l1(const void* a) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(a));
 }
+// Row stores of a warp's 32 rows (this lane's row in v; row r goes to dst0 + r * ld) through a
+// 4 KB tile of shared memory: the lanes write their rows in 16-byte groups, then every store
+// instruction writes whole rows (four 128-byte float32 rows, or eight 64-byte bf16 rows) instead
+// of one 16-byte piece of each of 32 rows. The groups are rotated by the row so that neither the
+// row writes nor the reads collide in a bank.
+__device__ __forceinline__ void store_rows32_f32(float* tile, const float (&v)[32], float* dst0,
+                                                 size_t ld, int lane) {
+  float4* t4 = reinterpret_cast<float4*>(tile + lane * 32);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    t4[(c + lane) & 7] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  __syncwarp();
+  const int rs = lane >> 3, c = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + rs;
+    reinterpret_cast<float4*>(dst0 + (size_t)r * ld)[c] =
+        reinterpret_cast<const float4*>(tile + r * 32)[(c + r) & 7];
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ void store_rows32_bf16(float* tile, const float (&v)[32],
+                                                  __nv_bfloat16* dst0, size_t ld, int lane) {
+  // row r's four groups sit at (c + 4 (r & 1) + (r >> 1)) & 7 of its 128-byte tile row
+  auto slot = [](int c, int r) { return (c + 4 * (r & 1) + (r >> 1)) & 7; };
+  uint4* t4 = reinterpret_cast<uint4*>(tile + lane * 32);
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    t4[slot(c, lane)] = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]),
+                                   pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                   pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
+                                   pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+  __syncwarp();
+  const int rs = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * i + rs;
+    reinterpret_cast<uint4*>(dst0 + (size_t)r * ld)[c] =
+        reinterpret_cast<const uint4*>(tile + r * 32)[slot(c, r)];
+  }
+  __syncwarp();
+}
+
 // Eight bf16 of u (x, y, z, w in order) as float32.
 __device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
   v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
@@ -1215,6 +1258,9 @@ __global__ void __launch_bounds__(kVoThreads, 2)
     if (p.colk || p.dLk) prefetch_l2(kr);
     const float sg = sigm(__ldg(p.beta + tr) + p.lr_bias), eta = 2.f * sg;
     float deta = 0.f;
+    // this warp's staging tile for row stores, in the K panel (read by no product once the last
+    // query half has been multiplied)
+    float* ktile = reinterpret_cast<float*>(smem + L::OFF_K) + q * 1024;
     do {
       // L at the key block's reference token and at the chunk's last token
       {
@@ -1319,7 +1365,7 @@ __global__ void __launch_bounds__(kVoThreads, 2)
         float a[32];
         tmem_ld32(tmem + loff + L::T_DG + 32 * h, a);  // = -dG = dV
         tmem_wait_ld();
-        st_global_bf16x32(p.dV + tr * VD + 32 * h, a);
+        store_rows32_bf16(ktile, a, p.dV + (tr - lane) * VD + 32 * h, VD, lane);
         if constexpr (LOSS == 0) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) a[k] = -a[k];
@@ -1387,11 +1433,9 @@ __global__ void __launch_bounds__(kVoThreads, 2)
         if (p.dLk) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) unpack_bf16x8(kq[k], t32 + 8 * k);
-          float4* dst = reinterpret_cast<float4*>(p.dLk + tr * VD + 32 * h);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(-t32[4 * k] * dk[4 * k], -t32[4 * k + 1] * dk[4 * k + 1],
-                                 -t32[4 * k + 2] * dk[4 * k + 2], -t32[4 * k + 3] * dk[4 * k + 3]);
+          for (int k = 0; k < 32; ++k) t32[k] = -t32[k] * dk[k];
+          store_rows32_f32(ktile, t32, p.dLk + (tr - lane) * VD + 32 * h, VD, lane);
         }
         if constexpr (LOSS == 0) {
           tmem_ld32(tmem + loff + L::T_DS + 32 * h, t32);  // dG W0^T
@@ -1399,7 +1443,7 @@ __global__ void __launch_bounds__(kVoThreads, 2)
 #pragma unroll
           for (int k = 0; k < 32; ++k) dk[k] += t32[k];
         }
-        st_global_bf16x32(p.dK + tr * VD + 32 * h, dk);
+        store_rows32_bf16(ktile, dk, p.dK + (tr - lane) * VD + 32 * h, VD, lane);
       }
       p.dbeta[tr] = deta * 2.f * sg * (1.f - sg);
       if (range) atomicOr(err, ERR_RANGE);
@@ -1659,17 +1703,16 @@ __global__ void __launch_bounds__(kVoThreads, 2)
           a[4 * k + 2] *= clamped_exp(v.z - f_Lm[32 * h + 4 * k + 2], range);
           a[4 * k + 3] *= clamped_exp(v.w - f_Lm[32 * h + 4 * k + 3], range);
         }
-        st_global_bf16x32(p.dQ + ts * VD + 32 * h, a);
+        // the first K panel, read by no product any more, stages the row stores
+        float* qtile = reinterpret_cast<float*>(smem) + q * 1024;
+        store_rows32_bf16(qtile, a, p.dQ + (ts - lane) * VD + 32 * h, VD, lane);
         if (p.dLq) {
-          float4* dst = reinterpret_cast<float4*>(p.dLq + ts * VD + 32 * h);
+          float qv[32];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint4 u = qq[k];
-            dst[2 * k] = make_float4(bf16lo(u.x) * a[8 * k], bf16hi(u.x) * a[8 * k + 1],
-                                     bf16lo(u.y) * a[8 * k + 2], bf16hi(u.y) * a[8 * k + 3]);
-            dst[2 * k + 1] = make_float4(bf16lo(u.z) * a[8 * k + 4], bf16hi(u.z) * a[8 * k + 5],
-                                         bf16lo(u.w) * a[8 * k + 6], bf16hi(u.w) * a[8 * k + 7]);
-          }
+          for (int k = 0; k < 4; ++k) unpack_bf16x8(qq[k], qv + 8 * k);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) a[k] *= qv[k];
+          store_rows32_f32(qtile, a, p.dLq + (ts - lane) * VD + 32 * h, VD, lane);
         }
       }
       if (range) atomicOr(err, ERR_RANGE);
