@@ -86,6 +86,61 @@ __device__ __forceinline__ float clamped_exp(float e, bool& range) {
   }
   return __expf(e);
 }
+__device__ __forceinline__ void prefetch_l2(const void* a) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+}
+__device__ __forceinline__ void prefetch_l1(const void* a) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(a));
+}
+// Row stores of a warp's 32 rows (this lane's row in v; row r goes to dst0 + r * ld) through a
+// 4 KB tile of shared memory: the lanes write their rows in 16-byte groups, then every store
+// instruction writes whole rows (four 128-byte float32 rows, or eight 64-byte bf16 rows) instead
+// of one 16-byte piece of each of 32 rows. The groups are rotated by the row so that neither the
+// row writes nor the reads collide in a bank.
+__device__ __forceinline__ void store_rows32_f32(float* tile, const float (&v)[32], float* dst0,
+                                                 size_t ld, int lane) {
+  float4* t4 = reinterpret_cast<float4*>(tile + lane * 32);
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    t4[(c + lane) & 7] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  __syncwarp();
+  const int rs = lane >> 3, c = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + rs;
+    reinterpret_cast<float4*>(dst0 + (size_t)r * ld)[c] =
+        reinterpret_cast<const float4*>(tile + r * 32)[(c + r) & 7];
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ void store_rows32_bf16(float* tile, const float (&v)[32],
+                                                  __nv_bfloat16* dst0, size_t ld, int lane) {
+  // row r's four groups sit at (c + 4 (r & 1) + (r >> 1)) & 7 of its 128-byte tile row
+  auto slot = [](int c, int r) { return (c + 4 * (r & 1) + (r >> 1)) & 7; };
+  uint4* t4 = reinterpret_cast<uint4*>(tile + lane * 32);
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    t4[slot(c, lane)] = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]),
+                                   pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                   pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
+                                   pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+  __syncwarp();
+  const int rs = lane >> 2, c = lane & 3;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * i + rs;
+    reinterpret_cast<uint4*>(dst0 + (size_t)r * ld)[c] =
+        reinterpret_cast<const uint4*>(tile + r * 32)[slot(c, r)];
+  }
+  __syncwarp();
+}
+
+// Eight bf16 of u (x, y, z, w in order) as float32.
+__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
+  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
+  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
+}
+
 __device__ __forceinline__ float4 log4(float4 g) {
   return make_float4(__logf(g.x), __logf(g.y), __logf(g.z), __logf(g.w));
 }
@@ -698,13 +753,15 @@ __global__ void __launch_bounds__(kVoThreads, 2)
       if (!mbar_wait(UB(U_ZQ), 0, ab)) break;
       __syncwarp();
       tc_fence_after();
-      __nv_bfloat16* orow = p.O + ((size_t)tokc + s) * VD;
+      // the rows go out through slot B (V_0, read by no product any more)
+      float* otile = reinterpret_cast<float*>(smem + L::OFF_B) + q * 1024;
+      __nv_bfloat16* orow0 = p.O + ((size_t)tokc + s - lane) * VD;
 #pragma unroll 1
       for (int c32 = 0; c32 < VD / 32; ++c32) {
         float o[32];
         tmem_ld32(tmem + loff + L::T_ACC + 32 * c32, o);
         tmem_wait_ld();
-        st_global_bf16x32(orow + 32 * c32, o);
+        store_rows32_bf16(otile, o, orow0 + 32 * c32, VD, lane);
       }
     } while (0);
   }
@@ -1047,61 +1104,6 @@ struct __align__(8) KgBars {
   int abort_flag;
 };
 constexpr uint32_t kg_bytes() { return KgL::OFF_BAR + sizeof(KgBars); }
-
-__device__ __forceinline__ void prefetch_l2(const void* a) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-}
-__device__ __forceinline__ void prefetch_l1(const void* a) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(a));
-}
-// Row stores of a warp's 32 rows (this lane's row in v; row r goes to dst0 + r * ld) through a
-// 4 KB tile of shared memory: the lanes write their rows in 16-byte groups, then every store
-// instruction writes whole rows (four 128-byte float32 rows, or eight 64-byte bf16 rows) instead
-// of one 16-byte piece of each of 32 rows. The groups are rotated by the row so that neither the
-// row writes nor the reads collide in a bank.
-__device__ __forceinline__ void store_rows32_f32(float* tile, const float (&v)[32], float* dst0,
-                                                 size_t ld, int lane) {
-  float4* t4 = reinterpret_cast<float4*>(tile + lane * 32);
-#pragma unroll
-  for (int c = 0; c < 8; ++c)
-    t4[(c + lane) & 7] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-  __syncwarp();
-  const int rs = lane >> 3, c = lane & 7;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = 4 * i + rs;
-    reinterpret_cast<float4*>(dst0 + (size_t)r * ld)[c] =
-        reinterpret_cast<const float4*>(tile + r * 32)[(c + r) & 7];
-  }
-  __syncwarp();
-}
-__device__ __forceinline__ void store_rows32_bf16(float* tile, const float (&v)[32],
-                                                  __nv_bfloat16* dst0, size_t ld, int lane) {
-  // row r's four groups sit at (c + 4 (r & 1) + (r >> 1)) & 7 of its 128-byte tile row
-  auto slot = [](int c, int r) { return (c + 4 * (r & 1) + (r >> 1)) & 7; };
-  uint4* t4 = reinterpret_cast<uint4*>(tile + lane * 32);
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-    t4[slot(c, lane)] = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]),
-                                   pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
-                                   pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
-                                   pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
-  __syncwarp();
-  const int rs = lane >> 2, c = lane & 3;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = 8 * i + rs;
-    reinterpret_cast<uint4*>(dst0 + (size_t)r * ld)[c] =
-        reinterpret_cast<const uint4*>(tile + r * 32)[slot(c, r)];
-  }
-  __syncwarp();
-}
-
-// Eight bf16 of u (x, y, z, w in order) as float32.
-__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* v) {
-  v[0] = bf16lo(u.x); v[1] = bf16hi(u.x); v[2] = bf16lo(u.y); v[3] = bf16hi(u.y);
-  v[4] = bf16lo(u.z); v[5] = bf16hi(u.z); v[6] = bf16lo(u.w); v[7] = bf16hi(u.w);
-}
 
 // SG: the tmV operand is the forward's saved G (bf16), so G is neither recomputed nor negated.
 template <int NB, int LOSS, bool SG>
