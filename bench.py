@@ -575,8 +575,10 @@ PROFILE_CASES = {
                       "many passes",
     "inplace-bwd-8k": "the In-Place forward and backward on the first 8192 tokens (8 chunks, one "
                       "persistent launch each)",
-    "vector-decay": "vector decay forward (tensor cores) and backward (SIMT kernels), B=1, H=4, "
-                    "T=512, d=64, C=256",
+    "vector-decay": "vector decay forward and backward on the SIMT kernels (float32, which the "
+                    "tensor-core path does not take), B=1, H=4, T=512, d=64, C=256",
+    "tiny-fp32": "the tiny float32 inference forward (B=1, H=2, T=512, d=64, C=64): the SIMT "
+                 "forward with its chunk staged in shared memory and register-tiled scores",
     "vector-decay-fwd-410m": "the vector-decay forward on the 410M shape (B=8, H=16, T=2048, "
                              "d=64, C=256): the state and readout kernels",
     "vector-decay-410m": "the vector-decay forward and backward (decay gradient included) on "
@@ -649,11 +651,16 @@ def run_case(name, ttt):
                 ttt.inplace_ttt_bwd(T, F, M, C, icfg.lr, inp["Z"], inp["Vhat"], Wc, inp["dO"], None,
                                     dZ, dV, dW, ws, n)
     elif name == "vector-decay":
-        cfg = synth.FWD_410M.replace(B=1, H=4, T=512, decay="vector")
+        cfg = synth.FWD_410M.replace(B=1, H=4, T=512, decay="vector", dtype="f32")
         layer = Layer(cfg, ttt, seed=cfg.seed)
         for _ in range(2):
             layer.fwd()
             layer.bwd()
+    elif name == "tiny-fp32":
+        cfg = synth.TINY_FP32
+        layer = Layer(cfg, ttt, seed=cfg.seed)
+        for _ in range(2):
+            layer.fwd(save=False)
     elif name == "vector-decay-fwd-410m":
         cfg = synth.FWD_410M.replace(decay="vector")
         layer = Layer(cfg, ttt, seed=cfg.seed)
