@@ -31,7 +31,8 @@ SHAPES = [
     (1, 2, 96, 16, 24, 32),
     (2, 1, 192, 64, 40, 64),
     (1, 1, 60, 8, 8, 20),      # C not a multiple of the 32-row query tile
-    (1, 1, 512, 128, 128, 256),
+    (1, 1, 512, 128, 128, 256),  # the backward's scratch only partly in shared memory
+    (4, 8, 128, 32, 64, 32),     # enough heads for the forward's 32-column value slices
 ]
 COMBOS = [("mse", "id"), ("mse", "silu"), ("ip", "id"), ("ip", "silu")]
 
