@@ -481,6 +481,21 @@ def time_inplace(ttt, steps, warmup):
     dW = torch.empty((M, F), device="cuda", dtype=torch.float32)
     ms_save = timed(fwd, True)
     ms_bwd = timed(bwd, None)
+    extra = {}
+    # with document resets (four documents of eight chunks): one launch per chunk
+    nd = ttt.inplace_ttt_docs_workspace_bytes(T, F, M, C)
+    wsd = torch.empty(nd, device="cuda", dtype=torch.uint8)
+    starts = [k * (T // C) // 4 for k in (1, 2, 3)]
+    extra["docs_ms"] = timed(lambda _: ttt.inplace_ttt_fwd_docs(T, F, M, C, icfg.lr, inp["Z"],
+                                                                 inp["Vhat"], W, O, None, starts,
+                                                                 wsd, nd), None)
+    extra["doc_starts"] = starts
+    del wsd
+    # the context-parallel shard update dW = eta Vhat^T Z over the whole sequence (K = T)
+    dWd = torch.empty((M, F), device="cuda", dtype=torch.float32)
+    extra["delta_ms"] = timed(lambda _: ttt.inplace_ttt_delta(T, F, M, icfg.lr, inp["Z"], inp["Vhat"],
+                                                               dWd, ws, n), None)
+    del dWd
     # the NTP-aligned target Vhat = Conv1D(X0) W_target (4 taps) on the same sequence
     tin = synth.inplace_target_inputs(icfg, k=4, device="cuda")
     nt = ttt.inplace_ttt_target_workspace_bytes(T, M)
@@ -497,7 +512,7 @@ def time_inplace(ttt, steps, warmup):
     ms_tgt_bwd = timed(lambda _: ttt.inplace_ttt_target_bwd(T, M, 4, tin["X0"], tin["conv_w"],
                                                             tin["W_target"], tin["dVhat"], dX0,
                                                             dcw, dWt, wsb, ntb), None)
-    return icfg, ms, ms_save, ms_bwd, (ms_tgt, ms_tgt_bwd)
+    return icfg, ms, ms_save, ms_bwd, (ms_tgt, ms_tgt_bwd), extra
 
 
 # --------------------------------------------------------------------------- oracle legs
@@ -819,7 +834,8 @@ def main():
     if not args.no_configs:
         out["other_configs"] = time_other_configs(ttt, peaks)
     if not args.no_inplace:
-        icfg, ims, ims_save, ims_bwd, (ims_tgt, ims_tgt_bwd) = time_inplace(ttt, steps=3, warmup=3)
+        icfg, ims, ims_save, ims_bwd, (ims_tgt, ims_tgt_bwd), ix = time_inplace(ttt, steps=3,
+                                                                               warmup=3)
         fl, by = inplace_work(icfg)
         tf = fl / (ims * 1e-3) / 1e12
         # these calls are timed alone (a few launches of a few ms each, not a seconds-long
@@ -831,7 +847,21 @@ def main():
                                        "traffic": measured_traffic("inplace_ttt_fwd", icfg.name),
                                        "traffic_unit": "bytes per call (one launch)",
                                        "peak_source": peak_src},
-                          "ms_saving_chunk_weights": ims_save}
+                          "ms_saving_chunk_weights": ims_save,
+                          # document resets: the weight restarts at each document's first chunk,
+                          # so the chunks run one launch each instead of one persistent launch
+                          "ms_with_document_resets": ix["docs_ms"],
+                          "document_start_chunks": ix["doc_starts"]}
+        # the shard update of the context-parallel scan, dW = eta Vhat^T Z with K = T:
+        # 2 T d_ff d_model flops in one launch of update tiles
+        tfd = 2 * icfg.T * icfg.d_ff * icfg.d_model / (ix["delta_ms"] * 1e-3) / 1e12
+        out["inplace_cp_shard_update"] = {"workload": "inplace-ttt-wdown-shard-update-k32768",
+                                          "ms": ix["delta_ms"],
+                                          "roofline": {"bound": "tensor", "achieved": tfd,
+                                                       "peak": peaks["bf16_tflops"],
+                                                       "unit": "TFLOP/s",
+                                                       "frac": tfd / peaks["bf16_tflops"],
+                                                       "peak_source": peak_src}}
         # backward per token: dZ 4 d_model d_ff (K = 2 d_model), dVhat 2 d_ff d_model and the
         # adjoint update 2 d_model d_ff flops: twice the forward's 4 d_ff d_model
         tfb = 2 * fl / (ims_bwd * 1e-3) / 1e12

@@ -223,6 +223,31 @@ def test_inplace_document_resets(starts):
     assert rel_err(dZ, ref["dZ"]) <= O_TOL
     assert rel_err(dVh, ref["dVhat"]) <= O_TOL
     assert rel_err(dW, ref["dW"]) <= W_TOL
+    # the applied weights it saved: the state before each chunk, the initial W at a document start
+    for i in range(T // C):
+        s0 = max([0] + [s for s in starts if s <= i])  # the first chunk of chunk i's document
+        ref_i = inp["W"].double().cpu().numpy() if i == s0 else oracle.inplace_fwd(
+            inp["Z"][s0 * C: i * C], inp["Vhat"][s0 * C: i * C], inp["W"], C=C, lr=lr32)[1]
+        assert rel_err(Wc[i], ref_i) <= 4e-3, i
+
+
+@pytest.mark.parametrize("starts", [[2], [1, 3], [3, 5, 6]])
+def test_inplace_document_resets_without_saved_weights(starts):
+    # the forward alone (two rotating bf16 copies instead of the caller's chunk states), 8 chunks
+    cfg = synth.INPLACE_QWEN4B.replace(T=1024, d_ff=320, d_model=384, C=128, lr=0.1)
+    inp = synth.inplace_inputs(cfg, device="cuda", seed=63)
+    T, F, M, C = cfg.T, cfg.d_ff, cfg.d_model, cfg.C
+    n = ttt.inplace_ttt_docs_workspace_bytes(T, F, M, C)
+    ws = torch.empty(n, device="cuda", dtype=torch.uint8)
+    W = inp["W"].clone()
+    O = torch.empty((T, M), device="cuda", dtype=torch.bfloat16)
+    ttt.inplace_ttt_fwd_docs(T, F, M, C, cfg.lr, inp["Z"], inp["Vhat"], W, O, None, starts, ws, n)
+    torch.cuda.synchronize()
+    assert ttt.ttt_get_device_error() == ttt.OK
+    lr32 = float(np.float32(cfg.lr))
+    Oref, Wref = oracle.inplace_fwd(inp["Z"], inp["Vhat"], inp["W"], C=C, lr=lr32, doc_starts=starts)
+    assert rel_err(O, Oref) <= O_TOL
+    assert rel_err(W, Wref) <= W_TOL
 
 
 def test_inplace_delta_and_single_rank_context_parallel():

@@ -75,6 +75,9 @@ struct Params {
   // column block (backward). A tile waits for the counts of the chunk processed before it.
   int persistent, nchunk, tiles_per_chunk, n_mblk, n_nblk, wb_saved, upd_col_major;
   int* done;
+  // a persistent launch covers chunks [chunk0, chunk0 + nchunk) of the sequence (one document
+  // when the sequence has document resets); chunk indices above are relative to chunk0
+  int chunk0;
 };
 
 // Offsets of the completion-count arrays in Params::done.
@@ -106,13 +109,13 @@ __device__ __forceinline__ TileCtx ctx_of(const Params& p, int t) {
     c.u = t - k * p.tiles_per_chunk;
     c.wb_cur = (c.chunk & 1) * p.d_model;
     c.wb_next = c.chunk > 0 ? ((c.chunk - 1) & 1) * p.d_model : -1;
-    c.wc = c.chunk * p.d_model;
+    c.wc = (p.chunk0 + c.chunk) * p.d_model;
   } else if (p.persistent) {
     c.chunk = t / p.tiles_per_chunk;
     c.u = t - c.chunk * p.tiles_per_chunk;
     if (p.wb_saved) {
-      c.wb_cur = c.chunk * p.d_model;
-      c.wb_next = c.chunk + 1 < p.nchunk ? (c.chunk + 1) * p.d_model : -1;
+      c.wb_cur = (p.chunk0 + c.chunk) * p.d_model;
+      c.wb_next = c.chunk + 1 < p.nchunk ? (p.chunk0 + c.chunk + 1) * p.d_model : -1;
     } else {
       c.wb_cur = (c.chunk & 1) * p.d_model;
       c.wb_next = ((c.chunk + 1) & 1) * p.d_model;
@@ -123,7 +126,7 @@ __device__ __forceinline__ TileCtx ctx_of(const Params& p, int t) {
     c.wb_cur = p.wb_cur_row0;
     c.wb_next = p.wb_next_row0;
   }
-  c.row_base = c.chunk * p.C;
+  c.row_base = (c.chunk + (p.persistent ? p.chunk0 : 0)) * p.C;
   return c;
 }
 
@@ -1040,13 +1043,10 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   Launch l;
   cudaError_t e = prepare(&l);
   if (e != cudaSuccess) return e;
-  to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W, Wb, nW, 1.f);
   if (reset && (e = cudaMemcpyAsync(W0, W, nW * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
     return e;
   const int n_mblk = (d_model + PTM - 1) / PTM, n_nblk = (d_ff + BN - 1) / BN;
-  e = cudaMemsetAsync(counters, 0, ((size_t)NC + 2 * (size_t)NC * (n_mblk + n_nblk)) * sizeof(int),
-                      s);
-  if (e != cudaSuccess) return e;
+  const size_t n_counters = ((size_t)NC + 2 * (size_t)NC * (n_mblk + n_nblk)) * sizeof(int);
   Params p{};
   p.C = C;
   p.d_ff = d_ff;
@@ -1062,40 +1062,34 @@ cudaError_t inplace_run(int T, int d_ff, int d_model, int C, float lr, const voi
   p.Mb = Wb;
   p.Orow = static_cast<__nv_bfloat16*>(O);
   p.err = err;
-  if (!reset) {
-    // one launch over all chunks; each tile waits for the previous chunk's tiles it depends on
-    p.persistent = 1;
-    p.nchunk = NC;
-    p.tiles_per_chunk = p.n_total;
-    p.n_total = NC * p.tiles_per_chunk;
-    p.n_mblk = n_mblk;
-    p.n_nblk = n_nblk;
-    p.wb_saved = W_chunks != nullptr;
-    p.done = counters + NC;
-    p.counter = counters;
+  // One persistent launch per document (the whole sequence without resets): each tile waits for
+  // the tiles of the document's previous chunk it depends on. A document after the first starts
+  // from the initial W, kept in the workspace.
+  p.persistent = 1;
+  p.n_mblk = n_mblk;
+  p.n_nblk = n_nblk;
+  p.wb_saved = W_chunks != nullptr;
+  p.done = counters + NC;
+  p.counter = counters;
+  const int per_chunk = p.n_total;
+  int launches = 0;
+  for (int a = 0; a < NC;) {
+    int b = a + 1;
+    while (b < NC && !(reset && reset[b])) ++b;
+    if (a > 0 && (e = cudaMemcpyAsync(W, W0, nW * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
+      return e;
+    // the bf16 copy the document's first chunk applies
+    to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(a > 0 ? W0 : W,
+                                             Wb + (W_chunks ? (size_t)a * d_model * d_ff : 0),
+                                             nW, 1.f);
+    if ((e = cudaMemsetAsync(counters, 0, n_counters, s)) != cudaSuccess) return e;
+    p.chunk0 = a;
+    p.nchunk = b - a;
+    p.tiles_per_chunk = per_chunk;
+    p.n_total = p.nchunk * per_chunk;
     launch_pairs(l, p, s, tza, tzb, twb, tvh, tza, tza, tzb, tzb, tmf);
-    count_launches(2);
-    return cudaGetLastError();
-  }
-  int launches = NC + 1;
-  for (int i = 0; i < NC; ++i) {
-    p.chunk = i;
-    if (W_chunks) {
-      p.wb_cur_row0 = i * d_model;
-      p.wb_next_row0 = i + 1 < NC ? (i + 1) * d_model : -1;
-    } else {
-      p.wb_cur_row0 = (i & 1) * d_model;
-      p.wb_next_row0 = ((i + 1) & 1) * d_model;
-    }
-    p.counter = counters + i;
-    if (reset && i > 0 && reset[i]) {
-      // a new document: this chunk applies, and its update starts from, the initial W
-      if ((e = cudaMemcpyAsync(W, W0, nW * 4, cudaMemcpyDeviceToDevice, s)) != cudaSuccess)
-        return e;
-      to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(W0, Wb + (size_t)p.wb_cur_row0 * d_ff, nW, 1.f);
-      ++launches;
-    }
-    launch_pairs(l, p, s, tza, tzb, twb, tvh, tza, tza, tzb, tzb, tmf);
+    launches += 2;
+    a = b;
   }
   count_launches(launches);
   return cudaGetLastError();
@@ -1129,22 +1123,9 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   cudaError_t e = prepare(&l);
   if (e != cudaSuccess) return e;
   const size_t nW = (size_t)d_model * d_ff;
-  const int first = (NC - 1) & 1;  // copy slot the last chunk reads
-  int launches = NC + 1;
-  if (dW_final) {
-    e = cudaMemcpyAsync(R, dW_final, nW * sizeof(float), cudaMemcpyDeviceToDevice, s);
-    if (e != cudaSuccess) return e;
-    to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(dW_final, Mb + first * nW, nW, lr);
-  } else {
-    if ((e = cudaMemsetAsync(R, 0, nW * sizeof(float), s)) != cudaSuccess ||
-        (e = cudaMemsetAsync(Mb + first * nW, 0, nW * 2, s)) != cudaSuccess)
-      return e;
-  }
   if (reset && (e = cudaMemsetAsync(dW, 0, nW * sizeof(float), s)) != cudaSuccess) return e;
   const int n_mblk = (d_model + PTM - 1) / PTM, n_nblk = (d_ff + BN - 1) / BN;
-  e = cudaMemsetAsync(counters, 0, ((size_t)NC + 2 * (size_t)NC * (n_mblk + n_nblk)) * sizeof(int),
-                      s);
-  if (e != cudaSuccess) return e;
+  const size_t n_counters = ((size_t)NC + 2 * (size_t)NC * (n_mblk + n_nblk)) * sizeof(int);
   Params p{};
   p.C = C;
   p.d_ff = d_ff;
@@ -1164,39 +1145,43 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   p.Orow = static_cast<__nv_bfloat16*>(dVhat);
   p.Odz = static_cast<__nv_bfloat16*>(dZ);
   p.err = err;
-  if (!reset) {
-    // one launch over all chunks, from the last one; each tile waits for the tiles of the chunk
-    // after it that it depends on
-    p.persistent = 2;
-    p.upd_col_major = 1;
-    p.nchunk = NC;
-    p.tiles_per_chunk = p.n_total;
-    p.n_total = NC * p.tiles_per_chunk;
-    p.n_mblk = n_mblk;
-    p.n_nblk = n_nblk;
-    p.done = counters + NC;
-    p.counter = counters;
+  // One persistent launch per document, the last document first, each from its last chunk;
+  // each tile waits for the tiles of the chunk after it that it depends on. The last document's
+  // adjoint starts from dW_final; an earlier document's from zero (the next document restarted
+  // from the initial W), and each document's adjoint at its first chunk joins dW.
+  p.persistent = 2;
+  p.upd_col_major = 1;
+  p.n_mblk = n_mblk;
+  p.n_nblk = n_nblk;
+  p.done = counters + NC;
+  p.counter = counters;
+  const int per_chunk = p.n_total;
+  int launches = 0;
+  for (int b = NC; b > 0;) {
+    int a = b - 1;
+    while (a > 0 && !(reset && reset[a])) --a;
+    const int first = (b - a - 1) & 1;  // copy slot the document's last chunk reads
+    if (b == NC && dW_final) {
+      e = cudaMemcpyAsync(R, dW_final, nW * sizeof(float), cudaMemcpyDeviceToDevice, s);
+      if (e != cudaSuccess) return e;
+      to_bf16_kernel<<<l.sms * 4, 256, 0, s>>>(dW_final, Mb + first * nW, nW, lr);
+      ++launches;
+    } else if ((e = cudaMemsetAsync(R, 0, nW * sizeof(float), s)) != cudaSuccess ||
+               (e = cudaMemsetAsync(Mb + first * nW, 0, nW * 2, s)) != cudaSuccess) {
+      return e;
+    }
+    if ((e = cudaMemsetAsync(counters, 0, n_counters, s)) != cudaSuccess) return e;
+    p.chunk0 = a;
+    p.nchunk = b - a;
+    p.tiles_per_chunk = per_chunk;
+    p.n_total = p.nchunk * per_chunk;
     launch_pairs(l, p, s, tza, tzb, tmb, tdx, tdo, tvk, twc, tmbn, tmf);
-    count_launches(dW_final ? 2 : 1);
-    return cudaGetLastError();
-  }
-  for (int i = NC - 1; i >= 0; --i) {
-    p.chunk = i;
-    p.wb_cur_row0 = (i & 1) * d_model;
-    p.wb_next_row0 = i > 0 ? ((i - 1) & 1) * d_model : -1;
-    p.wc_row0 = i * d_model;
-    p.counter = counters + i;
-    launch_pairs(l, p, s, tza, tzb, tmb, tdx, tdo, tvk, twc, tmbn, tmf);
-    if (reset && (i == 0 || reset[i])) {
-      // this document's first chunk applied the initial W: its adjoint joins dW, and the
-      // previous document's end state (and its bf16 copy) gets none
+    ++launches;
+    if (reset) {
       add_kernel<<<l.sms * 4, 256, 0, s>>>(dW, R, nW / 4);
       ++launches;
-      if (i > 0 && ((e = cudaMemsetAsync(R, 0, nW * sizeof(float), s)) != cudaSuccess ||
-                    (e = cudaMemsetAsync(Mb + (size_t)p.wb_next_row0 * d_ff, 0, nW * 2, s)) !=
-                        cudaSuccess))
-        return e;
     }
+    b = a;
   }
   count_launches(launches);
   return cudaGetLastError();
