@@ -78,6 +78,9 @@ struct Params {
   // a persistent launch covers chunks [chunk0, chunk0 + nchunk) of the sequence (one document
   // when the sequence has document resets); chunk indices above are relative to chunk0
   int chunk0;
+  // the dz tiles of a chunk are handed out before its row tiles (the backward: a dz tile needs
+  // one column block of the previous chunk's adjoint copy, a row tile whole rows of it)
+  int dz_first;
 };
 
 // Offsets of the completion-count arrays in Params::done.
@@ -176,6 +179,7 @@ struct Tile {
 template <int TM>
 __device__ __forceinline__ Tile decode(const Params& p, int t) {
   Tile x;
+  if (p.dz_first) t = t < p.n_dz ? t + p.n_row : t < p.n_dz + p.n_row ? t - p.n_dz : t;
   if (t < p.n_row) {
     x.kind = KIND_ROW;
     x.m0 = (t / p.n_row_n) * TM;  // token offset inside the chunk
@@ -1151,6 +1155,7 @@ cudaError_t inplace_bwd_run(int T, int d_ff, int d_model, int C, float lr, const
   // from the initial W), and each document's adjoint at its first chunk joins dW.
   p.persistent = 2;
   p.upd_col_major = 1;
+  p.dz_first = 1;
   p.n_mblk = n_mblk;
   p.n_nblk = n_nblk;
   p.done = counters + NC;
