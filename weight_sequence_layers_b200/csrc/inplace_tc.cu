@@ -188,8 +188,15 @@ __device__ __forceinline__ Tile decode(const Params& p, int t) {
   } else if (t < p.n_row + p.n_dz) {
     const int u = t - p.n_row;
     x.kind = KIND_DZ;
-    x.m0 = (u / p.n_dz_n) * TM;   // token offset inside the chunk
-    x.n0 = (u % p.n_dz_n) * BN;   // d_ff column
+    if (p.dz_first) {
+      // column blocks in the order the previous chunk's (column-major) update tiles finish them
+      const int n_tok = p.n_dz / p.n_dz_n;
+      x.m0 = (u % n_tok) * TM;
+      x.n0 = (u / n_tok) * BN;
+    } else {
+      x.m0 = (u / p.n_dz_n) * TM;   // token offset inside the chunk
+      x.n0 = (u % p.n_dz_n) * BN;   // d_ff column
+    }
     x.nkb = p.kb_dz;
   } else {
     const int u = t - p.n_row - p.n_dz;
