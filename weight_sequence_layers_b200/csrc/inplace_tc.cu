@@ -23,12 +23,13 @@
 //   update tiles [256 d_model x 256 d_ff]: M += s X_i^T (MN-major) x Z_i (MN-major), K = C,
 //                with (M, X, s) = (W, Vhat, eta) forward and (Wh, dO, 1) backward; the epilogue
 //                keeps M in float32 and writes the scaled bf16 copy the next launch reads.
-// Long tiles (row, then dz) are handed out first, update tiles fill the remaining SMs. When
-// a CTA takes an update tile it prefetches its float32 block of M into L2, so the epilogue's
-// read-modify-write, issued after the tile's K steps, reads from L2.
-// Without document resets the forward and the backward are each ONE persistent launch over all
-// chunks, a tile waiting (bounded) for the tiles of the previously processed chunk it depends
-// on, through per-block completion counts in the workspace.
+// Long tiles (row, then dz; the backward dz, then row) are handed out first, update tiles fill
+// the remaining SMs. When a CTA takes an update tile it prefetches its float32 block of M into
+// L2, so the epilogue's read-modify-write, issued after the tile's K steps, reads from L2.
+// The forward and the backward are each ONE persistent launch over all chunks (over each
+// document's chunks with document resets), a tile waiting (bounded) for the tiles of the
+// previously processed chunk it depends on, through per-block completion counts in the
+// workspace.
 // Warp roles in each CTA: warp 0 issues TMA loads into a 6-stage ring, warp 1 of the leader CTA
 // (rank 0) issues the pair MMAs into two TMEM accumulators of 128 x 256 fp32 per CTA, warps 2-9
 // drain this CTA's accumulator rows (two warps per TMEM lane quadrant, each taking 128 of the
