@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stddef.h>
 
+#include <mutex>
+
 namespace tttk {
 
 struct LayerArgs {
@@ -133,5 +135,17 @@ bool make_tmap_f32(CUtensorMap* m, const void* base, uint64_t inner, uint64_t ro
 bool make_tmap3_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
                      uint64_t batch, uint64_t row_stride_elems, uint64_t batch_stride_elems,
                      uint32_t box_inner, uint32_t box_rows);
+
+// The tensor-core backward's per-device pair of internal streams (the serial chain at the
+// higher priority, the chunk-parallel work that does not depend on it at the lower) and the
+// events that fork the caller's stream into them and join it again, created on first use. A
+// backward enqueues its whole sequence while holding fork_mutex(), so calls from several host
+// threads keep their dependencies.
+struct ForkSet {
+  cudaStream_t hi = nullptr, lo = nullptr;
+  cudaEvent_t e0 = nullptr, eg = nullptr, ehi = nullptr, elo = nullptr;
+};
+ForkSet* fork_set();      // nullptr if the streams or events cannot be created
+std::mutex& fork_mutex();
 
 }  // namespace tttk

@@ -1207,17 +1207,15 @@ __global__ void __launch_bounds__(256)
 
 #undef BAR
 
-// Per-device pair of internal streams (chain then dk at the higher priority; g then dq at the
-// lower) and the events that fork the caller's stream into them and join it again. The enqueue
-// sequence runs under one lock, so calls from several host threads keep their dependencies
-// (their GPU work then serialises through the shared streams).
-struct ForkSet {
-  cudaStream_t hi = nullptr, lo = nullptr;
-  cudaEvent_t e0 = nullptr, eg = nullptr, ehi = nullptr, elo = nullptr;
-};
+// The fork set (kernels.h): chain then dk at the higher priority, g then dq at the lower; the
+// GPU work of calls from several host threads serialises through the shared streams.
 constexpr int kMaxDevices = 64;
 ForkSet g_fork[kMaxDevices];
 std::mutex g_fork_mu;
+
+}  // namespace
+
+std::mutex& fork_mutex() { return g_fork_mu; }
 
 ForkSet* fork_set() {
   int dev = 0;
@@ -1238,6 +1236,8 @@ ForkSet* fork_set() {
   }
   return &f;
 }
+
+namespace {
 
 template <int D, int NB>
 cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
@@ -1322,7 +1322,7 @@ cudaError_t launch(const LayerArgs& a, cudaStream_t s) {
       (e = cudaFuncSetAttribute(kk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dk)) ||
       (e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm_dq)))
     return e;
-  std::lock_guard<std::mutex> lk(g_fork_mu);
+  std::lock_guard<std::mutex> lk(fork_mutex());
   ForkSet* f = fork_set();
   if (!f) return cudaErrorInitializationError;
   int launched = g_saved ? 3 : 4;

@@ -1976,10 +1976,21 @@ cudaError_t launch_vec_bwd(const LayerArgs& a, cudaStream_t s) {
     kr<<<BH * NC * NB, kVoThreads, sm_r, s>>>(tQt, tKt, tK, tK, tK, tR, vp, a.err);
     count_launches(1);
   }
-  kb<<<BH, kVsThreads, sm_b, s>>>(tK, tKh, tR, tdO, bp, a.err);
-  kk<<<BH * NC * NB, kVoThreads, sm_k, s>>>(tK, tKh, tV, tKt, tQh, tQ2h, tdOh, tW, tLam, gp,
-                                            a.err);
-  kq<<<BH * NC * NB, kVoThreads, sm_q, s>>>(tK, tV, tKt, tdO, tW, gp, a.err);
+  // The query side needs no adjoint: it runs on the lower-priority stream beside the serial
+  // adjoint chain (one CTA per head, leaving SMs free) and the key side that follows it.
+  std::lock_guard<std::mutex> lk(fork_mutex());
+  ForkSet* f = fork_set();
+  if (!f) return cudaErrorInitializationError;
+  if ((e = cudaEventRecord(f->e0, s)) || (e = cudaStreamWaitEvent(f->hi, f->e0, 0)) ||
+      (e = cudaStreamWaitEvent(f->lo, f->e0, 0)))
+    return e;
+  kb<<<BH, kVsThreads, sm_b, f->hi>>>(tK, tKh, tR, tdO, bp, a.err);
+  kq<<<BH * NC * NB, kVoThreads, sm_q, f->lo>>>(tK, tV, tKt, tdO, tW, gp, a.err);
+  kk<<<BH * NC * NB, kVoThreads, sm_k, f->hi>>>(tK, tKh, tV, tKt, tQh, tQ2h, tdOh, tW, tLam, gp,
+                                                a.err);
+  if ((e = cudaEventRecord(f->elo, f->lo)) || (e = cudaEventRecord(f->ehi, f->hi)) ||
+      (e = cudaStreamWaitEvent(s, f->ehi, 0)) || (e = cudaStreamWaitEvent(s, f->elo, 0)))
+    return e;
   count_launches(3);
   if (dg) {
     DgParams dp{};
