@@ -17,9 +17,11 @@
 // factor beyond exp(80) is clamped and recorded in the device error word (a range error).
 //
 // Forward, three kernels:
-//   prep   : one CTA per (batch, head, chunk): the per-feature log-decay scan and every decayed
-//            operand (qtilde, ktilde per reference token, Khat) written once as bf16, with
-//            exp(L_C) and exp(L_m); the backward reuses it (and keeps L itself).
+//   prep   : persistent, one CTA per SM over (batch, head, chunk, half of the features) units,
+//            the next two units' gamma, q and k in flight to shared memory while the current
+//            one runs: the per-feature log-decay scan and every decayed operand (qtilde, ktilde
+//            per reference token, Khat) written once as bf16, with exp(L_C) and exp(L_m); the
+//            backward reuses it (and keeps L itself).
 //   vstate : one CTA per (batch, head) walks the chunks with the fp32 state in TMEM: Z = K W0,
 //            -eta G, W = diag(exp(L_C)) W + Khat^T (-eta G); K and Khat arrive by TMA.
 //   vout   : one CTA per (batch, head, chunk, 128-query block), two per SM:
@@ -28,6 +30,8 @@
 // adjoint pass, a key-side and a query-side chunk-parallel kernel, and the decay-gradient scan.
 #include <cuda_bf16.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -155,87 +159,170 @@ __device__ __forceinline__ uint2 scale4(uint2 x, float4 e, bool& range) {
   return r;
 }
 
-constexpr int kPrepSeg = 16;  // slices per chunk
+constexpr int kPrepSeg = 16;  // slices per chunk (decay-gradient scan)
 constexpr int kPrepThreads = 128;  // 8 feature quads (32 features) x 16 slices
 
-// One CTA per (batch, head, chunk, half of the features). Each thread loads its whole slice
-// (gamma, q, k) into registers before any arithmetic, so every load is in flight at once.
+// 16-byte asynchronous global -> shared copies (no register staging), in commit groups.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The prep is persistent: one CTA per SM walks units u = (batch, head, chunk, half of the
+// features) with a stride of the grid. A unit's gamma, q and k rows reach shared memory through
+// asynchronous copies issued two units ahead (three stages), so an SM's DRAM traffic for the
+// next units overlaps the exponentials and stores of the current one. Thread (f = four adjacent
+// key features, seg = one of 64 slices of the chunk); the slice sums are scanned by eight warps
+// (one per feature quad) with shuffles.
+constexpr int kPrepNseg = 64;
+constexpr int kPrepPThreads = 8 * kPrepNseg;
+constexpr int kPrepStages = 3;
 template <int NB>
-__global__ void __launch_bounds__(kPrepThreads) vec_prep_kernel(const PrepParams p) {
-  constexpr int C = 128 * NB, SEG = C / kPrepSeg, NV = NB * (NB + 1) / 2;
-  __shared__ float4 tot[kPrepSeg][8];
+__host__ __device__ constexpr uint32_t prep_stage_bytes() { return 128 * NB * (128 + 2 * 64); }  // gamma, q, k
+
+template <int NB>
+__global__ void __launch_bounds__(kPrepPThreads, 1) vec_prep_kernel(const PrepParams p, int nunits) {
+  constexpr int C = 128 * NB, SEG = C / kPrepNseg, NV = NB * (NB + 1) / 2;
+  constexpr uint32_t GB = C * 128, QB = C * 64, STAGE = prep_stage_bytes<NB>();
+  extern __shared__ __align__(16) uint8_t prep_smem[];
+  __shared__ float4 tot[kPrepNseg][8];  // per-slice sums of log gamma
+  __shared__ float4 pre[kPrepNseg][8];  // their exclusive prefix sums
   const int f = threadIdx.x & 7, seg = threadIdx.x >> 3;
-  const int fq = (blockIdx.x & 1) * 8 + f;  // feature quad 0..15
-  const size_t bc = blockIdx.x >> 1;        // bh * NC + c
-  const size_t r0 = bc * C + seg * SEG;     // first token row of this slice
-  const float4* __restrict__ g = reinterpret_cast<const float4*>(p.gamma + r0 * VD) + fq;
-  const uint2* __restrict__ q = reinterpret_cast<const uint2*>(p.Q + r0 * VD) + fq;
-  const uint2* __restrict__ k = reinterpret_cast<const uint2*>(p.K + r0 * VD) + fq;
-  float4 lg[SEG];
-  uint2 qv[SEG], kv[SEG];
-#pragma unroll
-  for (int t = 0; t < SEG; ++t) {
-    lg[t] = __ldg(g + t * (VD / 4));
-    qv[t] = __ldg(q + t * (VD / 4));
-    kv[t] = __ldg(k + t * (VD / 4));
-  }
-  {
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint32_t s_base = smem_u32(prep_smem);
+  // unit u into stage st: C rows of 32 gamma (8 x 16 bytes), of 32 q and of 32 k (4 x 16 bytes
+  // each); one commit group per call, empty past the last unit
+  auto issue = [&](int u, int st) {
+    if (u < nunits) {
+      const size_t e0 = (size_t)(u >> 1) * C * VD + 32 * (u & 1);
+      const uint8_t* g = reinterpret_cast<const uint8_t*>(p.gamma + e0);
+      const uint8_t* q = reinterpret_cast<const uint8_t*>(p.Q + e0);
+      const uint8_t* k = reinterpret_cast<const uint8_t*>(p.K + e0);
+      const uint32_t s0 = s_base + st * STAGE;
+      for (int i = threadIdx.x; i < C * 8; i += kPrepPThreads)
+        cp_async16(s0 + i * 16, g + (size_t)(i >> 3) * VD * 4 + (i & 7) * 16);
+      for (int i = threadIdx.x; i < C * 4; i += kPrepPThreads) {
+        const size_t off = (size_t)(i >> 2) * VD * 2 + (i & 3) * 16;
+        cp_async16(s0 + GB + i * 16, q + off);
+        cp_async16(s0 + GB + QB + i * 16, k + off);
+      }
+    }
+    cp_async_commit();
+  };
+  bool range = false;
+  const int stride = gridDim.x;
+  issue(blockIdx.x, 0);
+  issue(blockIdx.x + stride, 1);
+  int st = 0;
+  for (int u = blockIdx.x; u < nunits; u += stride) {
+    cp_async_wait<1>();  // this thread's copies of unit u have landed ...
+    __syncthreads();     // ... and every thread's
+    const uint8_t* sb = prep_smem + st * STAGE;
+    const float4* gs = reinterpret_cast<const float4*>(sb) + seg * SEG * 8 + f;
+    const uint2* qs = reinterpret_cast<const uint2*>(sb + GB) + seg * SEG * 8 + f;
+    const uint2* ks = reinterpret_cast<const uint2*>(sb + GB + QB) + seg * SEG * 8 + f;
+    float4 lg[SEG];
+    uint2 qv[SEG], kv[SEG];
 #pragma unroll
     for (int t = 0; t < SEG; ++t) {
-      lg[t] = log4(lg[t]);
-      s = add4(s, lg[t]);
+      lg[t] = gs[t * 8];
+      qv[t] = qs[t * 8];
+      kv[t] = ks[t * 8];
     }
-    tot[seg][f] = s;
-  }
-  __syncthreads();
-  float4 Lstart = make_float4(0.f, 0.f, 0.f, 0.f), LC = Lstart, Lm[NB];
+    // the stage of the previous unit: every thread has read it before the barrier above
+    issue(u + 2 * stride, st == 0 ? 2 : st - 1);
+    st = st == kPrepStages - 1 ? 0 : st + 1;
+
+    const int fq = (u & 1) * 8 + f;        // feature quad 0..15
+    const size_t bc = u >> 1;              // bh * NC + c
+    const size_t r0 = bc * C + seg * SEG;  // first token row of this slice
+    {
+      float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int kk = 0; kk < kPrepSeg; ++kk) {
-    const float4 tk = tot[kk][f];
-    if (kk < seg) Lstart = add4(Lstart, tk);
-    LC = add4(LC, tk);
+      for (int t = 0; t < SEG; ++t) {
+        lg[t] = log4(lg[t]);
+        s = add4(s, lg[t]);
+      }
+      tot[seg][f] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {
+      // warp w: exclusive prefix over the 64 slices of feature quad w, two slices a lane
+      const int w = threadIdx.x >> 5, j = threadIdx.x & 31;
+      const float4 a = tot[2 * j][w], b = tot[2 * j + 1][w];
+      float4 inc = add4(a, b);
 #pragma unroll
-    for (int qb = 0; qb < NB; ++qb)
-      if (kk == (128 * qb + 64) / SEG - 1) Lm[qb] = LC;
-  }
-  const int kb = seg * SEG / 128;
-  bool range = false;
-  float4 l = make_float4(0.f, 0.f, 0.f, 0.f);
-  uint2* qt = reinterpret_cast<uint2*>(p.Qt + r0 * VD) + fq;
-  uint2* kh = reinterpret_cast<uint2*>(p.Kh + r0 * VD) + fq;
-  const float4 lmk = Lm[kb];
-#pragma unroll
-  for (int t = 0; t < SEG; ++t) {
-    const int o = t * (VD / 4);
-    l = add4(l, lg[t]);
-    const float4 L = add4(Lstart, l);
-    qt[o] = scale4(qv[t], make_float4(L.x - lmk.x, L.y - lmk.y, L.z - lmk.z, L.w - lmk.w), range);
-    kh[o] = scale4(kv[t], make_float4(LC.x - L.x, LC.y - L.y, LC.z - L.z, LC.w - L.w), range);
-    const int tr = (seg * SEG + t) & 127;  // row inside the key block
+      for (int d = 1; d < 32; d <<= 1) {
+        const float4 o = make_float4(__shfl_up_sync(0xffffffffu, inc.x, d),
+                                     __shfl_up_sync(0xffffffffu, inc.y, d),
+                                     __shfl_up_sync(0xffffffffu, inc.z, d),
+                                     __shfl_up_sync(0xffffffffu, inc.w, d));
+        if (j >= d) inc = add4(o, inc);
+      }
+      float4 ex = make_float4(__shfl_up_sync(0xffffffffu, inc.x, 1),
+                              __shfl_up_sync(0xffffffffu, inc.y, 1),
+                              __shfl_up_sync(0xffffffffu, inc.z, 1),
+                              __shfl_up_sync(0xffffffffu, inc.w, 1));
+      if (j == 0) ex = make_float4(0.f, 0.f, 0.f, 0.f);
+      pre[2 * j][w] = ex;
+      pre[2 * j + 1][w] = add4(ex, a);
+    }
+    __syncthreads();
+    // L_t = (prefix of the slice) + (running sum inside it). Slice boundaries fall on the
+    // reference tokens' successors (64 and 192 for C = 256, 64 for C = 128), and L_m and L_C are
+    // formed as the same two-term sum as L_t at those tokens, so the exponent at the reference
+    // token is exactly 0.
+    const float4 Lstart = pre[seg][f];
+    const float4 LC = add4(pre[kPrepNseg - 1][f], tot[kPrepNseg - 1][f]);
+    float4 Lm[NB];
 #pragma unroll
     for (int qb = 0; qb < NB; ++qb) {
-      if (qb < kb) continue;
-      const int v = qb * (qb + 1) / 2 + kb;
-      const float4 m = Lm[qb];
-      reinterpret_cast<uint2*>(p.Kt + ((bc * NV + v) * 128 + tr) * VD)[fq] =
-          scale4(kv[t], make_float4(m.x - L.x, m.y - L.y, m.z - L.z, m.w - L.w), range);
+      const int kk = (128 * qb + 64) / SEG - 1;
+      Lm[qb] = add4(pre[kk][f], tot[kk][f]);
     }
-    if (p.Lf) reinterpret_cast<float4*>(p.Lf + r0 * VD)[o + fq] = L;
-    if (NB == 2 && kb == 1 && p.Qt2) {  // exponents <= 0: the reference precedes the token
-      const float4 m = Lm[0];
-      reinterpret_cast<uint2*>(p.Qt2 + (bc * 128 + tr) * VD)[fq] =
-          scale4(qv[t], make_float4(L.x - m.x, L.y - m.y, L.z - m.z, L.w - m.w), range);
-    }
-  }
-  if (seg == 0) {
-    reinterpret_cast<float4*>(p.GC + bc * VD)[fq] =
-        make_float4(__expf(LC.x), __expf(LC.y), __expf(LC.z), __expf(LC.w));
+    const int kb = seg * SEG / 128;
+    float4 l = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint2* qt = reinterpret_cast<uint2*>(p.Qt + r0 * VD) + fq;
+    uint2* kh = reinterpret_cast<uint2*>(p.Kh + r0 * VD) + fq;
+    const float4 lmk = kb ? Lm[NB - 1] : Lm[0];  // kb < NB <= 2
 #pragma unroll
-    for (int qb = 0; qb < NB; ++qb)
-      reinterpret_cast<float4*>(p.Em + (bc * NB + qb) * VD)[fq] = make_float4(
-          __expf(Lm[qb].x), __expf(Lm[qb].y), __expf(Lm[qb].z), __expf(Lm[qb].w));
+    for (int t = 0; t < SEG; ++t) {
+      const int o = t * (VD / 4);
+      l = add4(l, lg[t]);
+      const float4 L = add4(Lstart, l);
+      qt[o] = scale4(qv[t], make_float4(L.x - lmk.x, L.y - lmk.y, L.z - lmk.z, L.w - lmk.w), range);
+      kh[o] = scale4(kv[t], make_float4(LC.x - L.x, LC.y - L.y, LC.z - L.z, LC.w - L.w), range);
+      const int tr = (seg * SEG + t) & 127;  // row inside the key block
+#pragma unroll
+      for (int qb = 0; qb < NB; ++qb) {
+        if (qb < kb) continue;
+        const int v = qb * (qb + 1) / 2 + kb;
+        const float4 m = Lm[qb];
+        reinterpret_cast<uint2*>(p.Kt + ((bc * NV + v) * 128 + tr) * VD)[fq] =
+            scale4(kv[t], make_float4(m.x - L.x, m.y - L.y, m.z - L.z, m.w - L.w), range);
+      }
+      if (p.Lf) reinterpret_cast<float4*>(p.Lf + r0 * VD)[o + fq] = L;
+      if (NB == 2 && kb == 1 && p.Qt2) {  // exponents <= 0: the reference precedes the token
+        const float4 m = Lm[0];
+        reinterpret_cast<uint2*>(p.Qt2 + (bc * 128 + tr) * VD)[fq] =
+            scale4(qv[t], make_float4(L.x - m.x, L.y - m.y, L.z - m.z, L.w - m.w), range);
+      }
+    }
+    if (seg == 0) {
+      reinterpret_cast<float4*>(p.GC + bc * VD)[fq] =
+          make_float4(__expf(LC.x), __expf(LC.y), __expf(LC.z), __expf(LC.w));
+#pragma unroll
+      for (int qb = 0; qb < NB; ++qb)
+        reinterpret_cast<float4*>(p.Em + (bc * NB + qb) * VD)[fq] = make_float4(
+            __expf(Lm[qb].x), __expf(Lm[qb].y), __expf(Lm[qb].z), __expf(Lm[qb].w));
+    }
   }
+  cp_async_wait<0>();  // no copy in flight when the CTA exits
   if (range) atomicOr(p.err, ERR_RANGE);
 }
 
@@ -1807,7 +1894,16 @@ cudaError_t launch_prep(const LayerArgs& a, const VecPrep& o, cudaStream_t s) {
   p.Lf = o.Lf;
   p.Qt2 = static_cast<__nv_bfloat16*>(o.Qt2);
   p.err = a.err;
-  vec_prep_kernel<NB><<<a.B * a.H * p.NC * 2, kPrepThreads, 0, s>>>(p);
+  const int nunits = a.B * a.H * p.NC * 2;
+  int dev = 0, sms = 0;
+  cudaError_t e;
+  if ((e = cudaGetDevice(&dev)) || (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)))
+    return e;
+  const size_t smem = kPrepStages * prep_stage_bytes<NB>();
+  if ((e = cudaFuncSetAttribute(vec_prep_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem)))
+    return e;
+  vec_prep_kernel<NB><<<std::min(nunits, sms), kPrepPThreads, smem, s>>>(p, nunits);
   count_launches(1);
   return cudaGetLastError();
 }
